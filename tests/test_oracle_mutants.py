@@ -1,0 +1,98 @@
+"""Strength of the oracle's pins: each test plants one plausible mistake in
+the oracle (on the CPU, by monkeypatching a single function) and checks that
+a pin from test_oracle_pins.py then fails."""
+import numpy as np
+import pytest
+
+import test_oracle_pins as pins
+from oracle import codebook, df11
+from oracle import huffman as H
+
+
+def fails(fn, *args):
+    with pytest.raises((AssertionError, ValueError)):
+        fn(*args)
+
+
+def test_canonical_without_shift_is_caught(monkeypatch):
+    def bad(lengths):
+        order = sorted((l, s) for s, l in enumerate(lengths) if l > 0)
+        codes = [0] * 256
+        for i, (_, s) in enumerate(order):
+            codes[s] = i                       # forgets the shift on a length change
+        return codes
+    monkeypatch.setattr(H, "canonical_codes", bad)
+    fails(pins.test_golden_df11_worked_example)
+    fails(pins.test_golden_clrs_huffman)
+
+
+def test_depth_off_by_one_is_caught(monkeypatch):
+    good = H.huffman_lengths
+    monkeypatch.setattr(H, "huffman_lengths", lambda c: [l + 1 if l else 0 for l in good(c)])
+    fails(pins.test_huffman_optimal_bruteforce, 0)
+    fails(pins.test_golden_clrs_huffman)
+
+
+def test_package_merge_selection_off_by_one_is_caught(monkeypatch):
+    good = H.package_merge
+
+    def bad(counts, max_len):
+        out = good(counts, max_len)
+        syms = [s for s in range(256) if out[s]]
+        out[syms[0]] += 1                        # as if one extra item were selected
+        return out
+    monkeypatch.setattr(H, "package_merge", bad)
+    fails(pins.test_length_limited_optimal_bruteforce, 0)
+
+
+def test_floor_log2_width_is_caught(monkeypatch):
+    monkeypatch.setattr(codebook, "index_bits", lambda U: max(0, U.bit_length() - 1))
+    fails(pins.test_golden_codebook_worked_example)
+    fails(pins.test_codebook_table_and_width, 3)
+
+
+def test_gap_off_by_one_is_caught(monkeypatch):
+    good = df11.chunk_index
+
+    def bad(lens, total_bits, chunk_bits, tpb):
+        n_chunks, n_blocks, gaps, blkoff = good(lens, total_bits, chunk_bits, tpb)
+        gaps = gaps.copy()
+        gaps[1:n_chunks] += 1
+        return n_chunks, n_blocks, gaps, blkoff
+    monkeypatch.setattr(df11, "chunk_index", bad)
+    fails(pins.test_chunks_decode_independently, 8, 32)
+    fails(pins.test_golden_df11_periodic_offsets)
+
+
+def test_dropped_sign_is_caught(monkeypatch):
+    good = df11.merge
+    monkeypatch.setattr(df11, "merge", lambda e, s: good(e, s & np.uint8(0x7F)))
+    fails(pins.test_roundtrip_small_square)
+    fails(pins.test_all_65536_patterns)
+
+
+def test_swapped_exponent_and_mantissa_split_is_caught(monkeypatch):
+    good = df11.split
+
+    def bad(w):
+        e, s = good(w)
+        return e, (s & 0x80) | ((s & 0x7F)[::-1].copy())   # mantissas in the wrong order
+    monkeypatch.setattr(df11, "split", bad)
+    fails(pins.test_sign_and_mantissa_untouched)
+
+
+def test_lsb_msb_confusion_in_codebook_is_caught(monkeypatch):
+    good = codebook.encode
+
+    def bad(w):
+        b = good(w)
+        from oracle import blob as B
+        h = B.unpack_header(b)
+        off = h["off_packed"]
+        n = h["packed_bytes"]
+        # reverse the bit order inside each byte (MSB-first packing)
+        bits = np.unpackbits(b[off:off + n]).reshape(-1, 8)[:, ::-1]
+        b[off:off + n] = np.packbits(bits.reshape(-1))
+        return b
+    monkeypatch.setattr(codebook, "encode", bad)
+    fails(pins.test_golden_codebook_worked_example)
