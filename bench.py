@@ -1,0 +1,410 @@
+#!/usr/bin/env python3
+"""Decode throughput of liblwc on B200.
+
+Workload: one Llama-3-8B-shaped decoder layer (q, k, v, o, gate, up, down;
+218,103,808 BF16 weights, N(0, sigma) with sigma ~ U(0.01, 0.04) and 0.1 %
+outliers x20; synthetic, seeded) compressed with the DFloat11 codec and
+resident in HBM. One step = one layer-batched decode (all seven matrices in
+one launch) into a reusable BF16 buffer. Metric: decoded BF16 GB/s (2 bytes
+per weight / step time), with the HBM roofline fraction of the decode kernel
+and bits/weight. A second line of figures times the codebook codec on the
+same layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lwc|reference]
+
+N > 1 (under torchrun): every rank decodes its own layer (layer index =
+rank) on its own GPU; no data crosses GPUs (weak scaling); the reported time
+is the maximum over ranks. --impl reference times the CPU oracle on the
+host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decoded BF16 GB/s (DFloat11 layer-batched decode, Llama-3-8B layer)"
+FALLBACK_HBM_GBS = 6650.0
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_device.cuh")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("lwc", "reference"), default="lwc")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-codebook", action="store_true")
+    ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+def kernel_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    try:
+        with open(PROFILE_TRAFFIC) as f:
+            t = json.load(f).get("df11_decode", {})
+        if t.get("kernel_sha") == kernel_sha() and t.get("workload") == workload:
+            return int(t["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def gpu_id_for(device) -> str:
+    import torch
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    if uuid is not None:
+        s = str(uuid)
+        return s if s.startswith("GPU-") else "GPU-" + s
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        return vis.split(",")[device.index or 0]
+    return str(device.index or 0)
+
+
+# ---------------------------------------------------------------- setup
+
+def make_layer(layer: int):
+    names, tensors = [], []
+    for name, t in synth.llama_layer_tensors(layer):
+        names.append(name)
+        tensors.append(synth.as_u16(t))
+    return names, tensors
+
+
+def encode_all(tensors, codec: str):
+    from decode_dfloat11_b200 import lwc
+    fn = lwc.lwc_encode_dfloat11 if codec == "df11" else lwc.lwc_encode_codebook
+    with cf.ThreadPoolExecutor(max_workers=min(8, len(tensors))) as ex:
+        return list(ex.map(fn, tensors))
+
+
+def time_steps(step, steps: int, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def cpu_baseline(blobs, n_total: int):
+    """The oracle decoder as it stands, single thread, on this host."""
+    from oracle import df11 as odf
+    t0 = time.perf_counter()
+    n = 0
+    for b in blobs:
+        h = odf.B.unpack_header(b)
+        odf.decode(b)
+        n += h["n"]
+        if time.perf_counter() - t0 > 30:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"oracle bit-serial DFloat11 decode of {n:,} of the layer's {n_total:,} weights "
+                      f"(lib-encoded blobs), one host thread, {dt:.2f} s"}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_lwc(args, rank, world, local_rank, dist):
+    import torch
+    from decode_dfloat11_b200 import build as lwc_build
+    from decode_dfloat11_b200 import lwc
+
+    lwc_build.build()
+    lwc.load()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    layer = args.layer if args.layer is not None else rank
+
+    names, tensors = make_layer(layer)
+    n_total = sum(w.size for w in tensors)
+    enc = encode_all(tensors, "df11")
+    descs = [d for d, _ in enc]
+    blobs_h = [b for _, b in enc]
+    blob_bytes = sum(b.size for b in blobs_h)
+    blobs_d = [torch.from_numpy(b).to(device) for b in blobs_h]
+    out = torch.empty(n_total, dtype=torch.bfloat16, device=device)   # the reusable layer buffer
+    views, off = [], 0
+    for w in tensors:
+        views.append(out[off:off + w.size])
+        off += w.size
+    batch = lwc.Batch(descs, blobs_d, views)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    groups = {(d.chunk_bytes, d.threads_per_block) for d in descs if not d.flags & 1}
+    launches_per_step = len(groups) + sum(1 for d in descs if d.flags & 1 and d.n)
+
+    def step():
+        lwc.lwc_decode_dfloat11_batched(batch, stream=stream)
+
+    # correctness of the very buffers being timed
+    lwc.lwc_decode_dfloat11_batched(batch, d_status=status, stream=stream)
+    torch.cuda.synchronize(device)
+    for w, v in zip(tensors, views):
+        if not torch.equal(v.view(torch.int16), torch.from_numpy(w.view(np.int16)).to(device)):
+            raise SystemExit("decoded layer differs from its input")
+    if int(status.item()):
+        raise SystemExit(f"decoder reported status {int(status.item())}")
+
+    # bring the GPU to its loaded clock, then the W warm-up steps, then K timed steps
+    sampler = ClockSampler(gpu_id_for(device))
+    t_heat = time.perf_counter()
+    while time.perf_counter() - t_heat < 1.0:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(device)
+    for _ in range(args.warmup):
+        step()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ms = time_steps(step, args.steps, stream)
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    ms_max = ms
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    ms_per_step = ms_max / args.steps
+    value = world * 2 * n_total / (ms_per_step * 1e-3) / 1e9
+
+    # roofline of the decode kernel (one launch per step here)
+    peak, peak_kind = measured_peak()
+    launch_ms = ms / (args.steps * launches_per_step)
+    alg_bytes = blob_bytes + 2 * n_total
+    achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
+    workload = "llama3-8b-layer-df11"
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(workload),
+                "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
+                "kernel": "df11_decode_kernel", "launch_ms": round(launch_ms, 5)}
+
+    result = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+        "data": "synthetic (seeded N(0, sigma) BF16, sigma ~ U(0.01, 0.04), 0.1% outliers x20)",
+        "config": {"workload": workload, "tensors": names, "weights_per_gpu": n_total,
+                   "compressed_bytes_per_gpu": blob_bytes,
+                   "bits_per_weight": round(8 * blob_bytes / n_total, 4),
+                   "size_vs_bf16": round(blob_bytes / (2 * n_total), 4),
+                   "parallelism": f"replicas x{world} (each GPU decodes its own layer; no collective)",
+                   "l2": f"no flush: {(blob_bytes + 2 * n_total) / 1e6:.0f} MB moved per step > 126 MB L2",
+                   "chunk_bytes": descs[0].chunk_bytes, "threads_per_block": descs[0].threads_per_block},
+        "roofline": roofline,
+        "gpu_launches": args.steps * launches_per_step,
+        "clocks": clocks,
+    }
+
+    # codebook codec on the same layer (secondary figures)
+    if not args.no_codebook:
+        cenc = encode_all(tensors, "codebook")
+        cblobs = [torch.from_numpy(b).to(device) for _, b in cenc]
+        cdescs = [d for d, _ in cenc]
+        def cstep():
+            for d, b, v in zip(cdescs, cblobs, views):
+                lwc.lwc_decode_codebook(d, b, v, stream)
+        cstep()
+        torch.cuda.synchronize(device)
+        for w, v in zip(tensors, views):
+            if not torch.equal(v.view(torch.int16), torch.from_numpy(w.view(np.int16)).to(device)):
+                raise SystemExit("codebook-decoded layer differs from its input")
+        for _ in range(args.warmup):
+            cstep()
+        cms = time_steps(cstep, args.steps, stream) / args.steps
+        cbytes = sum(b.numel() for b in cblobs)
+        result["codebook"] = {
+            "value": round(2 * n_total / (cms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(cms, 5),
+            "launches_per_step": len(cdescs), "bits_per_weight": round(8 * cbytes / n_total, 4),
+            "index_bits": [d.k for d in cdescs],
+            "hbm_frac": round((cbytes + 2 * n_total) / (cms * 1e-3) / 1e9 / peak, 4)}
+        del cblobs
+
+    # end to end through the C ABI with host buffers: pinned blobs -> device,
+    # decode, decoded layer -> pinned host, every step
+    if not args.no_e2e:
+        pinned_in = [torch.from_numpy(b).pin_memory() for b in blobs_h]
+        pinned_out = torch.empty(n_total, dtype=torch.bfloat16).pin_memory()
+
+        def estep():
+            for h, d in zip(pinned_in, blobs_d):
+                d.copy_(h, non_blocking=True)
+            lwc.lwc_decode_dfloat11_batched(batch, stream=stream)
+            pinned_out.copy_(out, non_blocking=True)
+        for _ in range(3):
+            estep()
+        e_steps = max(3, min(args.steps, 20))
+        torch.cuda.synchronize(device)
+        ems = time_steps(estep, e_steps, stream) / e_steps
+        if not torch.equal(pinned_out.view(torch.int16)[:tensors[0].size],
+                           torch.from_numpy(tensors[0].view(np.int16))):
+            raise SystemExit("end-to-end output differs from its input")
+        ev = world * 2 * n_total / (ems * 1e-3) / 1e9
+        if dist:
+            t = torch.tensor([ems], dtype=torch.float64, device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ev = world * 2 * n_total / (float(t.item()) * 1e-3) / 1e9
+        result["e2e"] = {"value": round(ev, 3), "unit": "GB/s", "h2d_bytes_per_step": blob_bytes,
+                         "d2h_bytes_per_step": 2 * n_total, "ms_per_step": round(ems, 4), "steps": e_steps}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(blobs_h, n_total)
+    return result
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle as it stands, on this host, on a bounded sample of the
+    same workload (the layer's q matrix per step)."""
+    from decode_dfloat11_b200 import build as lwc_build
+    from decode_dfloat11_b200 import lwc
+    from oracle import df11 as odf
+    lwc_build.build()
+    names, tensors = make_layer(args.layer or 0)
+    d, blob = lwc.lwc_encode_dfloat11(tensors[0])
+    n = d.n
+    for _ in range(args.warmup):
+        odf.decode(blob)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        odf.decode(blob)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = 2 * n / dt / 1e9
+    sample = f"oracle bit-serial DFloat11 decode of the layer's q matrix ({n:,} weights) per step, one host thread"
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u16", "data": "synthetic",
+        "config": {"workload": "llama3-8b-layer-df11", "sample": "q matrix 4096x4096"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(local_rank)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                 device_id=torch.device("cuda", local_rank))
+        dist = tdist
+    try:
+        result = run_lwc(args, rank, world, local_rank, dist)
+        if rank == 0:
+            print(json.dumps(result), flush=True)
+    finally:
+        if dist:
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,576 @@
+// DFloat11-style decoder for sm_100a.
+//
+// What it computes ("Koniec z kompromisami! DFloat11 ratuje dokładność modeli
+// AI ...", section "Przełom: DFloat11 – bezstratna kompresja z wydajnością
+// GPU"): every weight is rebuilt from its Huffman-coded 8-bit exponent and its
+// raw sign|mantissa byte, bit for bit.
+//
+// How (same page, section "Jak to działa w praktyce? Magia na poziomie GPU"):
+//  * small linked lookup tables held in shared memory: the blob's
+//    hierarchical 256-entry tables (one per 8 code bits), fronted by two
+//    4096-entry tables this kernel builds from them, which resolve every code
+//    that fits in the next 12 stream bits — several codes per lookup;
+//  * two phases: each thread counts the codes that start in its chunk of the
+//    stream, a block-wide scan turns the counts into output positions, and the
+//    threads decode again, this time writing exponents to a shared-memory
+//    staging buffer; the staged exponents are then merged with the
+//    sign|mantissa bytes and written out with 16-byte stores;
+//  * all matrices of a transformer block in one launch: the grid walks a work
+//    list of (tensor, block) items; CTAs are persistent, take contiguous runs
+//    of items and rebuild their tables only when the tensor changes.
+// Blocks never wait on one another: each block's first output index is stored
+// in the blob, so there is no inter-block scan.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "lwc_device.cuh"
+#include "lwc_internal.h"
+
+namespace lwc {
+namespace {
+
+constexpr int kFastBits = 12;
+constexpr int kFastSize = 1 << kFastBits;
+constexpr int kMaxBatch = 32;
+constexpr uint32_t kFastBytes = kFastSize * 4 + kFastSize;   // symbol table + count table
+
+struct Df11Tensor {
+    const uint32_t *stream;
+    const uint8_t *gaps;
+    const uint64_t *blkoff;
+    const uint8_t *sm;
+    const uint16_t *lut;
+    uint16_t *out;
+    uint64_t n;
+    uint64_t total_bits;
+    uint64_t stream_words;
+    uint32_t n_blocks;
+    uint32_t n_tables;
+    uint32_t first_work;   // index of this tensor's block 0 in the launch's work list
+    uint32_t pad;
+};
+
+struct Df11Batch {
+    Df11Tensor t[kMaxBatch];
+    uint32_t count;
+    uint32_t total_work;
+    uint32_t chunk_words;  // chunk_bytes / 4
+    uint32_t seg_words;    // words staged per block: T * chunk_words + 2, rounded up to 4
+    uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 16)
+    uint32_t lut_entries;  // lookup-table entries reserved in shared memory
+    uint32_t *status;
+};
+
+// ---- lookup tables ---------------------------------------------------------
+
+// Walk the hierarchical tables with the window's top bits; returns
+// symbol | length << 8. A path no valid code takes yields length 1 and sets
+// LWC_DEVICE_BAD_CODE in `bad` (so decoding always advances and ends).
+__device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab, uint64_t win, uint32_t &bad) {
+    uint32_t e = lut[win >> 56];
+#pragma unroll 1
+    for (int d = 1; (e & 0x8000u) && d < 4; d++) {
+        const uint32_t t = e & 0x7FFFu;
+        if (t >= ntab) {
+            bad |= LWC_DEVICE_BAD_CODE;
+            return 0x100u;
+        }
+        e = lut[t * 256u + (uint32_t)((win >> (56 - 8 * d)) & 0xFFu)];
+    }
+    const uint32_t len = (e >> 8) & 0x3Fu;
+    if ((e & 0x8000u) || len == 0 || len > 32) {
+        bad |= LWC_DEVICE_BAD_CODE;
+        return 0x100u;
+    }
+    return e & 0x3FFFu;
+}
+
+// Fast tables, indexed by the next 12 stream bits:
+//  cnt_tab[v] = count << 4 | bits, for all whole codes inside the 12 bits;
+//  sym_tab[v] = sym0 | sym1 << 8 | sym2 << 16 | n << 24 | bits << 26, for the
+//               first n <= 3 of them. 0 means "first code longer than 12 bits".
+__device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *cnt_tab, uint32_t *sym_tab) {
+    for (uint32_t v = threadIdx.x; v < kFastSize; v += blockDim.x) {
+        uint64_t w = (uint64_t)v << (64 - kFastBits);
+        uint32_t used = 0, cnt = 0, syms = 0, n3 = 0, used3 = 0, ignore = 0;
+        while (cnt < (uint32_t)kFastBits) {
+            const uint32_t r = lut_walk(lut, ntab, w, ignore);
+            const uint32_t len = r >> 8;
+            if (ignore || used + len > (uint32_t)kFastBits) break;
+            if (cnt < 3) {
+                syms |= (r & 0xFFu) << (8 * cnt);
+                n3 = cnt + 1;
+                used3 = used + len;
+            }
+            cnt++;
+            used += len;
+            w <<= len;
+        }
+        cnt_tab[v] = cnt ? (uint8_t)((cnt << 4) | used) : (uint8_t)0;
+        sym_tab[v] = n3 ? (syms | (n3 << 24) | (used3 << 26)) : 0u;
+    }
+}
+
+// ---- bit window --------------------------------------------------------------
+
+// 64-bit window over the staged segment, MSB = next stream bit. Holds >= 32
+// valid bits before every decode step.
+struct BitWindow {
+    uint64_t win;
+    uint32_t nb;   // valid bits
+    uint32_t wp;   // next word to load
+    __device__ __forceinline__ void init(const uint32_t *seg, uint32_t bit) {
+        wp = bit >> 5;
+        const uint64_t w = ((uint64_t)seg[wp] << 32) | seg[wp + 1];
+        const uint32_t sh = bit & 31u;
+        win = w << sh;
+        nb = 64 - sh;
+        wp += 2;
+    }
+    __device__ __forceinline__ void consume(const uint32_t *seg, uint32_t len) {
+        win <<= len;
+        nb -= len;
+        if (nb < 32) {
+            win |= (uint64_t)seg[wp++] << (32 - nb);
+            nb += 32;
+        }
+    }
+};
+
+// Exponent writer for pass 2: gathers bytes into 32-bit words so that most
+// shared-memory stores are whole words; the first and last partial words of a
+// thread's range are written byte by byte (their other bytes belong to the
+// neighbouring threads).
+struct StageWriter {
+    uint8_t *base;
+    uint32_t wpos;   // byte offset of acc's byte 0 (multiple of 4)
+    uint32_t head;   // bytes of the first word owned by the previous thread
+    uint32_t fill;   // bytes held in acc, counting the head
+    uint64_t acc;
+    __device__ __forceinline__ void init(uint8_t *b, uint32_t p) {
+        base = b;
+        wpos = p & ~3u;
+        head = p & 3u;
+        fill = head;
+        acc = 0;
+    }
+    __device__ __forceinline__ void put(uint32_t syms, uint32_t n) {
+        acc |= (uint64_t)syms << (8 * fill);
+        fill += n;
+        if (fill >= 4) {
+            const uint32_t w = (uint32_t)acc;
+            if (head) {
+                for (uint32_t j = head; j < 4; j++) base[wpos + j] = (uint8_t)(w >> (8 * j));
+                head = 0;
+            } else {
+                *reinterpret_cast<uint32_t *>(base + wpos) = w;
+            }
+            wpos += 4;
+            acc >>= 32;
+            fill -= 4;
+        }
+    }
+    __device__ __forceinline__ void finish() {
+        for (uint32_t j = head; j < fill; j++) base[wpos + j] = (uint8_t)(acc >> (8 * j));
+    }
+};
+
+// ---- merge ---------------------------------------------------------------------
+
+// Two weights from s = [s0 s1 ..] and e = [e0 e1 ..] bytes selected by `sel`:
+// w = (s & 0x80) << 8 | e << 7 | (s & 0x7F), two at a time in one word.
+__device__ __forceinline__ uint32_t merge2(uint32_t s, uint32_t e, uint32_t sel) {
+    const uint32_t x = __byte_perm(s, e, sel);   // [s_a, e_a, s_b, e_b]
+    return (x & 0x007F007Fu) | ((x >> 1) & 0x7F807F80u) | ((x << 8) & 0x80008000u);
+}
+
+__device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e) {
+    return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
+}
+
+// ---- block scan ------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t &total) {
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    uint32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+        if (lane >= (uint32_t)o) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t s = lane < nwarps ? warp_sums[lane] : 0u;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, s, o);
+            if (lane >= (uint32_t)o) s += y;
+        }
+        if (lane < nwarps) warp_sums[lane] = s;
+    }
+    __syncthreads();
+    total = warp_sums[nwarps - 1];
+    const uint32_t before = warp ? warp_sums[warp - 1] : 0u;
+    __syncthreads();   // warp_sums is reused by the next scan
+    return before + x - v;
+}
+
+// ---- the kernel -------------------------------------------------------------------
+
+template <int kMaxThreads>
+__global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048 / kMaxThreads / 2 : 1)
+    df11_decode_kernel(const __grid_constant__ Df11Batch B) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem);
+    uint8_t *cnt_tab = smem + kFastSize * 4;
+    uint16_t *lut = reinterpret_cast<uint16_t *>(smem + kFastBytes);
+    uint32_t *seg = reinterpret_cast<uint32_t *>(smem + kFastBytes + 2 * B.lut_entries);
+    uint8_t *stage = reinterpret_cast<uint8_t *>(seg + B.seg_words);
+    uint32_t *warp_sums = reinterpret_cast<uint32_t *>(stage + B.stage_bytes);
+
+    const uint32_t T = blockDim.x, tid = threadIdx.x;
+    const uint32_t CW = B.chunk_words, cbits = CW * 32u;
+    const uint32_t W = B.total_work, G = gridDim.x;
+    const uint32_t w_begin = (uint32_t)((uint64_t)W * blockIdx.x / G);
+    const uint32_t w_end = (uint32_t)((uint64_t)W * (blockIdx.x + 1) / G);
+
+    uint32_t bad = 0;
+    int cur = -1;
+    uint32_t ti = 0;
+    for (uint32_t w = w_begin; w < w_end; ++w) {
+        while (ti + 1 < B.count && w >= B.t[ti + 1].first_work) ++ti;
+        const Df11Tensor &tn = B.t[ti];
+        if ((int)ti != cur) {
+            // new tensor: stage its hierarchical tables, build the fast tables
+            __syncthreads();
+            const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
+            for (uint32_t i = tid; i < ntab * 128u; i += T)
+                reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
+            __syncthreads();
+            build_fast_tables(lut, ntab, cnt_tab, sym_tab);
+            __syncthreads();
+            cur = (int)ti;
+        }
+        const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
+        const uint32_t b = w - tn.first_work;
+        const uint64_t o0 = tn.blkoff[b], o1 = tn.blkoff[b + 1];
+        if (!(o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes)) {
+            bad |= LWC_DEVICE_BAD_OFFSET;   // same decision in every thread
+            continue;
+        }
+
+        // stage this block's stream segment (plus 2 words of look-ahead)
+        const uint64_t seg0 = (uint64_t)b * T * CW;
+        for (uint32_t i = tid; i < B.seg_words / 4; i += T) {
+            const uint64_t gw = seg0 + 4ull * i;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (gw + 4 <= tn.stream_words) v = dev::ld_stream_v4(tn.stream + gw);
+            reinterpret_cast<uint4 *>(seg)[i] = v;
+        }
+        const uint32_t gap = tn.gaps[(uint64_t)b * T + tid];
+        __syncthreads();
+
+        const uint64_t rem = tn.total_bits - (uint64_t)b * T * cbits;
+        const uint32_t start = tid * cbits + gap;
+        const uint32_t end = (uint32_t)min((uint64_t)(tid + 1) * cbits, rem);
+
+        // phase 1: count the codes that start in [start, end)
+        uint32_t count = 0;
+        if (start < end) {
+            BitWindow bw;
+            bw.init(seg, start);
+            uint32_t pos = start;
+            while (pos + kFastBits <= end) {
+                const uint32_t e = cnt_tab[bw.win >> (64 - kFastBits)];
+                uint32_t len;
+                if (e) {
+                    count += e >> 4;
+                    len = e & 15u;
+                } else {
+                    len = lut_walk(lut, ntab, bw.win, bad) >> 8;
+                    count += 1;
+                }
+                bw.consume(seg, len);
+                pos += len;
+            }
+            while (pos < end) {
+                const uint32_t len = lut_walk(lut, ntab, bw.win, bad) >> 8;
+                count += 1;
+                bw.consume(seg, len);
+                pos += len;
+            }
+        }
+
+        uint32_t total;
+        const uint32_t first = block_exclusive_scan(count, warp_sums, total);
+        if (total != (uint32_t)(o1 - o0)) {
+            bad |= LWC_DEVICE_BAD_COUNT;   // `total` is the same in every thread
+            continue;
+        }
+
+        // phase 2: decode again, writing exponents to stage[(o0 & 15) + first ...]
+        if (start < end) {
+            BitWindow bw;
+            bw.init(seg, start);
+            StageWriter out;
+            out.init(stage, (uint32_t)(o0 & 15u) + first);
+            uint32_t pos = start;
+            while (pos + kFastBits <= end) {
+                const uint32_t e = sym_tab[bw.win >> (64 - kFastBits)];
+                uint32_t len;
+                if (e) {
+                    out.put(e & 0xFFFFFFu, (e >> 24) & 3u);
+                    len = e >> 26;
+                } else {
+                    const uint32_t r = lut_walk(lut, ntab, bw.win, bad);
+                    out.put(r & 0xFFu, 1);
+                    len = r >> 8;
+                }
+                bw.consume(seg, len);
+                pos += len;
+            }
+            while (pos < end) {
+                const uint32_t r = lut_walk(lut, ntab, bw.win, bad);
+                out.put(r & 0xFFu, 1);
+                const uint32_t len = r >> 8;
+                bw.consume(seg, len);
+                pos += len;
+            }
+            out.finish();
+        }
+        __syncthreads();
+
+        // merge exponents with sign|mantissa bytes; 16 weights per step
+        const uint64_t base = o0 & ~15ull;
+        for (uint64_t g = base + 16ull * tid; g < o1; g += 16ull * T) {
+            if (g >= o0 && g + 16 <= o1) {
+                const uint4 s = dev::ld_stream_v4(tn.sm + g);
+                const uint4 e = *reinterpret_cast<const uint4 *>(stage + (g - base));
+                uint4 r0, r1;
+                r0.x = merge2(s.x, e.x, 0x5140u);
+                r0.y = merge2(s.x, e.x, 0x7362u);
+                r0.z = merge2(s.y, e.y, 0x5140u);
+                r0.w = merge2(s.y, e.y, 0x7362u);
+                r1.x = merge2(s.z, e.z, 0x5140u);
+                r1.y = merge2(s.z, e.z, 0x7362u);
+                r1.z = merge2(s.w, e.w, 0x5140u);
+                r1.w = merge2(s.w, e.w, 0x7362u);
+                dev::st_v4(tn.out + g, r0);
+                dev::st_v4(tn.out + g + 8, r1);
+            } else {
+                for (uint32_t j = 0; j < 16; j++) {
+                    const uint64_t i = g + j;
+                    if (i >= o0 && i < o1) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
+                }
+            }
+        }
+        __syncthreads();
+    }
+    if (bad && B.status) atomicOr(B.status, bad);
+}
+
+// One exponent value for the whole tensor: out = merge(const_exp, sm).
+__global__ void df11_const_kernel(const uint8_t *__restrict__ sm, uint16_t *__restrict__ out, uint64_t n,
+                                  uint32_t const_exp) {
+    const uint32_t e4 = const_exp * 0x01010101u;
+    const uint64_t stride = 16ull * gridDim.x * blockDim.x;
+    for (uint64_t g = 16ull * (blockIdx.x * (uint64_t)blockDim.x + threadIdx.x); g < n; g += stride) {
+        if (g + 16 <= n) {
+            const uint4 s = dev::ld_stream_v4(sm + g);
+            uint4 r0, r1;
+            r0.x = merge2(s.x, e4, 0x5140u);
+            r0.y = merge2(s.x, e4, 0x7362u);
+            r0.z = merge2(s.y, e4, 0x5140u);
+            r0.w = merge2(s.y, e4, 0x7362u);
+            r1.x = merge2(s.z, e4, 0x5140u);
+            r1.y = merge2(s.z, e4, 0x7362u);
+            r1.z = merge2(s.w, e4, 0x5140u);
+            r1.w = merge2(s.w, e4, 0x7362u);
+            dev::st_v4(out + g, r0);
+            dev::st_v4(out + g + 8, r1);
+        } else {
+            for (uint64_t i = g; i < n; i++) out[i] = merge1(sm[i], const_exp);
+        }
+    }
+}
+
+// ---- host side -----------------------------------------------------------------------
+
+struct DeviceConfig {
+    int sms = 0;
+    int max_smem = 0;
+    bool ready = false;
+};
+
+std::mutex g_cfg_mutex;
+std::vector<DeviceConfig> g_cfg;
+
+lwc_status device_config(DeviceConfig &out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(err));
+    std::lock_guard<std::mutex> lock(g_cfg_mutex);
+    if ((int)g_cfg.size() <= dev) g_cfg.resize(dev + 1);
+    DeviceConfig &c = g_cfg[dev];
+    if (!c.ready) {
+        err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (err == cudaSuccess) err = cudaDeviceGetAttribute(&c.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        const void *kernels[] = {(const void *)df11_decode_kernel<256>, (const void *)df11_decode_kernel<1024>};
+        for (const void *k : kernels) {
+            if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
+            if (err == cudaSuccess)
+                err = cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        }
+        if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device setup: %s", cudaGetErrorString(err));
+        c.ready = true;
+    }
+    out = c;
+    return LWC_OK;
+}
+
+uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// Launch one kernel over up to kMaxBatch tensors sharing (chunk_bytes, threads_per_block).
+lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, const void *const *d_ins,
+                        uint16_t *const *d_outs, uint32_t *d_status, cudaStream_t stream,
+                        const DeviceConfig &cfg) {
+    Df11Batch B;
+    std::memset(&B, 0, sizeof B);
+    const lwc_desc &d0 = descs[idx[0]];
+    const uint32_t T = d0.threads_per_block;
+    B.chunk_words = d0.chunk_bytes / 4;
+    B.seg_words = (uint32_t)round_up((uint64_t)T * B.chunk_words + 2, 4);
+    uint64_t work = 0, max_count = 0, max_tables = 0;
+    for (size_t j = 0; j < idx.size(); j++) {
+        const lwc_desc &d = descs[idx[j]];
+        const uint8_t *base = static_cast<const uint8_t *>(d_ins[idx[j]]);
+        Df11Tensor &t = B.t[j];
+        t.stream = reinterpret_cast<const uint32_t *>(base + d.off_stream);
+        t.gaps = base + d.off_gaps;
+        t.blkoff = reinterpret_cast<const uint64_t *>(base + d.off_blkoff);
+        t.sm = base + d.off_sm;
+        t.lut = reinterpret_cast<const uint16_t *>(base + d.off_lut);
+        t.out = d_outs[idx[j]];
+        t.n = d.n;
+        t.total_bits = d.total_bits;
+        t.stream_words = d.stream_bytes / 4;
+        t.n_blocks = (uint32_t)d.n_blocks;
+        t.n_tables = d.n_tables;
+        t.first_work = (uint32_t)work;
+        work += d.n_blocks;
+        max_count = std::max<uint64_t>(max_count, d.max_block_count);
+        max_tables = std::max<uint64_t>(max_tables, d.n_tables);
+    }
+    if (work > 0xFFFFFFFFull) return fail(LWC_ERR_UNSUPPORTED, "too many blocks in one launch");
+    B.count = (uint32_t)idx.size();
+    B.total_work = (uint32_t)work;
+    B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
+    B.lut_entries = (uint32_t)(max_tables * 256);
+    B.status = d_status;
+    const uint64_t smem = kFastBytes + 2ull * B.lut_entries + 4ull * B.seg_words + B.stage_bytes + 128;
+    if (smem > (uint64_t)cfg.max_smem)
+        return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
+                    (unsigned long long)smem, cfg.max_smem);
+    const void *kernel = T <= 256 ? (const void *)df11_decode_kernel<256> : (const void *)df11_decode_kernel<1024>;
+    int per_sm = 0;
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)T, (size_t)smem);
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
+    if (per_sm < 1) return fail(LWC_ERR_UNSUPPORTED, "decoder does not fit on an SM (%u threads, %llu B smem)", T,
+                                (unsigned long long)smem);
+    const uint64_t grid = std::min<uint64_t>(work, (uint64_t)per_sm * cfg.sms);
+    if (T <= 256)
+        df11_decode_kernel<256><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);
+    else
+        df11_decode_kernel<1024><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return LWC_OK;
+}
+
+lwc_status launch_const(const lwc_desc &d, const void *d_in, uint16_t *d_out, cudaStream_t stream,
+                        const DeviceConfig &cfg) {
+    if (d.n == 0) return LWC_OK;
+    const uint64_t groups = (d.n + 15) / 16;
+    const uint64_t blocks = std::min<uint64_t>((groups + 255) / 256, (uint64_t)cfg.sms * 8);
+    df11_const_kernel<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const uint8_t *>(d_in) + d.off_sm, d_out,
+                                                           d.n, d.const_exp);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return LWC_OK;
+}
+
+}  // namespace
+}  // namespace lwc
+
+using namespace lwc;
+
+extern "C" {
+
+lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const *d_ins, uint16_t *const *d_outs,
+                                       int count, uint32_t *d_status, lwc_stream_t stream) {
+    if (count < 0 || (count > 0 && (!descs || !d_ins || !d_outs)))
+        return fail(LWC_ERR_INVALID_ARG, "bad batch arguments");
+    for (int i = 0; i < count; i++) {
+        lwc_status st = check_df11_desc(&descs[i]);
+        if (st) return st;
+        if (descs[i].n == 0) continue;
+        if (!d_ins[i] || !d_outs[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (tensor %d)", i);
+        if (!aligned16(d_ins[i]) || !aligned16(d_outs[i]))
+            return fail(LWC_ERR_MISALIGNED, "device pointers must be 16-byte aligned (tensor %d)", i);
+    }
+    if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u))
+        return fail(LWC_ERR_MISALIGNED, "status word must be 4-byte aligned");
+    bool any = false;
+    for (int i = 0; i < count; i++) any = any || descs[i].n > 0;
+    if (!any) {
+        clear_error();
+        return LWC_OK;
+    }
+    DeviceConfig cfg;
+    lwc_status st = device_config(cfg);
+    if (st) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // single-exponent tensors; the rest grouped by (chunk_bytes, threads_per_block)
+    std::vector<std::pair<uint64_t, int>> keyed;
+    for (int i = 0; i < count; i++) {
+        const lwc_desc &d = descs[i];
+        if (d.n == 0) continue;
+        if (d.flags & kFlagSingleExponent) {
+            st = launch_const(d, d_ins[i], d_outs[i], s, cfg);
+            if (st) return st;
+            continue;
+        }
+        keyed.push_back({((uint64_t)d.chunk_bytes << 32) | d.threads_per_block, i});
+    }
+    std::stable_sort(keyed.begin(), keyed.end(),
+                     [](const std::pair<uint64_t, int> &a, const std::pair<uint64_t, int> &b) { return a.first < b.first; });
+    std::vector<int> group;
+    for (size_t i = 0; i < keyed.size(); i++) {
+        group.push_back(keyed[i].second);
+        const bool last = i + 1 == keyed.size() || keyed[i + 1].first != keyed[i].first;
+        if (last || group.size() == (size_t)kMaxBatch) {
+            st = launch_group(group, descs, d_ins, d_outs, d_status, s, cfg);
+            if (st) return st;
+            group.clear();
+        }
+    }
+    clear_error();
+    return LWC_OK;
+}
+
+lwc_status lwc_decode_dfloat11_checked(const lwc_desc *desc, const void *d_in, uint16_t *d_out, uint32_t *d_status,
+                                       lwc_stream_t stream) {
+    if (!desc) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    return lwc_decode_dfloat11_batched(desc, &d_in, &d_out, 1, d_status, stream);
+}
+
+lwc_status lwc_decode_dfloat11(const lwc_desc *desc, const void *d_in, uint16_t *d_out, lwc_stream_t stream) {
+    return lwc_decode_dfloat11_checked(desc, d_in, d_out, nullptr, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,225 @@
+"""ctypes binding of liblwc (include/lwc.h): argument marshalling only.
+
+Every function keeps the C name. Host buffers are numpy arrays; device
+buffers are passed as integer addresses (``tensor.data_ptr()``) or as torch
+tensors, and streams as ``torch.cuda.Stream`` objects or raw handles. All
+decoding happens in the library's CUDA kernels; there is no other path: if
+liblwc.so is missing or fails to load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblwc.so")
+
+LWC_OK = 0
+LWC_CODEC_DFLOAT11 = 1
+LWC_CODEC_CODEBOOK = 2
+LWC_DEVICE_BAD_COUNT = 1
+LWC_DEVICE_BAD_CODE = 2
+LWC_DEVICE_BAD_OFFSET = 4
+LWC_DEVICE_TIMEOUT = 8
+
+STATUS_NAMES = {0: "LWC_OK", 1: "LWC_ERR_INVALID_ARG", 2: "LWC_ERR_MISALIGNED", 3: "LWC_ERR_CORRUPT",
+                4: "LWC_ERR_UNSUPPORTED", 5: "LWC_ERR_NOMEM", 6: "LWC_ERR_CUDA"}
+
+# Every symbol include/lwc.h declares.
+EXPORTED = (
+    "lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
+    "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
+    "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_status_string",
+    "lwc_last_error", "lwc_version",
+)
+
+
+class LwcError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+class lwc_desc(ctypes.Structure):
+    _fields_ = [
+        ("magic", ctypes.c_uint32), ("version", ctypes.c_uint32), ("codec", ctypes.c_uint32),
+        ("flags", ctypes.c_uint32), ("n", ctypes.c_uint64), ("total_bytes", ctypes.c_uint64),
+        ("chunk_bytes", ctypes.c_uint32), ("threads_per_block", ctypes.c_uint32),
+        ("max_len", ctypes.c_uint32), ("n_tables", ctypes.c_uint32),
+        ("n_chunks", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64), ("total_bits", ctypes.c_uint64),
+        ("max_block_count", ctypes.c_uint32), ("const_exp", ctypes.c_uint32),
+        ("off_lengths", ctypes.c_uint64), ("off_lut", ctypes.c_uint64), ("off_gaps", ctypes.c_uint64),
+        ("off_blkoff", ctypes.c_uint64), ("off_stream", ctypes.c_uint64), ("stream_bytes", ctypes.c_uint64),
+        ("off_sm", ctypes.c_uint64),
+        ("U", ctypes.c_uint32), ("k", ctypes.c_uint32), ("off_table", ctypes.c_uint64),
+        ("off_packed", ctypes.c_uint64), ("packed_bytes", ctypes.c_uint64),
+    ]
+
+    def as_dict(self):
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+    @property
+    def bits_per_weight(self) -> float:
+        return 8.0 * self.total_bytes / max(1, self.n)
+
+
+class lwc_df11_params(ctypes.Structure):
+    _fields_ = [("chunk_bytes", ctypes.c_uint32), ("threads_per_block", ctypes.c_uint32),
+                ("max_len", ctypes.c_uint32)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_u64 = ctypes.c_uint64
+
+
+def load():
+    """Load liblwc.so (built by decode_dfloat11_b200.build). Raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"liblwc.so not built ({LIB_PATH}); run python -m decode_dfloat11_b200.build")
+    L = ctypes.CDLL(LIB_PATH)
+    D = ctypes.POINTER(lwc_desc)
+    L.lwc_encode_dfloat11.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), D,
+                                      ctypes.POINTER(_P), ctypes.POINTER(_u64)]
+    L.lwc_encode_codebook.argtypes = [_P, _u64, D, ctypes.POINTER(_P), ctypes.POINTER(_u64)]
+    L.lwc_free.argtypes = [_P]
+    L.lwc_free.restype = None
+    L.lwc_desc_from_blob.argtypes = [_P, _u64, D]
+    L.lwc_decode_dfloat11.argtypes = [D, _P, _P, _P]
+    L.lwc_decode_codebook.argtypes = [D, _P, _P, _P]
+    L.lwc_decode_dfloat11_checked.argtypes = [D, _P, _P, _P, _P]
+    L.lwc_decode_codebook_checked.argtypes = [D, _P, _P, _P, _P]
+    L.lwc_decode_dfloat11_batched.argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int, _P, _P]
+    L.lwc_status_string.argtypes = [ctypes.c_int]
+    L.lwc_status_string.restype = ctypes.c_char_p
+    L.lwc_last_error.argtypes = []
+    L.lwc_last_error.restype = ctypes.c_char_p
+    L.lwc_version.argtypes = []
+    for name in ("lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
+                 "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
+                 "lwc_decode_dfloat11_batched"):
+        getattr(L, name).restype = ctypes.c_int
+    _lib = L
+    return L
+
+
+def _check(status: int):
+    if status != LWC_OK:
+        raise LwcError(status, load().lwc_last_error().decode())
+
+
+def _addr(x) -> int | None:
+    """Device address of a torch tensor, or an integer address as given."""
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(s) -> int | None:
+    if s is None:
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _take_blob(ptr: ctypes.c_void_p, nbytes: int) -> np.ndarray:
+    L = load()
+    try:
+        out = np.empty(nbytes, np.uint8)
+        if nbytes:
+            ctypes.memmove(out.ctypes.data, ptr, nbytes)
+        return out
+    finally:
+        L.lwc_free(ptr)
+
+
+def _src(h_src) -> np.ndarray:
+    a = np.ascontiguousarray(h_src)
+    if a.dtype != np.uint16:
+        a = a.view(np.uint16) if a.dtype.itemsize == 2 else a.astype(np.uint16)
+    return a.reshape(-1)
+
+
+def lwc_encode_dfloat11(h_src, chunk_bytes: int = 36, threads_per_block: int = 256,
+                        max_len: int = 32) -> tuple[lwc_desc, np.ndarray]:
+    """Encode host BF16 bit patterns (uint16 array); returns (desc, blob bytes)."""
+    src = _src(h_src)
+    desc, ptr, nbytes = lwc_desc(), _P(), _u64()
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    _check(load().lwc_encode_dfloat11(src.ctypes.data, src.size, ctypes.byref(params), ctypes.byref(desc),
+                                      ctypes.byref(ptr), ctypes.byref(nbytes)))
+    return desc, _take_blob(ptr, nbytes.value)
+
+
+def lwc_encode_codebook(h_src) -> tuple[lwc_desc, np.ndarray]:
+    src = _src(h_src)
+    desc, ptr, nbytes = lwc_desc(), _P(), _u64()
+    _check(load().lwc_encode_codebook(src.ctypes.data, src.size, ctypes.byref(desc), ctypes.byref(ptr),
+                                      ctypes.byref(nbytes)))
+    return desc, _take_blob(ptr, nbytes.value)
+
+
+def lwc_desc_from_blob(h_blob: np.ndarray) -> lwc_desc:
+    b = np.ascontiguousarray(h_blob, dtype=np.uint8)
+    desc = lwc_desc()
+    _check(load().lwc_desc_from_blob(b.ctypes.data, b.size, ctypes.byref(desc)))
+    return desc
+
+
+def lwc_decode_dfloat11(desc: lwc_desc, d_in, d_out_bf16, stream=None) -> None:
+    _check(load().lwc_decode_dfloat11(ctypes.byref(desc), _addr(d_in), _addr(d_out_bf16), _stream(stream)))
+
+
+def lwc_decode_codebook(desc: lwc_desc, d_in, d_out_bf16, stream=None) -> None:
+    _check(load().lwc_decode_codebook(ctypes.byref(desc), _addr(d_in), _addr(d_out_bf16), _stream(stream)))
+
+
+def lwc_decode_dfloat11_checked(desc, d_in, d_out_bf16, d_status, stream=None) -> None:
+    _check(load().lwc_decode_dfloat11_checked(ctypes.byref(desc), _addr(d_in), _addr(d_out_bf16),
+                                              _addr(d_status), _stream(stream)))
+
+
+def lwc_decode_codebook_checked(desc, d_in, d_out_bf16, d_status, stream=None) -> None:
+    _check(load().lwc_decode_codebook_checked(ctypes.byref(desc), _addr(d_in), _addr(d_out_bf16),
+                                              _addr(d_status), _stream(stream)))
+
+
+class Batch:
+    """Marshalled arguments of lwc_decode_dfloat11_batched, built once and
+    reusable across calls (the layer loop decodes the same tensors again)."""
+
+    def __init__(self, descs, d_ins, d_outs):
+        n = len(descs)
+        if not (len(d_ins) == len(d_outs) == n):
+            raise ValueError("descs, d_ins and d_outs differ in length")
+        self.count = n
+        self.descs = (lwc_desc * max(1, n))(*descs)
+        self.ins = (_P * max(1, n))(*[_addr(x) for x in d_ins])
+        self.outs = (_P * max(1, n))(*[_addr(x) for x in d_outs])
+
+
+def lwc_decode_dfloat11_batched(descs, d_ins=None, d_outs=None, d_status=None, stream=None) -> None:
+    """Decode several DFloat11 tensors (e.g. one transformer layer) at once.
+    ``descs`` may also be a prepared ``Batch`` (then d_ins/d_outs are unused)."""
+    b = descs if isinstance(descs, Batch) else Batch(descs, d_ins, d_outs)
+    _check(load().lwc_decode_dfloat11_batched(b.descs, b.ins, b.outs, b.count, _addr(d_status), _stream(stream)))
+
+
+def lwc_status_string(status: int) -> str:
+    return load().lwc_status_string(status).decode()
+
+
+def lwc_last_error() -> str:
+    return load().lwc_last_error().decode()
+
+
+def lwc_version() -> int:
+    return load().lwc_version()

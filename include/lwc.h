@@ -1,0 +1,202 @@
+/*
+ * lwc.h — C ABI of liblwc: lossless compression of BF16 weight tensors and
+ * their decompression to bit-exact BF16 in GPU memory (NVIDIA B200, sm_100a).
+ *
+ * Two codecs, both lossless:
+ *
+ *  - DFloat11-style ("Koniec z kompromisami! DFloat11 ratuje dokładność
+ *    modeli AI, czyli kompresja, na którą czekałem", section "Przełom:
+ *    DFloat11 – bezstratna kompresja z wydajnością GPU"): each BF16 weight is
+ *    split into its 8-bit exponent, which is Huffman coded per tensor, and one
+ *    raw byte holding its sign and 7 mantissa bits. About 10.6–11 bits/weight.
+ *    The decoder is the GPU kernel of section "Jak to działa w praktyce? Magia
+ *    na poziomie GPU" of the same page: small linked lookup tables in shared
+ *    memory, two phases (threads count their codes, a block scan gives each
+ *    thread its output position, threads decode again and write), and one
+ *    launch for all matrices of a transformer block.
+ *
+ *  - Codebook ("Codebook Lossless Compression: когда 25% памяти значат
+ *    больше, чем кажется", section "Как работает эта магия?"; and
+ *    "無損 LLM 壓縮減少 10-25% RAM", key points): the table of the tensor's U
+ *    distinct 16-bit patterns plus ceil(log2 U)-bit packed indices, decoded by
+ *    table lookup.
+ *
+ * Memory and ownership
+ *  - Encoders run on the host. They malloc the blob; release it with lwc_free.
+ *  - The caller copies the blob, byte for byte, to a device buffer it owns
+ *    (d_in) and keeps the lwc_desc (a plain struct in host memory).
+ *  - Decoders run asynchronously on the caller's CUDA stream and write n
+ *    BF16 values (2n bytes) to the caller's device buffer d_out_bf16.
+ *    They allocate no memory (host or device) and never synchronise.
+ *  - d_in and d_out_bf16 must be 16-byte aligned (else LWC_ERR_MISALIGNED).
+ *
+ * Errors
+ *  - Return values report synchronous checks: arguments, descriptor
+ *    consistency, and cudaGetLastError() after the launch (LWC_ERR_CUDA).
+ *    lwc_last_error() gives a message for the calling thread's last failure.
+ *  - Corrupt device data (a damaged blob whose header is still valid) cannot
+ *    make a decoder read or write outside its buffers or hang; the affected
+ *    outputs are unspecified and, in the *_checked variants, a bit is OR-ed
+ *    into the caller's device status word (LWC_DEVICE_* below). The library
+ *    never traps or asserts on the device.
+ *
+ * Thread safety: all entry points may be called concurrently from several
+ * host threads (the decoders keep only per-device launch configuration,
+ * set once under a lock).
+ */
+#ifndef LWC_H
+#define LWC_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LWC_API __attribute__((visibility("default")))
+#else
+#define LWC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL means the legacy default stream. */
+typedef struct CUstream_st *lwc_stream_t;
+
+typedef enum lwc_status {
+    LWC_OK = 0,
+    LWC_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size or parameter */
+    LWC_ERR_MISALIGNED = 2,   /* device pointer not 16-byte aligned */
+    LWC_ERR_CORRUPT = 3,      /* blob header/descriptor inconsistent */
+    LWC_ERR_UNSUPPORTED = 4,  /* valid but outside what this build decodes */
+    LWC_ERR_NOMEM = 5,        /* host allocation failed (encoders) */
+    LWC_ERR_CUDA = 6          /* CUDA runtime error at launch */
+} lwc_status;
+
+enum {
+    LWC_CODEC_DFLOAT11 = 1,
+    LWC_CODEC_CODEBOOK = 2
+};
+
+/* Bits OR-ed into the optional device status word by the decoders. */
+enum {
+    LWC_DEVICE_BAD_COUNT = 1u,   /* a block decoded a different number of codes than blkoff says */
+    LWC_DEVICE_BAD_CODE = 2u,    /* a lookup-table path that no valid code takes */
+    LWC_DEVICE_BAD_OFFSET = 4u,  /* blkoff out of order, past n, or above max_block_count */
+    LWC_DEVICE_TIMEOUT = 8u      /* a bounded wait on an asynchronous copy gave up */
+};
+
+/* Descriptor of one compressed tensor: a host-side copy of the blob header
+ * (layout of the blob itself: 256-byte little-endian header, then sections at
+ * 16-byte aligned offsets; see the field comments). Plain data, owned by the
+ * caller; fill it with an encoder or with lwc_desc_from_blob. */
+typedef struct lwc_desc {
+    uint32_t magic;            /* 0x3143574C */
+    uint32_t version;          /* 1 */
+    uint32_t codec;            /* LWC_CODEC_* */
+    uint32_t flags;            /* bit 0 (DFloat11): one exponent value only */
+    uint64_t n;                /* number of weights */
+    uint64_t total_bytes;      /* blob size */
+    /* DFloat11 */
+    uint32_t chunk_bytes;      /* bitstream bytes per chunk = per decoding thread */
+    uint32_t threads_per_block;/* chunks per block = threads per CUDA block */
+    uint32_t max_len;          /* longest code length (<= 32) */
+    uint32_t n_tables;         /* 256-entry lookup tables */
+    uint64_t n_chunks;
+    uint64_t n_blocks;
+    uint64_t total_bits;       /* Huffman bitstream length */
+    uint32_t max_block_count;  /* most weights decoded by one block */
+    uint32_t const_exp;        /* exponent when flags bit 0 is set */
+    uint64_t off_lengths;      /* u8[256] code length per exponent value */
+    uint64_t off_lut;          /* u16[n_tables][256] */
+    uint64_t off_gaps;         /* u8[n_blocks * threads_per_block] */
+    uint64_t off_blkoff;       /* u64[n_blocks + 1] */
+    uint64_t off_stream;       /* u32 words, MSB-first codes */
+    uint64_t stream_bytes;
+    uint64_t off_sm;           /* u8[n] sign|mantissa bytes */
+    /* codebook */
+    uint32_t U;                /* table entries */
+    uint32_t k;                /* index bits = ceil(log2 U) */
+    uint64_t off_table;        /* u16[U], ascending */
+    uint64_t off_packed;       /* k-bit indices, LSB first */
+    uint64_t packed_bytes;
+} lwc_desc;
+
+/* DFloat11 encoder parameters; pass NULL for the defaults
+ * (chunk_bytes 36, threads_per_block 256, max_len 32). chunk_bytes: multiple
+ * of 4 in [8, 1024]; threads_per_block: multiple of 32 in [32, 1024];
+ * max_len: code length limit in [9, 32]. */
+typedef struct lwc_df11_params {
+    uint32_t chunk_bytes;
+    uint32_t threads_per_block;
+    uint32_t max_len;
+} lwc_df11_params;
+
+/* ---- host encoders -------------------------------------------------------- */
+
+/* Compress n BF16 bit patterns (h_src, host memory, read only) with the
+ * DFloat11 codec. On LWC_OK, *h_blob_out is a malloc'ed blob of
+ * *blob_bytes_out bytes (release with lwc_free) and *desc_out describes it.
+ * n = 0 gives a header-only blob. Fails only on bad arguments or
+ * LWC_ERR_NOMEM. */
+LWC_API lwc_status lwc_encode_dfloat11(const uint16_t *h_src, uint64_t n, const lwc_df11_params *params,
+                               lwc_desc *desc_out, void **h_blob_out, uint64_t *blob_bytes_out);
+
+/* Compress n BF16 bit patterns with the codebook codec (table of the U
+ * distinct patterns in ascending order + k = ceil(log2 U)-bit indices).
+ * Same ownership and errors as lwc_encode_dfloat11. */
+LWC_API lwc_status lwc_encode_codebook(const uint16_t *h_src, uint64_t n,
+                               lwc_desc *desc_out, void **h_blob_out, uint64_t *blob_bytes_out);
+
+/* Release a blob returned by an encoder (NULL is ignored). */
+LWC_API void lwc_free(void *h_blob);
+
+/* Parse and check the header of a blob held in host memory (h_blob, bytes
+ * long) into *desc_out. LWC_ERR_CORRUPT if the header is inconsistent with
+ * itself or with `bytes`. */
+LWC_API lwc_status lwc_desc_from_blob(const void *h_blob, uint64_t bytes, lwc_desc *desc_out);
+
+/* ---- device decoders (asynchronous on `stream`) --------------------------- */
+
+/* Decode a DFloat11 blob: d_in = the blob in device memory (16-byte aligned),
+ * d_out_bf16 = n outputs (2n bytes, 16-byte aligned). */
+LWC_API lwc_status lwc_decode_dfloat11(const lwc_desc *desc, const void *d_in, uint16_t *d_out_bf16,
+                               lwc_stream_t stream);
+
+/* Decode a codebook blob; arguments as lwc_decode_dfloat11. */
+LWC_API lwc_status lwc_decode_codebook(const lwc_desc *desc, const void *d_in, uint16_t *d_out_bf16,
+                               lwc_stream_t stream);
+
+/* As above, plus d_status: a device uint32 the caller owns (and zeroes); the
+ * decoder ORs LWC_DEVICE_* bits into it when it meets corrupt data. NULL is
+ * allowed. */
+LWC_API lwc_status lwc_decode_dfloat11_checked(const lwc_desc *desc, const void *d_in, uint16_t *d_out_bf16,
+                                       uint32_t *d_status, lwc_stream_t stream);
+LWC_API lwc_status lwc_decode_codebook_checked(const lwc_desc *desc, const void *d_in, uint16_t *d_out_bf16,
+                                       uint32_t *d_status, lwc_stream_t stream);
+
+/* Decode `count` DFloat11 tensors — e.g. all matrices of one transformer
+ * block (DF11 page, section "Jak to działa w praktyce?", third pillar) — in
+ * as few launches as possible (one per distinct (chunk_bytes,
+ * threads_per_block) pair among them, plus one for tensors with a single
+ * exponent value). descs[i], d_ins[i], d_outs[i] as for lwc_decode_dfloat11;
+ * d_status optional. */
+LWC_API lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const *d_ins,
+                                       uint16_t *const *d_outs, int count, uint32_t *d_status,
+                                       lwc_stream_t stream);
+
+/* ---- helpers -------------------------------------------------------------- */
+
+/* Static string naming a status code. */
+LWC_API const char *lwc_status_string(lwc_status s);
+
+/* Message describing the calling thread's last failed call ("" if none). */
+LWC_API const char *lwc_last_error(void);
+
+/* Library version as 10000*major + 100*minor + patch. */
+LWC_API int lwc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LWC_H */

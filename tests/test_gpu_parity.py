@@ -1,0 +1,237 @@
+"""GPU decoders against the oracle, bit for bit, through the C ABI.
+
+Small cases span many blocks/tiles with ragged tails; the full-size cases use
+the workloads' own sizes (one Llama-3-8B layer, the 256M-weight codebook and
+uniform-exponent stress tensors) with the launch configuration the benchmark
+times. Every comparison is on 16-bit patterns (never float ==)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from decode_dfloat11_b200 import build as lwc_build
+from decode_dfloat11_b200 import lwc
+from oracle import codebook as ocb
+from oracle import df11 as odf
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib(cuda_device):
+    lwc_build.build()
+    return lwc.load()
+
+
+def dev(blob: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(blob).to("cuda")
+
+
+def host_u16(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def gpu_decode(desc, blob_dev, codec="df11", status=None):
+    out = torch.empty(desc.n, dtype=torch.int16, device="cuda")
+    st = torch.cuda.current_stream()
+    if codec == "df11":
+        lwc.lwc_decode_dfloat11_checked(desc, blob_dev, out, status, st)
+    else:
+        lwc.lwc_decode_codebook_checked(desc, blob_dev, out, status, st)
+    torch.cuda.synchronize()
+    return out
+
+
+def small_inputs():
+    yield "config1", synth.as_u16(synth.small_square(0))
+    yield "uniform", synth.as_u16(synth.uniform_patterns(300_001, seed=1))
+    yield "all_patterns", synth.as_u16(synth.all_patterns())
+    yield "outliers", synth.as_u16(synth.normal_bf16((777_777,), seed=2, sigma=0.01, outlier_frac=1e-2))
+    yield "narrow", synth.as_u16(synth.normal_bf16((500_000,), seed=3, sigma=1e-3))
+    yield "single_exp", (np.arange(100_003, dtype=np.uint16) & 0x807F) | 0x3F00
+    yield "zeros", np.zeros(4097, np.uint16)
+    for n in (1, 2, 3, 15, 16, 17, 31, 33, 255, 257, 4095, 65537):
+        yield f"n{n}", synth.as_u16(synth.normal_bf16((n,), seed=n, sigma=0.02))
+
+
+@pytest.mark.parametrize("name,w", list(small_inputs()), ids=lambda x: x if isinstance(x, str) else "")
+def test_df11_small(name, w):
+    d, b = lwc.lwc_encode_dfloat11(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = host_u16(gpu_decode(d, dev(b), status=status))
+    assert int(status.item()) == 0
+    assert np.array_equal(got, odf.decode(b))
+    assert np.array_equal(got, w)
+    # the oracle's own blob decodes the same on the GPU
+    ob = odf.encode(w)
+    od = lwc.lwc_desc_from_blob(ob)
+    assert np.array_equal(host_u16(gpu_decode(od, dev(ob))), w)
+
+
+@pytest.mark.parametrize("chunk_bytes,tpb", [(8, 32), (12, 64), (20, 96), (36, 256), (64, 128), (36, 512),
+                                             (36, 1024)])
+def test_df11_block_parameters(chunk_bytes, tpb):
+    w = synth.as_u16(synth.normal_bf16((1_234_567,), seed=4, sigma=0.02, outlier_frac=1e-3))
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    got = host_u16(gpu_decode(d, dev(b)))
+    assert np.array_equal(got, odf.decode(b))
+    ob = odf.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    assert np.array_equal(host_u16(gpu_decode(lwc.lwc_desc_from_blob(ob), dev(ob))), w)
+
+
+def test_df11_long_codes():
+    # Fibonacci counts push codes to the length limit: the hierarchical tables
+    # go 4 levels deep and the fast table misses often
+    fib = [1, 1]
+    while len(fib) < 40:
+        fib.append(fib[-1] + fib[-2])
+    counts = np.array(fib[:40], np.int64) // 500 + 1
+    w = np.repeat((np.arange(40, dtype=np.uint16) << 7) | 0x8011, counts)
+    w = np.random.default_rng(0).permutation(w).astype(np.uint16)
+    for limit in (32, 24, 16):
+        d, b = lwc.lwc_encode_dfloat11(w, max_len=limit)
+        assert d.max_len == limit
+        assert np.array_equal(host_u16(gpu_decode(d, dev(b))), w)
+
+
+@pytest.mark.parametrize("name,w", list(small_inputs()), ids=lambda x: x if isinstance(x, str) else "")
+def test_codebook_small(name, w):
+    d, b = lwc.lwc_encode_codebook(w)
+    got = host_u16(gpu_decode(d, dev(b), codec="cb"))
+    assert np.array_equal(got, ocb.decode(b))
+    assert np.array_equal(got, w)
+
+
+@pytest.mark.parametrize("U", [1, 2, 3, 5, 17, 200, 256, 600, 2000, 4096, 5000, 8192, 20000, 40000, 65536])
+def test_codebook_every_width(U):
+    n = 3 * 8192 + 77
+    if U == 65536:
+        w = synth.as_u16(synth.uniform_patterns(200_000, seed=U))
+        w[:65536] = np.arange(65536, dtype=np.uint16)
+    else:
+        w = synth.as_u16(synth.codebook_stress(U, n, seed=U))
+    d, b = lwc.lwc_encode_codebook(w)
+    assert d.U == len(np.unique(w))
+    got = host_u16(gpu_decode(d, dev(b), codec="cb"))
+    assert np.array_equal(got, ocb.decode(b))
+
+
+def test_batched_mixed():
+    tensors = [
+        synth.as_u16(synth.normal_bf16((300_000,), seed=10, sigma=0.02)),
+        (np.arange(5000, dtype=np.uint16) & 0x807F) | 0x3E80,           # single exponent
+        np.zeros(0, np.uint16),
+        synth.as_u16(synth.uniform_patterns(99_999, seed=11)),
+        synth.as_u16(synth.normal_bf16((77,), seed=12, sigma=0.5)),
+    ]
+    params = [dict(), dict(), dict(), dict(chunk_bytes=12, threads_per_block=64), dict()]
+    enc = [lwc.lwc_encode_dfloat11(w, **p) for w, p in zip(tensors, params)]
+    blobs = [dev(b) for _, b in enc]
+    outs = [torch.full((max(1, w.size),), 0x5555, dtype=torch.int16, device="cuda") for w in tensors]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_batched([d for d, _ in enc], blobs, outs, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for w, o in zip(tensors, outs):
+        assert np.array_equal(host_u16(o)[:w.size], w)
+
+
+def test_side_stream_and_reuse():
+    w = synth.as_u16(synth.small_square(5))
+    d, b = lwc.lwc_encode_dfloat11(w)
+    bd = dev(b)
+    s = torch.cuda.Stream()
+    outs = [torch.empty(w.size, dtype=torch.int16, device="cuda") for _ in range(3)]
+    with torch.cuda.stream(s):
+        for o in outs:
+            lwc.lwc_decode_dfloat11(d, bd, o, s)
+    s.synchronize()
+    for o in outs:
+        assert np.array_equal(host_u16(o), w)
+
+
+def test_df11_corruption_is_contained():
+    w = synth.as_u16(synth.small_square(6))
+    d, b = lwc.lwc_encode_dfloat11(w)
+    rng = np.random.default_rng(0)
+    guard = 4096
+    cases = []
+    x = b.copy()                                   # payload bit flips
+    pos = d.off_stream + rng.integers(0, (d.total_bits + 7) // 8, 50)
+    x[pos] ^= np.uint8(0x10)
+    cases.append(x)
+    x = b.copy()                                   # block offsets out of range
+    x[d.off_blkoff + 8 * 3: d.off_blkoff + 8 * 4] = np.array([2 ** 40], np.uint64).view(np.uint8)
+    cases.append(x)
+    x = b.copy()                                   # every lookup entry invalid
+    x[d.off_lut: d.off_lut + 512 * d.n_tables] = 0xFF
+    cases.append(x)
+    x = b.copy()                                   # gaps garbage
+    x[d.off_gaps: d.off_gaps + d.n_blocks * d.threads_per_block] = rng.integers(0, 256, d.n_blocks * 256)
+    cases.append(x)
+    for i, x in enumerate(cases):
+        xd = dev(x)
+        out = torch.zeros(w.size + 2 * guard, dtype=torch.int16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        lwc.lwc_decode_dfloat11_checked(d, xd, out[guard:guard + w.size], status, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        got = host_u16(out)
+        assert np.all(got[:guard] == 0) and np.all(got[guard + w.size:] == 0), i   # nothing outside
+        assert int(status.item()) != 0 or not np.array_equal(got[guard:guard + w.size], w) or i == 0, i
+        if i in (1, 2):
+            assert int(status.item()) != 0, i
+
+
+# ------------------------------------------------------------ full-size configs
+
+def test_llama3_8b_layer_full_size():
+    """One Llama-3-8B layer (218,103,808 weights), DFloat11: per-tensor and
+    layer-batched decodes, each compared with the oracle's decode of the same
+    blob element by element."""
+    tensors = [synth.as_u16(t) for _, t in synth.llama_layer_tensors(0)]
+    enc = [lwc.lwc_encode_dfloat11(w) for w in tensors]
+    blobs = [dev(b) for _, b in enc]
+    outs = [torch.empty(w.size, dtype=torch.int16, device="cuda") for w in tensors]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_batched([d for d, _ in enc], blobs, outs, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for (d, b), w, o in zip(enc, tensors, outs):
+        got = host_u16(o)
+        assert np.array_equal(got, odf.decode(b))
+        assert np.array_equal(got, w)
+        o.zero_()
+        lwc.lwc_decode_dfloat11(d, dev(b), o, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        assert np.array_equal(host_u16(o), w)
+    bpw = 8.0 * sum(d.total_bytes for d, _ in enc) / sum(w.size for w in tensors)
+    assert 10.0 < bpw < 11.5
+
+
+@pytest.mark.parametrize("U", [256, 4096, 8192, 65536])
+def test_codebook_stress_full_size(U):
+    """256M weights from a U-entry table with Zipf(1.1) frequencies."""
+    n = 1 << 28
+    x = synth.codebook_stress(U, n, seed=40 + U, device="cuda")
+    w = synth.as_u16(x)
+    d, b = lwc.lwc_encode_codebook(w)
+    assert d.k == {256: 8, 4096: 12, 8192: 13, 65536: 16}[U] or d.U < U
+    out = gpu_decode(d, dev(b), codec="cb")
+    assert torch.equal(out, x.view(torch.int16))
+    # sampled windows, each read independently by the oracle
+    rng = np.random.default_rng(U)
+    got = host_u16(out)
+    for i0 in list(rng.integers(0, n - 4096, 24)) + [n - 4096]:
+        assert np.array_equal(got[i0:i0 + 4096], ocb.decode_range(b, int(i0), 4096))
+
+
+def test_df11_uniform_exponents_full_size():
+    """256M uniformly random patterns: all 256 exponents, 8-bit codes (an
+    expansion to ~16 bits/weight), the decoder's worst table case."""
+    n = 1 << 28
+    x = synth.uniform_patterns(n, seed=77, device="cuda")
+    w = synth.as_u16(x)
+    d, b = lwc.lwc_encode_dfloat11(w)
+    out = gpu_decode(d, dev(b))
+    assert torch.equal(out, x.view(torch.int16))
+    assert np.array_equal(host_u16(out), odf.decode(b))

@@ -1,0 +1,199 @@
+"""Host side of liblwc, no GPU needed: the library loads and exports every
+symbol include/lwc.h declares; its encoders' blobs decode in the oracle (and
+pass the oracle's re-derivation of gaps, block offsets and lookup tables);
+it parses the oracle's blobs; and it rejects damaged headers and bad
+arguments before touching a device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from conftest import ROOT
+from decode_dfloat11_b200 import build as lwc_build
+from decode_dfloat11_b200 import lwc
+from oracle import blob as B
+from oracle import codebook as ocb
+from oracle import df11 as odf
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    lwc_build.build()
+    return lwc.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "lwc.h")).read()
+    return sorted(set(re.findall(r"LWC_API\s+[\w\s\*]+?\b(lwc_\w+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    names = declared_symbols()
+    assert len(names) >= 12
+    L = lwc.load()
+    for name in names:
+        assert hasattr(L, name), name
+    assert set(names) == set(lwc.EXPORTED)
+    assert lwc.lwc_version() == 10000
+    assert lwc.lwc_status_string(3) == "corrupt blob or descriptor"
+
+
+def df11_inputs():
+    yield "config1", synth.as_u16(synth.small_square(0))
+    yield "uniform", synth.as_u16(synth.uniform_patterns(300_001, seed=1))
+    yield "all_patterns", synth.as_u16(synth.all_patterns())
+    yield "outliers", synth.as_u16(synth.normal_bf16((777_777,), seed=2, sigma=0.01, outlier_frac=1e-2))
+    yield "single_exp", (np.arange(10_000, dtype=np.uint16) & 0x807F) | 0x3F00
+    yield "zeros", np.zeros(123, np.uint16)
+    yield "empty", np.zeros(0, np.uint16)
+    for n in (1, 2, 3, 7, 31, 33, 255, 257):
+        yield f"n{n}", synth.as_u16(synth.uniform_patterns(n, seed=n))
+
+
+@pytest.mark.parametrize("name,w", list(df11_inputs()), ids=lambda x: x if isinstance(x, str) else "")
+def test_library_df11_blob_decodes_in_oracle(name, w):
+    d, b = lwc.lwc_encode_dfloat11(w)
+    assert d.total_bytes == b.size and d.n == w.size
+    assert np.array_equal(odf.decode(b), w)
+    assert odf.check_index(b) == []
+    assert lwc.lwc_desc_from_blob(b).as_dict() == d.as_dict()
+
+
+@pytest.mark.parametrize("chunk_bytes,tpb", [(8, 32), (12, 64), (36, 256), (64, 128), (36, 1024), (100, 512)])
+def test_library_df11_parameters(chunk_bytes, tpb):
+    w = synth.as_u16(synth.normal_bf16((250_007,), seed=5, sigma=0.02, outlier_frac=1e-3))
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    assert (d.chunk_bytes, d.threads_per_block) == (chunk_bytes, tpb)
+    assert np.array_equal(odf.decode(b), w)
+    assert odf.check_index(b) == []
+
+
+def test_library_code_is_optimal_like_the_oracle():
+    # both encoders build an optimal code: same total bits, possibly other codewords
+    for seed in range(3):
+        w = synth.as_u16(synth.normal_bf16((400_000,), seed=seed, sigma_range=(0.005, 0.04),
+                                           outlier_frac=1e-3))
+        d, _ = lwc.lwc_encode_dfloat11(w)
+        oh = B.unpack_header(odf.encode(w))
+        assert d.total_bits == oh["total_bits"]
+
+
+def test_library_length_limit():
+    # Fibonacci counts: a Huffman tree 39 deep; the library must limit it
+    fib = [1, 1]
+    while len(fib) < 40:
+        fib.append(fib[-1] + fib[-2])
+    counts = np.array(fib[:40], np.int64) // 1000 + 1
+    w = np.repeat((np.arange(40, dtype=np.uint16) << 7) | 0x8005, counts)
+    w = np.random.default_rng(0).permutation(w).astype(np.uint16)
+    for limit in (32, 16, 12):
+        d, b = lwc.lwc_encode_dfloat11(w, max_len=limit)
+        assert d.max_len <= limit
+        assert np.array_equal(odf.decode(b), w)
+        assert odf.check_index(b) == []
+
+
+@pytest.mark.parametrize("U", [1, 2, 3, 255, 256, 257, 4096, 8192, 65536])
+def test_library_codebook_blob_decodes_in_oracle(U):
+    n = 70_001 if U < 65536 else 300_000
+    w = synth.as_u16(synth.codebook_stress(U, n, seed=U)) if U < 65536 else \
+        synth.as_u16(synth.uniform_patterns(n, seed=9))
+    d, b = lwc.lwc_encode_codebook(w)
+    assert d.U == len(np.unique(w)) and d.k == ocb.index_bits(d.U)
+    assert np.array_equal(ocb.decode(b), w)
+    # same layout rule, same table, same packing: the bytes agree with the oracle's
+    assert np.array_equal(b, ocb.encode(w))
+
+
+def test_library_parses_oracle_blobs():
+    w = synth.as_u16(synth.small_square(3))
+    ob = odf.encode(w, chunk_bytes=20, threads_per_block=96)
+    d = lwc.lwc_desc_from_blob(ob)
+    h = B.unpack_header(ob)
+    for key, val in h.items():
+        if key in ("header_bytes",):
+            continue
+        assert getattr(d, key) == val, key
+    oc = ocb.encode(w)
+    dc = lwc.lwc_desc_from_blob(oc)
+    assert (dc.U, dc.k, dc.n) == (B.unpack_header(oc)["U"], B.unpack_header(oc)["k"], w.size)
+
+
+def corrupt(blob, off, fmt, value):
+    b = blob.copy()
+    b[off:off + np.dtype(fmt).itemsize] = np.array([value], fmt).view(np.uint8)
+    return b
+
+
+def test_damaged_headers_are_rejected():
+    w = synth.as_u16(synth.small_square(1))
+    _, b = lwc.lwc_encode_dfloat11(w)
+    h = B.unpack_header(b)
+    bad = [
+        corrupt(b, 0, "<u4", 0x12345678),                 # magic
+        corrupt(b, 4, "<u2", 2),                          # version
+        corrupt(b, 16, "<u8", h["total_bytes"] + 16),     # size mismatch
+        corrupt(b, 32, "<u4", 30),                        # chunk_bytes not a multiple of 4
+        corrupt(b, 36, "<u4", 48),                        # threads_per_block not a multiple of 32
+        corrupt(b, 40, "<u4", 40),                        # max_len beyond the format
+        corrupt(b, 48, "<u8", h["n_chunks"] + 1),         # chunk count
+        corrupt(b, 56, "<u8", h["n_blocks"] + 1),         # block count
+        corrupt(b, 64, "<u8", 8),                         # total_bits below n
+        corrupt(b, 72, "<u4", 0),                         # max_block_count
+        corrupt(b, 112, "<u8", h["total_bytes"] - 16),    # stream outside the blob
+        corrupt(b, 128, "<u8", 8),                        # misaligned section
+    ]
+    for i, x in enumerate(bad):
+        with pytest.raises(lwc.LwcError) as e:
+            lwc.lwc_desc_from_blob(x)
+        assert e.value.status == 3, i
+    with pytest.raises(lwc.LwcError):
+        lwc.lwc_desc_from_blob(b[:100])
+    _, c = lwc.lwc_encode_codebook(w)
+    for x in (corrupt(c, 36, "<u4", 11), corrupt(c, 32, "<u4", 100_000), corrupt(c, 56, "<u8", 16)):
+        with pytest.raises(lwc.LwcError) as e:
+            lwc.lwc_desc_from_blob(x)
+        assert e.value.status == 3
+
+
+def test_decoders_validate_before_any_device_call():
+    w = synth.as_u16(synth.small_square(2))
+    d, _ = lwc.lwc_encode_dfloat11(w)
+    dc, _ = lwc.lwc_encode_codebook(w)
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_decode_dfloat11(d, 0x1008, 0x2000)          # misaligned input
+    assert e.value.status == 2
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_decode_codebook(dc, 0x1000, 0x2002)         # misaligned output
+    assert e.value.status == 2
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_decode_dfloat11(dc, 0x1000, 0x2000)         # wrong codec
+    assert e.value.status == 1
+    bad = lwc.lwc_desc.from_buffer_copy(d)
+    bad.n_blocks += 1
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_decode_dfloat11(bad, 0x1000, 0x2000)
+    assert e.value.status == 3
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_decode_dfloat11_batched([d, d], [0x1000, None], [0x2000, 0x3000])
+    assert e.value.status == 1
+    # empty tensors need no device at all
+    d0, _ = lwc.lwc_encode_dfloat11(np.zeros(0, np.uint16))
+    lwc.lwc_decode_dfloat11(d0, None, None)
+    c0, _ = lwc.lwc_encode_codebook(np.zeros(0, np.uint16))
+    lwc.lwc_decode_codebook(c0, None, None)
+
+
+def test_encoder_rejects_bad_arguments():
+    w = np.zeros(10, np.uint16)
+    for kw in (dict(chunk_bytes=6), dict(chunk_bytes=10), dict(threads_per_block=48),
+               dict(threads_per_block=2048), dict(max_len=8), dict(max_len=33)):
+        with pytest.raises(lwc.LwcError) as e:
+            lwc.lwc_encode_dfloat11(w, **kw)
+        assert e.value.status == 1
+    L = lwc.load()
+    desc = lwc.lwc_desc()
+    assert L.lwc_encode_dfloat11(None, 5, None, ctypes.byref(desc), None, None) == 1
