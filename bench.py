@@ -150,6 +150,29 @@ def gpu_id_for(device) -> str:
     return str(device.index or 0)
 
 
+# ---------------------------------------------------------------- ranks
+
+def rank_layer(rank: int, layer_arg) -> int:
+    """Layer (seed) a rank decodes: its own, so replicas hold different data."""
+    return layer_arg if layer_arg is not None else rank
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    """Largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank: int, ms_per_step: float) -> float:
+    """Aggregate GB/s when every rank moves bytes_per_rank per step and the
+    step takes ms_per_step on the slowest rank."""
+    return world * bytes_per_rank / (ms_per_step * 1e-3) / 1e9
+
+
 # ---------------------------------------------------------------- setup
 
 def make_layer(layer: int):
@@ -208,7 +231,7 @@ def run_lwc(args, rank, world, local_rank, dist):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    layer = args.layer if args.layer is not None else rank
+    layer = rank_layer(rank, args.layer)
 
     names, tensors = make_layer(layer)
     n_total = sum(w.size for w in tensors)
@@ -256,13 +279,8 @@ def run_lwc(args, rank, world, local_rank, dist):
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    ms_max = ms
-    if dist:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
-    ms_per_step = ms_max / args.steps
-    value = world * 2 * n_total / (ms_per_step * 1e-3) / 1e9
+    ms_per_step = max_over_ranks(ms, dist, device) / args.steps
+    value = whole_job_gbs(world, 2 * n_total, ms_per_step)
 
     # roofline of the decode kernel (one launch per step here)
     peak, peak_kind = measured_peak()
@@ -335,11 +353,7 @@ def run_lwc(args, rank, world, local_rank, dist):
         if not torch.equal(pinned_out.view(torch.int16)[:tensors[0].size],
                            torch.from_numpy(tensors[0].view(np.int16))):
             raise SystemExit("end-to-end output differs from its input")
-        ev = world * 2 * n_total / (ems * 1e-3) / 1e9
-        if dist:
-            t = torch.tensor([ems], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ev = world * 2 * n_total / (float(t.item()) * 1e-3) / 1e9
+        ev = whole_job_gbs(world, 2 * n_total, max_over_ranks(ems, dist, device))
         result["e2e"] = {"value": round(ev, 3), "unit": "GB/s", "h2d_bytes_per_step": blob_bytes,
                          "d2h_bytes_per_step": 2 * n_total, "ms_per_step": round(ems, 4), "steps": e_steps}
 

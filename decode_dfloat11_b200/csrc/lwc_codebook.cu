@@ -133,7 +133,9 @@ __global__ void __launch_bounds__(kThreads) cb_decode_kernel(const __grid_consta
         }
         const bool ok = dev::mbar_wait_bounded(&bars[buf], (it >> 1) & 1u);
         if (__syncthreads_or(!ok)) {
+            // let the copy already issued for the next tile land (bounded) before leaving
             timed_out = 1;
+            if (t + 1 < t_end) dev::mbar_wait_bounded(&bars[buf ^ 1u], ((it + 1) >> 1) & 1u);
             break;
         }
         uint32_t w[K + 1];

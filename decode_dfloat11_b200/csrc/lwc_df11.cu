@@ -20,6 +20,12 @@
 //    of items and rebuild their tables only when the tensor changes.
 // Blocks never wait on one another: each block's first output index is stored
 // in the blob, so there is no inter-block scan.
+//
+// Memory pipeline per CTA: while item j is decoded, the bulk-copy (TMA)
+// engine brings the stream segment and chunk gaps of item j+1 into the other
+// half of a shared-memory double buffer, and the sign|mantissa bytes of item
+// j+1 are prefetched into L2, so the merge of j+1 reads them from L2. Block
+// offsets are loaded two items ahead. No wait is unbounded.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -47,7 +53,7 @@ struct Df11Tensor {
     uint16_t *out;
     uint64_t n;
     uint64_t total_bits;
-    uint64_t stream_words;
+    uint64_t stream_bytes;
     uint32_t n_blocks;
     uint32_t n_tables;
     uint32_t first_work;   // index of this tensor's block 0 in the launch's work list
@@ -60,18 +66,33 @@ struct Df11Batch {
     uint32_t total_work;
     uint32_t chunk_words;  // chunk_bytes / 4
     uint32_t seg_words;    // words staged per block: T * chunk_words + 2, rounded up to 4
-    uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 16)
+    uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 32)
     uint32_t lut_entries;  // lookup-table entries reserved in shared memory
     uint32_t *status;
 };
 
+// Shared-memory layout of one CTA (T threads); every offset a multiple of 16.
+struct Layout {
+    uint32_t lut, bufs, buf_bytes, stage, sums, bars, total;
+    __host__ __device__ Layout(uint32_t T, uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes) {
+        lut = kFastBytes;
+        bufs = lut + 2 * lut_entries;
+        buf_bytes = 4 * seg_words + T;   // segment words, then T gap bytes
+        stage = bufs + 2 * buf_bytes;
+        sums = stage + stage_bytes;
+        bars = sums + 128;
+        total = bars + 16;
+    }
+};
+
 // ---- lookup tables ---------------------------------------------------------
 
-// Walk the hierarchical tables with the window's top bits; returns
-// symbol | length << 8. A path no valid code takes yields length 1 and sets
-// LWC_DEVICE_BAD_CODE in `bad` (so decoding always advances and ends).
-__device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab, uint64_t win, uint32_t &bad) {
-    uint32_t e = lut[win >> 56];
+// Walk the hierarchical tables with the 32 stream bits at the current
+// position (MSB first); returns symbol | length << 8. A path no valid code
+// takes yields length 1 and sets LWC_DEVICE_BAD_CODE in `bad` (so decoding
+// always advances and ends).
+__device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab, uint32_t w, uint32_t &bad) {
+    uint32_t e = lut[w >> 24];
 #pragma unroll 1
     for (int d = 1; (e & 0x8000u) && d < 4; d++) {
         const uint32_t t = e & 0x7FFFu;
@@ -79,7 +100,7 @@ __device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab,
             bad |= LWC_DEVICE_BAD_CODE;
             return 0x100u;
         }
-        e = lut[t * 256u + (uint32_t)((win >> (56 - 8 * d)) & 0xFFu)];
+        e = lut[t * 256u + ((w >> (24 - 8 * d)) & 0xFFu)];
     }
     const uint32_t len = (e >> 8) & 0x3Fu;
     if ((e & 0x8000u) || len == 0 || len > 32) {
@@ -90,12 +111,15 @@ __device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab,
 }
 
 // Fast tables, indexed by the next 12 stream bits:
-//  cnt_tab[v] = count << 4 | bits, for all whole codes inside the 12 bits;
+//  cnt_tab[v] = count << 4 | bits, for all whole codes inside the 12 bits
+//               (entries are summed: the sum of the `bits` parts is known, so
+//               one add per lookup counts codes);
 //  sym_tab[v] = sym0 | sym1 << 8 | sym2 << 16 | n << 24 | bits << 26, for the
-//               first n <= 3 of them. 0 means "first code longer than 12 bits".
+//               first n <= 3 of them.
+// 0 means "the first code is longer than 12 bits".
 __device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *cnt_tab, uint32_t *sym_tab) {
     for (uint32_t v = threadIdx.x; v < kFastSize; v += blockDim.x) {
-        uint64_t w = (uint64_t)v << (64 - kFastBits);
+        uint32_t w = v << (32 - kFastBits);
         uint32_t used = 0, cnt = 0, syms = 0, n3 = 0, used3 = 0, ignore = 0;
         while (cnt < (uint32_t)kFastBits) {
             const uint32_t r = lut_walk(lut, ntab, w, ignore);
@@ -115,69 +139,11 @@ __device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *c
     }
 }
 
-// ---- bit window --------------------------------------------------------------
-
-// 64-bit window over the staged segment, MSB = next stream bit. Holds >= 32
-// valid bits before every decode step.
-struct BitWindow {
-    uint64_t win;
-    uint32_t nb;   // valid bits
-    uint32_t wp;   // next word to load
-    __device__ __forceinline__ void init(const uint32_t *seg, uint32_t bit) {
-        wp = bit >> 5;
-        const uint64_t w = ((uint64_t)seg[wp] << 32) | seg[wp + 1];
-        const uint32_t sh = bit & 31u;
-        win = w << sh;
-        nb = 64 - sh;
-        wp += 2;
-    }
-    __device__ __forceinline__ void consume(const uint32_t *seg, uint32_t len) {
-        win <<= len;
-        nb -= len;
-        if (nb < 32) {
-            win |= (uint64_t)seg[wp++] << (32 - nb);
-            nb += 32;
-        }
-    }
-};
-
-// Exponent writer for pass 2: gathers bytes into 32-bit words so that most
-// shared-memory stores are whole words; the first and last partial words of a
-// thread's range are written byte by byte (their other bytes belong to the
-// neighbouring threads).
-struct StageWriter {
-    uint8_t *base;
-    uint32_t wpos;   // byte offset of acc's byte 0 (multiple of 4)
-    uint32_t head;   // bytes of the first word owned by the previous thread
-    uint32_t fill;   // bytes held in acc, counting the head
-    uint64_t acc;
-    __device__ __forceinline__ void init(uint8_t *b, uint32_t p) {
-        base = b;
-        wpos = p & ~3u;
-        head = p & 3u;
-        fill = head;
-        acc = 0;
-    }
-    __device__ __forceinline__ void put(uint32_t syms, uint32_t n) {
-        acc |= (uint64_t)syms << (8 * fill);
-        fill += n;
-        if (fill >= 4) {
-            const uint32_t w = (uint32_t)acc;
-            if (head) {
-                for (uint32_t j = head; j < 4; j++) base[wpos + j] = (uint8_t)(w >> (8 * j));
-                head = 0;
-            } else {
-                *reinterpret_cast<uint32_t *>(base + wpos) = w;
-            }
-            wpos += 4;
-            acc >>= 32;
-            fill -= 4;
-        }
-    }
-    __device__ __forceinline__ void finish() {
-        for (uint32_t j = head; j < fill; j++) base[wpos + j] = (uint8_t)(acc >> (8 * j));
-    }
-};
+// The 32 stream bits starting at bit `pos` of the staged segment.
+__device__ __forceinline__ uint32_t window32(const uint32_t *seg, uint32_t pos) {
+    const uint32_t i = pos >> 5;
+    return __funnelshift_l(seg[i + 1], seg[i], pos & 31u);
+}
 
 // ---- merge ---------------------------------------------------------------------
 
@@ -190,6 +156,20 @@ __device__ __forceinline__ uint32_t merge2(uint32_t s, uint32_t e, uint32_t sel)
 
 __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e) {
     return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
+}
+
+__device__ __forceinline__ void merge16(const uint4 &s, const uint4 &e, uint16_t *dst) {
+    uint4 r0, r1;
+    r0.x = merge2(s.x, e.x, 0x5140u);
+    r0.y = merge2(s.x, e.x, 0x7362u);
+    r0.z = merge2(s.y, e.y, 0x5140u);
+    r0.w = merge2(s.y, e.y, 0x7362u);
+    r1.x = merge2(s.z, e.z, 0x5140u);
+    r1.y = merge2(s.z, e.z, 0x7362u);
+    r1.z = merge2(s.w, e.w, 0x5140u);
+    r1.w = merge2(s.w, e.w, 0x7362u);
+    reinterpret_cast<uint4 *>(dst)[0] = r0;
+    reinterpret_cast<uint4 *>(dst)[1] = r1;
 }
 
 // ---- block scan ------------------------------------------------------------------
@@ -216,8 +196,33 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
     __syncthreads();
     total = warp_sums[nwarps - 1];
     const uint32_t before = warp ? warp_sums[warp - 1] : 0u;
-    __syncthreads();   // warp_sums is reused by the next scan
     return before + x - v;
+}
+
+// ---- work list ----------------------------------------------------------------------
+
+// Advance ti (monotonically) to the tensor that owns work item w.
+__device__ __forceinline__ uint32_t locate(const Df11Batch &B, uint32_t w, uint32_t ti) {
+    while (ti + 1 < B.count && w >= B.t[ti + 1].first_work) ++ti;
+    return ti;
+}
+
+// Thread 0: start the bulk copies of item (ti, b) into buffer `buf`, and
+// prefetch its sign|mantissa bytes [o0, o1) into L2.
+__device__ __forceinline__ void issue_item(const Df11Batch &B, uint32_t ti, uint32_t b, uint64_t o0, uint64_t o1,
+                                           uint8_t *buf, uint32_t seg_bytes, uint64_t *bar) {
+    const Df11Tensor &tn = B.t[ti];
+    const uint32_t T = blockDim.x;
+    const uint64_t seg0 = (uint64_t)b * T * B.chunk_words * 4;   // byte offset, multiple of 128
+    const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
+    const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
+    dev::mbar_arrive_expect_tx(bar, bytes + T);
+    if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
+    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * T, T, bar);
+    if (o0 < o1 && o1 <= tn.n) {
+        const uint64_t a = o0 & ~15ull, z = (o1 + 15) & ~15ull;
+        dev::prefetch_l2(tn.sm + a, (uint32_t)min(z - a, (uint64_t)0x7FFFFFF0ull));
+    }
 }
 
 // ---- the kernel -------------------------------------------------------------------
@@ -226,150 +231,209 @@ template <int kMaxThreads>
 __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048 / kMaxThreads / 2 : 1)
     df11_decode_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t T = blockDim.x, tid = threadIdx.x;
+    const Layout L(T, B.seg_words, B.lut_entries, B.stage_bytes);
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem);
     uint8_t *cnt_tab = smem + kFastSize * 4;
-    uint16_t *lut = reinterpret_cast<uint16_t *>(smem + kFastBytes);
-    uint32_t *seg = reinterpret_cast<uint32_t *>(smem + kFastBytes + 2 * B.lut_entries);
-    uint8_t *stage = reinterpret_cast<uint8_t *>(seg + B.seg_words);
-    uint32_t *warp_sums = reinterpret_cast<uint32_t *>(stage + B.stage_bytes);
+    uint16_t *lut = reinterpret_cast<uint16_t *>(smem + L.lut);
+    uint8_t *stage = smem + L.stage;
+    uint32_t *warp_sums = reinterpret_cast<uint32_t *>(smem + L.sums);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L.bars);
+    const uint32_t seg_bytes = 4 * B.seg_words;
 
-    const uint32_t T = blockDim.x, tid = threadIdx.x;
     const uint32_t CW = B.chunk_words, cbits = CW * 32u;
     const uint32_t W = B.total_work, G = gridDim.x;
     const uint32_t w_begin = (uint32_t)((uint64_t)W * blockIdx.x / G);
     const uint32_t w_end = (uint32_t)((uint64_t)W * (blockIdx.x + 1) / G);
+    if (w_begin >= w_end) return;
+
+    // block offsets of the current item and the next one
+    uint32_t ti = locate(B, w_begin, 0);
+    uint64_t o0c, o1c, o0n = 0, o1n = 0;
+    {
+        const uint32_t b = w_begin - B.t[ti].first_work;
+        o0c = B.t[ti].blkoff[b];
+        o1c = B.t[ti].blkoff[b + 1];
+    }
+    uint32_t tn1 = ti;
+    if (w_begin + 1 < w_end) {
+        tn1 = locate(B, w_begin + 1, ti);
+        const uint32_t b = w_begin + 1 - B.t[tn1].first_work;
+        o0n = B.t[tn1].blkoff[b];
+        o1n = B.t[tn1].blkoff[b + 1];
+    }
+    if (tid == 0) {
+        dev::mbar_init(&bars[0], 1);
+        dev::mbar_init(&bars[1], 1);
+        dev::fence_mbar_init();
+        issue_item(B, ti, w_begin - B.t[ti].first_work, o0c, o1c, smem + L.bufs, seg_bytes, &bars[0]);
+        if (w_begin + 1 < w_end)
+            issue_item(B, tn1, w_begin + 1 - B.t[tn1].first_work, o0n, o1n, smem + L.bufs + L.buf_bytes,
+                       seg_bytes, &bars[1]);
+    }
 
     uint32_t bad = 0;
     int cur = -1;
-    uint32_t ti = 0;
     for (uint32_t w = w_begin; w < w_end; ++w) {
-        while (ti + 1 < B.count && w >= B.t[ti + 1].first_work) ++ti;
+        const uint32_t it = w - w_begin, bi = it & 1u;
+        ti = locate(B, w, ti);
         const Df11Tensor &tn = B.t[ti];
+        const uint32_t b = w - tn.first_work;
+
+        // block offsets two items ahead (consumed at the end of this item)
+        uint64_t o0a = 0, o1a = 0;
+        uint32_t ta = ti;
+        if (w + 2 < w_end) {
+            ta = locate(B, w + 2, ti);
+            const uint32_t ba = w + 2 - B.t[ta].first_work;
+            o0a = B.t[ta].blkoff[ba];
+            o1a = B.t[ta].blkoff[ba + 1];
+        }
+
         if ((int)ti != cur) {
             // new tensor: stage its hierarchical tables, build the fast tables
             __syncthreads();
-            const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
-            for (uint32_t i = tid; i < ntab * 128u; i += T)
+            const uint32_t nt = min(tn.n_tables, B.lut_entries / 256u);
+            for (uint32_t i = tid; i < nt * 128u; i += T)
                 reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
             __syncthreads();
-            build_fast_tables(lut, ntab, cnt_tab, sym_tab);
-            __syncthreads();
+            build_fast_tables(lut, nt, cnt_tab, sym_tab);
             cur = (int)ti;
         }
         const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
-        const uint32_t b = w - tn.first_work;
-        const uint64_t o0 = tn.blkoff[b], o1 = tn.blkoff[b + 1];
-        if (!(o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes)) {
-            bad |= LWC_DEVICE_BAD_OFFSET;   // same decision in every thread
-            continue;
+        const uint64_t o0 = o0c, o1 = o1c;
+        const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 32 <= B.stage_bytes;
+
+        // clear the staging words this item will OR its exponents into
+        if (ok) {
+            const uint32_t words16 = (uint32_t)(((o0 & 15u) + (o1 - o0) + 4 + 15) >> 4);
+            for (uint32_t i = tid; i < words16; i += T) reinterpret_cast<uint4 *>(stage)[i] = make_uint4(0, 0, 0, 0);
         }
 
-        // stage this block's stream segment (plus 2 words of look-ahead)
-        const uint64_t seg0 = (uint64_t)b * T * CW;
-        for (uint32_t i = tid; i < B.seg_words / 4; i += T) {
-            const uint64_t gw = seg0 + 4ull * i;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (gw + 4 <= tn.stream_words) v = dev::ld_stream_v4(tn.stream + gw);
-            reinterpret_cast<uint4 *>(seg)[i] = v;
+        // this item's segment and gaps
+        const bool arrived = dev::mbar_wait_bounded(&bars[bi], (it >> 1) & 1u);
+        if (__syncthreads_or(!arrived)) {
+            // give up on this CTA's run, but first let the other buffer's copy
+            // (issued for the next item) land, within the same bound
+            bad |= LWC_DEVICE_TIMEOUT;
+            if (w + 1 < w_end) dev::mbar_wait_bounded(&bars[bi ^ 1u], ((it + 1) >> 1) & 1u);
+            break;
         }
-        const uint32_t gap = tn.gaps[(uint64_t)b * T + tid];
-        __syncthreads();
+        const uint32_t *seg = reinterpret_cast<const uint32_t *>(smem + L.bufs + bi * L.buf_bytes);
 
-        const uint64_t rem = tn.total_bits - (uint64_t)b * T * cbits;
-        const uint32_t start = tid * cbits + gap;
-        const uint32_t end = (uint32_t)min((uint64_t)(tid + 1) * cbits, rem);
+        if (ok) {
+            const uint32_t gap = smem[L.bufs + bi * L.buf_bytes + seg_bytes + tid];
+            const uint64_t rem = tn.total_bits - (uint64_t)b * T * cbits;
+            const uint32_t start = tid * cbits + gap;
+            const uint32_t end = (uint32_t)min((uint64_t)(tid + 1) * cbits, rem);
 
-        // phase 1: count the codes that start in [start, end)
-        uint32_t count = 0;
-        if (start < end) {
-            BitWindow bw;
-            bw.init(seg, start);
-            uint32_t pos = start;
-            while (pos + kFastBits <= end) {
-                const uint32_t e = cnt_tab[bw.win >> (64 - kFastBits)];
-                uint32_t len;
-                if (e) {
-                    count += e >> 4;
-                    len = e & 15u;
-                } else {
-                    len = lut_walk(lut, ntab, bw.win, bad) >> 8;
-                    count += 1;
+            // phase 1: count the codes that start in [start, end)
+            uint32_t count = 0;
+            if (start < end) {
+                uint32_t pos = start, acc = 0, sbits = 0, scount = 0;
+                if (end >= (uint32_t)kFastBits) {
+                    const uint32_t last = end - kFastBits;
+                    while (pos <= last) {
+                        const uint32_t wv = window32(seg, pos);
+                        const uint32_t e = cnt_tab[wv >> (32 - kFastBits)];
+                        if (e) {
+                            acc += e;
+                            pos += e & 15u;
+                        } else {
+                            const uint32_t len = lut_walk(lut, ntab, wv, bad) >> 8;
+                            pos += len;
+                            sbits += len;
+                            scount++;
+                        }
+                    }
                 }
-                bw.consume(seg, len);
-                pos += len;
-            }
-            while (pos < end) {
-                const uint32_t len = lut_walk(lut, ntab, bw.win, bad) >> 8;
-                count += 1;
-                bw.consume(seg, len);
-                pos += len;
-            }
-        }
-
-        uint32_t total;
-        const uint32_t first = block_exclusive_scan(count, warp_sums, total);
-        if (total != (uint32_t)(o1 - o0)) {
-            bad |= LWC_DEVICE_BAD_COUNT;   // `total` is the same in every thread
-            continue;
-        }
-
-        // phase 2: decode again, writing exponents to stage[(o0 & 15) + first ...]
-        if (start < end) {
-            BitWindow bw;
-            bw.init(seg, start);
-            StageWriter out;
-            out.init(stage, (uint32_t)(o0 & 15u) + first);
-            uint32_t pos = start;
-            while (pos + kFastBits <= end) {
-                const uint32_t e = sym_tab[bw.win >> (64 - kFastBits)];
-                uint32_t len;
-                if (e) {
-                    out.put(e & 0xFFFFFFu, (e >> 24) & 3u);
-                    len = e >> 26;
-                } else {
-                    const uint32_t r = lut_walk(lut, ntab, bw.win, bad);
-                    out.put(r & 0xFFu, 1);
-                    len = r >> 8;
+                count = ((acc - (pos - start - sbits)) >> 4) + scount;
+                while (pos < end) {
+                    pos += lut_walk(lut, ntab, window32(seg, pos), bad) >> 8;
+                    count++;
                 }
-                bw.consume(seg, len);
-                pos += len;
             }
-            while (pos < end) {
-                const uint32_t r = lut_walk(lut, ntab, bw.win, bad);
-                out.put(r & 0xFFu, 1);
-                const uint32_t len = r >> 8;
-                bw.consume(seg, len);
-                pos += len;
-            }
-            out.finish();
-        }
-        __syncthreads();
 
-        // merge exponents with sign|mantissa bytes; 16 weights per step
-        const uint64_t base = o0 & ~15ull;
-        for (uint64_t g = base + 16ull * tid; g < o1; g += 16ull * T) {
-            if (g >= o0 && g + 16 <= o1) {
-                const uint4 s = dev::ld_stream_v4(tn.sm + g);
-                const uint4 e = *reinterpret_cast<const uint4 *>(stage + (g - base));
-                uint4 r0, r1;
-                r0.x = merge2(s.x, e.x, 0x5140u);
-                r0.y = merge2(s.x, e.x, 0x7362u);
-                r0.z = merge2(s.y, e.y, 0x5140u);
-                r0.w = merge2(s.y, e.y, 0x7362u);
-                r1.x = merge2(s.z, e.z, 0x5140u);
-                r1.y = merge2(s.z, e.z, 0x7362u);
-                r1.z = merge2(s.w, e.w, 0x5140u);
-                r1.w = merge2(s.w, e.w, 0x7362u);
-                dev::st_v4(tn.out + g, r0);
-                dev::st_v4(tn.out + g + 8, r1);
+            uint32_t total;
+            const uint32_t first = block_exclusive_scan(count, warp_sums, total);
+            if (total == (uint32_t)(o1 - o0)) {
+                // phase 2: decode again, OR-ing exponents into stage[(o0 & 15) + first ...]
+                if (start < end) {
+                    const uint32_t p = (uint32_t)(o0 & 15u) + first;
+                    uint32_t *wp = reinterpret_cast<uint32_t *>(stage + (p & ~3u));
+                    uint32_t f8 = (p & 3u) * 8u, acc = 0;
+                    auto put = [&](uint32_t syms, uint32_t n8) {
+                        const uint32_t lo = acc | (syms << f8);
+                        const uint32_t hi = __funnelshift_l(syms, 0u, f8);
+                        f8 += n8;
+                        if (f8 >= 32) {
+                            atomicOr(wp, lo);
+                            ++wp;
+                            acc = hi;
+                            f8 -= 32;
+                        } else {
+                            acc = lo;
+                        }
+                    };
+                    uint32_t pos = start;
+                    if (end >= (uint32_t)kFastBits) {
+                        const uint32_t last = end - kFastBits;
+                        while (pos <= last) {
+                            const uint32_t wv = window32(seg, pos);
+                            const uint32_t e = sym_tab[wv >> (32 - kFastBits)];
+                            if (e) {
+                                put(e & 0xFFFFFFu, (e >> 21) & 0x18u);
+                                pos += e >> 26;
+                            } else {
+                                const uint32_t r = lut_walk(lut, ntab, wv, bad);
+                                put(r & 0xFFu, 8);
+                                pos += r >> 8;
+                            }
+                        }
+                    }
+                    while (pos < end) {
+                        const uint32_t r = lut_walk(lut, ntab, window32(seg, pos), bad);
+                        put(r & 0xFFu, 8);
+                        pos += r >> 8;
+                    }
+                    if (f8) atomicOr(wp, acc);
+                }
+                __syncthreads();
+
+                // merge exponents with sign|mantissa bytes (prefetched to L2)
+                const uint64_t base = o0 & ~15ull;
+                const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
+                for (uint64_t g = g_lo + 16ull * tid; g < g_hi; g += 32ull * T) {
+                    const uint64_t g2 = g + 16ull * T;
+                    const uint4 s1 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g));
+                    uint4 s2 = make_uint4(0, 0, 0, 0);
+                    if (g2 < g_hi) s2 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g2));
+                    merge16(s1, *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    if (g2 < g_hi) merge16(s2, *reinterpret_cast<const uint4 *>(stage + (g2 - base)), tn.out + g2);
+                }
+                if (tid < 32) {   // partial 16-groups at both ends
+                    const uint64_t i = tid < 16 ? o0 + tid : max(g_hi, g_lo) + (tid - 16);
+                    const bool head = tid < 16 && i < min(g_lo, o1);
+                    const bool tail = tid >= 16 && i < o1;
+                    if (head || tail) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
+                }
             } else {
-                for (uint32_t j = 0; j < 16; j++) {
-                    const uint64_t i = g + j;
-                    if (i >= o0 && i < o1) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
-                }
+                bad |= LWC_DEVICE_BAD_COUNT;   // `total` is the same in every thread
             }
+        } else {
+            bad |= LWC_DEVICE_BAD_OFFSET;      // same decision in every thread
         }
-        __syncthreads();
+        __syncthreads();   // buffer bi and the staging area are free again
+
+        if (tid == 0 && w + 2 < w_end) {
+            dev::fence_proxy_async_smem();
+            issue_item(B, ta, w + 2 - B.t[ta].first_work, o0a, o1a, smem + L.bufs + bi * L.buf_bytes, seg_bytes,
+                       &bars[bi]);
+        }
+        o0c = o0n;
+        o1c = o1n;
+        o0n = o0a;
+        o1n = o1a;
     }
     if (bad && B.status) atomicOr(B.status, bad);
 }
@@ -378,21 +442,11 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
 __global__ void df11_const_kernel(const uint8_t *__restrict__ sm, uint16_t *__restrict__ out, uint64_t n,
                                   uint32_t const_exp) {
     const uint32_t e4 = const_exp * 0x01010101u;
+    const uint4 ev = make_uint4(e4, e4, e4, e4);
     const uint64_t stride = 16ull * gridDim.x * blockDim.x;
     for (uint64_t g = 16ull * (blockIdx.x * (uint64_t)blockDim.x + threadIdx.x); g < n; g += stride) {
         if (g + 16 <= n) {
-            const uint4 s = dev::ld_stream_v4(sm + g);
-            uint4 r0, r1;
-            r0.x = merge2(s.x, e4, 0x5140u);
-            r0.y = merge2(s.x, e4, 0x7362u);
-            r0.z = merge2(s.y, e4, 0x5140u);
-            r0.w = merge2(s.y, e4, 0x7362u);
-            r1.x = merge2(s.z, e4, 0x5140u);
-            r1.y = merge2(s.z, e4, 0x7362u);
-            r1.z = merge2(s.w, e4, 0x5140u);
-            r1.w = merge2(s.w, e4, 0x7362u);
-            dev::st_v4(out + g, r0);
-            dev::st_v4(out + g + 8, r1);
+            merge16(__ldg(reinterpret_cast<const uint4 *>(sm + g)), ev, out + g);
         } else {
             for (uint64_t i = g; i < n; i++) out[i] = merge1(sm[i], const_exp);
         }
@@ -458,7 +512,7 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
         t.out = d_outs[idx[j]];
         t.n = d.n;
         t.total_bits = d.total_bits;
-        t.stream_words = d.stream_bytes / 4;
+        t.stream_bytes = d.stream_bytes;
         t.n_blocks = (uint32_t)d.n_blocks;
         t.n_tables = d.n_tables;
         t.first_work = (uint32_t)work;
@@ -469,10 +523,10 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     if (work > 0xFFFFFFFFull) return fail(LWC_ERR_UNSUPPORTED, "too many blocks in one launch");
     B.count = (uint32_t)idx.size();
     B.total_work = (uint32_t)work;
-    B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
+    B.stage_bytes = (uint32_t)round_up(max_count + 32, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
-    const uint64_t smem = kFastBytes + 2ull * B.lut_entries + 4ull * B.seg_words + B.stage_bytes + 128;
+    const uint64_t smem = Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
                     (unsigned long long)smem, cfg.max_smem);
