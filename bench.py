@@ -310,14 +310,15 @@ def run_lwc(args, rank, world, local_rank, dist):
         "clocks": clocks,
     }
 
-    # codebook codec on the same layer (secondary figures)
+    # codebook codec: the same layer in one batched launch, and a 256M-weight
+    # stress tensor (U = 8192 Zipf(1.1) table, k = 13) as secondary figures
     if not args.no_codebook:
         cenc = encode_all(tensors, "codebook")
         cblobs = [torch.from_numpy(b).to(device) for _, b in cenc]
-        cdescs = [d for d, _ in cenc]
+        cbatch = lwc.Batch([d for d, _ in cenc], cblobs, views)
+
         def cstep():
-            for d, b, v in zip(cdescs, cblobs, views):
-                lwc.lwc_decode_codebook(d, b, v, stream)
+            lwc.lwc_decode_codebook_batched(cbatch, stream=stream)
         cstep()
         torch.cuda.synchronize(device)
         for w, v in zip(tensors, views):
@@ -328,11 +329,30 @@ def run_lwc(args, rank, world, local_rank, dist):
         cms = time_steps(cstep, args.steps, stream) / args.steps
         cbytes = sum(b.numel() for b in cblobs)
         result["codebook"] = {
+            "workload": "llama3-8b-layer-codebook (one batched launch)",
             "value": round(2 * n_total / (cms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(cms, 5),
-            "launches_per_step": len(cdescs), "bits_per_weight": round(8 * cbytes / n_total, 4),
-            "index_bits": [d.k for d in cdescs],
+            "bits_per_weight": round(8 * cbytes / n_total, 4), "index_bits": [d.k for d, _ in cenc],
             "hbm_frac": round((cbytes + 2 * n_total) / (cms * 1e-3) / 1e9 / peak, 4)}
-        del cblobs
+        del cblobs, cbatch
+        ns = 1 << 28
+        xs = synth.codebook_stress(8192, ns, seed=40 + 8192, device=device)
+        sd, sb = lwc.lwc_encode_codebook(synth.as_u16(xs))
+        sbd = torch.from_numpy(sb).to(device)
+        sout = torch.empty(ns, dtype=torch.int16, device=device)
+        lwc.lwc_decode_codebook(sd, sbd, sout, stream)
+        torch.cuda.synchronize(device)
+        if not torch.equal(sout, xs.view(torch.int16)):
+            raise SystemExit("codebook stress decode differs from its input")
+        del xs
+        for _ in range(args.warmup):
+            lwc.lwc_decode_codebook(sd, sbd, sout, stream)
+        sms = time_steps(lambda: lwc.lwc_decode_codebook(sd, sbd, sout, stream), args.steps, stream) / args.steps
+        result["codebook_stress"] = {
+            "workload": f"codebook 256M weights, U={sd.U}, k={sd.k}, Zipf(1.1)",
+            "value": round(2 * ns / (sms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(sms, 5),
+            "bits_per_weight": round(sd.bits_per_weight, 4),
+            "hbm_frac": round((sb.size + 2 * ns) / (sms * 1e-3) / 1e9 / peak, 4)}
+        del sbd, sout
 
     # end to end through the C ABI with host buffers: pinned blobs -> device,
     # decode, decoded layer -> pinned host, every step

@@ -39,10 +39,12 @@
 namespace lwc {
 namespace {
 
-constexpr int kFastBits = 12;
+constexpr int kFastBits = 11;
 constexpr int kFastSize = 1 << kFastBits;
 constexpr int kMaxBatch = 32;
-constexpr uint32_t kFastBytes = kFastSize * 4 + kFastSize;   // symbol table + count table
+// symbol table (u32) + end-mask table (u16) + count table (u8)
+constexpr uint32_t kFastBytes = kFastSize * (4 + 2 + 1);
+constexpr int kMergeRegs = 8;   // 16-weight groups per thread whose loads are issued early
 
 struct Df11Tensor {
     const uint32_t *stream;
@@ -66,7 +68,7 @@ struct Df11Batch {
     uint32_t total_work;
     uint32_t chunk_words;  // chunk_bytes / 4
     uint32_t seg_words;    // words staged per block: T * chunk_words + 2, rounded up to 4
-    uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 32)
+    uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 16)
     uint32_t lut_entries;  // lookup-table entries reserved in shared memory
     uint32_t *status;
 };
@@ -77,7 +79,7 @@ struct Layout {
     __host__ __device__ Layout(uint32_t T, uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes) {
         lut = kFastBytes;
         bufs = lut + 2 * lut_entries;
-        buf_bytes = 4 * seg_words + T;   // segment words, then T gap bytes
+        buf_bytes = 4 * seg_words + T + 16;   // segment words, then the block's T gap bytes + the next one
         stage = bufs + 2 * buf_bytes;
         sums = stage + stage_bytes;
         bars = sums + 128;
@@ -110,17 +112,19 @@ __device__ __forceinline__ uint32_t lut_walk(const uint16_t *lut, uint32_t ntab,
     return e & 0x3FFFu;
 }
 
-// Fast tables, indexed by the next 12 stream bits:
-//  cnt_tab[v] = count << 4 | bits, for all whole codes inside the 12 bits
-//               (entries are summed: the sum of the `bits` parts is known, so
-//               one add per lookup counts codes);
-//  sym_tab[v] = sym0 | sym1 << 8 | sym2 << 16 | n << 24 | bits << 26, for the
-//               first n <= 3 of them.
-// 0 means "the first code is longer than 12 bits".
-__device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *cnt_tab, uint32_t *sym_tab) {
+// Fast tables, indexed by the next kFastBits (11) stream bits:
+//  cnt_tab[v]  = count << 4 | bits, for all whole codes inside the window
+//                (entries are summed: the sum of the `bits` parts is known, so
+//                one add per lookup counts codes);
+//  mask_tab[v] = bit (e - 1) set for every whole code that ends e bits in;
+//  sym_tab[v]  = sym0 | sym1 << 8 | sym2 << 16 | n << 24 | bits << 26, for the
+//                first n <= 3 of them.
+// Zero count/symbol entries mean "the first code is longer than the window".
+__device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *cnt_tab, uint16_t *mask_tab,
+                                  uint32_t *sym_tab) {
     for (uint32_t v = threadIdx.x; v < kFastSize; v += blockDim.x) {
         uint32_t w = v << (32 - kFastBits);
-        uint32_t used = 0, cnt = 0, syms = 0, n3 = 0, used3 = 0, ignore = 0;
+        uint32_t used = 0, cnt = 0, syms = 0, n3 = 0, used3 = 0, mask = 0, ignore = 0;
         while (cnt < (uint32_t)kFastBits) {
             const uint32_t r = lut_walk(lut, ntab, w, ignore);
             const uint32_t len = r >> 8;
@@ -132,9 +136,11 @@ __device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *c
             }
             cnt++;
             used += len;
+            mask |= 1u << (used - 1);
             w <<= len;
         }
         cnt_tab[v] = cnt ? (uint8_t)((cnt << 4) | used) : (uint8_t)0;
+        mask_tab[v] = (uint16_t)mask;
         sym_tab[v] = n3 ? (syms | (n3 << 24) | (used3 << 26)) : 0u;
     }
 }
@@ -207,34 +213,33 @@ __device__ __forceinline__ uint32_t locate(const Df11Batch &B, uint32_t w, uint3
     return ti;
 }
 
-// Thread 0: start the bulk copies of item (ti, b) into buffer `buf`, and
-// prefetch its sign|mantissa bytes [o0, o1) into L2.
-__device__ __forceinline__ void issue_item(const Df11Batch &B, uint32_t ti, uint32_t b, uint64_t o0, uint64_t o1,
-                                           uint8_t *buf, uint32_t seg_bytes, uint64_t *bar) {
+// Thread 0: start the bulk copies of item (ti, b) into buffer `buf`: the
+// block's stream segment, its T chunk gaps and (when there is a next block)
+// the next block's first gap, which bounds this block's last chunk.
+__device__ __forceinline__ void issue_item(const Df11Batch &B, uint32_t ti, uint32_t b, uint8_t *buf,
+                                           uint32_t seg_bytes, uint64_t *bar) {
     const Df11Tensor &tn = B.t[ti];
     const uint32_t T = blockDim.x;
     const uint64_t seg0 = (uint64_t)b * T * B.chunk_words * 4;   // byte offset, multiple of 128
     const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
     const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
-    dev::mbar_arrive_expect_tx(bar, bytes + T);
+    const uint32_t gbytes = b + 1 < tn.n_blocks ? T + 16 : T;
+    dev::mbar_arrive_expect_tx(bar, bytes + gbytes);
     if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
-    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * T, T, bar);
-    if (o0 < o1 && o1 <= tn.n) {
-        const uint64_t a = o0 & ~15ull, z = (o1 + 15) & ~15ull;
-        dev::prefetch_l2(tn.sm + a, (uint32_t)min(z - a, (uint64_t)0x7FFFFFF0ull));
-    }
+    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * T, gbytes, bar);
 }
 
 // ---- the kernel -------------------------------------------------------------------
 
 template <int kMaxThreads>
-__global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048 / kMaxThreads / 2 : 1)
+__global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMaxThreads : 1)
     df11_decode_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t T = blockDim.x, tid = threadIdx.x;
     const Layout L(T, B.seg_words, B.lut_entries, B.stage_bytes);
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem);
-    uint8_t *cnt_tab = smem + kFastSize * 4;
+    uint16_t *mask_tab = reinterpret_cast<uint16_t *>(smem + kFastSize * 4);
+    uint8_t *cnt_tab = smem + kFastSize * 6;
     uint16_t *lut = reinterpret_cast<uint16_t *>(smem + L.lut);
     uint8_t *stage = smem + L.stage;
     uint32_t *warp_sums = reinterpret_cast<uint32_t *>(smem + L.sums);
@@ -247,29 +252,16 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
     const uint32_t w_end = (uint32_t)((uint64_t)W * (blockIdx.x + 1) / G);
     if (w_begin >= w_end) return;
 
-    // block offsets of the current item and the next one
     uint32_t ti = locate(B, w_begin, 0);
-    uint64_t o0c, o1c, o0n = 0, o1n = 0;
-    {
-        const uint32_t b = w_begin - B.t[ti].first_work;
-        o0c = B.t[ti].blkoff[b];
-        o1c = B.t[ti].blkoff[b + 1];
-    }
-    uint32_t tn1 = ti;
-    if (w_begin + 1 < w_end) {
-        tn1 = locate(B, w_begin + 1, ti);
-        const uint32_t b = w_begin + 1 - B.t[tn1].first_work;
-        o0n = B.t[tn1].blkoff[b];
-        o1n = B.t[tn1].blkoff[b + 1];
-    }
     if (tid == 0) {
         dev::mbar_init(&bars[0], 1);
         dev::mbar_init(&bars[1], 1);
         dev::fence_mbar_init();
-        issue_item(B, ti, w_begin - B.t[ti].first_work, o0c, o1c, smem + L.bufs, seg_bytes, &bars[0]);
-        if (w_begin + 1 < w_end)
-            issue_item(B, tn1, w_begin + 1 - B.t[tn1].first_work, o0n, o1n, smem + L.bufs + L.buf_bytes,
-                       seg_bytes, &bars[1]);
+        issue_item(B, ti, w_begin - B.t[ti].first_work, smem + L.bufs, seg_bytes, &bars[0]);
+        if (w_begin + 1 < w_end) {
+            const uint32_t t1 = locate(B, w_begin + 1, ti);
+            issue_item(B, t1, w_begin + 1 - B.t[t1].first_work, smem + L.bufs + L.buf_bytes, seg_bytes, &bars[1]);
+        }
     }
 
     uint32_t bad = 0;
@@ -279,15 +271,17 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
         ti = locate(B, w, ti);
         const Df11Tensor &tn = B.t[ti];
         const uint32_t b = w - tn.first_work;
+        const uint64_t o0 = tn.blkoff[b], o1 = tn.blkoff[b + 1];
+        const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
 
-        // block offsets two items ahead (consumed at the end of this item)
-        uint64_t o0a = 0, o1a = 0;
-        uint32_t ta = ti;
-        if (w + 2 < w_end) {
-            ta = locate(B, w + 2, ti);
-            const uint32_t ba = w + 2 - B.t[ta].first_work;
-            o0a = B.t[ta].blkoff[ba];
-            o1a = B.t[ta].blkoff[ba + 1];
+        // sign|mantissa bytes of this thread's first merge groups: loads
+        // issued now, consumed after both decode passes
+        const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
+        uint4 sv[kMergeRegs];
+#pragma unroll
+        for (int m = 0; m < kMergeRegs; m++) {
+            const uint64_t g = g_lo + 16ull * (tid + (uint32_t)m * T);
+            sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
         }
 
         if ((int)ti != cur) {
@@ -297,18 +291,10 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
             for (uint32_t i = tid; i < nt * 128u; i += T)
                 reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
             __syncthreads();
-            build_fast_tables(lut, nt, cnt_tab, sym_tab);
+            build_fast_tables(lut, nt, cnt_tab, mask_tab, sym_tab);
             cur = (int)ti;
         }
         const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
-        const uint64_t o0 = o0c, o1 = o1c;
-        const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 32 <= B.stage_bytes;
-
-        // clear the staging words this item will OR its exponents into
-        if (ok) {
-            const uint32_t words16 = (uint32_t)(((o0 & 15u) + (o1 - o0) + 4 + 15) >> 4);
-            for (uint32_t i = tid; i < words16; i += T) reinterpret_cast<uint4 *>(stage)[i] = make_uint4(0, 0, 0, 0);
-        }
 
         // this item's segment and gaps
         const bool arrived = dev::mbar_wait_bounded(&bars[bi], (it >> 1) & 1u);
@@ -319,98 +305,103 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
             if (w + 1 < w_end) dev::mbar_wait_bounded(&bars[bi ^ 1u], ((it + 1) >> 1) & 1u);
             break;
         }
-        const uint32_t *seg = reinterpret_cast<const uint32_t *>(smem + L.bufs + bi * L.buf_bytes);
+        const uint8_t *buf = smem + L.bufs + bi * L.buf_bytes;
+        const uint32_t *seg = reinterpret_cast<const uint32_t *>(buf);
 
         if (ok) {
-            const uint32_t gap = smem[L.bufs + bi * L.buf_bytes + seg_bytes + tid];
-            const uint64_t rem = tn.total_bits - (uint64_t)b * T * cbits;
-            const uint32_t start = tid * cbits + gap;
-            const uint32_t end = (uint32_t)min((uint64_t)(tid + 1) * cbits, rem);
+            // this thread decodes the codes in [start, end): from its chunk's
+            // first code to the next chunk's first code (or the stream end),
+            // so the range holds whole codes only
+            const uint64_t rem_block = tn.total_bits - (uint64_t)b * T * cbits;
+            const uint32_t start = tid * cbits + buf[seg_bytes + tid];
+            const bool has_next = tid + 1 < T || b + 1 < tn.n_blocks;
+            const uint64_t next = has_next ? (uint64_t)(tid + 1) * cbits + buf[seg_bytes + tid + 1] : rem_block;
+            const uint32_t end = (uint32_t)min(next, rem_block);
 
-            // phase 1: count the codes that start in [start, end)
+            // phase 1: count the codes in [start, end)
             uint32_t count = 0;
             if (start < end) {
-                uint32_t pos = start, acc = 0, sbits = 0, scount = 0;
-                if (end >= (uint32_t)kFastBits) {
-                    const uint32_t last = end - kFastBits;
-                    while (pos <= last) {
-                        const uint32_t wv = window32(seg, pos);
-                        const uint32_t e = cnt_tab[wv >> (32 - kFastBits)];
-                        if (e) {
-                            acc += e;
-                            pos += e & 15u;
-                        } else {
-                            const uint32_t len = lut_walk(lut, ntab, wv, bad) >> 8;
-                            pos += len;
-                            sbits += len;
-                            scount++;
-                        }
+                uint32_t pos = start, rem = end - start, acc = 0, sbits = 0, scount = 0;
+                for (;;) {
+                    const uint32_t wv = window32(seg, pos);
+                    const uint32_t idx = wv >> (32 - kFastBits);
+                    const uint32_t e = cnt_tab[idx];
+                    const uint32_t len = e & 15u;
+                    if (len - 1u < rem) {   // whole entry inside the range (len 0: long code)
+                        acc += e;
+                        pos += len;
+                        rem -= len;
+                        continue;
                     }
+                    if (rem == 0) break;
+                    if (e == 0) {          // first code longer than the window
+                        const uint32_t l = lut_walk(lut, ntab, wv, bad) >> 8;
+                        if (l > rem) {
+                            bad |= LWC_DEVICE_BAD_CODE;
+                            break;
+                        }
+                        pos += l;
+                        rem -= l;
+                        sbits += l;
+                        scount++;
+                        continue;
+                    }
+                    scount += __popc(mask_tab[idx] & ((1u << rem) - 1u));   // codes ending inside the range
+                    break;
                 }
                 count = ((acc - (pos - start - sbits)) >> 4) + scount;
-                while (pos < end) {
-                    pos += lut_walk(lut, ntab, window32(seg, pos), bad) >> 8;
-                    count++;
-                }
             }
 
             uint32_t total;
             const uint32_t first = block_exclusive_scan(count, warp_sums, total);
             if (total == (uint32_t)(o1 - o0)) {
-                // phase 2: decode again, OR-ing exponents into stage[(o0 & 15) + first ...]
+                // phase 2: decode again, writing exponents to stage[(o0 & 15) + first ...]
                 if (start < end) {
-                    const uint32_t p = (uint32_t)(o0 & 15u) + first;
-                    uint32_t *wp = reinterpret_cast<uint32_t *>(stage + (p & ~3u));
-                    uint32_t f8 = (p & 3u) * 8u, acc = 0;
-                    auto put = [&](uint32_t syms, uint32_t n8) {
-                        const uint32_t lo = acc | (syms << f8);
-                        const uint32_t hi = __funnelshift_l(syms, 0u, f8);
-                        f8 += n8;
-                        if (f8 >= 32) {
-                            atomicOr(wp, lo);
-                            ++wp;
-                            acc = hi;
-                            f8 -= 32;
-                        } else {
-                            acc = lo;
+                    uint8_t *bp = stage + (uint32_t)(o0 & 15u) + first;
+                    uint32_t pos = start, rem = end - start;
+                    for (;;) {
+                        const uint32_t wv = window32(seg, pos);
+                        const uint32_t idx = wv >> (32 - kFastBits);
+                        const uint32_t e = sym_tab[idx];
+                        const uint32_t len = e >> 26;
+                        if (len - 1u < rem) {
+                            const uint32_t n = (e >> 24) & 3u;
+                            bp[0] = (uint8_t)e;
+                            if (n > 1) bp[1] = (uint8_t)(e >> 8);
+                            if (n > 2) bp[2] = (uint8_t)(e >> 16);
+                            bp += n;
+                            pos += len;
+                            rem -= len;
+                            continue;
                         }
-                    };
-                    uint32_t pos = start;
-                    if (end >= (uint32_t)kFastBits) {
-                        const uint32_t last = end - kFastBits;
-                        while (pos <= last) {
-                            const uint32_t wv = window32(seg, pos);
-                            const uint32_t e = sym_tab[wv >> (32 - kFastBits)];
-                            if (e) {
-                                put(e & 0xFFFFFFu, (e >> 21) & 0x18u);
-                                pos += e >> 26;
-                            } else {
-                                const uint32_t r = lut_walk(lut, ntab, wv, bad);
-                                put(r & 0xFFu, 8);
-                                pos += r >> 8;
-                            }
+                        if (rem == 0) break;
+                        if (e == 0) {
+                            const uint32_t r = lut_walk(lut, ntab, wv, bad);
+                            const uint32_t l = r >> 8;
+                            if (l > rem) break;
+                            *bp++ = (uint8_t)r;
+                            pos += l;
+                            rem -= l;
+                            continue;
                         }
+                        const uint32_t j = __popc(mask_tab[idx] & ((1u << rem) - 1u));   // < 3
+                        if (j > 0) bp[0] = (uint8_t)e;
+                        if (j > 1) bp[1] = (uint8_t)(e >> 8);
+                        break;
                     }
-                    while (pos < end) {
-                        const uint32_t r = lut_walk(lut, ntab, window32(seg, pos), bad);
-                        put(r & 0xFFu, 8);
-                        pos += r >> 8;
-                    }
-                    if (f8) atomicOr(wp, acc);
                 }
                 __syncthreads();
 
-                // merge exponents with sign|mantissa bytes (prefetched to L2)
+                // merge exponents with sign|mantissa bytes, 16 weights per group
                 const uint64_t base = o0 & ~15ull;
-                const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
-                for (uint64_t g = g_lo + 16ull * tid; g < g_hi; g += 32ull * T) {
-                    const uint64_t g2 = g + 16ull * T;
-                    const uint4 s1 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g));
-                    uint4 s2 = make_uint4(0, 0, 0, 0);
-                    if (g2 < g_hi) s2 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g2));
-                    merge16(s1, *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
-                    if (g2 < g_hi) merge16(s2, *reinterpret_cast<const uint4 *>(stage + (g2 - base)), tn.out + g2);
+#pragma unroll
+                for (int m = 0; m < kMergeRegs; m++) {
+                    const uint64_t g = g_lo + 16ull * (tid + (uint32_t)m * T);
+                    if (g < g_hi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
                 }
+                for (uint64_t g = g_lo + 16ull * (tid + (uint32_t)kMergeRegs * T); g < g_hi; g += 16ull * T)
+                    merge16(__ldg(reinterpret_cast<const uint4 *>(tn.sm + g)),
+                            *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
                 if (tid < 32) {   // partial 16-groups at both ends
                     const uint64_t i = tid < 16 ? o0 + tid : max(g_hi, g_lo) + (tid - 16);
                     const bool head = tid < 16 && i < min(g_lo, o1);
@@ -426,14 +417,10 @@ __global__ void __launch_bounds__(kMaxThreads, 2048 / kMaxThreads / 2 > 0 ? 2048
         __syncthreads();   // buffer bi and the staging area are free again
 
         if (tid == 0 && w + 2 < w_end) {
+            const uint32_t t2 = locate(B, w + 2, ti);
             dev::fence_proxy_async_smem();
-            issue_item(B, ta, w + 2 - B.t[ta].first_work, o0a, o1a, smem + L.bufs + bi * L.buf_bytes, seg_bytes,
-                       &bars[bi]);
+            issue_item(B, t2, w + 2 - B.t[t2].first_work, smem + L.bufs + bi * L.buf_bytes, seg_bytes, &bars[bi]);
         }
-        o0c = o0n;
-        o1c = o1n;
-        o0n = o0a;
-        o1n = o1a;
     }
     if (bad && B.status) atomicOr(B.status, bad);
 }
@@ -523,7 +510,7 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     if (work > 0xFFFFFFFFull) return fail(LWC_ERR_UNSUPPORTED, "too many blocks in one launch");
     B.count = (uint32_t)idx.size();
     B.total_work = (uint32_t)work;
-    B.stage_bytes = (uint32_t)round_up(max_count + 32, 16);
+    B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
     const uint64_t smem = Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;

@@ -31,7 +31,8 @@ STATUS_NAMES = {0: "LWC_OK", 1: "LWC_ERR_INVALID_ARG", 2: "LWC_ERR_MISALIGNED", 
 EXPORTED = (
     "lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
     "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
-    "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_status_string",
+    "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
+    "lwc_status_string",
     "lwc_last_error", "lwc_version",
 )
 
@@ -95,6 +96,7 @@ def load():
     L.lwc_decode_dfloat11_checked.argtypes = [D, _P, _P, _P, _P]
     L.lwc_decode_codebook_checked.argtypes = [D, _P, _P, _P, _P]
     L.lwc_decode_dfloat11_batched.argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int, _P, _P]
+    L.lwc_decode_codebook_batched.argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int, _P, _P]
     L.lwc_status_string.argtypes = [ctypes.c_int]
     L.lwc_status_string.restype = ctypes.c_char_p
     L.lwc_last_error.argtypes = []
@@ -102,7 +104,7 @@ def load():
     L.lwc_version.argtypes = []
     for name in ("lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
                  "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
-                 "lwc_decode_dfloat11_batched"):
+                 "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -211,6 +213,12 @@ def lwc_decode_dfloat11_batched(descs, d_ins=None, d_outs=None, d_status=None, s
     ``descs`` may also be a prepared ``Batch`` (then d_ins/d_outs are unused)."""
     b = descs if isinstance(descs, Batch) else Batch(descs, d_ins, d_outs)
     _check(load().lwc_decode_dfloat11_batched(b.descs, b.ins, b.outs, b.count, _addr(d_status), _stream(stream)))
+
+
+def lwc_decode_codebook_batched(descs, d_ins=None, d_outs=None, d_status=None, stream=None) -> None:
+    """Decode several codebook tensors at once (one launch per index width)."""
+    b = descs if isinstance(descs, Batch) else Batch(descs, d_ins, d_outs)
+    _check(load().lwc_decode_codebook_batched(b.descs, b.ins, b.outs, b.count, _addr(d_status), _stream(stream)))
 
 
 def lwc_status_string(status: int) -> str:

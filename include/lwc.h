@@ -184,6 +184,13 @@ LWC_API lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void
                                        uint16_t *const *d_outs, int count, uint32_t *d_status,
                                        lwc_stream_t stream);
 
+/* Decode `count` codebook tensors in as few launches as possible (one per
+ * distinct index width k among them, plus one fill per single-entry table).
+ * Arguments as lwc_decode_dfloat11_batched. */
+LWC_API lwc_status lwc_decode_codebook_batched(const lwc_desc *descs, const void *const *d_ins,
+                                               uint16_t *const *d_outs, int count, uint32_t *d_status,
+                                               lwc_stream_t stream);
+
 /* ---- helpers -------------------------------------------------------------- */
 
 /* Static string naming a status code. */

@@ -136,6 +136,28 @@ def test_batched_mixed():
         assert np.array_equal(host_u16(o)[:w.size], w)
 
 
+def test_codebook_batched_mixed():
+    tensors = [
+        synth.as_u16(synth.codebook_stress(4096, 100_003, seed=20)),     # k = 12
+        np.full(777, 0x3F80, np.uint16),                                # U = 1: k = 0
+        np.zeros(0, np.uint16),
+        synth.as_u16(synth.codebook_stress(300, 50_000, seed=21)),      # k = 9
+        synth.as_u16(synth.codebook_stress(4000, 8_191, seed=22)),      # k = 12, one partial tile
+        synth.as_u16(synth.uniform_patterns(70_000, seed=23)),          # k = 16
+    ]
+    enc = [lwc.lwc_encode_codebook(w) for w in tensors]
+    blobs = [dev(b) for _, b in enc]
+    outs = [torch.full((max(1, w.size),), 0x5555, dtype=torch.int16, device="cuda") for w in tensors]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_codebook_batched([d for d, _ in enc], blobs, outs, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for (d, b), w, o in zip(enc, tensors, outs):
+        got = host_u16(o)[:w.size]
+        assert np.array_equal(got, w)
+        assert np.array_equal(got, ocb.decode(b))
+
+
 def test_side_stream_and_reuse():
     w = synth.as_u16(synth.small_square(5))
     d, b = lwc.lwc_encode_dfloat11(w)
@@ -210,7 +232,8 @@ def test_llama3_8b_layer_full_size():
 
 @pytest.mark.parametrize("U", [256, 4096, 8192, 65536])
 def test_codebook_stress_full_size(U):
-    """256M weights from a U-entry table with Zipf(1.1) frequencies."""
+    """256M weights from a U-entry table with Zipf(1.1) frequencies (the
+    launch configuration bench.py times for the codebook stress figure)."""
     n = 1 << 28
     x = synth.codebook_stress(U, n, seed=40 + U, device="cuda")
     w = synth.as_u16(x)
