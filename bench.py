@@ -38,7 +38,7 @@ import synth  # noqa: E402
 
 METRIC = "decoded BF16 GB/s (DFloat11 layer-batched decode, Llama-3-8B layer)"
 FALLBACK_HBM_GBS = 6650.0
-PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
+PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_device.cuh")
 
 
@@ -78,14 +78,17 @@ def measured_peak():
 
 
 def profiled_traffic(workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    """DRAM bytes (read + write) per launch of the decode kernel from the
+    committed ncu summary, if it was taken on the current kernel source and
+    this workload; else None. Lines: <kernel> <workload> <source sha> <bytes>."""
     try:
         with open(PROFILE_TRAFFIC) as f:
-            t = json.load(f).get("df11_decode", {})
-        if t.get("kernel_sha") == kernel_sha() and t.get("workload") == workload:
-            return int(t["dram_bytes_per_launch"])
-    except Exception:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 4 and parts[0] == "df11_decode_kernel" and parts[1] == workload \
+                        and parts[2] == kernel_sha():
+                    return int(parts[3])
+    except OSError:
         pass
     return None
 

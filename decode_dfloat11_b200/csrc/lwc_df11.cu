@@ -21,11 +21,13 @@
 // Blocks never wait on one another: each block's first output index is stored
 // in the blob, so there is no inter-block scan.
 //
-// Memory pipeline per CTA: while item j is decoded, the bulk-copy (TMA)
-// engine brings the stream segment and chunk gaps of item j+1 into the other
-// half of a shared-memory double buffer, and the sign|mantissa bytes of item
-// j+1 are prefetched into L2, so the merge of j+1 reads them from L2. Block
-// offsets are loaded two items ahead. No wait is unbounded.
+// Memory pipeline per CTA: as soon as pass 2 of item j no longer needs the
+// shared stream segment, the bulk-copy (TMA) engine starts bringing in the
+// segment and chunk gaps of item j+1, overlapping the merge of item j; the
+// sign|mantissa bytes each thread merges are loaded into registers at the
+// start of an item, under both decode passes; block offsets are loaded one
+// item ahead. One segment buffer (not two) keeps four CTAs resident per SM.
+// No wait is unbounded.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -44,7 +46,8 @@ constexpr int kFastSize = 1 << kFastBits;
 constexpr int kMaxBatch = 32;
 // symbol table (u32) + end-mask table (u16) + count table (u8)
 constexpr uint32_t kFastBytes = kFastSize * (4 + 2 + 1);
-constexpr int kMergeRegs = 8;   // 16-weight groups per thread whose loads are issued early
+constexpr int kMergeRegs = 6;   // 16-weight groups per thread whose loads are issued early
+constexpr int kCtasPerSm = 4;   // target residency for 256-thread CTAs (shared memory sized for it)
 
 struct Df11Tensor {
     const uint32_t *stream;
@@ -80,7 +83,7 @@ struct Layout {
         lut = kFastBytes;
         bufs = lut + 2 * lut_entries;
         buf_bytes = 4 * seg_words + T + 16;   // segment words, then the block's T gap bytes + the next one
-        stage = bufs + 2 * buf_bytes;
+        stage = bufs + buf_bytes;
         sums = stage + stage_bytes;
         bars = sums + 128;
         total = bars + 16;
@@ -232,7 +235,7 @@ __device__ __forceinline__ void issue_item(const Df11Batch &B, uint32_t ti, uint
 // ---- the kernel -------------------------------------------------------------------
 
 template <int kMaxThreads>
-__global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMaxThreads : 1)
+__global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 0 ? kCtasPerSm * 256 / kMaxThreads : 1)
     df11_decode_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t T = blockDim.x, tid = threadIdx.x;
@@ -255,23 +258,27 @@ __global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMa
     uint32_t ti = locate(B, w_begin, 0);
     if (tid == 0) {
         dev::mbar_init(&bars[0], 1);
-        dev::mbar_init(&bars[1], 1);
         dev::fence_mbar_init();
         issue_item(B, ti, w_begin - B.t[ti].first_work, smem + L.bufs, seg_bytes, &bars[0]);
-        if (w_begin + 1 < w_end) {
-            const uint32_t t1 = locate(B, w_begin + 1, ti);
-            issue_item(B, t1, w_begin + 1 - B.t[t1].first_work, smem + L.bufs + L.buf_bytes, seg_bytes, &bars[1]);
-        }
     }
 
+    // block offsets of the first item; later items' are loaded one item ahead
+    uint64_t o0n = B.t[ti].blkoff[w_begin - B.t[ti].first_work];
+    uint64_t o1n = B.t[ti].blkoff[w_begin - B.t[ti].first_work + 1];
     uint32_t bad = 0;
     int cur = -1;
     for (uint32_t w = w_begin; w < w_end; ++w) {
-        const uint32_t it = w - w_begin, bi = it & 1u;
+        const uint32_t it = w - w_begin;
         ti = locate(B, w, ti);
         const Df11Tensor &tn = B.t[ti];
         const uint32_t b = w - tn.first_work;
-        const uint64_t o0 = tn.blkoff[b], o1 = tn.blkoff[b + 1];
+        const uint64_t o0 = o0n, o1 = o1n;
+        if (w + 1 < w_end) {
+            const uint32_t t1 = locate(B, w + 1, ti);
+            const uint32_t b1 = w + 1 - B.t[t1].first_work;
+            o0n = B.t[t1].blkoff[b1];
+            o1n = B.t[t1].blkoff[b1 + 1];
+        }
         const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
 
         // sign|mantissa bytes of this thread's first merge groups: loads
@@ -296,16 +303,14 @@ __global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMa
         }
         const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
 
-        // this item's segment and gaps
-        const bool arrived = dev::mbar_wait_bounded(&bars[bi], (it >> 1) & 1u);
+        // this item's segment and gaps (its copy is the only one in flight)
+        const bool arrived = dev::mbar_wait_bounded(&bars[0], it & 1u);
         if (__syncthreads_or(!arrived)) {
-            // give up on this CTA's run, but first let the other buffer's copy
-            // (issued for the next item) land, within the same bound
             bad |= LWC_DEVICE_TIMEOUT;
-            if (w + 1 < w_end) dev::mbar_wait_bounded(&bars[bi ^ 1u], ((it + 1) >> 1) & 1u);
             break;
         }
-        const uint8_t *buf = smem + L.bufs + bi * L.buf_bytes;
+        bool next_issued = false;
+        const uint8_t *buf = smem + L.bufs;
         const uint32_t *seg = reinterpret_cast<const uint32_t *>(buf);
 
         if (ok) {
@@ -391,6 +396,13 @@ __global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMa
                     }
                 }
                 __syncthreads();
+                // the segment is free: fetch the next item's while merging this one
+                if (tid == 0 && w + 1 < w_end) {
+                    const uint32_t t1 = locate(B, w + 1, ti);
+                    dev::fence_proxy_async_smem();
+                    issue_item(B, t1, w + 1 - B.t[t1].first_work, smem + L.bufs, seg_bytes, &bars[0]);
+                }
+                next_issued = true;
 
                 // merge exponents with sign|mantissa bytes, 16 weights per group
                 const uint64_t base = o0 & ~15ull;
@@ -414,12 +426,12 @@ __global__ void __launch_bounds__(kMaxThreads, 768 / kMaxThreads > 0 ? 768 / kMa
         } else {
             bad |= LWC_DEVICE_BAD_OFFSET;      // same decision in every thread
         }
-        __syncthreads();   // buffer bi and the staging area are free again
+        __syncthreads();   // the segment and the staging area are free again
 
-        if (tid == 0 && w + 2 < w_end) {
-            const uint32_t t2 = locate(B, w + 2, ti);
+        if (tid == 0 && !next_issued && w + 1 < w_end) {   // items skipped as corrupt
+            const uint32_t t1 = locate(B, w + 1, ti);
             dev::fence_proxy_async_smem();
-            issue_item(B, t2, w + 2 - B.t[t2].first_work, smem + L.bufs + bi * L.buf_bytes, seg_bytes, &bars[bi]);
+            issue_item(B, t1, w + 1 - B.t[t1].first_work, smem + L.bufs, seg_bytes, &bars[0]);
         }
     }
     if (bad && B.status) atomicOr(B.status, bad);

@@ -1,0 +1,103 @@
+"""Compressed model weights resident in GPU memory, decoded layer by layer.
+
+This follows the DFloat11 page ("Koniec z kompromisami! DFloat11 ratuje
+dokładność modeli AI ...", section "Jak to działa w praktyce? Magia na
+poziomie GPU", third pillar): the weights stay compressed in HBM and all the
+matrices of one transformer block are decompressed together, in one launch,
+right before the block runs. Decoded layers land in a small set of reusable
+BF16 buffers (two by default: a ping-pong pair, so layer L+1 can be decoded
+while layer L is in use).
+
+Everything here is bookkeeping and argument marshalling around the C ABI
+(``lwc_decode_dfloat11_batched`` / ``lwc_decode_codebook_batched``); the
+decoding itself runs in liblwc's CUDA kernels.
+"""
+from __future__ import annotations
+
+import concurrent.futures as cf
+import os
+
+import numpy as np
+
+from . import lwc
+
+CODECS = ("dfloat11", "codebook")
+
+
+def encode_many(arrays, codec: str = "dfloat11", workers: int | None = None, **params):
+    """Encode host BF16 bit-pattern arrays in parallel host threads (the C
+    encoder releases the GIL). Returns [(desc, blob), ...] in input order."""
+    if codec not in CODECS:
+        raise ValueError(f"unknown codec {codec!r}")
+    fn = (lambda a: lwc.lwc_encode_dfloat11(a, **params)) if codec == "dfloat11" else lwc.lwc_encode_codebook
+    workers = workers or min(len(arrays), os.cpu_count() or 1) or 1
+    with cf.ThreadPoolExecutor(max_workers=workers) as ex:
+        return list(ex.map(fn, arrays))
+
+
+class ResidentModel:
+    """Compressed layers in device memory plus reusable BF16 output buffers.
+
+    Usage: ``add_layer`` for every layer (uploads its blobs), ``finalize`` to
+    allocate the buffers and marshal the launch arguments once, then
+    ``decode(layer, slot, stream)`` per layer; ``views(layer, slot)`` gives
+    the decoded matrices (BF16 views into buffer ``slot``).
+    """
+
+    def __init__(self, codec: str, device, slots: int = 2):
+        import torch
+        if codec not in CODECS:
+            raise ValueError(f"unknown codec {codec!r}")
+        self.codec = codec
+        self.device = torch.device(device)
+        self.slots = slots
+        self.layers: list[dict] = []
+        self.buffers = []
+        self._batches: list[list] = []
+
+    def add_layer(self, name: str, encoded, shapes) -> None:
+        """encoded: [(desc, host blob)] of the layer's matrices, shapes their shapes."""
+        import torch
+        descs = [d for d, _ in encoded]
+        blobs = [torch.from_numpy(b).to(self.device) for _, b in encoded]
+        self.layers.append(dict(name=name, descs=descs, blobs=blobs, shapes=[tuple(s) for s in shapes],
+                                n=[d.n for d in descs]))
+
+    @property
+    def compressed_bytes(self) -> int:
+        return sum(int(b.numel()) for layer in self.layers for b in layer["blobs"])
+
+    @property
+    def weights(self) -> int:
+        return sum(sum(layer["n"]) for layer in self.layers)
+
+    def finalize(self) -> None:
+        import torch
+        biggest = max(sum(layer["n"]) for layer in self.layers)
+        # 8 extra elements per matrix keep every view 16-byte aligned
+        biggest += 8 * max(len(layer["n"]) for layer in self.layers)
+        self.buffers = [torch.empty(biggest, dtype=torch.bfloat16, device=self.device) for _ in range(self.slots)]
+        self._batches = []
+        for layer in self.layers:
+            per_slot = []
+            for s in range(self.slots):
+                views = self._views(layer, s)
+                per_slot.append((lwc.Batch(layer["descs"], layer["blobs"], views), views))
+            self._batches.append(per_slot)
+
+    def _views(self, layer, slot):
+        out, off = [], 0
+        for n, shape in zip(layer["n"], layer["shapes"]):
+            out.append(self.buffers[slot][off:off + n].view(shape))
+            off += (n + 7) // 8 * 8
+        return out
+
+    def views(self, layer: int, slot: int):
+        return self._batches[layer][slot][1]
+
+    def decode(self, layer: int, slot: int, stream=None, status=None) -> None:
+        batch = self._batches[layer][slot][0]
+        if self.codec == "dfloat11":
+            lwc.lwc_decode_dfloat11_batched(batch, d_status=status, stream=stream)
+        else:
+            lwc.lwc_decode_codebook_batched(batch, d_status=status, stream=stream)

@@ -1,0 +1,93 @@
+"""Model-scale decodes: compressed weights resident in HBM, decoded layer by
+layer (one batched launch per layer) into reusable BF16 ping-pong buffers.
+
+Full Llama-3-8B shapes (32 layers + embedding + LM head, 8.03 B weights) with
+both codecs resident at once, and Llama-3-70B shapes (layers sampled from the
+80, plus embedding and LM head; every tensor at full size). Every decoded
+layer is compared, on the device, with the same seeded tensors generated
+again; the oracle decodes sampled blobs on the host for an independent check."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from decode_dfloat11_b200 import build as lwc_build
+from decode_dfloat11_b200 import lwc
+from decode_dfloat11_b200.layers import ResidentModel, encode_many
+from oracle import codebook as ocb
+from oracle import df11 as odf
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def lib(cuda_device):
+    lwc_build.build()
+    return lwc.load()
+
+
+def model_units(which: str, layers):
+    """(name, generator) per unit; a generator yields the unit's tensors on the GPU."""
+    if which == "8b":
+        hidden, shapes, sig, off = synth.LLAMA3_8B_HIDDEN, synth.LLAMA3_8B_LAYER, (0.01, 0.04), 0
+    else:
+        hidden, shapes, sig, off = synth.LLAMA3_70B_HIDDEN, synth.LLAMA3_70B_LAYER, (0.005, 0.03), \
+            synth.SEED_70B_OFFSET
+    units = [("embed", lambda: [synth.llama_embedding("embed", hidden, sig, off, device="cuda")])]
+    for L in layers:
+        units.append((f"layer{L}", lambda L=L: [t for _, t in synth.llama_layer_tensors(
+            L, shapes, sig, off, device="cuda")]))
+    units.append(("lm_head", lambda: [synth.llama_embedding("lm_head", hidden, sig, off, device="cuda")]))
+    return units
+
+
+def build(units, codecs):
+    models = {c: ResidentModel(c, "cuda") for c in codecs}
+    for name, gen in units:
+        tensors = gen()
+        host = [synth.as_u16(t) for t in tensors]
+        shapes = [t.shape for t in tensors]
+        del tensors
+        for c, m in models.items():
+            m.add_layer(name, encode_many(host, c), shapes)
+    for m in models.values():
+        m.finalize()
+    return models
+
+
+def check_all(units, models, oracle_units=()):
+    stream = torch.cuda.current_stream()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for i, (name, gen) in enumerate(units):
+        expect = gen()
+        for c, m in models.items():
+            slot = i % 2
+            m.decode(i, slot, stream, status)
+            torch.cuda.synchronize()
+            for v, t in zip(m.views(i, slot), expect):
+                assert torch.equal(v.view(torch.int16), t.view(torch.int16)), (c, name)
+            if name in oracle_units:
+                got = m.views(i, slot)[0].reshape(-1).view(torch.int16).cpu().numpy().view(np.uint16)
+                blob = m.layers[i]["blobs"][0].cpu().numpy()
+                ref = odf.decode(blob) if c == "dfloat11" else ocb.decode(blob)
+                assert np.array_equal(got, ref), (c, name)
+        del expect
+    assert int(status.item()) == 0
+
+
+def test_llama3_8b_model_both_codecs_resident():
+    units = model_units("8b", range(synth.LLAMA3_8B_LAYERS))
+    models = build(units, ("dfloat11", "codebook"))
+    df, cb = models["dfloat11"], models["codebook"]
+    assert df.weights == cb.weights == 8_029_995_008
+    assert 10.0 < 8 * df.compressed_bytes / df.weights < 11.5
+    assert 12.5 < 8 * cb.compressed_bytes / cb.weights < 14.5
+    check_all(units, models, oracle_units=("layer0", "lm_head"))
+
+
+def test_llama3_70b_layers_full_shapes():
+    units = model_units("70b", (0, 41, 79))
+    models = build(units, ("dfloat11",))
+    df = models["dfloat11"]
+    assert 10.0 < 8 * df.compressed_bytes / df.weights < 11.5
+    check_all(units, models, oracle_units=("layer41",))
