@@ -14,7 +14,8 @@
 //    stream, a block-wide scan turns the counts into output positions, and the
 //    threads decode again, this time writing exponents to a shared-memory
 //    staging buffer; the staged exponents are then merged with the
-//    sign|mantissa bytes and written out with 16-byte stores;
+//    sign|mantissa bytes and written out with 16-byte stores. Both passes
+//    take two table entries per 32-bit window read (up to 22 bits per step);
 //  * all matrices of a transformer block in one launch: the grid walks a work
 //    list of (tensor, block) items; CTAs are persistent, take contiguous runs
 //    of items and rebuild their tables only when the tensor changes.
@@ -332,6 +333,15 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
                     const uint32_t idx = wv >> (32 - kFastBits);
                     const uint32_t e = cnt_tab[idx];
                     const uint32_t len = e & 15u;
+                    // two entries from one 32-bit window (the first takes at most 11 bits)
+                    const uint32_t e2 = cnt_tab[(wv << len) >> (32 - kFastBits)];
+                    const uint32_t l2 = e2 & 15u;
+                    if ((len - 1u < rem) & (l2 - 1u < rem - len)) {
+                        acc += e + e2;
+                        pos += len + l2;
+                        rem -= len + l2;
+                        continue;
+                    }
                     if (len - 1u < rem) {   // whole entry inside the range (len 0: long code)
                         acc += e;
                         pos += len;
@@ -369,6 +379,22 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
                         const uint32_t idx = wv >> (32 - kFastBits);
                         const uint32_t e = sym_tab[idx];
                         const uint32_t len = e >> 26;
+                        const uint32_t e2 = sym_tab[(wv << len) >> (32 - kFastBits)];
+                        const uint32_t l2 = e2 >> 26;
+                        if ((len - 1u < rem) & (l2 - 1u < rem - len)) {   // two entries, one window
+                            const uint32_t n = (e >> 24) & 3u, n2 = (e2 >> 24) & 3u;
+                            bp[0] = (uint8_t)e;
+                            if (n > 1) bp[1] = (uint8_t)(e >> 8);
+                            if (n > 2) bp[2] = (uint8_t)(e >> 16);
+                            uint8_t *bq = bp + n;
+                            bq[0] = (uint8_t)e2;
+                            if (n2 > 1) bq[1] = (uint8_t)(e2 >> 8);
+                            if (n2 > 2) bq[2] = (uint8_t)(e2 >> 16);
+                            bp = bq + n2;
+                            pos += len + l2;
+                            rem -= len + l2;
+                            continue;
+                        }
                         if (len - 1u < rem) {
                             const uint32_t n = (e >> 24) & 3u;
                             bp[0] = (uint8_t)e;

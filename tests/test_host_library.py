@@ -197,3 +197,16 @@ def test_encoder_rejects_bad_arguments():
     L = lwc.load()
     desc = lwc.lwc_desc()
     assert L.lwc_encode_dfloat11(None, 5, None, ctypes.byref(desc), None, None) == 1
+
+
+def test_encode_many_matches_sequential():
+    from decode_dfloat11_b200.layers import encode_many
+    arrays = [synth.as_u16(synth.normal_bf16((50_000 + 17 * i,), seed=30 + i, sigma=0.02, outlier_frac=1e-3))
+              for i in range(6)]
+    for codec, fn in (("dfloat11", lwc.lwc_encode_dfloat11), ("codebook", lwc.lwc_encode_codebook)):
+        par = encode_many(arrays, codec, workers=4)
+        for (d, b), a in zip(par, arrays):
+            d2, b2 = fn(a)
+            assert np.array_equal(b, b2) and d.as_dict() == d2.as_dict()
+    with pytest.raises(ValueError):
+        encode_many(arrays, "zstd")
