@@ -157,27 +157,27 @@ __device__ __forceinline__ uint32_t window32(const uint32_t *seg, uint32_t pos) 
 
 // ---- merge ---------------------------------------------------------------------
 
-// Two weights from s = [s0 s1 ..] and e = [e0 e1 ..] bytes selected by `sel`:
-// w = (s & 0x80) << 8 | e << 7 | (s & 0x7F), two at a time in one word.
-__device__ __forceinline__ uint32_t merge2(uint32_t s, uint32_t e, uint32_t sel) {
-    const uint32_t x = __byte_perm(s, e, sel);   // [s_a, e_a, s_b, e_b]
-    return (x & 0x007F007Fu) | ((x >> 1) & 0x7F807F80u) | ((x << 8) & 0x80008000u);
-}
-
 __device__ __forceinline__ uint16_t merge1(uint32_t s, uint32_t e) {
     return (uint16_t)(((s & 0x80u) << 8) | (e << 7) | (s & 0x7Fu));
 }
 
+// Four weights from four sign|mantissa bytes s and four exponents e: a BF16
+// weight's low byte is (s & 0x7F) | (e & 1) << 7 and its high byte is
+// (e >> 1) | (s & 0x80), computed for four lanes of a word at once, then
+// interleaved into two words of output.
+__device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t &w01, uint32_t &w23) {
+    const uint32_t lo = (s & 0x7F7F7F7Fu) | ((e << 7) & 0x80808080u);
+    const uint32_t hi = ((e >> 1) & 0x7F7F7F7Fu) | (s & 0x80808080u);
+    w01 = __byte_perm(lo, hi, 0x5140u);
+    w23 = __byte_perm(lo, hi, 0x7362u);
+}
+
 __device__ __forceinline__ void merge16(const uint4 &s, const uint4 &e, uint16_t *dst) {
     uint4 r0, r1;
-    r0.x = merge2(s.x, e.x, 0x5140u);
-    r0.y = merge2(s.x, e.x, 0x7362u);
-    r0.z = merge2(s.y, e.y, 0x5140u);
-    r0.w = merge2(s.y, e.y, 0x7362u);
-    r1.x = merge2(s.z, e.z, 0x5140u);
-    r1.y = merge2(s.z, e.z, 0x7362u);
-    r1.z = merge2(s.w, e.w, 0x5140u);
-    r1.w = merge2(s.w, e.w, 0x7362u);
+    merge4(s.x, e.x, r0.x, r0.y);
+    merge4(s.y, e.y, r0.z, r0.w);
+    merge4(s.z, e.z, r1.x, r1.y);
+    merge4(s.w, e.w, r1.z, r1.w);
     reinterpret_cast<uint4 *>(dst)[0] = r0;
     reinterpret_cast<uint4 *>(dst)[1] = r1;
 }
