@@ -17,7 +17,6 @@ from __future__ import annotations
 import concurrent.futures as cf
 import os
 
-import numpy as np
 
 from . import lwc
 
@@ -101,3 +100,35 @@ class ResidentModel:
             lwc.lwc_decode_dfloat11_batched(batch, d_status=status, stream=stream)
         else:
             lwc.lwc_decode_codebook_batched(batch, d_status=status, stream=stream)
+
+    def pipelined(self, compute_stream, decode_stream=None):
+        """Iterate over the layers with decoding one layer ahead of use.
+
+        Yields ``(layer, views)``; the views are ready for work enqueued on
+        ``compute_stream``, and layer + 1 is already being decoded on
+        ``decode_stream`` meanwhile (a side stream if None). Enqueue all work
+        that reads the yielded views on ``compute_stream`` before advancing
+        the generator: a buffer is reused only after an event recorded on
+        ``compute_stream`` at that point says its consumer has finished.
+        """
+        import torch
+        ds = decode_stream or torch.cuda.Stream(self.device)
+        ready = [torch.cuda.Event() for _ in range(self.slots)]
+        free = [torch.cuda.Event() for _ in range(self.slots)]
+        used = [False] * self.slots
+        ds.wait_stream(compute_stream)   # inputs written before the call are visible
+        self.decode(0, 0, ds)
+        ready[0].record(ds)
+        for i in range(len(self.layers)):
+            slot = i % self.slots
+            nxt = i + 1
+            if nxt < len(self.layers):
+                ns = nxt % self.slots
+                if used[ns]:
+                    ds.wait_event(free[ns])
+                self.decode(nxt, ns, ds)
+                ready[ns].record(ds)
+            compute_stream.wait_event(ready[slot])
+            yield i, self.views(i, slot)
+            free[slot].record(compute_stream)
+            used[slot] = True

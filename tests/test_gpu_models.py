@@ -91,3 +91,29 @@ def test_llama3_70b_layers_full_shapes():
     df = models["dfloat11"]
     assert 10.0 < 8 * df.compressed_bytes / df.weights < 11.5
     check_all(units, models, oracle_units=("layer41",))
+
+
+def test_pipelined_decode_overlaps_and_never_clobbers():
+    """Layer L+1 decodes on a side stream while layer L is consumed; the
+    consumer copies every weight it sees and runs a GEMM on it, so a buffer
+    overwritten too early would show up as a mismatch."""
+    shapes = [(3072, 1024), (1024, 3072), (2048, 2048)]
+    units = []
+    for L in range(6):
+        units.append((f"layer{L}", lambda L=L: [synth.normal_bf16(s, 7000 + 10 * L + j, sigma=0.02,
+                                                                outlier_frac=1e-3, device="cuda")
+                                                for j, s in enumerate(shapes)]))
+    model = build(units, ("dfloat11",))["dfloat11"]
+    compute = torch.cuda.Stream()
+    x = torch.randn(64, 1024, device="cuda", dtype=torch.bfloat16)
+    compute.wait_stream(torch.cuda.current_stream())
+    copies, outs = [], []
+    with torch.cuda.stream(compute):
+        for i, views in model.pipelined(compute):
+            copies.append([v.clone() for v in views])
+            outs.append(torch.relu(x @ views[1]))   # some real work on the decoded (1024 x 3072) matrix
+    torch.cuda.synchronize()
+    for (name, gen), got in zip(units, copies):
+        for g, t in zip(got, gen()):
+            assert torch.equal(g.view(torch.int16), t.view(torch.int16)), name
+    assert all(o.shape == (64, 3072) for o in outs)
