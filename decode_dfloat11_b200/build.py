@@ -17,7 +17,7 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liblwc.so")
 
-CUDA_SOURCES = ["lwc_df11.cu", "lwc_codebook.cu"]
+CUDA_SOURCES = ["lwc_df11.cu", "lwc_codebook.cu", "lwc_encode.cu"]
 CXX_SOURCES = ["lwc_host.cpp"]
 HEADERS = ["lwc_internal.h", "lwc_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

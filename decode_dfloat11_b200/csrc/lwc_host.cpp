@@ -40,13 +40,13 @@ lwc_status fail(lwc_status s, const char *fmt, ...) {
 void clear_error() { g_last_error.clear(); }
 
 namespace {
-
-// ---------------------------------------------------------------- header I/O
-
 template <typename T>
 void put(uint8_t *h, size_t off, T v) { std::memcpy(h + off, &v, sizeof v); }
 template <typename T>
 T get(const uint8_t *h, size_t off) { T v; std::memcpy(&v, h + off, sizeof v); return v; }
+}  // namespace
+
+// ---------------------------------------------------------------- header I/O
 
 void write_header(uint8_t *h, const lwc_desc &d) {
     std::memset(h, 0, kHeaderBytes);
@@ -83,6 +83,8 @@ void write_header(uint8_t *h, const lwc_desc &d) {
     }
 }
 
+namespace {
+
 void read_header(const uint8_t *h, lwc_desc &d) {
     std::memset(&d, 0, sizeof d);
     d.magic = get<uint32_t>(h, 0);
@@ -117,18 +119,9 @@ void read_header(const uint8_t *h, lwc_desc &d) {
     }
 }
 
-uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+}  // namespace
 
-// Section placement: each section at the next multiple of kSectionAlign.
-struct Layout {
-    uint64_t pos = kHeaderBytes;
-    uint64_t place(uint64_t bytes) {
-        uint64_t off = round_up(pos, kSectionAlign);
-        pos = off + bytes;
-        return off;
-    }
-    uint64_t total() const { return round_up(pos, 16); }
-};
+namespace {
 
 // ------------------------------------------------------------ Huffman code
 
@@ -249,6 +242,85 @@ lwc_status check_args(const uint16_t *src, uint64_t n, lwc_desc *desc, void **bl
 
 }  // namespace
 
+// ------------------------------------------------------------ blob plans
+
+lwc_status check_df11_params(uint32_t C, uint32_t T, uint32_t L) {
+    if (C % 4 || C < 8 || C > 1024 || T % 32 || T < 32 || T > 1024 || L < 9 || L > kFormatMaxLen)
+        return fail(LWC_ERR_INVALID_ARG, "bad DFloat11 parameters (chunk %u, block %u, max_len %u)", C, T, L);
+    return LWC_OK;
+}
+
+lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uint32_t T, uint32_t L, Df11Plan &p) {
+    if (lwc_status st = check_df11_params(C, T, L)) return st;
+    int present = 0, only = 0;
+    for (int s = 0; s < 256; s++)
+        if (counts[s]) present++, only = s;
+    lwc_desc &d = p.d;
+    std::memset(&d, 0, sizeof d);
+    d.magic = kMagic;
+    d.version = kVersion;
+    d.codec = LWC_CODEC_DFLOAT11;
+    d.n = n;
+    d.chunk_bytes = C;
+    d.threads_per_block = T;
+    std::memset(p.len, 0, sizeof p.len);
+    std::memset(p.code, 0, sizeof p.code);
+    p.tables.clear();
+    p.single = present < 2;
+    if (!p.single) {
+        std::vector<int> order;
+        huffman_lengths(counts, p.len);
+        limit_lengths(counts, p.len, L);
+        canonical(p.len, p.code, order);
+        if (!build_tables(p.len, p.code, order, p.tables))
+            return fail(LWC_ERR_UNSUPPORTED, "code needs more than %u lookup tables", kMaxTables);
+        for (int s = 0; s < 256; s++) {
+            d.total_bits += counts[s] * p.len[s];
+            d.max_len = std::max(d.max_len, p.len[s]);
+        }
+        d.n_tables = (uint32_t)(p.tables.size() / 256);
+        const uint64_t cb = 8ull * C;
+        d.n_chunks = (d.total_bits + cb - 1) / cb;
+        d.n_blocks = (d.n_chunks + T - 1) / T;
+        d.stream_bytes = round_up(4 * ((d.total_bits + 31) / 32) + 16, 16);
+    } else {
+        d.flags = n ? kFlagSingleExponent : 0;
+        d.const_exp = (uint32_t)only;
+    }
+    BlobLayout lay;
+    d.off_lengths = lay.place(256);
+    d.off_lut = lay.place(2 * p.tables.size());
+    d.off_gaps = lay.place(d.n_blocks * T);
+    d.off_blkoff = lay.place(8 * (d.n_blocks + 1));
+    d.off_stream = lay.place(d.stream_bytes);
+    d.off_sm = lay.place(round_up(n, 16));
+    d.total_bytes = lay.total();
+    return LWC_OK;
+}
+
+void plan_codebook(const std::vector<uint8_t> &seen, uint64_t n, CbPlan &p) {
+    p.table.clear();
+    p.rank.assign(65536, 0);
+    for (uint32_t v = 0; v < 65536; v++)
+        if (seen[v]) {
+            p.rank[v] = (uint16_t)p.table.size();
+            p.table.push_back((uint16_t)v);
+        }
+    lwc_desc &d = p.d;
+    std::memset(&d, 0, sizeof d);
+    d.magic = kMagic;
+    d.version = kVersion;
+    d.codec = LWC_CODEC_CODEBOOK;
+    d.n = n;
+    d.U = (uint32_t)p.table.size();
+    while ((1ull << d.k) < d.U) d.k++;
+    d.packed_bytes = d.k ? round_up((n * d.k + 7) / 8 + 16, 16) : 0;
+    BlobLayout lay;
+    d.off_table = lay.place(2ull * d.U);
+    d.off_packed = lay.place(d.packed_bytes);
+    d.total_bytes = lay.total();
+}
+
 // ------------------------------------------------------- descriptor checks
 
 static bool inside(uint64_t off, uint64_t bytes, uint64_t total) {
@@ -318,57 +390,17 @@ lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_p
     const uint32_t C = params ? params->chunk_bytes : 36;
     const uint32_t T = params ? params->threads_per_block : 256;
     const uint32_t L = params ? params->max_len : 32;
-    if (C % 4 || C < 8 || C > 1024 || T % 32 || T < 32 || T > 1024 || L < 9 || L > kFormatMaxLen)
-        return fail(LWC_ERR_INVALID_ARG, "bad DFloat11 parameters (chunk %u, block %u, max_len %u)", C, T, L);
 
-    // exponent histogram
+    // exponent histogram, then the code and the section layout
     uint64_t counts[256] = {0};
     for (uint64_t i = 0; i < n; i++) counts[(src[i] >> 7) & 0xFF]++;
-    int present = 0, only = 0;
-    for (int s = 0; s < 256; s++)
-        if (counts[s]) present++, only = s;
-
-    lwc_desc d;
-    std::memset(&d, 0, sizeof d);
-    d.magic = kMagic;
-    d.version = kVersion;
-    d.codec = LWC_CODEC_DFLOAT11;
-    d.n = n;
-    d.chunk_bytes = C;
-    d.threads_per_block = T;
-
-    uint32_t len[256], code[256] = {0};
-    std::vector<int> order;
-    std::vector<uint16_t> tables;
-    if (present >= 2) {
-        huffman_lengths(counts, len);
-        limit_lengths(counts, len, L);
-        canonical(len, code, order);
-        if (!build_tables(len, code, order, tables))
-            return fail(LWC_ERR_UNSUPPORTED, "code needs more than %u lookup tables", kMaxTables);
-        for (int s = 0; s < 256; s++) {
-            d.total_bits += counts[s] * len[s];
-            d.max_len = std::max(d.max_len, len[s]);
-        }
-        d.n_tables = (uint32_t)(tables.size() / 256);
-        const uint64_t cb = 8ull * C;
-        d.n_chunks = (d.total_bits + cb - 1) / cb;
-        d.n_blocks = (d.n_chunks + T - 1) / T;
-        d.stream_bytes = round_up(4 * ((d.total_bits + 31) / 32) + 16, 16);
-    } else {
-        std::memset(len, 0, sizeof len);
-        d.flags = n ? kFlagSingleExponent : 0;
-        d.const_exp = (uint32_t)only;
-    }
-
-    Layout lay;
-    d.off_lengths = lay.place(256);
-    d.off_lut = lay.place(2 * tables.size());
-    d.off_gaps = lay.place(d.n_blocks * T);
-    d.off_blkoff = lay.place(8 * (d.n_blocks + 1));
-    d.off_stream = lay.place(d.stream_bytes);
-    d.off_sm = lay.place(round_up(n, 16));
-    d.total_bytes = lay.total();
+    Df11Plan plan;
+    st = plan_dfloat11(counts, n, C, T, L, plan);
+    if (st) return st;
+    lwc_desc &d = plan.d;
+    const bool present2 = !plan.single;
+    const uint32_t *len = plan.len, *code = plan.code;
+    const std::vector<uint16_t> &tables = plan.tables;
 
     uint8_t *blob = (uint8_t *)std::calloc(1, d.total_bytes);
     if (!blob) return fail(LWC_ERR_NOMEM, "cannot allocate %llu bytes", (unsigned long long)d.total_bytes);
@@ -380,7 +412,7 @@ lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_p
     uint8_t *sm = blob + d.off_sm;
     for (uint64_t i = 0; i < n; i++) sm[i] = (uint8_t)(((src[i] >> 8) & 0x80) | (src[i] & 0x7F));
 
-    if (present >= 2) {
+    if (present2) {
         // codes, MSB first in u32 words, with chunk gaps and block offsets
         uint32_t *words = reinterpret_cast<uint32_t *>(blob + d.off_stream);
         uint8_t *gaps = blob + d.off_gaps;
@@ -440,26 +472,10 @@ lwc_status lwc_encode_codebook(const uint16_t *src, uint64_t n, lwc_desc *desc_o
     if (st) return st;
     std::vector<uint8_t> seen(65536, 0);
     for (uint64_t i = 0; i < n; i++) seen[src[i]] = 1;
-    std::vector<uint16_t> table;
-    std::vector<uint16_t> rank(65536, 0);
-    for (uint32_t v = 0; v < 65536; v++)
-        if (seen[v]) {
-            rank[v] = (uint16_t)table.size();
-            table.push_back((uint16_t)v);
-        }
-    lwc_desc d;
-    std::memset(&d, 0, sizeof d);
-    d.magic = kMagic;
-    d.version = kVersion;
-    d.codec = LWC_CODEC_CODEBOOK;
-    d.n = n;
-    d.U = (uint32_t)table.size();
-    while ((1ull << d.k) < d.U) d.k++;
-    d.packed_bytes = d.k ? round_up((n * d.k + 7) / 8 + 16, 16) : 0;
-    Layout lay;
-    d.off_table = lay.place(2ull * d.U);
-    d.off_packed = lay.place(d.packed_bytes);
-    d.total_bytes = lay.total();
+    CbPlan plan;
+    plan_codebook(seen, n, plan);
+    lwc_desc &d = plan.d;
+    const std::vector<uint16_t> &table = plan.table, &rank = plan.rank;
     uint8_t *blob = (uint8_t *)std::calloc(1, d.total_bytes);
     if (!blob) return fail(LWC_ERR_NOMEM, "cannot allocate %llu bytes", (unsigned long long)d.total_bytes);
     if (d.U) std::memcpy(blob + d.off_table, table.data(), 2ull * d.U);

@@ -1,9 +1,11 @@
-// Internal declarations shared by the host encoder (lwc_host.cpp) and the
-// device decoders (lwc_df11.cu, lwc_codebook.cu). Not part of the C ABI.
+// Internal declarations shared by the host encoder (lwc_host.cpp), the
+// device decoders (lwc_df11.cu, lwc_codebook.cu) and the device encoder
+// (lwc_encode.cu). Not part of the C ABI.
 #pragma once
 
 #include <cstdint>
 #include <cstddef>
+#include <vector>
 
 #include "lwc.h"
 
@@ -29,5 +31,42 @@ lwc_status check_df11_desc(const lwc_desc *d);
 lwc_status check_codebook_desc(const lwc_desc *d);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+
+// Section placement inside a blob: each section at the next multiple of kSectionAlign.
+struct BlobLayout {
+    uint64_t pos = kHeaderBytes;
+    uint64_t place(uint64_t bytes) {
+        const uint64_t off = round_up(pos, kSectionAlign);
+        pos = off + bytes;
+        return off;
+    }
+    uint64_t total() const { return round_up(pos, 16); }
+};
+
+// Everything a DFloat11 blob holds besides the per-weight sections, derived
+// from the exponent histogram: the descriptor (all fields but
+// max_block_count), code lengths, canonical codewords and lookup tables.
+struct Df11Plan {
+    lwc_desc d;
+    uint32_t len[256];
+    uint32_t code[256];
+    std::vector<uint16_t> tables;
+    bool single;   // one exponent value (or n = 0): no stream
+};
+lwc_status check_df11_params(uint32_t chunk_bytes, uint32_t threads_per_block, uint32_t max_len);
+lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t chunk_bytes, uint32_t threads_per_block,
+                         uint32_t max_len, Df11Plan &plan);
+
+// Codebook blob plan from the set of present 16-bit patterns (seen[v] != 0).
+struct CbPlan {
+    lwc_desc d;
+    std::vector<uint16_t> table;   // ascending distinct patterns
+    std::vector<uint16_t> rank;    // pattern -> index
+};
+void plan_codebook(const std::vector<uint8_t> &seen, uint64_t n, CbPlan &plan);
+
+// Writes the 256-byte blob header for `d`.
+void write_header(uint8_t *header, const lwc_desc &d);
 
 }  // namespace lwc

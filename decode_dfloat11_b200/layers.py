@@ -34,6 +34,37 @@ def encode_many(arrays, codec: str = "dfloat11", workers: int | None = None, **p
         return list(ex.map(fn, arrays))
 
 
+def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=None, **params):
+    """Compress a BF16 tensor that is already on the GPU into a device blob
+    (``lwc_encode_*_device_plan`` + ``lwc_encode_device_write``).
+
+    Returns ``(desc, blob)`` with ``blob`` a uint8 CUDA tensor of
+    ``desc.total_bytes`` bytes, byte-for-byte what the host encoder would make.
+    ``workspace`` (a uint8 CUDA tensor of at least
+    ``lwc_encode_device_workspace_bytes(n)`` bytes) may be passed to reuse one
+    buffer across tensors; the tensor must not change while this runs."""
+    import torch
+    if codec not in CODECS:
+        raise ValueError(f"unknown codec {codec!r}")
+    src = tensor.reshape(-1)
+    if src.dtype != torch.bfloat16 and src.element_size() != 2:
+        raise ValueError("expected a 16-bit tensor")
+    src = src.contiguous()
+    n = src.numel()
+    need = lwc.lwc_encode_device_workspace_bytes(n)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=src.device)
+    work_bytes = workspace.numel()
+    stream = stream if stream is not None else torch.cuda.current_stream(src.device)
+    if codec == "dfloat11":
+        desc = lwc.lwc_encode_dfloat11_device_plan(src, n, workspace, work_bytes, stream=stream, **params)
+    else:
+        desc = lwc.lwc_encode_codebook_device_plan(src, n, workspace, work_bytes, stream=stream)
+    blob = torch.empty(desc.total_bytes, dtype=torch.uint8, device=src.device)
+    desc = lwc.lwc_encode_device_write(src, n, workspace, work_bytes, blob, blob.numel(), stream=stream)
+    return desc, blob
+
+
 class ResidentModel:
     """Compressed layers in device memory plus reusable BF16 output buffers.
 
@@ -61,6 +92,19 @@ class ResidentModel:
         blobs = [torch.from_numpy(b).to(self.device) for _, b in encoded]
         self.layers.append(dict(name=name, descs=descs, blobs=blobs, shapes=[tuple(s) for s in shapes],
                                 n=[d.n for d in descs]))
+
+    def add_layer_from_device(self, name: str, tensors, workspace=None, **params) -> None:
+        """Compress BF16 tensors that are already on this model's GPU (the
+        device encoder) and keep only their blobs."""
+        import torch
+        encoded = []
+        for t in tensors:
+            need = lwc.lwc_encode_device_workspace_bytes(t.numel())
+            if workspace is None or workspace.numel() < need:
+                workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
+            encoded.append(encode_on_device(t, self.codec, workspace, **params))
+        self.layers.append(dict(name=name, descs=[d for d, _ in encoded], blobs=[b for _, b in encoded],
+                                shapes=[tuple(t.shape) for t in tensors], n=[d.n for d, _ in encoded]))
 
     @property
     def compressed_bytes(self) -> int:

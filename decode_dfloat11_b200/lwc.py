@@ -32,8 +32,8 @@ EXPORTED = (
     "lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
     "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
     "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
-    "lwc_status_string",
-    "lwc_last_error", "lwc_version",
+    "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan", "lwc_encode_codebook_device_plan",
+    "lwc_encode_device_write", "lwc_status_string", "lwc_last_error", "lwc_version",
 )
 
 
@@ -97,6 +97,11 @@ def load():
     L.lwc_decode_codebook_checked.argtypes = [D, _P, _P, _P, _P]
     L.lwc_decode_dfloat11_batched.argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int, _P, _P]
     L.lwc_decode_codebook_batched.argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.c_int, _P, _P]
+    L.lwc_encode_device_workspace_bytes.argtypes = [_u64]
+    L.lwc_encode_device_workspace_bytes.restype = _u64
+    L.lwc_encode_dfloat11_device_plan.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
+    L.lwc_encode_codebook_device_plan.argtypes = [_P, _u64, _P, _u64, D, _P]
+    L.lwc_encode_device_write.argtypes = [_P, _u64, _P, _u64, _P, _u64, D, _P]
     L.lwc_status_string.argtypes = [ctypes.c_int]
     L.lwc_status_string.restype = ctypes.c_char_p
     L.lwc_last_error.argtypes = []
@@ -104,7 +109,8 @@ def load():
     L.lwc_version.argtypes = []
     for name in ("lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
                  "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
-                 "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched"):
+                 "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched", "lwc_encode_dfloat11_device_plan",
+                 "lwc_encode_codebook_device_plan", "lwc_encode_device_write"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -219,6 +225,36 @@ def lwc_decode_codebook_batched(descs, d_ins=None, d_outs=None, d_status=None, s
     """Decode several codebook tensors at once (one launch per index width)."""
     b = descs if isinstance(descs, Batch) else Batch(descs, d_ins, d_outs)
     _check(load().lwc_decode_codebook_batched(b.descs, b.ins, b.outs, b.count, _addr(d_status), _stream(stream)))
+
+
+def lwc_encode_device_workspace_bytes(n: int) -> int:
+    return load().lwc_encode_device_workspace_bytes(n)
+
+
+def lwc_encode_dfloat11_device_plan(d_src, n: int, d_work, work_bytes: int, chunk_bytes: int = 36,
+                                    threads_per_block: int = 256, max_len: int = 32, stream=None) -> lwc_desc:
+    """Plan a DFloat11 blob for n device BF16 patterns; returns its descriptor."""
+    desc = lwc_desc()
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    _check(load().lwc_encode_dfloat11_device_plan(_addr(d_src), n, ctypes.byref(params), _addr(d_work), work_bytes,
+                                                  ctypes.byref(desc), _stream(stream)))
+    return desc
+
+
+def lwc_encode_codebook_device_plan(d_src, n: int, d_work, work_bytes: int, stream=None) -> lwc_desc:
+    desc = lwc_desc()
+    _check(load().lwc_encode_codebook_device_plan(_addr(d_src), n, _addr(d_work), work_bytes, ctypes.byref(desc),
+                                                  _stream(stream)))
+    return desc
+
+
+def lwc_encode_device_write(d_src, n: int, d_work, work_bytes: int, d_blob, blob_bytes: int,
+                            stream=None) -> lwc_desc:
+    """Write the planned blob into d_blob; returns the final descriptor."""
+    desc = lwc_desc()
+    _check(load().lwc_encode_device_write(_addr(d_src), n, _addr(d_work), work_bytes, _addr(d_blob), blob_bytes,
+                                          ctypes.byref(desc), _stream(stream)))
+    return desc
 
 
 def lwc_status_string(status: int) -> str:

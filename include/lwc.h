@@ -22,7 +22,8 @@
  *    table lookup.
  *
  * Memory and ownership
- *  - Encoders run on the host. They malloc the blob; release it with lwc_free.
+ *  - The host encoders malloc the blob; release it with lwc_free. (The
+ *    device encoders below write into caller-owned device memory instead.)
  *  - The caller copies the blob, byte for byte, to a device buffer it owns
  *    (d_in) and keeps the lwc_desc (a plain struct in host memory).
  *  - Decoders run asynchronously on the caller's CUDA stream and write n
@@ -190,6 +191,47 @@ LWC_API lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void
 LWC_API lwc_status lwc_decode_codebook_batched(const lwc_desc *descs, const void *const *d_ins,
                                                uint16_t *const *d_outs, int count, uint32_t *d_status,
                                                lwc_stream_t stream);
+
+/* ---- device encoders ------------------------------------------------------ */
+
+/* Compression of a tensor that is already in GPU memory, into a blob in GPU
+ * memory. The blob is byte-for-byte the one the host encoder makes from the
+ * same weights and parameters. The codebook page ("Codebook Lossless
+ * Compression: когда 25% памяти значат больше, чем кажется", trade-offs)
+ * notes that building the dictionary and index map lengthens model loading;
+ * these entry points keep every pass over the weights on the GPU and leave
+ * only the code construction (from a 256-bin histogram or a 65536-bit
+ * presence map) to the host.
+ *
+ * Two calls per tensor, sharing one device workspace the caller owns
+ * (lwc_encode_device_workspace_bytes(n) bytes, 256-byte aligned):
+ *   1. *_device_plan reads d_src (n BF16 patterns, device, 16-byte aligned)
+ *      and fills *desc_out; desc_out->total_bytes is the blob size to
+ *      allocate. (max_block_count is still 0 here.)
+ *   2. lwc_encode_device_write reads d_src again and writes the blob to d_blob
+ *      (device, 16-byte aligned, at least total_bytes long); *desc_out then
+ *      holds the final descriptor, equal to the blob's header.
+ * d_src must hold the same weights in both calls (else LWC_ERR_INVALID_ARG,
+ * with nothing written outside d_blob's total_bytes); the workspace must not
+ * be used by another encode in between. Work is issued on `stream`, after
+ * whatever the caller has queued there, and both calls synchronise `stream`
+ * before returning (the host needs the histogram, and the blob is complete on
+ * return). They allocate nothing. Limit: n <= 2^36. */
+LWC_API uint64_t lwc_encode_device_workspace_bytes(uint64_t n);
+
+/* Plan a DFloat11 blob (params as for lwc_encode_dfloat11; NULL = defaults). */
+LWC_API lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const lwc_df11_params *params,
+                                                   void *d_work, uint64_t work_bytes, lwc_desc *desc_out,
+                                                   lwc_stream_t stream);
+
+/* Plan a codebook blob. */
+LWC_API lwc_status lwc_encode_codebook_device_plan(const void *d_src, uint64_t n, void *d_work,
+                                                   uint64_t work_bytes, lwc_desc *desc_out, lwc_stream_t stream);
+
+/* Write the blob the workspace's plan describes (either codec). */
+LWC_API lwc_status lwc_encode_device_write(const void *d_src, uint64_t n, void *d_work, uint64_t work_bytes,
+                                           void *d_blob, uint64_t blob_bytes, lwc_desc *desc_out,
+                                           lwc_stream_t stream);
 
 /* ---- helpers -------------------------------------------------------------- */
 

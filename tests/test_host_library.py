@@ -210,3 +210,34 @@ def test_encode_many_matches_sequential():
             assert np.array_equal(b, b2) and d.as_dict() == d2.as_dict()
     with pytest.raises(ValueError):
         encode_many(arrays, "zstd")
+
+
+def test_device_encoder_validates_before_any_device_call():
+    L = lwc.load()
+    n = 100_000
+    need = lwc.lwc_encode_device_workspace_bytes(n)
+    # the workspace holds the tile arrays (DFloat11) or the 65536-entry index map (codebook)
+    tiles = (n + 4095) // 4096
+    assert need >= 256 + 8192 + max(2 * 65536, 12 * tiles)
+    assert lwc.lwc_encode_device_workspace_bytes(1 << 30) >= 12 * ((1 << 30) // 4096)
+    assert need % 256 == 0
+    cases = [
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1000, n, None, need), 1),          # no workspace
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1000, n, 0x2000, need - 1), 1),    # too small
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1008, n, 0x2000, need), 2),        # misaligned source
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1000, n, 0x2010, need), 2),        # misaligned workspace
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(None, n, 0x2000, need), 1),          # no source
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1000, n, 0x2000, need, chunk_bytes=10), 1),
+        (lambda: lwc.lwc_encode_dfloat11_device_plan(0x1000, n, 0x2000, need, max_len=40), 1),
+        (lambda: lwc.lwc_encode_codebook_device_plan(0x1000, 1 << 37, 0x2000, 1 << 62), 4),  # above the limit
+        (lambda: lwc.lwc_encode_device_write(0x1000, n, 0x2000, need, None, 1 << 20), 1),  # no blob
+        (lambda: lwc.lwc_encode_device_write(0x1000, n, 0x2000, need, 0x9008, 1 << 20), 2),  # misaligned blob
+    ]
+    for i, (call, status) in enumerate(cases):
+        with pytest.raises(lwc.LwcError) as e:
+            call()
+        assert e.value.status == status, (i, str(e.value))
+    desc = lwc.lwc_desc()
+    assert L.lwc_encode_codebook_device_plan(0x1000, n, 0x2000, need, None, None) == 1
+    assert L.lwc_encode_device_write(0x1000, n, 0x2000, need, 0x3000, 1 << 20, None, None) == 1
+    del desc
