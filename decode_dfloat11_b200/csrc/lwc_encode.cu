@@ -25,6 +25,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "lwc_internal.h"
@@ -769,3 +770,77 @@ lwc_status lwc_encode_device_write(const void *d_src, uint64_t n, void *d_work, 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// No-allocation variant of the DFloat11 device encoder.
+//
+// For callers that cannot call cudaMalloc at encode time: typically a serving
+// process whose memory manager has already reserved the device memory for
+// weights and KV cache up front and allows no further cudaMalloc/cudaFree
+// (a late cudaMalloc can fail or fragment the reserved pool, and cudaFree
+// synchronises the whole device). Instead of a caller workspace this entry
+// point uses one file-scope scratch array in device memory, created when the
+// library's device code is loaded on a GPU and held by every GPU that loads
+// it until the process exits.
+namespace lwc {
+namespace {
+
+constexpr uint64_t kNoAllocMaxN = 1ull << 30;   // weights; every matrix of Llama-3-8B/70B fits
+static_assert(3154432 == (kWsArrays + ((4 * ((kNoAllocMaxN + kTile - 1) / kTile) + 255) / 256) * 256 +
+                          8 * ((kNoAllocMaxN + kTile - 1) / kTile + 1) + 255) / 256 * 256,
+              "the scratch size stated in lwc.h");
+constexpr uint64_t kNoAllocScratchBytes =
+    (kWsArrays + ((4 * ((kNoAllocMaxN + kTile - 1) / kTile) + 255) / 256) * 256 +
+     8 * ((kNoAllocMaxN + kTile - 1) / kTile + 1) + 255) / 256 * 256;   // workspace_bytes(kNoAllocMaxN)
+
+// Shared by every call on a device; keeps the last call's contents (the plan
+// step clears what must start at zero).
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void *g_scratch_ptr[kMaxDevices];
+
+// Device address of the scratch array for the current device, looked up once
+// per device (the symbol's host-side name is only a handle, not an address).
+lwc_status noalloc_scratch(void *&ptr) {
+    int dev = 0;
+    LWC_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(LWC_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        LWC_CUDA(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(scratch)");
+        g_scratch_ptr[dev] = p;
+    }
+    ptr = g_scratch_ptr[dev];
+    return LWC_OK;
+}
+
+}  // namespace
+}  // namespace lwc
+
+extern "C" lwc_status lwc_encode_dfloat11_device_noalloc(const void *d_src, uint64_t n, const lwc_df11_params *params,
+                                                         void *d_blob, uint64_t blob_bytes, lwc_desc *desc_out,
+                                                         lwc_stream_t stream) {
+    if (!desc_out) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    if (n > kNoAllocMaxN)
+        return fail(LWC_ERR_UNSUPPORTED,
+                    "tensor of %llu weights is above the no-allocation encoder's maximum of %llu "
+                    "(its scratch array holds %llu bytes)",
+                    (unsigned long long)n, (unsigned long long)kNoAllocMaxN,
+                    (unsigned long long)kNoAllocScratchBytes);
+    if (!d_blob) return fail(LWC_ERR_INVALID_ARG, "NULL blob buffer");
+    if (!aligned16(d_blob)) return fail(LWC_ERR_MISALIGNED, "blob buffer must be 16-byte aligned");
+    void *scratch = nullptr;
+    if (lwc_status st = noalloc_scratch(scratch)) return st;
+    lwc_desc plan;
+    if (lwc_status st = lwc_encode_dfloat11_device_plan(d_src, n, params, scratch, kNoAllocScratchBytes, &plan, stream))
+        return st;
+    if (blob_bytes < plan.total_bytes) {
+        *desc_out = plan;   // tells the caller the size it needs
+        return fail(LWC_ERR_INVALID_ARG, "blob buffer of %llu bytes, %llu needed", (unsigned long long)blob_bytes,
+                    (unsigned long long)plan.total_bytes);
+    }
+    return lwc_encode_device_write(d_src, n, scratch, kNoAllocScratchBytes, d_blob, blob_bytes, desc_out, stream);
+}

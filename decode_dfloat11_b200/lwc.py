@@ -33,7 +33,8 @@ EXPORTED = (
     "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
     "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
     "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan", "lwc_encode_codebook_device_plan",
-    "lwc_encode_device_write", "lwc_status_string", "lwc_last_error", "lwc_version",
+    "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_status_string", "lwc_last_error",
+    "lwc_version",
 )
 
 
@@ -102,6 +103,7 @@ def load():
     L.lwc_encode_dfloat11_device_plan.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
     L.lwc_encode_codebook_device_plan.argtypes = [_P, _u64, _P, _u64, D, _P]
     L.lwc_encode_device_write.argtypes = [_P, _u64, _P, _u64, _P, _u64, D, _P]
+    L.lwc_encode_dfloat11_device_noalloc.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
     L.lwc_status_string.argtypes = [ctypes.c_int]
     L.lwc_status_string.restype = ctypes.c_char_p
     L.lwc_last_error.argtypes = []
@@ -110,7 +112,8 @@ def load():
     for name in ("lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
                  "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
                  "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched", "lwc_encode_dfloat11_device_plan",
-                 "lwc_encode_codebook_device_plan", "lwc_encode_device_write"):
+                 "lwc_encode_codebook_device_plan", "lwc_encode_device_write",
+                 "lwc_encode_dfloat11_device_noalloc"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
     return L
@@ -254,6 +257,18 @@ def lwc_encode_device_write(d_src, n: int, d_work, work_bytes: int, d_blob, blob
     desc = lwc_desc()
     _check(load().lwc_encode_device_write(_addr(d_src), n, _addr(d_work), work_bytes, _addr(d_blob), blob_bytes,
                                           ctypes.byref(desc), _stream(stream)))
+    return desc
+
+
+def lwc_encode_dfloat11_device_noalloc(d_src, n: int, d_blob, blob_bytes: int, chunk_bytes: int = 36,
+                                       threads_per_block: int = 256, max_len: int = 32, stream=None) -> lwc_desc:
+    """DFloat11 device encode without any device allocation (the library's
+    own scratch array replaces the workspace); for callers that cannot call
+    cudaMalloc. Returns the blob's descriptor."""
+    desc = lwc_desc()
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    _check(load().lwc_encode_dfloat11_device_noalloc(_addr(d_src), n, ctypes.byref(params), _addr(d_blob),
+                                                     blob_bytes, ctypes.byref(desc), _stream(stream)))
     return desc
 
 

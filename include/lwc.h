@@ -233,6 +233,38 @@ LWC_API lwc_status lwc_encode_device_write(const void *d_src, uint64_t n, void *
                                            void *d_blob, uint64_t blob_bytes, lwc_desc *desc_out,
                                            lwc_stream_t stream);
 
+/* DFloat11 device encode that allocates nothing, for callers that cannot
+ * call cudaMalloc when they compress a tensor: e.g. a serving process whose
+ * memory manager has reserved the device memory for weights and KV cache up
+ * front and permits no further cudaMalloc/cudaFree (a late cudaMalloc can
+ * fail or fragment that pool; cudaFree synchronises the whole device).
+ * The pages have no counterpart to this entry point.
+ *
+ * Does lwc_encode_dfloat11_device_plan + lwc_encode_device_write in one call,
+ * with a fixed scratch array inside the library (3,154,432 bytes of device
+ * memory, created when the library's device code is loaded on a GPU and
+ * held by every GPU that loads it until the process exits) in place of the
+ * caller's workspace. It calls no cudaMalloc or cudaFree and no allocating
+ * library routine.
+ *   - n must be <= 2^30 weights (the scratch's limit; every matrix of
+ *     Llama-3-8B and -70B fits), else LWC_ERR_UNSUPPORTED before any device
+ *     work.
+ *   - d_src, d_blob, params, *desc_out and the stream behave as for the
+ *     two-call device encoder; if blob_bytes is below the blob's size the
+ *     call fails with LWC_ERR_INVALID_ARG and *desc_out holds the plan, whose
+ *     total_bytes is the size needed.
+ *   - The first call on a device (per process) looks up the scratch array's
+ *     device address for that device (cudaGetSymbolAddress, with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the
+ *     last call's contents (each call clears what must start at zero). Calls
+ *     whose GPU work overlaps — from several host threads, or on several
+ *     streams of one device — race on it and give wrong blobs: serialise
+ *     them. */
+LWC_API lwc_status lwc_encode_dfloat11_device_noalloc(const void *d_src, uint64_t n, const lwc_df11_params *params,
+                                                      void *d_blob, uint64_t blob_bytes, lwc_desc *desc_out,
+                                                      lwc_stream_t stream);
+
 /* ---- helpers -------------------------------------------------------------- */
 
 /* Static string naming a status code. */
