@@ -39,6 +39,7 @@ import synth  # noqa: E402
 METRIC = "decoded BF16 GB/s (DFloat11 layer-batched decode, Llama-3-8B layer)"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+DECODE_KERNEL = "df11_warp_kernel"   # blocks of 32 chunks, the encoder's default
 KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_device.cuh")
 
 
@@ -90,7 +91,7 @@ def profiled_traffic(workload: str):
         with open(PROFILE_TRAFFIC) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) == 4 and parts[0] == "df11_decode_kernel" and parts[1] == workload \
+                if len(parts) == 4 and parts[0] == DECODE_KERNEL and parts[1] == workload \
                         and parts[2] == kernel_sha():
                     return int(parts[3])
     except OSError:
@@ -299,7 +300,7 @@ def run_lwc(args, rank, world, local_rank, dist):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": profiled_traffic(workload),
                 "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
-                "kernel": "df11_decode_kernel", "launch_ms": round(launch_ms, 5)}
+                "kernel": DECODE_KERNEL, "launch_ms": round(launch_ms, 5)}
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,

@@ -463,6 +463,265 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
     if (bad && B.status) atomicOr(B.status, bad);
 }
 
+// ---- per-warp blocks ----------------------------------------------------------------
+//
+// Blobs encoded with threads_per_block = 32 have one block per 32 chunks, so a
+// single warp can decode a block on its own: its output offset is stored, the
+// scan is a warp scan, and nothing waits for the other warps of the CTA. The
+// CTA's 8 warps share the lookup tables (rebuilt, with CTA barriers, only
+// where the CTA's run of blocks crosses into the next tensor); each warp has
+// its own segment buffer, gap bytes, staging area and mbarrier, and walks the
+// blocks w, w + 8, w + 16, ... of the current tensor.
+constexpr uint32_t kWarpsPerCta = 8;
+
+struct WarpLayout {
+    uint32_t warp0, seg_bytes, stage, warp_bytes, bars, total;
+    __host__ __device__ WarpLayout(uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes) {
+        warp0 = kFastBytes + ((2 * lut_entries + 15) & ~15u);
+        seg_bytes = 4 * seg_words;
+        stage = seg_bytes + 48;   // the block's 32 gap bytes, then the next block's first 16
+        warp_bytes = stage + stage_bytes;
+        bars = warp0 + kWarpsPerCta * warp_bytes;
+        total = bars + 8 * kWarpsPerCta;
+    }
+};
+
+// Lane 0: start the bulk copies of block b of tensor `tn` into this warp's buffer.
+__device__ __forceinline__ void issue_warp_item(const Df11Batch &B, const Df11Tensor &tn, uint32_t b, uint8_t *buf,
+                                                uint32_t seg_bytes, uint64_t *bar) {
+    const uint64_t seg0 = (uint64_t)b * 32u * B.chunk_words * 4;   // multiple of 128
+    const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
+    const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
+    const uint32_t gbytes = b + 1 < tn.n_blocks ? 48u : 32u;
+    dev::mbar_arrive_expect_tx(bar, bytes + gbytes);
+    if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
+    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
+}
+
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    const WarpLayout L(B.seg_words, B.lut_entries, B.stage_bytes);
+    uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem);
+    uint16_t *mask_tab = reinterpret_cast<uint16_t *>(smem + kFastSize * 4);
+    uint8_t *cnt_tab = smem + kFastSize * 6;
+    uint16_t *lut = reinterpret_cast<uint16_t *>(smem + kFastBytes);
+    uint8_t *buf = smem + L.warp0 + warp * L.warp_bytes;
+    const uint32_t *seg = reinterpret_cast<const uint32_t *>(buf);
+    const uint8_t *gapb = buf + L.seg_bytes;
+    uint8_t *stage = buf + L.stage;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.bars) + warp;
+    const uint32_t seg_bytes = L.seg_bytes;
+    const uint32_t cbits = B.chunk_words * 32u;
+
+    const uint32_t W = B.total_work, G = gridDim.x;
+    const uint32_t w_begin = (uint32_t)((uint64_t)W * blockIdx.x / G);
+    const uint32_t w_end = (uint32_t)((uint64_t)W * (blockIdx.x + 1) / G);
+    if (w_begin >= w_end) return;
+    if (lane == 0) {
+        dev::mbar_init(bar, 1);
+        dev::fence_mbar_init();
+    }
+    __syncwarp();
+
+    uint32_t bad = 0, items = 0;
+    bool dead = false;   // a bounded wait gave up: this warp stops decoding
+    uint32_t ti = locate(B, w_begin, 0);
+    for (uint32_t w0 = w_begin; w0 < w_end;) {
+        const Df11Tensor &tn = B.t[ti];
+        const uint32_t t_end = ti + 1 < B.count ? B.t[ti + 1].first_work : W;
+        const uint32_t s_end = min(w_end, t_end);
+        // this tensor's tables (every warp is done with the previous ones)
+        __syncthreads();
+        const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
+        for (uint32_t i = tid; i < ntab * 128u; i += blockDim.x)
+            reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
+        __syncthreads();
+        build_fast_tables(lut, ntab, cnt_tab, mask_tab, sym_tab);
+        __syncthreads();
+
+        uint32_t w = w0 + warp;
+        if (w < s_end && lane == 0 && !dead) {
+            dev::fence_proxy_async_smem();
+            issue_warp_item(B, tn, w - tn.first_work, buf, seg_bytes, bar);
+        }
+        uint64_t o0n = 0, o1n = 0;
+        if (w < s_end) {
+            o0n = tn.blkoff[w - tn.first_work];
+            o1n = tn.blkoff[w - tn.first_work + 1];
+        }
+        for (; w < s_end && !dead; w += kWarpsPerCta) {
+            const uint32_t b = w - tn.first_work;
+            const uint64_t o0 = o0n, o1 = o1n;
+            const bool more = w + kWarpsPerCta < s_end;
+            if (more) {
+                o0n = tn.blkoff[b + kWarpsPerCta];
+                o1n = tn.blkoff[b + kWarpsPerCta + 1];
+            }
+            const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
+            const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
+            uint4 sv[kMergeRegs];
+#pragma unroll
+            for (int m = 0; m < kMergeRegs; m++) {
+                const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
+                sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
+            }
+            const bool arrived = dev::mbar_wait_bounded(bar, items & 1u);
+            items++;
+            if (__any_sync(0xFFFFFFFFu, !arrived)) {
+                bad |= LWC_DEVICE_TIMEOUT;
+                dead = true;
+                break;
+            }
+            bool next_issued = false;
+            if (ok) {
+                const uint64_t rem_block = tn.total_bits - (uint64_t)b * 32u * cbits;
+                const uint32_t start = lane * cbits + gapb[lane];
+                const bool has_next = lane + 1 < 32u || b + 1 < tn.n_blocks;
+                const uint64_t next = has_next ? (uint64_t)(lane + 1) * cbits + gapb[lane + 1] : rem_block;
+                const uint32_t end = (uint32_t)min(next, rem_block);
+
+                uint32_t count = 0;
+                if (start < end) {
+                    uint32_t pos = start, rem = end - start, acc = 0, sbits = 0, scount = 0;
+                    for (;;) {
+                        const uint32_t wv = window32(seg, pos);
+                        const uint32_t idx = wv >> (32 - kFastBits);
+                        const uint32_t e = cnt_tab[idx];
+                        const uint32_t len = e & 15u;
+                        const uint32_t e2 = cnt_tab[(wv << len) >> (32 - kFastBits)];
+                        const uint32_t l2 = e2 & 15u;
+                        if ((len - 1u < rem) & (l2 - 1u < rem - len)) {
+                            acc += e + e2;
+                            pos += len + l2;
+                            rem -= len + l2;
+                            continue;
+                        }
+                        if (len - 1u < rem) {
+                            acc += e;
+                            pos += len;
+                            rem -= len;
+                            continue;
+                        }
+                        if (rem == 0) break;
+                        if (e == 0) {
+                            const uint32_t l = lut_walk(lut, ntab, wv, bad) >> 8;
+                            if (l > rem) {
+                                bad |= LWC_DEVICE_BAD_CODE;
+                                break;
+                            }
+                            pos += l;
+                            rem -= l;
+                            sbits += l;
+                            scount++;
+                            continue;
+                        }
+                        scount += __popc(mask_tab[idx] & ((1u << rem) - 1u));
+                        break;
+                    }
+                    count = ((acc - (pos - start - sbits)) >> 4) + scount;
+                }
+
+                // warp scan of the counts
+                uint32_t x = count;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+                    if (lane >= (uint32_t)o) x += y;
+                }
+                const uint32_t total = __shfl_sync(0xFFFFFFFFu, x, 31);
+                const uint32_t first = x - count;
+                if (total == (uint32_t)(o1 - o0)) {
+                    if (start < end) {
+                        uint8_t *bp = stage + (uint32_t)(o0 & 15u) + first;
+                        uint32_t pos = start, rem = end - start;
+                        for (;;) {
+                            const uint32_t wv = window32(seg, pos);
+                            const uint32_t idx = wv >> (32 - kFastBits);
+                            const uint32_t e = sym_tab[idx];
+                            const uint32_t len = e >> 26;
+                            const uint32_t e2 = sym_tab[(wv << len) >> (32 - kFastBits)];
+                            const uint32_t l2 = e2 >> 26;
+                            if ((len - 1u < rem) & (l2 - 1u < rem - len)) {
+                                const uint32_t n = (e >> 24) & 3u, n2 = (e2 >> 24) & 3u;
+                                bp[0] = (uint8_t)e;
+                                if (n > 1) bp[1] = (uint8_t)(e >> 8);
+                                if (n > 2) bp[2] = (uint8_t)(e >> 16);
+                                uint8_t *bq = bp + n;
+                                bq[0] = (uint8_t)e2;
+                                if (n2 > 1) bq[1] = (uint8_t)(e2 >> 8);
+                                if (n2 > 2) bq[2] = (uint8_t)(e2 >> 16);
+                                bp = bq + n2;
+                                pos += len + l2;
+                                rem -= len + l2;
+                                continue;
+                            }
+                            if (len - 1u < rem) {
+                                const uint32_t n = (e >> 24) & 3u;
+                                bp[0] = (uint8_t)e;
+                                if (n > 1) bp[1] = (uint8_t)(e >> 8);
+                                if (n > 2) bp[2] = (uint8_t)(e >> 16);
+                                bp += n;
+                                pos += len;
+                                rem -= len;
+                                continue;
+                            }
+                            if (rem == 0) break;
+                            if (e == 0) {
+                                const uint32_t r = lut_walk(lut, ntab, wv, bad);
+                                const uint32_t l = r >> 8;
+                                if (l > rem) break;
+                                *bp++ = (uint8_t)r;
+                                pos += l;
+                                rem -= l;
+                                continue;
+                            }
+                            const uint32_t j = __popc(mask_tab[idx] & ((1u << rem) - 1u));   // < 3
+                            if (j > 0) bp[0] = (uint8_t)e;
+                            if (j > 1) bp[1] = (uint8_t)(e >> 8);
+                            break;
+                        }
+                    }
+                    __syncwarp();
+                    // the segment is free: fetch this warp's next block while merging this one
+                    if (lane == 0 && more) {
+                        dev::fence_proxy_async_smem();
+                        issue_warp_item(B, tn, b + kWarpsPerCta, buf, seg_bytes, bar);
+                    }
+                    next_issued = true;
+
+                    const uint64_t base = o0 & ~15ull;
+#pragma unroll
+                    for (int m = 0; m < kMergeRegs; m++) {
+                        const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
+                        if (g < g_hi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    }
+                    for (uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)kMergeRegs); g < g_hi; g += 16ull * 32u)
+                        merge16(__ldg(reinterpret_cast<const uint4 *>(tn.sm + g)),
+                                *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    // partial 16-groups at both ends
+                    const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
+                    const bool head = lane < 16 && i < min(g_lo, o1);
+                    const bool tail = lane >= 16 && i < o1;
+                    if (head || tail) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
+                } else {
+                    bad |= LWC_DEVICE_BAD_COUNT;
+                }
+            } else {
+                bad |= LWC_DEVICE_BAD_OFFSET;
+            }
+            __syncwarp();   // segment and staging area free again
+            if (lane == 0 && !next_issued && more) {
+                dev::fence_proxy_async_smem();
+                issue_warp_item(B, tn, b + kWarpsPerCta, buf, seg_bytes, bar);
+            }
+        }
+        w0 = s_end;
+        if (w0 < w_end) ti = locate(B, w0, ti);
+    }
+    if (bad && B.status) atomicOr(B.status, bad);
+}
+
 // One exponent value for the whole tensor: out = merge(const_exp, sm).
 __global__ void df11_const_kernel(const uint8_t *__restrict__ sm, uint16_t *__restrict__ out, uint64_t n,
                                   uint32_t const_exp) {
@@ -499,7 +758,8 @@ lwc_status device_config(DeviceConfig &out) {
     if (!c.ready) {
         err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
         if (err == cudaSuccess) err = cudaDeviceGetAttribute(&c.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        const void *kernels[] = {(const void *)df11_decode_kernel<256>, (const void *)df11_decode_kernel<1024>};
+        const void *kernels[] = {(const void *)df11_decode_kernel<256>, (const void *)df11_decode_kernel<1024>,
+                                 (const void *)df11_warp_kernel};
         for (const void *k : kernels) {
             if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
             if (err == cudaSuccess)
@@ -551,18 +811,26 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
-    const uint64_t smem = Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
+    const bool per_warp = T == 32;
+    const uint32_t threads = per_warp ? kWarpsPerCta * 32u : T;
+    const uint64_t smem = per_warp ? WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes).total
+                                   : Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
                     (unsigned long long)smem, cfg.max_smem);
-    const void *kernel = T <= 256 ? (const void *)df11_decode_kernel<256> : (const void *)df11_decode_kernel<1024>;
+    const void *kernel = per_warp ? (const void *)df11_warp_kernel
+                         : T <= 256 ? (const void *)df11_decode_kernel<256>
+                                    : (const void *)df11_decode_kernel<1024>;
     int per_sm = 0;
-    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)T, (size_t)smem);
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)threads, (size_t)smem);
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
-    if (per_sm < 1) return fail(LWC_ERR_UNSUPPORTED, "decoder does not fit on an SM (%u threads, %llu B smem)", T,
-                                (unsigned long long)smem);
-    const uint64_t grid = std::min<uint64_t>(work, (uint64_t)per_sm * cfg.sms);
-    if (T <= 256)
+    if (per_sm < 1) return fail(LWC_ERR_UNSUPPORTED, "decoder does not fit on an SM (%u threads, %llu B smem)",
+                                threads, (unsigned long long)smem);
+    const uint64_t units = per_warp ? (work + kWarpsPerCta - 1) / kWarpsPerCta : work;
+    const uint64_t grid = std::min<uint64_t>(units, (uint64_t)per_sm * cfg.sms);
+    if (per_warp)
+        df11_warp_kernel<<<(unsigned)grid, threads, (size_t)smem, stream>>>(B);
+    else if (T <= 256)
         df11_decode_kernel<256><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);
     else
         df11_decode_kernel<1024><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);

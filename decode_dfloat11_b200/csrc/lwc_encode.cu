@@ -687,9 +687,9 @@ lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const 
     h.magic = kWsMagic;
     h.codec = LWC_CODEC_DFLOAT11;
     h.n = n;
-    h.chunk_bytes = params ? params->chunk_bytes : 36;
-    h.threads_per_block = params ? params->threads_per_block : 256;
-    h.max_len = params ? params->max_len : 32;
+    h.chunk_bytes = params ? params->chunk_bytes : kDefaultChunkBytes;
+    h.threads_per_block = params ? params->threads_per_block : kDefaultThreadsPerBlock;
+    h.max_len = params ? params->max_len : kDefaultMaxLen;
     if (lwc_status st = check_df11_params(h.chunk_bytes, h.threads_per_block, h.max_len)) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *work = static_cast<uint8_t *>(d_work);

@@ -387,9 +387,9 @@ lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_p
                                lwc_desc *desc_out, void **blob_out, uint64_t *bytes_out) {
     lwc_status st = check_args(src, n, desc_out, blob_out, bytes_out);
     if (st) return st;
-    const uint32_t C = params ? params->chunk_bytes : 36;
-    const uint32_t T = params ? params->threads_per_block : 256;
-    const uint32_t L = params ? params->max_len : 32;
+    const uint32_t C = params ? params->chunk_bytes : kDefaultChunkBytes;
+    const uint32_t T = params ? params->threads_per_block : kDefaultThreadsPerBlock;
+    const uint32_t L = params ? params->max_len : kDefaultMaxLen;
 
     // exponent histogram, then the code and the section layout
     uint64_t counts[256] = {0};

@@ -20,6 +20,13 @@ constexpr uint32_t kFlagSingleExponent = 1u;
 constexpr uint32_t kFormatMaxLen = 32;      // longest Huffman code the format allows
 constexpr uint32_t kMaxTables = 256;        // lookup tables this build stages in shared memory
 
+// DFloat11 encoder defaults. Blocks of 32 chunks are decoded one per warp
+// (no CTA-wide barrier per block); a 36-byte chunk is an odd number of words,
+// so the 32 lanes of a warp read their chunks from different banks.
+constexpr uint32_t kDefaultChunkBytes = 36;
+constexpr uint32_t kDefaultThreadsPerBlock = 32;
+constexpr uint32_t kDefaultMaxLen = 32;
+
 // Record a message for lwc_last_error() and return `s`.
 lwc_status fail(lwc_status s, const char *fmt, ...);
 void clear_error();

@@ -159,7 +159,7 @@ def _src(h_src) -> np.ndarray:
     return a.reshape(-1)
 
 
-def lwc_encode_dfloat11(h_src, chunk_bytes: int = 36, threads_per_block: int = 256,
+def lwc_encode_dfloat11(h_src, chunk_bytes: int = 36, threads_per_block: int = 32,
                         max_len: int = 32) -> tuple[lwc_desc, np.ndarray]:
     """Encode host BF16 bit patterns (uint16 array); returns (desc, blob bytes)."""
     src = _src(h_src)
@@ -235,7 +235,7 @@ def lwc_encode_device_workspace_bytes(n: int) -> int:
 
 
 def lwc_encode_dfloat11_device_plan(d_src, n: int, d_work, work_bytes: int, chunk_bytes: int = 36,
-                                    threads_per_block: int = 256, max_len: int = 32, stream=None) -> lwc_desc:
+                                    threads_per_block: int = 32, max_len: int = 32, stream=None) -> lwc_desc:
     """Plan a DFloat11 blob for n device BF16 patterns; returns its descriptor."""
     desc = lwc_desc()
     params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
@@ -261,7 +261,7 @@ def lwc_encode_device_write(d_src, n: int, d_work, work_bytes: int, d_blob, blob
 
 
 def lwc_encode_dfloat11_device_noalloc(d_src, n: int, d_blob, blob_bytes: int, chunk_bytes: int = 36,
-                                       threads_per_block: int = 256, max_len: int = 32, stream=None) -> lwc_desc:
+                                       threads_per_block: int = 32, max_len: int = 32, stream=None) -> lwc_desc:
     """DFloat11 device encode without any device allocation (the library's
     own scratch array replaces the workspace); for callers that cannot call
     cudaMalloc. Returns the blob's descriptor."""

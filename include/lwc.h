@@ -123,7 +123,7 @@ typedef struct lwc_desc {
 } lwc_desc;
 
 /* DFloat11 encoder parameters; pass NULL for the defaults
- * (chunk_bytes 36, threads_per_block 256, max_len 32). chunk_bytes: multiple
+ * (chunk_bytes 36, threads_per_block 32, max_len 32). chunk_bytes: multiple
  * of 4 in [8, 1024]; threads_per_block: multiple of 32 in [32, 1024];
  * max_len: code length limit in [9, 32]. */
 typedef struct lwc_df11_params {

@@ -172,9 +172,10 @@ def test_side_stream_and_reuse():
         assert np.array_equal(host_u16(o), w)
 
 
-def test_df11_corruption_is_contained():
+@pytest.mark.parametrize("tpb", [32, 256])   # the per-warp and the per-CTA kernel
+def test_df11_corruption_is_contained(tpb):
     w = synth.as_u16(synth.small_square(6))
-    d, b = lwc.lwc_encode_dfloat11(w)
+    d, b = lwc.lwc_encode_dfloat11(w, threads_per_block=tpb)
     rng = np.random.default_rng(0)
     guard = 4096
     cases = []
@@ -189,7 +190,7 @@ def test_df11_corruption_is_contained():
     x[d.off_lut: d.off_lut + 512 * d.n_tables] = 0xFF
     cases.append(x)
     x = b.copy()                                   # gaps garbage
-    x[d.off_gaps: d.off_gaps + d.n_blocks * d.threads_per_block] = rng.integers(0, 256, d.n_blocks * 256)
+    x[d.off_gaps: d.off_gaps + d.n_blocks * d.threads_per_block] = rng.integers(0, 256, d.n_blocks * d.threads_per_block)
     cases.append(x)
     for i, x in enumerate(cases):
         xd = dev(x)
