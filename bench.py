@@ -51,6 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=("lwc", "reference"), default="lwc")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-encode", action="store_true", help="skip the device-encoder timing")
     ap.add_argument("--no-codebook", action="store_true")
     ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
     ap.add_argument("--workload", choices=("layer", "model8b", "model70b"), default="layer",
@@ -244,7 +245,9 @@ def run_lwc(args, rank, world, local_rank, dist):
 
     names, tensors = make_layer(layer)
     n_total = sum(w.size for w in tensors)
+    t_host = time.perf_counter()
     enc = encode_all(tensors, "df11")
+    host_encode_s = time.perf_counter() - t_host
     descs = [d for d, _ in enc]
     blobs_h = [b for _, b in enc]
     blob_bytes = sum(b.size for b in blobs_h)
@@ -362,6 +365,35 @@ def run_lwc(args, rank, world, local_rank, dist):
             "bits_per_weight": round(sd.bits_per_weight, 4),
             "hbm_frac": round((sb.size + 2 * ns) / (sms * 1e-3) / 1e9 / peak, 4)}
         del sbd, sout
+
+    # device encoders (load-time path): the same layer, already on the GPU,
+    # compressed there; blobs must equal the host encoder's byte for byte
+    if not args.no_encode:
+        from decode_dfloat11_b200.layers import encode_on_device
+        src = [torch.from_numpy(w.view(np.int16)).to(device) for w in tensors]
+        work = torch.empty(lwc.lwc_encode_device_workspace_bytes(max(w.size for w in tensors)),
+                           dtype=torch.uint8, device=device)
+        enc_res = {"workload": "llama3-8b-layer, 7 tensors on the GPU, plan + write per tensor",
+                   "host_df11_ms": round(host_encode_s * 1e3, 1), "host_threads": min(8, len(tensors))}
+        for codec in ("dfloat11", "codebook"):
+            got = [encode_on_device(t, codec, workspace=work) for t in src]
+            ref = blobs_h if codec == "dfloat11" else [b for _, b in encode_all(tensors, "codebook")]
+            if not all(np.array_equal(b.cpu().numpy(), r) for (_, b), r in zip(got, ref)):
+                raise SystemExit(f"device {codec} encoder differs from the host encoder")
+            del got
+            reps = 3
+            torch.cuda.synchronize(device)
+            t0 = time.perf_counter()
+            for _ in range(reps):
+                for t in src:
+                    encode_on_device(t, codec, workspace=work)
+            torch.cuda.synchronize(device)
+            ems_enc = (time.perf_counter() - t0) / reps * 1e3
+            enc_res[f"{codec}_ms"] = round(ems_enc, 3)
+            enc_res[f"{codec}_gbs"] = round(2 * n_total / (ems_enc * 1e-3) / 1e9, 1)
+        enc_res["same_bytes_as_host"] = True
+        result["encode"] = enc_res
+        del src, work
 
     # end to end through the C ABI with host buffers: pinned blobs -> device,
     # decode, decoded layer -> pinned host, every step

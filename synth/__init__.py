@@ -87,6 +87,21 @@ def normal_bf16(shape, seed: int, sigma: float | None = None,
     return x.to(torch.bfloat16)
 
 
+def normal_fp16(shape, seed: int, sigma: float, outlier_frac: float = 0.0, outlier_scale: float = 20.0,
+                device="cpu") -> torch.Tensor:
+    """N(0, sigma) weights rounded to FP16 (same draws as normal_bf16 with a
+    fixed sigma, different rounding): the FP16 proof-of-concept workload of
+    the codebook pages, as 16-bit patterns for either codec."""
+    g = _gen(seed, device)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    x.mul_(sigma)
+    if outlier_frac > 0.0:
+        mask = torch.rand(shape, generator=g, device=device, dtype=torch.float32) < outlier_frac
+        x[mask] *= outlier_scale
+        del mask
+    return x.to(torch.float16)
+
+
 def small_square(seed: int = 0, device="cpu") -> torch.Tensor:
     """1024 x 1024 weights, i.i.d. N(0, 0.02), BF16."""
     return normal_bf16((1024, 1024), seed, sigma=0.02, device=device)

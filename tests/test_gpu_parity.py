@@ -259,3 +259,19 @@ def test_df11_uniform_exponents_full_size():
     out = gpu_decode(d, dev(b))
     assert torch.equal(out, x.view(torch.int16))
     assert np.array_equal(host_u16(out), odf.decode(b))
+
+
+@pytest.mark.parametrize("codec", ["codebook", "dfloat11"])
+def test_fp16_patterns(codec):
+    """FP16 weights as 16-bit patterns through both decoders, against the oracle."""
+    w = synth.as_u16(synth.normal_fp16((1_000_003,), seed=12, sigma=0.02, outlier_frac=1e-3))
+    if codec == "codebook":
+        d, b = lwc.lwc_encode_codebook(w)
+        ref = ocb.decode(b)
+        got = host_u16(gpu_decode(d, dev(b), "cb"))
+    else:
+        d, b = lwc.lwc_encode_dfloat11(w)
+        ref = odf.decode(b)
+        got = host_u16(gpu_decode(d, dev(b), "df11"))
+    assert np.array_equal(ref, w)
+    assert np.array_equal(got, w)

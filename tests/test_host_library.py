@@ -241,3 +241,21 @@ def test_device_encoder_validates_before_any_device_call():
     assert L.lwc_encode_codebook_device_plan(0x1000, n, 0x2000, need, None, None) == 1
     assert L.lwc_encode_device_write(0x1000, n, 0x2000, need, 0x3000, 1 << 20, None, None) == 1
     del desc
+
+
+def test_fp16_weights_through_both_codecs():
+    """FP16 weights (the codebook pages' proof of concept used FP16): both
+    codecs take any 16-bit patterns, so FP16 round-trips bit for bit. The
+    codebook's index width follows the tensor's distinct FP16 values; the
+    DFloat11 split is BF16-specific, so on FP16 patterns it is lossless but
+    compresses less (its 'exponent' byte straddles FP16's exponent and
+    mantissa)."""
+    w = synth.as_u16(synth.normal_fp16((300_007,), seed=11, sigma=0.02, outlier_frac=1e-3))
+    d, b = lwc.lwc_encode_codebook(w)
+    assert d.U == len(np.unique(w)) and d.k == ocb.index_bits(d.U)
+    assert np.array_equal(ocb.decode(b), w)
+    assert np.array_equal(b, ocb.encode(w))
+    d2, b2 = lwc.lwc_encode_dfloat11(w)
+    assert np.array_equal(odf.decode(b2), w)
+    assert odf.check_index(b2) == []
+    assert d2.bits_per_weight > 11.0   # far less skewed 'exponent' byte than BF16's
