@@ -152,7 +152,7 @@ __device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *c
 // The 32 stream bits starting at bit `pos` of the staged segment.
 __device__ __forceinline__ uint32_t window32(const uint32_t *seg, uint32_t pos) {
     const uint32_t i = pos >> 5;
-    return __funnelshift_l(seg[i + 1], seg[i], pos & 31u);
+    return __funnelshift_l(seg[i + 1], seg[i], pos);   // the shift amount is taken mod 32
 }
 
 // ---- merge ---------------------------------------------------------------------
@@ -468,11 +468,13 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
 // Blobs encoded with threads_per_block = 32 have one block per 32 chunks, so a
 // single warp can decode a block on its own: its output offset is stored, the
 // scan is a warp scan, and nothing waits for the other warps of the CTA. The
-// CTA's 8 warps share the lookup tables (rebuilt, with CTA barriers, only
+// CTA's 12 warps share the lookup tables (rebuilt, with CTA barriers, only
 // where the CTA's run of blocks crosses into the next tensor); each warp has
 // its own segment buffer, gap bytes, staging area and mbarrier, and walks the
-// blocks w, w + 8, w + 16, ... of the current tensor.
-constexpr uint32_t kWarpsPerCta = 8;
+// blocks w, w + 12, w + 24, ... of the current tensor.
+constexpr uint32_t kWarpsPerCta = 12;   // 3 CTAs (36 warps) per SM fit registers and shared memory
+constexpr int kWarpCtasPerSm = 3;
+constexpr int kWarpMergeRegs = 3;       // 16-weight merge groups per lane whose loads are issued early
 
 struct WarpLayout {
     uint32_t warp0, seg_bytes, stage, warp_bytes, bars, total;
@@ -498,7 +500,7 @@ __device__ __forceinline__ void issue_warp_item(const Df11Batch &B, const Df11Te
     dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
 }
 
-__global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const WarpLayout L(B.seg_words, B.lut_entries, B.stage_bytes);
@@ -560,9 +562,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) df11_warp_kerne
             }
             const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
             const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
-            uint4 sv[kMergeRegs];
+            uint4 sv[kWarpMergeRegs];
 #pragma unroll
-            for (int m = 0; m < kMergeRegs; m++) {
+            for (int m = 0; m < kWarpMergeRegs; m++) {
                 const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
                 sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
             }
@@ -643,14 +645,15 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) df11_warp_kerne
                             const uint32_t e2 = sym_tab[(wv << len) >> (32 - kFastBits)];
                             const uint32_t l2 = e2 >> 26;
                             if ((len - 1u < rem) & (l2 - 1u < rem - len)) {
+                                // n is 1..3: bit 25 set means n >= 2, bits 24 and 25 set mean n = 3
                                 const uint32_t n = (e >> 24) & 3u, n2 = (e2 >> 24) & 3u;
                                 bp[0] = (uint8_t)e;
-                                if (n > 1) bp[1] = (uint8_t)(e >> 8);
-                                if (n > 2) bp[2] = (uint8_t)(e >> 16);
+                                if (e & (1u << 25)) bp[1] = (uint8_t)(e >> 8);
+                                if ((e & 0x3000000u) == 0x3000000u) bp[2] = (uint8_t)(e >> 16);
                                 uint8_t *bq = bp + n;
                                 bq[0] = (uint8_t)e2;
-                                if (n2 > 1) bq[1] = (uint8_t)(e2 >> 8);
-                                if (n2 > 2) bq[2] = (uint8_t)(e2 >> 16);
+                                if (e2 & (1u << 25)) bq[1] = (uint8_t)(e2 >> 8);
+                                if ((e2 & 0x3000000u) == 0x3000000u) bq[2] = (uint8_t)(e2 >> 16);
                                 bp = bq + n2;
                                 pos += len + l2;
                                 rem -= len + l2;
@@ -690,15 +693,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kCtasPerSm) df11_warp_kerne
                     }
                     next_issued = true;
 
+                    // 32-bit offsets from the block's first 16-weight group
                     const uint64_t base = o0 & ~15ull;
+                    const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
+                    uint16_t *ob = tn.out + base;
+                    const uint8_t *sb = tn.sm + base;
 #pragma unroll
-                    for (int m = 0; m < kMergeRegs; m++) {
-                        const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
-                        if (g < g_hi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    for (int m = 0; m < kWarpMergeRegs; m++) {
+                        const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
+                        if (r < rhi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob + r);
                     }
-                    for (uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)kMergeRegs); g < g_hi; g += 16ull * 32u)
-                        merge16(__ldg(reinterpret_cast<const uint4 *>(tn.sm + g)),
-                                *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
+                        merge16(__ldg(reinterpret_cast<const uint4 *>(sb + r)), *reinterpret_cast<const uint4 *>(stage + r),
+                                ob + r);
                     // partial 16-groups at both ends
                     const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
                     const bool head = lane < 16 && i < min(g_lo, o1);
@@ -865,6 +872,8 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
     for (int i = 0; i < count; i++) {
         lwc_status st = check_df11_desc(&descs[i]);
         if (st) return st;
+        if (descs[i].elem != LWC_ELEM_BF16)
+            return fail(LWC_ERR_UNSUPPORTED, "tensor %d: element type %u is not decoded by this build", i, descs[i].elem);
         if (descs[i].n == 0) continue;
         if (!d_ins[i] || !d_outs[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (tensor %d)", i);
         if (!aligned16(d_ins[i]) || !aligned16(d_outs[i]))

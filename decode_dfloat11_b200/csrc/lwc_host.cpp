@@ -74,6 +74,9 @@ void write_header(uint8_t *h, const lwc_desc &d) {
         put<uint64_t>(h, 112, d.off_stream);
         put<uint64_t>(h, 120, d.stream_bytes);
         put<uint64_t>(h, 128, d.off_sm);
+        put<uint32_t>(h, 136, d.elem);
+        put<uint64_t>(h, 144, d.off_lo);
+        put<uint64_t>(h, 152, d.lo_bytes);
     } else {
         put<uint32_t>(h, 32, d.U);
         put<uint32_t>(h, 36, d.k);
@@ -110,6 +113,9 @@ void read_header(const uint8_t *h, lwc_desc &d) {
         d.off_stream = get<uint64_t>(h, 112);
         d.stream_bytes = get<uint64_t>(h, 120);
         d.off_sm = get<uint64_t>(h, 128);
+        d.elem = get<uint32_t>(h, 136);
+        d.off_lo = get<uint64_t>(h, 144);
+        d.lo_bytes = get<uint64_t>(h, 152);
     } else if (d.codec == LWC_CODEC_CODEBOOK) {
         d.U = get<uint32_t>(h, 32);
         d.k = get<uint32_t>(h, 36);
@@ -250,7 +256,14 @@ lwc_status check_df11_params(uint32_t C, uint32_t T, uint32_t L) {
     return LWC_OK;
 }
 
-lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uint32_t T, uint32_t L, Df11Plan &p) {
+uint64_t lo_section_bytes(uint32_t elem, uint64_t n) {
+    if (elem == LWC_ELEM_FP32) return round_up(2 * n, 16);
+    if (elem == LWC_ELEM_FP16) return round_up((3 * n + 7) / 8 + 16, 16);
+    return 0;
+}
+
+lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uint32_t T, uint32_t L, Df11Plan &p,
+                         uint64_t lo_bytes) {
     if (lwc_status st = check_df11_params(C, T, L)) return st;
     int present = 0, only = 0;
     for (int s = 0; s < 256; s++)
@@ -294,6 +307,10 @@ lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uin
     d.off_blkoff = lay.place(8 * (d.n_blocks + 1));
     d.off_stream = lay.place(d.stream_bytes);
     d.off_sm = lay.place(round_up(n, 16));
+    if (lo_bytes) {
+        d.off_lo = lay.place(lo_bytes);
+        d.lo_bytes = lo_bytes;
+    }
     d.total_bytes = lay.total();
     return LWC_OK;
 }
@@ -337,6 +354,12 @@ lwc_status check_df11_desc(const lwc_desc *d) {
                     (unsigned long long)C, (unsigned long long)T);
     if (!inside(d->off_sm, round_up(d->n, 16), tot) || !inside(d->off_lengths, 256, tot))
         return fail(LWC_ERR_CORRUPT, "sign/mantissa or lengths section outside the blob");
+    if (d->elem > LWC_ELEM_FP16) return fail(LWC_ERR_CORRUPT, "unknown element type %u", d->elem);
+    if (d->elem != LWC_ELEM_BF16 && d->n) {
+        const uint64_t need = d->elem == LWC_ELEM_FP32 ? 2 * d->n : (3 * d->n + 7) / 8 + 8;
+        if (d->lo_bytes < need || !inside(d->off_lo, d->lo_bytes, tot))
+            return fail(LWC_ERR_CORRUPT, "low-mantissa section too short or outside the blob");
+    }
     if (d->n == 0 || (d->flags & kFlagSingleExponent)) {
         if (d->const_exp > 255) return fail(LWC_ERR_CORRUPT, "bad const_exp");
         return LWC_OK;
@@ -377,16 +400,12 @@ lwc_status check_codebook_desc(const lwc_desc *d) {
     return LWC_OK;
 }
 
-}  // namespace lwc
-
-using namespace lwc;
-
-extern "C" {
-
-lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_params *params,
-                               lwc_desc *desc_out, void **blob_out, uint64_t *bytes_out) {
-    lwc_status st = check_args(src, n, desc_out, blob_out, bytes_out);
-    if (st) return st;
+// The DFloat11 encoder proper, on BF16-shaped 16-bit patterns; for FP32 and
+// FP16 elements `lo` holds the raw low-mantissa section (lo_len bytes) and
+// `elem` is recorded in the header.
+lwc_status encode_df11(const uint16_t *src, uint64_t n, const lwc_df11_params *params, uint32_t elem,
+                       const uint8_t *lo, uint64_t lo_len, lwc_desc *desc_out, void **blob_out, uint64_t *bytes_out) {
+    lwc_status st;
     const uint32_t C = params ? params->chunk_bytes : kDefaultChunkBytes;
     const uint32_t T = params ? params->threads_per_block : kDefaultThreadsPerBlock;
     const uint32_t L = params ? params->max_len : kDefaultMaxLen;
@@ -395,8 +414,9 @@ lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_p
     uint64_t counts[256] = {0};
     for (uint64_t i = 0; i < n; i++) counts[(src[i] >> 7) & 0xFF]++;
     Df11Plan plan;
-    st = plan_dfloat11(counts, n, C, T, L, plan);
+    st = plan_dfloat11(counts, n, C, T, L, plan, lo_section_bytes(elem, n));
     if (st) return st;
+    plan.d.elem = elem;
     lwc_desc &d = plan.d;
     const bool present2 = !plan.single;
     const uint32_t *len = plan.len, *code = plan.code;
@@ -458,12 +478,60 @@ lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_p
             return fail(LWC_ERR_CORRUPT, "internal: bit count mismatch");
         }
     }
+    if (lo_len) std::memcpy(blob + d.off_lo, lo, lo_len);
     write_header(blob, d);
     *desc_out = d;
     *blob_out = blob;
     *bytes_out = d.total_bytes;
     clear_error();
     return LWC_OK;
+}
+
+}  // namespace lwc
+
+using namespace lwc;
+
+extern "C" {
+
+lwc_status lwc_encode_dfloat11(const uint16_t *src, uint64_t n, const lwc_df11_params *params,
+                               lwc_desc *desc_out, void **blob_out, uint64_t *bytes_out) {
+    lwc_status st = check_args(src, n, desc_out, blob_out, bytes_out);
+    if (st) return st;
+    return encode_df11(src, n, params, LWC_ELEM_BF16, nullptr, 0, desc_out, blob_out, bytes_out);
+}
+
+lwc_status lwc_encode_dfloat11_elements(const void *src, uint64_t n, uint32_t elem, const lwc_df11_params *params,
+                                        lwc_desc *desc_out, void **blob_out, uint64_t *bytes_out) {
+    lwc_status st = check_args(static_cast<const uint16_t *>(src), n, desc_out, blob_out, bytes_out);
+    if (st) return st;
+    if (elem == LWC_ELEM_BF16)
+        return encode_df11(static_cast<const uint16_t *>(src), n, params, elem, nullptr, 0, desc_out, blob_out,
+                           bytes_out);
+    if (elem != LWC_ELEM_FP32 && elem != LWC_ELEM_FP16) return fail(LWC_ERR_INVALID_ARG, "unknown element type %u", elem);
+    // BF16-shaped patterns + raw low mantissa bits
+    std::vector<uint16_t> v(n);
+    std::vector<uint8_t> lo;
+    if (elem == LWC_ELEM_FP32) {
+        const uint32_t *x = static_cast<const uint32_t *>(src);
+        lo.resize(2 * n);
+        for (uint64_t i = 0; i < n; i++) {
+            v[i] = (uint16_t)(x[i] >> 16);
+            const uint16_t l = (uint16_t)x[i];
+            std::memcpy(&lo[2 * i], &l, 2);
+        }
+    } else {
+        const uint16_t *x = static_cast<const uint16_t *>(src);
+        lo.assign((3 * n + 7) / 8, 0);
+        for (uint64_t i = 0; i < n; i++) {
+            const uint32_t w = x[i], mant = w & 0x3FF;
+            v[i] = (uint16_t)((w & 0x8000) | (((w >> 10) & 0x1F) << 7) | (mant >> 3));
+            const uint64_t b = 3 * i;   // 3 bits at stream bit b, least significant first
+            const uint32_t l = mant & 7;
+            lo[b >> 3] |= (uint8_t)(l << (b & 7));
+            if ((b & 7) > 5) lo[(b >> 3) + 1] |= (uint8_t)(l >> (8 - (b & 7)));
+        }
+    }
+    return encode_df11(v.data(), n, params, elem, lo.data(), lo.size(), desc_out, blob_out, bytes_out);
 }
 
 lwc_status lwc_encode_codebook(const uint16_t *src, uint64_t n, lwc_desc *desc_out, void **blob_out,

@@ -62,8 +62,13 @@ struct Df11Plan {
     bool single;   // one exponent value (or n = 0): no stream
 };
 lwc_status check_df11_params(uint32_t chunk_bytes, uint32_t threads_per_block, uint32_t max_len);
+// lo_bytes: size of the raw low-mantissa section placed after the
+// sign|mantissa bytes (FP32 and FP16 elements; 0 for BF16).
 lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t chunk_bytes, uint32_t threads_per_block,
-                         uint32_t max_len, Df11Plan &plan);
+                         uint32_t max_len, Df11Plan &plan, uint64_t lo_bytes = 0);
+
+// Size of the raw low-mantissa section for n elements of type elem.
+uint64_t lo_section_bytes(uint32_t elem, uint64_t n);
 
 // Codebook blob plan from the set of present 16-bit patterns (seen[v] != 0).
 struct CbPlan {

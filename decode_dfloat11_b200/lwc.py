@@ -19,6 +19,9 @@ LIB_PATH = os.path.join(_HERE, "liblwc.so")
 LWC_OK = 0
 LWC_CODEC_DFLOAT11 = 1
 LWC_CODEC_CODEBOOK = 2
+LWC_ELEM_BF16 = 0
+LWC_ELEM_FP32 = 1
+LWC_ELEM_FP16 = 2
 LWC_DEVICE_BAD_COUNT = 1
 LWC_DEVICE_BAD_CODE = 2
 LWC_DEVICE_BAD_OFFSET = 4
@@ -29,7 +32,7 @@ STATUS_NAMES = {0: "LWC_OK", 1: "LWC_ERR_INVALID_ARG", 2: "LWC_ERR_MISALIGNED", 
 
 # Every symbol include/lwc.h declares.
 EXPORTED = (
-    "lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
+    "lwc_encode_dfloat11", "lwc_encode_dfloat11_elements", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
     "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
     "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
     "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan", "lwc_encode_codebook_device_plan",
@@ -57,6 +60,8 @@ class lwc_desc(ctypes.Structure):
         ("off_sm", ctypes.c_uint64),
         ("U", ctypes.c_uint32), ("k", ctypes.c_uint32), ("off_table", ctypes.c_uint64),
         ("off_packed", ctypes.c_uint64), ("packed_bytes", ctypes.c_uint64),
+        ("elem", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("off_lo", ctypes.c_uint64),
+        ("lo_bytes", ctypes.c_uint64),
     ]
 
     def as_dict(self):
@@ -89,6 +94,8 @@ def load():
     L.lwc_encode_dfloat11.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), D,
                                       ctypes.POINTER(_P), ctypes.POINTER(_u64)]
     L.lwc_encode_codebook.argtypes = [_P, _u64, D, ctypes.POINTER(_P), ctypes.POINTER(_u64)]
+    L.lwc_encode_dfloat11_elements.argtypes = [_P, _u64, ctypes.c_uint32, ctypes.POINTER(lwc_df11_params), D,
+                                               ctypes.POINTER(_P), ctypes.POINTER(_u64)]
     L.lwc_free.argtypes = [_P]
     L.lwc_free.restype = None
     L.lwc_desc_from_blob.argtypes = [_P, _u64, D]
@@ -109,7 +116,7 @@ def load():
     L.lwc_last_error.argtypes = []
     L.lwc_last_error.restype = ctypes.c_char_p
     L.lwc_version.argtypes = []
-    for name in ("lwc_encode_dfloat11", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
+    for name in ("lwc_encode_dfloat11", "lwc_encode_dfloat11_elements", "lwc_encode_codebook", "lwc_desc_from_blob", "lwc_decode_dfloat11",
                  "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
                  "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched", "lwc_encode_dfloat11_device_plan",
                  "lwc_encode_codebook_device_plan", "lwc_encode_device_write",
@@ -167,6 +174,22 @@ def lwc_encode_dfloat11(h_src, chunk_bytes: int = 36, threads_per_block: int = 3
     params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
     _check(load().lwc_encode_dfloat11(src.ctypes.data, src.size, ctypes.byref(params), ctypes.byref(desc),
                                       ctypes.byref(ptr), ctypes.byref(nbytes)))
+    return desc, _take_blob(ptr, nbytes.value)
+
+
+def lwc_encode_dfloat11_elements(h_src, elem: int, chunk_bytes: int = 36, threads_per_block: int = 32,
+                                 max_len: int = 32) -> tuple[lwc_desc, np.ndarray]:
+    """DFloat11 encode of FP32 (uint32 / float32 array), FP16 or BF16 (16-bit) elements."""
+    a = np.ascontiguousarray(h_src).reshape(-1)
+    want = np.uint32 if elem == LWC_ELEM_FP32 else np.uint16
+    if a.dtype != want:
+        if a.dtype.itemsize != np.dtype(want).itemsize:
+            raise ValueError(f"element type {elem} needs {np.dtype(want).itemsize}-byte elements")
+        a = a.view(want)
+    desc, ptr, nbytes = lwc_desc(), _P(), _u64()
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    _check(load().lwc_encode_dfloat11_elements(a.ctypes.data, a.size, elem, ctypes.byref(params), ctypes.byref(desc),
+                                               ctypes.byref(ptr), ctypes.byref(nbytes)))
     return desc, _take_blob(ptr, nbytes.value)
 
 

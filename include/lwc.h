@@ -27,7 +27,9 @@
  *  - The caller copies the blob, byte for byte, to a device buffer it owns
  *    (d_in) and keeps the lwc_desc (a plain struct in host memory).
  *  - Decoders run asynchronously on the caller's CUDA stream and write n
- *    BF16 values (2n bytes) to the caller's device buffer d_out_bf16.
+ *    BF16 values (2n bytes) to the caller's device buffer d_out_bf16
+ *    (for DFloat11 blobs of another element type: n elements of that type,
+ *    4n bytes for FP32).
  *    They allocate no memory (host or device) and never synchronise.
  *  - d_in and d_out_bf16 must be 16-byte aligned (else LWC_ERR_MISALIGNED).
  *
@@ -78,6 +80,21 @@ enum {
     LWC_CODEC_CODEBOOK = 2
 };
 
+/* Element types of a DFloat11 blob (lwc_desc.elem). The DFloat11 idea --
+ * entropy-code the exponent, keep sign and mantissa raw -- carried from BF16
+ * to the other float formats. Each element becomes a 16-bit pattern laid out
+ * like BF16 (sign, exponent field, 7 mantissa bits), coded as a BF16 tensor,
+ * plus the mantissa bits that do not fit, kept raw in the "lo" section:
+ *   FP32: the top 16 bits are a BF16 pattern; low 16 bits raw (uint16[n]).
+ *   FP16: sign | 5-bit exponent | top 7 mantissa bits; the low 3 mantissa
+ *         bits packed 3 per weight, least significant bits first.
+ * Decoders write n elements of the blob's type (4 bytes each for FP32). */
+enum {
+    LWC_ELEM_BF16 = 0,
+    LWC_ELEM_FP32 = 1,
+    LWC_ELEM_FP16 = 2
+};
+
 /* Bits OR-ed into the optional device status word by the decoders. */
 enum {
     LWC_DEVICE_BAD_COUNT = 1u,   /* a block decoded a different number of codes than blkoff says */
@@ -120,6 +137,11 @@ typedef struct lwc_desc {
     uint64_t off_table;        /* u16[U], ascending */
     uint64_t off_packed;       /* k-bit indices, LSB first */
     uint64_t packed_bytes;
+    /* DFloat11 element type (header bytes 136..159; zero in BF16 blobs) */
+    uint32_t elem;             /* LWC_ELEM_* */
+    uint32_t reserved;
+    uint64_t off_lo;           /* raw low mantissa bits (FP32, FP16) */
+    uint64_t lo_bytes;
 } lwc_desc;
 
 /* DFloat11 encoder parameters; pass NULL for the defaults
@@ -141,6 +163,15 @@ typedef struct lwc_df11_params {
  * LWC_ERR_NOMEM. */
 LWC_API lwc_status lwc_encode_dfloat11(const uint16_t *h_src, uint64_t n, const lwc_df11_params *params,
                                lwc_desc *desc_out, void **h_blob_out, uint64_t *blob_bytes_out);
+
+/* DFloat11 compression of n elements of type `elem` (LWC_ELEM_*): h_src
+ * holds uint32 patterns for FP32, uint16 patterns for FP16 and BF16 (BF16 is
+ * exactly lwc_encode_dfloat11). Same ownership and errors; LWC_ERR_INVALID_ARG
+ * for an unknown element type. Not part of the pages' method, which is
+ * defined for BF16. */
+LWC_API lwc_status lwc_encode_dfloat11_elements(const void *h_src, uint64_t n, uint32_t elem,
+                                                const lwc_df11_params *params, lwc_desc *desc_out,
+                                                void **h_blob_out, uint64_t *blob_bytes_out);
 
 /* Compress n BF16 bit patterns with the codebook codec (table of the U
  * distinct patterns in ascending order + k = ceil(log2 U)-bit indices).

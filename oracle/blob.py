@@ -18,6 +18,9 @@ VERSION = 1
 CODEC_DFLOAT11 = 1
 CODEC_CODEBOOK = 2
 FLAG_SINGLE_EXPONENT = 1
+ELEM_BF16 = 0   # DFloat11 element types (header field "elem")
+ELEM_FP32 = 1
+ELEM_FP16 = 2
 HEADER_BYTES = 256
 SECTION_ALIGN = 256
 
@@ -32,7 +35,7 @@ DF11 = (
     ("total_bits", 64, "Q"), ("max_block_count", 72, "I"), ("const_exp", 76, "I"),
     ("off_lengths", 80, "Q"), ("off_lut", 88, "Q"), ("off_gaps", 96, "Q"),
     ("off_blkoff", 104, "Q"), ("off_stream", 112, "Q"), ("stream_bytes", 120, "Q"),
-    ("off_sm", 128, "Q"),
+    ("off_sm", 128, "Q"), ("elem", 136, "I"), ("off_lo", 144, "Q"), ("lo_bytes", 152, "Q"),
 )
 CODEBOOK = (
     ("U", 32, "I"), ("k", 36, "I"), ("off_table", 40, "Q"), ("off_packed", 48, "Q"),

@@ -100,8 +100,11 @@ def chunk_index(code_lengths_per_weight: np.ndarray, total_bits: int, chunk_bits
 
 def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
            threads_per_block: int = DEFAULT_THREADS_PER_BLOCK,
-           max_len: int = DEFAULT_MAX_LEN) -> np.ndarray:
-    """Compress BF16 bit patterns into a DFloat11 blob (uint8 array)."""
+           max_len: int = DEFAULT_MAX_LEN, _elem: int = B.ELEM_BF16, _lo=None) -> np.ndarray:
+    """Compress BF16 bit patterns into a DFloat11 blob (uint8 array).
+
+    (``_elem`` / ``_lo`` are used by ``encode_elements`` for FP32 and FP16:
+    the element type recorded in the header and the low-mantissa section.)"""
     if chunk_bytes % 4 or chunk_bytes < 8 or threads_per_block % 32 or not 32 <= threads_per_block <= 1024:
         raise ValueError("bad chunk/block parameters")
     if not 1 <= max_len <= FORMAT_MAX_LEN:
@@ -114,7 +117,10 @@ def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
     lengths = H.limited_lengths(counts, max_len)
     header = dict(magic=B.MAGIC, version=B.VERSION, codec=B.CODEC_DFLOAT11, n=n,
                   header_bytes=B.HEADER_BYTES, chunk_bytes=chunk_bytes,
-                  threads_per_block=threads_per_block)
+                  threads_per_block=threads_per_block, elem=_elem)
+    lo_sections = [] if _lo is None else [("lo", _lo)]
+    if _lo is not None:
+        header["lo_bytes"] = _lo.nbytes
     len_arr = np.array(lengths, np.uint8)
     sm = np.zeros(B.align(n, 16), np.uint8)
     sm[:n] = s
@@ -123,7 +129,7 @@ def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
                       const_exp=present[0] if present else 0)
         sections = [("lengths", len_arr), ("lut", np.zeros(0, np.uint16)),
                     ("gaps", np.zeros(0, np.uint8)), ("blkoff", np.zeros(0, np.uint64)),
-                    ("stream", np.zeros(0, np.uint32)), ("sm", sm)]
+                    ("stream", np.zeros(0, np.uint32)), ("sm", sm)] + lo_sections
         return B.assemble(header, sections)
 
     codes = H.canonical_codes(lengths)
@@ -144,7 +150,7 @@ def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
                   max_block_count=int(np.diff(blkoff).max()), const_exp=0,
                   stream_bytes=stream_bytes)
     sections = [("lengths", len_arr), ("lut", np.array(tables, np.uint16).reshape(-1)),
-                ("gaps", gaps), ("blkoff", blkoff), ("stream", words), ("sm", sm)]
+                ("gaps", gaps), ("blkoff", blkoff), ("stream", words), ("sm", sm)] + lo_sections
     return B.assemble(header, sections)
 
 
@@ -192,7 +198,9 @@ def decode_exponents(blob: np.ndarray, h: dict | None = None, want_lengths: bool
 
 
 def decode(blob: np.ndarray) -> np.ndarray:
-    """Decompress a DFloat11 blob back to the BF16 bit patterns (uint16)."""
+    """Decompress a DFloat11 blob back to the BF16 bit patterns (uint16).
+    For FP32 / FP16 blobs this is the intermediate 16-bit pattern; use
+    ``decode_elements`` for the elements themselves."""
     blob = np.asarray(blob, np.uint8)
     h = B.unpack_header(blob)
     if h["codec"] != B.CODEC_DFLOAT11:
@@ -200,6 +208,111 @@ def decode(blob: np.ndarray) -> np.ndarray:
     e = decode_exponents(blob, h)
     sm, _ = _parts(blob, h)
     return merge(e, np.ascontiguousarray(sm))
+
+
+# ---------------------------------------------------------------- FP32 and FP16
+#
+# The DFloat11 idea carried to the other float formats: entropy-code the
+# exponent, keep sign and mantissa as they are. Each element is mapped to a
+# 16-bit pattern laid out like BF16 (sign, 8-bit exponent field, 7 mantissa
+# bits), which goes through the BF16 codec above, plus the mantissa bits that
+# do not fit, stored raw in a "lo" section:
+#  * FP32 (1 + 8 + 23 bits): the top 16 bits are exactly a BF16 pattern; the
+#    low 16 mantissa bits are stored as uint16.
+#  * FP16 (1 + 5 + 10 bits): the pattern is sign | exponent (0..31, in the
+#    8-bit field) | top 7 mantissa bits; the low 3 mantissa bits are packed,
+#    3 bits per weight, least significant bits first.
+
+def split_elements(x: np.ndarray, elem: int):
+    """(v, lo): the BF16-shaped 16-bit patterns and the raw low mantissa bits."""
+    if elem == B.ELEM_BF16:
+        return np.ascontiguousarray(x, np.uint16).reshape(-1), None
+    if elem == B.ELEM_FP32:
+        x = np.ascontiguousarray(x, np.uint32).reshape(-1)
+        return (x >> 16).astype(np.uint16), (x & 0xFFFF).astype(np.uint16)
+    if elem == B.ELEM_FP16:
+        x = np.ascontiguousarray(x, np.uint16).reshape(-1).astype(np.uint32)
+        sign, expo, mant = x >> 15, (x >> 10) & 0x1F, x & 0x3FF
+        v = (sign << 15) | (expo << 7) | (mant >> 3)
+        return v.astype(np.uint16), (mant & 7).astype(np.uint8)
+    raise ValueError(f"unknown element type {elem}")
+
+
+def merge_elements(v: np.ndarray, lo, elem: int) -> np.ndarray:
+    """Inverse of split_elements."""
+    v = np.asarray(v, np.uint16)
+    if elem == B.ELEM_BF16:
+        return v.copy()
+    if elem == B.ELEM_FP32:
+        return (v.astype(np.uint32) << 16) | np.asarray(lo, np.uint32)
+    if elem == B.ELEM_FP16:
+        v = v.astype(np.uint32)
+        sign, expo, mant7 = v >> 15, (v >> 7) & 0xFF, v & 0x7F
+        if expo.size and int(expo.max()) > 0x1F:
+            raise ValueError("FP16 exponent field above 31")
+        return ((sign << 15) | (expo << 10) | (mant7 << 3) | np.asarray(lo, np.uint32)).astype(np.uint16)
+    raise ValueError(f"unknown element type {elem}")
+
+
+def pack3(lo: np.ndarray) -> np.ndarray:
+    """3-bit values, value i at stream bits 3i..3i+2 (bit b of the stream is
+    bit b mod 8 of byte b / 8)."""
+    lo = np.asarray(lo, np.uint8).reshape(-1)
+    bits = ((lo[:, None] >> np.arange(3, dtype=np.uint8)) & 1).reshape(-1)
+    return np.packbits(bits, bitorder="little")
+
+
+def unpack3(packed: np.ndarray, n: int) -> np.ndarray:
+    bits = np.unpackbits(np.asarray(packed, np.uint8), bitorder="little")[:3 * n].reshape(n, 3)
+    return (bits * np.array([1, 2, 4], np.uint8)).sum(axis=1).astype(np.uint8)
+
+
+def lo_section(lo, elem: int, n: int) -> np.ndarray:
+    """The raw low-mantissa section: FP32 uint16[n], FP16 packed 3-bit values;
+    padded with zeros to a multiple of 16 bytes, with at least 16 bytes after
+    the FP16 values."""
+    if elem == B.ELEM_FP32:
+        out = np.zeros(B.align(2 * n, 16), np.uint8)
+        out[:2 * n] = np.asarray(lo, np.uint16).view(np.uint8)
+        return out
+    packed = pack3(lo)
+    out = np.zeros(B.align(-(-3 * n // 8) + 16, 16), np.uint8)
+    out[:packed.size] = packed
+    return out
+
+
+def encode_elements(x: np.ndarray, elem: int, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
+                    threads_per_block: int = DEFAULT_THREADS_PER_BLOCK,
+                    max_len: int = DEFAULT_MAX_LEN) -> np.ndarray:
+    """DFloat11 blob of FP32 (uint32 patterns), FP16 or BF16 (uint16) elements."""
+    v, lo = split_elements(x, elem)
+    if elem == B.ELEM_BF16:
+        return encode(v, chunk_bytes, threads_per_block, max_len)
+    return encode(v, chunk_bytes, threads_per_block, max_len, _elem=elem,
+                  _lo=lo_section(lo, elem, v.size))
+
+
+def decode_elements(blob: np.ndarray) -> np.ndarray:
+    """The elements of a DFloat11 blob of any element type (uint32 for FP32,
+    uint16 otherwise)."""
+    blob = np.asarray(blob, np.uint8)
+    h = B.unpack_header(blob)
+    elem, n = h["elem"], h["n"]
+    v = decode(blob)
+    if elem == B.ELEM_BF16:
+        return v
+    raw = B.section(blob, h["off_lo"], h["lo_bytes"])
+    if elem == B.ELEM_FP32:
+        if h["lo_bytes"] < 2 * n:
+            raise ValueError("low-mantissa section too short")
+        lo = raw[:2 * n].view(np.uint16)
+    elif elem == B.ELEM_FP16:
+        if h["lo_bytes"] < -(-3 * n // 8):
+            raise ValueError("low-mantissa section too short")
+        lo = unpack3(raw, n)
+    else:
+        raise ValueError(f"unknown element type {elem}")
+    return merge_elements(v, lo, elem)
 
 
 def check_index(blob: np.ndarray) -> list[str]:

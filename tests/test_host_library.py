@@ -259,3 +259,49 @@ def test_fp16_weights_through_both_codecs():
     assert np.array_equal(odf.decode(b2), w)
     assert odf.check_index(b2) == []
     assert d2.bits_per_weight > 11.0   # far less skewed 'exponent' byte than BF16's
+
+
+def elements_inputs():
+    rng = np.random.default_rng(21)
+    x32 = (rng.standard_normal(200_003).astype(np.float32) * 0.02).view(np.uint32)
+    yield "fp32_normal", B.ELEM_FP32, x32
+    special = np.array([0x00000000, 0x80000000, 0x7F800000, 0xFF800000, 0x7FC00001, 0xFFFFFFFF,
+                        0x00000001, 0x807FFFFF, 0x3F800000], np.uint32)
+    yield "fp32_special", B.ELEM_FP32, np.concatenate([special, rng.integers(0, 2 ** 32, 70_001,
+                                                                             dtype=np.uint64).astype(np.uint32)])
+    yield "fp16_normal", B.ELEM_FP16, synth.as_u16(synth.normal_fp16((300_007,), seed=12, sigma=0.02,
+                                                                      outlier_frac=1e-3))
+    yield "fp16_all", B.ELEM_FP16, np.arange(65536, dtype=np.uint16)
+    for n in (1, 2, 5, 15, 16, 17, 33):
+        yield f"fp16_n{n}", B.ELEM_FP16, rng.integers(0, 65536, n, dtype=np.uint64).astype(np.uint16)
+        yield f"fp32_n{n}", B.ELEM_FP32, rng.integers(0, 2 ** 32, n, dtype=np.uint64).astype(np.uint32)
+    yield "fp16_single_exp", B.ELEM_FP16, ((np.arange(10_000) & 0x83FF) | (13 << 10)).astype(np.uint16)
+    yield "fp32_empty", B.ELEM_FP32, np.zeros(0, np.uint32)
+
+
+@pytest.mark.parametrize("name,elem,x", list(elements_inputs()), ids=lambda v: v if isinstance(v, str) else "")
+def test_library_element_blobs_decode_in_oracle(name, elem, x):
+    d, b = lwc.lwc_encode_dfloat11_elements(x, elem)
+    assert d.elem == elem and d.total_bytes == b.size and d.n == x.size
+    assert np.array_equal(odf.decode_elements(b), x)
+    assert odf.check_index(b) == []
+    assert lwc.lwc_desc_from_blob(b).as_dict() == d.as_dict()
+    # the oracle's own blob parses in the library with the same element fields
+    ob = odf.encode_elements(x, elem, threads_per_block=32)
+    od = lwc.lwc_desc_from_blob(ob)
+    assert (od.elem, od.lo_bytes) == (elem, B.unpack_header(ob)["lo_bytes"])
+
+
+def test_element_encoder_arguments():
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_encode_dfloat11_elements(np.zeros(4, np.uint16), 7)
+    assert e.value.status == 1
+    # BF16 through the element entry point is the BF16 encoder
+    w = synth.as_u16(synth.small_square(4))
+    assert np.array_equal(lwc.lwc_encode_dfloat11_elements(w, B.ELEM_BF16)[1], lwc.lwc_encode_dfloat11(w)[1])
+    # a damaged element field or short low-mantissa section is rejected
+    d, b = lwc.lwc_encode_dfloat11_elements(np.arange(1000, dtype=np.uint32) * 77777, B.ELEM_FP32)
+    for x in (corrupt(b, 136, "<u4", 3), corrupt(b, 152, "<u8", 16)):
+        with pytest.raises(lwc.LwcError) as e:
+            lwc.lwc_desc_from_blob(x)
+        assert e.value.status == 3

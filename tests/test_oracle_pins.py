@@ -362,3 +362,78 @@ def test_codebook_bits_per_weight_closed_form():
     payload_bits = h["k"] * h["n"] + 16 * h["U"]
     assert h["k"] == 12
     assert payload_bits <= 8 * h["total_bytes"] <= payload_bits + 8 * (256 * 4 + 16)
+
+
+# ---------------------------------------------------------------- FP32 / FP16 elements
+#
+# The oracle's element split must agree with the IEEE formats themselves:
+# each finite normal element's value is rebuilt, in float64, from the parts
+# the split produces (sign, exponent field, mantissa bits) and compared with
+# numpy's own reading of the same bits; the exponent field is compared with
+# frexp. A wrong bit position or field width fails here.
+
+def _rebuild(sign, expo, mant, bias, mant_bits):
+    return np.where(sign == 1, -1.0, 1.0) * (1.0 + mant / float(1 << mant_bits)) * np.exp2(expo.astype(np.float64) - bias)
+
+
+def test_fp16_split_matches_ieee_half():
+    x = np.arange(65536, dtype=np.uint16)
+    v, lo = df11.split_elements(x, B.ELEM_FP16)
+    sign = (v >> 15).astype(np.int64)
+    expo = ((v >> 7) & 0xFF).astype(np.int64)
+    mant = (((v & 0x7F).astype(np.int64)) << 3) | lo.astype(np.int64)
+    val = x.view(np.float16).astype(np.float64)
+    normal = (expo >= 1) & (expo <= 30)
+    assert expo.max() <= 31
+    assert np.array_equal(_rebuild(sign, expo, mant, 15, 10)[normal], val[normal])
+    _, e2 = np.frexp(val[normal])
+    assert np.array_equal(expo[normal], e2 - 1 + 15)
+    assert np.array_equal(df11.merge_elements(v, lo, B.ELEM_FP16), x)
+
+
+def test_fp32_split_matches_ieee_single():
+    rng = np.random.default_rng(5)
+    x = rng.integers(0, 2 ** 32, 200_000, dtype=np.uint64).astype(np.uint32)
+    v, lo = df11.split_elements(x, B.ELEM_FP32)
+    sign = (v >> 15).astype(np.int64)
+    expo = ((v >> 7) & 0xFF).astype(np.int64)
+    mant = (((v & 0x7F).astype(np.int64)) << 16) | lo.astype(np.int64)
+    val = x.view(np.float32).astype(np.float64)
+    normal = (expo >= 1) & (expo <= 254)
+    assert np.array_equal(_rebuild(sign, expo, mant, 127, 23)[normal], val[normal])
+    _, e2 = np.frexp(val[normal])
+    assert np.array_equal(expo[normal], e2 - 1 + 127)
+    assert np.array_equal(df11.merge_elements(v, lo, B.ELEM_FP32), x)
+
+
+def test_pack3_is_little_endian_bit_concatenation():
+    rng = np.random.default_rng(6)
+    for n in (1, 2, 3, 7, 8, 9, 100):
+        vals = rng.integers(0, 8, n)
+        as_int = sum(int(v) << (3 * i) for i, v in enumerate(vals))
+        expect = np.frombuffer(as_int.to_bytes(-(-3 * n // 8), "little"), np.uint8)
+        got = df11.pack3(vals)
+        assert np.array_equal(got, expect), n
+        assert np.array_equal(df11.unpack3(got, n), vals.astype(np.uint8))
+
+
+def test_element_blobs_round_trip_and_entropy():
+    x16 = synth.as_u16(synth.normal_fp16((200_000,), seed=3, sigma=0.02))
+    b = df11.encode_elements(x16, B.ELEM_FP16, threads_per_block=32)
+    assert np.array_equal(df11.decode_elements(b), x16)
+    h = B.unpack_header(b)
+    assert h["elem"] == B.ELEM_FP16 and h["lo_bytes"] >= -(-3 * x16.size // 8)
+    # only the 32 FP16 exponent values can have codes; Huffman within 1 bit of the entropy
+    v, _ = df11.split_elements(x16, B.ELEM_FP16)
+    e, _ = df11.split(v)
+    counts = df11.histogram(e)
+    assert counts[32:].sum() == 0
+    lengths = [int(x) for x in B.section(b, h["off_lengths"], 256)]
+    p = counts[counts > 0] / counts.sum()
+    entropy = float(-(p * np.log2(p)).sum())
+    avg = float(sum(int(counts[i]) * lengths[i] for i in range(256)) / counts.sum())
+    assert entropy <= avg < entropy + 1
+    x32 = (np.random.default_rng(8).standard_normal(100_001).astype(np.float32) * 0.02).view(np.uint32)
+    b = df11.encode_elements(x32, B.ELEM_FP32, threads_per_block=32)
+    assert np.array_equal(df11.decode_elements(b), x32)
+    assert 8.0 * b.size / x32.size < 28.0    # exponent coded, 24 raw bits kept
