@@ -52,6 +52,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-encode", action="store_true", help="skip the device-encoder timing")
+    ap.add_argument("--no-elements", action="store_true", help="skip the FP32/FP16 DFloat11 decodes")
     ap.add_argument("--no-codebook", action="store_true")
     ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
     ap.add_argument("--workload", choices=("layer", "model8b", "model70b"), default="layer",
@@ -365,6 +366,39 @@ def run_lwc(args, rank, world, local_rank, dist):
             "bits_per_weight": round(sd.bits_per_weight, 4),
             "hbm_frac": round((sb.size + 2 * ns) / (sms * 1e-3) / 1e9 / peak, 4)}
         del sbd, sout
+
+    # DFloat11 for the other float formats: a gate-shaped FP32 and FP16 matrix
+    if not args.no_elements:
+        rows, cols = 14336, 4096
+        ne = rows * cols
+        res_el = {}
+        for label, elem in (("fp32", lwc.LWC_ELEM_FP32), ("fp16", lwc.LWC_ELEM_FP16)):
+            if elem == lwc.LWC_ELEM_FP32:
+                xe = synth.normal_bf16((rows, cols), seed=7000, sigma=0.02).float()
+                xe = xe + torch.randn(xe.shape, generator=torch.Generator().manual_seed(7001)) * 1e-5
+                xh = xe.numpy().view(np.uint32).reshape(-1)
+                out_e = torch.empty(ne, dtype=torch.int32, device=device)
+            else:
+                xh = synth.as_u16(synth.normal_fp16((rows, cols), seed=7002, sigma=0.02, outlier_frac=1e-3))
+                out_e = torch.empty(ne, dtype=torch.int16, device=device)
+            de, be = lwc.lwc_encode_dfloat11_elements(xh, elem)
+            bd = torch.from_numpy(be).to(device)
+            lwc.lwc_decode_dfloat11(de, bd, out_e, stream)
+            torch.cuda.synchronize(device)
+            if not np.array_equal(out_e.cpu().numpy().view(xh.dtype), xh):
+                raise SystemExit(f"{label} decode differs from its input")
+            for _ in range(args.warmup):
+                lwc.lwc_decode_dfloat11(de, bd, out_e, stream)
+            ems_e = time_steps(lambda: lwc.lwc_decode_dfloat11(de, bd, out_e, stream), args.steps, stream) / args.steps
+            esz = xh.dtype.itemsize
+            res_el[label] = {
+                "workload": f"{label} {rows}x{cols} matrix (Llama-3-8B gate shape), DFloat11 elements",
+                "value": round(esz * ne / (ems_e * 1e-3) / 1e9, 2), "unit": "GB/s decoded",
+                "ms_per_step": round(ems_e, 5), "bits_per_weight": round(8 * be.size / ne, 4),
+                "size_vs_uncompressed": round(be.size / (esz * ne), 4),
+                "hbm_frac": round((be.size + esz * ne) / (ems_e * 1e-3) / 1e9 / peak, 4)}
+            del bd, out_e, xh
+        result["elements"] = res_el
 
     # device encoders (load-time path): the same layer, already on the GPU,
     # compressed there; blobs must equal the host encoder's byte for byte

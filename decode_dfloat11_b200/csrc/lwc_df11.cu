@@ -55,6 +55,7 @@ struct Df11Tensor {
     const uint8_t *gaps;
     const uint64_t *blkoff;
     const uint8_t *sm;
+    const uint8_t *lo;     // raw low-mantissa section (FP32, FP16 elements)
     const uint16_t *lut;
     uint16_t *out;
     uint64_t n;
@@ -182,6 +183,77 @@ __device__ __forceinline__ void merge16(const uint4 &s, const uint4 &e, uint16_t
     reinterpret_cast<uint4 *>(dst)[1] = r1;
 }
 
+// ---- other element types -----------------------------------------------------------
+//
+// FP32 and FP16 blobs code a BF16-shaped 16-bit pattern per element (sign,
+// exponent field, top 7 mantissa bits), decoded exactly like BF16, plus raw
+// low mantissa bits in the "lo" section. The merge turns the BF16-shaped
+// pattern v into the element:
+//   FP32: (v << 16) | lo16[i]
+//   FP16: (v & 0x8000) | ((v & 0x0FFF) << 3) | lo3[i]   (exponent field < 32)
+
+// Two FP16 elements from a word of two BF16-shaped patterns and their 3-bit tails.
+__device__ __forceinline__ uint32_t fp16_pair(uint32_t v2, uint32_t lo_pair) {
+    return (v2 & 0x80008000u) | ((v2 & 0x0FFF0FFFu) << 3) | lo_pair;
+}
+
+// 16 elements starting at element offset r of `out` (typed by E). FP32: their
+// low halves are at lo + 2 r. FP16: `lo` is the section start (4-byte
+// aligned) and the group's 48 tail bits start at byte 6 (g0 + r / 16).
+template <int E, typename I>
+__device__ __forceinline__ void merge_group(const uint4 &s, const uint4 &e, void *out, const uint8_t *lo, I r,
+                                            uint64_t g0 = 0) {
+    if constexpr (E == LWC_ELEM_BF16) {
+        merge16(s, e, static_cast<uint16_t *>(out) + r);
+    } else {
+        uint4 r0, r1;
+        merge4(s.x, e.x, r0.x, r0.y);
+        merge4(s.y, e.y, r0.z, r0.w);
+        merge4(s.z, e.z, r1.x, r1.y);
+        merge4(s.w, e.w, r1.z, r1.w);
+        if constexpr (E == LWC_ELEM_FP32) {
+            const uint4 *lp = reinterpret_cast<const uint4 *>(lo + 2 * r);
+            const uint4 l0 = __ldg(lp), l1 = __ldg(lp + 1);
+            uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(out) + r);
+            o[0] = make_uint4(__byte_perm(l0.x, r0.x, 0x5410u), __byte_perm(l0.x, r0.x, 0x7632u),
+                              __byte_perm(l0.y, r0.y, 0x5410u), __byte_perm(l0.y, r0.y, 0x7632u));
+            o[1] = make_uint4(__byte_perm(l0.z, r0.z, 0x5410u), __byte_perm(l0.z, r0.z, 0x7632u),
+                              __byte_perm(l0.w, r0.w, 0x5410u), __byte_perm(l0.w, r0.w, 0x7632u));
+            o[2] = make_uint4(__byte_perm(l1.x, r1.x, 0x5410u), __byte_perm(l1.x, r1.x, 0x7632u),
+                              __byte_perm(l1.y, r1.y, 0x5410u), __byte_perm(l1.y, r1.y, 0x7632u));
+            o[3] = make_uint4(__byte_perm(l1.z, r1.z, 0x5410u), __byte_perm(l1.z, r1.z, 0x7632u),
+                              __byte_perm(l1.w, r1.w, 0x5410u), __byte_perm(l1.w, r1.w, 0x7632u));
+        } else {
+            // the group's 48 tail bits start at an even byte; read the aligned 8 bytes around them
+            const uint64_t b0 = 6 * (g0 + r / 16);
+            const uint32_t *wp = reinterpret_cast<const uint32_t *>(lo + (b0 & ~3ull));
+            const uint64_t L = ((static_cast<uint64_t>(__ldg(wp + 1)) << 32) | __ldg(wp)) >> (8u * (uint32_t)(b0 & 3));
+            uint32_t t[8];
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                t[j] = (uint32_t)((L >> (6 * j)) & 7u) | ((uint32_t)((L >> (6 * j + 3)) & 7u) << 16);
+            uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + r);
+            o[0] = make_uint4(fp16_pair(r0.x, t[0]), fp16_pair(r0.y, t[1]), fp16_pair(r0.z, t[2]), fp16_pair(r0.w, t[3]));
+            o[1] = make_uint4(fp16_pair(r1.x, t[4]), fp16_pair(r1.y, t[5]), fp16_pair(r1.z, t[6]), fp16_pair(r1.w, t[7]));
+        }
+    }
+}
+
+// One element i from its sign|mantissa byte s and exponent e.
+template <int E>
+__device__ __forceinline__ void merge_one(uint32_t s, uint32_t e, void *out, const uint8_t *lo, uint64_t i) {
+    const uint32_t v = merge1(s, e);
+    if constexpr (E == LWC_ELEM_BF16) {
+        static_cast<uint16_t *>(out)[i] = (uint16_t)v;
+    } else if constexpr (E == LWC_ELEM_FP32) {
+        static_cast<uint32_t *>(out)[i] = (v << 16) | reinterpret_cast<const uint16_t *>(lo)[i];
+    } else {
+        const uint64_t b = 3 * i;   // lo has slack bytes after the last tail
+        const uint32_t t = ((uint32_t)lo[b >> 3] | ((uint32_t)lo[(b >> 3) + 1] << 8)) >> (b & 7);
+        static_cast<uint16_t *>(out)[i] = (uint16_t)((v & 0x8000u) | ((v & 0x0FFFu) << 3) | (t & 7u));
+    }
+}
+
 // ---- block scan ------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t &total) {
@@ -235,7 +307,7 @@ __device__ __forceinline__ void issue_item(const Df11Batch &B, uint32_t ti, uint
 
 // ---- the kernel -------------------------------------------------------------------
 
-template <int kMaxThreads>
+template <int kMaxThreads, int E>
 __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 0 ? kCtasPerSm * 256 / kMaxThreads : 1)
     df11_decode_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
@@ -435,16 +507,17 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
 #pragma unroll
                 for (int m = 0; m < kMergeRegs; m++) {
                     const uint64_t g = g_lo + 16ull * (tid + (uint32_t)m * T);
-                    if (g < g_hi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    if (g < g_hi)
+                        merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out, tn.lo, g);
                 }
                 for (uint64_t g = g_lo + 16ull * (tid + (uint32_t)kMergeRegs * T); g < g_hi; g += 16ull * T)
-                    merge16(__ldg(reinterpret_cast<const uint4 *>(tn.sm + g)),
-                            *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out + g);
+                    merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(tn.sm + g)),
+                                   *reinterpret_cast<const uint4 *>(stage + (g - base)), tn.out, tn.lo, g);
                 if (tid < 32) {   // partial 16-groups at both ends
                     const uint64_t i = tid < 16 ? o0 + tid : max(g_hi, g_lo) + (tid - 16);
                     const bool head = tid < 16 && i < min(g_lo, o1);
                     const bool tail = tid >= 16 && i < o1;
-                    if (head || tail) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
+                    if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
                 }
             } else {
                 bad |= LWC_DEVICE_BAD_COUNT;   // `total` is the same in every thread
@@ -500,6 +573,7 @@ __device__ __forceinline__ void issue_warp_item(const Df11Batch &B, const Df11Te
     dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
 }
 
+template <int E>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
@@ -696,21 +770,25 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
                     // 32-bit offsets from the block's first 16-weight group
                     const uint64_t base = o0 & ~15ull;
                     const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
-                    uint16_t *ob = tn.out + base;
+                    // typed output and low-mantissa pointers at the block's first group
+                    void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
+                                                  : static_cast<void *>(tn.out + base);
+                    const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
+                    const uint64_t g0 = base / 16;   // first group, for the FP16 tails
                     const uint8_t *sb = tn.sm + base;
 #pragma unroll
                     for (int m = 0; m < kWarpMergeRegs; m++) {
                         const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
-                        if (r < rhi) merge16(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob + r);
+                        if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
                     }
                     for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
-                        merge16(__ldg(reinterpret_cast<const uint4 *>(sb + r)), *reinterpret_cast<const uint4 *>(stage + r),
-                                ob + r);
+                        merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
+                                       *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
                     // partial 16-groups at both ends
                     const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
                     const bool head = lane < 16 && i < min(g_lo, o1);
                     const bool tail = lane >= 16 && i < o1;
-                    if (head || tail) tn.out[i] = merge1(tn.sm[i], stage[i - base]);
+                    if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
                 } else {
                     bad |= LWC_DEVICE_BAD_COUNT;
                 }
@@ -730,16 +808,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
 }
 
 // One exponent value for the whole tensor: out = merge(const_exp, sm).
-__global__ void df11_const_kernel(const uint8_t *__restrict__ sm, uint16_t *__restrict__ out, uint64_t n,
+template <int E>
+__global__ void df11_const_kernel(const uint8_t *__restrict__ sm, const uint8_t *__restrict__ lo, void *out, uint64_t n,
                                   uint32_t const_exp) {
     const uint32_t e4 = const_exp * 0x01010101u;
     const uint4 ev = make_uint4(e4, e4, e4, e4);
     const uint64_t stride = 16ull * gridDim.x * blockDim.x;
     for (uint64_t g = 16ull * (blockIdx.x * (uint64_t)blockDim.x + threadIdx.x); g < n; g += stride) {
         if (g + 16 <= n) {
-            merge16(__ldg(reinterpret_cast<const uint4 *>(sm + g)), ev, out + g);
+            merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sm + g)), ev, out, lo, g);
         } else {
-            for (uint64_t i = g; i < n; i++) out[i] = merge1(sm[i], const_exp);
+            for (uint64_t i = g; i < n; i++) merge_one<E>(sm[i], const_exp, out, lo, i);
         }
     }
 }
@@ -765,8 +844,13 @@ lwc_status device_config(DeviceConfig &out) {
     if (!c.ready) {
         err = cudaDeviceGetAttribute(&c.sms, cudaDevAttrMultiProcessorCount, dev);
         if (err == cudaSuccess) err = cudaDeviceGetAttribute(&c.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        const void *kernels[] = {(const void *)df11_decode_kernel<256>, (const void *)df11_decode_kernel<1024>,
-                                 (const void *)df11_warp_kernel};
+        const void *kernels[] = {
+            (const void *)df11_decode_kernel<256, LWC_ELEM_BF16>, (const void *)df11_decode_kernel<1024, LWC_ELEM_BF16>,
+            (const void *)df11_warp_kernel<LWC_ELEM_BF16>,
+            (const void *)df11_decode_kernel<256, LWC_ELEM_FP32>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP32>,
+            (const void *)df11_warp_kernel<LWC_ELEM_FP32>,
+            (const void *)df11_decode_kernel<256, LWC_ELEM_FP16>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP16>,
+            (const void *)df11_warp_kernel<LWC_ELEM_FP16>};
         for (const void *k : kernels) {
             if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
             if (err == cudaSuccess)
@@ -781,7 +865,32 @@ lwc_status device_config(DeviceConfig &out) {
 
 uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
-// Launch one kernel over up to kMaxBatch tensors sharing (chunk_bytes, threads_per_block).
+// The decode kernel for an element type and block shape, and its launch.
+template <int E>
+const void *df11_kernel(bool per_warp, uint32_t T) {
+    return per_warp   ? (const void *)df11_warp_kernel<E>
+           : T <= 256 ? (const void *)df11_decode_kernel<256, E>
+                      : (const void *)df11_decode_kernel<1024, E>;
+}
+
+const void *df11_kernel_for(uint32_t elem, bool per_warp, uint32_t T) {
+    if (elem == LWC_ELEM_FP32) return df11_kernel<LWC_ELEM_FP32>(per_warp, T);
+    if (elem == LWC_ELEM_FP16) return df11_kernel<LWC_ELEM_FP16>(per_warp, T);
+    return df11_kernel<LWC_ELEM_BF16>(per_warp, T);
+}
+
+template <int E>
+void launch_df11(bool per_warp, uint32_t T, unsigned grid, uint32_t threads, size_t smem, cudaStream_t stream,
+                 const Df11Batch &B) {
+    if (per_warp)
+        df11_warp_kernel<E><<<grid, threads, smem, stream>>>(B);
+    else if (T <= 256)
+        df11_decode_kernel<256, E><<<grid, T, smem, stream>>>(B);
+    else
+        df11_decode_kernel<1024, E><<<grid, T, smem, stream>>>(B);
+}
+
+// Launch one kernel over up to kMaxBatch tensors sharing (element type, chunk_bytes, threads_per_block).
 lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, const void *const *d_ins,
                         uint16_t *const *d_outs, uint32_t *d_status, cudaStream_t stream,
                         const DeviceConfig &cfg) {
@@ -800,6 +909,7 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
         t.gaps = base + d.off_gaps;
         t.blkoff = reinterpret_cast<const uint64_t *>(base + d.off_blkoff);
         t.sm = base + d.off_sm;
+        t.lo = d.elem != LWC_ELEM_BF16 ? base + d.off_lo : nullptr;
         t.lut = reinterpret_cast<const uint16_t *>(base + d.off_lut);
         t.out = d_outs[idx[j]];
         t.n = d.n;
@@ -825,9 +935,8 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
                     (unsigned long long)smem, cfg.max_smem);
-    const void *kernel = per_warp ? (const void *)df11_warp_kernel
-                         : T <= 256 ? (const void *)df11_decode_kernel<256>
-                                    : (const void *)df11_decode_kernel<1024>;
+    const uint32_t elem = d0.elem;
+    const void *kernel = df11_kernel_for(elem, per_warp, T);
     int per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)threads, (size_t)smem);
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
@@ -835,12 +944,12 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
                                 threads, (unsigned long long)smem);
     const uint64_t units = per_warp ? (work + kWarpsPerCta - 1) / kWarpsPerCta : work;
     const uint64_t grid = std::min<uint64_t>(units, (uint64_t)per_sm * cfg.sms);
-    if (per_warp)
-        df11_warp_kernel<<<(unsigned)grid, threads, (size_t)smem, stream>>>(B);
-    else if (T <= 256)
-        df11_decode_kernel<256><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);
+    if (elem == LWC_ELEM_FP32)
+        launch_df11<LWC_ELEM_FP32>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
+    else if (elem == LWC_ELEM_FP16)
+        launch_df11<LWC_ELEM_FP16>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     else
-        df11_decode_kernel<1024><<<(unsigned)grid, T, (size_t)smem, stream>>>(B);
+        launch_df11<LWC_ELEM_BF16>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
     return LWC_OK;
@@ -851,8 +960,14 @@ lwc_status launch_const(const lwc_desc &d, const void *d_in, uint16_t *d_out, cu
     if (d.n == 0) return LWC_OK;
     const uint64_t groups = (d.n + 15) / 16;
     const uint64_t blocks = std::min<uint64_t>((groups + 255) / 256, (uint64_t)cfg.sms * 8);
-    df11_const_kernel<<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const uint8_t *>(d_in) + d.off_sm, d_out,
-                                                           d.n, d.const_exp);
+    const uint8_t *sm = static_cast<const uint8_t *>(d_in) + d.off_sm;
+    const uint8_t *lo = d.elem != LWC_ELEM_BF16 ? static_cast<const uint8_t *>(d_in) + d.off_lo : nullptr;
+    if (d.elem == LWC_ELEM_FP32)
+        df11_const_kernel<LWC_ELEM_FP32><<<(unsigned)blocks, 256, 0, stream>>>(sm, lo, d_out, d.n, d.const_exp);
+    else if (d.elem == LWC_ELEM_FP16)
+        df11_const_kernel<LWC_ELEM_FP16><<<(unsigned)blocks, 256, 0, stream>>>(sm, lo, d_out, d.n, d.const_exp);
+    else
+        df11_const_kernel<LWC_ELEM_BF16><<<(unsigned)blocks, 256, 0, stream>>>(sm, lo, d_out, d.n, d.const_exp);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
     return LWC_OK;
@@ -872,8 +987,6 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
     for (int i = 0; i < count; i++) {
         lwc_status st = check_df11_desc(&descs[i]);
         if (st) return st;
-        if (descs[i].elem != LWC_ELEM_BF16)
-            return fail(LWC_ERR_UNSUPPORTED, "tensor %d: element type %u is not decoded by this build", i, descs[i].elem);
         if (descs[i].n == 0) continue;
         if (!d_ins[i] || !d_outs[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (tensor %d)", i);
         if (!aligned16(d_ins[i]) || !aligned16(d_outs[i]))
@@ -891,7 +1004,7 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
     lwc_status st = device_config(cfg);
     if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // single-exponent tensors; the rest grouped by (chunk_bytes, threads_per_block)
+    // single-exponent tensors; the rest grouped by (element type, chunk_bytes, threads_per_block)
     std::vector<std::pair<uint64_t, int>> keyed;
     for (int i = 0; i < count; i++) {
         const lwc_desc &d = descs[i];
@@ -901,7 +1014,7 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
             if (st) return st;
             continue;
         }
-        keyed.push_back({((uint64_t)d.chunk_bytes << 32) | d.threads_per_block, i});
+        keyed.push_back({((uint64_t)d.elem << 40) | ((uint64_t)d.chunk_bytes << 20) | d.threads_per_block, i});
     }
     std::stable_sort(keyed.begin(), keyed.end(),
                      [](const std::pair<uint64_t, int> &a, const std::pair<uint64_t, int> &b) { return a.first < b.first; });

@@ -11,6 +11,7 @@ import torch
 import synth
 from decode_dfloat11_b200 import build as lwc_build
 from decode_dfloat11_b200 import lwc
+from oracle import blob as B
 from oracle import codebook as ocb
 from oracle import df11 as odf
 
@@ -275,3 +276,72 @@ def test_fp16_patterns(codec):
         got = host_u16(gpu_decode(d, dev(b), "df11"))
     assert np.array_equal(ref, w)
     assert np.array_equal(got, w)
+
+
+# ------------------------------------------------------------ FP32 / FP16 elements
+
+def element_cases():
+    rng = np.random.default_rng(31)
+    x32 = (rng.standard_normal(1_000_003).astype(np.float32) * 0.02).view(np.uint32)
+    yield "fp32_normal", B.ELEM_FP32, x32
+    special = np.array([0, 0x80000000, 0x7F800000, 0xFF800000, 0x7FC00001, 0xFFFFFFFF, 1, 0x807FFFFF], np.uint32)
+    yield "fp32_random", B.ELEM_FP32, np.concatenate(
+        [special, rng.integers(0, 2 ** 32, 300_001, dtype=np.uint64).astype(np.uint32)])
+    yield "fp16_normal", B.ELEM_FP16, synth.as_u16(synth.normal_fp16((1_000_003,), seed=13, sigma=0.02,
+                                                                      outlier_frac=1e-3))
+    yield "fp16_all", B.ELEM_FP16, np.arange(65536, dtype=np.uint16)
+    yield "fp16_single_exp", B.ELEM_FP16, ((np.arange(70_001) & 0x83FF) | (13 << 10)).astype(np.uint16)
+    yield "fp32_single_exp", B.ELEM_FP32, ((np.arange(70_001, dtype=np.uint32) * 2654435761) & 0x807FFFFF) | (120 << 23)
+    for n in (1, 15, 16, 17, 33, 4097):
+        yield f"fp16_n{n}", B.ELEM_FP16, rng.integers(0, 65536, n, dtype=np.uint64).astype(np.uint16)
+        yield f"fp32_n{n}", B.ELEM_FP32, rng.integers(0, 2 ** 32, n, dtype=np.uint64).astype(np.uint32)
+
+
+def gpu_decode_elements(d, blob_dev, elem, n):
+    out = torch.zeros(n, dtype=torch.int32 if elem == B.ELEM_FP32 else torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_checked(d, blob_dev, out, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    got = out.cpu().numpy()
+    return got.view(np.uint32) if elem == B.ELEM_FP32 else got.view(np.uint16)
+
+
+@pytest.mark.parametrize("tpb", [32, 256])   # the per-warp and the per-CTA kernel
+@pytest.mark.parametrize("name,elem,x", list(element_cases()), ids=lambda v: v if isinstance(v, str) else "")
+def test_df11_elements(name, elem, x, tpb):
+    d, b = lwc.lwc_encode_dfloat11_elements(x, elem, threads_per_block=tpb)
+    ref = odf.decode_elements(b)
+    assert np.array_equal(ref, x)
+    assert np.array_equal(gpu_decode_elements(d, dev(b), elem, x.size), x)
+
+
+def test_df11_elements_mixed_batch():
+    """BF16, FP32 and FP16 tensors in one batched call (one launch per element type)."""
+    rng = np.random.default_rng(32)
+    xs = [(B.ELEM_BF16, synth.as_u16(synth.normal_bf16((500_001,), seed=40, sigma=0.02))),
+          (B.ELEM_FP32, (rng.standard_normal(300_007).astype(np.float32) * 0.03).view(np.uint32)),
+          (B.ELEM_FP16, synth.as_u16(synth.normal_fp16((400_009,), seed=41, sigma=0.01))),
+          (B.ELEM_FP32, (rng.standard_normal(12_345).astype(np.float32)).view(np.uint32))]
+    enc = [lwc.lwc_encode_dfloat11_elements(x, e) for e, x in xs]
+    blobs = [dev(b) for _, b in enc]
+    outs = [torch.zeros(x.size, dtype=torch.int32 if e == B.ELEM_FP32 else torch.int16, device="cuda")
+            for e, x in xs]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_batched([d for d, _ in enc], blobs, outs, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for (e, x), o in zip(xs, outs):
+        got = o.cpu().numpy()
+        assert np.array_equal(got.view(np.uint32) if e == B.ELEM_FP32 else got.view(np.uint16), x), e
+
+
+def test_df11_fp32_full_size():
+    """An FP32 matrix of the Llama-3-8B gate shape (58,720,256 weights, 235 MB out)."""
+    x = synth.normal_bf16((14336, 4096), seed=42, sigma=0.02).float()   # FP32 values with BF16 precision ...
+    x = x + torch.randn(x.shape, generator=torch.Generator().manual_seed(43)) * 1e-5   # ... plus low bits
+    xh = x.numpy().view(np.uint32).reshape(-1)
+    d, b = lwc.lwc_encode_dfloat11_elements(xh, B.ELEM_FP32)
+    got = gpu_decode_elements(d, dev(b), B.ELEM_FP32, xh.size)
+    assert np.array_equal(got, xh)
+    assert 8.0 * d.total_bytes / d.n < 28.0
