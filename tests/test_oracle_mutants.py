@@ -96,3 +96,37 @@ def test_lsb_msb_confusion_in_codebook_is_caught(monkeypatch):
         return b
     monkeypatch.setattr(codebook, "encode", bad)
     fails(pins.test_golden_codebook_worked_example)
+
+
+def test_fp16_exponent_off_by_one_bit_is_caught(monkeypatch):
+    good = df11.split_elements
+
+    def bad(x, elem):
+        if elem != 2:
+            return good(x, elem)
+        x = np.ascontiguousarray(x, np.uint16).astype(np.uint32)
+        sign, expo, mant = x >> 15, (x >> 11) & 0x1F, x & 0x3FF      # exponent read one bit too high
+        return ((sign << 15) | (expo << 7) | (mant >> 3)).astype(np.uint16), (mant & 7).astype(np.uint8)
+    monkeypatch.setattr(df11, "split_elements", bad)
+    fails(pins.test_fp16_split_matches_ieee_half)
+
+
+def test_fp32_halves_swapped_is_caught(monkeypatch):
+    good = df11.split_elements
+
+    def bad(x, elem):
+        if elem != 1:
+            return good(x, elem)
+        x = np.ascontiguousarray(x, np.uint32)
+        return (x & 0xFFFF).astype(np.uint16), (x >> 16).astype(np.uint16)   # high and low halves swapped
+    monkeypatch.setattr(df11, "split_elements", bad)
+    fails(pins.test_fp32_split_matches_ieee_single)
+
+
+def test_pack3_msb_first_is_caught(monkeypatch):
+    def bad(lo):
+        lo = np.asarray(lo, np.uint8).reshape(-1)
+        bits = ((lo[:, None] >> np.arange(3, dtype=np.uint8)[::-1]) & 1).reshape(-1)   # bits reversed
+        return np.packbits(bits, bitorder="little")
+    monkeypatch.setattr(df11, "pack3", bad)
+    fails(pins.test_pack3_is_little_endian_bit_concatenation)
