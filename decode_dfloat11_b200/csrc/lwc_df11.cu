@@ -150,11 +150,21 @@ __device__ void build_fast_tables(const uint16_t *lut, uint32_t ntab, uint8_t *c
     }
 }
 
-// The 32 stream bits starting at bit `pos` of the staged segment.
-__device__ __forceinline__ uint32_t window32(const uint32_t *seg, uint32_t pos) {
-    const uint32_t i = pos >> 5;
-    return __funnelshift_l(seg[i + 1], seg[i], pos);   // the shift amount is taken mod 32
-}
+// The 32 stream bits starting at bit `pos` of the staged segment (MSB first),
+// keeping the last two words read: a decode step consumes at most 32 bits, so
+// the word index advances by 0 or 1 per step and one shared-memory load per
+// step suffices.
+struct Window {
+    uint32_t wi, w0, w1;
+    __device__ __forceinline__ Window(const uint32_t *seg, uint32_t pos) : wi((pos >> 5) - 1u), w0(0), w1(seg[pos >> 5]) {}
+    __device__ __forceinline__ uint32_t at(const uint32_t *seg, uint32_t pos) {
+        const uint32_t ni = pos >> 5;
+        w0 = ni != wi ? w1 : w0;
+        w1 = seg[ni + 1];
+        wi = ni;
+        return __funnelshift_l(w1, w0, pos);
+    }
+};
 
 // ---- merge ---------------------------------------------------------------------
 
@@ -400,8 +410,9 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
             uint32_t count = 0;
             if (start < end) {
                 uint32_t pos = start, rem = end - start, acc = 0, sbits = 0, scount = 0;
+                Window win(seg, start);
                 for (;;) {
-                    const uint32_t wv = window32(seg, pos);
+                    const uint32_t wv = win.at(seg, pos);
                     const uint32_t idx = wv >> (32 - kFastBits);
                     const uint32_t e = cnt_tab[idx];
                     const uint32_t len = e & 15u;
@@ -446,8 +457,9 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
                 if (start < end) {
                     uint8_t *bp = stage + (uint32_t)(o0 & 15u) + first;
                     uint32_t pos = start, rem = end - start;
+                    Window win(seg, start);
                     for (;;) {
-                        const uint32_t wv = window32(seg, pos);
+                        const uint32_t wv = win.at(seg, pos);
                         const uint32_t idx = wv >> (32 - kFastBits);
                         const uint32_t e = sym_tab[idx];
                         const uint32_t len = e >> 26;
@@ -660,8 +672,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
                 uint32_t count = 0;
                 if (start < end) {
                     uint32_t pos = start, rem = end - start, acc = 0, sbits = 0, scount = 0;
+                    Window win(seg, start);
                     for (;;) {
-                        const uint32_t wv = window32(seg, pos);
+                        const uint32_t wv = win.at(seg, pos);
                         const uint32_t idx = wv >> (32 - kFastBits);
                         const uint32_t e = cnt_tab[idx];
                         const uint32_t len = e & 15u;
@@ -711,8 +724,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
                     if (start < end) {
                         uint8_t *bp = stage + (uint32_t)(o0 & 15u) + first;
                         uint32_t pos = start, rem = end - start;
+                        Window win(seg, start);
                         for (;;) {
-                            const uint32_t wv = window32(seg, pos);
+                            const uint32_t wv = win.at(seg, pos);
                             const uint32_t idx = wv >> (32 - kFastBits);
                             const uint32_t e = sym_tab[idx];
                             const uint32_t len = e >> 26;

@@ -254,6 +254,7 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
     __shared__ uint64_t s_lc[256];
     __shared__ uint32_t s_words[kTile + 2];  // 32 bits per weight at most, plus the lead-in word
     __shared__ uint32_t s_warp[kTileThreads / 32];
+    __shared__ uint64_t s_div[4];            // tile start bit / and % chunk bits, / and % block bits
     s_lc[threadIdx.x] = t.lc[threadIdx.x];
     __syncthreads();
     const uint64_t n16 = (a.n + 15) & ~15ull;
@@ -280,6 +281,12 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
         const uint32_t lead = (uint32_t)(t0 & 31);
         const uint32_t nwords = (lead + tile_bits + 31) / 32;
         for (uint32_t j = threadIdx.x; j < nwords; j += kTileThreads) s_words[j] = 0;
+        if (threadIdx.x == 0) {   // the tile's 64-bit divisions, once
+            s_div[0] = t0 / a.chunk_bits;
+            s_div[1] = t0 % a.chunk_bits;
+            s_div[2] = t0 / a.block_bits;
+            s_div[3] = t0 % a.block_bits;
+        }
         __syncthreads();
 
         if (cnt) {
@@ -288,9 +295,12 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
                 a.blkoff[0] = 0;
             }
             const uint32_t o0 = lead + excl;
-            uint64_t pos = t0 + excl;
-            uint64_t ci = pos / a.chunk_bits + 1, next_c = ci * a.chunk_bits;
-            uint64_t bi = pos / a.block_bits + 1, next_b = bi * a.block_bits;
+            // chunk and block starts after this thread's first code, as 32-bit
+            // distances from it (chunks are <= 8192 bits, blocks <= 2^23)
+            const uint32_t cbits = (uint32_t)a.chunk_bits, bbits = (uint32_t)a.block_bits;
+            const uint32_t xc = (uint32_t)s_div[1] + excl, xb = (uint32_t)s_div[3] + excl;
+            uint64_t ci = s_div[0] + xc / cbits + 1, bi = s_div[2] + xb / bbits + 1;
+            uint32_t next_c = cbits - xc % cbits, next_b = bbits - xb % bbits, rel = 0;
             uint64_t acc = 0;
             uint32_t nacc = o0 & 31, wi = o0 >> 5;
             bool first = true;
@@ -313,18 +323,18 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
                     wi++;
                     first = false;
                 }
-                const uint64_t end = pos + l;
+                const uint32_t end = rel + l;
                 if (end >= next_c) {
                     if (ci < a.n_chunks) a.gaps[ci] = (uint8_t)(end - next_c);
                     ci++;
-                    next_c += a.chunk_bits;
+                    next_c += cbits;
                 }
                 if (end >= next_b) {
                     if (bi < a.n_blocks) a.blkoff[bi] = i0 + j + 1;
                     bi++;
-                    next_b += a.block_bits;
+                    next_b += bbits;
                 }
-                pos = end;
+                rel = end;
             }
             if (nacc) atomicOr(&s_words[wi], (uint32_t)(acc << (32 - nacc)));
             if (i0 + cnt == a.n) a.blkoff[a.n_blocks] = a.n;
