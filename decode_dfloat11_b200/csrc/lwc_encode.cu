@@ -415,6 +415,66 @@ __global__ void __launch_bounds__(512) cb_presence_kernel(const uint16_t *__rest
         if (s_bits[i]) atomicOr(&bitmap[i], s_bits[i]);
 }
 
+// The ascending table of present patterns and the pattern -> index map, from
+// the presence bitmap: a pattern's index is the number of set bits before it.
+// 2048 threads (8 CTAs of 256), one bitmap word of 32 patterns each; a CTA
+// counts the set bits of all earlier CTAs' words itself, then scans its own.
+// Absent patterns map to 0xFFFF. A count that differs from the planned U is
+// flagged.
+constexpr uint32_t kRankCtas = 8, kRankThreads = 256;
+
+__global__ void __launch_bounds__(kRankThreads) cb_rank_kernel(const uint32_t *bitmap, uint16_t *rank,
+                                                               uint16_t *table, uint32_t U, WsHeader *ws) {
+    __shared__ uint32_t s_warp[kRankThreads / 32];
+    __shared__ uint32_t s_before;
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // set bits in the words of earlier CTAs
+    uint32_t before = 0;
+    for (uint32_t i = threadIdx.x; i < blockIdx.x * kRankThreads; i += kRankThreads) before += __popc(bitmap[i]);
+#pragma unroll
+    for (int d = 16; d; d >>= 1) before += __shfl_xor_sync(0xFFFFFFFFu, before, d);
+    if (lane == 0) s_warp[warp] = before;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t t = 0;
+        for (uint32_t k = 0; k < kRankThreads / 32; k++) t += s_warp[k];
+        s_before = t;
+    }
+    __syncthreads();
+    // exclusive scan of this CTA's word counts
+    const uint32_t wi = blockIdx.x * kRankThreads + threadIdx.x;
+    const uint32_t word = bitmap[wi], c = __popc(word);
+    uint32_t x = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, d);
+        if (lane >= (uint32_t)d) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;   // every thread has read s_warp above (second barrier)
+    __syncthreads();
+    uint32_t r = s_before + x - c, total = s_before;
+    for (uint32_t k = 0; k < kRankThreads / 32; k++) {
+        r += k < warp ? s_warp[k] : 0;
+        total += s_warp[k];
+    }
+    uint32_t pairs[16];
+#pragma unroll
+    for (int b = 0; b < 32; b += 2) {
+        const bool s0 = (word >> b) & 1u, s1 = (word >> (b + 1)) & 1u;
+        const uint32_t r0 = s0 ? r : 0xFFFFu;
+        if (s0 && r < U) table[r] = (uint16_t)(32 * wi + b);
+        r += s0;
+        const uint32_t r1 = s1 ? r : 0xFFFFu;
+        if (s1 && r < U) table[r] = (uint16_t)(32 * wi + b + 1);
+        r += s1;
+        pairs[b / 2] = r0 | (r1 << 16);
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(rank + 32 * wi);
+#pragma unroll
+    for (int q = 0; q < 4; q++) dst[q] = make_uint4(pairs[4 * q], pairs[4 * q + 1], pairs[4 * q + 2], pairs[4 * q + 3]);
+    if (blockIdx.x == kRankCtas - 1 && threadIdx.x == kRankThreads - 1 && total != U) atomicOr(&ws->error, kErrUnplanned);
+}
+
 // Packs K-bit indices, LSB first. A warp handles 1024 weights: 32 lanes x 32
 // consecutive weights, whose K-bit indices fill exactly K words per lane.
 // Patterns are staged in shared memory (16-byte slots XOR-swizzled within
@@ -639,40 +699,38 @@ lwc_status write_dfloat11(const uint16_t *src, uint64_t n, const WsHeader &h, co
 
 lwc_status write_codebook(const uint16_t *src, uint64_t n, const WsHeader &h, const uint32_t *bitmap, uint8_t *work,
                           uint8_t *blob, uint64_t blob_bytes, lwc_desc *desc_out, cudaStream_t s) {
-    std::vector<uint8_t> seen(65536, 0);
-    for (uint32_t v = 0; v < 65536; v++) seen[v] = (bitmap[v >> 5] >> (v & 31)) & 1;
-    CbPlan plan;
-    plan_codebook(seen, n, plan);
-    lwc_desc &d = plan.d;
+    uint32_t U = 0;
+    for (uint32_t i = 0; i < 2048; i++) U += (uint32_t)__builtin_popcount(bitmap[i]);
+    lwc_desc d;
+    codebook_layout(U, n, d);
     if (blob_bytes < d.total_bytes)
         return fail(LWC_ERR_INVALID_ARG, "blob buffer of %llu bytes, %llu needed", (unsigned long long)blob_bytes,
                     (unsigned long long)d.total_bytes);
-    if (d.U) LWC_CUDA(cudaMemcpyAsync(blob + d.off_table, plan.table.data(), 2ull * d.U, cudaMemcpyHostToDevice, s),
-                      "table write");
-    if (!d.k) {
-        if (lwc_status st = zero(blob, d.off_table + 2ull * d.U, d.total_bytes, s)) return st;
-        return finish_blob(blob, d, desc_out, s);
-    }
-    std::vector<uint16_t> rank = plan.rank;
-    for (uint32_t v = 0; v < 65536; v++)
-        if (!seen[v]) rank[v] = 0xFFFF;
     WsHeader hw = h;
     hw.error = 0;
     if (lwc_status st = put_header(work, hw, s)) return st;
-    LWC_CUDA(cudaMemcpyAsync(work + kWsArrays, rank.data(), 2 * 65536, cudaMemcpyHostToDevice, s),
-             "index map write");
-    const uint64_t packed_words = d.packed_bytes / 4, groups = (n + 1023) / 1024;
-    const uint64_t written = std::min<uint64_t>(packed_words, groups * 32 * d.k);
-    if (lwc_status st = zero(blob, d.off_table + 2ull * d.U, d.off_packed, s)) return st;
-    if (lwc_status st = zero(blob, d.off_packed + 4 * written, d.total_bytes, s)) return st;
-    const PackKernel kernel = kPackKernels[d.k - 1];
-    unsigned grid;
-    if (lwc_status st = grid_for((const void *)kernel, kPackWarps * 32, 0, (groups + kPackWarps - 1) / kPackWarps, grid))
-        return st;
-    kernel<<<grid, kPackWarps * 32, 0, s>>>(src, n, reinterpret_cast<const uint16_t *>(work + kWsArrays), d.U,
-                                           reinterpret_cast<uint32_t *>(blob + d.off_packed), packed_words,
-                                           reinterpret_cast<WsHeader *>(work));
+    WsHeader *ws = reinterpret_cast<WsHeader *>(work);
+    uint16_t *rank = reinterpret_cast<uint16_t *>(work + kWsArrays);
+    // table (into the blob) and index map (into the workspace) from the bitmap on the device
+    cb_rank_kernel<<<kRankCtas, kRankThreads, 0, s>>>(reinterpret_cast<const uint32_t *>(work + kWsCounts), rank,
+                                                      reinterpret_cast<uint16_t *>(blob + d.off_table), U, ws);
     LWC_CUDA(cudaGetLastError(), "encode launch");
+    if (!d.k) {
+        if (lwc_status st = zero(blob, d.off_table + 2ull * d.U, d.total_bytes, s)) return st;
+    } else {
+        const uint64_t packed_words = d.packed_bytes / 4, groups = (n + 1023) / 1024;
+        const uint64_t written = std::min<uint64_t>(packed_words, groups * 32 * d.k);
+        if (lwc_status st = zero(blob, d.off_table + 2ull * d.U, d.off_packed, s)) return st;
+        if (lwc_status st = zero(blob, d.off_packed + 4 * written, d.total_bytes, s)) return st;
+        const PackKernel kernel = kPackKernels[d.k - 1];
+        unsigned grid;
+        if (lwc_status st = grid_for((const void *)kernel, kPackWarps * 32, 0, (groups + kPackWarps - 1) / kPackWarps,
+                                     grid))
+            return st;
+        kernel<<<grid, kPackWarps * 32, 0, s>>>(src, n, rank, d.U, reinterpret_cast<uint32_t *>(blob + d.off_packed),
+                                               packed_words, ws);
+        LWC_CUDA(cudaGetLastError(), "encode launch");
+    }
     WsHeader r;
     if (lwc_status st = fetch_header(work, r, nullptr, 0, s)) return st;
     if (r.error) return fail(LWC_ERR_INVALID_ARG, "source changed between plan and write (unplanned 16-bit patterns)");
@@ -744,10 +802,10 @@ lwc_status lwc_encode_codebook_device_plan(const void *d_src, uint64_t n, void *
     std::vector<uint32_t> bitmap(2048);
     WsHeader r;
     if (lwc_status st = fetch_header(work, r, bitmap.data(), 8192, s)) return st;
-    std::vector<uint8_t> seen(65536, 0);
-    for (uint32_t v = 0; v < 65536; v++) seen[v] = (bitmap[v >> 5] >> (v & 31)) & 1;
+    uint32_t U = 0;
+    for (uint32_t i = 0; i < 2048; i++) U += (uint32_t)__builtin_popcount(bitmap[i]);
     CbPlan plan;
-    plan_codebook(seen, n, plan);
+    codebook_layout(U, n, plan.d);
     *desc_out = plan.d;
     clear_error();
     return LWC_OK;

@@ -315,6 +315,21 @@ lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uin
     return LWC_OK;
 }
 
+void codebook_layout(uint32_t U, uint64_t n, lwc_desc &d) {
+    std::memset(&d, 0, sizeof d);
+    d.magic = kMagic;
+    d.version = kVersion;
+    d.codec = LWC_CODEC_CODEBOOK;
+    d.n = n;
+    d.U = U;
+    while ((1ull << d.k) < d.U) d.k++;
+    d.packed_bytes = d.k ? round_up((n * d.k + 7) / 8 + 16, 16) : 0;
+    BlobLayout lay;
+    d.off_table = lay.place(2ull * d.U);
+    d.off_packed = lay.place(d.packed_bytes);
+    d.total_bytes = lay.total();
+}
+
 void plan_codebook(const std::vector<uint8_t> &seen, uint64_t n, CbPlan &p) {
     p.table.clear();
     p.rank.assign(65536, 0);
@@ -323,19 +338,7 @@ void plan_codebook(const std::vector<uint8_t> &seen, uint64_t n, CbPlan &p) {
             p.rank[v] = (uint16_t)p.table.size();
             p.table.push_back((uint16_t)v);
         }
-    lwc_desc &d = p.d;
-    std::memset(&d, 0, sizeof d);
-    d.magic = kMagic;
-    d.version = kVersion;
-    d.codec = LWC_CODEC_CODEBOOK;
-    d.n = n;
-    d.U = (uint32_t)p.table.size();
-    while ((1ull << d.k) < d.U) d.k++;
-    d.packed_bytes = d.k ? round_up((n * d.k + 7) / 8 + 16, 16) : 0;
-    BlobLayout lay;
-    d.off_table = lay.place(2ull * d.U);
-    d.off_packed = lay.place(d.packed_bytes);
-    d.total_bytes = lay.total();
+    codebook_layout((uint32_t)p.table.size(), n, p.d);
 }
 
 // ------------------------------------------------------- descriptor checks

@@ -78,6 +78,9 @@ struct CbPlan {
 };
 void plan_codebook(const std::vector<uint8_t> &seen, uint64_t n, CbPlan &plan);
 
+// Codebook descriptor (U, k and the section layout) for U distinct patterns.
+void codebook_layout(uint32_t U, uint64_t n, lwc_desc &d);
+
 // Writes the 256-byte blob header for `d`.
 void write_header(uint8_t *header, const lwc_desc &d);
 

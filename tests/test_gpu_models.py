@@ -117,3 +117,40 @@ def test_pipelined_decode_overlaps_and_never_clobbers():
         for g, t in zip(got, gen()):
             assert torch.equal(g.view(torch.int16), t.view(torch.int16)), name
     assert all(o.shape == (64, 3072) for o in outs)
+
+
+def test_layer_decodes_replay_from_a_cuda_graph():
+    """The decoders only enqueue kernels (no allocation, no synchronisation),
+    so a whole model's layer-by-layer decode can be captured once into a CUDA
+    graph and replayed; the first (uncaptured) call does the per-device setup."""
+    shapes = [(3072, 1024), (1024, 3072), (2048, 2048)]
+    units = [(f"layer{L}", lambda L=L: [synth.normal_bf16(s, 8000 + 10 * L + j, sigma=0.02, outlier_frac=1e-3,
+                                                          device="cuda") for j, s in enumerate(shapes)])
+             for L in range(4)]
+    models = build(units, ("dfloat11", "codebook"))
+    stream = torch.cuda.Stream()
+    sinks = {c: [torch.empty(sum(int(np.prod(s)) for s in shapes), dtype=torch.bfloat16, device="cuda")
+                 for _ in units] for c in models}
+    with torch.cuda.stream(stream):
+        for c, m in models.items():          # setup outside the capture
+            m.decode(0, 0, stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c, m in models.items():
+            for i in range(len(units)):
+                m.decode(i, i % 2, stream)
+                off = 0
+                for v in m.views(i, i % 2):   # copy each decoded layer out of the ping-pong buffer
+                    sinks[c][i][off:off + v.numel()].copy_(v.reshape(-1))
+                    off += v.numel()
+    for _ in range(2):
+        for c in sinks:
+            for t in sinks[c]:
+                t.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        for c in models:
+            for (name, gen), got in zip(units, sinks[c]):
+                want = torch.cat([t.reshape(-1) for t in gen()])
+                assert torch.equal(got.view(torch.int16), want.view(torch.int16)), (c, name)
