@@ -553,12 +553,12 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
 // Blobs encoded with threads_per_block = 32 have one block per 32 chunks, so a
 // single warp can decode a block on its own: its output offset is stored, the
 // scan is a warp scan, and nothing waits for the other warps of the CTA. The
-// CTA's 12 warps share the lookup tables (rebuilt, with CTA barriers, only
+// CTA's 18 warps share the lookup tables (rebuilt, with CTA barriers, only
 // where the CTA's run of blocks crosses into the next tensor); each warp has
 // its own segment buffer, gap bytes, staging area and mbarrier, and walks the
-// blocks w, w + 12, w + 24, ... of the current tensor.
-constexpr uint32_t kWarpsPerCta = 12;   // 3 CTAs (36 warps) per SM fit registers and shared memory
-constexpr int kWarpCtasPerSm = 3;
+// blocks w, w + 18, w + 36, ... of the current tensor.
+constexpr uint32_t kWarpsPerCta = 18;   // 2 CTAs (36 warps) per SM fit registers and shared memory
+constexpr int kWarpCtasPerSm = 2;
 constexpr int kWarpMergeRegs = 3;       // 16-weight merge groups per lane whose loads are issued early
 
 struct WarpLayout {
