@@ -60,7 +60,7 @@ struct WsHeader {
     uint32_t error;            // kErr* bits
     uint64_t total_bits;       // written by the scan
     uint32_t max_block_count;  // written by the last pass
-    uint32_t reserved;
+    uint32_t elem;             // LWC_ELEM_* of the source
 };
 static_assert(sizeof(WsHeader) <= kWsCounts, "workspace header too large");
 
@@ -80,23 +80,65 @@ struct CodeTable {
 
 // ------------------------------------------------------------ device helpers
 
-// Loads weights i0 .. i0+15 as 8 words (two BF16 per word, low half first);
-// weights at or past n read as 0. Returns how many are below n.
-__device__ __forceinline__ uint32_t load16(const uint16_t *__restrict__ src, uint64_t n, uint64_t i0, uint32_t w[8]) {
-    if (i0 + kPerThread <= n) {
-        const uint4 a = __ldg(reinterpret_cast<const uint4 *>(src + i0));
-        const uint4 b = __ldg(reinterpret_cast<const uint4 *>(src + i0) + 1);
-        w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
-        return kPerThread;
+// Element i of the source as a BF16-shaped pattern (sign, exponent field, top
+// 7 mantissa bits; see the element types in lwc.h), from its raw bits.
+template <int E>
+__device__ __forceinline__ uint32_t shaped(uint32_t x) {
+    if constexpr (E == LWC_ELEM_FP32) return x >> 16;
+    else if constexpr (E == LWC_ELEM_FP16) return (x & 0x8000u) | ((x >> 3) & 0x0FFFu);
+    else return x;
+}
+
+// Two 16-bit elements packed in a word (low half first), each made BF16-shaped.
+template <int E>
+__device__ __forceinline__ uint32_t shaped_pair(uint32_t w) {
+    if constexpr (E == LWC_ELEM_FP16) return (w & 0x80008000u) | ((w >> 3) & 0x0FFF0FFFu);
+    else return w;
+}
+
+// Loads elements i0 .. i0+15 as 8 words of BF16-shaped patterns (two per
+// word, low half first); elements at or past n read as 0. Returns how many
+// are below n. The source holds uint32 elements for FP32, uint16 otherwise.
+template <int E>
+__device__ __forceinline__ uint32_t load16(const void *__restrict__ src, uint64_t n, uint64_t i0, uint32_t w[8]) {
+    if constexpr (E == LWC_ELEM_FP32) {
+        const uint32_t *x = static_cast<const uint32_t *>(src);
+        if (i0 + kPerThread <= n) {
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + i0) + q);
+                w[2 * q] = __byte_perm(a.x, a.y, 0x7632u);       // high halves of two elements
+                w[2 * q + 1] = __byte_perm(a.z, a.w, 0x7632u);
+            }
+            return kPerThread;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) w[j] = 0;
+        if (i0 >= n) return 0;
+        const uint32_t cnt = (uint32_t)(n - i0);
+#pragma unroll
+        for (uint32_t k = 0; k < kPerThread; k++)
+            if (k < cnt) w[k >> 1] |= (x[i0 + k] >> 16) << (16 * (k & 1));
+        return cnt;
+    } else {
+        const uint16_t *x = static_cast<const uint16_t *>(src);
+        if (i0 + kPerThread <= n) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + i0));
+            const uint4 b = __ldg(reinterpret_cast<const uint4 *>(x + i0) + 1);
+            w[0] = a.x, w[1] = a.y, w[2] = a.z, w[3] = a.w, w[4] = b.x, w[5] = b.y, w[6] = b.z, w[7] = b.w;
+#pragma unroll
+            for (int j = 0; j < 8; j++) w[j] = shaped_pair<E>(w[j]);
+            return kPerThread;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j++) w[j] = 0;
+        if (i0 >= n) return 0;
+        const uint32_t cnt = (uint32_t)(n - i0);
+#pragma unroll
+        for (uint32_t k = 0; k < kPerThread; k++)
+            if (k < cnt) w[k >> 1] |= shaped<E>(x[i0 + k]) << (16 * (k & 1));
+        return cnt;
     }
-#pragma unroll
-    for (int j = 0; j < 8; j++) w[j] = 0;
-    if (i0 >= n) return 0;
-    const uint32_t cnt = (uint32_t)(n - i0);
-#pragma unroll
-    for (uint32_t k = 0; k < kPerThread; k++)
-        if (k < cnt) w[k >> 1] |= (uint32_t)src[i0 + k] << (16 * (k & 1));
-    return cnt;
 }
 
 __device__ __forceinline__ uint32_t exponent_of(const uint32_t w[8], uint32_t j) {
@@ -131,25 +173,21 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *s
 // copies are interleaved so that the 32 lanes of a warp always hit 32
 // different banks, whatever exponents they see (weights cluster on a few
 // exponent values, which would serialise a single shared histogram).
-__global__ void __launch_bounds__(512) df11_histogram_kernel(const uint16_t *__restrict__ src, uint64_t n,
+template <int E>
+__global__ void __launch_bounds__(512) df11_histogram_kernel(const void *__restrict__ src, uint64_t n,
                                                              unsigned long long *counts) {
     __shared__ uint32_t h[256 * 32];
     for (uint32_t i = threadIdx.x; i < 256 * 32; i += blockDim.x) h[i] = 0;
     __syncthreads();
     const uint32_t lane = threadIdx.x & 31;
-    const uint64_t nv = n / 8, stride = (uint64_t)gridDim.x * blockDim.x;
-    const uint4 *v = reinterpret_cast<const uint4 *>(src);
-    for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nv; i += stride) {
-        const uint4 q = __ldg(v + i);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const uint64_t groups = (n + kPerThread - 1) / kPerThread, stride = (uint64_t)gridDim.x * blockDim.x;
+    for (uint64_t g = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; g < groups; g += stride) {
+        uint32_t w[8];
+        const uint32_t cnt = load16<E>(src, n, g * kPerThread, w);
 #pragma unroll
-        for (int j = 0; j < 4; j++) {
-            atomicAdd(&h[((w[j] >> 7) & 0xFF) * 32 + lane], 1u);
-            atomicAdd(&h[((w[j] >> 23) & 0xFF) * 32 + lane], 1u);
-        }
+        for (uint32_t j = 0; j < kPerThread; j++)
+            if (j < cnt) atomicAdd(&h[exponent_of(w, j) * 32 + lane], 1u);
     }
-    if (blockIdx.x == 0)
-        for (uint64_t i = nv * 8 + threadIdx.x; i < n; i += blockDim.x) atomicAdd(&h[((src[i] >> 7) & 0xFF) * 32 + lane], 1u);
     __syncthreads();
     for (uint32_t e = threadIdx.x; e < 256; e += blockDim.x) {
         uint32_t sum = 0;
@@ -159,7 +197,8 @@ __global__ void __launch_bounds__(512) df11_histogram_kernel(const uint16_t *__r
 }
 
 // Bit length of every tile (sum of its code lengths).
-__global__ void __launch_bounds__(kTileThreads) df11_tile_bits_kernel(const uint16_t *__restrict__ src, uint64_t n,
+template <int E>
+__global__ void __launch_bounds__(kTileThreads) df11_tile_bits_kernel(const void *__restrict__ src, uint64_t n,
                                                                       uint64_t n_tiles, CodeTable t,
                                                                       uint32_t *tile_bits, WsHeader *ws) {
     __shared__ uint32_t s_len[256];
@@ -169,7 +208,7 @@ __global__ void __launch_bounds__(kTileThreads) df11_tile_bits_kernel(const uint
     bool bad = false;
     for (uint64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
         uint32_t w[8];
-        const uint32_t cnt = load16(src, n, tile * kTile + threadIdx.x * kPerThread, w);
+        const uint32_t cnt = load16<E>(src, n, tile * kTile + threadIdx.x * kPerThread, w);
         uint32_t bits = 0;
 #pragma unroll
         for (uint32_t j = 0; j < kPerThread; j++) {
@@ -221,7 +260,7 @@ __global__ void __launch_bounds__(1024) df11_scan_kernel(const uint32_t *tile_bi
 }
 
 struct EmitArgs {
-    const uint16_t *src;
+    const void *src;
     uint64_t n;
     const uint64_t *tile_pos;
     uint64_t n_tiles;
@@ -250,6 +289,7 @@ __device__ __forceinline__ uint32_t sm_byte(uint32_t w, int hi) {
 // the next code); one that crosses a block start gives that block's first
 // weight index. Codes are at most 32 bits and chunks at least 64, so a code
 // crosses at most one chunk start.
+template <int E>
 __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, CodeTable t) {
     __shared__ uint64_t s_lc[256];
     __shared__ uint32_t s_words[kTile + 2];  // 32 bits per weight at most, plus the lead-in word
@@ -262,7 +302,7 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
     for (uint64_t tile = blockIdx.x; tile < a.n_tiles; tile += gridDim.x) {
         const uint64_t i0 = tile * kTile + threadIdx.x * kPerThread;
         uint32_t w[8];
-        const uint32_t cnt = load16(a.src, a.n, i0, w);
+        const uint32_t cnt = load16<E>(a.src, a.n, i0, w);
         if (i0 < n16) {
             uint32_t o[4];
 #pragma unroll
@@ -359,19 +399,59 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
 }
 
 // Sign|mantissa bytes only (tensors with a single exponent value: no stream).
-__global__ void __launch_bounds__(kTileThreads) df11_sm_kernel(const uint16_t *__restrict__ src, uint64_t n,
+template <int E>
+__global__ void __launch_bounds__(kTileThreads) df11_sm_kernel(const void *__restrict__ src, uint64_t n,
                                                                uint8_t *sm) {
     const uint64_t n16 = (n + 15) & ~15ull;
     for (uint64_t i0 = ((uint64_t)blockIdx.x * kTileThreads + threadIdx.x) * kPerThread; i0 < n16;
          i0 += (uint64_t)gridDim.x * kTileThreads * kPerThread) {
         uint32_t w[8];
-        load16(src, n, i0, w);
+        load16<E>(src, n, i0, w);
         uint32_t o[4];
 #pragma unroll
         for (int k = 0; k < 4; k++)
             o[k] = sm_byte(w[2 * k], 0) | sm_byte(w[2 * k], 1) << 8 | sm_byte(w[2 * k + 1], 0) << 16 |
                    sm_byte(w[2 * k + 1], 1) << 24;
         *reinterpret_cast<uint4 *>(sm + i0) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// The raw low-mantissa section: FP32 low halves (uint16 per element), FP16
+// low 3 mantissa bits (48 bits per 16 elements, at byte 6 (i0 / 16), least
+// significant bits first). Elements past n contribute zeros.
+template <int E>
+__global__ void __launch_bounds__(kTileThreads) df11_lo_kernel(const void *__restrict__ src, uint64_t n, uint8_t *lo) {
+    const uint64_t groups = (n + kPerThread - 1) / kPerThread;
+    for (uint64_t g = (uint64_t)blockIdx.x * kTileThreads + threadIdx.x; g < groups;
+         g += (uint64_t)gridDim.x * kTileThreads) {
+        const uint64_t i0 = g * kPerThread;
+        if constexpr (E == LWC_ELEM_FP32) {
+            const uint32_t *x = static_cast<const uint32_t *>(src);
+            uint16_t *o = reinterpret_cast<uint16_t *>(lo) + i0;
+            if (i0 + kPerThread <= n) {
+                uint32_t p[8];
+#pragma unroll
+                for (int q = 0; q < 4; q++) {
+                    const uint4 a = __ldg(reinterpret_cast<const uint4 *>(x + i0) + q);
+                    p[2 * q] = __byte_perm(a.x, a.y, 0x5410u);   // low halves of two elements
+                    p[2 * q + 1] = __byte_perm(a.z, a.w, 0x5410u);
+                }
+                reinterpret_cast<uint4 *>(o)[0] = make_uint4(p[0], p[1], p[2], p[3]);
+                reinterpret_cast<uint4 *>(o)[1] = make_uint4(p[4], p[5], p[6], p[7]);
+            } else {
+                for (uint64_t i = i0; i < n; i++) o[i - i0] = (uint16_t)x[i];
+            }
+        } else {
+            const uint16_t *x = static_cast<const uint16_t *>(src);
+            uint64_t bits = 0;
+#pragma unroll
+            for (uint32_t k = 0; k < kPerThread; k++)
+                if (i0 + k < n) bits |= (uint64_t)(x[i0 + k] & 7u) << (3 * k);
+            uint16_t *o = reinterpret_cast<uint16_t *>(lo + 6 * g);   // even byte: 16-bit stores
+            o[0] = (uint16_t)bits;
+            o[1] = (uint16_t)(bits >> 16);
+            o[2] = (uint16_t)(bits >> 32);
+        }
     }
 }
 
@@ -617,20 +697,47 @@ lwc_status finish_blob(void *d_blob, const lwc_desc &d, lwc_desc *desc_out, cuda
     return LWC_OK;
 }
 
-lwc_status write_dfloat11(const uint16_t *src, uint64_t n, const WsHeader &h, const uint64_t *counts,
+// The raw low-mantissa section of FP32 / FP16 blobs, and the zero padding after it.
+template <int E>
+lwc_status write_lo(const void *src, uint64_t n, uint8_t *blob, const lwc_desc &d, cudaStream_t s) {
+    if constexpr (E == LWC_ELEM_BF16) {
+        return LWC_OK;
+    } else {
+        const uint64_t groups = (n + kPerThread - 1) / kPerThread;
+        const uint64_t written = E == LWC_ELEM_FP32 ? 2 * n : 6 * groups;
+        if (lwc_status st = zero(blob, d.off_sm + round_up(n, 16), d.off_lo, s)) return st;   // padding before it
+        if (lwc_status st = zero(blob, d.off_lo + written, d.off_lo + d.lo_bytes, s)) return st;
+        if (!n) return LWC_OK;
+        unsigned grid;
+        if (lwc_status st = grid_for((const void *)df11_lo_kernel<E>, kTileThreads, 0,
+                                     (groups + kTileThreads - 1) / kTileThreads, grid))
+            return st;
+        df11_lo_kernel<E><<<grid, kTileThreads, 0, s>>>(src, n, blob + d.off_lo);
+        LWC_CUDA(cudaGetLastError(), "encode launch");
+        return LWC_OK;
+    }
+}
+
+template <int E>
+lwc_status write_dfloat11(const void *src, uint64_t n, const WsHeader &h, const uint64_t *counts,
                           uint8_t *work, uint8_t *blob, uint64_t blob_bytes, lwc_desc *desc_out, cudaStream_t s) {
     Df11Plan plan;
-    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan)) return st;
+    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan,
+                                      lo_section_bytes(E, n)))
+        return st;
+    plan.d.elem = E;
     lwc_desc &d = plan.d;
     if (blob_bytes < d.total_bytes)
         return fail(LWC_ERR_INVALID_ARG, "blob buffer of %llu bytes, %llu needed", (unsigned long long)blob_bytes,
                     (unsigned long long)d.total_bytes);
+    if (lwc_status st = write_lo<E>(src, n, blob, d, s)) return st;
     if (plan.single) {
         if (lwc_status st = zero(blob, kHeaderBytes, d.off_sm, s)) return st;
         if (n) {
             unsigned grid;
-            if (lwc_status st = grid_for((const void *)df11_sm_kernel, kTileThreads, 0, n_tiles_of(n), grid)) return st;
-            df11_sm_kernel<<<grid, kTileThreads, 0, s>>>(src, n, blob + d.off_sm);
+            if (lwc_status st = grid_for((const void *)df11_sm_kernel<E>, kTileThreads, 0, n_tiles_of(n), grid))
+                return st;
+            df11_sm_kernel<E><<<grid, kTileThreads, 0, s>>>(src, n, blob + d.off_sm);
             LWC_CUDA(cudaGetLastError(), "encode launch");
         }
         return finish_blob(blob, d, desc_out, s);
@@ -661,8 +768,8 @@ lwc_status write_dfloat11(const uint16_t *src, uint64_t n, const WsHeader &h, co
     uint64_t *tile_pos = reinterpret_cast<uint64_t *>(work + ws_tile_pos_off(n));
     uint32_t *stream = reinterpret_cast<uint32_t *>(blob + d.off_stream);
     unsigned grid;
-    if (lwc_status st = grid_for((const void *)df11_tile_bits_kernel, kTileThreads, 0, tiles, grid)) return st;
-    df11_tile_bits_kernel<<<grid, kTileThreads, 0, s>>>(src, n, tiles, t, tile_bits, ws);
+    if (lwc_status st = grid_for((const void *)df11_tile_bits_kernel<E>, kTileThreads, 0, tiles, grid)) return st;
+    df11_tile_bits_kernel<E><<<grid, kTileThreads, 0, s>>>(src, n, tiles, t, tile_bits, ws);
     LWC_CUDA(cudaGetLastError(), "encode launch");
     df11_scan_kernel<<<1, 1024, 0, s>>>(tile_bits, tile_pos, tiles, stream, stream_words, ws);
     LWC_CUDA(cudaGetLastError(), "encode launch");
@@ -681,8 +788,8 @@ lwc_status write_dfloat11(const uint16_t *src, uint64_t n, const WsHeader &h, co
     a.block_bits = a.chunk_bits * d.threads_per_block;
     a.sm = blob + d.off_sm;
     a.ws = ws;
-    if (lwc_status st = grid_for((const void *)df11_emit_kernel, kTileThreads, 0, tiles, grid)) return st;
-    df11_emit_kernel<<<grid, kTileThreads, 0, s>>>(a, t);
+    if (lwc_status st = grid_for((const void *)df11_emit_kernel<E>, kTileThreads, 0, tiles, grid)) return st;
+    df11_emit_kernel<E><<<grid, kTileThreads, 0, s>>>(a, t);
     LWC_CUDA(cudaGetLastError(), "encode launch");
     const unsigned mgrid = (unsigned)std::min<uint64_t>(1024, (d.n_blocks + 255) / 256);
     df11_max_block_kernel<<<mgrid, 256, 0, s>>>(a.blkoff, d.n_blocks, ws);
@@ -746,14 +853,16 @@ extern "C" {
 
 uint64_t lwc_encode_device_workspace_bytes(uint64_t n) { return workspace_bytes(n); }
 
-lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const lwc_df11_params *params,
-                                           void *d_work, uint64_t work_bytes, lwc_desc *desc_out,
-                                           lwc_stream_t stream) {
+lwc_status lwc_encode_dfloat11_elements_device_plan(const void *d_src, uint64_t n, uint32_t elem,
+                                                    const lwc_df11_params *params, void *d_work, uint64_t work_bytes,
+                                                    lwc_desc *desc_out, lwc_stream_t stream) {
     if (!desc_out) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    if (elem > LWC_ELEM_FP16) return fail(LWC_ERR_INVALID_ARG, "unknown element type %u", elem);
     if (lwc_status st = check_common(d_src, n, d_work, work_bytes)) return st;
     WsHeader h{};
     h.magic = kWsMagic;
     h.codec = LWC_CODEC_DFLOAT11;
+    h.elem = elem;
     h.n = n;
     h.chunk_bytes = params ? params->chunk_bytes : kDefaultChunkBytes;
     h.threads_per_block = params ? params->threads_per_block : kDefaultThreadsPerBlock;
@@ -763,10 +872,18 @@ lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const 
     uint8_t *work = static_cast<uint8_t *>(d_work);
     LWC_CUDA(cudaMemsetAsync(work + kWsCounts, 0, 256 * sizeof(uint64_t), s), "memset");
     if (n) {
+        const void *kernel = elem == LWC_ELEM_FP32   ? (const void *)df11_histogram_kernel<LWC_ELEM_FP32>
+                             : elem == LWC_ELEM_FP16 ? (const void *)df11_histogram_kernel<LWC_ELEM_FP16>
+                                                     : (const void *)df11_histogram_kernel<LWC_ELEM_BF16>;
         unsigned grid;
-        if (lwc_status st = grid_for((const void *)df11_histogram_kernel, 512, 0, (n / 8 + 511) / 512, grid)) return st;
-        df11_histogram_kernel<<<grid, 512, 0, s>>>(static_cast<const uint16_t *>(d_src), n,
-                                                   reinterpret_cast<unsigned long long *>(work + kWsCounts));
+        if (lwc_status st = grid_for(kernel, 512, 0, (n / kPerThread + 511) / 512, grid)) return st;
+        unsigned long long *counts = reinterpret_cast<unsigned long long *>(work + kWsCounts);
+        if (elem == LWC_ELEM_FP32)
+            df11_histogram_kernel<LWC_ELEM_FP32><<<grid, 512, 0, s>>>(d_src, n, counts);
+        else if (elem == LWC_ELEM_FP16)
+            df11_histogram_kernel<LWC_ELEM_FP16><<<grid, 512, 0, s>>>(d_src, n, counts);
+        else
+            df11_histogram_kernel<LWC_ELEM_BF16><<<grid, 512, 0, s>>>(d_src, n, counts);
         LWC_CUDA(cudaGetLastError(), "encode launch");
     }
     if (lwc_status st = put_header(work, h, s)) return st;
@@ -774,10 +891,20 @@ lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const 
     WsHeader r;
     if (lwc_status st = fetch_header(work, r, counts, sizeof counts, s)) return st;
     Df11Plan plan;
-    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan)) return st;
+    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan,
+                                      lo_section_bytes(elem, n)))
+        return st;
+    plan.d.elem = elem;
     *desc_out = plan.d;
     clear_error();
     return LWC_OK;
+}
+
+lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n, const lwc_df11_params *params,
+                                           void *d_work, uint64_t work_bytes, lwc_desc *desc_out,
+                                           lwc_stream_t stream) {
+    return lwc_encode_dfloat11_elements_device_plan(d_src, n, LWC_ELEM_BF16, params, d_work, work_bytes, desc_out,
+                                                    stream);
 }
 
 lwc_status lwc_encode_codebook_device_plan(const void *d_src, uint64_t n, void *d_work, uint64_t work_bytes,
@@ -825,9 +952,15 @@ lwc_status lwc_encode_device_write(const void *d_src, uint64_t n, void *d_work, 
     if (h.magic != kWsMagic || h.n != n)
         return fail(LWC_ERR_INVALID_ARG, "workspace holds no plan for this tensor (call a *_device_plan first)");
     lwc_status st;
-    if (h.codec == LWC_CODEC_DFLOAT11)
-        st = write_dfloat11(static_cast<const uint16_t *>(d_src), n, h, region.data(), work,
-                            static_cast<uint8_t *>(d_blob), blob_bytes, desc_out, s);
+    if (h.codec == LWC_CODEC_DFLOAT11 && h.elem == LWC_ELEM_FP32)
+        st = write_dfloat11<LWC_ELEM_FP32>(d_src, n, h, region.data(), work, static_cast<uint8_t *>(d_blob), blob_bytes,
+                                           desc_out, s);
+    else if (h.codec == LWC_CODEC_DFLOAT11 && h.elem == LWC_ELEM_FP16)
+        st = write_dfloat11<LWC_ELEM_FP16>(d_src, n, h, region.data(), work, static_cast<uint8_t *>(d_blob), blob_bytes,
+                                           desc_out, s);
+    else if (h.codec == LWC_CODEC_DFLOAT11 && h.elem == LWC_ELEM_BF16)
+        st = write_dfloat11<LWC_ELEM_BF16>(d_src, n, h, region.data(), work, static_cast<uint8_t *>(d_blob), blob_bytes,
+                                           desc_out, s);
     else if (h.codec == LWC_CODEC_CODEBOOK)
         st = write_codebook(static_cast<const uint16_t *>(d_src), n, h, reinterpret_cast<const uint32_t *>(region.data()),
                             work, static_cast<uint8_t *>(d_blob), blob_bytes, desc_out, s);

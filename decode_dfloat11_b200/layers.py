@@ -35,8 +35,10 @@ def encode_many(arrays, codec: str = "dfloat11", workers: int | None = None, **p
 
 
 def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=None, **params):
-    """Compress a BF16 tensor that is already on the GPU into a device blob
-    (``lwc_encode_*_device_plan`` + ``lwc_encode_device_write``).
+    """Compress a tensor that is already on the GPU into a device blob
+    (``lwc_encode_*_device_plan`` + ``lwc_encode_device_write``). BF16 (or any
+    16-bit patterns) for both codecs; float32 / float16 tensors with the
+    DFloat11 codec use its FP32 / FP16 element types.
 
     Returns ``(desc, blob)`` with ``blob`` a uint8 CUDA tensor of
     ``desc.total_bytes`` bytes, byte-for-byte what the host encoder would make.
@@ -46,10 +48,16 @@ def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=Non
     import torch
     if codec not in CODECS:
         raise ValueError(f"unknown codec {codec!r}")
-    src = tensor.reshape(-1)
-    if src.dtype != torch.bfloat16 and src.element_size() != 2:
-        raise ValueError("expected a 16-bit tensor")
-    src = src.contiguous()
+    src = tensor.reshape(-1).contiguous()
+    elem = lwc.LWC_ELEM_BF16
+    if src.dtype == torch.float32 or src.dtype == torch.int32:
+        elem = lwc.LWC_ELEM_FP32
+    elif src.dtype == torch.float16:
+        elem = lwc.LWC_ELEM_FP16
+    elif src.element_size() != 2:
+        raise ValueError("expected a 16-bit or 32-bit tensor")
+    if elem != lwc.LWC_ELEM_BF16 and codec != "dfloat11":
+        raise ValueError("FP32 / FP16 element types are a DFloat11 feature (the codebook takes 16-bit patterns)")
     n = src.numel()
     need = lwc.lwc_encode_device_workspace_bytes(n)
     if workspace is None or workspace.numel() < need:
@@ -57,7 +65,8 @@ def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=Non
     work_bytes = workspace.numel()
     stream = stream if stream is not None else torch.cuda.current_stream(src.device)
     if codec == "dfloat11":
-        desc = lwc.lwc_encode_dfloat11_device_plan(src, n, workspace, work_bytes, stream=stream, **params)
+        desc = lwc.lwc_encode_dfloat11_elements_device_plan(src, n, elem, workspace, work_bytes, stream=stream,
+                                                            **params)
     else:
         desc = lwc.lwc_encode_codebook_device_plan(src, n, workspace, work_bytes, stream=stream)
     blob = torch.empty(desc.total_bytes, dtype=torch.uint8, device=src.device)

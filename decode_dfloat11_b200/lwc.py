@@ -35,7 +35,8 @@ EXPORTED = (
     "lwc_encode_dfloat11", "lwc_encode_dfloat11_elements", "lwc_encode_codebook", "lwc_free", "lwc_desc_from_blob",
     "lwc_decode_dfloat11", "lwc_decode_codebook", "lwc_decode_dfloat11_checked",
     "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
-    "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan", "lwc_encode_codebook_device_plan",
+    "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan",
+    "lwc_encode_dfloat11_elements_device_plan", "lwc_encode_codebook_device_plan",
     "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_status_string", "lwc_last_error",
     "lwc_version",
 )
@@ -109,6 +110,8 @@ def load():
     L.lwc_encode_device_workspace_bytes.restype = _u64
     L.lwc_encode_dfloat11_device_plan.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
     L.lwc_encode_codebook_device_plan.argtypes = [_P, _u64, _P, _u64, D, _P]
+    L.lwc_encode_dfloat11_elements_device_plan.argtypes = [_P, _u64, ctypes.c_uint32, ctypes.POINTER(lwc_df11_params),
+                                                           _P, _u64, D, _P]
     L.lwc_encode_device_write.argtypes = [_P, _u64, _P, _u64, _P, _u64, D, _P]
     L.lwc_encode_dfloat11_device_noalloc.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
     L.lwc_status_string.argtypes = [ctypes.c_int]
@@ -120,6 +123,7 @@ def load():
                  "lwc_decode_codebook", "lwc_decode_dfloat11_checked", "lwc_decode_codebook_checked",
                  "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched", "lwc_encode_dfloat11_device_plan",
                  "lwc_encode_codebook_device_plan", "lwc_encode_device_write",
+                 "lwc_encode_dfloat11_elements_device_plan",
                  "lwc_encode_dfloat11_device_noalloc"):
         getattr(L, name).restype = ctypes.c_int
     _lib = L
@@ -264,6 +268,17 @@ def lwc_encode_dfloat11_device_plan(d_src, n: int, d_work, work_bytes: int, chun
     params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
     _check(load().lwc_encode_dfloat11_device_plan(_addr(d_src), n, ctypes.byref(params), _addr(d_work), work_bytes,
                                                   ctypes.byref(desc), _stream(stream)))
+    return desc
+
+
+def lwc_encode_dfloat11_elements_device_plan(d_src, n: int, elem: int, d_work, work_bytes: int, chunk_bytes: int = 36,
+                                             threads_per_block: int = 32, max_len: int = 32,
+                                             stream=None) -> lwc_desc:
+    """Plan a DFloat11 blob of FP32 / FP16 / BF16 elements held on the device."""
+    desc = lwc_desc()
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    _check(load().lwc_encode_dfloat11_elements_device_plan(_addr(d_src), n, elem, ctypes.byref(params), _addr(d_work),
+                                                           work_bytes, ctypes.byref(desc), _stream(stream)))
     return desc
 
 

@@ -255,6 +255,15 @@ LWC_API lwc_status lwc_encode_dfloat11_device_plan(const void *d_src, uint64_t n
                                                    void *d_work, uint64_t work_bytes, lwc_desc *desc_out,
                                                    lwc_stream_t stream);
 
+/* Plan a DFloat11 blob of n elements of type `elem` (LWC_ELEM_*; d_src holds
+ * uint32 patterns for FP32, uint16 otherwise); lwc_encode_device_write then
+ * writes the same bytes lwc_encode_dfloat11_elements makes on the host.
+ * lwc_encode_dfloat11_device_plan is this with LWC_ELEM_BF16. */
+LWC_API lwc_status lwc_encode_dfloat11_elements_device_plan(const void *d_src, uint64_t n, uint32_t elem,
+                                                            const lwc_df11_params *params, void *d_work,
+                                                            uint64_t work_bytes, lwc_desc *desc_out,
+                                                            lwc_stream_t stream);
+
 /* Plan a codebook blob. */
 LWC_API lwc_status lwc_encode_codebook_device_plan(const void *d_src, uint64_t n, void *d_work,
                                                    uint64_t work_bytes, lwc_desc *desc_out, lwc_stream_t stream);

@@ -192,3 +192,30 @@ def test_device_encoder_errors():
     d = lwc.lwc_encode_dfloat11_device_plan(src, n, work, need)
     d2 = lwc.lwc_encode_device_write(src, n, work, need, blob, blob.numel())
     assert np.array_equal(host_bytes(blob[:d2.total_bytes]), lwc.lwc_encode_dfloat11(w)[1])
+
+
+def element_sources():
+    rng = np.random.default_rng(51)
+    x32 = (rng.standard_normal(300_007).astype(np.float32) * 0.02).view(np.uint32)
+    yield "fp32_normal", 1, x32
+    yield "fp32_random", 1, rng.integers(0, 2 ** 32, 70_001, dtype=np.uint64).astype(np.uint32)
+    yield "fp16_normal", 2, synth.as_u16(synth.normal_fp16((300_007,), seed=52, sigma=0.02, outlier_frac=1e-3))
+    yield "fp16_all", 2, np.arange(65536, dtype=np.uint16)
+    yield "fp16_single_exp", 2, ((np.arange(10_001) & 0x83FF) | (13 << 10)).astype(np.uint16)
+    for n in (1, 15, 16, 17, 4097):
+        yield f"fp32_n{n}", 1, rng.integers(0, 2 ** 32, n, dtype=np.uint64).astype(np.uint32)
+        yield f"fp16_n{n}", 2, rng.integers(0, 65536, n, dtype=np.uint64).astype(np.uint16)
+
+
+@pytest.mark.parametrize("name,elem,x", list(element_sources()), ids=lambda v: v if isinstance(v, str) else "")
+def test_device_element_blob_equals_host_blob(name, elem, x):
+    hd, hb = lwc.lwc_encode_dfloat11_elements(x, elem)
+    t = torch.from_numpy(x.view(np.int32) if elem == 1 else x.view(np.int16)).to("cuda")
+    if elem == 2:
+        t = t.view(torch.float16)
+    elif elem == 1:
+        t = t.view(torch.float32)
+    dd, db = encode_on_device(t, "dfloat11")
+    assert dd.as_dict() == hd.as_dict()
+    assert np.array_equal(host_bytes(db), hb)
+    assert np.array_equal(odf.decode_elements(hb), x)
