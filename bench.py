@@ -55,7 +55,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-elements", action="store_true", help="skip the FP32/FP16 DFloat11 decodes")
     ap.add_argument("--no-codebook", action="store_true")
     ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
-    ap.add_argument("--workload", choices=("layer", "model8b", "model70b"), default="layer",
+    ap.add_argument("--workload", choices=("layer", "model8b", "model70b", "stress"), default="layer",
                     help="layer: one Llama-3-8B layer (default line); model8b / model70b: the whole "
                          "model resident compressed, decoded layer by layer into ping-pong buffers")
     ap.add_argument("--codec", choices=("dfloat11", "codebook"), default="dfloat11",
@@ -584,6 +584,63 @@ def run_model(args, rank, world, local_rank, dist):
     }
 
 
+# ---------------------------------------------------------------- stress tensors
+
+def run_stress(args, rank, world, local_rank, dist):
+    """config 4: 256M-weight stress tensors, each generated and compressed on
+    the GPU and decoded K times: codebook tables of U = 256 / 4096 / 8192 /
+    65536 entries with Zipf(1.1) frequencies (k = 8 / 12 / 13 / 16; also
+    16384 and 32768 for k = 14 and 15), and the
+    DFloat11 edge case of uniformly random patterns (all 256 exponents, 8-bit
+    codes: an expansion)."""
+    import torch
+    from decode_dfloat11_b200 import build as lwc_build
+    from decode_dfloat11_b200 import lwc
+    from decode_dfloat11_b200.layers import encode_on_device
+
+    lwc_build.build()
+    lwc.load()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    peak, peak_kind = measured_peak()
+    n = 1 << 28
+    cases = [("codebook", U) for U in (256, 4096, 8192, 16384, 32768, 65536)] + [("dfloat11", None)]
+    rows, max_ms = {}, 0.0
+    for codec, U in cases:
+        x = synth.codebook_stress(U, n, seed=40 + U + rank, device=device) if U else \
+            synth.uniform_patterns(n, seed=44 + rank, device=device)
+        d, blob = encode_on_device(x, codec)
+        out = torch.empty(n, dtype=torch.int16, device=device)
+        dec = lwc.lwc_decode_codebook if codec == "codebook" else lwc.lwc_decode_dfloat11
+        dec(d, blob, out, stream)
+        torch.cuda.synchronize(device)
+        if not torch.equal(out, x.view(torch.int16)):
+            raise SystemExit(f"stress {codec} U={U} decode differs from its input")
+        del x
+        for _ in range(args.warmup):
+            dec(d, blob, out, stream)
+        ms = time_steps(lambda: dec(d, blob, out, stream), args.steps, stream) / args.steps
+        ms = max_over_ranks(ms, dist, device)
+        max_ms = max(max_ms, ms)
+        key = f"codebook_U{U}" if U else "dfloat11_uniform_exponents"
+        rows[key] = {"k": d.k if U else None, "bits_per_weight": round(d.bits_per_weight, 4),
+                     "ms": round(ms, 5), "decoded_gbs": round(2 * n / (ms * 1e-3) / 1e9, 1),
+                     "hbm_frac": round((d.total_bytes + 2 * n) / (ms * 1e-3) / 1e9 / peak, 4)}
+        del blob, out
+    first = rows["codebook_U8192"]
+    return {
+        "metric": "decoded BF16 GB/s (codebook U=8192 stress tensor; all config-4 cases in 'cases')",
+        "value": round(world * first["decoded_gbs"], 2), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": first["ms"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "u16",
+        "data": "synthetic (Zipf(1.1) draws from U-entry tables; uniform 16-bit patterns)",
+        "config": {"workload": "stress-256M", "weights_per_gpu": n, "parallelism": f"replicas x{world}",
+                   "l2": "no flush: >= 805 MB moved per decode > 126 MB L2", "peak_source": peak_kind},
+        "cases": rows, "gpu_launches": args.steps * len(cases),
+    }
+
+
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -635,6 +692,8 @@ def main(argv=None):
     try:
         if args.workload == "layer":
             result = run_lwc(args, rank, world, local_rank, dist)
+        elif args.workload == "stress":
+            result = run_stress(args, rank, world, local_rank, dist)
         else:
             result = run_model(args, rank, world, local_rank, dist)
         if rank == 0:

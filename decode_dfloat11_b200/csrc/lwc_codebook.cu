@@ -28,8 +28,13 @@
 namespace lwc {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+// Warps per CTA by index width: the 32 and 64 KB tables of k = 14 and 15
+// leave room for only two CTAs per SM, so those CTAs carry more warps sharing
+// one copy (measured: 76-78 % of the HBM roofline instead of ~70 %). With
+// k = 16 (128 KB, one CTA per SM) more warps only add contention on the
+// table gathers, so it keeps 8.
+template <int K>
+constexpr int warps_for() { return K == 15 ? 12 : K == 14 ? 16 : 8; }
 constexpr int kPerLane = 32;                            // indices per lane per tile
 constexpr uint32_t kTile = 32 * kPerLane;               // indices per tile (one warp)
 constexpr int kMaxBatch = 32;
@@ -109,6 +114,7 @@ struct CbLayout {
     static constexpr uint32_t kTileBytes = 128u * K;                       // packed bytes of one tile
     static constexpr uint32_t kTabBytes = (2u << K) < 16u ? 16u : (2u << K);
     static constexpr uint32_t kBars = 0;                                    // 2 per warp + 1 for the table
+    static constexpr uint32_t kWarps = warps_for<K>();
     static constexpr uint32_t kBufs = 8 * (2 * kWarps + 2);
     static constexpr uint32_t kTab = kBufs + 2 * kWarps * kTileBytes;
     static constexpr uint32_t kTotal = kTab + kTabBytes;
@@ -126,11 +132,14 @@ __device__ __forceinline__ void issue_tile(const CbTensor &tn, uint64_t tile, ui
 
 // Persistent decoder: each CTA takes a contiguous run of tiles (1024 indices
 // each) from the launch's tile list; within one tensor, warp w handles tiles
-// w, w + 8, ... of the run with its own double buffer and mbarriers, so the
-// only CTA-wide barriers are at tensor boundaries (table reload).
+// w, w + W, ... (W warps per CTA) of the run with its own double buffer and
+// mbarriers, so the only CTA-wide barriers are at tensor boundaries (table
+// reload).
 template <int K>
-__global__ void __launch_bounds__(kThreads) cb_decode_kernel(const __grid_constant__ CbBatch B) {
+__global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2 : 4)   // CTAs per SM
+    cb_decode_kernel(const __grid_constant__ CbBatch B) {
     using Lay = CbLayout<K>;
+    constexpr uint32_t kWarps = Lay::kWarps;
     extern __shared__ __align__(16) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
     uint32_t *bufs = reinterpret_cast<uint32_t *>(smem + Lay::kBufs);
@@ -145,7 +154,7 @@ __global__ void __launch_bounds__(kThreads) cb_decode_kernel(const __grid_consta
     uint64_t *my_bar = &bars[2 * warp];
     uint32_t *my_buf = bufs + 2 * warp * (Lay::kTileBytes / 4);
     if (tid == 0) {
-        for (int i = 0; i < 2 * kWarps + 1; i++) dev::mbar_init(&bars[i], 1);
+        for (uint32_t i = 0; i < 2 * kWarps + 1; i++) dev::mbar_init(&bars[i], 1);
         dev::fence_mbar_init();
     }
     __syncthreads();
@@ -242,6 +251,10 @@ const KernelFn kKernels[17] = {nullptr,          kernel_for<1>(),  kernel_for<2>
 
 template <int K>
 constexpr uint32_t smem_for() { return CbLayout<K>::kTotal; }
+const int kWarpsFor[17] = {0,  warps_for<1>(),  warps_for<2>(),  warps_for<3>(),  warps_for<4>(),  warps_for<5>(),
+                           warps_for<6>(),  warps_for<7>(),  warps_for<8>(),  warps_for<9>(),  warps_for<10>(),
+                           warps_for<11>(), warps_for<12>(), warps_for<13>(), warps_for<14>(), warps_for<15>(),
+                           warps_for<16>()};
 const uint32_t kSmem[17] = {0,           smem_for<1>(),  smem_for<2>(),  smem_for<3>(),  smem_for<4>(),
                             smem_for<5>(),  smem_for<6>(),  smem_for<7>(),  smem_for<8>(),  smem_for<9>(),
                             smem_for<10>(), smem_for<11>(), smem_for<12>(), smem_for<13>(), smem_for<14>(),
@@ -271,7 +284,7 @@ lwc_status device_state(DevState &out) {
                 err = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                            cudaSharedmemCarveoutMaxShared);
             if (err == cudaSuccess)
-                err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.per_sm[k], fn, kThreads, kSmem[k]);
+                err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.per_sm[k], fn, 32 * kWarpsFor[k], kSmem[k]);
         }
         if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device setup: %s", cudaGetErrorString(err));
         s.ready = true;
@@ -303,9 +316,10 @@ lwc_status launch_cb_group(const std::vector<int> &idx, const lwc_desc *descs, c
     B.total_tiles = tiles;
     B.status = d_status;
     const int per_sm = std::max(1, ds.per_sm[K]);
+    const uint32_t warps = (uint32_t)kWarpsFor[K];
     // enough CTAs that every warp of every resident CTA gets tiles
-    const uint64_t grid = std::min<uint64_t>((tiles + kWarps - 1) / kWarps, (uint64_t)per_sm * ds.sms);
-    kKernels[K]<<<(unsigned)grid, kThreads, kSmem[K], stream>>>(B);
+    const uint64_t grid = std::min<uint64_t>((tiles + warps - 1) / warps, (uint64_t)per_sm * ds.sms);
+    kKernels[K]<<<(unsigned)grid, 32 * warps, kSmem[K], stream>>>(B);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
     return LWC_OK;

@@ -103,18 +103,23 @@ def test_codebook_small(name, w):
     assert np.array_equal(got, w)
 
 
-@pytest.mark.parametrize("U", [1, 2, 3, 5, 17, 200, 256, 600, 2000, 4096, 5000, 8192, 20000, 40000, 65536])
+@pytest.mark.parametrize("U", [1, 2, 3, 5, 17, 200, 256, 600, 2000, 4096, 5000, 8192, 10000, 16384, 20000, 40000,
+                               65536])
 def test_codebook_every_width(U):
     n = 3 * 8192 + 77
     if U == 65536:
         w = synth.as_u16(synth.uniform_patterns(200_000, seed=U))
         w[:65536] = np.arange(65536, dtype=np.uint16)
-    else:
-        w = synth.as_u16(synth.codebook_stress(U, n, seed=U))
+    else:   # Zipf draws plus every table entry once, so U (and k) are exact
+        draws = synth.as_u16(synth.codebook_stress(U, n, seed=U))
+        table = synth.codebook_table(U, seed=U).numpy().astype(np.uint16)
+        w = np.random.default_rng(U).permutation(np.concatenate([draws, table])).astype(np.uint16)
     d, b = lwc.lwc_encode_codebook(w)
-    assert d.U == len(np.unique(w))
+    assert d.U == len(np.unique(w)) == U
+    assert d.k == ocb.index_bits(U)
     got = host_u16(gpu_decode(d, dev(b), codec="cb"))
     assert np.array_equal(got, ocb.decode(b))
+    assert np.array_equal(got, w)
 
 
 def test_batched_mixed():
