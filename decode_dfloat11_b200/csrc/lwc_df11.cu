@@ -7,28 +7,34 @@
 //
 // How (same page, section "Jak to działa w praktyce? Magia na poziomie GPU"):
 //  * small linked lookup tables held in shared memory: the blob's
-//    hierarchical 256-entry tables (one per 8 code bits), fronted by two
-//    4096-entry tables this kernel builds from them, which resolve every code
-//    that fits in the next 12 stream bits — several codes per lookup;
+//    hierarchical 256-entry tables (one per 8 code bits), fronted by three
+//    2048-entry tables this kernel builds from them (symbols, code-end masks,
+//    code counts), which resolve every code that fits in the next 11 stream
+//    bits: several codes per lookup;
 //  * two phases: each thread counts the codes that start in its chunk of the
-//    stream, a block-wide scan turns the counts into output positions, and the
-//    threads decode again, this time writing exponents to a shared-memory
-//    staging buffer; the staged exponents are then merged with the
-//    sign|mantissa bytes and written out with 16-byte stores. Both passes
-//    take two table entries per 32-bit window read (up to 22 bits per step);
+//    stream, a scan turns the counts into output positions, and the threads
+//    decode again, this time writing exponents to a shared-memory staging
+//    buffer; the staged exponents are then merged with the sign|mantissa
+//    bytes (and, for FP32 / FP16 elements, the raw low mantissa bits) and
+//    written out with 16-byte stores. Both passes take two table entries per
+//    32-bit window (up to 22 bits per step);
 //  * all matrices of a transformer block in one launch: the grid walks a work
 //    list of (tensor, block) items; CTAs are persistent, take contiguous runs
 //    of items and rebuild their tables only when the tensor changes.
 // Blocks never wait on one another: each block's first output index is stored
 // in the blob, so there is no inter-block scan.
 //
-// Memory pipeline per CTA: as soon as pass 2 of item j no longer needs the
-// shared stream segment, the bulk-copy (TMA) engine starts bringing in the
-// segment and chunk gaps of item j+1, overlapping the merge of item j; the
-// sign|mantissa bytes each thread merges are loaded into registers at the
-// start of an item, under both decode passes; block offsets are loaded one
-// item ahead. One segment buffer (not two) keeps four CTAs resident per SM.
-// No wait is unbounded.
+// Two kernels. df11_warp_kernel (blocks of 32 chunks, the encoder's default):
+// one warp decodes one block with a warp scan and its own segment buffer,
+// staging area and mbarrier, so no CTA-wide barrier sits on the per-block
+// path; 18 warps per CTA share the tables. df11_decode_kernel (blocks of 64+
+// chunks): one block per CTA and a block scan.
+//
+// Memory pipeline: as soon as pass 2 of an item no longer needs the shared
+// stream segment, the bulk-copy (TMA) engine starts bringing in the segment
+// and chunk gaps of the next item, overlapping the merge; the sign|mantissa
+// bytes are loaded into registers at the start of an item, under both decode
+// passes; block offsets are loaded one item ahead. No wait is unbounded.
 #include <cuda_runtime.h>
 
 #include <algorithm>
