@@ -430,55 +430,30 @@ def run_lwc(args, rank, world, local_rank, dist):
         del src, work
 
     # end to end through the C ABI with host buffers: pinned blobs -> device,
-    # decode, decoded layer -> pinned host, every step. The copies of tensor i
-    # overlap the decode of tensor i - 1 and the read-back of tensor i - 2
-    # (three streams, smallest tensors first), so both PCIe directions run at
-    # once; the timing events sit on the decode stream, which waits for the
-    # last read-back before the end event.
+    # decode, decoded layer -> pinned host, every step (layers.HostPipeline:
+    # tensor i's upload, i-1's decode and i-2's read-back overlap on three
+    # streams; the timing events sit on the decode stream, which waits for the
+    # last read-back before the end event).
     if not args.no_e2e:
-        pinned_in = [torch.from_numpy(b).pin_memory() for b in blobs_h]
-        pinned_out = torch.empty(n_total, dtype=torch.bfloat16).pin_memory()
-        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-        out_offsets = []
-        off = 0
-        for w in tensors:
-            out_offsets.append(off)
-            off += w.size
-        order = sorted(range(len(tensors)), key=lambda i: tensors[i].size)
+        from decode_dfloat11_b200.layers import HostPipeline
+        pipe = HostPipeline(descs, [torch.from_numpy(b) for b in blobs_h], "dfloat11", device)
 
         def estep():
-            s_in.wait_stream(stream)       # the previous step is done with every buffer
-            done_in, done_dec = [], []
-            for i in order:
-                with torch.cuda.stream(s_in):
-                    blobs_d[i].copy_(pinned_in[i], non_blocking=True)
-                ev = torch.cuda.Event()
-                ev.record(s_in)
-                done_in.append(ev)
-            for j, i in enumerate(order):
-                stream.wait_event(done_in[j])
-                lwc.lwc_decode_dfloat11(descs[i], blobs_d[i], views[i], stream)
-                ev = torch.cuda.Event()
-                ev.record(stream)
-                done_dec.append(ev)
-            for j, i in enumerate(order):
-                s_out.wait_event(done_dec[j])
-                with torch.cuda.stream(s_out):
-                    pinned_out[out_offsets[i]:out_offsets[i] + tensors[i].size].copy_(views[i], non_blocking=True)
-            stream.wait_stream(s_out)
+            pipe.run(stream)
         for _ in range(3):
             estep()
         e_steps = max(3, min(args.steps, 20))
         torch.cuda.synchronize(device)
         ems = time_steps(estep, e_steps, stream) / e_steps
         torch.cuda.synchronize(device)
-        for w, off in zip(tensors, out_offsets):
-            if not torch.equal(pinned_out.view(torch.int16)[off:off + w.size], torch.from_numpy(w.view(np.int16))):
+        for w, off in zip(tensors, pipe.offsets):
+            if not torch.equal(pipe.host_out.view(torch.int16)[off:off + w.size], torch.from_numpy(w.view(np.int16))):
                 raise SystemExit("end-to-end output differs from its input")
         ev = whole_job_gbs(world, 2 * n_total, max_over_ranks(ems, dist, device))
-        result["e2e"] = {"value": round(ev, 3), "unit": "GB/s", "h2d_bytes_per_step": blob_bytes,
-                         "d2h_bytes_per_step": 2 * n_total, "ms_per_step": round(ems, 4), "steps": e_steps,
-                         "pipeline": "per-tensor H2D / decode / D2H on three streams"}
+        result["e2e"] = {"value": round(ev, 3), "unit": "GB/s", "h2d_bytes_per_step": pipe.h2d_bytes,
+                         "d2h_bytes_per_step": pipe.d2h_bytes, "ms_per_step": round(ems, 4), "steps": e_steps,
+                         "pipeline": "layers.HostPipeline: per-tensor H2D / decode / D2H on three streams"}
+        del pipe
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(blobs_h, n_total)

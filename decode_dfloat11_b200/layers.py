@@ -185,3 +185,71 @@ class ResidentModel:
             yield i, self.views(i, slot)
             free[slot].record(compute_stream)
             used[slot] = True
+
+
+class HostPipeline:
+    """Compressed tensors held in (pinned) host memory, decoded through the GPU
+    back into host memory, with the transfers overlapped: tensor i's upload,
+    tensor i-1's decode and tensor i-2's read-back run on three streams, so
+    both PCIe directions are busy at once (smallest tensors first, so the
+    read-back starts early).
+
+    ``run()`` enqueues one pass on ``stream`` (and two helper streams) and
+    returns; work after it on ``stream`` sees the host output complete once
+    the stream is synchronised.
+    """
+
+    def __init__(self, descs, host_blobs, codec: str, device, host_out=None):
+        import torch
+        if codec not in CODECS:
+            raise ValueError(f"unknown codec {codec!r}")
+        self.codec = codec
+        self.device = torch.device(device)
+        self.descs = list(descs)
+        self.pinned_in = [b if isinstance(b, torch.Tensor) and b.is_pinned() else
+                          torch.as_tensor(b).pin_memory() for b in host_blobs]
+        self.blobs = [torch.empty(b.numel(), dtype=torch.uint8, device=self.device) for b in self.pinned_in]
+        ns = [d.n for d in self.descs]
+        self.offsets = []            # element offsets, multiples of 8 (16-byte aligned views)
+        off = 0
+        for n in ns:
+            self.offsets.append(off)
+            off += (n + 7) // 8 * 8
+        self.out = torch.empty(off, dtype=torch.bfloat16, device=self.device)
+        self.host_out = host_out if host_out is not None else torch.empty(off, dtype=torch.bfloat16).pin_memory()
+        self.views = [self.out[o:o + n] for o, n in zip(self.offsets, ns)]
+        self.order = sorted(range(len(ns)), key=lambda i: ns[i])
+        self.s_in = torch.cuda.Stream(self.device)
+        self.s_out = torch.cuda.Stream(self.device)
+
+    @property
+    def h2d_bytes(self) -> int:
+        return sum(int(b.numel()) for b in self.pinned_in)
+
+    @property
+    def d2h_bytes(self) -> int:
+        return 2 * sum(d.n for d in self.descs)
+
+    def run(self, stream) -> None:
+        import torch
+        decode = lwc.lwc_decode_dfloat11 if self.codec == "dfloat11" else lwc.lwc_decode_codebook
+        self.s_in.wait_stream(stream)        # earlier work on `stream` is done with every buffer
+        done_in, done_dec = [], []
+        for i in self.order:
+            with torch.cuda.stream(self.s_in):
+                self.blobs[i].copy_(self.pinned_in[i], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.s_in)
+            done_in.append(ev)
+        for j, i in enumerate(self.order):
+            stream.wait_event(done_in[j])
+            decode(self.descs[i], self.blobs[i], self.views[i], stream)
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            done_dec.append(ev)
+        for j, i in enumerate(self.order):
+            self.s_out.wait_event(done_dec[j])
+            o, n = self.offsets[i], self.descs[i].n
+            with torch.cuda.stream(self.s_out):
+                self.host_out[o:o + n].copy_(self.views[i], non_blocking=True)
+        stream.wait_stream(self.s_out)

@@ -154,3 +154,23 @@ def test_layer_decodes_replay_from_a_cuda_graph():
             for (name, gen), got in zip(units, sinks[c]):
                 want = torch.cat([t.reshape(-1) for t in gen()])
                 assert torch.equal(got.view(torch.int16), want.view(torch.int16)), (c, name)
+
+
+@pytest.mark.parametrize("codec", ["dfloat11", "codebook"])
+def test_host_pipeline_round_trip(codec):
+    """Host blobs -> GPU decode -> host output with overlapped transfers
+    (layers.HostPipeline), run twice on the same buffers."""
+    from decode_dfloat11_b200.layers import HostPipeline
+    ws = [synth.as_u16(synth.normal_bf16((n,), seed=9100 + n, sigma=0.02, outlier_frac=1e-3))
+          for n in (1_000_003, 17, 4_194_304, 65_537)]
+    enc = encode_many(ws, codec)
+    pipe = HostPipeline([d for d, _ in enc], [b for _, b in enc], codec, "cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(2):
+        pipe.host_out.zero_()
+        pipe.run(stream)
+        stream.synchronize()
+        got = pipe.host_out.view(torch.int16).numpy().view(np.uint16)
+        for w, off in zip(ws, pipe.offsets):
+            assert np.array_equal(got[off:off + w.size], w)
+    assert pipe.h2d_bytes == sum(b.size for _, b in enc) and pipe.d2h_bytes == 2 * sum(w.size for w in ws)
