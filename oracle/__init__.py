@@ -3,7 +3,9 @@
 A plain, slow, obviously correct CPU implementation of what the decode path
 computes: the DFloat11-style exponent-Huffman codec (``oracle.df11``, with
 the code construction in ``oracle.huffman``) and the codebook codec
-(``oracle.codebook``), over the container in ``oracle.blob``. The per-weight
+(``oracle.codebook``), over the container in ``oracle.blob``; and the linear
+layer that consumes a decompressed matrix (``oracle.linear``, float64, with
+the float32 rounding bounds a device result is held to). The per-weight
 loops are plain C (``native.c``, one bit at a time); the rest is Python.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
@@ -19,14 +21,17 @@ over all length vectors on small alphabets, with and without a length
 limit) and within one bit of the exponent entropy; the canonical codes and
 bit order match hand-derived worked examples under ``tests/golden/``; the
 codebook width is ceil(log2 U) and its table is the sorted set of distinct
-patterns (checked against a brute-force count). The exact bytes of a
+patterns (checked against a brute-force count); BF16 values follow the
+IEEE-754 fields (hand-derived values, numpy's float32 view on all 65536
+patterns), and the linear layer matches a hand-derived worked example,
+closed forms, one-hot columns and exact rational sums. The exact bytes of a
 stream are pinned only through those worked examples: the pages print no
 encoded example of their own.
 """
-from . import blob, codebook, df11, huffman
+from . import blob, codebook, df11, huffman, linear
 from ._native import build
 
-__all__ = ["blob", "codebook", "df11", "huffman", "build", "decode"]
+__all__ = ["blob", "codebook", "df11", "huffman", "linear", "build", "decode"]
 
 
 def decode(blob_bytes):

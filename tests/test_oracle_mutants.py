@@ -130,3 +130,50 @@ def test_pack3_msb_first_is_caught(monkeypatch):
         return np.packbits(bits, bitorder="little")
     monkeypatch.setattr(df11, "pack3", bad)
     fails(pins.test_pack3_is_little_endian_bit_concatenation)
+
+
+# ---- linear-layer oracle (oracle/linear.py) ----------------------------------
+
+import test_oracle_linear as lpins
+from oracle import linear as OL
+
+
+def _bad_linear(transform):
+    def bad(w_bits, x_bits):
+        w = OL.bf16_values(w_bits)
+        x = OL.bf16_values(x_bits)
+        w, x = transform(w, x)
+        return x @ w.T, np.abs(x) @ np.abs(w).T
+    return bad
+
+
+def test_linear_transposed_operand_is_caught(monkeypatch):
+    monkeypatch.setattr(OL, "linear", lambda w_bits, x_bits: (
+        OL.bf16_values(x_bits) @ OL.bf16_values(w_bits), np.abs(OL.bf16_values(x_bits)) @ np.abs(OL.bf16_values(w_bits))))
+    fails(lpins.test_golden_square_example_catches_a_transpose)
+
+
+def test_linear_shifted_column_is_caught(monkeypatch):
+    monkeypatch.setattr(OL, "linear", _bad_linear(lambda w, x: (w, np.roll(x, 1, axis=1))))
+    fails(lpins.test_one_hot_selects_a_column, 6)
+    fails(lpins.test_golden_rectangular_example)
+
+
+def test_linear_dropped_last_column_is_caught(monkeypatch):
+    monkeypatch.setattr(OL, "linear", _bad_linear(lambda w, x: (w[:, :-1], x[:, :-1])))
+    fails(lpins.test_ones_closed_form)
+    fails(lpins.test_exact_rational_sums, 0)
+
+
+def test_bf16_exponent_bias_off_by_one_is_caught(monkeypatch):
+    good = OL.bf16_values
+    monkeypatch.setattr(OL, "bf16_values", lambda b: good(b) * 0.5)
+    fails(lpins.test_bf16_field_values)
+    fails(lpins.test_bf16_values_match_float32_upper_half_on_every_pattern)
+
+
+def test_bf16_sign_dropped_is_caught(monkeypatch):
+    good = OL.bf16_values
+    monkeypatch.setattr(OL, "bf16_values", lambda b: np.abs(good(b)))
+    fails(lpins.test_bf16_field_values)
+    fails(lpins.test_golden_rectangular_example)
