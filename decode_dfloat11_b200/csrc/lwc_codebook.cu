@@ -238,6 +238,279 @@ __global__ void cb_fill_kernel(uint16_t *__restrict__ out, uint64_t n, const uin
     }
 }
 
+// ---- fused decode + linear layer ---------------------------------------------
+//
+// y[m, r] = sum_c W[r, c] x[m, c] for M <= 8 activation rows, with W the
+// tensor's rows x cols weights, decoded in registers and never written out.
+// One warp owns one row at a time and walks it in windows of 1024 indices
+// (32 per lane); each window's packed bits are bulk-copied from the
+// 16-byte boundary at or below its first bit, and every lane re-aligns its K
+// + 1 words by the window's bit offset (the same for all lanes, since 32
+// fields are K whole words), so the fields keep compile-time positions for
+// any cols. Each lane sums its 32 products of a window in FP32 as one FMA
+// chain per activation row and adds that to its running sum for the row; a
+// 5-level butterfly sums the lanes, and lane 0 stores the row's outputs: the
+// summation tree has height at most ceil(cols / 1024) + 37, and the result
+// does not depend on the launch shape.
+
+constexpr int kMaxRows = 8;          // activation rows per call
+constexpr uint32_t kLinWarps = 8;    // warps per CTA
+
+struct CbLinTensor {
+    const uint8_t *packed;
+    uint64_t packed_bytes;
+    const uint16_t *table;
+    const uint16_t *x;     // M x cols BF16, row-major
+    float *y;              // M x rows FP32, row-major
+    uint64_t rows;
+    uint64_t first_row;    // index of this tensor's row 0 in the launch's row list
+    uint64_t first_win;    // index of its first window in the launch's window list
+    uint32_t cols;
+    uint32_t table_bytes;
+};
+
+struct CbLinBatch {
+    CbLinTensor t[kMaxBatch];
+    uint32_t count;
+    uint32_t M;
+    uint64_t total_rows;
+    uint64_t total_wins;
+    uint32_t *status;
+};
+
+// The first row (in the launch's row list) whose first window is at or after
+// window u: CTAs take equal runs of windows, rounded to whole rows.
+__device__ __forceinline__ uint64_t row_at_window(const CbLinBatch &B, uint64_t u) {
+    if (u >= B.total_wins) return B.total_rows;
+    uint32_t t = 0;
+    while (t + 1 < B.count && B.t[t + 1].first_win <= u) ++t;
+    const CbLinTensor &tn = B.t[t];
+    const uint32_t nwin = (tn.cols + kTile - 1) / kTile;
+    return tn.first_row + (u - tn.first_win + nwin - 1) / nwin;
+}
+
+template <int K>
+struct CbLinLayout {
+    // a window's 128 K bytes from the aligned start at or below its first bit
+    // (at most 15 bytes earlier), plus the word after its last field
+    static constexpr uint32_t kBufBytes = 128u * K + 48u;
+    static constexpr uint32_t kTabBytes = (2u << K) < 16u ? 16u : (2u << K);
+    static constexpr uint32_t kWarps = kLinWarps;
+    static constexpr uint32_t kBars = 0;
+    static constexpr uint32_t kBufs = 8 * (2 * kWarps + 2);
+    static constexpr uint32_t kTab = kBufs + 2 * kWarps * kBufBytes;
+    static constexpr uint32_t kTotal = kTab + kTabBytes;
+};
+
+// Index range of window q of row r: first index and count.
+__device__ __forceinline__ uint64_t window_first(const CbLinTensor &tn, uint64_t r, uint32_t q) {
+    return r * tn.cols + (uint64_t)q * kTile;
+}
+__device__ __forceinline__ uint32_t window_count(const CbLinTensor &tn, uint32_t q) {
+    return min(kTile, tn.cols - q * kTile);
+}
+
+// Lane 0: bulk copy of window q of row r into dst, completing on bar.
+template <int K>
+__device__ __forceinline__ void issue_window(const CbLinTensor &tn, uint64_t r, uint32_t q, uint32_t *dst,
+                                             uint64_t *bar) {
+    const uint64_t bit0 = window_first(tn, r, q) * K;
+    const uint64_t a0 = (bit0 >> 3) & ~15ull;
+    const uint64_t need = (bit0 + (uint64_t)window_count(tn, q) * K + 7) / 8 + 4;   // through the next word
+    uint64_t end = (need + 15) & ~15ull;
+    if (end > tn.packed_bytes) end = tn.packed_bytes;   // the words past the section are never used
+    const uint32_t bytes = (uint32_t)(end - a0);
+    dev::mbar_arrive_expect_tx(bar, bytes);
+    dev::bulk_g2s(dst, tn.packed + a0, bytes, bar);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
+
+// acc + dot(v, x[0..31]) as one FMA chain; v holds the 32 weights as BF16
+// pairs, x is 16-byte aligned.
+__device__ __forceinline__ float dot32(const uint32_t (&v)[16], const uint16_t *x, float acc) {
+    const uint4 *xp = reinterpret_cast<const uint4 *>(x);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint4 q = __ldg(xp + i);
+        acc = fmaf(bf16_lo(v[4 * i + 0]), bf16_lo(q.x), acc);
+        acc = fmaf(bf16_hi(v[4 * i + 0]), bf16_hi(q.x), acc);
+        acc = fmaf(bf16_lo(v[4 * i + 1]), bf16_lo(q.y), acc);
+        acc = fmaf(bf16_hi(v[4 * i + 1]), bf16_hi(q.y), acc);
+        acc = fmaf(bf16_lo(v[4 * i + 2]), bf16_lo(q.z), acc);
+        acc = fmaf(bf16_hi(v[4 * i + 2]), bf16_hi(q.z), acc);
+        acc = fmaf(bf16_lo(v[4 * i + 3]), bf16_lo(q.w), acc);
+        acc = fmaf(bf16_hi(v[4 * i + 3]), bf16_hi(q.w), acc);
+    }
+    return acc;
+}
+
+// Lane 0 of the warp stores the butterfly sums of acc[m] as y[m, row]; acc is reset.
+template <int MM>
+__device__ __forceinline__ void finish_row(float (&acc)[MM], uint32_t M, float *y, uint64_t rows, uint64_t row,
+                                           uint32_t lane) {
+#pragma unroll
+    for (int m = 0; m < MM; m++) {
+        if ((uint32_t)m < M) {
+            float v = acc[m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            if (lane == 0) y[(uint64_t)m * rows + row] = v;
+        }
+        acc[m] = 0.f;
+    }
+}
+
+// MM: the largest number of activation rows the instance handles (1, 2, 4, 8).
+template <int K, int MM>
+__global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : MM == 1 ? 4 : 3)
+    cb_linear_kernel(const __grid_constant__ CbLinBatch B) {
+    using Lay = CbLinLayout<K>;
+    constexpr uint32_t kWarps = Lay::kWarps;
+    constexpr uint32_t kBufWords = Lay::kBufBytes / 4;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
+    uint32_t *bufs = reinterpret_cast<uint32_t *>(smem + Lay::kBufs);
+    uint16_t *tab = reinterpret_cast<uint16_t *>(smem + Lay::kTab);
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    const uint32_t M = B.M;
+
+    const uint64_t r_begin = row_at_window(B, B.total_wins * blockIdx.x / gridDim.x);
+    const uint64_t r_end = row_at_window(B, B.total_wins * (blockIdx.x + 1) / gridDim.x);
+    if (r_begin >= r_end) return;
+
+    uint64_t *tab_bar = &bars[2 * kWarps];
+    uint64_t *my_bar = &bars[2 * warp];
+    uint32_t *my_buf = bufs + 2 * warp * kBufWords;
+    if (tid == 0) {
+        for (uint32_t i = 0; i < 2 * kWarps + 1; i++) dev::mbar_init(&bars[i], 1);
+        dev::fence_mbar_init();
+    }
+    __syncthreads();
+
+    uint32_t it = 0, tab_uses = 0, status = 0;
+    bool dead = false;
+    uint32_t ti = 0;
+    uint64_t r = r_begin;
+    float acc[MM];
+#pragma unroll
+    for (int m = 0; m < MM; m++) acc[m] = 0.f;
+    while (r < r_end) {
+        while (ti + 1 < B.count && r >= B.t[ti + 1].first_row) ++ti;
+        const CbLinTensor &tn = B.t[ti];
+        const uint64_t seg_end = ti + 1 < B.count ? min(r_end, B.t[ti + 1].first_row) : r_end;
+        const uint64_t s0 = r - tn.first_row, ns = seg_end - r;   // this tensor's rows [s0, s0 + ns)
+        const uint32_t nwin = (tn.cols + kTile - 1) / kTile;
+        const bool vec = (tn.cols & 7u) == 0;                    // 16-byte aligned activation chunks
+
+        __syncthreads();
+        if (tid == 0) {
+            dev::fence_proxy_async_smem();
+            dev::mbar_arrive_expect_tx(tab_bar, tn.table_bytes);
+            dev::bulk_g2s(tab, tn.table, tn.table_bytes, tab_bar);
+        }
+        // this warp's (row, window) items: rows s0 + warp, + kWarps, ...; windows 0 .. nwin - 1.
+        // (ir, iq): the next item to issue; (cr, cq): the item being consumed.
+        uint64_t ir = s0 + warp, cr = ir;
+        uint32_t iq = 0, cq = 0, issued = 0;
+        const uint64_t row_end = s0 + ns;
+        for (; issued < 2 && ir < row_end; issued++) {   // the first two items
+            if (lane == 0 && !dead)
+                issue_window<K>(tn, ir, iq, my_buf + ((it + issued) & 1u) * kBufWords, &my_bar[(it + issued) & 1u]);
+            if (++iq == nwin) { iq = 0; ir += kWarps; }
+        }
+        const bool tab_ok = dev::mbar_wait_bounded(tab_bar, tab_uses & 1u);
+        tab_uses++;
+        if (__syncthreads_or(!tab_ok)) {
+            // let this warp's copies land (bounded), then stop
+            status |= LWC_DEVICE_TIMEOUT;
+            if (!dead)
+                for (uint32_t k = 0; k < issued; k++) dev::mbar_wait_bounded(&my_bar[(it + k) & 1u], ((it + k) >> 1) & 1u);
+            break;
+        }
+
+        while (cr < row_end && !dead) {
+            const uint32_t bi = it & 1u;
+            const bool ok = dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
+            if (__any_sync(0xFFFFFFFFu, !ok)) {
+                // let the copy issued into the other buffer land (bounded), then stop
+                status |= LWC_DEVICE_TIMEOUT;
+                if (cq + 1 < nwin || cr + kWarps < row_end) dev::mbar_wait_bounded(&my_bar[bi ^ 1u], ((it + 1) >> 1) & 1u);
+                dead = true;
+                break;
+            }
+            const uint64_t bit0 = window_first(tn, cr, cq) * K;
+            const uint32_t boff = (uint32_t)(bit0 - (((bit0 >> 3) & ~15ull) << 3));   // < 128
+            const uint32_t cnt = window_count(tn, cq);
+            const uint32_t *src = my_buf + bi * kBufWords + (boff >> 5) + lane * K;
+            const uint32_t sh = boff & 31u;
+            uint32_t w[K + 1];
+#pragma unroll
+            for (int i = 0; i < K; i++) w[i] = __funnelshift_r(src[i], src[i + 1], sh);
+            w[K] = 0;
+            uint32_t v[16];   // weights 2i, 2i + 1 as a BF16 pair
+            Gather<K, 0>::run(w, tab, v);
+            __syncwarp();
+            if (lane == 0 && ir < row_end) {
+                dev::fence_proxy_async_smem();
+                issue_window<K>(tn, ir, iq, my_buf + bi * kBufWords, &my_bar[bi]);
+            }
+            if (ir < row_end && ++iq == nwin) { iq = 0; ir += kWarps; }
+
+            const uint32_t c0 = cq * kTile + lane * 32u;
+            const uint32_t valid = cnt > lane * 32u ? min(32u, cnt - lane * 32u) : 0u;
+            const uint16_t *xr = tn.x + c0;
+            // each window's products form their own FMA chain, then join the row's sum
+            if (valid == 32u && vec) {
+#pragma unroll
+                for (int m = 0; m < MM; m++)
+                    if ((uint32_t)m < M) acc[m] += dot32(v, xr + (uint64_t)m * tn.cols, 0.f);
+            } else if (valid) {
+#pragma unroll
+                for (int m = 0; m < MM; m++) {
+                    if ((uint32_t)m < M) {
+                        const uint16_t *xm = xr + (uint64_t)m * tn.cols;
+                        float p = 0.f;
+#pragma unroll
+                        for (int j = 0; j < 32; j++)
+                            if ((uint32_t)j < valid)
+                                p = fmaf(bf16_lo(v[j / 2] >> (16 * (j & 1))), bf16_lo(xm[j]), p);
+                        acc[m] += p;
+                    }
+                }
+            }
+            if (++cq == nwin) {
+                finish_row<MM>(acc, M, tn.y, tn.rows, cr, lane);
+                cq = 0;
+                cr += kWarps;
+            }
+            ++it;
+        }
+        r = seg_end;
+    }
+    if (status && lane == 0 && B.status) atomicOr(B.status, status);
+}
+
+// U == 1: every weight is table[0]; one warp per row, lane-strided columns
+// (summation tree height ceil(cols / 32) + 5).
+__global__ void cb_linear_fill_kernel(const uint16_t *__restrict__ table, const uint16_t *__restrict__ x, uint32_t M,
+                                      uint64_t rows, uint32_t cols, float *__restrict__ y) {
+    const float wv = __uint_as_float((uint32_t)table[0] << 16);
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x / 32);
+    float acc[kMaxRows];
+#pragma unroll
+    for (int m = 0; m < kMaxRows; m++) acc[m] = 0.f;
+    for (uint64_t r = blockIdx.x * (uint64_t)(blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+#pragma unroll
+        for (int m = 0; m < kMaxRows; m++)
+            if ((uint32_t)m < M)
+                for (uint32_t c = lane; c < cols; c += 32u) acc[m] = fmaf(wv, bf16_lo(x[(uint64_t)m * cols + c]), acc[m]);
+        finish_row<kMaxRows>(acc, M, y, rows, r, lane);
+    }
+}
+
 using KernelFn = void (*)(CbBatch);
 
 template <int K>
@@ -260,9 +533,31 @@ const uint32_t kSmem[17] = {0,           smem_for<1>(),  smem_for<2>(),  smem_fo
                             smem_for<10>(), smem_for<11>(), smem_for<12>(), smem_for<13>(), smem_for<14>(),
                             smem_for<15>(), smem_for<16>()};
 
+using LinKernelFn = void (*)(CbLinBatch);
+template <int MM>
+struct LinTable {
+    static constexpr LinKernelFn k[17] = {
+        nullptr,                  cb_linear_kernel<1, MM>,  cb_linear_kernel<2, MM>,  cb_linear_kernel<3, MM>,
+        cb_linear_kernel<4, MM>,  cb_linear_kernel<5, MM>,  cb_linear_kernel<6, MM>,  cb_linear_kernel<7, MM>,
+        cb_linear_kernel<8, MM>,  cb_linear_kernel<9, MM>,  cb_linear_kernel<10, MM>, cb_linear_kernel<11, MM>,
+        cb_linear_kernel<12, MM>, cb_linear_kernel<13, MM>, cb_linear_kernel<14, MM>, cb_linear_kernel<15, MM>,
+        cb_linear_kernel<16, MM>};
+};
+constexpr int kMmCount = 4;   // instances for M <= 1, 2, 4, 8
+constexpr int mm_index(uint32_t M) { return M <= 1 ? 0 : M <= 2 ? 1 : M <= 4 ? 2 : 3; }
+const LinKernelFn *const kLinKernels[kMmCount] = {LinTable<1>::k, LinTable<2>::k, LinTable<4>::k, LinTable<8>::k};
+template <int K>
+constexpr uint32_t lin_smem_for() { return CbLinLayout<K>::kTotal; }
+const uint32_t kLinSmem[17] = {0,
+                               lin_smem_for<1>(),  lin_smem_for<2>(),  lin_smem_for<3>(),  lin_smem_for<4>(),
+                               lin_smem_for<5>(),  lin_smem_for<6>(),  lin_smem_for<7>(),  lin_smem_for<8>(),
+                               lin_smem_for<9>(),  lin_smem_for<10>(), lin_smem_for<11>(), lin_smem_for<12>(),
+                               lin_smem_for<13>(), lin_smem_for<14>(), lin_smem_for<15>(), lin_smem_for<16>()};
+
 struct DevState {
     int sms = 0;
     int per_sm[17] = {0};
+    int lin_per_sm[4][17] = {{0}};
     bool ready = false;
 };
 std::mutex g_mutex;
@@ -285,6 +580,16 @@ lwc_status device_state(DevState &out) {
                                            cudaSharedmemCarveoutMaxShared);
             if (err == cudaSuccess)
                 err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.per_sm[k], fn, 32 * kWarpsFor[k], kSmem[k]);
+            for (int mi = 0; mi < kMmCount && err == cudaSuccess; mi++) {
+                const void *lf = (const void *)kLinKernels[mi][k];
+                err = cudaFuncSetAttribute(lf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLinSmem[k]);
+                if (err == cudaSuccess)
+                    err = cudaFuncSetAttribute(lf, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                               cudaSharedmemCarveoutMaxShared);
+                if (err == cudaSuccess)
+                    err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.lin_per_sm[mi][k], lf, 32 * kLinWarps,
+                                                                        kLinSmem[k]);
+            }
         }
         if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device setup: %s", cudaGetErrorString(err));
         s.ready = true;
@@ -322,6 +627,45 @@ lwc_status launch_cb_group(const std::vector<int> &idx, const lwc_desc *descs, c
     kKernels[K]<<<(unsigned)grid, 32 * warps, kSmem[K], stream>>>(B);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return LWC_OK;
+}
+
+lwc_status launch_cb_linear_group(const std::vector<int> &idx, const lwc_desc *descs, const void *const *d_blobs,
+                                  const uint64_t *cols, const uint16_t *const *d_xs, uint32_t M, float *const *d_ys,
+                                  uint32_t *d_status, cudaStream_t stream, const DevState &ds) {
+    CbLinBatch B;
+    std::memset(&B, 0, sizeof B);
+    const uint32_t K = descs[idx[0]].k;
+    uint64_t rows = 0, wins = 0;
+    for (size_t j = 0; j < idx.size(); j++) {
+        const int i = idx[j];
+        const lwc_desc &d = descs[i];
+        const uint8_t *base = static_cast<const uint8_t *>(d_blobs[i]);
+        CbLinTensor &t = B.t[j];
+        t.packed = base + d.off_packed;
+        t.packed_bytes = d.packed_bytes;
+        t.table = reinterpret_cast<const uint16_t *>(base + d.off_table);
+        t.table_bytes = (uint32_t)((2ull * d.U + 15) / 16 * 16);
+        t.x = d_xs[i];
+        t.y = d_ys[i];
+        t.cols = (uint32_t)cols[i];
+        t.rows = d.n / cols[i];
+        t.first_row = rows;
+        t.first_win = wins;
+        rows += t.rows;
+        wins += t.rows * ((t.cols + kTile - 1) / kTile);
+    }
+    B.count = (uint32_t)idx.size();
+    B.M = M;
+    B.total_rows = rows;
+    B.total_wins = wins;
+    B.status = d_status;
+    const int mi = mm_index(M);
+    const int per_sm = std::max(1, ds.lin_per_sm[mi][K]);
+    const uint64_t grid = std::min<uint64_t>((rows + kLinWarps - 1) / kLinWarps, (uint64_t)per_sm * ds.sms);
+    kLinKernels[mi][K]<<<(unsigned)grid, 32 * kLinWarps, kLinSmem[K], stream>>>(B);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));
     return LWC_OK;
 }
 
@@ -390,6 +734,67 @@ lwc_status lwc_decode_codebook_checked(const lwc_desc *desc, const void *d_in, u
 
 lwc_status lwc_decode_codebook(const lwc_desc *desc, const void *d_in, uint16_t *d_out, lwc_stream_t stream) {
     return lwc_decode_codebook_checked(desc, d_in, d_out, nullptr, stream);
+}
+
+lwc_status lwc_linear_codebook_batched(const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
+                                       const uint16_t *const *d_xs, int M, float *const *d_ys, int count,
+                                       uint32_t *d_status, lwc_stream_t stream) {
+    if (count < 0 || (count > 0 && (!descs || !d_blobs || !cols || !d_xs || !d_ys)))
+        return fail(LWC_ERR_INVALID_ARG, "bad batch arguments");
+    if (M < 1 || M > kMaxRows) return fail(LWC_ERR_INVALID_ARG, "M must be 1..%d (got %d)", kMaxRows, M);
+    bool any = false;
+    for (int i = 0; i < count; i++) {
+        lwc_status st = check_codebook_desc(&descs[i]);
+        if (st) return st;
+        if (cols[i] == 0 || cols[i] >= (1ull << 31) || descs[i].n % cols[i] != 0)
+            return fail(LWC_ERR_INVALID_ARG, "cols must be 1..2^31-1 and divide n (tensor %d)", i);
+        if (descs[i].n == 0) continue;
+        any = true;
+        if (!d_blobs[i] || !d_xs[i] || !d_ys[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (tensor %d)", i);
+        if (!aligned16(d_blobs[i]) || !aligned16(d_xs[i]) || (reinterpret_cast<uintptr_t>(d_ys[i]) & 3u))
+            return fail(LWC_ERR_MISALIGNED, "blob and x must be 16-byte aligned, y 4-byte aligned (tensor %d)", i);
+    }
+    if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u))
+        return fail(LWC_ERR_MISALIGNED, "status word must be 4-byte aligned");
+    if (!any) {
+        clear_error();
+        return LWC_OK;
+    }
+    DevState ds;
+    lwc_status st = device_state(ds);
+    if (st) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<std::vector<int>> by_k(17);
+    for (int i = 0; i < count; i++) {
+        const lwc_desc &d = descs[i];
+        if (d.n == 0) continue;
+        if (d.k == 0) {
+            const uint64_t rows = d.n / cols[i];
+            const uint64_t blocks = std::min<uint64_t>((rows + 7) / 8, (uint64_t)ds.sms * 8);
+            cb_linear_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+                reinterpret_cast<const uint16_t *>(static_cast<const uint8_t *>(d_blobs[i]) + d.off_table), d_xs[i],
+                (uint32_t)M, rows, (uint32_t)cols[i], d_ys[i]);
+            cudaError_t err = cudaGetLastError();
+            if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));
+            continue;
+        }
+        by_k[d.k].push_back(i);
+    }
+    for (int k = 1; k <= 16; k++) {
+        for (size_t a = 0; a < by_k[k].size(); a += kMaxBatch) {
+            std::vector<int> g(by_k[k].begin() + a, by_k[k].begin() + std::min(by_k[k].size(), a + kMaxBatch));
+            st = launch_cb_linear_group(g, descs, d_blobs, cols, d_xs, (uint32_t)M, d_ys, d_status, s, ds);
+            if (st) return st;
+        }
+    }
+    clear_error();
+    return LWC_OK;
+}
+
+lwc_status lwc_linear_codebook(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x, int M,
+                               float *d_y, uint32_t *d_status, lwc_stream_t stream) {
+    if (!desc) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    return lwc_linear_codebook_batched(desc, &d_blob, &cols, &d_x, M, &d_y, 1, d_status, stream);
 }
 
 }  // extern "C"

@@ -81,6 +81,7 @@ struct Df11Batch {
     uint32_t seg_words;    // words staged per block: T * chunk_words + 2, rounded up to 4
     uint32_t stage_bytes;  // exponent staging capacity (>= max_block_count + 16)
     uint32_t lut_entries;  // lookup-table entries reserved in shared memory
+    uint32_t warps;        // per-warp kernel: warps per CTA (fewer than kWarpsPerCta for large chunks)
     uint32_t *status;
 };
 
@@ -562,20 +563,22 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
 // CTA's 18 warps share the lookup tables (rebuilt, with CTA barriers, only
 // where the CTA's run of blocks crosses into the next tensor); each warp has
 // its own segment buffer, gap bytes, staging area and mbarrier, and walks the
-// blocks w, w + 18, w + 36, ... of the current tensor.
+// blocks w, w + 18, w + 36, ... of the current tensor (fewer warps per CTA,
+// and a shorter stride, when long chunks make a warp's buffers too large for
+// 18 of them).
 constexpr uint32_t kWarpsPerCta = 18;   // 2 CTAs (36 warps) per SM fit registers and shared memory
 constexpr int kWarpCtasPerSm = 2;
 constexpr int kWarpMergeRegs = 3;       // 16-weight merge groups per lane whose loads are issued early
 
 struct WarpLayout {
     uint32_t warp0, seg_bytes, stage, warp_bytes, bars, total;
-    __host__ __device__ WarpLayout(uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes) {
+    __host__ __device__ WarpLayout(uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes, uint32_t warps) {
         warp0 = kFastBytes + ((2 * lut_entries + 15) & ~15u);
         seg_bytes = 4 * seg_words;
         stage = seg_bytes + 48;   // the block's 32 gap bytes, then the next block's first 16
         warp_bytes = stage + stage_bytes;
-        bars = warp0 + kWarpsPerCta * warp_bytes;
-        total = bars + 8 * kWarpsPerCta;
+        bars = warp0 + warps * warp_bytes;
+        total = bars + 8 * warps;
     }
 };
 
@@ -591,11 +594,242 @@ __device__ __forceinline__ void issue_warp_item(const Df11Batch &B, const Df11Te
     dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
 }
 
-template <int E>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
+// ---- fused linear layer ---------------------------------------------------------------
+//
+// y[m, r] = sum_c W[r, c] x[m, c] for M <= 8 activation rows: the weights a
+// warp decodes into its staging area are dotted with the activations instead
+// of being stored. W is rows x cols row-major, so a block's weights [o0, o1)
+// end one row, span whole rows and start another. The block's weights are
+// taken in rounds, in order (the single weights before its first 16-weight
+// group, rounds of 32 groups, the single weights after its last group); each
+// lane forms its part of a round as one FMA chain per activation row and adds
+// it to its running sum for the open row; when a round reaches the next row,
+// the finished row's lane sums are summed across the warp and added to y with
+// one atomic add per activation row. Summation tree height per output: at
+// most 16 (chain) + ceil(cols / 512) + 4 (running sum) + 5 (warp) + the number
+// of blocks sharing the row (a block of 32 chunks of at least 8 bytes holds at
+// least 63 codes of at most 32 bits), within ceil(cols / 512) + ceil(cols /
+// 32) + 32. Rows whose length is not a multiple of 16 take one atomic add
+// per weight (height cols).
+
+constexpr int kMaxLinBatch = 16;
+constexpr int kMaxRows = 8;
+constexpr uint32_t kNoRow = 0xFFFFFFFFu;
+
+struct Df11Lin {
+    const uint16_t *x[kMaxLinBatch];   // M x cols BF16, row-major
+    float *y[kMaxLinBatch];            // M x rows FP32, row-major, zeroed before the launch
+    uint64_t rows[kMaxLinBatch];
+    uint32_t cols[kMaxLinBatch];
+    uint32_t magic[kMaxLinBatch];      // division by cols, see div_cols
+    uint32_t shifts[kMaxLinBatch];     // sh1 | sh2 << 8
+    uint32_t M;
+};
+
+// n / cols for any 32-bit n, with m' and the shifts precomputed on the host
+// (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994, section 4, unsigned division: t = MULUH(m', n),
+// q = SRL(t + SRL(n - t, sh1), sh2)).
+__device__ __forceinline__ uint32_t div_cols(uint32_t n, uint32_t magic, uint32_t shifts) {
+    const uint32_t t = __umulhi(magic, n);
+    return (t + ((n - t) >> (shifts & 0xFFu))) >> (shifts >> 8);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
+
+// Warp sums of c[m]; lane 0 adds them to y[m, row].
+template <int MM>
+__device__ __forceinline__ void lin_flush(const float (&c)[MM], uint32_t M, float *y, uint64_t rows,
+                                          uint64_t row, uint32_t lane) {
+#pragma unroll
+    for (int m = 0; m < MM; m++) {
+        if ((uint32_t)m < M) {
+            float v = c[m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            if (lane == 0) atomicAdd(y + (uint64_t)m * rows + row, v);
+        }
+    }
+}
+
+// One round: each valid lane brings p[m] for row offset lr; the round's
+// weights lie in rows rf .. rl (warp-uniform, rf at or after the open row
+// cur). Rows before rl are flushed; acc becomes rl's lane sums.
+template <int MM>
+__device__ __forceinline__ void lin_round(float (&acc)[MM], uint32_t &cur, const float (&p)[MM],
+                                          bool valid, uint32_t lr, uint32_t rf, uint32_t rl, uint32_t M, float *y,
+                                          uint64_t rows, uint64_t row_base, uint32_t lane) {
+    if (rf == rl && rl == cur) {
+#pragma unroll
+        for (int m = 0; m < MM; m++) acc[m] += valid ? p[m] : 0.f;
+        return;
+    }
+    for (uint32_t rr = cur == kNoRow ? rf : cur; rr <= rl; rr++) {
+        float c[MM];
+#pragma unroll
+        for (int m = 0; m < MM; m++) c[m] = (valid && lr == rr ? p[m] : 0.f) + (rr == cur ? acc[m] : 0.f);
+        if (rr < rl) {
+            lin_flush<MM>(c, M, y, rows, row_base + rr, lane);
+        } else {
+#pragma unroll
+            for (int m = 0; m < MM; m++) acc[m] = c[m];
+        }
+    }
+    cur = rl;
+}
+
+// The linear layer's part of one decoded block [o0, o1) (exponents staged at
+// stage[i - (o0 & ~15)], sign|mantissa bytes of the first groups in sv).
+template <int MM>
+__device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const Df11Tensor &tn, const uint8_t *stage,
+                                          const uint4 (&sv)[kWarpMergeRegs], uint64_t o0, uint64_t o1,
+                                          uint64_t g_lo, uint64_t g_hi, uint32_t lane) {
+    const uint32_t cols = X.cols[ti], M = X.M, magic = X.magic[ti], shifts = X.shifts[ti];
+    const uint64_t rows = X.rows[ti];
+    const uint16_t *x = X.x[ti];
+    float *y = X.y[ti];
+    const uint64_t base = o0 & ~15ull;
+    const uint64_t row_base = base / cols;
+    const uint32_t d0 = (uint32_t)(base - row_base * cols);   // column of `base`; offsets below are from base
+    const uint8_t *sb = tn.sm + base;
+
+    if (cols & 15u) {
+        // rows not made of whole 16-weight groups: one atomic add per weight
+        for (uint64_t i = o0 + lane; i < o1; i += 32) {
+            const uint32_t r = (uint32_t)(i - base), d = d0 + r;
+            const uint32_t lr = div_cols(d, magic, shifts), col = d - lr * cols;
+            const float w = bf16_lo(merge1(sb[r], stage[r]));
+            for (uint32_t m = 0; m < M; m++)
+                atomicAdd(y + (uint64_t)m * rows + row_base + lr, w * bf16_lo(x[(uint64_t)m * cols + col]));
+        }
+        return;
+    }
+
+    float acc[MM], p[MM];
+#pragma unroll
+    for (int m = 0; m < MM; m++) acc[m] = 0.f;
+    uint32_t cur = kNoRow;
+
+    // single weights at block-relative offset r (valid lanes); the round spans [first, last]
+    auto single = [&](uint32_t r, bool valid, uint32_t first, uint32_t last) {
+        const uint32_t d = d0 + r;
+        const uint32_t lr = div_cols(d, magic, shifts);
+#pragma unroll
+        for (int m = 0; m < MM; m++) p[m] = 0.f;
+        if (valid) {
+            const float w = bf16_lo(merge1(sb[r], stage[r]));
+            const uint16_t *xc = x + (d - lr * cols);
+#pragma unroll
+            for (int m = 0; m < MM; m++)
+                if ((uint32_t)m < M) p[m] = w * bf16_lo(xc[(uint64_t)m * cols]);
+        }
+        lin_round<MM>(acc, cur, p, valid, lr, div_cols(d0 + first, magic, shifts), div_cols(d0 + last, magic, shifts), M,
+                  y, rows, row_base, lane);
+    };
+    // a round of 32 groups starting at block-relative rb; this lane's group at rb + 16 lane
+    const uint32_t rhi = (uint32_t)(g_hi - base);
+    auto groups = [&](uint32_t rb, const uint4 &s, bool valid) {
+        const uint32_t r = rb + 16u * lane, d = d0 + r;
+        const uint32_t lr = div_cols(d, magic, shifts);
+#pragma unroll
+        for (int m = 0; m < MM; m++) p[m] = 0.f;
+        if (valid) {
+            const uint4 e = *reinterpret_cast<const uint4 *>(stage + r);
+            uint32_t wv[8];
+            merge4(s.x, e.x, wv[0], wv[1]);
+            merge4(s.y, e.y, wv[2], wv[3]);
+            merge4(s.z, e.z, wv[4], wv[5]);
+            merge4(s.w, e.w, wv[6], wv[7]);
+            const uint4 *xc = reinterpret_cast<const uint4 *>(x + (d - lr * cols));   // 16 columns, 32-byte aligned
+#pragma unroll
+            for (int m = 0; m < MM; m++) {
+                if ((uint32_t)m < M) {
+                    const uint4 a = __ldg(xc + (uint64_t)m * (cols / 8)), b = __ldg(xc + (uint64_t)m * (cols / 8) + 1);
+                    const uint32_t xa[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    float t = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) {
+                        t = fmaf(bf16_lo(wv[j]), bf16_lo(xa[j]), t);
+                        t = fmaf(bf16_hi(wv[j]), bf16_hi(xa[j]), t);
+                    }
+                    p[m] = t;
+                }
+            }
+        }
+        const uint32_t last = min(rhi, rb + 512u) - 16u;   // the round's last group (groups never straddle rows)
+        lin_round<MM>(acc, cur, p, valid, lr, div_cols(d0 + rb, magic, shifts), div_cols(d0 + last, magic, shifts), M,
+                  y, rows, row_base, lane);
+    };
+
+    // weights before the first group, on lanes 0..15
+    const uint64_t hend = min(g_lo, o1);
+    if (hend > o0) {
+        const bool valid = lane < 16 && o0 + lane < hend;
+        single((uint32_t)(o0 - base) + (valid ? lane : 0u), valid, (uint32_t)(o0 - base), (uint32_t)(hend - 1 - base));
+    }
+    // whole groups
+    const uint32_t rlo = (uint32_t)(g_lo - base);
+#pragma unroll
+    for (int m = 0; m < kWarpMergeRegs; m++) {
+        const uint32_t rb = rlo + 512u * m;
+        if (rb < rhi) groups(rb, sv[m], rb + 16u * lane < rhi);
+    }
+    for (uint32_t rb = rlo + 512u * kWarpMergeRegs; rb < rhi; rb += 512u) {
+        const bool valid = rb + 16u * lane < rhi;
+        groups(rb, valid ? __ldg(reinterpret_cast<const uint4 *>(sb + rb + 16u * lane)) : make_uint4(0, 0, 0, 0), valid);
+    }
+    // weights after the last group, on lanes 16..31
+    const uint64_t tb = max(g_hi, g_lo);
+    if (o1 > tb) {
+        const bool valid = lane >= 16 && tb + (lane - 16) < o1;
+        single((uint32_t)(tb - base) + (valid ? lane - 16 : 0u), valid, (uint32_t)(tb - base), (uint32_t)(o1 - 1 - base));
+    }
+    if (cur != kNoRow) lin_flush<MM>(acc, M, y, rows, row_base + cur, lane);
+}
+
+// Single-exponent tensors: one warp per row, lane-strided columns.
+__global__ void df11_linear_const_kernel(const uint8_t *__restrict__ sm, uint32_t const_exp,
+                                         const uint16_t *__restrict__ x, uint32_t M, uint64_t rows, uint32_t cols,
+                                         float *__restrict__ y) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint64_t warps = (uint64_t)gridDim.x * (blockDim.x / 32);
+    for (uint64_t r = blockIdx.x * (uint64_t)(blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += warps) {
+        float acc[kMaxRows];
+#pragma unroll
+        for (int m = 0; m < kMaxRows; m++) acc[m] = 0.f;
+        for (uint32_t c = lane; c < cols; c += 32u) {
+            const float w = bf16_lo(merge1(sm[r * cols + c], const_exp));
+#pragma unroll
+            for (int m = 0; m < kMaxRows; m++)
+                if ((uint32_t)m < M) acc[m] = fmaf(w, bf16_lo(x[(uint64_t)m * cols + c]), acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < kMaxRows; m++) {
+            if ((uint32_t)m < M) {
+                float v = acc[m];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+                if (lane == 0) y[(uint64_t)m * rows + r] = v;
+            }
+        }
+    }
+}
+
+__global__ void zero_f32_kernel(float *__restrict__ y, uint64_t n) {
+    for (uint64_t i = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; i < n; i += (uint64_t)gridDim.x * blockDim.x)
+        y[i] = 0.f;
+}
+
+// The per-warp decoder's body. LIN = false: store the weights (decoder).
+// LIN = true: dot them with the activations instead (fused linear layer, BF16
+// elements only).
+template <int E, int LIN>   // LIN: 0 = decoder, else the linear layer for up to LIN activation rows
+__device__ __forceinline__ void df11_warp_body(const Df11Batch &B, const Df11Lin *X) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
-    const WarpLayout L(B.seg_words, B.lut_entries, B.stage_bytes);
+    const uint32_t NW = B.warps;   // warps per CTA
+    const WarpLayout L(B.seg_words, B.lut_entries, B.stage_bytes, NW);
     uint32_t *sym_tab = reinterpret_cast<uint32_t *>(smem);
     uint16_t *mask_tab = reinterpret_cast<uint16_t *>(smem + kFastSize * 4);
     uint8_t *cnt_tab = smem + kFastSize * 6;
@@ -644,13 +878,13 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
             o0n = tn.blkoff[w - tn.first_work];
             o1n = tn.blkoff[w - tn.first_work + 1];
         }
-        for (; w < s_end && !dead; w += kWarpsPerCta) {
+        for (; w < s_end && !dead; w += NW) {
             const uint32_t b = w - tn.first_work;
             const uint64_t o0 = o0n, o1 = o1n;
-            const bool more = w + kWarpsPerCta < s_end;
+            const bool more = w + NW < s_end;
             if (more) {
-                o0n = tn.blkoff[b + kWarpsPerCta];
-                o1n = tn.blkoff[b + kWarpsPerCta + 1];
+                o0n = tn.blkoff[b + NW];
+                o1n = tn.blkoff[b + NW + 1];
             }
             const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
             const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
@@ -783,32 +1017,36 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
                     // the segment is free: fetch this warp's next block while merging this one
                     if (lane == 0 && more) {
                         dev::fence_proxy_async_smem();
-                        issue_warp_item(B, tn, b + kWarpsPerCta, buf, seg_bytes, bar);
+                        issue_warp_item(B, tn, b + NW, buf, seg_bytes, bar);
                     }
                     next_issued = true;
 
-                    // 32-bit offsets from the block's first 16-weight group
-                    const uint64_t base = o0 & ~15ull;
-                    const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
-                    // typed output and low-mantissa pointers at the block's first group
-                    void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
-                                                  : static_cast<void *>(tn.out + base);
-                    const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
-                    const uint64_t g0 = base / 16;   // first group, for the FP16 tails
-                    const uint8_t *sb = tn.sm + base;
-#pragma unroll
-                    for (int m = 0; m < kWarpMergeRegs; m++) {
-                        const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
-                        if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                    if constexpr (LIN) {
+                        lin_block<LIN>(*X, ti, tn, stage, sv, o0, o1, g_lo, g_hi, lane);
+                    } else {
+                        // 32-bit offsets from the block's first 16-weight group
+                        const uint64_t base = o0 & ~15ull;
+                        const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
+                        // typed output and low-mantissa pointers at the block's first group
+                        void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
+                                                      : static_cast<void *>(tn.out + base);
+                        const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
+                        const uint64_t g0 = base / 16;   // first group, for the FP16 tails
+                        const uint8_t *sb = tn.sm + base;
+    #pragma unroll
+                        for (int m = 0; m < kWarpMergeRegs; m++) {
+                            const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
+                            if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                        }
+                        for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
+                            merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
+                                           *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                        // partial 16-groups at both ends
+                        const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
+                        const bool head = lane < 16 && i < min(g_lo, o1);
+                        const bool tail = lane >= 16 && i < o1;
+                        if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
                     }
-                    for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
-                        merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
-                                       *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
-                    // partial 16-groups at both ends
-                    const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
-                    const bool head = lane < 16 && i < min(g_lo, o1);
-                    const bool tail = lane >= 16 && i < o1;
-                    if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
                 } else {
                     bad |= LWC_DEVICE_BAD_COUNT;
                 }
@@ -818,7 +1056,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
             __syncwarp();   // segment and staging area free again
             if (lane == 0 && !next_issued && more) {
                 dev::fence_proxy_async_smem();
-                issue_warp_item(B, tn, b + kWarpsPerCta, buf, seg_bytes, bar);
+                issue_warp_item(B, tn, b + NW, buf, seg_bytes, bar);
             }
         }
         w0 = s_end;
@@ -826,6 +1064,25 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
     }
     if (bad && B.status) atomicOr(B.status, bad);
 }
+
+template <int E>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_kernel(const __grid_constant__ Df11Batch B) {
+    df11_warp_body<E, 0>(B, nullptr);
+}
+
+// Fused decode + linear layer (BF16 elements, blocks of 32 chunks) for up
+// to MM activation rows; with more than one row the accumulators need more
+// registers than two CTAs per SM leave.
+template <int MM>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, MM == 1 ? kWarpCtasPerSm : 1)
+    df11_warp_linear_kernel(const __grid_constant__ Df11Batch B, const __grid_constant__ Df11Lin X) {
+    df11_warp_body<LWC_ELEM_BF16, MM>(B, &X);
+}
+
+using LinKernel = void (*)(Df11Batch, Df11Lin);
+const LinKernel kLinKernels[4] = {df11_warp_linear_kernel<1>, df11_warp_linear_kernel<2>, df11_warp_linear_kernel<4>,
+                                  df11_warp_linear_kernel<8>};
+int lin_index(uint32_t M) { return M <= 1 ? 0 : M <= 2 ? 1 : M <= 4 ? 2 : 3; }
 
 // One exponent value for the whole tensor: out = merge(const_exp, sm).
 template <int E>
@@ -870,7 +1127,8 @@ lwc_status device_config(DeviceConfig &out) {
             (const void *)df11_decode_kernel<256, LWC_ELEM_FP32>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP32>,
             (const void *)df11_warp_kernel<LWC_ELEM_FP32>,
             (const void *)df11_decode_kernel<256, LWC_ELEM_FP16>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP16>,
-            (const void *)df11_warp_kernel<LWC_ELEM_FP16>};
+            (const void *)df11_warp_kernel<LWC_ELEM_FP16>, (const void *)kLinKernels[0], (const void *)kLinKernels[1],
+            (const void *)kLinKernels[2], (const void *)kLinKernels[3]};
         for (const void *k : kernels) {
             if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
             if (err == cudaSuccess)
@@ -908,6 +1166,14 @@ void launch_df11(bool per_warp, uint32_t T, unsigned grid, uint32_t threads, siz
         df11_decode_kernel<256, E><<<grid, T, smem, stream>>>(B);
     else
         df11_decode_kernel<1024, E><<<grid, T, smem, stream>>>(B);
+}
+
+// Warps per CTA of the per-warp kernel: kWarpsPerCta, or fewer when one
+// warp's segment buffer and staging area are large (long chunks).
+uint32_t warps_that_fit(const Df11Batch &B, int max_smem) {
+    uint32_t w = kWarpsPerCta;
+    while (w > 1 && WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total > (uint64_t)max_smem) w--;
+    return w;
 }
 
 // Launch one kernel over up to kMaxBatch tensors sharing (element type, chunk_bytes, threads_per_block).
@@ -949,8 +1215,9 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
     const bool per_warp = T == 32;
-    const uint32_t threads = per_warp ? kWarpsPerCta * 32u : T;
-    const uint64_t smem = per_warp ? WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes).total
+    B.warps = per_warp ? warps_that_fit(B, cfg.max_smem) : 0;
+    const uint32_t threads = per_warp ? B.warps * 32u : T;
+    const uint64_t smem = per_warp ? WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, B.warps).total
                                    : Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
@@ -962,7 +1229,7 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
     if (per_sm < 1) return fail(LWC_ERR_UNSUPPORTED, "decoder does not fit on an SM (%u threads, %llu B smem)",
                                 threads, (unsigned long long)smem);
-    const uint64_t units = per_warp ? (work + kWarpsPerCta - 1) / kWarpsPerCta : work;
+    const uint64_t units = per_warp ? (work + B.warps - 1) / B.warps : work;
     const uint64_t grid = std::min<uint64_t>(units, (uint64_t)per_sm * cfg.sms);
     if (elem == LWC_ELEM_FP32)
         launch_df11<LWC_ELEM_FP32>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
@@ -972,6 +1239,79 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
         launch_df11<LWC_ELEM_BF16>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+    return LWC_OK;
+}
+
+// m' and the shifts of div_cols for divisor d (1 <= d < 2^31): l = ceil(log2 d),
+// m' = floor(2^32 (2^l - d) / d) + 1, sh1 = min(l, 1), sh2 = max(l - 1, 0).
+void division_magic(uint32_t d, uint32_t &magic, uint32_t &shifts) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) l++;
+    magic = (uint32_t)(((((uint64_t)1 << l) - d) << 32) / d + 1);
+    shifts = (l < 1 ? l : 1u) | ((l > 0 ? l - 1 : 0u) << 8);
+}
+
+// One fused-linear launch over up to kMaxLinBatch tensors sharing chunk_bytes
+// (BF16 elements, blocks of 32 chunks); their outputs are already zeroed.
+lwc_status launch_linear_group(const std::vector<int> &idx, const lwc_desc *descs, const void *const *d_blobs,
+                               const uint64_t *cols, const uint16_t *const *d_xs, uint32_t M, float *const *d_ys,
+                               uint32_t *d_status, cudaStream_t stream, const DeviceConfig &cfg) {
+    Df11Batch B;
+    Df11Lin X;
+    std::memset(&B, 0, sizeof B);
+    std::memset(&X, 0, sizeof X);
+    const lwc_desc &d0 = descs[idx[0]];
+    B.chunk_words = d0.chunk_bytes / 4;
+    B.seg_words = (uint32_t)round_up((uint64_t)32 * B.chunk_words + 2, 4);
+    uint64_t work = 0, max_count = 0, max_tables = 0;
+    for (size_t j = 0; j < idx.size(); j++) {
+        const int i = idx[j];
+        const lwc_desc &d = descs[i];
+        const uint8_t *base = static_cast<const uint8_t *>(d_blobs[i]);
+        Df11Tensor &t = B.t[j];
+        t.stream = reinterpret_cast<const uint32_t *>(base + d.off_stream);
+        t.gaps = base + d.off_gaps;
+        t.blkoff = reinterpret_cast<const uint64_t *>(base + d.off_blkoff);
+        t.sm = base + d.off_sm;
+        t.lut = reinterpret_cast<const uint16_t *>(base + d.off_lut);
+        t.n = d.n;
+        t.total_bits = d.total_bits;
+        t.stream_bytes = d.stream_bytes;
+        t.n_blocks = (uint32_t)d.n_blocks;
+        t.n_tables = d.n_tables;
+        t.first_work = (uint32_t)work;
+        work += d.n_blocks;
+        max_count = std::max<uint64_t>(max_count, d.max_block_count);
+        max_tables = std::max<uint64_t>(max_tables, d.n_tables);
+        X.x[j] = d_xs[i];
+        X.y[j] = d_ys[i];
+        X.cols[j] = (uint32_t)cols[i];
+        X.rows[j] = d.n / cols[i];
+        division_magic(X.cols[j], X.magic[j], X.shifts[j]);
+    }
+    if (work > 0xFFFFFFFFull) return fail(LWC_ERR_UNSUPPORTED, "too many blocks in one launch");
+    B.count = (uint32_t)idx.size();
+    B.total_work = (uint32_t)work;
+    B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
+    B.lut_entries = (uint32_t)(max_tables * 256);
+    B.status = d_status;
+    X.M = M;
+    B.warps = warps_that_fit(B, cfg.max_smem);
+    const uint32_t threads = B.warps * 32u;
+    const uint64_t smem = WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, B.warps).total;
+    if (smem > (uint64_t)cfg.max_smem)
+        return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
+                    (unsigned long long)smem, cfg.max_smem);
+    const LinKernel kernel = kLinKernels[lin_index(M)];
+    int per_sm = 0;
+    cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void *)kernel, (int)threads,
+                                                                    (size_t)smem);
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
+    if (per_sm < 1) return fail(LWC_ERR_UNSUPPORTED, "linear kernel does not fit on an SM");
+    const uint64_t grid = std::min<uint64_t>((work + B.warps - 1) / B.warps, (uint64_t)per_sm * cfg.sms);
+    kernel<<<(unsigned)grid, threads, (size_t)smem, stream>>>(B, X);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));
     return LWC_OK;
 }
 
@@ -1060,6 +1400,81 @@ lwc_status lwc_decode_dfloat11_checked(const lwc_desc *desc, const void *d_in, u
 
 lwc_status lwc_decode_dfloat11(const lwc_desc *desc, const void *d_in, uint16_t *d_out, lwc_stream_t stream) {
     return lwc_decode_dfloat11_checked(desc, d_in, d_out, nullptr, stream);
+}
+
+lwc_status lwc_linear_dfloat11_batched(const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
+                                       const uint16_t *const *d_xs, int M, float *const *d_ys, int count,
+                                       uint32_t *d_status, lwc_stream_t stream) {
+    if (count < 0 || (count > 0 && (!descs || !d_blobs || !cols || !d_xs || !d_ys)))
+        return fail(LWC_ERR_INVALID_ARG, "bad batch arguments");
+    if (M < 1 || M > kMaxRows) return fail(LWC_ERR_INVALID_ARG, "M must be 1..%d (got %d)", kMaxRows, M);
+    bool any = false;
+    for (int i = 0; i < count; i++) {
+        const lwc_desc &d = descs[i];
+        lwc_status st = check_df11_desc(&d);
+        if (st) return st;
+        if (cols[i] == 0 || cols[i] >= (1ull << 31) || d.n % cols[i] != 0)
+            return fail(LWC_ERR_INVALID_ARG, "cols must be 1..2^31-1 and divide n (tensor %d)", i);
+        if (d.n == 0) continue;
+        any = true;
+        if (d.elem != LWC_ELEM_BF16)
+            return fail(LWC_ERR_UNSUPPORTED, "the fused linear layer takes BF16 weights (tensor %d)", i);
+        if (!(d.flags & kFlagSingleExponent) && d.threads_per_block != 32)
+            return fail(LWC_ERR_UNSUPPORTED, "the fused linear layer needs blocks of 32 chunks (tensor %d has %u)", i,
+                        d.threads_per_block);
+        if (!d_blobs[i] || !d_xs[i] || !d_ys[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (tensor %d)", i);
+        if (!aligned16(d_blobs[i]) || !aligned16(d_xs[i]) || (reinterpret_cast<uintptr_t>(d_ys[i]) & 3u))
+            return fail(LWC_ERR_MISALIGNED, "blob and x must be 16-byte aligned, y 4-byte aligned (tensor %d)", i);
+    }
+    if (d_status && (reinterpret_cast<uintptr_t>(d_status) & 3u))
+        return fail(LWC_ERR_MISALIGNED, "status word must be 4-byte aligned");
+    if (!any) {
+        clear_error();
+        return LWC_OK;
+    }
+    DeviceConfig cfg;
+    lwc_status st = device_config(cfg);
+    if (st) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<std::pair<uint64_t, int>> keyed;
+    for (int i = 0; i < count; i++) {
+        const lwc_desc &d = descs[i];
+        if (d.n == 0) continue;
+        const uint64_t rows = d.n / cols[i];
+        if (d.flags & kFlagSingleExponent) {
+            const uint64_t blocks = std::min<uint64_t>((rows + 7) / 8, (uint64_t)cfg.sms * 8);
+            df11_linear_const_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+                static_cast<const uint8_t *>(d_blobs[i]) + d.off_sm, d.const_exp, d_xs[i], (uint32_t)M, rows,
+                (uint32_t)cols[i], d_ys[i]);
+        } else {
+            const uint64_t ny = rows * (uint64_t)M;
+            const uint64_t blocks = std::min<uint64_t>((ny + 255) / 256, (uint64_t)cfg.sms * 8);
+            zero_f32_kernel<<<(unsigned)blocks, 256, 0, s>>>(d_ys[i], ny);
+            keyed.push_back({d.chunk_bytes, i});
+        }
+        cudaError_t err = cudaGetLastError();
+        if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));
+    }
+    std::stable_sort(keyed.begin(), keyed.end(),
+                     [](const std::pair<uint64_t, int> &a, const std::pair<uint64_t, int> &b) { return a.first < b.first; });
+    std::vector<int> group;
+    for (size_t i = 0; i < keyed.size(); i++) {
+        group.push_back(keyed[i].second);
+        const bool last = i + 1 == keyed.size() || keyed[i + 1].first != keyed[i].first;
+        if (last || group.size() == (size_t)kMaxLinBatch) {
+            st = launch_linear_group(group, descs, d_blobs, cols, d_xs, (uint32_t)M, d_ys, d_status, s, cfg);
+            if (st) return st;
+            group.clear();
+        }
+    }
+    clear_error();
+    return LWC_OK;
+}
+
+lwc_status lwc_linear_dfloat11(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x, int M,
+                               float *d_y, uint32_t *d_status, lwc_stream_t stream) {
+    if (!desc) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    return lwc_linear_dfloat11_batched(desc, &d_blob, &cols, &d_x, M, &d_y, 1, d_status, stream);
 }
 
 }  // extern "C"

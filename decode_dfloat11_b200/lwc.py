@@ -37,8 +37,9 @@ EXPORTED = (
     "lwc_decode_codebook_checked", "lwc_decode_dfloat11_batched", "lwc_decode_codebook_batched",
     "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan",
     "lwc_encode_dfloat11_elements_device_plan", "lwc_encode_codebook_device_plan",
-    "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_status_string", "lwc_last_error",
-    "lwc_version",
+    "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_linear_codebook",
+    "lwc_linear_codebook_batched", "lwc_linear_dfloat11", "lwc_linear_dfloat11_batched", "lwc_status_string",
+    "lwc_last_error", "lwc_version",
 )
 
 
@@ -114,6 +115,13 @@ def load():
                                                            _P, _u64, D, _P]
     L.lwc_encode_device_write.argtypes = [_P, _u64, _P, _u64, _P, _u64, D, _P]
     L.lwc_encode_dfloat11_device_noalloc.argtypes = [_P, _u64, ctypes.POINTER(lwc_df11_params), _P, _u64, D, _P]
+    for name in ("lwc_linear_codebook", "lwc_linear_dfloat11"):
+        getattr(L, name).argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
+        getattr(L, name).restype = ctypes.c_int
+    for name in ("lwc_linear_codebook_batched", "lwc_linear_dfloat11_batched"):
+        getattr(L, name).argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_u64), ctypes.POINTER(_P), ctypes.c_int,
+                                     ctypes.POINTER(_P), ctypes.c_int, _P, _P]
+        getattr(L, name).restype = ctypes.c_int
     L.lwc_status_string.argtypes = [ctypes.c_int]
     L.lwc_status_string.restype = ctypes.c_char_p
     L.lwc_last_error.argtypes = []
@@ -255,6 +263,47 @@ def lwc_decode_codebook_batched(descs, d_ins=None, d_outs=None, d_status=None, s
     """Decode several codebook tensors at once (one launch per index width)."""
     b = descs if isinstance(descs, Batch) else Batch(descs, d_ins, d_outs)
     _check(load().lwc_decode_codebook_batched(b.descs, b.ins, b.outs, b.count, _addr(d_status), _stream(stream)))
+
+
+def lwc_linear_codebook(desc: lwc_desc, d_blob, cols: int, d_x, M: int, d_y, d_status=None, stream=None) -> None:
+    """y = x W^T with W (n / cols x cols) decoded from a codebook blob in registers;
+    x: M x cols BF16 (device), y: M x rows FP32 (device)."""
+    _check(load().lwc_linear_codebook(ctypes.byref(desc), _addr(d_blob), cols, _addr(d_x), M, _addr(d_y),
+                                      _addr(d_status), _stream(stream)))
+
+
+def lwc_linear_dfloat11(desc: lwc_desc, d_blob, cols: int, d_x, M: int, d_y, d_status=None, stream=None) -> None:
+    """As lwc_linear_codebook, for a DFloat11 blob of BF16 elements."""
+    _check(load().lwc_linear_dfloat11(ctypes.byref(desc), _addr(d_blob), cols, _addr(d_x), M, _addr(d_y),
+                                      _addr(d_status), _stream(stream)))
+
+
+class LinearBatch:
+    """Marshalled arguments of lwc_linear_*_batched, reusable across calls."""
+
+    def __init__(self, descs, d_blobs, cols, d_xs, d_ys, M: int):
+        n = len(descs)
+        if not (len(d_blobs) == len(cols) == len(d_xs) == len(d_ys) == n):
+            raise ValueError("argument lists differ in length")
+        self.count = n
+        self.M = M
+        self.descs = (lwc_desc * max(1, n))(*descs)
+        self.blobs = (_P * max(1, n))(*[_addr(x) for x in d_blobs])
+        self.cols = (_u64 * max(1, n))(*cols)
+        self.xs = (_P * max(1, n))(*[_addr(x) for x in d_xs])
+        self.ys = (_P * max(1, n))(*[_addr(x) for x in d_ys])
+
+
+def lwc_linear_codebook_batched(batch: LinearBatch, d_status=None, stream=None) -> None:
+    b = batch
+    _check(load().lwc_linear_codebook_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
+                                              _stream(stream)))
+
+
+def lwc_linear_dfloat11_batched(batch: LinearBatch, d_status=None, stream=None) -> None:
+    b = batch
+    _check(load().lwc_linear_dfloat11_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
+                                              _stream(stream)))
 
 
 def lwc_encode_device_workspace_bytes(n: int) -> int:

@@ -223,6 +223,59 @@ LWC_API lwc_status lwc_decode_codebook_batched(const lwc_desc *descs, const void
                                                uint16_t *const *d_outs, int count, uint32_t *d_status,
                                                lwc_stream_t stream);
 
+/* ---- decode fused into the linear layer that consumes the weights --------- */
+
+/* y = x W^T without writing W out: the decoded weights stay in registers.
+ * The DF11 page ("Koniec z kompromisami! DFloat11 ratuje dokładność modeli
+ * AI ...", section "Jak to działa w praktyce? Magia na poziomie GPU") has the
+ * weights decompressed on the GPU during inference for the model's use, and
+ * measures token-generation throughput (section "Realne korzyści, które
+ * zmieniają zasady gry"); token generation runs the linear layers on a few
+ * activation rows, where the product is bound by reading the weights.
+ *
+ *   y[m * rows + r] = sum over c < cols of W[r * cols + c] * x[m * cols + c]
+ *
+ * for m < M, r < rows = n / cols, W the n weights the blob decodes to (BF16),
+ * read as rows x cols row-major (out_features x in_features).
+ *   - d_blob: the blob in device memory, 16-byte aligned (not modified).
+ *   - cols: 1 .. 2^31 - 1, and n must be a multiple of it.
+ *   - d_x: M x cols BF16 activations, row-major, 16-byte aligned (not modified).
+ *   - M: 1 .. 8.
+ *   - d_y: M x rows FP32 outputs, 4-byte aligned; every output is written
+ *     (overwritten, not accumulated into). The caller owns all buffers.
+ *   - d_status: optional, as for the checked decoders.
+ * Products of two BF16 values are exact in FP32; the sums are FP32, and
+ * every output is a summation tree of height at most h, so that
+ * |y - exact| <= gamma_h * sum |W x|, gamma_h = h u / (1 - h u), u = 2^-24:
+ *   codebook: h = ceil(cols / 1024) + 37 (ceil(cols / 32) + 5 for a
+ *     one-entry table); the result does not depend on the launch shape;
+ *   DFloat11: h = ceil(cols / 512) + ceil(cols / 32) + 32 when cols is a
+ *     multiple of 16, else h = cols; blocks that share an output row add
+ *     their parts atomically, so the last bits may vary from run to run.
+ * Errors as for the decoders (LWC_ERR_INVALID_ARG for a bad M or cols). */
+LWC_API lwc_status lwc_linear_codebook(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x,
+                                       int M, float *d_y, uint32_t *d_status, lwc_stream_t stream);
+
+/* `count` codebook tensors, each with its own cols[i], activations d_xs[i]
+ * and outputs d_ys[i] (all with the same M), in one launch per index width. */
+LWC_API lwc_status lwc_linear_codebook_batched(const lwc_desc *descs, const void *const *d_blobs,
+                                               const uint64_t *cols, const uint16_t *const *d_xs, int M,
+                                               float *const *d_ys, int count, uint32_t *d_status,
+                                               lwc_stream_t stream);
+
+/* As lwc_linear_codebook, for a DFloat11 blob of BF16 elements whose blocks
+ * hold 32 chunks (threads_per_block = 32, the encoder's default), or with a
+ * single exponent value; other blobs give LWC_ERR_UNSUPPORTED (re-encode). */
+LWC_API lwc_status lwc_linear_dfloat11(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x,
+                                       int M, float *d_y, uint32_t *d_status, lwc_stream_t stream);
+
+/* `count` DFloat11 tensors as lwc_linear_codebook_batched, in one launch per
+ * distinct chunk_bytes (at most 16 tensors each), after zeroing the outputs. */
+LWC_API lwc_status lwc_linear_dfloat11_batched(const lwc_desc *descs, const void *const *d_blobs,
+                                               const uint64_t *cols, const uint16_t *const *d_xs, int M,
+                                               float *const *d_ys, int count, uint32_t *d_status,
+                                               lwc_stream_t stream);
+
 /* ---- device encoders ------------------------------------------------------ */
 
 /* Compression of a tensor that is already in GPU memory, into a blob in GPU

@@ -102,6 +102,12 @@ def normal_fp16(shape, seed: int, sigma: float, outlier_frac: float = 0.0, outli
     return x.to(torch.float16)
 
 
+def activations_bf16(M: int, cols: int, seed: int, device="cpu") -> torch.Tensor:
+    """M activation rows of width cols for a linear layer: i.i.d. N(0, 1) with
+    0.1 % outliers x20 (the scale of normalised hidden states), BF16."""
+    return normal_bf16((M, cols), seed, sigma=1.0, outlier_frac=1e-3, outlier_scale=20.0, device=device)
+
+
 def small_square(seed: int = 0, device="cpu") -> torch.Tensor:
     """1024 x 1024 weights, i.i.d. N(0, 0.02), BF16."""
     return normal_bf16((1024, 1024), seed, sigma=0.02, device=device)

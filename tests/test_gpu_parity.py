@@ -70,7 +70,7 @@ def test_df11_small(name, w):
 
 
 @pytest.mark.parametrize("chunk_bytes,tpb", [(8, 32), (12, 64), (20, 96), (36, 256), (64, 128), (36, 512),
-                                             (36, 1024)])
+                                             (36, 1024), (100, 32), (512, 32), (1024, 32)])
 def test_df11_block_parameters(chunk_bytes, tpb):
     w = synth.as_u16(synth.normal_bf16((1_234_567,), seed=4, sigma=0.02, outlier_frac=1e-3))
     d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
