@@ -54,6 +54,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-encode", action="store_true", help="skip the device-encoder timing")
     ap.add_argument("--no-elements", action="store_true", help="skip the FP32/FP16 DFloat11 decodes")
     ap.add_argument("--no-codebook", action="store_true")
+    ap.add_argument("--no-linear", action="store_true", help="skip the decode-fused linear layer timing")
     ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
     ap.add_argument("--workload", choices=("layer", "model8b", "model70b", "stress"), default="layer",
                     help="layer: one Llama-3-8B layer (default line); model8b / model70b: the whole "
@@ -366,6 +367,61 @@ def run_lwc(args, rank, world, local_rank, dist):
             "bits_per_weight": round(sd.bits_per_weight, 4),
             "hbm_frac": round((sb.size + 2 * ns) / (sms * 1e-3) / 1e9 / peak, 4)}
         del sbd, sout
+
+    # decode fused into the linear layer (token generation: M activation rows):
+    # the layer's seven y = x W^T with the weights decoded in registers, one
+    # batched call per codec, against decode-then-matmul and the uncompressed
+    # BF16 matmul (torch), for context
+    if not args.no_linear:
+        from decode_dfloat11_b200.layers import encode_on_device
+        lin = {"workload": "llama3-8b-layer: 7 x (y = x W^T), batched call, weights decoded in registers",
+               "kernels": {"dfloat11": "df11_warp_linear_kernel", "codebook": "cb_linear_kernel"}}
+        src = [torch.from_numpy(w.view(np.int16)).to(device).view(torch.bfloat16).view(r, c)
+               for w, (_, r, c) in zip(tensors, synth.LLAMA3_8B_LAYER)]
+        for codec in ("dfloat11", "codebook"):
+            enc_l = [encode_on_device(t, codec) for t in src]
+            ld = [d for d, _ in enc_l]
+            lb = [b for _, b in enc_l]
+            lbytes = sum(b.numel() for b in lb)
+            fn = lwc.lwc_linear_dfloat11_batched if codec == "dfloat11" else lwc.lwc_linear_codebook_batched
+            dec = lwc.lwc_decode_dfloat11_batched if codec == "dfloat11" else lwc.lwc_decode_codebook_batched
+            dbatch = lwc.Batch(ld, lb, views)
+            for M in (1, 4):
+                xs = [synth.activations_bf16(M, t.shape[1], seed=500 + j, device=device) for j, t in enumerate(src)]
+                ys = [torch.empty((M, t.shape[0]), dtype=torch.float32, device=device) for t in src]
+                lbatch = lwc.LinearBatch(ld, lb, [t.shape[1] for t in src], xs, ys, M)
+                fn(lbatch, stream=stream)
+                torch.cuda.synchronize(device)
+                for t, x, y in zip(src, xs, ys):   # consistency with torch on the same weights
+                    ref = x.float() @ t.float().T
+                    if not torch.allclose(y, ref, rtol=1e-3, atol=1e-3 * float(ref.abs().max())):
+                        raise SystemExit(f"fused {codec} linear layer disagrees with torch")
+                for _ in range(args.warmup):
+                    fn(lbatch, stream=stream)
+                fms = time_steps(lambda: fn(lbatch, stream=stream), args.steps, stream) / args.steps
+
+                def unfused():
+                    dec(dbatch, stream=stream)
+                    for x, v, t in zip(xs, views, src):
+                        torch.matmul(x, v.view(t.shape).T)
+                for _ in range(args.warmup):
+                    unfused()
+                ums = time_steps(unfused, args.steps, stream) / args.steps
+                dense = lambda: [torch.matmul(x, t.T) for x, t in zip(xs, src)]
+                for _ in range(args.warmup):
+                    dense()
+                bms = time_steps(dense, args.steps, stream) / args.steps
+                io = sum(2 * x.numel() + 4 * y.numel() for x, y in zip(xs, ys))
+                ach = (lbytes + io) / (fms * 1e-3) / 1e9
+                lin[f"{codec}_M{M}"] = {
+                    "fused_ms": round(fms, 5), "decode_then_matmul_ms": round(ums, 5),
+                    "bf16_matmul_ms": round(bms, 5), "speedup_vs_decode_then_matmul": round(ums / fms, 3),
+                    "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                                 "frac": round(ach / peak, 4), "algorithmic_bytes_per_call": lbytes + io}}
+                del xs, ys, lbatch
+            del enc_l, ld, lb, dbatch
+        result["linear"] = lin
+        del src
 
     # DFloat11 for the other float formats: a gate-shaped FP32 and FP16 matrix
     if not args.no_elements:
