@@ -327,6 +327,20 @@ __device__ __forceinline__ void issue_window(const CbLinTensor &tn, uint64_t r, 
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
+// acc + w.lo * x.lo, then + w.hi * x.hi: two FMAs on BF16 pairs with an FP32
+// accumulator (PTX mixed-precision fma.rn.f32.bf16: the product of two BF16
+// values is exact, one rounding per FMA, as with the FP32 FMA of the
+// converted values, minus the conversions).
+__device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) {
+    float d;
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t.reg .f32 t;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 t, wl, xl, %3;\n\tfma.rn.f32.bf16 %0, wh, xh, t;\n\t}"
+        : "=f"(d)
+        : "r"(w2), "r"(x2), "f"(acc));
+    return d;
+}
+
 // acc + dot(v, x[0..31]) as one FMA chain; v holds the 32 weights as BF16
 // pairs, x is 16-byte aligned.
 __device__ __forceinline__ float dot32(const uint32_t (&v)[16], const uint16_t *x, float acc) {
@@ -334,14 +348,10 @@ __device__ __forceinline__ float dot32(const uint32_t (&v)[16], const uint16_t *
 #pragma unroll
     for (int i = 0; i < 4; i++) {
         const uint4 q = __ldg(xp + i);
-        acc = fmaf(bf16_lo(v[4 * i + 0]), bf16_lo(q.x), acc);
-        acc = fmaf(bf16_hi(v[4 * i + 0]), bf16_hi(q.x), acc);
-        acc = fmaf(bf16_lo(v[4 * i + 1]), bf16_lo(q.y), acc);
-        acc = fmaf(bf16_hi(v[4 * i + 1]), bf16_hi(q.y), acc);
-        acc = fmaf(bf16_lo(v[4 * i + 2]), bf16_lo(q.z), acc);
-        acc = fmaf(bf16_hi(v[4 * i + 2]), bf16_hi(q.z), acc);
-        acc = fmaf(bf16_lo(v[4 * i + 3]), bf16_lo(q.w), acc);
-        acc = fmaf(bf16_hi(v[4 * i + 3]), bf16_hi(q.w), acc);
+        acc = fma2_bf16(v[4 * i + 0], q.x, acc);
+        acc = fma2_bf16(v[4 * i + 1], q.y, acc);
+        acc = fma2_bf16(v[4 * i + 2], q.z, acc);
+        acc = fma2_bf16(v[4 * i + 3], q.w, acc);
     }
     return acc;
 }

@@ -638,6 +638,20 @@ __device__ __forceinline__ uint32_t div_cols(uint32_t n, uint32_t magic, uint32_
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
+// acc + w.lo * x.lo, then + w.hi * x.hi: two FMAs on BF16 pairs with an FP32
+// accumulator (PTX mixed-precision fma.rn.f32.bf16: the product of two BF16
+// values is exact, one rounding per FMA, as with the FP32 FMA of the
+// converted values, minus the conversions).
+__device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) {
+    float d;
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t.reg .f32 t;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\tmov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 t, wl, xl, %3;\n\tfma.rn.f32.bf16 %0, wh, xh, t;\n\t}"
+        : "=f"(d)
+        : "r"(w2), "r"(x2), "f"(acc));
+    return d;
+}
+
 // Warp sums of c[m]; lane 0 adds them to y[m, row].
 template <int MM>
 __device__ __forceinline__ void lin_flush(const float (&c)[MM], uint32_t M, float *y, uint64_t rows,
@@ -749,10 +763,7 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
                     const uint32_t xa[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
                     float t = 0.f;
 #pragma unroll
-                    for (int j = 0; j < 8; j++) {
-                        t = fmaf(bf16_lo(wv[j]), bf16_lo(xa[j]), t);
-                        t = fmaf(bf16_hi(wv[j]), bf16_hi(xa[j]), t);
-                    }
+                    for (int j = 0; j < 8; j++) t = fma2_bf16(wv[j], xa[j], t);
                     p[m] = t;
                 }
             }
