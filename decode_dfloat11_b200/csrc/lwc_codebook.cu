@@ -255,6 +255,7 @@ __global__ void cb_fill_kernel(uint16_t *__restrict__ out, uint64_t n, const uin
 
 constexpr int kMaxRows = 8;          // activation rows per call
 constexpr uint32_t kLinWarps = 8;    // warps per CTA
+constexpr uint32_t kXStageMax = 32768;   // shared-memory bytes for a tensor's activations (M x whole windows)
 
 struct CbLinTensor {
     const uint8_t *packed;
@@ -267,12 +268,15 @@ struct CbLinTensor {
     uint64_t first_win;    // index of its first window in the launch's window list
     uint32_t cols;
     uint32_t table_bytes;
+    uint32_t stage_x;      // 1: the CTA copies x into shared memory (fits kXStageMax)
+    uint32_t pad;
 };
 
 struct CbLinBatch {
     CbLinTensor t[kMaxBatch];
     uint32_t count;
     uint32_t M;
+    uint32_t x_stage_bytes;   // shared memory after the table for staged activations
     uint64_t total_rows;
     uint64_t total_wins;
     uint32_t *status;
@@ -341,6 +345,38 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
     return d;
 }
 
+// The same from activations staged in shared memory: the lane's four 16-byte
+// chunks sit at xq[(i + rot) & 3] (see stage_activations).
+__device__ __forceinline__ float dot32_staged(const uint32_t (&v)[16], const uint4 *xq, uint32_t rot, float acc) {
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint4 q = xq[(i + rot) & 3u];
+        acc = fma2_bf16(v[4 * i + 0], q.x, acc);
+        acc = fma2_bf16(v[4 * i + 1], q.y, acc);
+        acc = fma2_bf16(v[4 * i + 2], q.z, acc);
+        acc = fma2_bf16(v[4 * i + 3], q.w, acc);
+    }
+    return acc;
+}
+
+// Copy the M x cols activations (cols a multiple of 8) into shared memory so
+// that lane l's chunk i (16 bytes: columns 32 l + 8 i .. + 8 of window q) of
+// row m lands in 16-byte slot (m nwin + q) 128 + 4 l + ((i + l / 2) & 3):
+// the 8 lanes of each quarter-warp then read 8 different bank groups, and the
+// copy's consecutive chunks write 8 different ones too. Read straight from
+// global memory, each lane's 64 contiguous bytes would span 16 cache lines per
+// warp-wide load (64-byte lane stride).
+__device__ __forceinline__ void stage_activations(const uint16_t *x, uint32_t M, uint32_t cols, uint32_t nwin,
+                                                  uint4 *dst) {
+    const uint32_t cpr = cols / 8;   // 16-byte chunks per activation row
+    const uint4 *src = reinterpret_cast<const uint4 *>(x);
+    for (uint32_t g = threadIdx.x; g < M * cpr; g += blockDim.x) {
+        const uint32_t m = g / cpr, c = g - m * cpr;
+        const uint32_t q = c >> 7, l = (c & 127u) >> 2, i = c & 3u;
+        dst[(m * nwin + q) * 128u + 4u * l + ((i + (l >> 1)) & 3u)] = __ldg(src + g);
+    }
+}
+
 // acc + dot(v, x[0..31]) as one FMA chain; v holds the 32 weights as BF16
 // pairs, x is 16-byte aligned.
 __device__ __forceinline__ float dot32(const uint32_t (&v)[16], const uint16_t *x, float acc) {
@@ -374,7 +410,7 @@ __device__ __forceinline__ void finish_row(float (&acc)[MM], uint32_t M, float *
 
 // MM: the largest number of activation rows the instance handles (1, 2, 4, 8).
 template <int K, int MM>
-__global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : MM == 1 ? 4 : 3)
+__global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : 3)
     cb_linear_kernel(const __grid_constant__ CbLinBatch B) {
     using Lay = CbLinLayout<K>;
     constexpr uint32_t kWarps = Lay::kWarps;
@@ -383,6 +419,7 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : MM
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
     uint32_t *bufs = reinterpret_cast<uint32_t *>(smem + Lay::kBufs);
     uint16_t *tab = reinterpret_cast<uint16_t *>(smem + Lay::kTab);
+    uint4 *xst = reinterpret_cast<uint4 *>(smem + Lay::kTotal);
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const uint32_t M = B.M;
 
@@ -430,9 +467,10 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : MM
                 issue_window<K>(tn, ir, iq, my_buf + ((it + issued) & 1u) * kBufWords, &my_bar[(it + issued) & 1u]);
             if (++iq == nwin) { iq = 0; ir += kWarps; }
         }
+        if (tn.stage_x) stage_activations(tn.x, M, tn.cols, nwin, xst);
         const bool tab_ok = dev::mbar_wait_bounded(tab_bar, tab_uses & 1u);
         tab_uses++;
-        if (__syncthreads_or(!tab_ok)) {
+        if (__syncthreads_or(!tab_ok)) {   // also publishes the staged activations
             // let this warp's copies land (bounded), then stop
             status |= LWC_DEVICE_TIMEOUT;
             if (!dead)
@@ -472,7 +510,12 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : MM
             const uint32_t valid = cnt > lane * 32u ? min(32u, cnt - lane * 32u) : 0u;
             const uint16_t *xr = tn.x + c0;
             // each window's products form their own FMA chain, then join the row's sum
-            if (valid == 32u && vec) {
+            if (valid == 32u && tn.stage_x) {
+                const uint4 *xq = xst + cq * 128u + 4u * lane;
+#pragma unroll
+                for (int m = 0; m < MM; m++)
+                    if ((uint32_t)m < M) acc[m] += dot32_staged(v, xq + m * nwin * 128u, lane >> 1, 0.f);
+            } else if (valid == 32u && vec) {
 #pragma unroll
                 for (int m = 0; m < MM; m++)
                     if ((uint32_t)m < M) acc[m] += dot32(v, xr + (uint64_t)m * tn.cols, 0.f);
@@ -592,7 +635,8 @@ lwc_status device_state(DevState &out) {
                 err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&s.per_sm[k], fn, 32 * kWarpsFor[k], kSmem[k]);
             for (int mi = 0; mi < kMmCount && err == cudaSuccess; mi++) {
                 const void *lf = (const void *)kLinKernels[mi][k];
-                err = cudaFuncSetAttribute(lf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLinSmem[k]);
+                err = cudaFuncSetAttribute(lf, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)(kLinSmem[k] + kXStageMax));
                 if (err == cudaSuccess)
                     err = cudaFuncSetAttribute(lf, cudaFuncAttributePreferredSharedMemoryCarveout,
                                                cudaSharedmemCarveoutMaxShared);
@@ -646,7 +690,7 @@ lwc_status launch_cb_linear_group(const std::vector<int> &idx, const lwc_desc *d
     CbLinBatch B;
     std::memset(&B, 0, sizeof B);
     const uint32_t K = descs[idx[0]].k;
-    uint64_t rows = 0, wins = 0;
+    uint64_t rows = 0, wins = 0, xstage = 0;
     for (size_t j = 0; j < idx.size(); j++) {
         const int i = idx[j];
         const lwc_desc &d = descs[i];
@@ -663,17 +707,31 @@ lwc_status launch_cb_linear_group(const std::vector<int> &idx, const lwc_desc *d
         t.first_row = rows;
         t.first_win = wins;
         rows += t.rows;
-        wins += t.rows * ((t.cols + kTile - 1) / kTile);
+        const uint32_t nwin = (t.cols + kTile - 1) / kTile;
+        wins += t.rows * nwin;
+        const uint64_t xbytes = (uint64_t)M * nwin * kTile * 2;   // whole windows
+        if (t.cols % 8 == 0 && xbytes <= kXStageMax) {
+            t.stage_x = 1;
+            xstage = std::max<uint64_t>(xstage, xbytes);
+        }
     }
     B.count = (uint32_t)idx.size();
     B.M = M;
     B.total_rows = rows;
     B.total_wins = wins;
+    B.x_stage_bytes = (uint32_t)xstage;
     B.status = d_status;
     const int mi = mm_index(M);
-    const int per_sm = std::max(1, ds.lin_per_sm[mi][K]);
+    const size_t smem = kLinSmem[K] + xstage;
+    int per_sm = ds.lin_per_sm[mi][K];
+    if (xstage) {
+        cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void *)kLinKernels[mi][K],
+                                                                      32 * kLinWarps, smem);
+        if (e != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(e));
+    }
+    per_sm = std::max(1, per_sm);
     const uint64_t grid = std::min<uint64_t>((rows + kLinWarps - 1) / kLinWarps, (uint64_t)per_sm * ds.sms);
-    kLinKernels[mi][K]<<<(unsigned)grid, 32 * kLinWarps, kLinSmem[K], stream>>>(B);
+    kLinKernels[mi][K]<<<(unsigned)grid, 32 * kLinWarps, smem, stream>>>(B);
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));
     return LWC_OK;
