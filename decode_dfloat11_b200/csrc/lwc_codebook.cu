@@ -255,7 +255,7 @@ __global__ void cb_fill_kernel(uint16_t *__restrict__ out, uint64_t n, const uin
 
 constexpr int kMaxRows = 8;          // activation rows per call
 constexpr uint32_t kLinWarps = 8;    // warps per CTA
-constexpr uint32_t kXStageMax = 32768;   // shared-memory bytes for a tensor's activations (M x whole windows)
+constexpr uint32_t kXStageMax = 65536;   // shared-memory bytes for a tensor's activations (M x whole windows)
 
 struct CbLinTensor {
     const uint8_t *packed;
@@ -329,7 +329,6 @@ __device__ __forceinline__ void issue_window(const CbLinTensor &tn, uint64_t r, 
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
 // acc + w.lo * x.lo, then + w.hi * x.hi: two FMAs on BF16 pairs with an FP32
 // accumulator (PTX mixed-precision fma.rn.f32.bf16: the product of two BF16

@@ -636,7 +636,6 @@ __device__ __forceinline__ uint32_t div_cols(uint32_t n, uint32_t magic, uint32_
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t p) { return __uint_as_float(p << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t p) { return __uint_as_float(p & 0xFFFF0000u); }
 
 // acc + w.lo * x.lo, then + w.hi * x.hi: two FMAs on BF16 pairs with an FP32
 // accumulator (PTX mixed-precision fma.rn.f32.bf16: the product of two BF16
