@@ -651,38 +651,49 @@ __device__ __forceinline__ float fma2_bf16(uint32_t w2, uint32_t x2, float acc) 
     return d;
 }
 
-// Warp sum of c; lane 0 adds it to ym[row].
-__device__ __forceinline__ void lin_flush(float c, float *ym, uint64_t row, uint32_t lane) {
+// Warp sums of c[m]; lane 0 adds them to y[m, row].
+template <int MM>
+__device__ __forceinline__ void lin_flush(const float (&c)[MM], uint32_t M, float *y, uint64_t rows,
+                                          uint64_t row, uint32_t lane) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-    if (lane == 0) atomicAdd(ym + row, c);
+    for (int m = 0; m < MM; m++) {
+        if ((uint32_t)m < M) {
+            float v = c[m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+            if (lane == 0) atomicAdd(y + (uint64_t)m * rows + row, v);
+        }
+    }
 }
 
-// One activation row's part of a round: each valid lane brings p for row
-// offset lr; the round's weights lie in rows rf .. rl (warp-uniform, at or
-// after the open row cur). Rows before rl get their warp sums added to
-// ym[row_base + row]; acc becomes the lane's sum for rl.
-__device__ __forceinline__ void lin_update(float &acc, float p, bool valid, uint32_t lr, uint32_t rf, uint32_t rl,
-                                           uint32_t cur, float *ym, uint64_t row_base, uint32_t lane) {
+// One round: each valid lane brings p[m] for row offset lr; the round's
+// weights lie in rows rf .. rl (warp-uniform, rf at or after the open row
+// cur). Rows before rl are flushed; acc becomes rl's lane sums.
+template <int MM>
+__device__ __forceinline__ void lin_round(float (&acc)[MM], uint32_t &cur, const float (&p)[MM],
+                                          bool valid, uint32_t lr, uint32_t rf, uint32_t rl, uint32_t M, float *y,
+                                          uint64_t rows, uint64_t row_base, uint32_t lane) {
     if (rf == rl && rl == cur) {
-        acc += valid ? p : 0.f;
+#pragma unroll
+        for (int m = 0; m < MM; m++) acc[m] += valid ? p[m] : 0.f;
         return;
     }
-    float keep = 0.f;
     for (uint32_t rr = cur == kNoRow ? rf : cur; rr <= rl; rr++) {
-        const float c = (valid && lr == rr ? p : 0.f) + (rr == cur ? acc : 0.f);
-        if (rr < rl)
-            lin_flush(c, ym, row_base + rr, lane);
-        else
-            keep = c;
+        float c[MM];
+#pragma unroll
+        for (int m = 0; m < MM; m++) c[m] = (valid && lr == rr ? p[m] : 0.f) + (rr == cur ? acc[m] : 0.f);
+        if (rr < rl) {
+            lin_flush<MM>(c, M, y, rows, row_base + rr, lane);
+        } else {
+#pragma unroll
+            for (int m = 0; m < MM; m++) acc[m] = c[m];
+        }
     }
-    acc = keep;
+    cur = rl;
 }
 
 // The linear layer's part of one decoded block [o0, o1) (exponents staged at
-// stage[i - (o0 & ~15)], sign|mantissa bytes of the first groups in sv). The
-// activation rows are taken one at a time, so only their running sums stay
-// live across rounds.
+// stage[i - (o0 & ~15)], sign|mantissa bytes of the first groups in sv).
 template <int MM>
 __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const Df11Tensor &tn, const uint8_t *stage,
                                           const uint4 (&sv)[kWarpMergeRegs], uint64_t o0, uint64_t o1,
@@ -708,7 +719,7 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
         return;
     }
 
-    float acc[MM];
+    float acc[MM], p[MM];
 #pragma unroll
     for (int m = 0; m < MM; m++) acc[m] = 0.f;
     uint32_t cur = kNoRow;
@@ -717,51 +728,48 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
     auto single = [&](uint32_t r, bool valid, uint32_t first, uint32_t last) {
         const uint32_t d = d0 + r;
         const uint32_t lr = div_cols(d, magic, shifts);
-        const uint32_t rf = div_cols(d0 + first, magic, shifts), rl = div_cols(d0 + last, magic, shifts);
-        const float w = valid ? bf16_lo(merge1(sb[r], stage[r])) : 0.f;
-        const uint16_t *xc = x + (d - lr * cols);
 #pragma unroll
-        for (int m = 0; m < MM; m++) {
-            if ((uint32_t)m < M) {
-                const float p = valid ? w * bf16_lo(xc[(uint64_t)m * cols]) : 0.f;
-                lin_update(acc[m], p, valid, lr, rf, rl, cur, y + (uint64_t)m * rows, row_base, lane);
-            }
+        for (int m = 0; m < MM; m++) p[m] = 0.f;
+        if (valid) {
+            const float w = bf16_lo(merge1(sb[r], stage[r]));
+            const uint16_t *xc = x + (d - lr * cols);
+#pragma unroll
+            for (int m = 0; m < MM; m++)
+                if ((uint32_t)m < M) p[m] = w * bf16_lo(xc[(uint64_t)m * cols]);
         }
-        cur = rl;
+        lin_round<MM>(acc, cur, p, valid, lr, div_cols(d0 + first, magic, shifts), div_cols(d0 + last, magic, shifts), M,
+                  y, rows, row_base, lane);
     };
     // a round of 32 groups starting at block-relative rb; this lane's group at rb + 16 lane
     const uint32_t rhi = (uint32_t)(g_hi - base);
     auto groups = [&](uint32_t rb, const uint4 &s, bool valid) {
         const uint32_t r = rb + 16u * lane, d = d0 + r;
         const uint32_t lr = div_cols(d, magic, shifts);
-        const uint32_t last = min(rhi, rb + 512u) - 16u;   // the round's last group (groups never straddle rows)
-        const uint32_t rf = div_cols(d0 + rb, magic, shifts), rl = div_cols(d0 + last, magic, shifts);
-        uint32_t wv[8];
-        const uint4 e = valid ? *reinterpret_cast<const uint4 *>(stage + r) : make_uint4(0, 0, 0, 0);
-        merge4(s.x, e.x, wv[0], wv[1]);
-        merge4(s.y, e.y, wv[2], wv[3]);
-        merge4(s.z, e.z, wv[4], wv[5]);
-        merge4(s.w, e.w, wv[6], wv[7]);
-        const uint4 *xc = reinterpret_cast<const uint4 *>(x + (d - lr * cols));   // 16 columns, 32-byte aligned
 #pragma unroll
-        for (int m = 0; m < MM; m++) {
-            if ((uint32_t)m < M) {
-                float t = 0.f;
-                if (valid) {
+        for (int m = 0; m < MM; m++) p[m] = 0.f;
+        if (valid) {
+            const uint4 e = *reinterpret_cast<const uint4 *>(stage + r);
+            uint32_t wv[8];
+            merge4(s.x, e.x, wv[0], wv[1]);
+            merge4(s.y, e.y, wv[2], wv[3]);
+            merge4(s.z, e.z, wv[4], wv[5]);
+            merge4(s.w, e.w, wv[6], wv[7]);
+            const uint4 *xc = reinterpret_cast<const uint4 *>(x + (d - lr * cols));   // 16 columns, 32-byte aligned
+#pragma unroll
+            for (int m = 0; m < MM; m++) {
+                if ((uint32_t)m < M) {
                     const uint4 a = __ldg(xc + (uint64_t)m * (cols / 8)), b = __ldg(xc + (uint64_t)m * (cols / 8) + 1);
-                    t = fma2_bf16(wv[0], a.x, t);
-                    t = fma2_bf16(wv[1], a.y, t);
-                    t = fma2_bf16(wv[2], a.z, t);
-                    t = fma2_bf16(wv[3], a.w, t);
-                    t = fma2_bf16(wv[4], b.x, t);
-                    t = fma2_bf16(wv[5], b.y, t);
-                    t = fma2_bf16(wv[6], b.z, t);
-                    t = fma2_bf16(wv[7], b.w, t);
+                    const uint32_t xa[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+                    float t = 0.f;
+#pragma unroll
+                    for (int j = 0; j < 8; j++) t = fma2_bf16(wv[j], xa[j], t);
+                    p[m] = t;
                 }
-                lin_update(acc[m], t, valid, lr, rf, rl, cur, y + (uint64_t)m * rows, row_base, lane);
             }
         }
-        cur = rl;
+        const uint32_t last = min(rhi, rb + 512u) - 16u;   // the round's last group (groups never straddle rows)
+        lin_round<MM>(acc, cur, p, valid, lr, div_cols(d0 + rb, magic, shifts), div_cols(d0 + last, magic, shifts), M,
+                  y, rows, row_base, lane);
     };
 
     // weights before the first group, on lanes 0..15
@@ -787,11 +795,7 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
         const bool valid = lane >= 16 && tb + (lane - 16) < o1;
         single((uint32_t)(tb - base) + (valid ? lane - 16 : 0u), valid, (uint32_t)(tb - base), (uint32_t)(o1 - 1 - base));
     }
-    if (cur != kNoRow) {
-#pragma unroll
-        for (int m = 0; m < MM; m++)
-            if ((uint32_t)m < M) lin_flush(acc[m], y + (uint64_t)m * rows, row_base + cur, lane);
-    }
+    if (cur != kNoRow) lin_flush<MM>(acc, M, y, rows, row_base + cur, lane);
 }
 
 // Single-exponent tensors: one warp per row, lane-strided columns.
@@ -1077,11 +1081,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
 }
 
 // Fused decode + linear layer (BF16 elements, blocks of 32 chunks) for up
-// to MM activation rows: two CTAs per SM up to two rows (measured: M = 2
-// 0.42 -> 0.38 ms per Llama-3-8B layer), one CTA with room for the running
-// sums beyond (two CTAs spilled: M = 8 0.79 -> 1.02 ms).
+// to MM activation rows; with more than one row the accumulators need more
+// registers than two CTAs per SM leave.
 template <int MM>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, MM <= 2 ? kWarpCtasPerSm : 1)
+__global__ void __launch_bounds__(kWarpsPerCta * 32, MM == 1 ? kWarpCtasPerSm : 1)
     df11_warp_linear_kernel(const __grid_constant__ Df11Batch B, const __grid_constant__ Df11Lin X) {
     df11_warp_body<LWC_ELEM_BF16, MM>(B, &X);
 }
