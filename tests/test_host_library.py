@@ -187,6 +187,49 @@ def test_decoders_validate_before_any_device_call():
     lwc.lwc_decode_codebook(c0, None, None)
 
 
+def test_linear_layer_validates_before_any_device_call():
+    # y = x W^T entry points: every argument error is reported before a CUDA call
+    w = synth.as_u16(synth.normal_bf16((64 * 48,), seed=3, sigma=0.02))
+    d, _ = lwc.lwc_encode_dfloat11(w)
+    dc, _ = lwc.lwc_encode_codebook(w)
+    for desc, fn in ((d, lwc.lwc_linear_dfloat11), (dc, lwc.lwc_linear_codebook)):
+        for M in (0, 9, -1):                                           # 1..8 activation rows
+            with pytest.raises(lwc.LwcError) as e:
+                fn(desc, 0x1000, 48, 0x2000, M, 0x3000)
+            assert e.value.status == 1 and "M must be" in str(e.value)
+        for cols in (0, 47, 64 * 48 + 1, 1 << 31):                    # must divide n, < 2^31
+            with pytest.raises(lwc.LwcError) as e:
+                fn(desc, 0x1000, cols, 0x2000, 1, 0x3000)
+            assert e.value.status == 1
+        for args in ((0x1008, 0x2000, 0x3000), (0x1000, 0x2008, 0x3000), (0x1000, 0x2000, 0x3002)):
+            with pytest.raises(lwc.LwcError) as e:                     # blob, x 16-byte; y 4-byte aligned
+                fn(desc, args[0], 48, args[1], 1, args[2])
+            assert e.value.status == 2
+        with pytest.raises(lwc.LwcError) as e:
+            fn(desc, None, 48, 0x2000, 1, 0x3000)
+        assert e.value.status == 1
+    with pytest.raises(lwc.LwcError) as e:                             # wrong codec
+        lwc.lwc_linear_dfloat11(dc, 0x1000, 48, 0x2000, 1, 0x3000)
+    assert e.value.status == 1
+    # DFloat11 blobs the fused layer does not take
+    d256, _ = lwc.lwc_encode_dfloat11(w, threads_per_block=256)
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_linear_dfloat11(d256, 0x1000, 48, 0x2000, 1, 0x3000)
+    assert e.value.status == 4 and "32 chunks" in str(e.value)
+    x32 = np.arange(64 * 48, dtype=np.uint32) * 2654435761 % (1 << 31)
+    d32, _ = lwc.lwc_encode_dfloat11_elements(x32.astype(np.uint32), lwc.LWC_ELEM_FP32)
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_linear_dfloat11(d32, 0x1000, 48, 0x2000, 1, 0x3000)
+    assert e.value.status == 4 and "BF16" in str(e.value)
+    # batched: argument lists must agree; empty tensors need no device
+    with pytest.raises(ValueError):
+        lwc.LinearBatch([d, d], [0x1000], [48, 48], [0x2000, 0x2000], [0x3000, 0x3000], 1)
+    d0, _ = lwc.lwc_encode_dfloat11(np.zeros(0, np.uint16))
+    c0, _ = lwc.lwc_encode_codebook(np.zeros(0, np.uint16))
+    lwc.lwc_linear_dfloat11_batched(lwc.LinearBatch([d0], [None], [16], [None], [None], 2))
+    lwc.lwc_linear_codebook_batched(lwc.LinearBatch([c0, c0], [None, None], [1, 7], [None, None], [None, None], 8))
+
+
 def test_encoder_rejects_bad_arguments():
     w = np.zeros(10, np.uint16)
     for kw in (dict(chunk_bytes=6), dict(chunk_bytes=10), dict(threads_per_block=48),
