@@ -186,7 +186,13 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
         const bool tab_ok = dev::mbar_wait_bounded(tab_bar, tab_uses & 1u);
         tab_uses++;
         if (__syncthreads_or(!tab_ok)) {
+            // let the table copy and this warp's first two tiles land (bounded), then stop
             status |= LWC_DEVICE_TIMEOUT;
+            if (tid == 0) dev::mbar_wait_bounded(tab_bar, (tab_uses - 1) & 1u);
+            if (!dead) {
+                if (warp < ns) dev::mbar_wait_bounded(&my_bar[it & 1u], (it >> 1) & 1u);
+                if (warp + kWarps < ns) dev::mbar_wait_bounded(&my_bar[(it + 1) & 1u], ((it + 1) >> 1) & 1u);
+            }
             break;
         }
 
@@ -194,8 +200,9 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
             const uint32_t bi = it & 1u;
             const bool ok = dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
-                // let the copy issued into the other buffer land (bounded), then stop
+                // let this tile's copy and the one issued into the other buffer land (bounded), then stop
                 status |= LWC_DEVICE_TIMEOUT;
+                dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
                 if (j + kWarps < ns) dev::mbar_wait_bounded(&my_bar[bi ^ 1u], ((it + 1) >> 1) & 1u);
                 dead = true;
                 break;
@@ -470,8 +477,9 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : 3)
         const bool tab_ok = dev::mbar_wait_bounded(tab_bar, tab_uses & 1u);
         tab_uses++;
         if (__syncthreads_or(!tab_ok)) {   // also publishes the staged activations
-            // let this warp's copies land (bounded), then stop
+            // let the table copy and this warp's copies land (bounded), then stop
             status |= LWC_DEVICE_TIMEOUT;
+            if (tid == 0) dev::mbar_wait_bounded(tab_bar, (tab_uses - 1) & 1u);
             if (!dead)
                 for (uint32_t k = 0; k < issued; k++) dev::mbar_wait_bounded(&my_bar[(it + k) & 1u], ((it + k) >> 1) & 1u);
             break;
@@ -481,8 +489,9 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : 3)
             const uint32_t bi = it & 1u;
             const bool ok = dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
-                // let the copy issued into the other buffer land (bounded), then stop
+                // let this window's copy and the one issued into the other buffer land (bounded), then stop
                 status |= LWC_DEVICE_TIMEOUT;
+                dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
                 if (cq + 1 < nwin || cr + kWarps < row_end) dev::mbar_wait_bounded(&my_bar[bi ^ 1u], ((it + 1) >> 1) & 1u);
                 dead = true;
                 break;
@@ -560,6 +569,19 @@ __global__ void cb_linear_fill_kernel(const uint16_t *__restrict__ table, const 
             if ((uint32_t)m < M)
                 for (uint32_t c = lane; c < cols; c += 32u) acc[m] = fmaf(wv, bf16_lo(x[(uint64_t)m * cols + c]), acc[m]);
         finish_row<kMaxRows>(acc, M, y, rows, r, lane);
+    }
+}
+
+// Self-test of the bounded wait the kernels use on their asynchronous copies:
+// one thread waits on an mbarrier phase that completes only through its own
+// arrival (`arrive`), for at most `polls` polls; a wait that gives up reports
+// LWC_DEVICE_TIMEOUT and the kernel returns normally.
+__global__ void wait_selftest_kernel(uint32_t *status, uint32_t polls, uint32_t arrive) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        dev::mbar_init(&bar, 1);
+        if (arrive) dev::mbar_arrive(&bar);
+        if (!dev::mbar_wait_bounded(&bar, 0, polls)) atomicOr(status, LWC_DEVICE_TIMEOUT);
     }
 }
 
@@ -862,6 +884,17 @@ lwc_status lwc_linear_codebook(const lwc_desc *desc, const void *d_blob, uint64_
                                float *d_y, uint32_t *d_status, lwc_stream_t stream) {
     if (!desc) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
     return lwc_linear_codebook_batched(desc, &d_blob, &cols, &d_x, M, &d_y, 1, d_status, stream);
+}
+
+lwc_status lwc_selftest_bounded_wait(uint32_t *d_status, uint32_t polls, int arrive, lwc_stream_t stream) {
+    if (!d_status || (reinterpret_cast<uintptr_t>(d_status) & 3u))
+        return fail(LWC_ERR_INVALID_ARG, "status word must be a 4-byte aligned device pointer");
+    if (polls == 0 || polls > (1u << 24)) return fail(LWC_ERR_INVALID_ARG, "polls must be 1..2^24");
+    wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(d_status, polls, arrive ? 1u : 0u);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "self-test launch: %s", cudaGetErrorString(err));
+    clear_error();
+    return LWC_OK;
 }
 
 }  // extern "C"

@@ -396,7 +396,9 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
         // this item's segment and gaps (its copy is the only one in flight)
         const bool arrived = dev::mbar_wait_bounded(&bars[0], it & 1u);
         if (__syncthreads_or(!arrived)) {
+            // let the late copy land (bounded) before the CTA's shared memory goes away
             bad |= LWC_DEVICE_TIMEOUT;
+            if (tid == 0) dev::mbar_wait_bounded(&bars[0], it & 1u);
             break;
         }
         bool next_issued = false;
@@ -907,7 +909,9 @@ __device__ __forceinline__ void df11_warp_body(const Df11Batch &B, const Df11Lin
             const bool arrived = dev::mbar_wait_bounded(bar, items & 1u);
             items++;
             if (__any_sync(0xFFFFFFFFu, !arrived)) {
+                // let the late copy land (bounded) before this warp stops
                 bad |= LWC_DEVICE_TIMEOUT;
+                if (lane == 0) dev::mbar_wait_bounded(bar, (items - 1) & 1u);
                 dead = true;
                 break;
             }

@@ -38,7 +38,8 @@ EXPORTED = (
     "lwc_encode_device_workspace_bytes", "lwc_encode_dfloat11_device_plan",
     "lwc_encode_dfloat11_elements_device_plan", "lwc_encode_codebook_device_plan",
     "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_linear_codebook",
-    "lwc_linear_codebook_batched", "lwc_linear_dfloat11", "lwc_linear_dfloat11_batched", "lwc_status_string",
+    "lwc_linear_codebook_batched", "lwc_linear_dfloat11", "lwc_linear_dfloat11_batched",
+    "lwc_selftest_bounded_wait", "lwc_status_string",
     "lwc_last_error", "lwc_version",
 )
 
@@ -122,6 +123,8 @@ def load():
         getattr(L, name).argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_u64), ctypes.POINTER(_P), ctypes.c_int,
                                      ctypes.POINTER(_P), ctypes.c_int, _P, _P]
         getattr(L, name).restype = ctypes.c_int
+    L.lwc_selftest_bounded_wait.argtypes = [_P, ctypes.c_uint32, ctypes.c_int, _P]
+    L.lwc_selftest_bounded_wait.restype = ctypes.c_int
     L.lwc_status_string.argtypes = [ctypes.c_int]
     L.lwc_status_string.restype = ctypes.c_char_p
     L.lwc_last_error.argtypes = []
@@ -304,6 +307,11 @@ def lwc_linear_dfloat11_batched(batch: LinearBatch, d_status=None, stream=None) 
     b = batch
     _check(load().lwc_linear_dfloat11_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
                                               _stream(stream)))
+
+
+def lwc_selftest_bounded_wait(d_status, polls: int, arrive: bool, stream=None) -> None:
+    """Run the bounded-wait self-test kernel (see lwc.h)."""
+    _check(load().lwc_selftest_bounded_wait(_addr(d_status), polls, int(bool(arrive)), _stream(stream)))
 
 
 def lwc_encode_device_workspace_bytes(n: int) -> int:

@@ -358,6 +358,15 @@ LWC_API lwc_status lwc_encode_dfloat11_device_noalloc(const void *d_src, uint64_
                                                       void *d_blob, uint64_t blob_bytes, lwc_desc *desc_out,
                                                       lwc_stream_t stream);
 
+/* Self-test of the bounded wait every kernel above uses on its asynchronous
+ * copies (failure detection without a GPU fault): one thread waits, for at
+ * most `polls` (1 .. 2^24) polls, on a shared-memory mbarrier phase that
+ * completes only if `arrive` is non-zero (the thread's own arrival). A wait
+ * that gives up ORs LWC_DEVICE_TIMEOUT into *d_status (device, 4-byte
+ * aligned, owned and zeroed by the caller) and the kernel returns normally,
+ * so the context stays usable. No copy, trap or fault is involved. */
+LWC_API lwc_status lwc_selftest_bounded_wait(uint32_t *d_status, uint32_t polls, int arrive, lwc_stream_t stream);
+
 /* ---- helpers -------------------------------------------------------------- */
 
 /* Static string naming a status code. */

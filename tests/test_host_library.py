@@ -230,6 +230,13 @@ def test_linear_layer_validates_before_any_device_call():
     lwc.lwc_linear_codebook_batched(lwc.LinearBatch([c0, c0], [None, None], [1, 7], [None, None], [None, None], 8))
 
 
+def test_wait_selftest_validates_before_any_device_call():
+    for args in ((None, 64, False), (0x1002, 64, False), (0x1000, 0, True), (0x1000, (1 << 24) + 1, True)):
+        with pytest.raises(lwc.LwcError) as e:
+            lwc.lwc_selftest_bounded_wait(*args)
+        assert e.value.status == 1
+
+
 def test_encoder_rejects_bad_arguments():
     w = np.zeros(10, np.uint16)
     for kw in (dict(chunk_bytes=6), dict(chunk_bytes=10), dict(threads_per_block=48),
