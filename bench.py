@@ -231,6 +231,54 @@ def cpu_baseline(blobs, n_total: int):
                       f"(lib-encoded blobs), one host thread, {dt:.2f} s"}
 
 
+def _oracle_decode_worker(job) -> int:
+    """Decode one blob that sits in a shared-memory segment: (name, offset, size)."""
+    from multiprocessing import shared_memory
+
+    from oracle import df11 as odf
+    name, off, size = job
+    shm = shared_memory.SharedMemory(name=name)
+    try:
+        blob = np.ndarray((size,), dtype=np.uint8, buffer=shm.buf, offset=off)
+        odf.decode(blob)
+        n = int(odf.B.unpack_header(blob)["n"])
+        del blob
+    finally:
+        shm.close()
+    return n
+
+
+def cpu_baseline_all_cores(blobs, n_total: int):
+    """The same oracle decoder, one tensor per worker process, on the host's
+    cores (spawned processes: no fork after the GPU was used). The blobs sit
+    in one shared-memory segment; timed from handing out the jobs to the last
+    result, with the workers already started."""
+    import multiprocessing as mp
+    from multiprocessing import shared_memory
+    workers = max(1, min(os.cpu_count() or 1, len(blobs)))
+    total = sum(b.size for b in blobs)
+    shm = shared_memory.SharedMemory(create=True, size=max(1, total))
+    try:
+        jobs, off = [], 0
+        for b in blobs:
+            np.ndarray((b.size,), dtype=np.uint8, buffer=shm.buf, offset=off)[:] = b
+            jobs.append((shm.name, off, b.size))
+            off += b.size
+        order = sorted(range(len(jobs)), key=lambda i: -jobs[i][2])   # largest first
+        ctx = mp.get_context("spawn")
+        with ctx.Pool(workers) as pool:
+            pool.map(_oracle_decode_worker, [jobs[order[-1]]] * workers, chunksize=1)   # start, import
+            t0 = time.perf_counter()
+            n = sum(pool.map(_oracle_decode_worker, [jobs[i] for i in order], chunksize=1))
+            dt = time.perf_counter() - t0
+    finally:
+        shm.close()
+        shm.unlink()
+    return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": f"oracle bit-serial DFloat11 decode of the whole layer ({n:,} weights), one tensor per "
+                      f"process on {workers} spawned workers (blobs in shared memory), {dt:.2f} s"}
+
+
 # ---------------------------------------------------------------- our arm
 
 def run_lwc(args, rank, world, local_rank, dist):
@@ -513,6 +561,7 @@ def run_lwc(args, rank, world, local_rank, dist):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(blobs_h, n_total)
+        result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(blobs_h, n_total)
     return result
 
 
