@@ -266,11 +266,14 @@ def cpu_baseline_all_cores(blobs, n_total: int):
             off += b.size
         order = sorted(range(len(jobs)), key=lambda i: -jobs[i][2])   # largest first
         ctx = mp.get_context("spawn")
-        with ctx.Pool(workers) as pool:
-            pool.map(_oracle_decode_worker, [jobs[order[-1]]] * workers, chunksize=1)   # start, import
-            t0 = time.perf_counter()
-            n = sum(pool.map(_oracle_decode_worker, [jobs[i] for i in order], chunksize=1))
-            dt = time.perf_counter() - t0
+        with ctx.Pool(workers) as pool:   # leaving the block terminates the workers
+            try:
+                pool.map_async(_oracle_decode_worker, [jobs[order[-1]]] * workers, chunksize=1).get(timeout=600)
+                t0 = time.perf_counter()
+                n = sum(pool.map_async(_oracle_decode_worker, [jobs[i] for i in order], chunksize=1).get(timeout=600))
+                dt = time.perf_counter() - t0
+            except mp.TimeoutError:
+                return {"unavailable": "oracle worker processes did not finish within 600 s"}
     finally:
         shm.close()
         shm.unlink()
