@@ -15,6 +15,11 @@
 // possibly across several tensors of one layer; each warp keeps its own
 // double buffer, filled by bulk copies two tiles ahead, and unpacks, gathers
 // from the shared table and writes 16-byte stores.
+//
+// Also here: cb_linear_kernel, the decode fused into the linear layer that
+// consumes the weights (y = x W^T for up to 8 activation rows, weights kept
+// in registers; see the section comment below), and the self-test kernel of
+// the bounded mbarrier wait all these kernels use.
 #include <cuda_runtime.h>
 
 #include <algorithm>
