@@ -74,6 +74,29 @@ def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=Non
     return desc, blob
 
 
+def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status=None):
+    """y = x W^T with W (``shape`` = (rows, cols), the tensor ``blob``
+    decodes to) decoded in registers; x: M x cols BF16 on the GPU, M <= 8.
+    Returns ``out`` (M x rows FP32, allocated if None)."""
+    import torch
+    if codec not in CODECS:
+        raise ValueError(f"unknown codec {codec!r}")
+    if len(shape) != 2:
+        raise ValueError("the weight must be a rows x cols matrix")
+    rows, cols = int(shape[0]), int(shape[1])
+    if x.dim() != 2 or x.shape[1] != cols or x.dtype != torch.bfloat16:
+        raise ValueError(f"x must be M x {cols} BF16")
+    x = x.contiguous()
+    M = int(x.shape[0])
+    if out is None:
+        out = torch.empty((M, rows), dtype=torch.float32, device=x.device)
+    elif tuple(out.shape) != (M, rows) or out.dtype != torch.float32 or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {M} x {rows} FP32 tensor")
+    fn = lwc.lwc_linear_dfloat11 if codec == "dfloat11" else lwc.lwc_linear_codebook
+    fn(desc, blob, cols, x, M, out, d_status=status, stream=stream)
+    return out
+
+
 class ResidentModel:
     """Compressed layers in device memory plus reusable BF16 output buffers.
 
@@ -153,6 +176,16 @@ class ResidentModel:
             lwc.lwc_decode_dfloat11_batched(batch, d_status=status, stream=stream)
         else:
             lwc.lwc_decode_codebook_batched(batch, d_status=status, stream=stream)
+
+    def linear(self, layer: int, index: int, x, out=None, stream=None, status=None):
+        """y = x W^T for matrix ``index`` of ``layer`` without decoding it to
+        memory: the weights are decoded in registers by the fused kernel
+        (lwc_linear_dfloat11 / lwc_linear_codebook). x: M x cols BF16 on this
+        model's GPU, 1 <= M <= 8 (token generation); returns (or fills
+        ``out``) the M x rows FP32 result."""
+        return fused_linear(self.layers[layer]["descs"][index], self.layers[layer]["blobs"][index],
+                            self.layers[layer]["shapes"][index], x, self.codec, out=out, stream=stream,
+                            status=status)
 
     def pipelined(self, compute_stream, decode_stream=None):
         """Iterate over the layers with decoding one layer ahead of use.

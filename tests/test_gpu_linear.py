@@ -209,3 +209,32 @@ def test_linear_argument_errors():
     with pytest.raises(lwc.LwcError) as e:
         lwc.lwc_linear_dfloat11(d32, torch.from_numpy(b32).to("cuda"), 48, x, 2, y)
     assert e.value.status == 4
+
+
+@pytest.mark.parametrize("codec", ["dfloat11", "codebook"])
+def test_resident_model_linear(codec):
+    from decode_dfloat11_b200.layers import ResidentModel, fused_linear
+    shapes = [(96, 256), (40, 1040), (17, 48)]
+    layers = [[synth.normal_bf16(s, 700 + 10 * L + j, sigma=0.02, outlier_frac=1e-3, device="cuda")
+               for j, s in enumerate(shapes)] for L in range(2)]
+    m = ResidentModel(codec, "cuda")
+    for L, ts in enumerate(layers):
+        m.add_layer_from_device(f"layer{L}", ts)
+    m.finalize()
+    for L, ts in enumerate(layers):
+        for j, t in enumerate(ts):
+            rows, cols = t.shape
+            x = synth.activations_bf16(2, cols, seed=50 + j, device="cuda")
+            y = m.linear(L, j, x)
+            torch.cuda.synchronize()
+            check(y.cpu().numpy().astype(np.float64), synth.as_u16(t).reshape(rows, cols), x, cols, codec,
+                  m.layers[L]["descs"][j])
+    # argument checks of the torch-level helper
+    d, b = m.layers[0]["descs"][0], m.layers[0]["blobs"][0]
+    with pytest.raises(ValueError):
+        fused_linear(d, b, (96, 256), torch.zeros((2, 255), dtype=torch.bfloat16, device="cuda"), codec)
+    with pytest.raises(ValueError):
+        fused_linear(d, b, (96, 256), torch.zeros((2, 256), dtype=torch.float32, device="cuda"), codec)
+    with pytest.raises(ValueError):
+        fused_linear(d, b, (96, 256), torch.zeros((2, 256), dtype=torch.bfloat16, device="cuda"), codec,
+                     out=torch.empty((2, 95), dtype=torch.float32, device="cuda"))
