@@ -237,6 +237,27 @@ def test_wait_selftest_validates_before_any_device_call():
         assert e.value.status == 1
 
 
+def test_fused_linear_helper_checks_shapes_before_the_library():
+    import torch
+    from decode_dfloat11_b200.layers import fused_linear
+    w = synth.as_u16(synth.normal_bf16((16 * 32,), seed=4, sigma=0.02))
+    d, b = lwc.lwc_encode_codebook(w)
+    ok = torch.zeros((2, 32), dtype=torch.bfloat16)
+    bad_cases = [
+        dict(shape=(16, 32), x=torch.zeros((2, 31), dtype=torch.bfloat16)),          # wrong cols
+        dict(shape=(16, 32), x=torch.zeros((2, 32), dtype=torch.float16)),           # not BF16
+        dict(shape=(16, 32), x=torch.zeros(32, dtype=torch.bfloat16)),               # not M x cols
+        dict(shape=(512,), x=ok),                                                    # W not a matrix
+        dict(shape=(16, 32), x=ok, out=torch.empty((2, 15), dtype=torch.float32)),   # wrong out shape
+        dict(shape=(16, 32), x=ok, out=torch.empty((2, 16), dtype=torch.float64)),   # wrong out dtype
+    ]
+    for case in bad_cases:
+        with pytest.raises(ValueError):
+            fused_linear(d, b, case["shape"], case["x"], "codebook", out=case.get("out"))
+    with pytest.raises(ValueError):
+        fused_linear(d, b, (16, 32), ok, "huffman")
+
+
 def test_encoder_rejects_bad_arguments():
     w = np.zeros(10, np.uint16)
     for kw in (dict(chunk_bytes=6), dict(chunk_bytes=10), dict(threads_per_block=48),
