@@ -248,35 +248,57 @@ def _oracle_decode_worker(job) -> int:
     return n
 
 
+class OraclePool:
+    """Spawned worker processes (no fork after the GPU was used) that decode
+    blobs with the oracle, one blob per task; the blobs sit in one
+    shared-memory segment. ``decode_all()`` decodes every blob once and
+    returns the weight count; waits are bounded."""
+
+    def __init__(self, blobs):
+        self.blobs = blobs
+        self.workers = max(1, min(os.cpu_count() or 1, len(blobs)))
+
+    def __enter__(self):
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        total = sum(b.size for b in self.blobs)
+        self.shm = shared_memory.SharedMemory(create=True, size=max(1, total))
+        jobs, off = [], 0
+        for b in self.blobs:
+            np.ndarray((b.size,), dtype=np.uint8, buffer=self.shm.buf, offset=off)[:] = b
+            jobs.append((self.shm.name, off, b.size))
+            off += b.size
+        self.jobs = sorted(jobs, key=lambda j: -j[2])   # largest first
+        self.pool = mp.get_context("spawn").Pool(self.workers)
+        self._map([self.jobs[-1]] * self.workers)          # start the workers, import the oracle
+        return self
+
+    def _map(self, jobs) -> int:
+        return sum(self.pool.map_async(_oracle_decode_worker, jobs, chunksize=1).get(timeout=600))
+
+    def decode_all(self) -> int:
+        return self._map(self.jobs)
+
+    def __exit__(self, *exc):
+        self.pool.terminate()
+        self.pool.join()
+        self.shm.close()
+        self.shm.unlink()
+        return False
+
+
 def cpu_baseline_all_cores(blobs, n_total: int):
     """The same oracle decoder, one tensor per worker process, on the host's
-    cores (spawned processes: no fork after the GPU was used). The blobs sit
-    in one shared-memory segment; timed from handing out the jobs to the last
-    result, with the workers already started."""
+    cores; timed with the workers already started."""
     import multiprocessing as mp
-    from multiprocessing import shared_memory
-    workers = max(1, min(os.cpu_count() or 1, len(blobs)))
-    total = sum(b.size for b in blobs)
-    shm = shared_memory.SharedMemory(create=True, size=max(1, total))
     try:
-        jobs, off = [], 0
-        for b in blobs:
-            np.ndarray((b.size,), dtype=np.uint8, buffer=shm.buf, offset=off)[:] = b
-            jobs.append((shm.name, off, b.size))
-            off += b.size
-        order = sorted(range(len(jobs)), key=lambda i: -jobs[i][2])   # largest first
-        ctx = mp.get_context("spawn")
-        with ctx.Pool(workers) as pool:   # leaving the block terminates the workers
-            try:
-                pool.map_async(_oracle_decode_worker, [jobs[order[-1]]] * workers, chunksize=1).get(timeout=600)
-                t0 = time.perf_counter()
-                n = sum(pool.map_async(_oracle_decode_worker, [jobs[i] for i in order], chunksize=1).get(timeout=600))
-                dt = time.perf_counter() - t0
-            except mp.TimeoutError:
-                return {"unavailable": "oracle worker processes did not finish within 600 s"}
-    finally:
-        shm.close()
-        shm.unlink()
+        with OraclePool(blobs) as pool:
+            t0 = time.perf_counter()
+            n = pool.decode_all()
+            dt = time.perf_counter() - t0
+            workers = pool.workers
+    except mp.TimeoutError:
+        return {"unavailable": "oracle worker processes did not finish within 600 s"}
     return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
             "sample": f"oracle bit-serial DFloat11 decode of the whole layer ({n:,} weights), one tensor per "
                       f"process on {workers} spawned workers (blobs in shared memory), {dt:.2f} s"}
@@ -727,29 +749,36 @@ def run_stress(args, rank, world, local_rank, dist):
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args):
-    """The CPU oracle as it stands, on this host, on a bounded sample of the
-    same workload (the layer's q matrix per step)."""
+    """The CPU oracle as it stands, on this host's cores: one step decodes the
+    whole layer, one tensor per spawned worker process (the q matrix alone
+    when more than 200 steps are asked for, to keep the run within minutes)."""
     from decode_dfloat11_b200 import build as lwc_build
     from decode_dfloat11_b200 import lwc
-    from oracle import df11 as odf
     lwc_build.build()
     names, tensors = make_layer(args.layer or 0)
-    d, blob = lwc.lwc_encode_dfloat11(tensors[0])
-    n = d.n
-    for _ in range(args.warmup):
-        odf.decode(blob)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        odf.decode(blob)
-    dt = (time.perf_counter() - t0) / args.steps
+    whole = args.steps + args.warmup <= 200
+    use = tensors if whole else tensors[:1]
+    blobs = [lwc.lwc_encode_dfloat11(t)[1] for t in use]
+    n = sum(t.size for t in use)
+    with OraclePool(blobs) as pool:
+        for _ in range(args.warmup):
+            pool.decode_all()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            pool.decode_all()
+        dt = (time.perf_counter() - t0) / args.steps
+        workers = pool.workers
     value = 2 * n / dt / 1e9
-    sample = f"oracle bit-serial DFloat11 decode of the layer's q matrix ({n:,} weights) per step, one host thread"
+    what = "the whole layer" if whole else "the layer's q matrix"
+    sample = (f"oracle bit-serial DFloat11 decode of {what} ({n:,} weights) per step, one tensor per process "
+              f"on {workers} spawned workers")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u16", "data": "synthetic",
-        "config": {"workload": "llama3-8b-layer-df11", "sample": "q matrix 4096x4096"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "config": {"workload": "llama3-8b-layer-df11", "sample": what},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
