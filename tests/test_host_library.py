@@ -258,6 +258,21 @@ def test_fused_linear_helper_checks_shapes_before_the_library():
         fused_linear(d, b, (16, 32), ok, "huffman")
 
 
+def test_header_is_plain_c(tmp_path):
+    # the boundary is a C ABI: include/lwc.h must compile as strict C99 (and C++)
+    import shutil
+    import subprocess
+    src = tmp_path / "use_lwc.c"
+    src.write_text('#include "lwc.h"\nint main(void) { lwc_desc d; (void)d; return (int)LWC_OK; }\n')
+    for cc, std in (("gcc", "-std=c99"), ("g++", "-std=c++17")):
+        if shutil.which(cc) is None:
+            pytest.skip(f"{cc} not installed")
+        lang = ["-x", "c++"] if cc == "g++" else []
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only", "-I",
+                            os.path.join(ROOT, "include"), *lang, str(src)], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
+
+
 def test_encoder_rejects_bad_arguments():
     w = np.zeros(10, np.uint16)
     for kw in (dict(chunk_bytes=6), dict(chunk_bytes=10), dict(threads_per_block=48),
