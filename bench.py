@@ -610,7 +610,7 @@ def model_units(which: str, device):
 
 
 def run_model(args, rank, world, local_rank, dist):
-    """configs 3 and 5: the whole model resident compressed in HBM; one step
+    """Whole models (Llama-3-8B or Llama-3-70B shapes) resident compressed in HBM; one step
     decodes every layer in order (one batched launch each) into two
     reusable BF16 buffers."""
     import torch
@@ -692,7 +692,7 @@ def run_model(args, rank, world, local_rank, dist):
 # ---------------------------------------------------------------- stress tensors
 
 def run_stress(args, rank, world, local_rank, dist):
-    """config 4: 256M-weight stress tensors, each generated and compressed on
+    """256M-weight stress tensors, each generated and compressed on
     the GPU and decoded K times: codebook tables of U = 256 / 4096 / 8192 /
     65536 entries with Zipf(1.1) frequencies (k = 8 / 12 / 13 / 16; also
     16384 and 32768 for k = 14 and 15), and the

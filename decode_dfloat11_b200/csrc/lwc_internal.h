@@ -18,7 +18,7 @@ constexpr uint32_t kHeaderBytes = 256;
 constexpr uint32_t kSectionAlign = 256;
 constexpr uint32_t kFlagSingleExponent = 1u;
 constexpr uint32_t kFormatMaxLen = 32;      // longest Huffman code the format allows
-constexpr uint32_t kMaxTables = 256;        // lookup tables this build stages in shared memory
+constexpr uint32_t kMaxTables = 256;        // lookup tables the decoders stage in shared memory
 
 // DFloat11 encoder defaults. Blocks of 32 chunks are decoded one per warp
 // (no CTA-wide barrier per block); a 36-byte chunk is an odd number of words,

@@ -70,7 +70,7 @@ typedef enum lwc_status {
     LWC_ERR_INVALID_ARG = 1,  /* NULL pointer, bad size or parameter */
     LWC_ERR_MISALIGNED = 2,   /* device pointer not 16-byte aligned */
     LWC_ERR_CORRUPT = 3,      /* blob header/descriptor inconsistent */
-    LWC_ERR_UNSUPPORTED = 4,  /* valid but outside what this build decodes */
+    LWC_ERR_UNSUPPORTED = 4,  /* valid but outside what this library decodes */
     LWC_ERR_NOMEM = 5,        /* host allocation failed (encoders) */
     LWC_ERR_CUDA = 6          /* CUDA runtime error at launch */
 } lwc_status;
