@@ -183,6 +183,7 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
         }
         // this warp's first two tiles of the run
         if (lane == 0 && !dead) {
+            dev::fence_proxy_async_smem();   // this warp's reads of its buffers come before the copies' writes
             if (warp < ns) issue_tile<K>(tn, s0 + warp, my_buf + (it & 1u) * (Lay::kTileBytes / 4), &my_bar[it & 1u]);
             if (warp + kWarps < ns)
                 issue_tile<K>(tn, s0 + warp + kWarps, my_buf + ((it + 1) & 1u) * (Lay::kTileBytes / 4),
@@ -474,8 +475,10 @@ __global__ void __launch_bounds__(kLinWarps * 32, K == 16 ? 1 : K >= 14 ? 2 : 3)
         uint32_t iq = 0, cq = 0, issued = 0;
         const uint64_t row_end = s0 + ns;
         for (; issued < 2 && ir < row_end; issued++) {   // the first two items
-            if (lane == 0 && !dead)
+            if (lane == 0 && !dead) {
+                dev::fence_proxy_async_smem();   // this warp's reads of the buffer come before the copy's writes
                 issue_window<K>(tn, ir, iq, my_buf + ((it + issued) & 1u) * kBufWords, &my_bar[(it + issued) & 1u]);
+            }
             if (++iq == nwin) { iq = 0; ir += kWarps; }
         }
         if (tn.stage_x) stage_activations(tn.x, M, tn.cols, nwin, xst);
