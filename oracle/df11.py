@@ -98,6 +98,41 @@ def chunk_index(code_lengths_per_weight: np.ndarray, total_bits: int, chunk_bits
     return n_chunks, n_blocks, gaps, blkoff
 
 
+def chunk_output_offsets(code_lengths_per_weight: np.ndarray, total_bits: int, chunk_bits: int,
+                         threads_per_block: int) -> np.ndarray:
+    """Per chunk, where its codes' outputs start inside its block: the number
+    of codes of the block that start before the chunk's first code (its gap).
+    This is the result of the two-phase decoder's first phase plus the block
+    scan (DFloat11 page, "Jak to działa w praktyce?": each thread first learns
+    how much it decodes, then writes at its place), i.e. what a blob would
+    store to let the decoder skip that phase. Chunks past the stream end get
+    their block's code count."""
+    n = code_lengths_per_weight.size
+    starts = np.zeros(n + 1, np.uint64)
+    np.cumsum(code_lengths_per_weight, dtype=np.uint64, out=starts[1:])
+    assert int(starts[-1]) == total_bits
+    n_chunks, n_blocks, _, blkoff = chunk_index(code_lengths_per_weight, total_bits, chunk_bits, threads_per_block)
+    first = np.full(n_blocks * threads_per_block, n, np.uint64)   # index of each chunk's first code
+    chunk_starts = np.arange(n_chunks, dtype=np.uint64) * np.uint64(chunk_bits)
+    first[:n_chunks] = np.searchsorted(starts[:n], chunk_starts, side="left")
+    block_of = np.arange(n_blocks * threads_per_block) // threads_per_block
+    first = np.minimum(first, blkoff[block_of + 1])
+    return (first - blkoff[block_of]).astype(np.uint32)
+
+
+def chunk_output_offsets_of_blob(blob: np.ndarray) -> np.ndarray:
+    """chunk_output_offsets for a DFloat11 blob, from its sequential decode."""
+    blob = np.asarray(blob, np.uint8)
+    h = B.unpack_header(blob)
+    if h["codec"] != B.CODEC_DFLOAT11:
+        raise ValueError("not a DFloat11 blob")
+    if h["total_bits"] == 0:
+        return np.zeros(0, np.uint32)
+    _, lens = decode_exponents(blob, h, want_lengths=True)
+    return chunk_output_offsets(np.asarray(lens, np.uint64), h["total_bits"], 8 * h["chunk_bytes"],
+                                h["threads_per_block"])
+
+
 def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
            threads_per_block: int = DEFAULT_THREADS_PER_BLOCK,
            max_len: int = DEFAULT_MAX_LEN, _elem: int = B.ELEM_BF16, _lo=None) -> np.ndarray:

@@ -177,3 +177,15 @@ def test_bf16_sign_dropped_is_caught(monkeypatch):
     monkeypatch.setattr(OL, "bf16_values", lambda b: np.abs(good(b)))
     fails(lpins.test_bf16_field_values)
     fails(lpins.test_golden_rectangular_example)
+
+
+def test_chunk_offsets_off_by_one_is_caught(monkeypatch):
+    good = df11.chunk_output_offsets
+
+    def bad(*a):
+        o = good(*a).copy()
+        o[1:] += 1
+        return o
+    monkeypatch.setattr(df11, "chunk_output_offsets", bad)
+    fails(pins.test_chunk_output_offsets_match_independent_chunk_decodes, 8, 32)
+    fails(pins.test_chunk_output_offsets_single_code_length)

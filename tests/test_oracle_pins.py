@@ -264,6 +264,51 @@ def test_chunks_decode_independently(chunk_bytes, tpb):
     assert np.array_equal(np.array(got, np.uint8), e_ref)
 
 
+@pytest.mark.parametrize("chunk_bytes,tpb", [(8, 32), (36, 32), (36, 64)])
+def test_chunk_output_offsets_match_independent_chunk_decodes(chunk_bytes, tpb):
+    """The per-chunk output offsets a blob could store (the first phase plus
+    the block scan, done once by the encoder) equal the running code count of
+    each block when every chunk is decoded on its own from its gap."""
+    w = synth.as_u16(synth.normal_bf16((30_000,), seed=23, sigma=0.02, outlier_frac=3e-3))
+    b = df11.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    h = B.unpack_header(b)
+    offs = df11.chunk_output_offsets_of_blob(b)
+    assert offs.size == h["n_blocks"] * tpb
+    lengths = [int(x) for x in B.section(b, h["off_lengths"], 256)]
+    words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
+    gaps = B.section(b, h["off_gaps"], h["n_blocks"] * tpb)
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    cb = 8 * chunk_bytes
+    for blk in range(h["n_blocks"]):
+        running = 0
+        for t in range(tpb):
+            c = blk * tpb + t
+            assert offs[c] == running, (blk, t)
+            if c * cb < h["total_bits"]:
+                running += len(decode_chunk(words, h["total_bits"], c * cb + int(gaps[c]),
+                                            min((c + 1) * cb, h["total_bits"]), lengths))
+        assert running == int(blkoff[blk + 1] - blkoff[blk])
+
+
+def test_chunk_output_offsets_single_code_length():
+    # all 16 exponents equally frequent: every code is 4 bits, so chunk c's
+    # first code is code ceil(c * cb / 4) and its offset is that minus the
+    # block's first code (closed form, no decode)
+    e = np.repeat(np.arange(120, 136, dtype=np.uint16), 1000)
+    w = ((np.random.default_rng(3).permutation(e) << 7) | 0x0011).astype(np.uint16)
+    for chunk_bytes, tpb in ((8, 32), (36, 64)):
+        b = df11.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+        h = B.unpack_header(b)
+        assert h["max_len"] == 4 and h["total_bits"] == 4 * w.size
+        offs = df11.chunk_output_offsets_of_blob(b)
+        cb = 8 * chunk_bytes
+        for c in range(offs.size):
+            blk = c // tpb
+            first = min(-(-c * cb // 4), w.size)
+            blk_first = min(-(-blk * tpb * cb // 4), w.size)
+            assert offs[c] == first - blk_first
+
+
 # ----------------------------------------------------- worked examples
 
 def test_golden_df11_worked_example():
