@@ -5,6 +5,7 @@
 from __future__ import annotations
 
 import argparse
+import concurrent.futures
 import os
 import shutil
 import subprocess
@@ -49,28 +50,28 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
     if not force and not ptxas_info and not stale():
         return LIB
     os.makedirs(BUILD, exist_ok=True)
-    objs = []
     common = ["-O3", "-std=c++17", "-I", INCLUDE, "-I", CSRC]
-    log = []
+    jobs = []   # (source, object, command), compiled in parallel
     for src in CUDA_SOURCES:
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
         cmd = [nvcc(), *ARCH, "-lineinfo", *common, "-Xcompiler", "-fPIC,-fvisibility=hidden",
                "--expt-relaxed-constexpr", "-c", os.path.join(CSRC, src), "-o", obj]
         if ptxas_info:
             cmd.insert(1, "-Xptxas=-v")
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        log.append(r.stdout + r.stderr)
-        if r.returncode != 0:
-            raise RuntimeError(f"nvcc failed on {src}:\n{r.stderr}")
-        objs.append(obj)
+        jobs.append((src, obj, cmd, "nvcc"))
     for src in CXX_SOURCES:
         obj = os.path.join(BUILD, src.replace(".cpp", ".o"))
         cmd = ["g++", "-O2", "-fPIC", "-fvisibility=hidden", "-Wall", *common, "-c",
                os.path.join(CSRC, src), "-o", obj]
-        r = subprocess.run(cmd, capture_output=True, text=True)
+        jobs.append((src, obj, cmd, "g++"))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(jobs)) as pool:
+        results = list(pool.map(lambda j: subprocess.run(j[2], capture_output=True, text=True), jobs))
+    log = []
+    objs = []
+    for (src, obj, _, tool), r in zip(jobs, results):
         log.append(r.stdout + r.stderr)
         if r.returncode != 0:
-            raise RuntimeError(f"g++ failed on {src}:\n{r.stderr}")
+            raise RuntimeError(f"{tool} failed on {src}:\n{r.stderr}")
         objs.append(obj)
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, "-lpthread"]
