@@ -51,7 +51,7 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
         return LIB
     os.makedirs(BUILD, exist_ok=True)
     common = ["-O3", "-std=c++17", "-I", INCLUDE, "-I", CSRC]
-    jobs = []   # (source, object, command), compiled in parallel
+    jobs = []   # (source, object, command, tool), compiled in parallel
     for src in CUDA_SOURCES:
         obj = os.path.join(BUILD, src.replace(".cu", ".o"))
         cmd = [nvcc(), *ARCH, "-lineinfo", *common, "-Xcompiler", "-fPIC,-fvisibility=hidden",
