@@ -89,3 +89,35 @@ def test_swizzle_is_bank_conflict_free_per_quarter_warp():
         for quarter in range(4):
             groups = {(4 * l + ((i + (l >> 1)) & 3)) % 8 for l in range(8 * quarter, 8 * quarter + 8)}
             assert len(groups) == 8
+
+
+def magic_for(d):
+    """division_magic in csrc/lwc_df11.cu: l = ceil(log2 d), m' = floor(2^32 (2^l - d) / d) + 1."""
+    l = 0
+    while (1 << l) < d:
+        l += 1
+    return (((1 << l) - d) << 32) // d + 1, min(l, 1), max(l - 1, 0)
+
+
+def div_cols(n, d):
+    """div_cols in csrc/lwc_df11.cu: t = umulhi(m', n), q = (t + ((n - t) >> sh1)) >> sh2."""
+    m, sh1, sh2 = magic_for(d)
+    t = (m * n) >> 32
+    return (t + ((n - t) >> sh1)) >> sh2
+
+
+def test_division_by_cols_is_exact_for_every_32_bit_numerator():
+    # Granlund and Montgomery's unsigned division by an invariant, as the
+    # DFloat11 linear kernel uses it for rows and columns: exact for all
+    # n < 2^32 and 1 <= d < 2^31, and m' fits 32 bits
+    rng = np.random.default_rng(0)
+    divisors = list(range(1, 70)) + [127, 128, 129, 1040, 4096, 4099, 8192, 14336, 28672, (1 << 30) + 1,
+                                     (1 << 31) - 1] + [int(x) for x in rng.integers(1, 1 << 31, 200)]
+    for d in divisors:
+        m, _, _ = magic_for(d)
+        assert 0 < m < 1 << 32
+        ns = [0, 1, d - 1, d, d + 1, 2 * d - 1, (1 << 32) - 1, (1 << 32) - d, (1 << 31)]
+        ns += [int(x) for x in rng.integers(0, 1 << 32, 50)]
+        for n in ns:
+            if 0 <= n < 1 << 32:
+                assert div_cols(n, d) == n // d, (n, d)
