@@ -5,7 +5,9 @@ window buffer, and covers every bit a lane's fields need; every lane's word
 reads stay inside the buffer; the swizzled activation slots stay inside the
 staged region and are a permutation within each window (no two chunks share
 a slot). The constants and formulas mirror csrc/lwc_codebook.cu
-(issue_window, the re-alignment in cb_linear_kernel, stage_activations)."""
+(issue_window, the re-alignment in cb_linear_kernel, stage_activations).
+Also the multiply-shift division by cols of the DFloat11 linear kernel
+(csrc/lwc_df11.cu: division_magic, div_cols), exact over its range."""
 import numpy as np
 import pytest
 
