@@ -232,43 +232,56 @@ def cpu_baseline(blobs, n_total: int):
 
 
 def _oracle_decode_worker(job) -> int:
-    """Decode one blob that sits in a shared-memory segment: (name, offset, size)."""
+    """Decode one piece of a blob that sits in a shared-memory segment:
+    (segment name, offset, size, first block, end block); a block range of
+    (0, 0) means the whole blob."""
     from multiprocessing import shared_memory
 
     from oracle import df11 as odf
-    name, off, size = job
+    name, off, size, b0, b1 = job
     shm = shared_memory.SharedMemory(name=name)
     try:
         blob = np.ndarray((size,), dtype=np.uint8, buffer=shm.buf, offset=off)
-        odf.decode(blob)
-        n = int(odf.B.unpack_header(blob)["n"])
+        n = (odf.decode(blob) if (b0, b1) == (0, 0) else odf.decode_blocks(blob, b0, b1)).size
         del blob
     finally:
         shm.close()
-    return n
+    return int(n)
 
 
 class OraclePool:
-    """Spawned worker processes (no fork after the GPU was used) that decode
-    blobs with the oracle, one blob per task; the blobs sit in one
-    shared-memory segment. ``decode_all()`` decodes every blob once and
+    """Spawned worker processes (no fork after the GPU was used), one per host
+    core, that decode blobs with the oracle; the blobs sit in one
+    shared-memory segment and each task is a range of a blob's blocks (about
+    four tasks per worker), which the stored block offsets and gaps let any
+    process decode on its own. ``decode_all()`` decodes every blob once and
     returns the weight count; waits are bounded."""
 
     def __init__(self, blobs):
         self.blobs = blobs
-        self.workers = max(1, min(os.cpu_count() or 1, len(blobs)))
+        self.workers = max(1, os.cpu_count() or 1)
 
     def __enter__(self):
         import multiprocessing as mp
         from multiprocessing import shared_memory
+
+        from oracle import blob as OB
         total = sum(b.size for b in self.blobs)
         self.shm = shared_memory.SharedMemory(create=True, size=max(1, total))
+        weights = [int(OB.unpack_header(b)["n"]) for b in self.blobs]
+        piece = max(1, sum(weights) // (4 * self.workers))   # about 4 pieces per worker
         jobs, off = [], 0
-        for b in self.blobs:
+        for b, n in zip(self.blobs, weights):
             np.ndarray((b.size,), dtype=np.uint8, buffer=self.shm.buf, offset=off)[:] = b
-            jobs.append((self.shm.name, off, b.size))
+            nb = int(OB.unpack_header(b).get("n_blocks", 0) or 0)
+            if nb == 0:
+                jobs.append((n, (self.shm.name, off, b.size, 0, 0)))
+            else:   # block ranges of about `piece` weights, decoded independently
+                k = max(1, min(nb, -(-n // piece)))
+                cuts = [nb * i // k for i in range(k + 1)]
+                jobs += [(n * (y - x) // nb, (self.shm.name, off, b.size, x, y)) for x, y in zip(cuts, cuts[1:])]
             off += b.size
-        self.jobs = sorted(jobs, key=lambda j: -j[2])   # largest first
+        self.jobs = [j for _, j in sorted(jobs, key=lambda t: -t[0])]   # largest first
         self.pool = mp.get_context("spawn").Pool(self.workers)
         self._map([self.jobs[-1]] * self.workers)          # start the workers, import the oracle
         return self
@@ -300,8 +313,8 @@ def cpu_baseline_all_cores(blobs, n_total: int):
     except mp.TimeoutError:
         return {"unavailable": "oracle worker processes did not finish within 600 s"}
     return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
-            "sample": f"oracle bit-serial DFloat11 decode of the whole layer ({n:,} weights), one tensor per "
-                      f"process on {workers} spawned workers (blobs in shared memory), {dt:.2f} s"}
+            "sample": f"oracle bit-serial DFloat11 decode of the whole layer ({n:,} weights) in block ranges "
+                      f"on {workers} spawned workers (blobs in shared memory), {dt:.2f} s"}
 
 
 # ---------------------------------------------------------------- our arm
@@ -770,8 +783,8 @@ def run_reference(args):
         workers = pool.workers
     value = 2 * n / dt / 1e9
     what = "the whole layer" if whole else "the layer's q matrix"
-    sample = (f"oracle bit-serial DFloat11 decode of {what} ({n:,} weights) per step, one tensor per process "
-              f"on {workers} spawned workers")
+    sample = (f"oracle bit-serial DFloat11 decode of {what} ({n:,} weights) per step, in block ranges on "
+              f"{workers} spawned workers")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,

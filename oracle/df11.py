@@ -245,6 +245,48 @@ def decode(blob: np.ndarray) -> np.ndarray:
     return merge(e, np.ascontiguousarray(sm))
 
 
+def decode_blocks(blob: np.ndarray, b0: int, b1: int) -> np.ndarray:
+    """Weights blkoff[b0] .. blkoff[b1] of a DFloat11 blob, decoded bit-serially
+    from the first code of block b0 (its chunk's gap) without touching the
+    blocks before it: the independence the stored block offsets and gaps give
+    (DFloat11 page, "Jak to działa w praktyce?"), used to spread the decode of
+    one tensor over several processes."""
+    blob = np.asarray(blob, np.uint8)
+    h = B.unpack_header(blob)
+    if h["codec"] != B.CODEC_DFLOAT11:
+        raise ValueError("not a DFloat11 blob")
+    if h["flags"] & B.FLAG_SINGLE_EXPONENT or h["n"] == 0:
+        if (b0, b1) != (0, 0):
+            raise ValueError("a blob without a stream has no blocks")
+        return decode(blob)
+    if not 0 <= b0 <= b1 <= h["n_blocks"]:
+        raise ValueError("block range outside the blob")
+    T, cb = h["threads_per_block"], 8 * h["chunk_bytes"]
+    blkoff = B.section(blob, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    gaps = B.section(blob, h["off_gaps"], h["n_blocks"] * T)
+    i0, i1 = int(blkoff[b0]), int(blkoff[b1])
+    if i1 == i0:
+        return np.zeros(0, np.uint16)
+    _, lengths = _parts(blob, h)
+    first, cnt, base, sorted_syms = H.decode_tables(lengths)
+    words = B.section(blob, h["off_stream"], h["stream_bytes"], np.uint32)
+    e = np.empty(i1 - i0, np.uint8)
+    f = np.array(first, np.uint32)
+    c = np.array(cnt, np.uint32)
+    bb = np.array(base, np.uint32)
+    ss = np.array(sorted_syms + [0], np.uint8)
+    end = ctypes.c_uint64(0)
+    start = b0 * T * cb + int(gaps[b0 * T])
+    rc = lib().orc_df11_decode_syms(ptr(words, ctypes.c_uint32), h["total_bits"], start, i1 - i0,
+                                    ptr(f, ctypes.c_uint32), ptr(c, ctypes.c_uint32),
+                                    ptr(bb, ctypes.c_uint32), ptr(ss, ctypes.c_uint8), 32,
+                                    ptr(e, ctypes.c_uint8), None, ctypes.byref(end))
+    if rc != 0:
+        raise ValueError(f"corrupt stream (code {rc} at bit {end.value})")
+    sm, _ = _parts(blob, h)
+    return merge(e, np.ascontiguousarray(sm[i0:i1]))
+
+
 # ---------------------------------------------------------------- FP32 and FP16
 #
 # The DFloat11 idea carried to the other float formats: entropy-code the

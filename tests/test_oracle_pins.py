@@ -309,6 +309,26 @@ def test_chunk_output_offsets_single_code_length():
             assert offs[c] == first - blk_first
 
 
+@pytest.mark.parametrize("chunk_bytes,tpb", [(8, 64), (36, 32), (36, 256)])
+def test_block_ranges_decode_independently(chunk_bytes, tpb):
+    """Any split of a blob's blocks into ranges, each decoded from its own
+    first gap, concatenates to the whole tensor (what lets one tensor's decode
+    be spread over processes)."""
+    w = synth.as_u16(synth.normal_bf16((120_007,), seed=31, sigma=0.02, outlier_frac=2e-3))
+    b = df11.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    nb = B.unpack_header(b)["n_blocks"]
+    rng = np.random.default_rng(tpb)
+    for _ in range(3):
+        cuts = sorted({0, nb, *rng.integers(0, nb + 1, 4).tolist()})
+        parts = [df11.decode_blocks(b, x, y) for x, y in zip(cuts[:-1], cuts[1:])]
+        assert np.array_equal(np.concatenate(parts), w)
+    assert df11.decode_blocks(b, 3, 3).size == 0
+    with pytest.raises(ValueError):
+        df11.decode_blocks(b, 2, nb + 1)
+    single = np.full(1000, 0x3C12, np.uint16)
+    assert np.array_equal(df11.decode_blocks(df11.encode(single), 0, 0), single)
+
+
 # ----------------------------------------------------- worked examples
 
 def test_golden_df11_worked_example():
