@@ -259,7 +259,11 @@ class OraclePool:
 
     def __init__(self, blobs):
         self.blobs = blobs
-        self.workers = max(1, os.cpu_count() or 1)
+        try:   # the cores this process may run on (a container's CPU set), at most 32 workers
+            cores = len(os.sched_getaffinity(0))
+        except AttributeError:
+            cores = os.cpu_count() or 1
+        self.workers = max(1, min(cores, 32))
 
     def __enter__(self):
         import multiprocessing as mp
