@@ -18,6 +18,7 @@ VERSION = 1
 CODEC_DFLOAT11 = 1
 CODEC_CODEBOOK = 2
 FLAG_SINGLE_EXPONENT = 1
+FLAG_CHUNK_COUNTS = 2         # DFloat11: a u8 code count per chunk is stored ("counts")
 ELEM_BF16 = 0   # DFloat11 element types (header field "elem")
 ELEM_FP32 = 1
 ELEM_FP16 = 2
@@ -36,6 +37,7 @@ DF11 = (
     ("off_lengths", 80, "Q"), ("off_lut", 88, "Q"), ("off_gaps", 96, "Q"),
     ("off_blkoff", 104, "Q"), ("off_stream", 112, "Q"), ("stream_bytes", 120, "Q"),
     ("off_sm", 128, "Q"), ("elem", 136, "I"), ("off_lo", 144, "Q"), ("lo_bytes", 152, "Q"),
+    ("off_counts", 160, "Q"),
 )
 CODEBOOK = (
     ("U", 32, "I"), ("k", 36, "I"), ("off_table", 40, "Q"), ("off_packed", 48, "Q"),

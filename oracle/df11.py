@@ -16,7 +16,10 @@ Follows "Koniec z kompromisami! DFloat11 ratuje dokładność modeli AI ..."
   after a synchronisation, write it at the right place. For that the blob
   carries, per fixed-size chunk of the bitstream, the offset of the first code
   that starts in it (``gaps``) and, per block of chunks, the index of the first
-  weight it decodes (``blkoff``).
+  weight it decodes (``blkoff``). Optionally (``chunk_counts``) it also
+  carries, per chunk, the number of codes that start in it (``counts``):
+  the result of the first phase, worked out once by the encoder, so that a
+  decoder can go straight to the scan and the writing phase.
 
 Encoding steps, in the order the pages give them: split each weight into its
 exponent and its sign|mantissa byte; count exponents; build the Huffman code
@@ -133,11 +136,41 @@ def chunk_output_offsets_of_blob(blob: np.ndarray) -> np.ndarray:
                                 h["threads_per_block"])
 
 
+def chunk_code_counts(code_lengths_per_weight: np.ndarray, total_bits: int, chunk_bits: int,
+                      threads_per_block: int) -> np.ndarray:
+    """Per chunk, the number of codes that start in it: #{i < n : c*chunk_bits
+    <= starts[i] < (c+1)*chunk_bits}, starts[i] being the exclusive prefix sum
+    of the code lengths. This is what each thread finds in the first phase of
+    the two-phase decoder (DFloat11 page, "Jak to działa w praktyce?": threads
+    first learn how much they will decode). The array covers n_blocks *
+    threads_per_block chunks; chunks at or past the stream end count 0."""
+    n = code_lengths_per_weight.size
+    starts = np.zeros(n + 1, np.uint64)
+    np.cumsum(code_lengths_per_weight, dtype=np.uint64, out=starts[1:])
+    assert int(starts[-1]) == total_bits
+    n_chunks = -(-total_bits // chunk_bits)
+    n_blocks = -(-n_chunks // threads_per_block)
+    chunk_of = (starts[:n] // np.uint64(chunk_bits)).astype(np.int64)
+    return np.bincount(chunk_of, minlength=n_blocks * threads_per_block).astype(np.uint64)
+
+
+def counts_fit_in_bytes(lengths, chunk_bits: int) -> bool:
+    """Whether every per-chunk code count fits in a byte for this code: codes
+    are at least min_len bits long, so at most ceil(chunk_bits / min_len) of
+    them start in one chunk."""
+    present = [l for l in lengths if l > 0]
+    return bool(present) and -(-chunk_bits // min(present)) <= 255
+
+
 def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
            threads_per_block: int = DEFAULT_THREADS_PER_BLOCK,
-           max_len: int = DEFAULT_MAX_LEN, _elem: int = B.ELEM_BF16, _lo=None) -> np.ndarray:
+           max_len: int = DEFAULT_MAX_LEN, _elem: int = B.ELEM_BF16, _lo=None,
+           chunk_counts: bool = True) -> np.ndarray:
     """Compress BF16 bit patterns into a DFloat11 blob (uint8 array).
 
+    With ``chunk_counts`` the blob also stores each chunk's code count (a
+    byte per chunk, flag FLAG_CHUNK_COUNTS) whenever every count fits in a
+    byte (``counts_fit_in_bytes``); otherwise it is left out.
     (``_elem`` / ``_lo`` are used by ``encode_elements`` for FP32 and FP16:
     the element type recorded in the header and the low-mantissa section.)"""
     if chunk_bytes % 4 or chunk_bytes < 8 or threads_per_block % 32 or not 32 <= threads_per_block <= 1024:
@@ -180,12 +213,20 @@ def encode(w: np.ndarray, chunk_bytes: int = DEFAULT_CHUNK_BYTES,
     chunk_bits = 8 * chunk_bytes
     n_chunks, n_blocks, gaps, blkoff = chunk_index(len_arr[e], total_bits, chunk_bits,
                                                    threads_per_block)
-    header.update(flags=0, max_len=max(lengths), n_tables=len(tables), n_chunks=n_chunks,
+    with_counts = chunk_counts and counts_fit_in_bytes(lengths, chunk_bits)
+    header.update(flags=B.FLAG_CHUNK_COUNTS if with_counts else 0, max_len=max(lengths),
+                  n_tables=len(tables), n_chunks=n_chunks,
                   n_blocks=n_blocks, total_bits=total_bits,
                   max_block_count=int(np.diff(blkoff).max()), const_exp=0,
                   stream_bytes=stream_bytes)
+    count_sections = []
+    if with_counts:
+        counts = chunk_code_counts(len_arr[e], total_bits, chunk_bits, threads_per_block)
+        assert int(counts.max()) <= 255
+        count_sections = [("counts", counts.astype(np.uint8))]
     sections = [("lengths", len_arr), ("lut", np.array(tables, np.uint16).reshape(-1)),
-                ("gaps", gaps), ("blkoff", blkoff), ("stream", words), ("sm", sm)] + lo_sections
+                ("gaps", gaps)] + count_sections + [("blkoff", blkoff), ("stream", words),
+                                                    ("sm", sm)] + lo_sections
     return B.assemble(header, sections)
 
 
@@ -393,8 +434,9 @@ def decode_elements(blob: np.ndarray) -> np.ndarray:
 
 
 def check_index(blob: np.ndarray) -> list[str]:
-    """Re-derive gaps, blkoff, max_block_count and the lookup tables of a blob
-    from its sequential decode and code lengths; list every disagreement."""
+    """Re-derive gaps, blkoff, max_block_count, the per-chunk code counts (if
+    stored) and the lookup tables of a blob from its sequential decode and
+    code lengths; list every disagreement."""
     blob = np.asarray(blob, np.uint8)
     h = B.unpack_header(blob)
     problems = []
@@ -416,6 +458,10 @@ def check_index(blob: np.ndarray) -> list[str]:
         problems.append("blkoff")
     if int(np.diff(blkoff).max()) != h["max_block_count"]:
         problems.append("max_block_count")
+    if h["flags"] & B.FLAG_CHUNK_COUNTS:
+        stored_counts = B.section(blob, h["off_counts"], n_blocks * T)
+        if not np.array_equal(stored_counts.astype(np.uint64), chunk_code_counts(lens, h["total_bits"], 8 * C, T)):
+            problems.append("counts")
     _, lengths = _parts(blob, h)
     if max(lengths) != h["max_len"]:
         problems.append("max_len")

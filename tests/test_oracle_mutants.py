@@ -64,6 +64,19 @@ def test_gap_off_by_one_is_caught(monkeypatch):
     fails(pins.test_golden_df11_periodic_offsets)
 
 
+def test_chunk_counts_by_code_end_is_caught(monkeypatch):
+    def bad(lens, total_bits, chunk_bits, tpb):
+        # counts the codes that end in each chunk instead of those that start there
+        ends = np.cumsum(np.asarray(lens, np.uint64), dtype=np.uint64)
+        n_blocks = -(-(-(-total_bits // chunk_bits)) // tpb)
+        chunk_of = ((ends - np.uint64(1)) // np.uint64(chunk_bits)).astype(np.int64)
+        return np.bincount(chunk_of, minlength=n_blocks * tpb).astype(np.uint64)
+    monkeypatch.setattr(df11, "chunk_code_counts", bad)
+    fails(pins.test_golden_df11_periodic_offsets)
+    fails(pins.test_chunk_counts_match_independent_chunk_decodes, 8, 32)
+    fails(pins.test_chunk_counts_single_code_length)
+
+
 def test_dropped_sign_is_caught(monkeypatch):
     good = df11.merge
     monkeypatch.setattr(df11, "merge", lambda e, s: good(e, s & np.uint8(0x7F)))

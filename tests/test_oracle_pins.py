@@ -84,7 +84,10 @@ def test_uniform_exponents_maximal_spread():
     counts, lengths, _ = df11.code_for(w)
     assert H.entropy_bits(counts) > 7.99
     assert all(l in (7, 8, 9) for l in lengths)
-    assert 15.9 < df11.bits_per_weight(b) < 16.3
+    # 8 raw bits + 8 code bits, plus a gap byte and a count byte per 36-byte
+    # chunk of 36 codes (2 x 8/36 = 0.44 bits), the block offsets and the
+    # 256-byte section alignment (about 0.05 bits at this size)
+    assert 15.9 < df11.bits_per_weight(b) < 16.6
 
 
 # ------------------------------------------------------- code properties
@@ -309,6 +312,66 @@ def test_chunk_output_offsets_single_code_length():
             assert offs[c] == first - blk_first
 
 
+@pytest.mark.parametrize("chunk_bytes,tpb", [(8, 32), (36, 32), (36, 64)])
+def test_chunk_counts_match_independent_chunk_decodes(chunk_bytes, tpb):
+    """The per-chunk code counts a blob stores equal the number of codes each
+    chunk yields when it is decoded on its own, from its gap up to the next
+    chunk's first code (what each thread of the two-phase decoder counts in
+    the first phase), and each block's counts add up to its stored offsets."""
+    w = synth.as_u16(synth.normal_bf16((30_000,), seed=29, sigma=0.02, outlier_frac=3e-3))
+    b = df11.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+    h = B.unpack_header(b)
+    assert h["flags"] & B.FLAG_CHUNK_COUNTS
+    counts = B.section(b, h["off_counts"], h["n_blocks"] * tpb)
+    lengths = [int(x) for x in B.section(b, h["off_lengths"], 256)]
+    words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
+    gaps = B.section(b, h["off_gaps"], h["n_blocks"] * tpb)
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    cb, tb = 8 * chunk_bytes, h["total_bits"]
+    for c in range(h["n_blocks"] * tpb):
+        got = len(decode_chunk(words, tb, c * cb + int(gaps[c]), min((c + 1) * cb, tb), lengths)) \
+            if c * cb < tb else 0
+        assert counts[c] == got, c
+    sums = counts.astype(np.int64).reshape(-1, tpb).sum(axis=1)
+    assert np.array_equal(sums, np.diff(blkoff.astype(np.int64)))
+
+
+def test_chunk_counts_single_code_length():
+    # all 16 exponents equally frequent: every code is 4 bits, so the codes
+    # that start in chunk c are the multiples of 4 in [c cb, min((c+1) cb, TB)):
+    # ceil(min((c+1) cb, TB) / 4) - ceil(c cb / 4) of them (closed form, no decode)
+    e = np.repeat(np.arange(120, 136, dtype=np.uint16), 1000)
+    w = ((np.random.default_rng(5).permutation(e) << 7) | 0x0033).astype(np.uint16)
+    for chunk_bytes, tpb in ((8, 32), (20, 32), (36, 64)):
+        b = df11.encode(w, chunk_bytes=chunk_bytes, threads_per_block=tpb)
+        h = B.unpack_header(b)
+        assert h["max_len"] == 4 and h["flags"] & B.FLAG_CHUNK_COUNTS
+        counts = B.section(b, h["off_counts"], h["n_blocks"] * tpb)
+        cb, tb = 8 * chunk_bytes, h["total_bits"]
+        for c in range(counts.size):
+            lo, hi = min(c * cb, tb), min((c + 1) * cb, tb)
+            assert counts[c] == -(-hi // 4) - -(-lo // 4), c
+
+
+def test_chunk_counts_only_when_they_fit_a_byte():
+    # exponent 126 in 3/4 of the weights gets a 1-bit code, so up to 288 codes
+    # can start in a 288-bit chunk: more than a byte counts, and the counts
+    # are left out; in 64-bit chunks at most 64 start, and they are stored
+    rng = np.random.default_rng(6)
+    e = rng.choice(np.array([126, 125, 127], np.uint16), size=20_000, p=[0.75, 0.125, 0.125])
+    w = ((e << 7) | rng.integers(0, 256, e.size, dtype=np.uint16) & 0x807F).astype(np.uint16)
+    lengths = df11.code_for(w)[1]
+    assert min(l for l in lengths if l) == 1
+    wide = df11.encode(w, chunk_bytes=36, threads_per_block=32)
+    assert not B.unpack_header(wide)["flags"] & B.FLAG_CHUNK_COUNTS
+    narrow = df11.encode(w, chunk_bytes=8, threads_per_block=32)
+    assert B.unpack_header(narrow)["flags"] & B.FLAG_CHUNK_COUNTS
+    assert df11.check_index(narrow) == [] and np.array_equal(df11.decode(narrow), w)
+    off = df11.encode(w, chunk_bytes=8, threads_per_block=32, chunk_counts=False)
+    assert not B.unpack_header(off)["flags"] & B.FLAG_CHUNK_COUNTS
+    assert np.array_equal(df11.decode(off), w)
+
+
 @pytest.mark.parametrize("chunk_bytes,tpb", [(8, 64), (36, 32), (36, 256)])
 def test_block_ranges_decode_independently(chunk_bytes, tpb):
     """Any split of a blob's blocks into ranges, each decoded from its own
@@ -371,6 +434,12 @@ def test_golden_df11_periodic_offsets():
         nxt = min(x for x in starts if x >= c * cb)
         assert gaps[c] == nxt - c * cb
     assert np.all(gaps[p["n_chunks"]:] == 0)
+    # per-chunk code counts: the first three by hand, all from the period structure
+    assert h["flags"] & B.FLAG_CHUNK_COUNTS
+    counts = B.section(b, h["off_counts"], h["n_blocks"] * p["threads_per_block"])
+    assert counts[:3].tolist() == p["counts_first3"]
+    for c in range(counts.size):
+        assert counts[c] == sum(1 for x in starts[:-1] if c * cb <= x < (c + 1) * cb)
 
 
 def test_golden_clrs_huffman():
