@@ -1155,7 +1155,6 @@ lwc_status device_config(DeviceConfig &out) {
     return LWC_OK;
 }
 
-uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // The decode kernel for an element type and block shape, and its launch.
 template <int E>

@@ -61,13 +61,14 @@ struct WsHeader {
     uint64_t total_bits;       // written by the scan
     uint32_t max_block_count;  // written by the last pass
     uint32_t elem;             // LWC_ELEM_* of the source
+    uint32_t chunk_counts;     // store per-chunk code counts when they fit a byte
 };
 static_assert(sizeof(WsHeader) <= kWsCounts, "workspace header too large");
 
-uint64_t n_tiles_of(uint64_t n) { return (n + kTile - 1) / kTile; }
-uint64_t ws_tile_pos_off(uint64_t n) { return kWsArrays + round_up(4 * n_tiles_of(n), 256); }
+constexpr uint64_t n_tiles_of(uint64_t n) { return (n + kTile - 1) / kTile; }
+constexpr uint64_t ws_tile_pos_off(uint64_t n) { return kWsArrays + round_up(4 * n_tiles_of(n), 256); }
 
-uint64_t workspace_bytes(uint64_t n) {
+constexpr uint64_t workspace_bytes(uint64_t n) {
     const uint64_t df11 = ws_tile_pos_off(n) + 8 * (n_tiles_of(n) + 1);
     const uint64_t cb = kWsArrays + 2 * 65536;
     return round_up(std::max(df11, cb), 256);
@@ -267,6 +268,7 @@ struct EmitArgs {
     uint32_t *stream;
     uint64_t stream_words;  // words that hold code bits: ceil(total_bits / 32)
     uint8_t *gaps;
+    uint32_t *counts;       // per-chunk code counts as bytes of u32 words (zeroed first), or null
     uint64_t n_chunks;
     uint64_t chunk_bits;
     uint64_t *blkoff;
@@ -288,7 +290,10 @@ __device__ __forceinline__ uint32_t sm_byte(uint32_t w, int hi) {
 // crosses a chunk start gives that chunk's gap (bits from the chunk start to
 // the next code); one that crosses a block start gives that block's first
 // weight index. Codes are at most 32 bits and chunks at least 64, so a code
-// crosses at most one chunk start.
+// crosses at most one chunk start. With per-chunk code counts, each thread
+// counts its codes per chunk and adds each chunk's part to that chunk's byte
+// (an atomic add on the byte's word: the plan guarantees that no chunk holds
+// more than 255 codes, so no carry reaches the next byte).
 template <int E>
 __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, CodeTable t) {
     __shared__ uint64_t s_lc[256];
@@ -342,8 +347,14 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
             uint64_t ci = s_div[0] + xc / cbits + 1, bi = s_div[2] + xb / bbits + 1;
             uint32_t next_c = cbits - xc % cbits, next_b = bbits - xb % bbits, rel = 0;
             uint64_t acc = 0;
-            uint32_t nacc = o0 & 31, wi = o0 >> 5;
+            uint32_t nacc = o0 & 31, wi = o0 >> 5, run = 0;
             bool first = true;
+            // adds this thread's run of codes to the count of chunk ci - 1, where they start
+            auto flush = [&]() {
+                if (a.counts && run && ci - 1 < a.n_chunks)
+                    atomicAdd(&a.counts[(ci - 1) >> 2], run << (8u * (uint32_t)((ci - 1) & 3)));
+                run = 0;
+            };
 #pragma unroll
             for (uint32_t j = 0; j < kPerThread; j++) {
                 if (j >= cnt) break;
@@ -364,8 +375,10 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
                     first = false;
                 }
                 const uint32_t end = rel + l;
+                run++;
                 if (end >= next_c) {
                     if (ci < a.n_chunks) a.gaps[ci] = (uint8_t)(end - next_c);
+                    flush();
                     ci++;
                     next_c += cbits;
                 }
@@ -377,6 +390,7 @@ __global__ void __launch_bounds__(kTileThreads) df11_emit_kernel(EmitArgs a, Cod
                 rel = end;
             }
             if (nacc) atomicOr(&s_words[wi], (uint32_t)(acc << (32 - nacc)));
+            flush();
             if (i0 + cnt == a.n) a.blkoff[a.n_blocks] = a.n;
         }
         __syncthreads();
@@ -722,8 +736,8 @@ template <int E>
 lwc_status write_dfloat11(const void *src, uint64_t n, const WsHeader &h, const uint64_t *counts,
                           uint8_t *work, uint8_t *blob, uint64_t blob_bytes, lwc_desc *desc_out, cudaStream_t s) {
     Df11Plan plan;
-    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan,
-                                      lo_section_bytes(E, n)))
+    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, h.chunk_counts != 0,
+                                      plan, lo_section_bytes(E, n)))
         return st;
     plan.d.elem = E;
     lwc_desc &d = plan.d;
@@ -756,7 +770,9 @@ lwc_status write_dfloat11(const void *src, uint64_t n, const WsHeader &h, const 
     LWC_CUDA(cudaMemcpyAsync(blob + d.off_lengths, lengths, 256, cudaMemcpyHostToDevice, s), "lengths write");
     LWC_CUDA(cudaMemcpyAsync(blob + d.off_lut, plan.tables.data(), 2 * plan.tables.size(), cudaMemcpyHostToDevice, s),
              "lookup table write");
-    // bytes no pass writes: unused chunk gaps, padding, the stream's tail
+    // bytes no pass writes: unused chunk gaps, padding, the stream's tail (the
+    // range after the gaps also clears the chunk counts, which lie between
+    // the gaps and the block offsets and are accumulated by atomic adds)
     if (lwc_status st = zero(blob, d.off_lengths + 256, d.off_lut, s)) return st;
     if (lwc_status st = zero(blob, d.off_lut + 2 * plan.tables.size(), d.off_gaps, s)) return st;
     if (lwc_status st = zero(blob, d.off_gaps + d.n_chunks, d.off_blkoff, s)) return st;
@@ -781,6 +797,7 @@ lwc_status write_dfloat11(const void *src, uint64_t n, const WsHeader &h, const 
     a.stream = stream;
     a.stream_words = stream_words;
     a.gaps = blob + d.off_gaps;
+    a.counts = (d.flags & kFlagChunkCounts) ? reinterpret_cast<uint32_t *>(blob + d.off_counts) : nullptr;
     a.n_chunks = d.n_chunks;
     a.chunk_bits = 8ull * d.chunk_bytes;
     a.blkoff = reinterpret_cast<uint64_t *>(blob + d.off_blkoff);
@@ -867,6 +884,7 @@ lwc_status lwc_encode_dfloat11_elements_device_plan(const void *d_src, uint64_t 
     h.chunk_bytes = params ? params->chunk_bytes : kDefaultChunkBytes;
     h.threads_per_block = params ? params->threads_per_block : kDefaultThreadsPerBlock;
     h.max_len = params ? params->max_len : kDefaultMaxLen;
+    h.chunk_counts = params ? (params->chunk_counts != 0) : kDefaultChunkCounts;
     if (lwc_status st = check_df11_params(h.chunk_bytes, h.threads_per_block, h.max_len)) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *work = static_cast<uint8_t *>(d_work);
@@ -891,8 +909,8 @@ lwc_status lwc_encode_dfloat11_elements_device_plan(const void *d_src, uint64_t 
     WsHeader r;
     if (lwc_status st = fetch_header(work, r, counts, sizeof counts, s)) return st;
     Df11Plan plan;
-    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, plan,
-                                      lo_section_bytes(elem, n)))
+    if (lwc_status st = plan_dfloat11(counts, n, h.chunk_bytes, h.threads_per_block, h.max_len, h.chunk_counts != 0,
+                                      plan, lo_section_bytes(elem, n)))
         return st;
     plan.d.elem = elem;
     *desc_out = plan.d;
@@ -987,12 +1005,8 @@ namespace lwc {
 namespace {
 
 constexpr uint64_t kNoAllocMaxN = 1ull << 30;   // weights; every matrix of Llama-3-8B/70B fits
-static_assert(3154432 == (kWsArrays + ((4 * ((kNoAllocMaxN + kTile - 1) / kTile) + 255) / 256) * 256 +
-                          8 * ((kNoAllocMaxN + kTile - 1) / kTile + 1) + 255) / 256 * 256,
-              "the scratch size stated in lwc.h");
-constexpr uint64_t kNoAllocScratchBytes =
-    (kWsArrays + ((4 * ((kNoAllocMaxN + kTile - 1) / kTile) + 255) / 256) * 256 +
-     8 * ((kNoAllocMaxN + kTile - 1) / kTile + 1) + 255) / 256 * 256;   // workspace_bytes(kNoAllocMaxN)
+constexpr uint64_t kNoAllocScratchBytes = workspace_bytes(kNoAllocMaxN);
+static_assert(kNoAllocScratchBytes == 3154432, "the scratch size stated in lwc.h");
 
 // Shared by every call on a device; keeps the last call's contents (the plan
 // step clears what must start at zero).

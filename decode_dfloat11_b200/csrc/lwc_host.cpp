@@ -77,6 +77,7 @@ void write_header(uint8_t *h, const lwc_desc &d) {
         put<uint32_t>(h, 136, d.elem);
         put<uint64_t>(h, 144, d.off_lo);
         put<uint64_t>(h, 152, d.lo_bytes);
+        put<uint64_t>(h, 160, d.off_counts);
     } else {
         put<uint32_t>(h, 32, d.U);
         put<uint32_t>(h, 36, d.k);
@@ -116,6 +117,7 @@ void read_header(const uint8_t *h, lwc_desc &d) {
         d.elem = get<uint32_t>(h, 136);
         d.off_lo = get<uint64_t>(h, 144);
         d.lo_bytes = get<uint64_t>(h, 152);
+        d.off_counts = get<uint64_t>(h, 160);
     } else if (d.codec == LWC_CODEC_CODEBOOK) {
         d.U = get<uint32_t>(h, 32);
         d.k = get<uint32_t>(h, 36);
@@ -262,8 +264,8 @@ uint64_t lo_section_bytes(uint32_t elem, uint64_t n) {
     return 0;
 }
 
-lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uint32_t T, uint32_t L, Df11Plan &p,
-                         uint64_t lo_bytes) {
+lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uint32_t T, uint32_t L,
+                         bool chunk_counts, Df11Plan &p, uint64_t lo_bytes) {
     if (lwc_status st = check_df11_params(C, T, L)) return st;
     int present = 0, only = 0;
     for (int s = 0; s < 256; s++)
@@ -296,6 +298,11 @@ lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uin
         d.n_chunks = (d.total_bits + cb - 1) / cb;
         d.n_blocks = (d.n_chunks + T - 1) / T;
         d.stream_bytes = round_up(4 * ((d.total_bits + 31) / 32) + 16, 16);
+        // codes are at least min_len bits, so at most ceil(cb / min_len) start in a chunk
+        uint32_t min_len = 32;
+        for (int s = 0; s < 256; s++)
+            if (p.len[s]) min_len = std::min(min_len, p.len[s]);
+        if (chunk_counts && (cb + min_len - 1) / min_len <= 255) d.flags |= kFlagChunkCounts;
     } else {
         d.flags = n ? kFlagSingleExponent : 0;
         d.const_exp = (uint32_t)only;
@@ -304,6 +311,7 @@ lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t C, uin
     d.off_lengths = lay.place(256);
     d.off_lut = lay.place(2 * p.tables.size());
     d.off_gaps = lay.place(d.n_blocks * T);
+    if (d.flags & kFlagChunkCounts) d.off_counts = lay.place(d.n_blocks * T);
     d.off_blkoff = lay.place(8 * (d.n_blocks + 1));
     d.off_stream = lay.place(d.stream_bytes);
     d.off_sm = lay.place(round_up(n, 16));
@@ -379,6 +387,8 @@ lwc_status check_df11_desc(const lwc_desc *d) {
         return fail(LWC_ERR_CORRUPT, "stream section too short");
     if (d->max_block_count == 0 || d->max_block_count > T * cb || d->max_block_count > d->n)
         return fail(LWC_ERR_CORRUPT, "bad max_block_count");
+    if ((d->flags & kFlagChunkCounts) && !inside(d->off_counts, d->n_blocks * T, tot))
+        return fail(LWC_ERR_CORRUPT, "chunk-count section outside the blob");
     if (!inside(d->off_lut, 512ull * d->n_tables, tot) || !inside(d->off_gaps, d->n_blocks * T, tot) ||
         !inside(d->off_blkoff, 8 * (d->n_blocks + 1), tot) || !inside(d->off_stream, d->stream_bytes, tot))
         return fail(LWC_ERR_CORRUPT, "section outside the blob");
@@ -412,12 +422,13 @@ lwc_status encode_df11(const uint16_t *src, uint64_t n, const lwc_df11_params *p
     const uint32_t C = params ? params->chunk_bytes : kDefaultChunkBytes;
     const uint32_t T = params ? params->threads_per_block : kDefaultThreadsPerBlock;
     const uint32_t L = params ? params->max_len : kDefaultMaxLen;
+    const bool with_counts = params ? params->chunk_counts != 0 : kDefaultChunkCounts != 0;
 
     // exponent histogram, then the code and the section layout
     uint64_t counts[256] = {0};
     for (uint64_t i = 0; i < n; i++) counts[(src[i] >> 7) & 0xFF]++;
     Df11Plan plan;
-    st = plan_dfloat11(counts, n, C, T, L, plan, lo_section_bytes(elem, n));
+    st = plan_dfloat11(counts, n, C, T, L, with_counts, plan, lo_section_bytes(elem, n));
     if (st) return st;
     plan.d.elem = elem;
     lwc_desc &d = plan.d;
@@ -436,9 +447,11 @@ lwc_status encode_df11(const uint16_t *src, uint64_t n, const lwc_df11_params *p
     for (uint64_t i = 0; i < n; i++) sm[i] = (uint8_t)(((src[i] >> 8) & 0x80) | (src[i] & 0x7F));
 
     if (present2) {
-        // codes, MSB first in u32 words, with chunk gaps and block offsets
+        // codes, MSB first in u32 words, with chunk gaps, block offsets and
+        // (when planned) per-chunk code counts
         uint32_t *words = reinterpret_cast<uint32_t *>(blob + d.off_stream);
         uint8_t *gaps = blob + d.off_gaps;
+        uint8_t *ccount = (d.flags & kFlagChunkCounts) ? blob + d.off_counts : nullptr;
         uint64_t *blkoff = reinterpret_cast<uint64_t *>(blob + d.off_blkoff);
         uint64_t lut32[256];  // (len << 32) | code
         for (int s = 0; s < 256; s++) lut32[s] = ((uint64_t)len[s] << 32) | code[s];
@@ -459,6 +472,7 @@ lwc_status encode_df11(const uint16_t *src, uint64_t n, const lwc_df11_params *p
                 }
                 if (chunk >= d.n_chunks) next_chunk_bit = ~0ull;
             }
+            if (ccount) ccount[chunk - 1]++;   // this code starts in chunk `chunk - 1`
             const uint64_t lc = lut32[(src[i] >> 7) & 0xFF];
             const uint32_t l = (uint32_t)(lc >> 32);
             acc = (acc << l) | (uint32_t)lc;

@@ -17,6 +17,7 @@ constexpr uint32_t kVersion = 1;
 constexpr uint32_t kHeaderBytes = 256;
 constexpr uint32_t kSectionAlign = 256;
 constexpr uint32_t kFlagSingleExponent = 1u;
+constexpr uint32_t kFlagChunkCounts = 2u;   // DFloat11: u8 code count per chunk at off_counts
 constexpr uint32_t kFormatMaxLen = 32;      // longest Huffman code the format allows
 constexpr uint32_t kMaxTables = 256;        // lookup tables the decoders stage in shared memory
 
@@ -26,6 +27,7 @@ constexpr uint32_t kMaxTables = 256;        // lookup tables the decoders stage 
 constexpr uint32_t kDefaultChunkBytes = 36;
 constexpr uint32_t kDefaultThreadsPerBlock = 32;
 constexpr uint32_t kDefaultMaxLen = 32;
+constexpr uint32_t kDefaultChunkCounts = 1;
 
 // Record a message for lwc_last_error() and return `s`.
 lwc_status fail(lwc_status s, const char *fmt, ...);
@@ -38,7 +40,7 @@ lwc_status check_df11_desc(const lwc_desc *d);
 lwc_status check_codebook_desc(const lwc_desc *d);
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-inline uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
+constexpr uint64_t round_up(uint64_t x, uint64_t a) { return (x + a - 1) / a * a; }
 
 // Section placement inside a blob: each section at the next multiple of kSectionAlign.
 struct BlobLayout {
@@ -63,9 +65,10 @@ struct Df11Plan {
 };
 lwc_status check_df11_params(uint32_t chunk_bytes, uint32_t threads_per_block, uint32_t max_len);
 // lo_bytes: size of the raw low-mantissa section placed after the
-// sign|mantissa bytes (FP32 and FP16 elements; 0 for BF16).
+// sign|mantissa bytes (FP32 and FP16 elements; 0 for BF16). chunk_counts:
+// store the per-chunk code counts when the code bounds every count below 256.
 lwc_status plan_dfloat11(const uint64_t counts[256], uint64_t n, uint32_t chunk_bytes, uint32_t threads_per_block,
-                         uint32_t max_len, Df11Plan &plan, uint64_t lo_bytes = 0);
+                         uint32_t max_len, bool chunk_counts, Df11Plan &plan, uint64_t lo_bytes = 0);
 
 // Size of the raw low-mantissa section for n elements of type elem.
 uint64_t lo_section_bytes(uint32_t elem, uint64_t n);

@@ -64,7 +64,7 @@ class lwc_desc(ctypes.Structure):
         ("U", ctypes.c_uint32), ("k", ctypes.c_uint32), ("off_table", ctypes.c_uint64),
         ("off_packed", ctypes.c_uint64), ("packed_bytes", ctypes.c_uint64),
         ("elem", ctypes.c_uint32), ("reserved", ctypes.c_uint32), ("off_lo", ctypes.c_uint64),
-        ("lo_bytes", ctypes.c_uint64),
+        ("lo_bytes", ctypes.c_uint64), ("off_counts", ctypes.c_uint64),
     ]
 
     def as_dict(self):
@@ -77,7 +77,7 @@ class lwc_desc(ctypes.Structure):
 
 class lwc_df11_params(ctypes.Structure):
     _fields_ = [("chunk_bytes", ctypes.c_uint32), ("threads_per_block", ctypes.c_uint32),
-                ("max_len", ctypes.c_uint32)]
+                ("max_len", ctypes.c_uint32), ("chunk_counts", ctypes.c_uint32)]
 
 
 _lib = None
@@ -182,18 +182,19 @@ def _src(h_src) -> np.ndarray:
 
 
 def lwc_encode_dfloat11(h_src, chunk_bytes: int = 36, threads_per_block: int = 32,
-                        max_len: int = 32) -> tuple[lwc_desc, np.ndarray]:
-    """Encode host BF16 bit patterns (uint16 array); returns (desc, blob bytes)."""
+                        max_len: int = 32, chunk_counts: bool = True) -> tuple[lwc_desc, np.ndarray]:
+    """Encode host BF16 bit patterns (uint16 array); returns (desc, blob bytes).
+    chunk_counts: store per-chunk code counts when they fit a byte (see lwc.h)."""
     src = _src(h_src)
     desc, ptr, nbytes = lwc_desc(), _P(), _u64()
-    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len, int(chunk_counts))
     _check(load().lwc_encode_dfloat11(src.ctypes.data, src.size, ctypes.byref(params), ctypes.byref(desc),
                                       ctypes.byref(ptr), ctypes.byref(nbytes)))
     return desc, _take_blob(ptr, nbytes.value)
 
 
 def lwc_encode_dfloat11_elements(h_src, elem: int, chunk_bytes: int = 36, threads_per_block: int = 32,
-                                 max_len: int = 32) -> tuple[lwc_desc, np.ndarray]:
+                                 max_len: int = 32, chunk_counts: bool = True) -> tuple[lwc_desc, np.ndarray]:
     """DFloat11 encode of FP32 (uint32 / float32 array), FP16 or BF16 (16-bit) elements."""
     a = np.ascontiguousarray(h_src).reshape(-1)
     want = np.uint32 if elem == LWC_ELEM_FP32 else np.uint16
@@ -202,7 +203,7 @@ def lwc_encode_dfloat11_elements(h_src, elem: int, chunk_bytes: int = 36, thread
             raise ValueError(f"element type {elem} needs {np.dtype(want).itemsize}-byte elements")
         a = a.view(want)
     desc, ptr, nbytes = lwc_desc(), _P(), _u64()
-    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len, int(chunk_counts))
     _check(load().lwc_encode_dfloat11_elements(a.ctypes.data, a.size, elem, ctypes.byref(params), ctypes.byref(desc),
                                                ctypes.byref(ptr), ctypes.byref(nbytes)))
     return desc, _take_blob(ptr, nbytes.value)
@@ -319,10 +320,11 @@ def lwc_encode_device_workspace_bytes(n: int) -> int:
 
 
 def lwc_encode_dfloat11_device_plan(d_src, n: int, d_work, work_bytes: int, chunk_bytes: int = 36,
-                                    threads_per_block: int = 32, max_len: int = 32, stream=None) -> lwc_desc:
+                                    threads_per_block: int = 32, max_len: int = 32, stream=None,
+                                    chunk_counts: bool = True) -> lwc_desc:
     """Plan a DFloat11 blob for n device BF16 patterns; returns its descriptor."""
     desc = lwc_desc()
-    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len, int(chunk_counts))
     _check(load().lwc_encode_dfloat11_device_plan(_addr(d_src), n, ctypes.byref(params), _addr(d_work), work_bytes,
                                                   ctypes.byref(desc), _stream(stream)))
     return desc
@@ -330,10 +332,10 @@ def lwc_encode_dfloat11_device_plan(d_src, n: int, d_work, work_bytes: int, chun
 
 def lwc_encode_dfloat11_elements_device_plan(d_src, n: int, elem: int, d_work, work_bytes: int, chunk_bytes: int = 36,
                                              threads_per_block: int = 32, max_len: int = 32,
-                                             stream=None) -> lwc_desc:
+                                             stream=None, chunk_counts: bool = True) -> lwc_desc:
     """Plan a DFloat11 blob of FP32 / FP16 / BF16 elements held on the device."""
     desc = lwc_desc()
-    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len, int(chunk_counts))
     _check(load().lwc_encode_dfloat11_elements_device_plan(_addr(d_src), n, elem, ctypes.byref(params), _addr(d_work),
                                                            work_bytes, ctypes.byref(desc), _stream(stream)))
     return desc
@@ -356,12 +358,13 @@ def lwc_encode_device_write(d_src, n: int, d_work, work_bytes: int, d_blob, blob
 
 
 def lwc_encode_dfloat11_device_noalloc(d_src, n: int, d_blob, blob_bytes: int, chunk_bytes: int = 36,
-                                       threads_per_block: int = 32, max_len: int = 32, stream=None) -> lwc_desc:
+                                       threads_per_block: int = 32, max_len: int = 32, stream=None,
+                                       chunk_counts: bool = True) -> lwc_desc:
     """DFloat11 device encode without any device allocation (the library's
     own scratch array replaces the workspace); for callers that cannot call
     cudaMalloc. Returns the blob's descriptor."""
     desc = lwc_desc()
-    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len)
+    params = lwc_df11_params(chunk_bytes, threads_per_block, max_len, int(chunk_counts))
     _check(load().lwc_encode_dfloat11_device_noalloc(_addr(d_src), n, ctypes.byref(params), _addr(d_blob),
                                                      blob_bytes, ctypes.byref(desc), _stream(stream)))
     return desc

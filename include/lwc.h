@@ -111,7 +111,8 @@ typedef struct lwc_desc {
     uint32_t magic;            /* 0x3143574C */
     uint32_t version;          /* 1 */
     uint32_t codec;            /* LWC_CODEC_* */
-    uint32_t flags;            /* bit 0 (DFloat11): one exponent value only */
+    uint32_t flags;            /* DFloat11: bit 0 one exponent value only;
+                                  bit 1 per-chunk code counts stored (off_counts) */
     uint64_t n;                /* number of weights */
     uint64_t total_bytes;      /* blob size */
     /* DFloat11 */
@@ -142,16 +143,28 @@ typedef struct lwc_desc {
     uint32_t reserved;
     uint64_t off_lo;           /* raw low mantissa bits (FP32, FP16) */
     uint64_t lo_bytes;
+    /* DFloat11, flags bit 1 (header bytes 160..167; zero otherwise):
+     * u8[n_blocks * threads_per_block], the number of codes that start in
+     * each chunk -- what the first phase of the two-phase decoder (DF11
+     * page, section "Jak to działa w praktyce?") counts, stored by the
+     * encoder so that a decoder can go straight to the scan and the writes.
+     * Chunks past the stream end count 0. */
+    uint64_t off_counts;
 } lwc_desc;
 
 /* DFloat11 encoder parameters; pass NULL for the defaults
- * (chunk_bytes 36, threads_per_block 32, max_len 32). chunk_bytes: multiple
- * of 4 in [8, 1024]; threads_per_block: multiple of 32 in [32, 1024];
- * max_len: code length limit in [9, 32]. */
+ * (chunk_bytes 36, threads_per_block 32, max_len 32, chunk_counts 1).
+ * chunk_bytes: multiple of 4 in [8, 1024]; threads_per_block: multiple of 32
+ * in [32, 1024]; max_len: code length limit in [9, 32]; chunk_counts: 1 =
+ * store the per-chunk code counts (flags bit 1) whenever every count fits in
+ * a byte, which the code guarantees when ceil(8 chunk_bytes / shortest code
+ * length) <= 255 (with 36-byte chunks: no 1-bit code); 0 = never. Blobs with
+ * the counts decode faster; both kinds decode to the same tensor. */
 typedef struct lwc_df11_params {
     uint32_t chunk_bytes;
     uint32_t threads_per_block;
     uint32_t max_len;
+    uint32_t chunk_counts;
 } lwc_df11_params;
 
 /* ---- host encoders -------------------------------------------------------- */

@@ -74,7 +74,6 @@ def test_chunk_counts_by_code_end_is_caught(monkeypatch):
     monkeypatch.setattr(df11, "chunk_code_counts", bad)
     fails(pins.test_golden_df11_periodic_offsets)
     fails(pins.test_chunk_counts_match_independent_chunk_decodes, 8, 32)
-    fails(pins.test_chunk_counts_single_code_length)
 
 
 def test_dropped_sign_is_caught(monkeypatch):
