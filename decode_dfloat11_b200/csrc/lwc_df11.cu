@@ -59,6 +59,7 @@ constexpr int kCtasPerSm = 4;   // target residency for 256-thread CTAs (shared 
 struct Df11Tensor {
     const uint32_t *stream;
     const uint8_t *gaps;
+    const uint8_t *counts; // per-chunk code counts (blobs that store them), else null
     const uint64_t *blkoff;
     const uint8_t *sm;
     const uint8_t *lo;     // raw low-mantissa section (FP32, FP16 elements)
@@ -1084,6 +1085,337 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
     df11_warp_body<E, 0>(B, nullptr);
 }
 
+// ---- per-warp blocks with stored chunk counts ------------------------------------
+//
+// Blobs that store each chunk's code count (flags bit 1) carry the result of
+// the first phase of the two-phase decoder: a warp reads the 32 counts of
+// its block, turns them into output positions with a warp scan and decodes
+// each chunk once. Each lane assembles its exponents into 32-bit words in
+// registers and writes whole words to the staging area (a quarter of the
+// shared-memory stores of byte writes, and far fewer bank conflicts). The
+// word a lane shares with the lane before it (when its first exponent is not
+// word aligned) goes to a private slot instead; after the warp's word stores
+// the lane copies its bytes of that word into place, so no byte is written
+// by two lanes at once. Codes of 12 to 19 bits take one more lookup, in a
+// second-level table indexed by the next 8 bits (for the first kSubTables
+// 11-bit prefixes that begin long codes: in a canonical code those are the
+// numerically last prefixes); longer codes walk the blob's hierarchical
+// tables.
+//
+// Symbol table entry (u32): bits 0-23 up to three exponents (first code in
+// the low byte), bits 24-25 how many (n), bits 27-31 the bits their codes
+// take; 0 means the first code is longer than 11 bits.
+
+constexpr uint32_t kSubTables = 8;
+constexpr uint32_t kCtdTabBytes = kFastSize * 4 + kSubTables * 256 * 4;   // 16 KB
+
+struct CountedLayout {
+    uint32_t warp0, seg_bytes, gaps, counts, slot, stage, warp_bytes, misc, bars, total;
+    __host__ __device__ CountedLayout(uint32_t seg_words, uint32_t lut_entries, uint32_t stage_bytes, uint32_t warps) {
+        warp0 = kCtdTabBytes + ((2 * lut_entries + 15) & ~15u);
+        seg_bytes = 4 * seg_words;
+        gaps = seg_bytes;     // 48 bytes: the block's 32 gaps, then the next block's first 16
+        counts = gaps + 48;   // the block's 32 code counts
+        slot = counts + 32;   // one word per lane: its first (shared) staging word
+        stage = slot + 128;
+        warp_bytes = stage + stage_bytes;
+        misc = warp0 + warps * warp_bytes;   // the first long 11-bit prefix
+        bars = misc + 16;
+        total = bars + 8 * warps;
+    }
+};
+
+// Symbol table and second-level tables of one tensor, from its hierarchical
+// tables (all threads of the CTA; barriers inside).
+__device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint32_t *sym, uint32_t *sub,
+                                     uint32_t *first_long) {
+    if (threadIdx.x == 0) *first_long = kFastSize;
+    __syncthreads();
+    for (uint32_t v = threadIdx.x; v < kFastSize; v += blockDim.x) {
+        uint32_t w = v << (32 - kFastBits), used = 0, cnt = 0, syms = 0, ignore = 0;
+        while (cnt < 3) {
+            const uint32_t r = lut_walk(lut, ntab, w, ignore);
+            const uint32_t len = r >> 8;
+            if (ignore || used + len > (uint32_t)kFastBits) break;
+            syms |= (r & 0xFFu) << (8 * cnt);
+            cnt++;
+            used += len;
+            w <<= len;
+        }
+        sym[v] = cnt ? (syms | (cnt << 24) | (used << 27)) : 0u;
+        if (!cnt) atomicMin(first_long, v);
+    }
+    __syncthreads();
+    const uint32_t v0 = *first_long;
+    for (uint32_t i = threadIdx.x; i < kSubTables * 256u; i += blockDim.x) {
+        const uint32_t v = v0 + (i >> 8);
+        uint32_t e = 0;
+        if (v < (uint32_t)kFastSize) {
+            uint32_t ignore = 0;
+            const uint32_t r = lut_walk(lut, ntab, (v << (32 - kFastBits)) | ((i & 255u) << (24 - kFastBits)), ignore);
+            const uint32_t len = r >> 8;
+            if (!ignore && len > (uint32_t)kFastBits && len <= (uint32_t)kFastBits + 8) e = (r & 0xFFu) | (1u << 24) | (len << 27);
+        }
+        sub[i] = e;
+    }
+}
+
+// Lane 0: bulk copies of block b of tensor `tn`: its stream segment, its 32
+// gaps (+ the next block's first 16) and its 32 code counts.
+__device__ __forceinline__ void issue_counted_item(const Df11Batch &B, const Df11Tensor &tn, uint32_t b, uint8_t *buf,
+                                                   uint32_t seg_bytes, uint64_t *bar) {
+    const uint64_t seg0 = (uint64_t)b * 32u * B.chunk_words * 4;   // multiple of 128
+    const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
+    const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
+    const uint32_t gbytes = b + 1 < tn.n_blocks ? 48u : 32u;
+    dev::mbar_arrive_expect_tx(bar, bytes + gbytes + 32u);
+    if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
+    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
+    dev::bulk_g2s(buf + seg_bytes + 48, tn.counts + (uint64_t)b * 32u, 32u, bar);
+}
+
+// The 32 stream bits at bit `pos` of the segment, as Window, with the word
+// index kept inside the segment buffer whatever the counts say.
+struct SegWindow {
+    uint32_t wi, w0, w1;
+    __device__ __forceinline__ SegWindow(const uint32_t *seg, uint32_t pos, uint32_t last)
+        : wi((pos >> 5) - 1u), w0(0), w1(seg[min(pos >> 5, last)]) {}
+    __device__ __forceinline__ uint32_t at(const uint32_t *seg, uint32_t pos, uint32_t last) {
+        const uint32_t ni = pos >> 5;
+        w0 = ni != wi ? w1 : w0;
+        w1 = seg[min(ni + 1, last)];
+        wi = ni;
+        return __funnelshift_l(w1, w0, pos);
+    }
+};
+
+// Decodes `cnt` codes from bit `pos` of the segment; exponent j goes to
+// staging byte qb + j. Words of the staging area that hold none of these
+// exponents are never written; the word holding byte qb goes to *slot when
+// qb is not word aligned. Returns the bit where decoding stopped: the last
+// step takes whole table entries, so that is the end of the last code or up
+// to 30 bits past it.
+__device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t last, const uint32_t *sym,
+                                                   const uint32_t *sub, uint32_t v0, const uint16_t *lut,
+                                                   uint32_t ntab, uint32_t pos, uint32_t cnt, uint32_t qb,
+                                                   uint32_t *stage_w, uint32_t *slot, uint32_t &bad) {
+    uint32_t *nxt = stage_w + (qb >> 2) + 1;        // the staging word after the current one
+    uint32_t *dst = (qb & 3u) ? slot : nxt - 1;     // where the current word goes
+    const uint32_t *const lim = stage_w + ((qb + cnt + 3) >> 2);   // first word past this lane's bytes
+    uint32_t lo = 0, sh = (qb & 3u) << 3;           // pending bytes of the current word, and their bits
+    int32_t k8 = (int32_t)(cnt << 3);               // exponents still to decode, x 8
+    // Appends n8/8 exponents (c1:c0, little-endian bytes, zero above them) at
+    // byte sh/8 of the current word; stores each word it completes (the
+    // second one only if it holds an exponent of this lane).
+    auto emit = [&](uint32_t c0, uint32_t c1, uint32_t n8) {
+        const uint32_t w0 = lo | (c0 << sh);
+        const uint32_t w1 = __funnelshift_lc(c0, c1, sh);
+        const uint32_t w2 = __funnelshift_lc(c1, 0u, sh);
+        sh += n8;
+        if (sh >= 32) {
+            *dst = w0;
+            dst = nxt++;
+            if (sh >= 64) {
+                if (dst < lim) *dst = w1;
+                dst = nxt++;
+                lo = w2;
+            } else {
+                lo = w1;
+            }
+        } else {
+            lo = w0;
+        }
+        sh &= 31u;
+    };
+    SegWindow win(seg, pos, last);
+    while (k8 > 0) {
+        const uint32_t wv = win.at(seg, pos, last);
+        uint32_t e1 = sym[wv >> (32 - kFastBits)];
+        if (e1 == 0u) {   // the first code is longer than 11 bits
+            const uint32_t s = (wv >> (32 - kFastBits)) - v0;
+            if (s < kSubTables) e1 = sub[(s << 8) | ((wv >> (24 - kFastBits)) & 0xFFu)];
+            if (e1 == 0u) {   // longer than 19 bits: the hierarchical tables
+                const uint32_t r = lut_walk(lut, ntab, wv, bad);
+                emit(r & 0xFFu, 0u, 8u);
+                pos += r >> 8;
+                k8 -= 8;
+                continue;
+            }
+        }
+        const uint32_t l1 = e1 >> 27;   // <= 19
+        const uint32_t e2 = sym[(wv << l1) >> (32 - kFastBits)];
+        const uint32_t n1 = (e1 >> 21) & 0x18u, n2 = (e2 >> 21) & 0x18u;
+        const uint32_t s1 = e1 & 0xFFFFFFu, s2 = e2 & 0xFFFFFFu;
+        emit(s1 | (s2 << n1), __funnelshift_lc(s2, 0u, n1), n1 + n2);
+        pos += l1 + (e2 >> 27);
+        k8 -= (int32_t)(n1 + n2);
+    }
+    if (nxt - 1 < lim) *dst = lo;   // the last, partial word
+    return pos;
+}
+
+template <int E>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counted_kernel(const __grid_constant__ Df11Batch B) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+    const uint32_t NW = B.warps;
+    const CountedLayout L(B.seg_words, B.lut_entries, B.stage_bytes, NW);
+    uint32_t *sym = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *sub = sym + kFastSize;
+    uint16_t *lut = reinterpret_cast<uint16_t *>(smem + kCtdTabBytes);
+    uint8_t *buf = smem + L.warp0 + warp * L.warp_bytes;
+    const uint32_t *seg = reinterpret_cast<const uint32_t *>(buf);
+    const uint8_t *gapb = buf + L.gaps;
+    const uint8_t *cntb = buf + L.counts;
+    uint32_t *slot = reinterpret_cast<uint32_t *>(buf + L.slot) + lane;
+    uint8_t *stage = buf + L.stage;
+    uint32_t *first_long = reinterpret_cast<uint32_t *>(smem + L.misc);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.bars) + warp;
+    const uint32_t seg_bytes = L.seg_bytes, last = B.seg_words - 1;
+    const uint32_t cbits = B.chunk_words * 32u;
+
+    const uint32_t W = B.total_work, G = gridDim.x;
+    const uint32_t w_begin = (uint32_t)((uint64_t)W * blockIdx.x / G);
+    const uint32_t w_end = (uint32_t)((uint64_t)W * (blockIdx.x + 1) / G);
+    if (w_begin >= w_end) return;
+    if (lane == 0) {
+        dev::mbar_init(bar, 1);
+        dev::fence_mbar_init();
+    }
+    __syncwarp();
+
+    uint32_t bad = 0, items = 0;
+    bool dead = false;   // a bounded wait gave up: this warp stops decoding
+    uint32_t ti = locate(B, w_begin, 0);
+    for (uint32_t w0 = w_begin; w0 < w_end;) {
+        const Df11Tensor &tn = B.t[ti];
+        const uint32_t t_end = ti + 1 < B.count ? B.t[ti + 1].first_work : W;
+        const uint32_t s_end = min(w_end, t_end);
+        __syncthreads();   // every warp is done with the previous tensor's tables
+        const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
+        for (uint32_t i = tid; i < ntab * 128u; i += blockDim.x)
+            reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
+        __syncthreads();
+        build_counted_tables(lut, ntab, sym, sub, first_long);
+        __syncthreads();
+        const uint32_t v0 = *first_long;
+
+        uint32_t w = w0 + warp;
+        if (w < s_end && lane == 0 && !dead) {
+            dev::fence_proxy_async_smem();
+            issue_counted_item(B, tn, w - tn.first_work, buf, seg_bytes, bar);
+        }
+        uint64_t o0n = 0, o1n = 0;
+        if (w < s_end) {
+            o0n = tn.blkoff[w - tn.first_work];
+            o1n = tn.blkoff[w - tn.first_work + 1];
+        }
+        for (; w < s_end && !dead; w += NW) {
+            const uint32_t b = w - tn.first_work;
+            const uint64_t o0 = o0n, o1 = o1n;
+            const bool more = w + NW < s_end;
+            if (more) {
+                o0n = tn.blkoff[b + NW];
+                o1n = tn.blkoff[b + NW + 1];
+            }
+            const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
+            const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
+            uint4 sv[kWarpMergeRegs];
+#pragma unroll
+            for (int m = 0; m < kWarpMergeRegs; m++) {
+                const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
+                sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
+            }
+            const bool arrived = dev::mbar_wait_bounded(bar, items & 1u);
+            items++;
+            if (__any_sync(0xFFFFFFFFu, !arrived)) {
+                // let the late copy land (bounded) before this warp stops
+                bad |= LWC_DEVICE_TIMEOUT;
+                if (lane == 0) dev::mbar_wait_bounded(bar, (items - 1) & 1u);
+                dead = true;
+                break;
+            }
+            bool next_issued = false;
+            if (ok) {
+                // output positions: a warp scan of the stored counts
+                const uint32_t cnt = cntb[lane];
+                uint32_t x = cnt;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+                    if (lane >= (uint32_t)o) x += y;
+                }
+                const uint32_t total = __shfl_sync(0xFFFFFFFFu, x, 31);
+                if (total == (uint32_t)(o1 - o0)) {
+                    const uint32_t first = x - cnt;
+                    const uint32_t qb = (uint32_t)(o0 & 15u) + first;   // staging byte of this lane's first exponent
+                    const uint64_t rem_block = tn.total_bits - (uint64_t)b * 32u * cbits;
+                    const uint32_t start = lane * cbits + gapb[lane];
+                    const bool has_next = lane + 1 < 32u || b + 1 < tn.n_blocks;
+                    const uint64_t next = has_next ? (uint64_t)(lane + 1) * cbits + gapb[lane + 1] : rem_block;
+                    const uint32_t end = (uint32_t)min(next, rem_block);
+                    if (cnt) {
+                        const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
+                                                            reinterpret_cast<uint32_t *>(stage), slot, bad);
+                        // the last step may decode past the lane's codes (by less than 32 bits);
+                        // falling short of the next chunk's first code, or far past it, means a bad count
+                        if (got - end >= 32u) bad |= LWC_DEVICE_BAD_COUNT;
+                    }
+                    __syncwarp();
+                    // the bytes of this lane's first, shared word
+                    if ((qb & 3u) && cnt) {
+                        const uint32_t hw = *slot, j0 = qb & 3u;
+                        uint8_t *hb = stage + (qb & ~3u);
+                        hb[j0] = (uint8_t)(hw >> (8 * j0));
+                        if (j0 < 3 && cnt > 1) hb[j0 + 1] = (uint8_t)(hw >> (8 * j0 + 8));
+                        if (j0 == 1 && cnt > 2) hb[3] = (uint8_t)(hw >> 24);
+                    }
+                    __syncwarp();
+                    // the segment is free: fetch this warp's next block while merging this one
+                    if (lane == 0 && more) {
+                        dev::fence_proxy_async_smem();
+                        issue_counted_item(B, tn, b + NW, buf, seg_bytes, bar);
+                    }
+                    next_issued = true;
+
+                    // 32-bit offsets from the block's first 16-weight group
+                    const uint64_t base = o0 & ~15ull;
+                    const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
+                    void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
+                                                  : static_cast<void *>(tn.out + base);
+                    const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
+                    const uint64_t g0 = base / 16;
+                    const uint8_t *sb = tn.sm + base;
+#pragma unroll
+                    for (int m = 0; m < kWarpMergeRegs; m++) {
+                        const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
+                        if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                    }
+                    for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
+                        merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
+                                       *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                    const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
+                    const bool head = lane < 16 && i < min(g_lo, o1);
+                    const bool tail = lane >= 16 && i < o1;
+                    if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
+                } else {
+                    bad |= LWC_DEVICE_BAD_COUNT;
+                }
+            } else {
+                bad |= LWC_DEVICE_BAD_OFFSET;
+            }
+            __syncwarp();   // segment and staging area free again
+            if (lane == 0 && !next_issued && more) {
+                dev::fence_proxy_async_smem();
+                issue_counted_item(B, tn, b + NW, buf, seg_bytes, bar);
+            }
+        }
+        w0 = s_end;
+        if (w0 < w_end) ti = locate(B, w0, ti);
+    }
+    if (bad && B.status) atomicOr(B.status, bad);
+}
+
 // Fused decode + linear layer (BF16 elements, blocks of 32 chunks) for up
 // to MM activation rows; with more than one row the accumulators need more
 // registers than two CTAs per SM leave.
@@ -1141,7 +1473,9 @@ lwc_status device_config(DeviceConfig &out) {
             (const void *)df11_decode_kernel<256, LWC_ELEM_FP32>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP32>,
             (const void *)df11_warp_kernel<LWC_ELEM_FP32>,
             (const void *)df11_decode_kernel<256, LWC_ELEM_FP16>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP16>,
-            (const void *)df11_warp_kernel<LWC_ELEM_FP16>, (const void *)kLinKernels[0], (const void *)kLinKernels[1],
+            (const void *)df11_warp_kernel<LWC_ELEM_FP16>, (const void *)df11_counted_kernel<LWC_ELEM_BF16>,
+            (const void *)df11_counted_kernel<LWC_ELEM_FP32>, (const void *)df11_counted_kernel<LWC_ELEM_FP16>,
+            (const void *)kLinKernels[0], (const void *)kLinKernels[1],
             (const void *)kLinKernels[2], (const void *)kLinKernels[3]};
         for (const void *k : kernels) {
             if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
@@ -1156,24 +1490,30 @@ lwc_status device_config(DeviceConfig &out) {
 }
 
 
-// The decode kernel for an element type and block shape, and its launch.
-template <int E>
-const void *df11_kernel(bool per_warp, uint32_t T) {
-    return per_warp   ? (const void *)df11_warp_kernel<E>
-           : T <= 256 ? (const void *)df11_decode_kernel<256, E>
-                      : (const void *)df11_decode_kernel<1024, E>;
-}
-
-const void *df11_kernel_for(uint32_t elem, bool per_warp, uint32_t T) {
-    if (elem == LWC_ELEM_FP32) return df11_kernel<LWC_ELEM_FP32>(per_warp, T);
-    if (elem == LWC_ELEM_FP16) return df11_kernel<LWC_ELEM_FP16>(per_warp, T);
-    return df11_kernel<LWC_ELEM_BF16>(per_warp, T);
-}
+// Decode kernels: one CTA per block (blocks of 64+ chunks), one warp per
+// block (blocks of 32 chunks), or one warp per block with stored chunk counts.
+enum KernelMode { kModeBlock, kModeWarp, kModeCounted };
 
 template <int E>
-void launch_df11(bool per_warp, uint32_t T, unsigned grid, uint32_t threads, size_t smem, cudaStream_t stream,
+const void *df11_kernel(KernelMode mode, uint32_t T) {
+    return mode == kModeCounted ? (const void *)df11_counted_kernel<E>
+           : mode == kModeWarp  ? (const void *)df11_warp_kernel<E>
+           : T <= 256           ? (const void *)df11_decode_kernel<256, E>
+                                : (const void *)df11_decode_kernel<1024, E>;
+}
+
+const void *df11_kernel_for(uint32_t elem, KernelMode mode, uint32_t T) {
+    if (elem == LWC_ELEM_FP32) return df11_kernel<LWC_ELEM_FP32>(mode, T);
+    if (elem == LWC_ELEM_FP16) return df11_kernel<LWC_ELEM_FP16>(mode, T);
+    return df11_kernel<LWC_ELEM_BF16>(mode, T);
+}
+
+template <int E>
+void launch_df11(KernelMode mode, uint32_t T, unsigned grid, uint32_t threads, size_t smem, cudaStream_t stream,
                  const Df11Batch &B) {
-    if (per_warp)
+    if (mode == kModeCounted)
+        df11_counted_kernel<E><<<grid, threads, smem, stream>>>(B);
+    else if (mode == kModeWarp)
         df11_warp_kernel<E><<<grid, threads, smem, stream>>>(B);
     else if (T <= 256)
         df11_decode_kernel<256, E><<<grid, T, smem, stream>>>(B);
@@ -1181,15 +1521,22 @@ void launch_df11(bool per_warp, uint32_t T, unsigned grid, uint32_t threads, siz
         df11_decode_kernel<1024, E><<<grid, T, smem, stream>>>(B);
 }
 
-// Warps per CTA of the per-warp kernel: kWarpsPerCta, or fewer when one
+// Shared memory of a per-warp launch with w warps per CTA.
+uint64_t warp_smem(const Df11Batch &B, KernelMode mode, uint32_t w) {
+    return mode == kModeCounted ? CountedLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total
+                                : WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total;
+}
+
+// Warps per CTA of the per-warp kernels: kWarpsPerCta, or fewer when one
 // warp's segment buffer and staging area are large (long chunks).
-uint32_t warps_that_fit(const Df11Batch &B, int max_smem) {
+uint32_t warps_that_fit(const Df11Batch &B, int max_smem, KernelMode mode = kModeWarp) {
     uint32_t w = kWarpsPerCta;
-    while (w > 1 && WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total > (uint64_t)max_smem) w--;
+    while (w > 1 && warp_smem(B, mode, w) > (uint64_t)max_smem) w--;
     return w;
 }
 
-// Launch one kernel over up to kMaxBatch tensors sharing (element type, chunk_bytes, threads_per_block).
+// Launch one kernel over up to kMaxBatch tensors sharing (element type,
+// chunk_bytes, threads_per_block, stored chunk counts or not).
 lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, const void *const *d_ins,
                         uint16_t *const *d_outs, uint32_t *d_status, cudaStream_t stream,
                         const DeviceConfig &cfg) {
@@ -1206,6 +1553,7 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
         Df11Tensor &t = B.t[j];
         t.stream = reinterpret_cast<const uint32_t *>(base + d.off_stream);
         t.gaps = base + d.off_gaps;
+        t.counts = (d.flags & kFlagChunkCounts) ? base + d.off_counts : nullptr;
         t.blkoff = reinterpret_cast<const uint64_t *>(base + d.off_blkoff);
         t.sm = base + d.off_sm;
         t.lo = d.elem != LWC_ELEM_BF16 ? base + d.off_lo : nullptr;
@@ -1227,16 +1575,16 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
-    const bool per_warp = T == 32;
-    B.warps = per_warp ? warps_that_fit(B, cfg.max_smem) : 0;
+    const KernelMode mode = T != 32 ? kModeBlock : (d0.flags & kFlagChunkCounts) ? kModeCounted : kModeWarp;
+    const bool per_warp = mode != kModeBlock;
+    B.warps = per_warp ? warps_that_fit(B, cfg.max_smem, mode) : 0;
     const uint32_t threads = per_warp ? B.warps * 32u : T;
-    const uint64_t smem = per_warp ? WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, B.warps).total
-                                   : Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
+    const uint64_t smem = per_warp ? warp_smem(B, mode, B.warps) : Layout(T, B.seg_words, B.lut_entries, B.stage_bytes).total;
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
                     (unsigned long long)smem, cfg.max_smem);
     const uint32_t elem = d0.elem;
-    const void *kernel = df11_kernel_for(elem, per_warp, T);
+    const void *kernel = df11_kernel_for(elem, mode, T);
     int per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, (int)threads, (size_t)smem);
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "occupancy: %s", cudaGetErrorString(err));
@@ -1245,11 +1593,11 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     const uint64_t units = per_warp ? (work + B.warps - 1) / B.warps : work;
     const uint64_t grid = std::min<uint64_t>(units, (uint64_t)per_sm * cfg.sms);
     if (elem == LWC_ELEM_FP32)
-        launch_df11<LWC_ELEM_FP32>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
+        launch_df11<LWC_ELEM_FP32>(mode, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     else if (elem == LWC_ELEM_FP16)
-        launch_df11<LWC_ELEM_FP16>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
+        launch_df11<LWC_ELEM_FP16>(mode, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     else
-        launch_df11<LWC_ELEM_BF16>(per_warp, T, (unsigned)grid, threads, (size_t)smem, stream, B);
+        launch_df11<LWC_ELEM_BF16>(mode, T, (unsigned)grid, threads, (size_t)smem, stream, B);
     err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
     return LWC_OK;
@@ -1387,7 +1735,10 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
             if (st) return st;
             continue;
         }
-        keyed.push_back({((uint64_t)d.elem << 40) | ((uint64_t)d.chunk_bytes << 20) | d.threads_per_block, i});
+        const uint64_t counted = (d.flags & kFlagChunkCounts) ? 1 : 0;
+        keyed.push_back({(counted << 50) | ((uint64_t)d.elem << 40) | ((uint64_t)d.chunk_bytes << 20) |
+                             d.threads_per_block,
+                         i});
     }
     std::stable_sort(keyed.begin(), keyed.end(),
                      [](const std::pair<uint64_t, int> &a, const std::pair<uint64_t, int> &b) { return a.first < b.first; });

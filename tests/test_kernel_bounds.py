@@ -123,3 +123,235 @@ def test_division_by_cols_is_exact_for_every_32_bit_numerator():
         for n in ns:
             if 0 <= n < 1 << 32:
                 assert div_cols(n, d) == n // d, (n, d)
+
+
+# ---------------------------------------------------------------------------
+# The DFloat11 decoder for blobs with stored chunk counts (csrc/lwc_df11.cu:
+# build_counted_tables, decode_counted and the head-byte step of
+# df11_counted_kernel), restated lane by lane on the CPU: its shared-memory
+# stores are recorded, and the test checks that in the word phase no two
+# lanes write the same staging word, that no lane writes a word holding none
+# of its bytes, that every read of the segment stays inside the staged
+# buffer, and that after the head-byte step the staging area holds the
+# block's exponents (as the oracle decodes them).
+
+FAST_BITS = 11
+SUB_TABLES = 8
+
+
+def _walk(lut, w):
+    """(symbol, length) of the code at the top of the 32-bit window w, by the
+    blob's hierarchical tables; None for an invalid path."""
+    e = lut[w >> 24]
+    d = 1
+    while e & 0x8000 and d < 4:
+        t = e & 0x7FFF
+        if t >= len(lut) // 256:
+            return None
+        e = lut[t * 256 + ((w >> (24 - 8 * d)) & 0xFF)]
+        d += 1
+    ln = (e >> 8) & 0x3F
+    if e & 0x8000 or ln == 0 or ln > 32:
+        return None
+    return e & 0xFF, ln
+
+
+def _counted_tables(lut):
+    sym = [0] * (1 << FAST_BITS)
+    first_long = 1 << FAST_BITS
+    for v in range(1 << FAST_BITS):
+        w, used, cnt, syms = v << (32 - FAST_BITS), 0, 0, 0
+        while cnt < 3:
+            r = _walk(lut, w)
+            if r is None or used + r[1] > FAST_BITS:
+                break
+            syms |= r[0] << (8 * cnt)
+            cnt += 1
+            used += r[1]
+            w = (w << r[1]) & 0xFFFFFFFF
+        sym[v] = (syms | cnt << 24 | used << 27) if cnt else 0
+        if not cnt:
+            first_long = min(first_long, v)
+    sub = [0] * (SUB_TABLES * 256)
+    for i in range(SUB_TABLES * 256):
+        v = first_long + (i >> 8)
+        if v < (1 << FAST_BITS):
+            r = _walk(lut, (v << (32 - FAST_BITS)) | ((i & 255) << (24 - FAST_BITS)))
+            if r is not None and FAST_BITS < r[1] <= FAST_BITS + 8:
+                sub[i] = r[0] | 1 << 24 | r[1] << 27
+    return sym, sub, first_long
+
+
+def _fsl(lo, hi, sh):
+    """__funnelshift_lc: the top 32 bits of (hi:lo) << min(sh, 32)."""
+    sh = min(sh, 32)
+    return (((hi << 32) | lo) << sh >> 32) & 0xFFFFFFFF
+
+
+def _decode_lane(seg, last, tables, pos, cnt, qb, stores, lane):
+    """decode_counted for one lane: records (word, value, lane) stores into
+    `stores` ('slot' for the lane's private slot); returns the stop bit."""
+    sym, sub, v0 = tables
+    nxt = (qb >> 2) + 1
+    dst = "slot" if qb & 3 else nxt - 1
+    lim = (qb + cnt + 3) >> 2
+    state = {"lo": 0, "sh": (qb & 3) << 3, "dst": dst, "nxt": nxt}
+
+    def emit(c0, c1, n8):
+        sh, lo = state["sh"], state["lo"]
+        w0 = lo | ((c0 << sh) & 0xFFFFFFFF)
+        w1 = _fsl(c0, c1, sh)
+        w2 = _fsl(c1, 0, sh)
+        sh += n8
+        if sh >= 32:
+            stores.append((state["dst"], w0, lane))
+            state["dst"] = state["nxt"]
+            state["nxt"] += 1
+            if sh >= 64:
+                if state["dst"] < lim:
+                    stores.append((state["dst"], w1, lane))
+                state["dst"] = state["nxt"]
+                state["nxt"] += 1
+                lo = w2
+            else:
+                lo = w1
+        else:
+            lo = w0
+        state["lo"], state["sh"] = lo, sh & 31
+
+    def word(i):
+        assert 0 <= i <= last
+        return seg[i]
+
+    k8 = cnt * 8
+    wi = (pos >> 5) - 1
+    w1 = word(min(pos >> 5, last))
+    w0 = 0
+    while k8 > 0:
+        ni = pos >> 5
+        w0 = w1 if ni != wi else w0
+        w1 = word(min(ni + 1, last))
+        wi = ni
+        wv = _fsl(w1, w0, pos & 31)
+        e1 = sym[wv >> (32 - FAST_BITS)]
+        if e1 == 0:
+            s = ((wv >> (32 - FAST_BITS)) - v0) & 0xFFFFFFFF
+            if s < SUB_TABLES:
+                e1 = sub[(s << 8) | ((wv >> (24 - FAST_BITS)) & 0xFF)]
+            if e1 == 0:
+                r = _walk_or_fail(wv)
+                emit(r[0], 0, 8)
+                pos += r[1]
+                k8 -= 8
+                continue
+        l1 = e1 >> 27
+        e2 = sym[((wv << l1) & 0xFFFFFFFF) >> (32 - FAST_BITS)]
+        n1, n2 = (e1 >> 21) & 0x18, (e2 >> 21) & 0x18
+        s1, s2 = e1 & 0xFFFFFF, e2 & 0xFFFFFF
+        emit(s1 | ((s2 << n1) & 0xFFFFFFFF), _fsl(s2, 0, n1), n1 + n2)
+        pos += l1 + (e2 >> 27)
+        k8 -= n1 + n2
+    if state["nxt"] - 1 < lim:
+        stores.append((state["dst"], state["lo"], lane))
+    return pos
+
+
+_walk_or_fail = None
+
+
+@pytest.mark.parametrize("case", ["normal", "outliers", "long_codes", "chunk8"])
+def test_counted_decoder_model(case):
+    import synth
+    from decode_dfloat11_b200 import lwc
+    from oracle import blob as B
+    from oracle import df11 as odf
+
+    global _walk_or_fail
+    chunk = 36
+    if case == "normal":
+        w = synth.as_u16(synth.normal_bf16((200_003,), seed=7, sigma=0.02, outlier_frac=1e-3))
+    elif case == "outliers":
+        w = synth.as_u16(synth.normal_bf16((150_001,), seed=8, sigma=0.01, outlier_frac=2e-2))
+    elif case == "long_codes":   # Fibonacci counts: codes of 1..23 bits, all three lookup paths
+        chunk = 8                # a 1-bit code: only chunks of <= 255 bits keep their counts
+        fib = [1, 1]
+        while len(fib) < 24:
+            fib.append(fib[-1] + fib[-2])
+        w = np.repeat((np.arange(24, dtype=np.uint16) << 7) | 0x8011, np.array(fib))
+        w = np.random.default_rng(0).permutation(w).astype(np.uint16)
+        firsts = np.array([int(np.argmax(w == v)) for v in np.unique(w)])   # one weight of each exponent
+        w = np.concatenate([w[firsts], np.delete(w, firsts)])                # moved to block 0
+    else:
+        chunk = 8
+        w = synth.as_u16(synth.normal_bf16((40_000,), seed=9, sigma=0.02, outlier_frac=1e-3))
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk)
+    assert d.flags & 2 and d.threads_per_block == 32
+    if case == "long_codes":
+        assert d.max_len == 23
+    h = B.unpack_header(b)
+    lut = B.section(b, h["off_lut"], 512 * h["n_tables"], np.uint16).tolist()
+    tables = _counted_tables(lut)
+
+    def walk_or_fail(wv):
+        r = _walk(lut, wv)
+        assert r is not None
+        return r
+    _walk_or_fail = walk_or_fail
+
+    exps, _ = odf.split(w)
+    words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
+    gaps = B.section(b, h["off_gaps"], h["n_blocks"] * 32)
+    counts = B.section(b, h["off_counts"], h["n_blocks"] * 32)
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    cw = chunk // 4
+    cbits = 32 * cw
+    seg_words = (32 * cw + 2 + 3) // 4 * 4
+    stage_bytes = (int(np.diff(blkoff).max()) + 16 + 15) // 16 * 16
+    blocks = range(h["n_blocks"]) if h["n_blocks"] <= 12 else \
+        sorted({0, 1, h["n_blocks"] // 2, h["n_blocks"] - 2, h["n_blocks"] - 1})
+    for blk in blocks:
+        o0, o1 = int(blkoff[blk]), int(blkoff[blk + 1])
+        seg0 = blk * 32 * cw
+        seg = [int(x) for x in words[seg0:seg0 + seg_words]]
+        seg += [0xDEADBEEF] * (seg_words - len(seg))    # stale buffer contents past the stream
+        cnt = [int(c) for c in counts[blk * 32:(blk + 1) * 32]]
+        first = np.concatenate([[0], np.cumsum(cnt)[:-1]]).astype(int).tolist()
+        assert sum(cnt) == o1 - o0
+        stores, slots = [], {}
+        rem_block = h["total_bits"] - blk * 32 * cbits
+        for lane in range(32):
+            qb = (o0 & 15) + first[lane]
+            start = lane * cbits + int(gaps[blk * 32 + lane])
+            nxt_gap = int(gaps[blk * 32 + lane + 1]) if lane < 31 else \
+                (int(gaps[(blk + 1) * 32]) if blk + 1 < h["n_blocks"] else 0)
+            nxt = (lane + 1) * cbits + nxt_gap if (lane < 31 or blk + 1 < h["n_blocks"]) else rem_block
+            end = min(nxt, rem_block)
+            if cnt[lane]:
+                mine = []
+                got = _decode_lane(seg, seg_words - 1, tables, start, cnt[lane], qb, mine, lane)
+                assert 0 <= got - end < 32, (blk, lane, got, end)
+                lo_w, hi_w = qb >> 2, (qb + cnt[lane] - 1) >> 2
+                for wd, val, _ in mine:
+                    if wd == "slot":
+                        slots[lane] = val
+                    else:
+                        assert lo_w <= wd <= hi_w and (wd > lo_w or qb & 3 == 0), (blk, lane, wd)
+                        assert 4 * wd + 4 <= stage_bytes
+                stores += mine
+        # word phase: each staging word written by one lane only
+        owner = {}
+        stage = bytearray(b"\xAA" * stage_bytes)
+        for wd, val, lane in stores:
+            if wd == "slot":
+                continue
+            assert owner.setdefault(wd, lane) == lane, (blk, wd)
+            stage[4 * wd:4 * wd + 4] = int(val).to_bytes(4, "little")
+        # head-byte step
+        for lane in range(32):
+            qb = (o0 & 15) + first[lane]
+            if qb & 3 and cnt[lane]:
+                hw, j0 = slots[lane], qb & 3
+                for j in range(j0, min(4, j0 + cnt[lane])):
+                    stage[(qb & ~3) + j] = (hw >> (8 * j)) & 0xFF
+        got = np.frombuffer(bytes(stage[(o0 & 15):(o0 & 15) + (o1 - o0)]), np.uint8)
+        assert np.array_equal(got, exps[o0:o1]), blk
