@@ -76,6 +76,45 @@ def test_chunk_counts_by_code_end_is_caught(monkeypatch):
     fails(pins.test_chunk_counts_match_independent_chunk_decodes, 8, 32)
 
 
+def _build_lut_with(fill_delta=0, pointer_delta=0):
+    """build_lut with one planted mistake: the fill count of every leaf off
+    by fill_delta, or the table index stored in new pointers off by
+    pointer_delta."""
+    def build(lengths):
+        codes = H.canonical_codes(lengths)
+        order = sorted((l, s) for s, l in enumerate(lengths) if l > 0)
+        tables = [[H.LUT_INVALID] * 256]
+        for l, s in order:
+            c, t, depth = codes[s], 0, 0
+            while l > 8 * (depth + 1):
+                prefix = (c >> (l - 8 * (depth + 1))) & 0xFF
+                entry = tables[t][prefix]
+                if entry == H.LUT_INVALID:
+                    tables.append([H.LUT_INVALID] * 256)
+                    entry = 0x8000 | (len(tables) - 1 + pointer_delta)
+                    tables[t][prefix] = entry
+                t = min(entry & 0x7FFF, len(tables) - 1)
+                depth += 1
+            rest = l - 8 * depth
+            low = c & ((1 << rest) - 1)
+            for fill in range(max(1, (1 << (8 - rest)) + fill_delta)):
+                tables[t][((low << (8 - rest)) | fill) & 0xFF] = (l << 8) | s
+        return tables
+    return build
+
+
+def test_lut_fill_count_off_by_one_is_caught(monkeypatch):
+    monkeypatch.setattr(H, "build_lut", _build_lut_with(fill_delta=-1))
+    fails(pins.test_golden_lookup_tables)
+    fails(pins.test_lut_lookup_matches_prefix_search)
+
+
+def test_lut_pointer_off_by_one_is_caught(monkeypatch):
+    monkeypatch.setattr(H, "build_lut", _build_lut_with(pointer_delta=1))
+    fails(pins.test_golden_lookup_tables)
+    fails(pins.test_lut_lookup_matches_prefix_search)
+
+
 def test_dropped_sign_is_caught(monkeypatch):
     good = df11.merge
     monkeypatch.setattr(df11, "merge", lambda e, s: good(e, s & np.uint8(0x7F)))

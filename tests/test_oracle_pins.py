@@ -442,6 +442,60 @@ def test_golden_df11_periodic_offsets():
         assert counts[c] == sum(1 for x in starts[:-1] if c * cb <= x < (c + 1) * cb)
 
 
+def _runs_to_table(runs):
+    t = [None] * 256
+    for lo, hi, v in runs:
+        for i in range(lo, hi + 1):
+            t[i] = v
+    assert None not in t
+    return t
+
+
+def test_golden_lookup_tables():
+    """Every entry of the hierarchical lookup tables (not only each code's
+    first one) against tables derived by hand: the worked example's single
+    table, and a two-level code with 9- and 10-bit codes behind a pointer."""
+    g = load_golden("df11_worked_example.json")
+    lengths = [0] * 256
+    for sym, l in g["lengths"].items():
+        lengths[int(sym)] = l
+    tables = H.build_lut(lengths)
+    assert len(tables) == 1
+    assert tables[0] == _runs_to_table(g["lut"]["worked_example_table0"]["runs"])
+    two = g["lut"]["two_level"]
+    lengths = [0] * 256
+    for sym, l in two["lengths"].items():
+        lengths[int(sym)] = l
+    tables = H.build_lut(lengths)
+    assert len(tables) == len(two["tables"])
+    for got, runs in zip(tables, two["tables"]):
+        assert got == _runs_to_table(runs)
+
+
+def test_lut_lookup_matches_prefix_search():
+    """lut_lookup on every 16-bit stream prefix returns the one code that is
+    a prefix of it, found by comparing the prefix with every codeword
+    (brute force), for the two-level golden code and a 4-level code."""
+    g = load_golden("df11_worked_example.json")["lut"]["two_level"]
+    two = [0] * 256
+    for sym, l in g["lengths"].items():
+        two[int(sym)] = l
+    fib = [0] * 256                       # Fibonacci-like lengths 1..24, 25: a path 4 tables deep
+    for i in range(24):
+        fib[100 + i] = i + 1
+    fib[124] = 24
+    for lengths in (two, fib):
+        codes = H.canonical_codes(lengths)
+        tables = H.build_lut(lengths)
+        words = [(s, lengths[s], codes[s]) for s in range(256) if lengths[s]]
+        rng = np.random.default_rng(7)
+        for top in range(1 << 16):
+            x = (top << 16) | int(rng.integers(0, 1 << 16))
+            want = [(s, l) for s, l, c in words if (x >> (32 - l)) == c]
+            assert len(want) == 1
+            assert H.lut_lookup(tables, x) == want[0], hex(x)
+
+
 def test_golden_clrs_huffman():
     g = load_golden("df11_worked_example.json")["clrs"]
     counts = np.zeros(256, np.uint64)
