@@ -487,13 +487,18 @@ def test_lut_lookup_matches_prefix_search():
     for lengths in (two, fib):
         codes = H.canonical_codes(lengths)
         tables = H.build_lut(lengths)
-        words = [(s, lengths[s], codes[s]) for s in range(256) if lengths[s]]
         rng = np.random.default_rng(7)
-        for top in range(1 << 16):
-            x = (top << 16) | int(rng.integers(0, 1 << 16))
-            want = [(s, l) for s, l, c in words if (x >> (32 - l)) == c]
-            assert len(want) == 1
-            assert H.lut_lookup(tables, x) == want[0], hex(x)
+        xs = (np.arange(1 << 16, dtype=np.uint64) << np.uint64(16)) | rng.integers(0, 1 << 16, 1 << 16).astype(np.uint64)
+        want_sym = np.full(xs.size, -1, np.int64)
+        want_len = np.zeros(xs.size, np.int64)
+        for sym in range(256):
+            if lengths[sym]:
+                hit = (xs >> np.uint64(32 - lengths[sym])) == np.uint64(codes[sym])
+                assert not np.any(hit & (want_sym >= 0))     # prefix-free: one code per prefix
+                want_sym[hit], want_len[hit] = sym, lengths[sym]
+        assert np.all(want_sym >= 0)                          # complete: every prefix starts a code
+        for x, ws, wl in zip(xs.tolist(), want_sym.tolist(), want_len.tolist()):
+            assert H.lut_lookup(tables, x) == (ws, wl), hex(x)
 
 
 def test_golden_clrs_huffman():
