@@ -1189,68 +1189,76 @@ struct SegWindow {
     }
 };
 
+// Stores v at shared-memory address a when p is non-zero, as a predicated
+// instruction (the lanes of a warp take different store paths every step;
+// predication keeps them on one instruction stream).
+__device__ __forceinline__ void st_shared_if(uint32_t a, uint32_t v, uint32_t p) {
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q st.shared.u32 [%0], %1;\n\t}" ::"r"(a), "r"(v),
+                 "r"(p)
+                 : "memory");
+}
+
 // Decodes `cnt` codes from bit `pos` of the segment; exponent j goes to
-// staging byte qb + j. Words of the staging area that hold none of these
-// exponents are never written; the word holding byte qb goes to *slot when
-// qb is not word aligned. Returns the bit where decoding stopped: the last
-// step takes whole table entries, so that is the end of the last code or up
-// to 30 bits past it.
+// staging byte qb + j (stage = the staging area's shared-memory address).
+// Words of the staging area that hold none of these exponents are never
+// written; the word holding byte qb goes to the lane's slot (shared address
+// `slot`) when qb is not word aligned. Each step reads 64 stream bits and
+// takes three table entries (up to nine codes). Returns the bit where
+// decoding stopped: the last step takes whole table entries, so that is the
+// end of the last code or up to 40 bits past it.
 __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t last, const uint32_t *sym,
                                                    const uint32_t *sub, uint32_t v0, const uint16_t *lut,
                                                    uint32_t ntab, uint32_t pos, uint32_t cnt, uint32_t qb,
-                                                   uint32_t *stage_w, uint32_t *slot, uint32_t &bad) {
-    uint32_t *nxt = stage_w + (qb >> 2) + 1;        // the staging word after the current one
-    uint32_t *dst = (qb & 3u) ? slot : nxt - 1;     // where the current word goes
-    const uint32_t *const lim = stage_w + ((qb + cnt + 3) >> 2);   // first word past this lane's bytes
+                                                   uint32_t stage, uint32_t slot, uint32_t &bad) {
+    uint32_t nxt = stage + 4 * ((qb >> 2) + 1);     // the staging word after the current one
+    uint32_t dst = (qb & 3u) ? slot : nxt - 4;      // where the current word goes
+    const uint32_t lim = stage + 4 * ((qb + cnt + 3) >> 2);   // first word past this lane's bytes
     uint32_t lo = 0, sh = (qb & 3u) << 3;           // pending bytes of the current word, and their bits
     int32_t k8 = (int32_t)(cnt << 3);               // exponents still to decode, x 8
-    // Appends n8/8 exponents (c1:c0, little-endian bytes, zero above them) at
-    // byte sh/8 of the current word; stores each word it completes (the
-    // second one only if it holds an exponent of this lane).
-    auto emit = [&](uint32_t c0, uint32_t c1, uint32_t n8) {
-        const uint32_t w0 = lo | (c0 << sh);
-        const uint32_t w1 = __funnelshift_lc(c0, c1, sh);
-        const uint32_t w2 = __funnelshift_lc(c1, 0u, sh);
+    // Appends the n8/8 (<= 3) exponents of entry e (low bytes) at byte sh/8
+    // of the current word and stores the word if it is complete and holds
+    // one of this lane's exponents (always true when `first`: the step's
+    // first entry starts at one of them).
+    auto emit = [&](uint32_t e, uint32_t n8, bool first) {
+        const uint32_t c = e & 0xFFFFFFu;
+        const uint32_t w = lo | (c << sh);
+        const uint32_t spill = __funnelshift_lc(c, 0u, sh);
         sh += n8;
-        if (sh >= 32) {
-            *dst = w0;
-            dst = nxt++;
-            if (sh >= 64) {
-                if (dst < lim) *dst = w1;
-                dst = nxt++;
-                lo = w2;
-            } else {
-                lo = w1;
-            }
-        } else {
-            lo = w0;
-        }
+        const uint32_t a = sh >= 32;
+        st_shared_if(dst, w, a & (first || nxt - 4 < lim));
+        dst = a ? nxt : dst;
+        nxt += a << 2;
+        lo = a ? spill : w;
         sh &= 31u;
     };
-    SegWindow win(seg, pos, last);
     while (k8 > 0) {
-        const uint32_t wv = win.at(seg, pos, last);
-        uint32_t e1 = sym[wv >> (32 - kFastBits)];
+        const uint32_t ni = min(pos >> 5, last - 2);
+        const uint32_t hi = __funnelshift_l(seg[ni + 1], seg[ni], pos);       // stream bits pos .. pos + 31
+        const uint32_t lw = __funnelshift_l(seg[ni + 2], seg[ni + 1], pos);   // pos + 32 .. pos + 63
+        uint32_t e1 = sym[hi >> (32 - kFastBits)];
         if (e1 == 0u) {   // the first code is longer than 11 bits
-            const uint32_t s = (wv >> (32 - kFastBits)) - v0;
-            if (s < kSubTables) e1 = sub[(s << 8) | ((wv >> (24 - kFastBits)) & 0xFFu)];
+            const uint32_t s = (hi >> (32 - kFastBits)) - v0;
+            if (s < kSubTables) e1 = sub[(s << 8) | ((hi >> (24 - kFastBits)) & 0xFFu)];
             if (e1 == 0u) {   // longer than 19 bits: the hierarchical tables
-                const uint32_t r = lut_walk(lut, ntab, wv, bad);
-                emit(r & 0xFFu, 0u, 8u);
+                const uint32_t r = lut_walk(lut, ntab, hi, bad);
+                emit(r & 0xFFu, 8u, true);
                 pos += r >> 8;
                 k8 -= 8;
                 continue;
             }
         }
         const uint32_t l1 = e1 >> 27;   // <= 19
-        const uint32_t e2 = sym[(wv << l1) >> (32 - kFastBits)];
-        const uint32_t n1 = (e1 >> 21) & 0x18u, n2 = (e2 >> 21) & 0x18u;
-        const uint32_t s1 = e1 & 0xFFFFFFu, s2 = e2 & 0xFFFFFFu;
-        emit(s1 | (s2 << n1), __funnelshift_lc(s2, 0u, n1), n1 + n2);
-        pos += l1 + (e2 >> 27);
-        k8 -= (int32_t)(n1 + n2);
+        const uint32_t e2 = sym[__funnelshift_l(lw, hi, l1) >> (32 - kFastBits)];
+        const uint32_t l2 = e2 >> 27;   // <= 11 (0 if the code is long: e3 then reads the same bits)
+        const uint32_t e3 = sym[__funnelshift_l(lw, hi, l1 + l2) >> (32 - kFastBits)];
+        const uint32_t n1 = (e1 >> 21) & 0x18u, n2 = (e2 >> 21) & 0x18u, n3 = (e3 >> 21) & 0x18u;
+        emit(e1, n1, true);
+        emit(e2, n2, false);
+        emit(e3, n3, false);
+        pos += l1 + l2 + (e3 >> 27);
+        k8 -= (int32_t)(n1 + n2 + n3);
     }
-    if (nxt - 1 < lim) *dst = lo;   // the last, partial word
+    st_shared_if(dst, lo, nxt - 4 < lim);   // the last, partial word
     return pos;
 }
 
@@ -1268,6 +1276,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
     const uint8_t *gapb = buf + L.gaps;
     const uint8_t *cntb = buf + L.counts;
     uint32_t *slot = reinterpret_cast<uint32_t *>(buf + L.slot) + lane;
+    const uint32_t slot_a = dev::smem_u32(slot), stage_a = dev::smem_u32(buf + L.stage);
     uint8_t *stage = buf + L.stage;
     uint32_t *first_long = reinterpret_cast<uint32_t *>(smem + L.misc);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.bars) + warp;
@@ -1319,12 +1328,23 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                 o1n = tn.blkoff[b + NW + 1];
             }
             const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
-            const uint64_t g_lo = (o0 + 15) & ~15ull, g_hi = o1 & ~15ull;
+            // merge units: 16-weight groups, or for BF16 8-weight units (one
+            // 16-byte store each, so a warp's store covers 512 contiguous bytes);
+            // the sign|mantissa bytes of each lane's first units are loaded now
+            constexpr uint32_t U = E == LWC_ELEM_BF16 ? 8u : 16u;
+            const uint64_t g_lo = (o0 + U - 1) & ~(uint64_t)(U - 1), g_hi = o1 & ~(uint64_t)(U - 1);
             uint4 sv[kWarpMergeRegs];
 #pragma unroll
             for (int m = 0; m < kWarpMergeRegs; m++) {
-                const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
-                sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
+                if constexpr (E == LWC_ELEM_BF16) {
+                    const uint64_t g = g_lo + 8ull * (lane + 64u * (uint32_t)m), h = g + 256;
+                    const uint2 a = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + g)) : make_uint2(0, 0);
+                    const uint2 c = (ok && h < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + h)) : make_uint2(0, 0);
+                    sv[m] = make_uint4(a.x, a.y, c.x, c.y);
+                } else {
+                    const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
+                    sv[m] = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint4 *>(tn.sm + g)) : make_uint4(0, 0, 0, 0);
+                }
             }
             const bool arrived = dev::mbar_wait_bounded(bar, items & 1u);
             items++;
@@ -1356,10 +1376,10 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                     const uint32_t end = (uint32_t)min(next, rem_block);
                     if (cnt) {
                         const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
-                                                            reinterpret_cast<uint32_t *>(stage), slot, bad);
-                        // the last step may decode past the lane's codes (by less than 32 bits);
+                                                            stage_a, slot_a, bad);
+                        // the last step may decode past the lane's codes (by at most 40 bits);
                         // falling short of the next chunk's first code, or far past it, means a bad count
-                        if (got - end >= 32u) bad |= LWC_DEVICE_BAD_COUNT;
+                        if (got - end > 40u) bad |= LWC_DEVICE_BAD_COUNT;
                     }
                     __syncwarp();
                     // the bytes of this lane's first, shared word
@@ -1381,19 +1401,49 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                     // 32-bit offsets from the block's first 16-weight group
                     const uint64_t base = o0 & ~15ull;
                     const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
-                    void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
-                                                  : static_cast<void *>(tn.out + base);
-                    const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
-                    const uint64_t g0 = base / 16;
                     const uint8_t *sb = tn.sm + base;
+                    if constexpr (E == LWC_ELEM_BF16) {
+                        uint16_t *ob = tn.out + base;
+                        auto merge8 = [&](uint32_t r, uint32_t sx, uint32_t sy) {
+                            const uint2 e = *reinterpret_cast<const uint2 *>(stage + r);
+                            uint4 o;
+                            merge4(sx, e.x, o.x, o.y);
+                            merge4(sy, e.y, o.z, o.w);
+                            *reinterpret_cast<uint4 *>(ob + r) = o;
+                        };
 #pragma unroll
-                    for (int m = 0; m < kWarpMergeRegs; m++) {
-                        const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
-                        if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                        for (int m = 0; m < kWarpMergeRegs; m++) {
+                            const uint32_t r = rlo + 8u * (lane + 64u * (uint32_t)m);
+                            if (r < rhi) merge8(r, sv[m].x, sv[m].y);
+                            if (r + 256 < rhi) merge8(r + 256, sv[m].z, sv[m].w);
+                        }
+                        // the rest, loads issued four at a time
+                        for (uint32_t r0 = rlo + 8u * (lane + 64u * (uint32_t)kWarpMergeRegs); r0 < rhi; r0 += 1024u) {
+                            uint2 q[4];
+#pragma unroll
+                            for (int j = 0; j < 4; j++) {
+                                const uint32_t r = r0 + 256u * j;
+                                q[j] = r < rhi ? __ldg(reinterpret_cast<const uint2 *>(sb + r)) : make_uint2(0, 0);
+                            }
+#pragma unroll
+                            for (int j = 0; j < 4; j++)
+                                if (r0 + 256u * j < rhi) merge8(r0 + 256u * j, q[j].x, q[j].y);
+                        }
+                    } else {
+                        void *ob = E == LWC_ELEM_FP32 ? static_cast<void *>(reinterpret_cast<uint32_t *>(tn.out) + base)
+                                                      : static_cast<void *>(tn.out + base);
+                        const uint8_t *lb = E == LWC_ELEM_FP32 ? tn.lo + 2 * base : tn.lo;
+                        const uint64_t g0 = base / 16;
+#pragma unroll
+                        for (int m = 0; m < kWarpMergeRegs; m++) {
+                            const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
+                            if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                        }
+                        for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
+                            merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
+                                           *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
                     }
-                    for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
-                        merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
-                                       *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                    // single weights before the first unit (lanes 0-15) and after the last (lanes 16-31)
                     const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
                     const bool head = lane < 16 && i < min(g_lo, o1);
                     const bool tail = lane >= 16 && i < o1;
