@@ -1119,7 +1119,7 @@ struct CountedLayout {
         slot = counts + 32;   // one word per lane: its first (shared) staging word
         stage = slot + 128;
         warp_bytes = stage + stage_bytes;
-        misc = warp0 + warps * warp_bytes;   // the first long 11-bit prefix
+        misc = warp0 + warps * warp_bytes;   // the first long 11-bit prefix; the next unclaimed block
         bars = misc + 16;
         total = bars + 8 * warps;
     }
@@ -1161,9 +1161,11 @@ __device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint32_
 }
 
 // Lane 0: bulk copies of block b of tensor `tn`: its stream segment, its 32
-// gaps (+ the next block's first 16) and its 32 code counts.
+// gaps (+ the next block's first 16) and its 32 code counts; and an L2
+// prefetch of the block's sign|mantissa bytes, which the merge reads.
+// (o0, o1: the block's output range, from blkoff.)
 __device__ __forceinline__ void issue_counted_item(const Df11Batch &B, const Df11Tensor &tn, uint32_t b, uint8_t *buf,
-                                                   uint32_t seg_bytes, uint64_t *bar) {
+                                                   uint32_t seg_bytes, uint64_t *bar, uint64_t o0, uint64_t o1) {
     const uint64_t seg0 = (uint64_t)b * 32u * B.chunk_words * 4;   // multiple of 128
     const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
     const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
@@ -1172,6 +1174,8 @@ __device__ __forceinline__ void issue_counted_item(const Df11Batch &B, const Df1
     if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
     dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
     dev::bulk_g2s(buf + seg_bytes + 48, tn.counts + (uint64_t)b * 32u, 32u, bar);
+    const uint64_t s0 = o0 & ~15ull, s1 = (o1 + 15) & ~15ull;
+    if (o0 < o1 && o1 <= tn.n && s1 - s0 < (1u << 20)) dev::prefetch_l2(tn.sm + s0, (uint32_t)(s1 - s0));
 }
 
 // The 32 stream bits at bit `pos` of the segment, as Window, with the word
@@ -1279,6 +1283,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
     const uint32_t slot_a = dev::smem_u32(slot), stage_a = dev::smem_u32(buf + L.stage);
     uint8_t *stage = buf + L.stage;
     uint32_t *first_long = reinterpret_cast<uint32_t *>(smem + L.misc);
+    uint32_t *claim = first_long + 1;   // the CTA's next unclaimed block of the current tensor
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.bars) + warp;
     const uint32_t seg_bytes = L.seg_bytes, last = B.seg_words - 1;
     const uint32_t cbits = B.chunk_words * 32u;
@@ -1300,7 +1305,21 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
         const Df11Tensor &tn = B.t[ti];
         const uint32_t t_end = ti + 1 < B.count ? B.t[ti + 1].first_work : W;
         const uint32_t s_end = min(w_end, t_end);
-        __syncthreads();   // every warp is done with the previous tensor's tables
+        __syncthreads();   // every warp is done with the previous tensor's tables and its own buffers
+        // warps take the tensor's first blocks in order, then claim one block
+        // at a time (so they finish together); the first block's copies
+        // overlap the table build
+        if (tid == 0) *claim = w0 + NW;
+        uint32_t w = w0 + warp;
+        uint64_t o0n = 0, o1n = 0;
+        if (w < s_end) {
+            o0n = tn.blkoff[w - tn.first_work];
+            o1n = tn.blkoff[w - tn.first_work + 1];
+            if (lane == 0 && !dead) {
+                dev::fence_proxy_async_smem();
+                issue_counted_item(B, tn, w - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
+            }
+        }
         const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
         for (uint32_t i = tid; i < ntab * 128u; i += blockDim.x)
             reinterpret_cast<uint32_t *>(lut)[i] = reinterpret_cast<const uint32_t *>(tn.lut)[i];
@@ -1309,23 +1328,16 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
         __syncthreads();
         const uint32_t v0 = *first_long;
 
-        uint32_t w = w0 + warp;
-        if (w < s_end && lane == 0 && !dead) {
-            dev::fence_proxy_async_smem();
-            issue_counted_item(B, tn, w - tn.first_work, buf, seg_bytes, bar);
-        }
-        uint64_t o0n = 0, o1n = 0;
-        if (w < s_end) {
-            o0n = tn.blkoff[w - tn.first_work];
-            o1n = tn.blkoff[w - tn.first_work + 1];
-        }
-        for (; w < s_end && !dead; w += NW) {
+        while (w < s_end && !dead) {
             const uint32_t b = w - tn.first_work;
             const uint64_t o0 = o0n, o1 = o1n;
-            const bool more = w + NW < s_end;
+            uint32_t wn = 0;   // this warp's next block
+            if (lane == 0) wn = atomicAdd(claim, 1u);
+            wn = __shfl_sync(0xFFFFFFFFu, wn, 0);
+            const bool more = wn < s_end;
             if (more) {
-                o0n = tn.blkoff[b + NW];
-                o1n = tn.blkoff[b + NW + 1];
+                o0n = tn.blkoff[wn - tn.first_work];
+                o1n = tn.blkoff[wn - tn.first_work + 1];
             }
             const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
             // merge units: 16-weight groups, or for BF16 8-weight units (one
@@ -1394,7 +1406,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                     // the segment is free: fetch this warp's next block while merging this one
                     if (lane == 0 && more) {
                         dev::fence_proxy_async_smem();
-                        issue_counted_item(B, tn, b + NW, buf, seg_bytes, bar);
+                        issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
                     }
                     next_issued = true;
 
@@ -1457,8 +1469,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
             __syncwarp();   // segment and staging area free again
             if (lane == 0 && !next_issued && more) {
                 dev::fence_proxy_async_smem();
-                issue_counted_item(B, tn, b + NW, buf, seg_bytes, bar);
+                issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
             }
+            w = wn;
         }
         w0 = s_end;
         if (w0 < w_end) ti = locate(B, w0, ti);
