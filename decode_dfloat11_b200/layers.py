@@ -110,6 +110,10 @@ class ResidentModel:
         import torch
         if codec not in CODECS:
             raise ValueError(f"unknown codec {codec!r}")
+        if slots < 2:
+            # pipelined() decodes layer L + 1 while layer L is still in use:
+            # that needs a second buffer
+            raise ValueError(f"ResidentModel needs at least 2 output buffers (got slots={slots})")
         self.codec = codec
         self.device = torch.device(device)
         self.slots = slots

@@ -391,3 +391,14 @@ def test_element_encoder_arguments():
         with pytest.raises(lwc.LwcError) as e:
             lwc.lwc_desc_from_blob(x)
         assert e.value.status == 3
+
+
+def test_resident_model_needs_two_buffers():
+    # the pipelined layer loop decodes layer L + 1 while layer L is in use:
+    # a single output buffer would let the two overlap, so it is refused
+    from decode_dfloat11_b200.layers import ResidentModel
+    with pytest.raises(ValueError):
+        ResidentModel("dfloat11", "cpu", slots=1)
+    with pytest.raises(ValueError):
+        ResidentModel("dfloat11", "cpu", slots=0)
+    assert ResidentModel("codebook", "cpu", slots=2).slots == 2
