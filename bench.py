@@ -1,21 +1,27 @@
 #!/usr/bin/env python3
 """Decode throughput of liblwc on B200.
 
-Workload: one Llama-3-8B-shaped decoder layer (q, k, v, o, gate, up, down;
-218,103,808 BF16 weights, N(0, sigma) with sigma ~ U(0.01, 0.04) and 0.1 %
-outliers x20; synthetic, seeded) compressed with the DFloat11 codec and
-resident in HBM. One step = one layer-batched decode (all seven matrices in
-one launch) into a reusable BF16 buffer. Metric: decoded BF16 GB/s (2 bytes
-per weight / step time), with the HBM roofline fraction of the decode kernel
-and bits/weight. A second line of figures times the codebook codec on the
-same layer.
+Default workload (the largest single-GPU configuration): a Llama-3-70B-shaped
+model (80 decoder layers of q 8192x8192, k/v 1024x8192, o 8192x8192, gate/up
+28672x8192, down 8192x28672, plus the 128256x8192 embedding and LM head:
+70,552,387,584 BF16 weights, N(0, sigma) with sigma ~ U(0.005, 0.03) per matrix
+and 0.1 % outliers x20; synthetic, seeded, generated and compressed on the GPU)
+held compressed with the DFloat11 codec in HBM (~94 GB). One step = one pass
+over the model: every unit (embedding, 80 layers, LM head) decoded in order,
+one layer-batched launch each, into two reusable BF16 buffers (ping-pong).
+Metric: decoded BF16 GB/s (2 bytes per weight / step time), with the HBM
+roofline fraction of the decode kernel and bits/weight.
+
+Extra keys (one GPU): the Llama-3-8B layer (decode, codebook codec, device
+encoders, FP32/FP16 element types, the decode-fused linear layer) and the
+whole Llama-3-8B model with both codecs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lwc|reference]
+                    [--workload model70b|layer|layer70b|model8b|stress]
 
-N > 1 (under torchrun): every rank decodes its own layer (layer index =
-rank) on its own GPU; no data crosses GPUs (weak scaling); the reported time
-is the maximum over ranks. --impl reference times the CPU oracle on the
-host cores instead (rank 0 only).
+N > 1 (under torchrun): every rank decodes its own replica on its own GPU; no
+data crosses GPUs (weak scaling); the reported time is the maximum over ranks.
+--impl reference times the CPU oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -36,10 +42,11 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-METRIC = "decoded BF16 GB/s (DFloat11 layer-batched decode, Llama-3-8B layer)"
+METRIC = "decoded BF16 GB/s and % of HBM roofline (1\u00d7B200); bits/weight vs BF16"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0             # B200 HBM3e, nominal
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
-DECODE_KERNEL = "df11_warp_kernel"   # blocks of 32 chunks, the encoder's default
+DECODE_KERNEL = "df11_counted_kernel"   # blobs with stored chunk counts, the encoder's default
 KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_device.cuh")
 
 
@@ -56,9 +63,13 @@ def parse_args(argv=None):
     ap.add_argument("--no-codebook", action="store_true")
     ap.add_argument("--no-linear", action="store_true", help="skip the decode-fused linear layer timing")
     ap.add_argument("--layer", type=int, default=None, help="layer seed (default: rank)")
-    ap.add_argument("--workload", choices=("layer", "model8b", "model70b", "stress"), default="layer",
-                    help="layer: one Llama-3-8B layer (default line); model8b / model70b: the whole "
-                         "model resident compressed, decoded layer by layer into ping-pong buffers")
+    ap.add_argument("--workload", choices=("model70b", "layer", "layer70b", "model8b", "stress"),
+                    default="model70b",
+                    help="model70b (default) / model8b: the whole model resident compressed, decoded "
+                         "layer by layer into ping-pong buffers; layer: one Llama-3-8B layer; layer70b: "
+                         "one Llama-3-70B layer; stress: 256M-weight codebook and uniform-exponent tensors")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default workload only: skip the Llama-3-8B layer and model keys")
     ap.add_argument("--codec", choices=("dfloat11", "codebook"), default="dfloat11",
                     help="codec of the model workloads")
     a = ap.parse_args(argv)
@@ -86,20 +97,39 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def profiled_traffic(workload: str):
+def profiled_traffic(workload: str, alg_bytes_per_launch: float | None = None):
     """DRAM bytes (read + write) per launch of the decode kernel from the
     committed ncu summary, if it was taken on the current kernel source and
-    this workload; else None. Lines: <kernel> <workload> <source sha> <bytes>."""
+    this workload; else None. Lines: <kernel> <workload> <source sha> <bytes>
+    [<algorithmic bytes of the captured launch>]. With the last field and
+    alg_bytes_per_launch, the captured traffic is scaled to this run's average
+    launch (traffic grows with the bytes a launch decodes)."""
     try:
         with open(PROFILE_TRAFFIC) as f:
             for line in f:
                 parts = line.split()
-                if len(parts) == 4 and parts[0] == DECODE_KERNEL and parts[1] == workload \
+                if len(parts) in (4, 5) and parts[0] == DECODE_KERNEL and parts[1] == workload \
                         and parts[2] == kernel_sha():
+                    if len(parts) == 5 and alg_bytes_per_launch:
+                        return int(round(int(parts[3]) * alg_bytes_per_launch / int(parts[4])))
                     return int(parts[3])
     except OSError:
         pass
     return None
+
+
+def roofline_entry(alg_bytes_per_launch: float, launch_ms: float, traffic, peak_kind_pair):
+    """The roofline object: achieved = algorithmic bytes per launch / launch
+    time, against the measured copy bandwidth (and, for context, nominal 8 TB/s)."""
+    peak, peak_kind = peak_kind_pair
+    achieved = alg_bytes_per_launch / (launch_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, a copy's bandwidth)"
+            if peak_kind == "measured" else peak_kind,
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "algorithmic_bytes_per_launch": int(round(alg_bytes_per_launch)), "kernel": DECODE_KERNEL,
+            "launch_ms": round(launch_ms, 5)}
 
 
 # ---------------------------------------------------------------- clocks
@@ -214,7 +244,7 @@ def time_steps(step, steps: int, stream):
     return start.elapsed_time(end)
 
 
-def cpu_baseline(blobs, n_total: int):
+def cpu_baseline(blobs, n_total: int, what: str = "the Llama-3-8B layer"):
     """The oracle decoder as it stands, single thread, on this host."""
     from oracle import df11 as odf
     t0 = time.perf_counter()
@@ -227,8 +257,8 @@ def cpu_baseline(blobs, n_total: int):
             break
     dt = time.perf_counter() - t0
     return {"value": round(2 * n / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"oracle bit-serial DFloat11 decode of {n:,} of the layer's {n_total:,} weights "
-                      f"(lib-encoded blobs), one host thread, {dt:.2f} s"}
+            "sample": f"oracle bit-serial DFloat11 decode of {n:,} of the {n_total:,} weights of {what} "
+                      f"(library-encoded blobs), one host thread, {dt:.2f} s"}
 
 
 def _oracle_decode_worker(job) -> int:
@@ -389,13 +419,9 @@ def run_lwc(args, rank, world, local_rank, dist):
     # roofline of the decode kernel (one launch per step here)
     peak, peak_kind = measured_peak()
     launch_ms = ms / (args.steps * launches_per_step)
-    alg_bytes = blob_bytes + 2 * n_total
-    achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
+    alg_bytes = (blob_bytes + 2 * n_total) / launches_per_step
     workload = "llama3-8b-layer-df11"
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(workload),
-                "peak_source": peak_kind, "algorithmic_bytes_per_launch": alg_bytes,
-                "kernel": DECODE_KERNEL, "launch_ms": round(launch_ms, 5)}
+    roofline = roofline_entry(alg_bytes, launch_ms, profiled_traffic(workload, alg_bytes), (peak, peak_kind))
 
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
@@ -611,37 +637,45 @@ def run_lwc(args, rank, world, local_rank, dist):
 
 def model_units(which: str, device):
     """(name, generator) per unit of a Llama-3-shaped model; generators make
-    the unit's seeded tensors on the given device."""
+    the unit's seeded tensors on the given device. layer70b: decoder layer 0
+    of the Llama-3-70B model alone."""
     if which == "model8b":
         hidden, shapes, layers, sig, off = (synth.LLAMA3_8B_HIDDEN, synth.LLAMA3_8B_LAYER,
                                             synth.LLAMA3_8B_LAYERS, (0.01, 0.04), 0)
     else:
         hidden, shapes, layers, sig, off = (synth.LLAMA3_70B_HIDDEN, synth.LLAMA3_70B_LAYER,
                                             synth.LLAMA3_70B_LAYERS, (0.005, 0.03), synth.SEED_70B_OFFSET)
-    units = [("embed", lambda: [synth.llama_embedding("embed", hidden, sig, off, device=device)])]
-    for L in range(layers):
-        units.append((f"layer{L}", lambda L=L: [t for _, t in synth.llama_layer_tensors(
-            L, shapes, sig, off, device=device)]))
-    units.append(("lm_head", lambda: [synth.llama_embedding("lm_head", hidden, sig, off, device=device)]))
-    return units
+    layer_units = [(f"layer{L}", lambda L=L: [t for _, t in synth.llama_layer_tensors(
+        L, shapes, sig, off, device=device)]) for L in range(layers)]
+    if which == "layer70b":
+        return layer_units[:1]
+    return ([("embed", lambda: [synth.llama_embedding("embed", hidden, sig, off, device=device)])] + layer_units +
+            [("lm_head", lambda: [synth.llama_embedding("lm_head", hidden, sig, off, device=device)])])
 
 
-def run_model(args, rank, world, local_rank, dist):
-    """Whole models (Llama-3-8B or Llama-3-70B shapes) resident compressed in HBM; one step
-    decodes every layer in order (one batched launch each) into two
-    reusable BF16 buffers."""
+MODEL_WORKLOADS = {"model70b": "llama3-70b-model", "model8b": "llama3-8b-model", "layer70b": "llama3-70b-layer"}
+
+
+def run_model(args, rank, world, local_rank, dist, which=None, codec=None, baselines=True):
+    """Whole models (Llama-3-8B or Llama-3-70B shapes; or one 70B layer)
+    resident compressed in HBM; one step decodes every unit in order (one
+    batched launch each) into two reusable BF16 buffers. With `baselines`
+    (the default line): the oracle timed on one layer's blobs on this host,
+    and an end-to-end pass of one layer through layers.HostPipeline."""
     import torch
     from decode_dfloat11_b200 import build as lwc_build
     from decode_dfloat11_b200 import lwc
     from decode_dfloat11_b200.layers import ResidentModel
 
+    which = which or args.workload
+    codec = codec or args.codec
     lwc_build.build()
     lwc.load()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
-    units = model_units(args.workload, device)
-    model = ResidentModel(args.codec, device)
+    units = model_units(which, device)
+    model = ResidentModel(codec, device)
     t0 = time.perf_counter()
     work = None
     for name, gen in units:   # generated on the GPU and compressed there (device encoder)
@@ -657,7 +691,7 @@ def run_model(args, rank, world, local_rank, dist):
     n_total, blob_bytes = model.weights, model.compressed_bytes
     status = torch.zeros(1, dtype=torch.int32, device=device)
 
-    # every layer checked once against its regenerated tensors
+    # every unit checked once against its regenerated tensors
     for i, (name, gen) in enumerate(units):
         model.decode(i, i % 2, stream, status)
         expect = gen()
@@ -684,26 +718,66 @@ def run_model(args, rank, world, local_rank, dist):
         dist.barrier()
     clocks = sampler.stop()
     ms_per_step = max_over_ranks(ms, dist, device) / args.steps
-    peak, peak_kind = measured_peak()
-    launch_ms = ms / (args.steps * len(units))
-    achieved = (blob_bytes + 2 * n_total) / (ms / args.steps * 1e-3) / 1e9
-    return {
-        "metric": f"decoded BF16 GB/s ({args.codec}, whole model decoded layer by layer)",
+    peak_pair = measured_peak()
+    launches = len(units)   # one batched launch per unit (every unit has several exponents)
+    launch_ms = ms / (args.steps * launches)
+    alg_per_launch = (blob_bytes + 2 * n_total) / launches
+    wl = f"{MODEL_WORKLOADS[which]}-{codec}"
+    traffic = profiled_traffic("llama3-70b-layer-dfloat11", alg_per_launch) \
+        if which in ("model70b", "layer70b") and codec == "dfloat11" else None
+    result = {
+        "metric": METRIC,
         "value": round(whole_job_gbs(world, 2 * n_total, ms_per_step), 2), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u16",
-        "data": "synthetic (seeded N(0, sigma) BF16 + 0.1% outliers x20)",
-        "config": {"workload": f"llama3-{args.workload[5:]}-model-{args.codec}", "units": len(units),
+        "data": "synthetic (seeded N(0, sigma) BF16 + 0.1% outliers x20, generated on the GPU)",
+        "config": {"workload": wl, "units": len(units),
                    "weights_per_gpu": n_total, "compressed_bytes_per_gpu": blob_bytes,
-                   "bits_per_weight": round(8 * blob_bytes / n_total, 4), "buffers": "2 x largest layer (ping-pong)",
+                   "bits_per_weight": round(8 * blob_bytes / n_total, 4),
+                   "size_vs_bf16": round(blob_bytes / (2 * n_total), 4),
+                   "buffers": "2 x largest unit (ping-pong)",
                    "setup_s": round(setup_s, 1), "setup": "tensors generated and compressed on the GPU",
-                   "parallelism": f"replicas x{world}"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None, "peak_source": peak_kind,
-                     "launch_ms": round(launch_ms, 5)},
-        "gpu_launches": args.steps * len(units),
+                   "l2": f"no flush: {(blob_bytes + 2 * n_total) / 1e9:.1f} GB moved per step > 126 MB L2",
+                   "parallelism": f"replicas x{world} (each GPU decodes its own copy; no collective)"},
+        "roofline": roofline_entry(alg_per_launch, launch_ms, traffic, peak_pair),
+        "gpu_launches": args.steps * launches,
         "clocks": clocks,
     }
+
+    if baselines and codec == "dfloat11" and which != "model8b":
+        li = next(i for i, (name, _) in enumerate(units) if name == "layer0")
+        layer = model.layers[li]
+        host_blobs = [b.cpu().numpy() for b in layer["blobs"]]
+        n_layer = sum(layer["n"])
+        if not args.no_e2e:
+            # end to end through the C ABI with host buffers, one layer per step:
+            # pinned blobs -> device, decode, decoded layer -> pinned host
+            from decode_dfloat11_b200.layers import HostPipeline
+            pipe = HostPipeline(layer["descs"], [torch.from_numpy(b) for b in host_blobs], "dfloat11", device)
+            for _ in range(3):
+                pipe.run(stream)
+            e_steps = max(3, min(args.steps, 10))
+            torch.cuda.synchronize(device)
+            ems = time_steps(lambda: pipe.run(stream), e_steps, stream) / e_steps
+            torch.cuda.synchronize(device)
+            expect = units[li][1]()
+            for t, off in zip(expect, pipe.offsets):
+                if not torch.equal(pipe.host_out.view(torch.int16)[off:off + t.numel()], t.reshape(-1).view(torch.int16).cpu()):
+                    raise SystemExit("end-to-end output differs from its input")
+            del expect
+            ev = whole_job_gbs(world, 2 * n_layer, max_over_ranks(ems, dist, device))
+            result["e2e"] = {"value": round(ev, 3), "unit": "GB/s", "h2d_bytes_per_step": pipe.h2d_bytes,
+                             "d2h_bytes_per_step": pipe.d2h_bytes, "ms_per_step": round(ems, 4), "steps": e_steps,
+                             "sample": "one step = decoder layer 0 of the model (7 matrices, "
+                                       f"{n_layer:,} weights) from pinned host blobs to pinned host BF16",
+                             "pipeline": "layers.HostPipeline: per-tensor H2D / decode / D2H on three streams"}
+            del pipe
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(host_blobs, n_layer, "one Llama-3-70B layer")
+            result["cpu_baseline_all_cores"] = cpu_baseline_all_cores(host_blobs, n_layer)
+    del model
+    torch.cuda.empty_cache()
+    return result
 
 
 # ---------------------------------------------------------------- stress tensors
@@ -766,15 +840,30 @@ def run_stress(args, rank, world, local_rank, dist):
 # ---------------------------------------------------------------- reference arm
 
 def run_reference(args):
-    """The CPU oracle as it stands, on this host's cores: one step decodes the
-    whole layer, one tensor per spawned worker process (the q matrix alone
-    when more than 200 steps are asked for, to keep the run within minutes)."""
+    """The CPU oracle as it stands, on this host's cores, for the same
+    workload and metric as our arm, each step a bounded sample of it: for the
+    whole-model workloads one matrix of layer 0 (the q matrix; generated on
+    the CPU with the same recipe), for the Llama-3-8B layer the whole layer
+    (its q matrix alone when more than 200 steps are asked for), decoded in
+    block ranges on one spawned worker process per core."""
     from decode_dfloat11_b200 import build as lwc_build
     from decode_dfloat11_b200 import lwc
     lwc_build.build()
-    names, tensors = make_layer(args.layer or 0)
-    whole = args.steps + args.warmup <= 200
-    use = tensors if whole else tensors[:1]
+    if args.workload in ("model70b", "layer70b", "model8b"):
+        seventy = args.workload != "model8b"
+        shapes = synth.LLAMA3_70B_LAYER if seventy else synth.LLAMA3_8B_LAYER
+        sig = (0.005, 0.03) if seventy else (0.01, 0.04)
+        off = synth.SEED_70B_OFFSET if seventy else 0
+        _, q = next(iter(synth.llama_layer_tensors(0, shapes, sig, off)))
+        use = [synth.as_u16(q)]
+        what = f"layer 0's q matrix ({use[0].size:,} weights, generated on the CPU with the same recipe)"
+        workload = f"{MODEL_WORKLOADS[args.workload]}-dfloat11"
+    else:
+        _, tensors = make_layer(args.layer or 0)
+        whole = args.steps + args.warmup <= 200
+        use = tensors if whole else tensors[:1]
+        what = "the whole Llama-3-8B layer" if whole else "the Llama-3-8B layer's q matrix"
+        workload = "llama3-8b-layer-df11"
     blobs = [lwc.lwc_encode_dfloat11(t)[1] for t in use]
     n = sum(t.size for t in use)
     with OraclePool(blobs) as pool:
@@ -786,14 +875,13 @@ def run_reference(args):
         dt = (time.perf_counter() - t0) / args.steps
         workers = pool.workers
     value = 2 * n / dt / 1e9
-    what = "the whole layer" if whole else "the layer's q matrix"
-    sample = (f"oracle bit-serial DFloat11 decode of {what} ({n:,} weights) per step, in block ranges on "
+    sample = (f"oracle bit-serial DFloat11 decode of {what} per step, in block ranges on "
               f"{workers} spawned workers")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u16", "data": "synthetic",
-        "config": {"workload": "llama3-8b-layer-df11", "sample": what},
+        "config": {"workload": workload, "sample": what},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": workers, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -825,6 +913,23 @@ def main(argv=None):
             result = run_stress(args, rank, world, local_rank, dist)
         else:
             result = run_model(args, rank, world, local_rank, dist)
+            if args.workload == "model70b" and world == 1 and not args.no_extras:
+                # the other workloads' figures, on the same GPU, after the 70B model is freed
+                import argparse as _ap
+                sub = _ap.Namespace(**{**vars(args), "no_e2e": False, "no_cpu_baseline": True})
+                layer = run_lwc(sub, rank, world, local_rank, dist)
+                result["llama3_8b_layer"] = {k: v for k, v in layer.items()
+                                             if k not in ("metric", "n_gpus", "steps", "warmup", "higher_is_better",
+                                                          "scaling", "vs_baseline", "dtype", "data")}
+                m8 = {}
+                for codec in ("dfloat11", "codebook"):
+                    r = run_model(sub, rank, world, local_rank, dist, which="model8b", codec=codec, baselines=False)
+                    m8[codec] = {"value": r["value"], "unit": r["unit"], "ms_per_step": r["ms_per_step"],
+                                 "bits_per_weight": r["config"]["bits_per_weight"],
+                                 "weights": r["config"]["weights_per_gpu"], "roofline": r["roofline"],
+                                 "clocks": r["clocks"]}
+                result["llama3_8b_model"] = {"workload": "llama3-8b-model (32 layers + embedding + LM head), "
+                                                         "decoded layer by layer into ping-pong buffers", **m8}
         if rank == 0:
             print(json.dumps(result), flush=True)
     finally:

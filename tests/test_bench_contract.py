@@ -10,6 +10,8 @@ import bench
 
 
 def test_reference_arm_prints_one_contract_line():
+    # the default workload (the Llama-3-70B model): each step decodes a
+    # sample of it, layer 0's q matrix
     out = io.StringIO()
     with contextlib.redirect_stdout(out):
         rc = bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
@@ -19,8 +21,10 @@ def test_reference_arm_prints_one_contract_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
     assert d["higher_is_better"] is True and d["value"] > 0 and d["steps"] == 1 and d["warmup"] == 3
+    assert d["config"]["workload"] == "llama3-70b-model-dfloat11"
     cb = d["cpu_baseline"]
-    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "whole layer" in cb["sample"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and "q matrix" in cb["sample"]
+    assert "67,108,864 weights" in cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
