@@ -1102,12 +1102,15 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
 // numerically last prefixes); longer codes walk the blob's hierarchical
 // tables.
 //
-// Symbol table entry (u32): bits 0-23 up to three exponents (first code in
-// the low byte), bits 24-25 how many (n), bits 27-31 the bits their codes
-// take; 0 means the first code is longer than 11 bits.
+// Symbol table entry (64 bits, indexed by the next 11 stream bits): the low
+// word holds up to four exponents (first code in the low byte, zero bytes
+// above them); the high word holds the bits their codes take (bits 0-4) and
+// 8 x how many there are (bits 8-13). An all-zero entry means the first code
+// is longer than 11 bits. Second-level entries are 32-bit: exponent | 1 <<
+// 24 | code length << 27, or 0.
 
-constexpr uint32_t kSubTables = 8;
-constexpr uint32_t kCtdTabBytes = kFastSize * 4 + kSubTables * 256 * 4;   // 16 KB
+constexpr uint32_t kSubTables = 2;
+constexpr uint32_t kCtdTabBytes = kFastSize * 8 + kSubTables * 256 * 4;   // 18 KB
 
 struct CountedLayout {
     uint32_t warp0, seg_bytes, gaps, counts, slot, stage, warp_bytes, misc, bars, total;
@@ -1127,13 +1130,13 @@ struct CountedLayout {
 
 // Symbol table and second-level tables of one tensor, from its hierarchical
 // tables (all threads of the CTA; barriers inside).
-__device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint32_t *sym, uint32_t *sub,
+__device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint2 *sym, uint32_t *sub,
                                      uint32_t *first_long) {
     if (threadIdx.x == 0) *first_long = kFastSize;
     __syncthreads();
     for (uint32_t v = threadIdx.x; v < kFastSize; v += blockDim.x) {
         uint32_t w = v << (32 - kFastBits), used = 0, cnt = 0, syms = 0, ignore = 0;
-        while (cnt < 3) {
+        while (cnt < 4) {
             const uint32_t r = lut_walk(lut, ntab, w, ignore);
             const uint32_t len = r >> 8;
             if (ignore || used + len > (uint32_t)kFastBits) break;
@@ -1142,7 +1145,7 @@ __device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint32_
             used += len;
             w <<= len;
         }
-        sym[v] = cnt ? (syms | (cnt << 24) | (used << 27)) : 0u;
+        sym[v] = cnt ? make_uint2(syms, used | (cnt << 11)) : make_uint2(0u, 0u);
         if (!cnt) atomicMin(first_long, v);
     }
     __syncthreads();
@@ -1207,10 +1210,10 @@ __device__ __forceinline__ void st_shared_if(uint32_t a, uint32_t v, uint32_t p)
 // Words of the staging area that hold none of these exponents are never
 // written; the word holding byte qb goes to the lane's slot (shared address
 // `slot`) when qb is not word aligned. Each step reads 64 stream bits and
-// takes three table entries (up to nine codes). Returns the bit where
+// takes three table entries (up to twelve codes). Returns the bit where
 // decoding stopped: the last step takes whole table entries, so that is the
 // end of the last code or up to 40 bits past it.
-__device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t last, const uint32_t *sym,
+__device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t last, const uint2 *sym,
                                                    const uint32_t *sub, uint32_t v0, const uint16_t *lut,
                                                    uint32_t ntab, uint32_t pos, uint32_t cnt, uint32_t qb,
                                                    uint32_t stage, uint32_t slot, uint32_t &bad) {
@@ -1219,12 +1222,11 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
     const uint32_t lim = stage + 4 * ((qb + cnt + 3) >> 2);   // first word past this lane's bytes
     uint32_t lo = 0, sh = (qb & 3u) << 3;           // pending bytes of the current word, and their bits
     int32_t k8 = (int32_t)(cnt << 3);               // exponents still to decode, x 8
-    // Appends the n8/8 (<= 3) exponents of entry e (low bytes) at byte sh/8
-    // of the current word and stores the word if it is complete and holds
-    // one of this lane's exponents (always true when `first`: the step's
-    // first entry starts at one of them).
-    auto emit = [&](uint32_t e, uint32_t n8, bool first) {
-        const uint32_t c = e & 0xFFFFFFu;
+    // Appends the n8/8 (<= 4) exponents c (low bytes, zero above them) at
+    // byte sh/8 of the current word and stores the word if it is complete and
+    // holds one of this lane's exponents (always true when `first`: the
+    // step's first entry starts at one of them).
+    auto emit = [&](uint32_t c, uint32_t n8, bool first) {
         const uint32_t w = lo | (c << sh);
         const uint32_t spill = __funnelshift_lc(c, 0u, sh);
         sh += n8;
@@ -1239,27 +1241,29 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
         const uint32_t ni = min(pos >> 5, last - 2);
         const uint32_t hi = __funnelshift_l(seg[ni + 1], seg[ni], pos);       // stream bits pos .. pos + 31
         const uint32_t lw = __funnelshift_l(seg[ni + 2], seg[ni + 1], pos);   // pos + 32 .. pos + 63
-        uint32_t e1 = sym[hi >> (32 - kFastBits)];
-        if (e1 == 0u) {   // the first code is longer than 11 bits
+        uint2 e1 = sym[hi >> (32 - kFastBits)];
+        if (e1.y == 0u) {   // the first code is longer than 11 bits
             const uint32_t s = (hi >> (32 - kFastBits)) - v0;
-            if (s < kSubTables) e1 = sub[(s << 8) | ((hi >> (24 - kFastBits)) & 0xFFu)];
-            if (e1 == 0u) {   // longer than 19 bits: the hierarchical tables
-                const uint32_t r = lut_walk(lut, ntab, hi, bad);
-                emit(r & 0xFFu, 8u, true);
-                pos += r >> 8;
+            const uint32_t r = s < kSubTables ? sub[(s << 8) | ((hi >> (24 - kFastBits)) & 0xFFu)] : 0u;
+            if (r == 0u) {   // longer than 19 bits (or a prefix without a second-level table)
+                const uint32_t t = lut_walk(lut, ntab, hi, bad);
+                emit(t & 0xFFu, 8u, true);
+                pos += t >> 8;
                 k8 -= 8;
                 continue;
             }
+            e1 = make_uint2(r & 0xFFu, (r >> 27) | (8u << 8));
         }
-        const uint32_t l1 = e1 >> 27;   // <= 19
-        const uint32_t e2 = sym[__funnelshift_l(lw, hi, l1) >> (32 - kFastBits)];
-        const uint32_t l2 = e2 >> 27;   // <= 11 (0 if the code is long: e3 then reads the same bits)
-        const uint32_t e3 = sym[__funnelshift_l(lw, hi, l1 + l2) >> (32 - kFastBits)];
-        const uint32_t n1 = (e1 >> 21) & 0x18u, n2 = (e2 >> 21) & 0x18u, n3 = (e3 >> 21) & 0x18u;
-        emit(e1, n1, true);
-        emit(e2, n2, false);
-        emit(e3, n3, false);
-        pos += l1 + l2 + (e3 >> 27);
+        const uint32_t l1 = e1.y & 31u;   // <= 19
+        const uint32_t x2 = __funnelshift_l(lw, hi, l1);   // stream bits pos + l1 .. pos + l1 + 31
+        const uint2 e2 = sym[x2 >> (32 - kFastBits)];
+        const uint32_t l2 = e2.y & 31u;   // <= 11 (0 if the code is long: e3 then reads the same bits)
+        const uint2 e3 = sym[(x2 << l2) >> (32 - kFastBits)];
+        const uint32_t n1 = e1.y >> 8, n2 = e2.y >> 8, n3 = e3.y >> 8;
+        emit(e1.x, n1, true);
+        emit(e2.x, n2, false);
+        emit(e3.x, n3, false);
+        pos += l1 + l2 + (e3.y & 31u);
         k8 -= (int32_t)(n1 + n2 + n3);
     }
     st_shared_if(dst, lo, nxt - 4 < lim);   // the last, partial word
@@ -1272,8 +1276,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const uint32_t NW = B.warps;
     const CountedLayout L(B.seg_words, B.lut_entries, B.stage_bytes, NW);
-    uint32_t *sym = reinterpret_cast<uint32_t *>(smem);
-    uint32_t *sub = sym + kFastSize;
+    uint2 *sym = reinterpret_cast<uint2 *>(smem);
+    uint32_t *sub = reinterpret_cast<uint32_t *>(smem + kFastSize * 8);
     uint16_t *lut = reinterpret_cast<uint16_t *>(smem + kCtdTabBytes);
     uint8_t *buf = smem + L.warp0 + warp * L.warp_bytes;
     const uint32_t *seg = reinterpret_cast<const uint32_t *>(buf);

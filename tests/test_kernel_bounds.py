@@ -136,7 +136,7 @@ def test_division_by_cols_is_exact_for_every_32_bit_numerator():
 # block's exponents (as the oracle decodes them).
 
 FAST_BITS = 11
-SUB_TABLES = 8
+SUB_TABLES = 2
 
 
 def _walk(lut, w):
@@ -157,11 +157,13 @@ def _walk(lut, w):
 
 
 def _counted_tables(lut):
-    sym = [0] * (1 << FAST_BITS)
+    """Symbol table (low word: up to four exponents; high word: bits used |
+    8 x count << 8) and second-level tables, as build_counted_tables."""
+    sym = [(0, 0)] * (1 << FAST_BITS)
     first_long = 1 << FAST_BITS
     for v in range(1 << FAST_BITS):
         w, used, cnt, syms = v << (32 - FAST_BITS), 0, 0, 0
-        while cnt < 3:
+        while cnt < 4:
             r = _walk(lut, w)
             if r is None or used + r[1] > FAST_BITS:
                 break
@@ -169,7 +171,7 @@ def _counted_tables(lut):
             cnt += 1
             used += r[1]
             w = (w << r[1]) & 0xFFFFFFFF
-        sym[v] = (syms | cnt << 24 | used << 27) if cnt else 0
+        sym[v] = (syms, used | (8 * cnt) << 8) if cnt else (0, 0)
         if not cnt:
             first_long = min(first_long, v)
     sub = [0] * (SUB_TABLES * 256)
@@ -196,8 +198,7 @@ def _decode_lane(seg, last, tables, pos, cnt, qb, stores, lane):
     st = {"lo": 0, "sh": (qb & 3) << 3, "nxt": (qb >> 2) + 1}
     st["dst"] = "slot" if qb & 3 else st["nxt"] - 1
 
-    def emit(e, n8, first):
-        c = e & 0xFFFFFF
+    def emit(c, n8, first):
         sh = st["sh"]
         w = st["lo"] | ((c << sh) & 0xFFFFFFFF)
         spill = _fsl(c, 0, sh)
@@ -222,25 +223,26 @@ def _decode_lane(seg, last, tables, pos, cnt, qb, stores, lane):
         hi = _fsl(word(ni + 1), word(ni), pos & 31)
         lw = _fsl(word(ni + 2), word(ni + 1), pos & 31)
         e1 = sym[hi >> (32 - FAST_BITS)]
-        if e1 == 0:
+        if e1[1] == 0:
             s = ((hi >> (32 - FAST_BITS)) - v0) & 0xFFFFFFFF
-            if s < SUB_TABLES:
-                e1 = sub[(s << 8) | ((hi >> (24 - FAST_BITS)) & 0xFF)]
-            if e1 == 0:
-                r = _walk_or_fail(hi)
-                emit(r[0], 8, True)
-                pos += r[1]
+            r = sub[(s << 8) | ((hi >> (24 - FAST_BITS)) & 0xFF)] if s < SUB_TABLES else 0
+            if r == 0:
+                t = _walk_or_fail(hi)
+                emit(t[0], 8, True)
+                pos += t[1]
                 k8 -= 8
                 continue
-        l1 = e1 >> 27
-        e2 = sym[_fsl(lw, hi, l1) >> (32 - FAST_BITS)]
-        l2 = e2 >> 27
-        e3 = sym[_fsl(lw, hi, l1 + l2) >> (32 - FAST_BITS)]
-        n1, n2, n3 = ((e >> 21) & 0x18 for e in (e1, e2, e3))
-        emit(e1, n1, True)
-        emit(e2, n2, False)
-        emit(e3, n3, False)
-        pos += l1 + l2 + (e3 >> 27)
+            e1 = (r & 0xFF, (r >> 27) | 8 << 8)
+        l1 = e1[1] & 31
+        x2 = _fsl(lw, hi, l1)
+        e2 = sym[x2 >> (32 - FAST_BITS)]
+        l2 = e2[1] & 31
+        e3 = sym[((x2 << l2) & 0xFFFFFFFF) >> (32 - FAST_BITS)]
+        n1, n2, n3 = (e[1] >> 8 for e in (e1, e2, e3))
+        emit(e1[0], n1, True)
+        emit(e2[0], n2, False)
+        emit(e3[0], n3, False)
+        pos += l1 + l2 + (e3[1] & 31)
         k8 -= n1 + n2 + n3
     if st["nxt"] - 1 < lim:
         stores.append((st["dst"], st["lo"], lane))
