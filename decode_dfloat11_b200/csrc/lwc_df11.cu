@@ -191,6 +191,23 @@ __device__ __forceinline__ void merge4(uint32_t s, uint32_t e, uint32_t &w01, ui
     w23 = __byte_perm(lo, hi, 0x7362u);
 }
 
+// The same from rotated exponents r = (e >> 1) | (e & 1) << 7, as the counted
+// decoder stages them: each byte is then one bit-select of s and r
+// (low byte: s's mantissa bits under r's top bit; high byte: r's low seven
+// bits under s's sign bit).
+__device__ __forceinline__ void merge4r(uint32_t s, uint32_t r, uint32_t &w01, uint32_t &w23) {
+    const uint32_t lo = (s & 0x7F7F7F7Fu) | (r & 0x80808080u);
+    const uint32_t hi = (r & 0x7F7F7F7Fu) | (s & 0x80808080u);
+    w01 = __byte_perm(lo, hi, 0x5140u);
+    w23 = __byte_perm(lo, hi, 0x7362u);
+}
+
+// The exponent in the low byte of e (higher bits ignored), rotated right by one bit.
+__device__ __forceinline__ uint32_t rot_exponent(uint32_t e) {
+    e &= 0xFFu;
+    return ((e >> 1) | (e << 7)) & 0xFFu;
+}
+
 __device__ __forceinline__ void merge16(const uint4 &s, const uint4 &e, uint16_t *dst) {
     uint4 r0, r1;
     merge4(s.x, e.x, r0.x, r0.y);
@@ -218,18 +235,29 @@ __device__ __forceinline__ uint32_t fp16_pair(uint32_t v2, uint32_t lo_pair) {
 // 16 elements starting at element offset r of `out` (typed by E). FP32: their
 // low halves are at lo + 2 r. FP16: `lo` is the section start (4-byte
 // aligned) and the group's 48 tail bits start at byte 6 (g0 + r / 16).
-template <int E, typename I>
+// (ROT: the exponents are rotated, see merge4r.)
+template <int E, bool ROT = false, typename I>
 __device__ __forceinline__ void merge_group(const uint4 &s, const uint4 &e, void *out, const uint8_t *lo, I r,
                                             uint64_t g0 = 0) {
-    if constexpr (E == LWC_ELEM_BF16) {
+    if constexpr (E == LWC_ELEM_BF16 && !ROT) {
         merge16(s, e, static_cast<uint16_t *>(out) + r);
     } else {
         uint4 r0, r1;
-        merge4(s.x, e.x, r0.x, r0.y);
-        merge4(s.y, e.y, r0.z, r0.w);
-        merge4(s.z, e.z, r1.x, r1.y);
-        merge4(s.w, e.w, r1.z, r1.w);
-        if constexpr (E == LWC_ELEM_FP32) {
+        if constexpr (ROT) {
+            merge4r(s.x, e.x, r0.x, r0.y);
+            merge4r(s.y, e.y, r0.z, r0.w);
+            merge4r(s.z, e.z, r1.x, r1.y);
+            merge4r(s.w, e.w, r1.z, r1.w);
+        } else {
+            merge4(s.x, e.x, r0.x, r0.y);
+            merge4(s.y, e.y, r0.z, r0.w);
+            merge4(s.z, e.z, r1.x, r1.y);
+            merge4(s.w, e.w, r1.z, r1.w);
+        }
+        if constexpr (E == LWC_ELEM_BF16) {
+            reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + r)[0] = r0;
+            reinterpret_cast<uint4 *>(static_cast<uint16_t *>(out) + r)[1] = r1;
+        } else if constexpr (E == LWC_ELEM_FP32) {
             const uint4 *lp = reinterpret_cast<const uint4 *>(lo + 2 * r);
             const uint4 l0 = __ldg(lp), l1 = __ldg(lp + 1);
             uint4 *o = reinterpret_cast<uint4 *>(static_cast<uint32_t *>(out) + r);
@@ -257,10 +285,10 @@ __device__ __forceinline__ void merge_group(const uint4 &s, const uint4 &e, void
     }
 }
 
-// One element i from its sign|mantissa byte s and exponent e.
-template <int E>
+// One element i from its sign|mantissa byte s and exponent e (rotated if ROT).
+template <int E, bool ROT = false>
 __device__ __forceinline__ void merge_one(uint32_t s, uint32_t e, void *out, const uint8_t *lo, uint64_t i) {
-    const uint32_t v = merge1(s, e);
+    const uint32_t v = merge1(s, ROT ? ((e << 1) | (e >> 7)) & 0xFFu : e);
     if constexpr (E == LWC_ELEM_BF16) {
         static_cast<uint16_t *>(out)[i] = (uint16_t)v;
     } else if constexpr (E == LWC_ELEM_FP32) {
@@ -1140,7 +1168,7 @@ __device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint2 *
             const uint32_t r = lut_walk(lut, ntab, w, ignore);
             const uint32_t len = r >> 8;
             if (ignore || used + len > (uint32_t)kFastBits) break;
-            syms |= (r & 0xFFu) << (8 * cnt);
+            syms |= rot_exponent(r) << (8 * cnt);
             cnt++;
             used += len;
             w <<= len;
@@ -1157,7 +1185,7 @@ __device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint2 *
             uint32_t ignore = 0;
             const uint32_t r = lut_walk(lut, ntab, (v << (32 - kFastBits)) | ((i & 255u) << (24 - kFastBits)), ignore);
             const uint32_t len = r >> 8;
-            if (!ignore && len > (uint32_t)kFastBits && len <= (uint32_t)kFastBits + 8) e = (r & 0xFFu) | (1u << 24) | (len << 27);
+            if (!ignore && len > (uint32_t)kFastBits && len <= (uint32_t)kFastBits + 8) e = rot_exponent(r) | (1u << 24) | (len << 27);
         }
         sub[i] = e;
     }
@@ -1247,7 +1275,7 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
             const uint32_t r = s < kSubTables ? sub[(s << 8) | ((hi >> (24 - kFastBits)) & 0xFFu)] : 0u;
             if (r == 0u) {   // longer than 19 bits (or a prefix without a second-level table)
                 const uint32_t t = lut_walk(lut, ntab, hi, bad);
-                emit(t & 0xFFu, 8u, true);
+                emit(rot_exponent(t), 8u, true);
                 pos += t >> 8;
                 k8 -= 8;
                 continue;
@@ -1423,8 +1451,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                         auto merge8 = [&](uint32_t r, uint32_t sx, uint32_t sy) {
                             const uint2 e = *reinterpret_cast<const uint2 *>(stage + r);
                             uint4 o;
-                            merge4(sx, e.x, o.x, o.y);
-                            merge4(sy, e.y, o.z, o.w);
+                            merge4r(sx, e.x, o.x, o.y);
+                            merge4r(sy, e.y, o.z, o.w);
                             *reinterpret_cast<uint4 *>(ob + r) = o;
                         };
 #pragma unroll
@@ -1453,17 +1481,17 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
 #pragma unroll
                         for (int m = 0; m < kWarpMergeRegs; m++) {
                             const uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)m);
-                            if (r < rhi) merge_group<E>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
+                            if (r < rhi) merge_group<E, true>(sv[m], *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
                         }
                         for (uint32_t r = rlo + 16u * (lane + 32u * (uint32_t)kWarpMergeRegs); r < rhi; r += 512u)
-                            merge_group<E>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
+                            merge_group<E, true>(__ldg(reinterpret_cast<const uint4 *>(sb + r)),
                                            *reinterpret_cast<const uint4 *>(stage + r), ob, lb, r, g0);
                     }
                     // single weights before the first unit (lanes 0-15) and after the last (lanes 16-31)
                     const uint64_t i = lane < 16 ? o0 + lane : max(g_hi, g_lo) + (lane - 16);
                     const bool head = lane < 16 && i < min(g_lo, o1);
                     const bool tail = lane >= 16 && i < o1;
-                    if (head || tail) merge_one<E>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
+                    if (head || tail) merge_one<E, true>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
                 } else {
                     bad |= LWC_DEVICE_BAD_COUNT;
                 }

@@ -65,7 +65,16 @@ def test_device_blob_equals_host_blob(name, w, codec):
     hd, hb = host_fn(w)
     dd, db = encode_on_device(on_gpu(w), codec)
     assert dd.as_dict() == hd.as_dict()
-    assert np.array_equal(host_bytes(db), hb)
+    dbh = host_bytes(db)
+    assert np.array_equal(dbh, hb)
+    # the device-made blob itself, checked by the oracle: its indexes (gaps,
+    # block offsets, chunk counts, tables) re-derived from a sequential
+    # decode, and its decode
+    if codec == "dfloat11":
+        assert odf.check_index(dbh) == []
+        assert np.array_equal(odf.decode(dbh), w)
+    else:
+        assert np.array_equal(ocb.decode(dbh), w)
     if w.size:
         assert np.array_equal(decode(dd, db, codec), w)
 

@@ -2,8 +2,8 @@
 layer (one batched launch per layer) into reusable BF16 ping-pong buffers.
 
 Full Llama-3-8B shapes (32 layers + embedding + LM head, 8.03 B weights) with
-both codecs resident at once, and Llama-3-70B shapes (layers sampled from the
-80, plus embedding and LM head; every tensor at full size). Every decoded
+both codecs resident at once, and Llama-3-70B shapes (three layers resident
+with the embedding and LM head; and all 82 units decoded one at a time). Every decoded
 layer is compared, on the device, with the same seeded tensors generated
 again; the oracle decodes sampled blobs on the host for an independent check."""
 import numpy as np
@@ -91,6 +91,34 @@ def test_llama3_70b_layers_full_shapes():
     df = models["dfloat11"]
     assert 10.0 < 8 * df.compressed_bytes / df.weights < 11.5
     check_all(units, models, oracle_units=("layer41",))
+
+
+def test_llama3_70b_every_unit_decodes_exactly():
+    """All 82 units of the Llama-3-70B-shaped model (embedding, the 80
+    decoder layers, LM head: 70.55 B weights), each generated on the GPU,
+    compressed there (device encoder, the blob format the bench keeps
+    resident) and decoded in one batched launch, compared bit for bit with
+    the regenerated tensors. One unit at a time, so the test holds a few GB."""
+    from decode_dfloat11_b200.layers import encode_on_device
+    units = model_units("70b", range(synth.LLAMA3_70B_LAYERS))
+    stream = torch.cuda.current_stream()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    biggest = synth.VOCAB * synth.LLAMA3_70B_HIDDEN   # the embedding and LM head
+    work = torch.empty(lwc.lwc_encode_device_workspace_bytes(biggest), dtype=torch.uint8, device="cuda")
+    total = 0
+    for name, gen in units:
+        tensors = gen()
+        enc = [encode_on_device(t, "dfloat11", workspace=work) for t in tensors]
+        outs = [torch.empty(t.numel(), dtype=torch.int16, device="cuda") for t in tensors]
+        lwc.lwc_decode_dfloat11_batched(lwc.Batch([d for d, _ in enc], [b for _, b in enc], outs),
+                                        d_status=status, stream=stream)
+        assert all(d.flags & 2 for d, _ in enc), name       # stored chunk counts: the counted decoder
+        for o, t in zip(outs, tensors):
+            assert torch.equal(o, t.reshape(-1).view(torch.int16)), name
+        total += sum(t.numel() for t in tensors)
+        del tensors, enc, outs
+    assert total == 70_552_387_584
+    assert int(status.item()) == 0
 
 
 def test_pipelined_decode_overlaps_and_never_clobbers():

@@ -133,7 +133,8 @@ def test_division_by_cols_is_exact_for_every_32_bit_numerator():
 # lanes write the same staging word, that no lane writes a word holding none
 # of its bytes, that every read of the segment stays inside the staged
 # buffer, and that after the head-byte step the staging area holds the
-# block's exponents (as the oracle decodes them).
+# block's exponents (as the oracle decodes them, each rotated right by one
+# bit, the form the merge uses).
 
 FAST_BITS = 11
 SUB_TABLES = 2
@@ -167,7 +168,7 @@ def _counted_tables(lut):
             r = _walk(lut, w)
             if r is None or used + r[1] > FAST_BITS:
                 break
-            syms |= r[0] << (8 * cnt)
+            syms |= _rot(r[0]) << (8 * cnt)
             cnt += 1
             used += r[1]
             w = (w << r[1]) & 0xFFFFFFFF
@@ -180,8 +181,13 @@ def _counted_tables(lut):
         if v < (1 << FAST_BITS):
             r = _walk(lut, (v << (32 - FAST_BITS)) | ((i & 255) << (24 - FAST_BITS)))
             if r is not None and FAST_BITS < r[1] <= FAST_BITS + 8:
-                sub[i] = r[0] | 1 << 24 | r[1] << 27
+                sub[i] = _rot(r[0]) | 1 << 24 | r[1] << 27
     return sym, sub, first_long
+
+
+def _rot(e):
+    """Exponent byte rotated right by one bit, as the tables hold it."""
+    return ((e >> 1) | (e << 7)) & 0xFF
 
 
 def _fsl(lo, hi, sh):
@@ -228,7 +234,7 @@ def _decode_lane(seg, last, tables, pos, cnt, qb, stores, lane):
             r = sub[(s << 8) | ((hi >> (24 - FAST_BITS)) & 0xFF)] if s < SUB_TABLES else 0
             if r == 0:
                 t = _walk_or_fail(hi)
-                emit(t[0], 8, True)
+                emit(_rot(t[0]), 8, True)
                 pos += t[1]
                 k8 -= 8
                 continue
@@ -347,4 +353,4 @@ def test_counted_decoder_model(case):
                 for j in range(j0, min(4, j0 + cnt[lane])):
                     stage[(qb & ~3) + j] = (hw >> (8 * j)) & 0xFF
         got = np.frombuffer(bytes(stage[(o0 & 15):(o0 & 15) + (o1 - o0)]), np.uint8)
-        assert np.array_equal(got, exps[o0:o1]), blk
+        assert np.array_equal(got, np.array([_rot(int(x)) for x in exps[o0:o1]], np.uint8)), blk
