@@ -786,7 +786,9 @@ def run_stress(args, rank, world, local_rank, dist):
     """256M-weight stress tensors, each generated and compressed on
     the GPU and decoded K times: codebook tables of U = 256 / 4096 / 8192 /
     65536 entries with Zipf(1.1) frequencies (k = 8 / 12 / 13 / 16; also
-    16384 and 32768 for k = 14 and 15), and the
+    16384, 32768 and 40000 for k = 14, 15 and a k = 16 table that is not the
+    identity: U = 65536 means every pattern, a table the decoder copies
+    through), and the
     DFloat11 edge case of uniformly random patterns (all 256 exponents, 8-bit
     codes: an expansion)."""
     import torch
@@ -801,7 +803,7 @@ def run_stress(args, rank, world, local_rank, dist):
     stream = torch.cuda.current_stream(device)
     peak, peak_kind = measured_peak()
     n = 1 << 28
-    cases = [("codebook", U) for U in (256, 4096, 8192, 16384, 32768, 65536)] + [("dfloat11", None)]
+    cases = [("codebook", U) for U in (256, 4096, 8192, 16384, 32768, 40000, 65536)] + [("dfloat11", None)]
     rows, max_ms = {}, 0.0
     for codec, U in cases:
         x = synth.codebook_stress(U, n, seed=40 + U + rank, device=device) if U else \

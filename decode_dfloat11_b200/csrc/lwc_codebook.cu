@@ -40,6 +40,12 @@ namespace {
 // table gathers, so it keeps 8.
 template <int K>
 constexpr int warps_for() { return K == 15 ? 12 : K == 14 ? 16 : 8; }
+// Tile buffers per warp (bulk copies in flight per warp). Measured on
+// 256M-weight tensors: a third buffer lifts k = 14 and 15 (whose 2-CTA SMs
+// have few warps) from 76-78 % to 84-88 % of the HBM roofline; it costs k = 13
+// a few points and does not help k = 16.
+template <int K>
+constexpr int bufs_for() { return K == 14 || K == 15 ? 3 : 2; }
 constexpr int kPerLane = 32;                            // indices per lane per tile
 constexpr uint32_t kTile = 32 * kPerLane;               // indices per tile (one warp)
 constexpr int kMaxBatch = 32;
@@ -118,10 +124,11 @@ template <int K>
 struct CbLayout {
     static constexpr uint32_t kTileBytes = 128u * K;                       // packed bytes of one tile
     static constexpr uint32_t kTabBytes = (2u << K) < 16u ? 16u : (2u << K);
-    static constexpr uint32_t kBars = 0;                                    // 2 per warp + 1 for the table
+    static constexpr uint32_t kBars = 0;                                    // NB per warp + 1 for the table
     static constexpr uint32_t kWarps = warps_for<K>();
-    static constexpr uint32_t kBufs = 8 * (2 * kWarps + 2);
-    static constexpr uint32_t kTab = kBufs + 2 * kWarps * kTileBytes;
+    static constexpr uint32_t NB = bufs_for<K>();
+    static constexpr uint32_t kBufs = (8 * (NB * kWarps + 1) + 15) / 16 * 16;
+    static constexpr uint32_t kTab = kBufs + NB * kWarps * kTileBytes;
     static constexpr uint32_t kTotal = kTab + kTabBytes;
 };
 
@@ -137,14 +144,15 @@ __device__ __forceinline__ void issue_tile(const CbTensor &tn, uint64_t tile, ui
 
 // Persistent decoder: each CTA takes a contiguous run of tiles (1024 indices
 // each) from the launch's tile list; within one tensor, warp w handles tiles
-// w, w + W, ... (W warps per CTA) of the run with its own double buffer and
-// mbarriers, so the only CTA-wide barriers are at tensor boundaries (table
-// reload).
+// w, w + W, ... (W warps per CTA) of the run with its own NB tile buffers
+// (copies issued NB tiles ahead) and mbarriers, so the only CTA-wide barriers
+// are at tensor boundaries (table reload).
 template <int K>
 __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2 : 4)   // CTAs per SM
     cb_decode_kernel(const __grid_constant__ CbBatch B) {
     using Lay = CbLayout<K>;
-    constexpr uint32_t kWarps = Lay::kWarps;
+    constexpr uint32_t kWarps = Lay::kWarps, NB = Lay::NB;
+    constexpr uint32_t kTileWords = Lay::kTileBytes / 4;
     extern __shared__ __align__(16) uint8_t smem[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Lay::kBars);
     uint32_t *bufs = reinterpret_cast<uint32_t *>(smem + Lay::kBufs);
@@ -155,11 +163,11 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
     const uint64_t t_end = B.total_tiles * (blockIdx.x + 1) / gridDim.x;
     if (t_begin >= t_end) return;
 
-    uint64_t *tab_bar = &bars[2 * kWarps];
-    uint64_t *my_bar = &bars[2 * warp];
-    uint32_t *my_buf = bufs + 2 * warp * (Lay::kTileBytes / 4);
+    uint64_t *tab_bar = &bars[NB * kWarps];
+    uint64_t *my_bar = &bars[NB * warp];
+    uint32_t *my_buf = bufs + NB * warp * kTileWords;
     if (tid == 0) {
-        for (uint32_t i = 0; i < 2 * kWarps + 1; i++) dev::mbar_init(&bars[i], 1);
+        for (uint32_t i = 0; i < NB * kWarps + 1; i++) dev::mbar_init(&bars[i], 1);
         dev::fence_mbar_init();
     }
     __syncthreads();
@@ -181,46 +189,46 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
             dev::mbar_arrive_expect_tx(tab_bar, tn.table_bytes);
             dev::bulk_g2s(tab, tn.table, tn.table_bytes, tab_bar);
         }
-        // this warp's first two tiles of the run
+        // this warp's first NB tiles of the run (use u of buffer b completes phase u & 1 of its mbarrier)
         if (lane == 0 && !dead) {
             dev::fence_proxy_async_smem();   // this warp's reads of its buffers come before the copies' writes
-            if (warp < ns) issue_tile<K>(tn, s0 + warp, my_buf + (it & 1u) * (Lay::kTileBytes / 4), &my_bar[it & 1u]);
-            if (warp + kWarps < ns)
-                issue_tile<K>(tn, s0 + warp + kWarps, my_buf + ((it + 1) & 1u) * (Lay::kTileBytes / 4),
-                              &my_bar[(it + 1) & 1u]);
+#pragma unroll
+            for (uint32_t q = 0; q < NB; q++)
+                if (warp + q * kWarps < ns)
+                    issue_tile<K>(tn, s0 + warp + q * kWarps, my_buf + ((it + q) % NB) * kTileWords,
+                                  &my_bar[(it + q) % NB]);
         }
         const bool tab_ok = dev::mbar_wait_bounded(tab_bar, tab_uses & 1u);
         tab_uses++;
         if (__syncthreads_or(!tab_ok)) {
-            // let the table copy and this warp's first two tiles land (bounded), then stop
+            // let the table copy and this warp's first tiles land (bounded), then stop
             status |= LWC_DEVICE_TIMEOUT;
             if (tid == 0) dev::mbar_wait_bounded(tab_bar, (tab_uses - 1) & 1u);
-            if (!dead) {
-                if (warp < ns) dev::mbar_wait_bounded(&my_bar[it & 1u], (it >> 1) & 1u);
-                if (warp + kWarps < ns) dev::mbar_wait_bounded(&my_bar[(it + 1) & 1u], ((it + 1) >> 1) & 1u);
-            }
+            if (!dead)
+                for (uint32_t q = 0; q < NB; q++)
+                    if (warp + q * kWarps < ns) dev::mbar_wait_bounded(&my_bar[(it + q) % NB], ((it + q) / NB) & 1u);
             break;
         }
 
         for (uint64_t j = warp; j < ns && !dead; j += kWarps, ++it) {
-            const uint32_t bi = it & 1u;
-            const bool ok = dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
+            const uint32_t bi = it % NB;
+            const bool ok = dev::mbar_wait_bounded(&my_bar[bi], (it / NB) & 1u);
             if (__any_sync(0xFFFFFFFFu, !ok)) {
-                // let this tile's copy and the one issued into the other buffer land (bounded), then stop
+                // let this tile's copy and the ones issued into the other buffers land (bounded), then stop
                 status |= LWC_DEVICE_TIMEOUT;
-                dev::mbar_wait_bounded(&my_bar[bi], (it >> 1) & 1u);
-                if (j + kWarps < ns) dev::mbar_wait_bounded(&my_bar[bi ^ 1u], ((it + 1) >> 1) & 1u);
+                for (uint32_t q = 0; q < NB; q++)
+                    if (j + q * kWarps < ns) dev::mbar_wait_bounded(&my_bar[(it + q) % NB], ((it + q) / NB) & 1u);
                 dead = true;
                 break;
             }
             uint32_t w[K + 1];
-            load_words<K>(my_buf + bi * (Lay::kTileBytes / 4) + lane * K, w);
+            load_words<K>(my_buf + bi * kTileWords + lane * K, w);
             uint32_t o[16];
             Gather<K, 0>::run(w, tab, o);
             __syncwarp();
-            if (lane == 0 && j + 2 * kWarps < ns) {
+            if (lane == 0 && j + NB * kWarps < ns) {
                 dev::fence_proxy_async_smem();
-                issue_tile<K>(tn, s0 + j + 2 * kWarps, my_buf + bi * (Lay::kTileBytes / 4), &my_bar[bi]);
+                issue_tile<K>(tn, s0 + j + NB * kWarps, my_buf + bi * kTileWords, &my_bar[bi]);
             }
             const uint64_t i0 = (s0 + j) * kTile + (uint64_t)lane * kPerLane;
             if (i0 + kPerLane <= tn.n) {
@@ -236,6 +244,34 @@ __global__ void __launch_bounds__(warps_for<K>() * 32, K == 16 ? 1 : K >= 14 ? 2
         t = seg_end;
     }
     if (status && lane == 0 && B.status) atomicOr(B.status, status);
+}
+
+// U == 65536: the table holds every 16-bit pattern in ascending order, so
+// table[j] = j and out[i] = index i: the packed 16-bit fields (least
+// significant bit first) are the weights themselves, little-endian. The
+// decode is a copy, 64 bytes per thread step; the CTAs also check the table
+// (a slice each) and report LWC_DEVICE_BAD_CODE if it is not the identity.
+__global__ void __launch_bounds__(256) cb_identity_kernel(const uint8_t *__restrict__ packed, uint16_t *__restrict__ out,
+                                                          uint64_t n, const uint16_t *__restrict__ table,
+                                                          uint32_t *status) {
+    const uint64_t tid = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x, nt = (uint64_t)gridDim.x * blockDim.x;
+    uint32_t bad = 0;
+    for (uint64_t j = tid; j < 65536; j += nt) bad |= table[j] != (uint16_t)j;
+    const uint4 *src = reinterpret_cast<const uint4 *>(packed);
+    uint4 *dst = reinterpret_cast<uint4 *>(out);
+    const uint64_t n16 = n / 8;   // whole 16-byte groups of 8 weights
+    uint64_t g = tid;
+    for (; g + 3 * nt < n16; g += 4 * nt) {
+        const uint4 a = __ldg(src + g), b = __ldg(src + g + nt), c = __ldg(src + g + 2 * nt), d = __ldg(src + g + 3 * nt);
+        dst[g] = a;
+        dst[g + nt] = b;
+        dst[g + 2 * nt] = c;
+        dst[g + 3 * nt] = d;
+    }
+    for (; g < n16; g += nt) dst[g] = __ldg(src + g);
+    const uint16_t *src16 = reinterpret_cast<const uint16_t *>(packed);
+    for (uint64_t i = 8 * n16 + tid; i < n; i += nt) out[i] = src16[i];
+    if (bad && status) atomicOr(status, LWC_DEVICE_BAD_CODE);
 }
 
 // U == 1: every weight is the single table entry.
@@ -797,11 +833,21 @@ lwc_status lwc_decode_codebook_batched(const lwc_desc *descs, const void *const 
     lwc_status st = device_state(ds);
     if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    // one-entry tables: a fill; the rest grouped by index width
+    // one-entry tables: a fill; tables of all 65536 patterns: a copy; the rest
+    // grouped by index width
     std::vector<std::vector<int>> by_k(17);
     for (int i = 0; i < count; i++) {
         const lwc_desc &d = descs[i];
         if (d.n == 0) continue;
+        if (d.U == 65536) {
+            const uint64_t blocks = std::min<uint64_t>((d.n + 32 * 256 - 1) / (32 * 256), (uint64_t)ds.sms * 8);
+            const uint8_t *base = static_cast<const uint8_t *>(d_ins[i]);
+            cb_identity_kernel<<<(unsigned)std::max<uint64_t>(blocks, 1), 256, 0, s>>>(
+                base + d.off_packed, d_outs[i], d.n, reinterpret_cast<const uint16_t *>(base + d.off_table), d_status);
+            cudaError_t err = cudaGetLastError();
+            if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "decode launch: %s", cudaGetErrorString(err));
+            continue;
+        }
         if (d.k == 0) {
             const uint64_t blocks = std::min<uint64_t>((d.n + 8 * 256 - 1) / (8 * 256), (uint64_t)ds.sms * 8);
             cb_fill_kernel<<<(unsigned)blocks, 256, 0, s>>>(

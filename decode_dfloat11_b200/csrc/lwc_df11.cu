@@ -724,8 +724,9 @@ __device__ __forceinline__ void lin_round(float (&acc)[MM], uint32_t &cur, const
 }
 
 // The linear layer's part of one decoded block [o0, o1) (exponents staged at
-// stage[i - (o0 & ~15)], sign|mantissa bytes of the first groups in sv).
-template <int MM>
+// stage[i - (o0 & ~15)], rotated as merge4r takes them if ROT; sign|mantissa
+// bytes of the first groups in sv).
+template <int MM, bool ROT = false>
 __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const Df11Tensor &tn, const uint8_t *stage,
                                           const uint4 (&sv)[kWarpMergeRegs], uint64_t o0, uint64_t o1,
                                           uint64_t g_lo, uint64_t g_hi, uint32_t lane) {
@@ -743,7 +744,7 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
         for (uint64_t i = o0 + lane; i < o1; i += 32) {
             const uint32_t r = (uint32_t)(i - base), d = d0 + r;
             const uint32_t lr = div_cols(d, magic, shifts), col = d - lr * cols;
-            const float w = bf16_lo(merge1(sb[r], stage[r]));
+            const float w = bf16_lo(merge1(sb[r], ROT ? ((stage[r] << 1) | (stage[r] >> 7)) & 0xFFu : stage[r]));
             for (uint32_t m = 0; m < M; m++)
                 atomicAdd(y + (uint64_t)m * rows + row_base + lr, w * bf16_lo(x[(uint64_t)m * cols + col]));
         }
@@ -762,7 +763,7 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
 #pragma unroll
         for (int m = 0; m < MM; m++) p[m] = 0.f;
         if (valid) {
-            const float w = bf16_lo(merge1(sb[r], stage[r]));
+            const float w = bf16_lo(merge1(sb[r], ROT ? ((stage[r] << 1) | (stage[r] >> 7)) & 0xFFu : stage[r]));
             const uint16_t *xc = x + (d - lr * cols);
 #pragma unroll
             for (int m = 0; m < MM; m++)
@@ -781,10 +782,17 @@ __device__ __forceinline__ void lin_block(const Df11Lin &X, uint32_t ti, const D
         if (valid) {
             const uint4 e = *reinterpret_cast<const uint4 *>(stage + r);
             uint32_t wv[8];
-            merge4(s.x, e.x, wv[0], wv[1]);
-            merge4(s.y, e.y, wv[2], wv[3]);
-            merge4(s.z, e.z, wv[4], wv[5]);
-            merge4(s.w, e.w, wv[6], wv[7]);
+            if constexpr (ROT) {
+                merge4r(s.x, e.x, wv[0], wv[1]);
+                merge4r(s.y, e.y, wv[2], wv[3]);
+                merge4r(s.z, e.z, wv[4], wv[5]);
+                merge4r(s.w, e.w, wv[6], wv[7]);
+            } else {
+                merge4(s.x, e.x, wv[0], wv[1]);
+                merge4(s.y, e.y, wv[2], wv[3]);
+                merge4(s.z, e.z, wv[4], wv[5]);
+                merge4(s.w, e.w, wv[6], wv[7]);
+            }
             const uint4 *xc = reinterpret_cast<const uint4 *>(x + (d - lr * cols));   // 16 columns, 32-byte aligned
 #pragma unroll
             for (int m = 0; m < MM; m++) {
@@ -1298,8 +1306,11 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
     return pos;
 }
 
-template <int E>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counted_kernel(const __grid_constant__ Df11Batch B) {
+// The counted decoder's body. LIN = 0: merge and store the weights (decoder).
+// LIN > 0: dot them with up to LIN activation rows instead (fused linear
+// layer, BF16 elements only), as in df11_warp_body.
+template <int E, int LIN>
+__device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11Lin *X) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const uint32_t NW = B.warps;
@@ -1375,12 +1386,12 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
             // merge units: 16-weight groups, or for BF16 8-weight units (one
             // 16-byte store each, so a warp's store covers 512 contiguous bytes);
             // the sign|mantissa bytes of each lane's first units are loaded now
-            constexpr uint32_t U = E == LWC_ELEM_BF16 ? 8u : 16u;
+            constexpr uint32_t U = E == LWC_ELEM_BF16 && !LIN ? 8u : 16u;
             const uint64_t g_lo = (o0 + U - 1) & ~(uint64_t)(U - 1), g_hi = o1 & ~(uint64_t)(U - 1);
             uint4 sv[kWarpMergeRegs];
 #pragma unroll
             for (int m = 0; m < kWarpMergeRegs; m++) {
-                if constexpr (E == LWC_ELEM_BF16) {
+                if constexpr (U == 8) {
                     const uint64_t g = g_lo + 8ull * (lane + 64u * (uint32_t)m), h = g + 256;
                     const uint2 a = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + g)) : make_uint2(0, 0);
                     const uint2 c = (ok && h < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + h)) : make_uint2(0, 0);
@@ -1442,6 +1453,9 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                     }
                     next_issued = true;
 
+                    if constexpr (LIN) {
+                        lin_block<LIN, true>(*X, ti, tn, stage, sv, o0, o1, g_lo, g_hi, lane);
+                    } else {
                     // 32-bit offsets from the block's first 16-weight group
                     const uint64_t base = o0 & ~15ull;
                     const uint32_t rlo = (uint32_t)(g_lo - base), rhi = (uint32_t)(g_hi - base);
@@ -1492,6 +1506,7 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
                     const bool head = lane < 16 && i < min(g_lo, o1);
                     const bool tail = lane >= 16 && i < o1;
                     if (head || tail) merge_one<E, true>(tn.sm[i], stage[i - base], tn.out, tn.lo, i);
+                    }
                 } else {
                     bad |= LWC_DEVICE_BAD_COUNT;
                 }
@@ -1511,6 +1526,19 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counte
     if (bad && B.status) atomicOr(B.status, bad);
 }
 
+template <int E>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counted_kernel(const __grid_constant__ Df11Batch B) {
+    df11_counted_body<E, 0>(B, nullptr);
+}
+
+// Fused decode + linear layer on blobs with stored chunk counts (BF16, blocks
+// of 32 chunks), for up to MM activation rows.
+template <int MM>
+__global__ void __launch_bounds__(kWarpsPerCta * 32, MM == 1 ? kWarpCtasPerSm : 1)
+    df11_counted_linear_kernel(const __grid_constant__ Df11Batch B, const __grid_constant__ Df11Lin X) {
+    df11_counted_body<LWC_ELEM_BF16, MM>(B, &X);
+}
+
 // Fused decode + linear layer (BF16 elements, blocks of 32 chunks) for up
 // to MM activation rows; with more than one row the accumulators need more
 // registers than two CTAs per SM leave.
@@ -1523,6 +1551,8 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, MM == 1 ? kWarpCtasPerSm : 
 using LinKernel = void (*)(Df11Batch, Df11Lin);
 const LinKernel kLinKernels[4] = {df11_warp_linear_kernel<1>, df11_warp_linear_kernel<2>, df11_warp_linear_kernel<4>,
                                   df11_warp_linear_kernel<8>};
+const LinKernel kCtdLinKernels[4] = {df11_counted_linear_kernel<1>, df11_counted_linear_kernel<2>,
+                                     df11_counted_linear_kernel<4>, df11_counted_linear_kernel<8>};
 int lin_index(uint32_t M) { return M <= 1 ? 0 : M <= 2 ? 1 : M <= 4 ? 2 : 3; }
 
 // One exponent value for the whole tensor: out = merge(const_exp, sm).
@@ -1571,7 +1601,8 @@ lwc_status device_config(DeviceConfig &out) {
             (const void *)df11_warp_kernel<LWC_ELEM_FP16>, (const void *)df11_counted_kernel<LWC_ELEM_BF16>,
             (const void *)df11_counted_kernel<LWC_ELEM_FP32>, (const void *)df11_counted_kernel<LWC_ELEM_FP16>,
             (const void *)kLinKernels[0], (const void *)kLinKernels[1],
-            (const void *)kLinKernels[2], (const void *)kLinKernels[3]};
+            (const void *)kLinKernels[2], (const void *)kLinKernels[3], (const void *)kCtdLinKernels[0],
+            (const void *)kCtdLinKernels[1], (const void *)kCtdLinKernels[2], (const void *)kCtdLinKernels[3]};
         for (const void *k : kernels) {
             if (err == cudaSuccess) err = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
             if (err == cudaSuccess)
@@ -1727,6 +1758,7 @@ lwc_status launch_linear_group(const std::vector<int> &idx, const lwc_desc *desc
         Df11Tensor &t = B.t[j];
         t.stream = reinterpret_cast<const uint32_t *>(base + d.off_stream);
         t.gaps = base + d.off_gaps;
+        t.counts = (d.flags & kFlagChunkCounts) ? base + d.off_counts : nullptr;
         t.blkoff = reinterpret_cast<const uint64_t *>(base + d.off_blkoff);
         t.sm = base + d.off_sm;
         t.lut = reinterpret_cast<const uint16_t *>(base + d.off_lut);
@@ -1752,13 +1784,14 @@ lwc_status launch_linear_group(const std::vector<int> &idx, const lwc_desc *desc
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
     X.M = M;
-    B.warps = warps_that_fit(B, cfg.max_smem);
+    const KernelMode mode = (d0.flags & kFlagChunkCounts) ? kModeCounted : kModeWarp;
+    B.warps = warps_that_fit(B, cfg.max_smem, mode);
     const uint32_t threads = B.warps * 32u;
-    const uint64_t smem = WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, B.warps).total;
+    const uint64_t smem = warp_smem(B, mode, B.warps);
     if (smem > (uint64_t)cfg.max_smem)
         return fail(LWC_ERR_UNSUPPORTED, "decoder needs %llu bytes of shared memory (device allows %d)",
                     (unsigned long long)smem, cfg.max_smem);
-    const LinKernel kernel = kLinKernels[lin_index(M)];
+    const LinKernel kernel = mode == kModeCounted ? kCtdLinKernels[lin_index(M)] : kLinKernels[lin_index(M)];
     int per_sm = 0;
     cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, (const void *)kernel, (int)threads,
                                                                     (size_t)smem);
@@ -1909,7 +1942,7 @@ lwc_status lwc_linear_dfloat11_batched(const lwc_desc *descs, const void *const 
             const uint64_t ny = rows * (uint64_t)M;
             const uint64_t blocks = std::min<uint64_t>((ny + 255) / 256, (uint64_t)cfg.sms * 8);
             zero_f32_kernel<<<(unsigned)blocks, 256, 0, s>>>(d_ys[i], ny);
-            keyed.push_back({d.chunk_bytes, i});
+            keyed.push_back({((uint64_t)((d.flags & kFlagChunkCounts) ? 1 : 0) << 40) | d.chunk_bytes, i});
         }
         cudaError_t err = cudaGetLastError();
         if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "linear launch: %s", cudaGetErrorString(err));

@@ -41,8 +41,15 @@ def height(codec: str, cols: int, desc) -> int:
 
 
 def encode(w_u16: np.ndarray, codec: str, **params):
-    fn = lwc.lwc_encode_dfloat11 if codec == "dfloat11" else lwc.lwc_encode_codebook
-    d, b = fn(w_u16, **params)
+    # "dfloat11_nocounts": a DFloat11 blob without stored chunk counts, which
+    # the two-pass fused kernel takes (blobs with counts take the counted one)
+    if codec == "dfloat11_nocounts":
+        d, b = lwc.lwc_encode_dfloat11(w_u16, chunk_counts=False, **params)
+        assert not d.flags & 2
+    elif codec == "dfloat11":
+        d, b = lwc.lwc_encode_dfloat11(w_u16, **params)
+    else:
+        d, b = lwc.lwc_encode_codebook(w_u16, **params)
     return d, torch.from_numpy(b).to("cuda")
 
 
@@ -50,7 +57,7 @@ def run_linear(codec, desc, blob, cols, x, M):
     rows = desc.n // cols
     y = torch.full((M, rows), float("nan"), dtype=torch.float32, device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    fn = lwc.lwc_linear_dfloat11 if codec == "dfloat11" else lwc.lwc_linear_codebook
+    fn = lwc.lwc_linear_codebook if codec == "codebook" else lwc.lwc_linear_dfloat11
     fn(desc, blob, cols, x, M, y, status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
@@ -68,7 +75,7 @@ SHAPES = [(1, 16), (1, 1), (7, 33), (5, 100), (200, 8), (33, 48), (64, 1024), (1
           (300, 4096), (3, 14336), (2, 4099)]
 
 
-@pytest.mark.parametrize("codec", ["dfloat11", "codebook"])
+@pytest.mark.parametrize("codec", ["dfloat11", "dfloat11_nocounts", "codebook"])
 @pytest.mark.parametrize("rows,cols", SHAPES)
 @pytest.mark.parametrize("M", [1, 3, 8])
 def test_linear_matches_oracle(codec, rows, cols, M):
@@ -79,7 +86,7 @@ def test_linear_matches_oracle(codec, rows, cols, M):
     check(y, w.reshape(rows, cols), x, cols, codec, d)
 
 
-@pytest.mark.parametrize("codec", ["dfloat11", "codebook"])
+@pytest.mark.parametrize("codec", ["dfloat11", "dfloat11_nocounts", "codebook"])
 @pytest.mark.parametrize("rows,cols", [(40, 48), (9, 100), (3, 1040), (70, 16)])
 def test_one_hot_sweep_checks_every_weight_exactly(codec, rows, cols):
     # x row m is one at column c_m: y[m, r] = W[r, c_m] exactly, whatever the order of the sums
@@ -187,7 +194,7 @@ def test_linear_argument_errors():
     y = torch.empty((2, 64), dtype=torch.float32, device="cuda")
     for codec in ("dfloat11", "codebook"):
         d, blob = encode(w, codec)
-        fn = lwc.lwc_linear_dfloat11 if codec == "dfloat11" else lwc.lwc_linear_codebook
+        fn = lwc.lwc_linear_codebook if codec == "codebook" else lwc.lwc_linear_dfloat11
         for M in (0, 9):
             with pytest.raises(lwc.LwcError) as e:
                 fn(d, blob, 48, x, M, y)

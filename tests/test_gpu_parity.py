@@ -103,6 +103,24 @@ def test_codebook_small(name, w):
     assert np.array_equal(got, w)
 
 
+def test_codebook_identity_table_is_checked():
+    """A table of all 65536 patterns is the identity (sorted distinct values),
+    so the decoder copies the index stream; a blob whose table is not the
+    identity is corrupt and is reported (LWC_DEVICE_BAD_CODE)."""
+    w = synth.as_u16(synth.uniform_patterns(300_007, seed=11))
+    w[:65536] = np.arange(65536, dtype=np.uint16)
+    d, b = lwc.lwc_encode_codebook(w)
+    assert d.U == 65536 and d.k == 16
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert np.array_equal(host_u16(gpu_decode(d, dev(b), codec="cb", status=status)), w)
+    assert int(status.item()) == 0
+    bad = b.copy()
+    tab = bad[d.off_table:d.off_table + 2 * 65536].view(np.uint16)
+    tab[[1000, 2000]] = tab[[2000, 1000]]    # no longer sorted: not a valid table
+    gpu_decode(d, dev(bad), codec="cb", status=status)
+    assert int(status.item()) & lwc.LWC_DEVICE_BAD_CODE
+
+
 @pytest.mark.parametrize("U", [1, 2, 3, 5, 17, 200, 256, 600, 2000, 4096, 5000, 8192, 10000, 16384, 20000, 40000,
                                65536])
 def test_codebook_every_width(U):
