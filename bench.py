@@ -491,7 +491,9 @@ def run_lwc(args, rank, world, local_rank, dist):
     if not args.no_linear:
         from decode_dfloat11_b200.layers import encode_on_device
         lin = {"workload": "llama3-8b-layer: 7 x (y = x W^T), batched call, weights decoded in registers",
-               "kernels": {"dfloat11": "df11_warp_linear_kernel", "codebook": "cb_linear_kernel"}}
+               "kernels": {"dfloat11": "df11_counted_linear_kernel", "codebook": "cb_linear_kernel"},
+               "route": "layers.fused_linear (route auto) takes the fused kernel, except DFloat11 with "
+                        "M > DF11_FUSED_MAX_M, where it decodes then multiplies"}
         src = [torch.from_numpy(w.view(np.int16)).to(device).view(torch.bfloat16).view(r, c)
                for w, (_, r, c) in zip(tensors, synth.LLAMA3_8B_LAYER)]
         for codec in ("dfloat11", "codebook"):
@@ -502,7 +504,7 @@ def run_lwc(args, rank, world, local_rank, dist):
             fn = lwc.lwc_linear_dfloat11_batched if codec == "dfloat11" else lwc.lwc_linear_codebook_batched
             dec = lwc.lwc_decode_dfloat11_batched if codec == "dfloat11" else lwc.lwc_decode_codebook_batched
             dbatch = lwc.Batch(ld, lb, views)
-            for M in (1, 4):
+            for M in (1, 2, 4):
                 xs = [synth.activations_bf16(M, t.shape[1], seed=500 + j, device=device) for j, t in enumerate(src)]
                 ys = [torch.empty((M, t.shape[0]), dtype=torch.float32, device=device) for t in src]
                 lbatch = lwc.LinearBatch(ld, lb, [t.shape[1] for t in src], xs, ys, M)
@@ -529,9 +531,13 @@ def run_lwc(args, rank, world, local_rank, dist):
                 bms = time_steps(dense, args.steps, stream) / args.steps
                 io = sum(2 * x.numel() + 4 * y.numel() for x, y in zip(xs, ys))
                 ach = (lbytes + io) / (fms * 1e-3) / 1e9
+                from decode_dfloat11_b200.layers import DF11_FUSED_MAX_M
+                route = "decode" if codec == "dfloat11" and M > DF11_FUSED_MAX_M else "fused"
                 lin[f"{codec}_M{M}"] = {
                     "fused_ms": round(fms, 5), "decode_then_matmul_ms": round(ums, 5),
                     "bf16_matmul_ms": round(bms, 5), "speedup_vs_decode_then_matmul": round(ums / fms, 3),
+                    "layers_fused_linear_route": route,
+                    "routed_speedup_vs_decode_then_matmul": round(ums / (fms if route == "fused" else ums), 3),
                     "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
                                  "frac": round(ach / peak, 4), "algorithmic_bytes_per_call": lbytes + io}}
                 del xs, ys, lbatch

@@ -74,13 +74,27 @@ def encode_on_device(tensor, codec: str = "dfloat11", workspace=None, stream=Non
     return desc, blob
 
 
-def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status=None):
+# Activation rows from which the DFloat11 decode-fused linear layer is slower
+# than decoding the matrix and running the GEMM (Llama-3-8B layer on B200:
+# fused 1.43 x faster at M = 1, 0.88 x at M = 4).
+DF11_FUSED_MAX_M = 2
+
+
+def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status=None, route: str = "auto"):
     """y = x W^T with W (``shape`` = (rows, cols), the tensor ``blob``
-    decodes to) decoded in registers; x: M x cols BF16 on the GPU, M <= 8.
-    Returns ``out`` (M x rows FP32, allocated if None)."""
+    decodes to); x: M x cols BF16 on the GPU, M <= 8. Returns ``out`` (M x
+    rows FP32, allocated if None).
+
+    route "fused": the decode-fused kernel (W decoded in registers, never
+    written); "decode": decode W into a BF16 buffer, then a BF16 x BF16 ->
+    FP32 GEMM (torch.mm; its summation order is cuBLAS's, so the bound is
+    gamma_cols); "auto": fused, except DFloat11 with more than
+    DF11_FUSED_MAX_M rows, where the fused kernel is the slower of the two."""
     import torch
     if codec not in CODECS:
         raise ValueError(f"unknown codec {codec!r}")
+    if route not in ("auto", "fused", "decode"):
+        raise ValueError(f"unknown route {route!r}")
     if len(shape) != 2:
         raise ValueError("the weight must be a rows x cols matrix")
     rows, cols = int(shape[0]), int(shape[1])
@@ -92,6 +106,16 @@ def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status
         out = torch.empty((M, rows), dtype=torch.float32, device=x.device)
     elif tuple(out.shape) != (M, rows) or out.dtype != torch.float32 or not out.is_contiguous():
         raise ValueError(f"out must be a contiguous {M} x {rows} FP32 tensor")
+    if route == "auto":
+        route = "decode" if codec == "dfloat11" and M > DF11_FUSED_MAX_M else "fused"
+    if route == "decode":
+        s = stream if stream is not None else torch.cuda.current_stream(x.device)
+        w = torch.empty((rows, cols), dtype=torch.bfloat16, device=x.device)
+        dec = lwc.lwc_decode_dfloat11_checked if codec == "dfloat11" else lwc.lwc_decode_codebook_checked
+        dec(desc, blob, w, status, s)
+        with torch.cuda.stream(s):
+            out.copy_(torch.mm(x, w.t(), out_dtype=torch.float32))
+        return out
     fn = lwc.lwc_linear_dfloat11 if codec == "dfloat11" else lwc.lwc_linear_codebook
     fn(desc, blob, cols, x, M, out, d_status=status, stream=stream)
     return out
@@ -181,15 +205,16 @@ class ResidentModel:
         else:
             lwc.lwc_decode_codebook_batched(batch, d_status=status, stream=stream)
 
-    def linear(self, layer: int, index: int, x, out=None, stream=None, status=None):
-        """y = x W^T for matrix ``index`` of ``layer`` without decoding it to
-        memory: the weights are decoded in registers by the fused kernel
-        (lwc_linear_dfloat11 / lwc_linear_codebook). x: M x cols BF16 on this
-        model's GPU, 1 <= M <= 8 (token generation); returns (or fills
-        ``out``) the M x rows FP32 result."""
+    def linear(self, layer: int, index: int, x, out=None, stream=None, status=None, route: str = "auto"):
+        """y = x W^T for matrix ``index`` of ``layer``, by default without
+        decoding it to memory: the weights are decoded in registers by the
+        fused kernel (lwc_linear_dfloat11 / lwc_linear_codebook); see
+        fused_linear for ``route``. x: M x cols BF16 on this model's GPU,
+        1 <= M <= 8 (token generation); returns (or fills ``out``) the M x rows
+        FP32 result."""
         return fused_linear(self.layers[layer]["descs"][index], self.layers[layer]["blobs"][index],
                             self.layers[layer]["shapes"][index], x, self.codec, out=out, stream=stream,
-                            status=status)
+                            status=status, route=route)
 
     def pipelined(self, compute_stream, decode_stream=None):
         """Iterate over the layers with decoding one layer ahead of use.

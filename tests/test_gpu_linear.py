@@ -245,3 +245,28 @@ def test_resident_model_linear(codec):
     with pytest.raises(ValueError):
         fused_linear(d, b, (96, 256), torch.zeros((2, 256), dtype=torch.bfloat16, device="cuda"), codec,
                      out=torch.empty((2, 95), dtype=torch.float32, device="cuda"))
+
+
+@pytest.mark.parametrize("codec", ["dfloat11", "codebook"])
+def test_fused_linear_routes(codec):
+    """layers.fused_linear picks the fused kernel or decode-then-GEMM; both
+    routes give y = x W^T within their bounds (the GEMM's: gamma_cols, its
+    summation order being cuBLAS's), and "auto" sends DFloat11 with more than
+    DF11_FUSED_MAX_M rows to the decode route."""
+    from decode_dfloat11_b200 import layers
+    rows, cols = 300, 1040
+    w = synth.as_u16(synth.normal_bf16((rows * cols,), seed=31, sigma=0.02, outlier_frac=1e-3))
+    d, blob = encode(w, codec)
+    for M in (1, 2, 3, 8):
+        x = synth.activations_bf16(M, cols, seed=40 + M, device="cuda")
+        want, mag = OL.linear(w.reshape(rows, cols), synth.as_u16(x).reshape(M, cols))
+        for route in ("auto", "fused", "decode"):
+            y = layers.fused_linear(d, blob, (rows, cols), x, codec, route=route)
+            torch.cuda.synchronize()
+            taken = "decode" if route == "decode" or (route == "auto" and codec == "dfloat11"
+                                                      and M > layers.DF11_FUSED_MAX_M) else "fused"
+            h = cols if taken == "decode" else height(codec, cols, d)
+            err = np.abs(y.cpu().numpy().astype(np.float64) - want)
+            assert np.all(err <= OL.float32_tree_bound(mag, h)), (route, M)
+    with pytest.raises(ValueError):
+        layers.fused_linear(d, blob, (rows, cols), x, codec, route="gemm")
