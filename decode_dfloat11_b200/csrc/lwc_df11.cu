@@ -1199,22 +1199,25 @@ __device__ void build_counted_tables(const uint16_t *lut, uint32_t ntab, uint2 *
     }
 }
 
-// Lane 0: bulk copies of block b of tensor `tn`: its stream segment, its 32
-// gaps (+ the next block's first 16) and its 32 code counts; and an L2
-// prefetch of the block's sign|mantissa bytes, which the merge reads.
-// (o0, o1: the block's output range, from blkoff.)
+// Lanes 0-2 of a warp (all lanes call it): the bulk copies of block b of
+// tensor `tn` into the warp's buffer -- lane 0 its stream segment, lane 1 its
+// 32 gaps (+ the next block's first 16), lane 2 its 32 code counts -- on one
+// mbarrier, whose transaction count lane 0 sets first.
 __device__ __forceinline__ void issue_counted_item(const Df11Batch &B, const Df11Tensor &tn, uint32_t b, uint8_t *buf,
-                                                   uint32_t seg_bytes, uint64_t *bar, uint64_t o0, uint64_t o1) {
+                                                   uint32_t seg_bytes, uint64_t *bar, uint32_t lane) {
     const uint64_t seg0 = (uint64_t)b * 32u * B.chunk_words * 4;   // multiple of 128
     const uint64_t avail = tn.stream_bytes > seg0 ? tn.stream_bytes - seg0 : 0;
     const uint32_t bytes = (uint32_t)(avail < seg_bytes ? avail : seg_bytes);
     const uint32_t gbytes = b + 1 < tn.n_blocks ? 48u : 32u;
-    dev::mbar_arrive_expect_tx(bar, bytes + gbytes + 32u);
-    if (bytes) dev::bulk_g2s(buf, reinterpret_cast<const uint8_t *>(tn.stream) + seg0, bytes, bar);
-    dev::bulk_g2s(buf + seg_bytes, tn.gaps + (uint64_t)b * 32u, gbytes, bar);
-    dev::bulk_g2s(buf + seg_bytes + 48, tn.counts + (uint64_t)b * 32u, 32u, bar);
-    const uint64_t s0 = o0 & ~15ull, s1 = (o1 + 15) & ~15ull;
-    if (o0 < o1 && o1 <= tn.n && s1 - s0 < (1u << 20)) dev::prefetch_l2(tn.sm + s0, (uint32_t)(s1 - s0));
+    if (lane == 0) {
+        dev::fence_proxy_async_smem();   // this warp's reads of the buffer come before the copies' writes
+        dev::mbar_arrive_expect_tx(bar, bytes + gbytes + 32u);
+    }
+    __syncwarp();
+    const uint8_t *src = lane == 0 ? reinterpret_cast<const uint8_t *>(tn.stream) + seg0
+                         : lane == 1 ? tn.gaps + (uint64_t)b * 32u : tn.counts + (uint64_t)b * 32u;
+    const uint32_t n = lane == 0 ? bytes : lane == 1 ? gbytes : 32u;
+    if (lane < 3 && n) dev::bulk_g2s(buf + (lane == 0 ? 0u : lane == 1 ? seg_bytes : seg_bytes + 48), src, n, bar);
 }
 
 // The 32 stream bits at bit `pos` of the segment, as Window, with the word
@@ -1358,10 +1361,7 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
         if (w < s_end) {
             o0n = tn.blkoff[w - tn.first_work];
             o1n = tn.blkoff[w - tn.first_work + 1];
-            if (lane == 0 && !dead) {
-                dev::fence_proxy_async_smem();
-                issue_counted_item(B, tn, w - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
-            }
+            if (!dead) issue_counted_item(B, tn, w - tn.first_work, buf, seg_bytes, bar, lane);
         }
         const uint32_t ntab = min(tn.n_tables, B.lut_entries / 256u);
         for (uint32_t i = tid; i < ntab * 128u; i += blockDim.x)
@@ -1383,18 +1383,23 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
                 o1n = tn.blkoff[wn - tn.first_work + 1];
             }
             const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes;
+            if (lane == 0 && ok && o1 > o0 && o1 - o0 < (1u << 20))   // this block's sign|mantissa bytes into L2
+                dev::prefetch_l2(tn.sm + (o0 & ~15ull), (uint32_t)(((o1 + 15) & ~15ull) - (o0 & ~15ull)));
             // merge units: 16-weight groups, or for BF16 8-weight units (one
             // 16-byte store each, so a warp's store covers 512 contiguous bytes);
             // the sign|mantissa bytes of each lane's first units are loaded now
             constexpr uint32_t U = E == LWC_ELEM_BF16 && !LIN ? 8u : 16u;
             const uint64_t g_lo = (o0 + U - 1) & ~(uint64_t)(U - 1), g_hi = o1 & ~(uint64_t)(U - 1);
             uint4 sv[kWarpMergeRegs];
+            // 32-bit offsets from the block's first unit (a block decodes fewer than 2^32 weights)
+            const uint32_t span = ok && g_hi > g_lo ? (uint32_t)(g_hi - g_lo) : 0u;
+            const uint8_t *smu = tn.sm + g_lo;
 #pragma unroll
             for (int m = 0; m < kWarpMergeRegs; m++) {
                 if constexpr (U == 8) {
-                    const uint64_t g = g_lo + 8ull * (lane + 64u * (uint32_t)m), h = g + 256;
-                    const uint2 a = (ok && g < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + g)) : make_uint2(0, 0);
-                    const uint2 c = (ok && h < g_hi) ? __ldg(reinterpret_cast<const uint2 *>(tn.sm + h)) : make_uint2(0, 0);
+                    const uint32_t g = 8u * (lane + 64u * (uint32_t)m), h = g + 256;
+                    const uint2 a = g < span ? __ldg(reinterpret_cast<const uint2 *>(smu + g)) : make_uint2(0, 0);
+                    const uint2 c = h < span ? __ldg(reinterpret_cast<const uint2 *>(smu + h)) : make_uint2(0, 0);
                     sv[m] = make_uint4(a.x, a.y, c.x, c.y);
                 } else {
                     const uint64_t g = g_lo + 16ull * (lane + 32u * (uint32_t)m);
@@ -1447,10 +1452,7 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
                     }
                     __syncwarp();
                     // the segment is free: fetch this warp's next block while merging this one
-                    if (lane == 0 && more) {
-                        dev::fence_proxy_async_smem();
-                        issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
-                    }
+                    if (more) issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, lane);
                     next_issued = true;
 
                     if constexpr (LIN) {
@@ -1514,10 +1516,7 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
                 bad |= LWC_DEVICE_BAD_OFFSET;
             }
             __syncwarp();   // segment and staging area free again
-            if (lane == 0 && !next_issued && more) {
-                dev::fence_proxy_async_smem();
-                issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, o0n, o1n);
-            }
+            if (!next_issued && more) issue_counted_item(B, tn, wn - tn.first_work, buf, seg_bytes, bar, lane);
             w = wn;
         }
         w0 = s_end;
