@@ -118,7 +118,7 @@ def profiled_traffic(workload: str, alg_bytes_per_launch: float | None = None):
     return None
 
 
-def roofline_entry(alg_bytes_per_launch: float, launch_ms: float, traffic, peak_kind_pair):
+def roofline_entry(alg_bytes_per_launch: float, launch_ms: float, traffic, peak_kind_pair, kernel=DECODE_KERNEL):
     """The roofline object: achieved = algorithmic bytes per launch / launch
     time, against the measured copy bandwidth (and, for context, nominal 8 TB/s)."""
     peak, peak_kind = peak_kind_pair
@@ -128,7 +128,7 @@ def roofline_entry(alg_bytes_per_launch: float, launch_ms: float, traffic, peak_
             "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, a copy's bandwidth)"
             if peak_kind == "measured" else peak_kind,
             "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-            "algorithmic_bytes_per_launch": int(round(alg_bytes_per_launch)), "kernel": DECODE_KERNEL,
+            "algorithmic_bytes_per_launch": int(round(alg_bytes_per_launch)), "kernel": kernel,
             "launch_ms": round(launch_ms, 5)}
 
 
@@ -745,7 +745,8 @@ def run_model(args, rank, world, local_rank, dist, which=None, codec=None, basel
                    "setup_s": round(setup_s, 1), "setup": "tensors generated and compressed on the GPU",
                    "l2": f"no flush: {(blob_bytes + 2 * n_total) / 1e9:.1f} GB moved per step > 126 MB L2",
                    "parallelism": f"replicas x{world} (each GPU decodes its own copy; no collective)"},
-        "roofline": roofline_entry(alg_per_launch, launch_ms, traffic, peak_pair),
+        "roofline": roofline_entry(alg_per_launch, launch_ms, traffic, peak_pair,
+                                   DECODE_KERNEL if codec == "dfloat11" else "cb_decode_kernel"),
         "gpu_launches": args.steps * launches,
         "clocks": clocks,
     }
