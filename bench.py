@@ -44,10 +44,12 @@ import synth  # noqa: E402
 
 METRIC = "decoded BF16 GB/s and % of HBM roofline (1\u00d7B200); bits/weight vs BF16"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 NOMINAL_HBM_GBS = 8000.0             # B200 HBM3e, nominal
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "dram_traffic.txt")
 DECODE_KERNEL = "df11_counted_kernel"   # blobs with stored chunk counts, the encoder's default
-KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_device.cuh")
+KERNEL_SOURCES = ("decode_dfloat11_b200/csrc/lwc_df11.cu", "decode_dfloat11_b200/csrc/lwc_df11_dev.cuh",
+                  "decode_dfloat11_b200/csrc/lwc_device.cuh")
 
 
 def parse_args(argv=None):
@@ -86,6 +88,37 @@ def kernel_sha() -> str:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def measured_tensor_peak():
+    """Dense BF16 tensor-core peak (TFLOP/s): the burst cuBLAS figure of
+    MEASURED_PEAKS.json (a kernel timed alone), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def mixed_roofline(bytes_moved: float, flops: float, ms: float, hbm_peak: float, tc_peak: float):
+    """Roofline of a kernel that both streams bytes and runs the tensor cores:
+    the bound is whichever of bytes / HBM peak and flops / tensor peak takes
+    longer; both fractions are reported."""
+    t_hbm = bytes_moved / (hbm_peak * 1e9)
+    t_tc = flops / (tc_peak * 1e12)
+    gbs = bytes_moved / (ms * 1e-3) / 1e9
+    tfs = flops / (ms * 1e-3) / 1e12
+    if t_hbm >= t_tc:
+        head = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(gbs / hbm_peak, 4)}
+    else:
+        head = {"bound": "tensor", "achieved": round(tfs, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": round(tfs / tc_peak, 4)}
+    head.update({"hbm_frac": round(gbs / hbm_peak, 4), "tensor_frac": round(tfs / tc_peak, 4),
+                 "algorithmic_bytes_per_call": int(bytes_moved), "flops_per_call": int(flops),
+                 "target_ms": round(max(t_hbm, t_tc) * 1e3, 5)})
+    return head
 
 
 def measured_peak():
@@ -542,6 +575,50 @@ def run_lwc(args, rank, world, local_rank, dist):
                                  "frac": round(ach / peak, 4), "algorithmic_bytes_per_call": lbytes + io}}
                 del xs, ys, lbatch
             del enc_l, ld, lb, dbatch
+
+        # the tensor-core product (prefill-size M): the weights in tile order,
+        # each 128 x 64 tile decoded straight into the MMA's shared-memory
+        # operand; against decode-then-matmul (row-major blobs) and the BF16 matmul
+        from decode_dfloat11_b200.layers import TiledWeights
+        tc_peak, _ = measured_tensor_peak()
+        tw = TiledWeights(device)
+        tidx = [tw.add(t) for t in src]
+        tbytes = tw.compressed_bytes
+        enc_d = [encode_on_device(t, "dfloat11") for t in src]
+        dbatch = lwc.Batch([d for d, _ in enc_d], [b for _, b in enc_d], views)
+        lin["kernels"]["dfloat11_tensor_core"] = "df11_gemm_kernel (tcgen05.mma, TMEM accumulator, x by TMA)"
+        for M in (16, 64, 128, 256):
+            xs = [synth.activations_bf16(M, t.shape[1], seed=700 + j, device=device) for j, t in enumerate(src)]
+            ys = [torch.empty((M, t.shape[0]), dtype=torch.float32, device=device) for t in src]
+            tb = lwc.LinearBatch(tw.descs, tw.blobs, [t.shape[1] for t in src], xs, ys, M)
+            lwc.lwc_gemm_dfloat11_batched(tb, stream=stream)
+            torch.cuda.synchronize(device)
+            for t, x, y in zip(src, xs, ys):   # consistency with torch on the same weights
+                ref = x.float() @ t.float().T
+                if not torch.allclose(y, ref, rtol=1e-3, atol=1e-3 * float(ref.abs().max())):
+                    raise SystemExit("tensor-core product disagrees with torch")
+            for _ in range(args.warmup):
+                lwc.lwc_gemm_dfloat11_batched(tb, stream=stream)
+            gms = time_steps(lambda: lwc.lwc_gemm_dfloat11_batched(tb, stream=stream), args.steps, stream) / args.steps
+
+            def unfused_tc():
+                lwc.lwc_decode_dfloat11_batched(dbatch, stream=stream)
+                for x, v, t in zip(xs, views, src):
+                    torch.mm(x, v.view(t.shape).T, out_dtype=torch.float32)
+            for _ in range(args.warmup):
+                unfused_tc()
+            ums = time_steps(unfused_tc, args.steps, stream) / args.steps
+            dense = lambda: [torch.mm(x, t.T, out_dtype=torch.float32) for x, t in zip(xs, src)]
+            for _ in range(args.warmup):
+                dense()
+            bms = time_steps(dense, args.steps, stream) / args.steps
+            io = sum(2 * x.numel() + 4 * y.numel() for x, y in zip(xs, ys))
+            lin[f"dfloat11_tc_M{M}"] = {
+                "tc_ms": round(gms, 5), "decode_then_matmul_ms": round(ums, 5), "bf16_matmul_ms": round(bms, 5),
+                "speedup_vs_decode_then_matmul": round(ums / gms, 3),
+                "roofline": mixed_roofline(tbytes + io, 2.0 * M * n_total, gms, peak, tc_peak)}
+            del xs, ys, tb
+        del tw, enc_d, dbatch
         result["linear"] = lin
         del src
 

@@ -18,9 +18,9 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "liblwc.so")
 
-CUDA_SOURCES = ["lwc_df11.cu", "lwc_codebook.cu", "lwc_encode.cu"]
+CUDA_SOURCES = ["lwc_df11.cu", "lwc_codebook.cu", "lwc_encode.cu", "lwc_gemm.cu"]
 CXX_SOURCES = ["lwc_host.cpp"]
-HEADERS = ["lwc_internal.h", "lwc_device.cuh"]
+HEADERS = ["lwc_internal.h", "lwc_device.cuh", "lwc_df11_dev.cuh", "lwc_umma.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

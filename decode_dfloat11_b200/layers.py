@@ -121,6 +121,83 @@ def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status
     return out
 
 
+# Chunk size of the blobs TiledWeights makes. A 32-chunk block of 20-byte
+# chunks holds about 2,000 exponent codes, so the product's 16 decoder warps
+# keep about four 8192-weight tiles in flight (36-byte chunks: about seven,
+# more than the shared-memory stages hold at M > 16); the price is 0.13 bits
+# per weight of chunk gaps and counts. Measured on a Llama-3-8B layer (B200):
+# 20 bytes was the fastest of 16, 20, 24 and 36 for M = 16..256.
+GEMM_CHUNK_BYTES = 20
+
+
+class TiledWeights:
+    """Weight matrices held for the tensor-core product (lwc_gemm_dfloat11):
+    each rows x cols BF16 matrix (rows % 128 == 0, cols % 64 == 0) is put in
+    tile order on the GPU (lwc_tile_order) and compressed there by the
+    DFloat11 device encoder. ``gemm`` then computes y = x W^T for 1 to 256
+    activation rows with W decoded straight into the MMA's shared-memory
+    operands (the BF16 matrix is never written to device memory)."""
+
+    def __init__(self, device):
+        self.device = device
+        self.descs, self.blobs, self.shapes = [], [], []
+
+    def add(self, w, workspace=None, stream=None, chunk_bytes: int = GEMM_CHUNK_BYTES) -> int:
+        """Tile-order and compress one rows x cols BF16 CUDA tensor; returns its index.
+        chunk_bytes: DFloat11 chunk size of the blob (see GEMM_CHUNK_BYTES)."""
+        import torch
+        if w.dim() != 2 or w.element_size() != 2 or not w.is_cuda:
+            raise ValueError("expected a rows x cols 16-bit CUDA tensor")
+        rows, cols = int(w.shape[0]), int(w.shape[1])
+        stream = stream if stream is not None else torch.cuda.current_stream(w.device)
+        src = w.contiguous()
+        tiled = torch.empty_like(src)
+        lwc.lwc_tile_order(src, rows, cols, tiled, stream)
+        with torch.cuda.stream(stream):
+            d, b = encode_on_device(tiled, "dfloat11", workspace=workspace, stream=stream, chunk_bytes=chunk_bytes)
+        del tiled
+        self.descs.append(d)
+        self.blobs.append(b)
+        self.shapes.append((rows, cols))
+        return len(self.descs) - 1
+
+    @property
+    def compressed_bytes(self) -> int:
+        return sum(int(d.total_bytes) for d in self.descs)
+
+    def _check_x(self, index: int, x):
+        import torch
+        rows, cols = self.shapes[index]
+        if x.dim() != 2 or x.shape[1] != cols or x.dtype != torch.bfloat16:
+            raise ValueError(f"x must be M x {cols} BF16")
+        return rows, cols, x.contiguous()
+
+    def gemm(self, index: int, x, out=None, stream=None, status=None):
+        """y = x W^T for matrix ``index``; x: M x cols BF16 (M <= 256). Returns
+        ``out`` (M x rows FP32, allocated if None)."""
+        import torch
+        rows, cols, x = self._check_x(index, x)
+        M = int(x.shape[0])
+        if out is None:
+            out = torch.empty((M, rows), dtype=torch.float32, device=x.device)
+        lwc.lwc_gemm_dfloat11(self.descs[index], self.blobs[index], cols, x, M, out, d_status=status, stream=stream)
+        return out
+
+    def gemm_batched(self, indices, xs, outs=None, stream=None, status=None):
+        """Several matrices (at most 8), one launch; all x share M."""
+        import torch
+        xs = [self._check_x(i, x)[2] for i, x in zip(indices, xs)]
+        M = int(xs[0].shape[0])
+        if any(int(x.shape[0]) != M for x in xs):
+            raise ValueError("all activations of a batched call share M")
+        if outs is None:
+            outs = [torch.empty((M, self.shapes[i][0]), dtype=torch.float32, device=xs[0].device) for i in indices]
+        batch = lwc.LinearBatch([self.descs[i] for i in indices], [self.blobs[i] for i in indices],
+                                [self.shapes[i][1] for i in indices], xs, outs, M)
+        lwc.lwc_gemm_dfloat11_batched(batch, d_status=status, stream=stream)
+        return outs
+
+
 class ResidentModel:
     """Compressed layers in device memory plus reusable BF16 output buffers.
 

@@ -22,6 +22,12 @@ LWC_CODEC_CODEBOOK = 2
 LWC_ELEM_BF16 = 0
 LWC_ELEM_FP32 = 1
 LWC_ELEM_FP16 = 2
+LWC_ERR_INVALID_ARG = 1
+LWC_ERR_MISALIGNED = 2
+LWC_ERR_CORRUPT = 3
+LWC_ERR_UNSUPPORTED = 4
+LWC_ERR_NOMEM = 5
+LWC_ERR_CUDA = 6
 LWC_DEVICE_BAD_COUNT = 1
 LWC_DEVICE_BAD_CODE = 2
 LWC_DEVICE_BAD_OFFSET = 4
@@ -39,6 +45,7 @@ EXPORTED = (
     "lwc_encode_dfloat11_elements_device_plan", "lwc_encode_codebook_device_plan",
     "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_linear_codebook",
     "lwc_linear_codebook_batched", "lwc_linear_dfloat11", "lwc_linear_dfloat11_batched",
+    "lwc_tile_order", "lwc_gemm_dfloat11", "lwc_gemm_dfloat11_batched",
     "lwc_selftest_bounded_wait", "lwc_status_string",
     "lwc_last_error", "lwc_version",
 )
@@ -119,7 +126,11 @@ def load():
     for name in ("lwc_linear_codebook", "lwc_linear_dfloat11"):
         getattr(L, name).argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
         getattr(L, name).restype = ctypes.c_int
-    for name in ("lwc_linear_codebook_batched", "lwc_linear_dfloat11_batched"):
+    L.lwc_gemm_dfloat11.argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
+    L.lwc_gemm_dfloat11.restype = ctypes.c_int
+    L.lwc_tile_order.argtypes = [_P, _u64, _u64, _P, _P]
+    L.lwc_tile_order.restype = ctypes.c_int
+    for name in ("lwc_linear_codebook_batched", "lwc_linear_dfloat11_batched", "lwc_gemm_dfloat11_batched"):
         getattr(L, name).argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_u64), ctypes.POINTER(_P), ctypes.c_int,
                                      ctypes.POINTER(_P), ctypes.c_int, _P, _P]
         getattr(L, name).restype = ctypes.c_int
@@ -308,6 +319,27 @@ def lwc_linear_dfloat11_batched(batch: LinearBatch, d_status=None, stream=None) 
     b = batch
     _check(load().lwc_linear_dfloat11_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
                                               _stream(stream)))
+
+
+def lwc_tile_order(d_src, rows: int, cols: int, d_dst, stream=None) -> None:
+    """Write the 128 x 64 tile order of a rows x cols BF16 device matrix
+    (the weight order lwc_gemm_dfloat11 reads) to d_dst."""
+    _check(load().lwc_tile_order(_addr(d_src), rows, cols, _addr(d_dst), _stream(stream)))
+
+
+def lwc_gemm_dfloat11(desc: lwc_desc, d_blob, cols: int, d_x, M: int, d_y, d_status=None, stream=None) -> None:
+    """y = x W^T on the tensor cores, W decoded from a tile-order DFloat11
+    blob into shared-memory operands; x: M x cols BF16, y: M x rows FP32
+    (device), M = 1 .. 256."""
+    _check(load().lwc_gemm_dfloat11(ctypes.byref(desc), _addr(d_blob), cols, _addr(d_x), M, _addr(d_y),
+                                    _addr(d_status), _stream(stream)))
+
+
+def lwc_gemm_dfloat11_batched(batch: LinearBatch, d_status=None, stream=None) -> None:
+    """Several tile-order DFloat11 matrices (at most 8) in one launch."""
+    b = batch
+    _check(load().lwc_gemm_dfloat11_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
+                                            _stream(stream)))
 
 
 def lwc_selftest_bounded_wait(d_status, polls: int, arrive: bool, stream=None) -> None:

@@ -289,6 +289,55 @@ LWC_API lwc_status lwc_linear_dfloat11_batched(const lwc_desc *descs, const void
                                                float *const *d_ys, int count, uint32_t *d_status,
                                                lwc_stream_t stream);
 
+/* ---- decode fused into a tensor-core matrix product ------------------------ */
+
+/* Tile order: the order in which lwc_gemm_dfloat11 expects a matrix's
+ * weights. W (rows x cols, row-major, rows % 128 == 0, cols % 64 == 0) is cut
+ * into 128 x 64 tiles; tile (i, j) holds rows 128 i .. 128 i + 127 and
+ * columns 64 j .. 64 j + 63; tiles follow each other by i, then j, and each
+ * tile is row-major. Writes that order of d_src (rows x cols BF16 on the
+ * device) to d_dst (same size, not overlapping); both 16-byte aligned. Encode
+ * the result with any DFloat11 encoder to get a blob for lwc_gemm_dfloat11
+ * (its plain decode then yields the tile order, not the source order).
+ * LWC_ERR_INVALID_ARG for other shapes, NULL or equal pointers. */
+LWC_API lwc_status lwc_tile_order(const uint16_t *d_src, uint64_t rows, uint64_t cols, uint16_t *d_dst,
+                                  lwc_stream_t stream);
+
+/* y = x W^T on the tensor cores (tcgen05, sm_100 only), with W decoded from
+ * a DFloat11 blob straight into shared-memory operand tiles; the BF16 matrix
+ * is never written to device memory. This is the decompression the DFloat11
+ * page places just before a layer's use ("Koniec z kompromisami! DFloat11
+ * ratuje dokładność modeli AI ...", section "Jak to działa w praktyce? Magia
+ * na poziomie GPU"), fused with the layer for batches of 1 to 256 rows.
+ *   - desc / d_blob: a DFloat11 blob of BF16 weights in tile order (see
+ *     lwc_tile_order), blocks of 32 chunks, stored chunk counts (the
+ *     encoder's defaults) and more than one exponent value; else
+ *     LWC_ERR_UNSUPPORTED. d_blob 16-byte aligned.
+ *   - cols: W's columns (a multiple of 64, at most 2^24); rows = n / cols
+ *     must be a multiple of 128 (at most 2^20); else LWC_ERR_INVALID_ARG.
+ *   - d_x: M x cols BF16 activations, row-major, 16-byte aligned.
+ *   - M: 1 .. 256.
+ *   - d_y: M x rows FP32 outputs (row-major), 4-byte aligned; every output
+ *     is written (not accumulated into). The caller owns all buffers.
+ *   - d_status: optional, as for the checked decoders; on a nonzero status
+ *     d_y is undefined.
+ * Products of two BF16 values are exact in FP32; the tensor cores add them
+ * into an FP32 accumulator in steps of 16, in an order and with an internal
+ * rounding the hardware fixes: |y - exact| <= gamma_cols * sum |W x| with
+ * gamma_k = k u / (1 - k u) and u = 2^-23 (twice FP32's unit roundoff, to
+ * cover truncating internal additions). Results repeat bit for bit from run
+ * to run. */
+LWC_API lwc_status lwc_gemm_dfloat11(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x,
+                                     int M, float *d_y, uint32_t *d_status, lwc_stream_t stream);
+
+/* `count` (at most 8) such matrices in one launch, each with its own cols[i],
+ * activations d_xs[i] and outputs d_ys[i], all with the same M and
+ * chunk_bytes; at most 4096 units of 128 rows in all. */
+LWC_API lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d_blobs,
+                                             const uint64_t *cols, const uint16_t *const *d_xs, int M,
+                                             float *const *d_ys, int count, uint32_t *d_status,
+                                             lwc_stream_t stream);
+
 /* ---- device encoders ------------------------------------------------------ */
 
 /* Compression of a tensor that is already in GPU memory, into a blob in GPU

@@ -73,13 +73,15 @@ def linear_rows(w_rows: np.ndarray, row_ids, x_bits: np.ndarray):
     return y, mag
 
 
-def float32_tree_bound(mag: np.ndarray, height: int) -> np.ndarray:
+def float32_tree_bound(mag: np.ndarray, height: int, unit_roundoff: float = 2.0 ** -24) -> np.ndarray:
     """Largest |float32 result - exact| for a sum of exact products taken
     along any summation tree in which no product passes through more than
     `height` float32 additions (or fused multiply-adds) on its way to the
     result: gamma_height * mag, u = 2^-24 (Higham, same section: each term
-    picks up one factor (1 + delta), |delta| <= u, per addition on its path)."""
-    u = 2.0 ** -24
+    picks up one factor (1 + delta), |delta| <= u, per addition on its path).
+    `unit_roundoff` replaces u for additions that may round less well than
+    round-to-nearest (2^-23 covers truncation to float32)."""
+    u = unit_roundoff
     k = max(int(height), 0)
     gamma = k * u / (1.0 - k * u)
     return gamma * np.asarray(mag, dtype=np.float64)
@@ -98,3 +100,42 @@ def from_blob(blob_bytes: np.ndarray, rows: int, cols: int, x_bits: np.ndarray):
         raise ValueError("rows * cols must equal the blob's weight count")
     w = decode(blob_bytes).reshape(rows, cols)
     return linear(w, x_bits)
+
+
+def tile_order(w_bits: np.ndarray, tile_rows: int = 128, tile_cols: int = 64) -> np.ndarray:
+    """The weights of a rows x cols matrix in tile order, flat: the matrix is
+    cut into tile_rows x tile_cols tiles; tile (i, j) holds rows
+    i*tile_rows .. (i+1)*tile_rows - 1 and columns j*tile_cols ..
+    (j+1)*tile_cols - 1; tiles follow one another by i, then by j, and each
+    tile is read row by row. This is the weight order the library's
+    tensor-core product reads (a layout of this library; the pages do not
+    fix one). Written tile by tile, as the definition reads."""
+    w = np.asarray(w_bits)
+    if w.ndim != 2:
+        raise ValueError("expected a rows x cols matrix")
+    rows, cols = w.shape
+    if rows % tile_rows or cols % tile_cols:
+        raise ValueError("rows and cols must be multiples of the tile size")
+    pieces = []
+    for i in range(rows // tile_rows):
+        for j in range(cols // tile_cols):
+            tile = w[i * tile_rows:(i + 1) * tile_rows, j * tile_cols:(j + 1) * tile_cols]
+            pieces.append(tile.reshape(-1))
+    return np.concatenate(pieces) if pieces else w.reshape(-1).copy()
+
+
+def from_tile_order(flat: np.ndarray, rows: int, cols: int, tile_rows: int = 128, tile_cols: int = 64) -> np.ndarray:
+    """The rows x cols matrix whose tile order is `flat` (inverse of
+    tile_order), again tile by tile."""
+    flat = np.asarray(flat).reshape(-1)
+    if flat.size != rows * cols or rows % tile_rows or cols % tile_cols:
+        raise ValueError("size and tile multiples do not match")
+    w = np.empty((rows, cols), dtype=flat.dtype)
+    k = 0
+    for i in range(rows // tile_rows):
+        for j in range(cols // tile_cols):
+            n = tile_rows * tile_cols
+            w[i * tile_rows:(i + 1) * tile_rows, j * tile_cols:(j + 1) * tile_cols] = \
+                flat[k:k + n].reshape(tile_rows, tile_cols)
+            k += n
+    return w

@@ -354,3 +354,102 @@ def test_counted_decoder_model(case):
                     stage[(qb & ~3) + j] = (hw >> (8 * j)) & 0xFF
         got = np.frombuffer(bytes(stage[(o0 & 15):(o0 & 15) + (o1 - o0)]), np.uint8)
         assert np.array_equal(got, np.array([_rot(int(x)) for x in exps[o0:o1]], np.uint8)), blk
+
+
+# ---- decode into tensor-core tiles (csrc/lwc_gemm.cu, df11_gemm_kernel) ------------
+#
+# Restates, on the CPU, how the decoder warps place the weights of a
+# tile-order DFloat11 blob into the 128 x 64 swizzled stage tiles: each unit
+# (128 rows, all columns) takes the blocks from the last one starting at or
+# before its first weight to the last one starting before its end; a block
+# writes its part of the unit as 8-weight pieces (one 16-byte chunk each)
+# plus up to 7 single weights at either end, and adds to each tile it touches
+# the number of weights it wrote there. Checked: every tile gets each of its
+# 8192 slots exactly once, with the right weight, and its count reaches 8192
+# exactly; a block touches at most two tiles.
+
+def _sw128(r, c):
+    return r * 128 + ((((c >> 3) ^ r) & 7) << 4) + ((c & 7) << 1)
+
+
+def _last_le(blkoff, n_blocks, v):
+    a, b = 0, n_blocks
+    while b - a > 1:
+        mid = a + (b - a) // 2
+        if blkoff[mid] <= v:
+            a = mid
+        else:
+            b = mid
+    return a
+
+
+def _gemm_placement(blkoff, n_blocks, tiled, rows, cols, cta_units):
+    kt = cols // 64
+    slots = {}      # tile sequence number -> {byte offset: weight}
+    counts = {}
+    t0 = 0
+    for u in cta_units:
+        lo, hi = u * 128 * cols, (u + 1) * 128 * cols
+        first, last = _last_le(blkoff, n_blocks, lo), _last_le(blkoff, n_blocks, hi - 1)
+        for b in range(first, last + 1):
+            o0, o1 = int(blkoff[b]), int(blkoff[b + 1])
+            assert o0 <= o1 and o0 < hi and o1 > lo
+            p_lo, p_hi = max(o0, lo), min(o1, hi)
+            qa, qz = t0 + (p_lo - lo) // 8192, t0 + (p_hi - 1 - lo) // 8192
+            assert qz - qa <= 1
+
+            def put(i):
+                t = i - lo
+                q, idx = t0 + t // 8192, t % 8192
+                off = _sw128(idx >> 6, idx & 63)
+                assert off not in slots.setdefault(q, {})
+                slots[q][off] = int(tiled[i])
+
+            g_lo, g_hi = (p_lo + 7) & ~7, p_hi & ~7
+            for pos in range(g_lo, g_hi, 8):
+                t = pos - lo
+                q, idx = t0 + t // 8192, t % 8192
+                base = _sw128(idx >> 6, idx & 63)
+                assert base % 16 == 0
+                for j in range(8):   # one 16-byte chunk: weights pos .. pos + 7 in order
+                    assert base + 2 * j not in slots.setdefault(q, {})
+                    slots[q][base + 2 * j] = int(tiled[pos + j])
+            for lane in range(16):
+                i = p_lo + lane if lane < 8 else max(g_hi, g_lo) + (lane - 8)
+                if (lane < 8 and i < min(g_lo, p_hi)) or (lane >= 8 and i < p_hi):
+                    put(i)
+            for q in range(qa, qz + 1):
+                tlo = lo + (q - t0) * 8192
+                counts[q] = counts.get(q, 0) + min(p_hi, tlo + 8192) - max(p_lo, tlo)
+        t0 += kt
+    return slots, counts
+
+
+@pytest.mark.parametrize("rows,cols,chunk,order", [(384, 320, 36, "plain"), (256, 64, 8, "plain"),
+                                                   (512, 192, 36, "shuffled"), (128, 1024, 12, "plain")])
+def test_gemm_tile_placement_model(rows, cols, chunk, order):
+    import synth
+    from decode_dfloat11_b200 import lwc
+    from oracle import blob as B
+    from oracle import linear as OL
+
+    w = synth.as_u16(synth.normal_bf16((rows, cols), seed=rows + cols, sigma=0.02, outlier_frac=0.01)).reshape(rows, cols)
+    tiled = OL.tile_order(w)
+    d, b = lwc.lwc_encode_dfloat11(tiled, chunk_bytes=chunk)
+    assert d.flags & 2
+    h = B.unpack_header(b)
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    units = list(range(rows // 128))
+    if order == "shuffled":
+        units = units[::-1]
+    slots, counts = _gemm_placement(blkoff, h["n_blocks"], tiled, rows, cols, units)
+    kt = cols // 64
+    assert sorted(counts) == list(range(len(units) * kt))
+    assert all(c == 8192 for c in counts.values())
+    for k, u in enumerate(units):
+        for j in range(kt):
+            q = k * kt + j
+            assert len(slots[q]) == 8192
+            for r in (0, 1, 7, 8, 63, 127):
+                for c in (0, 5, 8, 31, 63):
+                    assert slots[q][_sw128(r, c)] == w[u * 128 + r, j * 64 + c]

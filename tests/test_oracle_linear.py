@@ -143,3 +143,36 @@ def test_from_blob_both_codecs():
         assert np.array_equal(y, want)
     with pytest.raises(ValueError):
         OL.from_blob(df11.encode(w), rows, cols + 1, x)
+
+
+def test_golden_tile_order():
+    """The tile order of a hand-worked 4 x 6 example (2 x 3 tiles), and back."""
+    g = G["tile_order"]
+    w = np.arange(g["rows"] * g["cols"], dtype=np.uint16).reshape(g["rows"], g["cols"])
+    got = OL.tile_order(w, g["tile_rows"], g["tile_cols"])
+    assert got.tolist() == g["tile_order"]
+    back = OL.from_tile_order(np.array(g["tile_order"], np.uint16), g["rows"], g["cols"], g["tile_rows"], g["tile_cols"])
+    assert np.array_equal(back, w)
+
+
+def test_tile_order_is_a_permutation_with_closed_form_positions():
+    """Every weight appears once, and weight (r, c) of a 256 x 192 matrix
+    lands where its tile and its place in the tile say: tiles before it
+    (all earlier tile rows, then earlier tiles of its own tile row) hold
+    8192 weights each, then r % 128 full tile rows of 64, then c % 64."""
+    rows, cols = 256, 192
+    w = np.arange(rows * cols, dtype=np.uint32).reshape(rows, cols)
+    t = OL.tile_order(w)
+    assert np.array_equal(np.sort(t), np.arange(rows * cols))
+    for r, c in [(0, 0), (0, 63), (0, 64), (1, 0), (127, 191), (128, 0), (200, 100), (255, 191)]:
+        tiles_before = (r // 128) * (cols // 64) + c // 64
+        pos = tiles_before * 8192 + (r % 128) * 64 + c % 64
+        assert t[pos] == w[r, c]
+    assert np.array_equal(OL.from_tile_order(t, rows, cols), w)
+
+
+def test_tile_order_whole_matrix_tile_is_row_major():
+    w = np.arange(128 * 64, dtype=np.uint16).reshape(128, 64)
+    assert np.array_equal(OL.tile_order(w), w.reshape(-1))
+    with pytest.raises(ValueError):
+        OL.tile_order(np.zeros((100, 64), np.uint16))
