@@ -29,7 +29,8 @@
 //    accumulator in tensor memory as soon as the tile is complete, and gives
 //    each stage back to the decoders as soon as the MMAs that read it end.
 //  * warps 0..3 (one per 32-lane quarter of tensor memory): after a unit's
-//    last MMA, read the accumulator with tcgen05.ld and write y (FP32).
+//    last MMA, read its accumulator with tcgen05.ld and write y (FP32). Two
+//    accumulators alternate, so this overlaps the next unit's MMAs.
 // The units (128-row slices of every matrix of the call) are spread over the
 // CTAs on the host, longest first onto the least loaded CTA, and passed in
 // the launch parameters. Every wait is bounded; any failure raises a shared
@@ -62,7 +63,8 @@ constexpr uint32_t kMaxM = 256;            // activation rows (MMA N)
 constexpr uint32_t kMaxUnits = 4096;       // 128-row units per call
 constexpr uint32_t kMaxCtas = 256;
 constexpr uint32_t kMaxCtaUnits = 64;      // units one CTA takes
-constexpr uint32_t kMaxStages = 8;
+constexpr uint32_t kMaxStages = 8;         // weight-tile stages
+constexpr uint32_t kXStages = 2;           // x-tile stages (refilled from L2 by the tensor copy)
 constexpr int kPreloadUnits = 8;           // 8-weight pieces per lane whose sign|mantissa loads are issued early
 constexpr uint32_t kMaxDecWarps = 16;     // decoder warps: up to 16 (more only slowed the issue-bound decode)
 constexpr uint32_t kMinDecWarps = 4;
@@ -70,48 +72,72 @@ constexpr uint32_t kMmaWarp = 4;
 constexpr uint32_t kDec0 = 5;              // first decoder warp
 constexpr uint32_t kMaxThreads = (kDec0 + kMaxDecWarps) * 32;
 constexpr uint32_t kDecBarrier = 1;        // named barrier of the decoder warps
+// y of a matrix whose K range is split starts as this pattern (a NaN that no
+// sum of finite or infinite products yields: those NaNs are canonical)
+constexpr uint32_t kSplitEmpty = 0xFFFFFFFFu;
 
 struct GemmMat {
     Df11Tensor t;          // the blob's sections (tile order); t.out unused
     float *y;              // M x rows, row-major
-    uint32_t rows, cols, k_tiles, pad;
+    uint32_t rows, cols, k_tiles, kt_split;   // kt_split: k-tiles of part 0 when the K range is split, else 0
 };
 
 struct __align__(64) GemmBatch {
     CUtensorMap xmap[kMaxMats];   // x of each matrix: M x cols BF16, box 64 x n_pad, 128-byte swizzle
     GemmMat m[kMaxMats];
-    uint32_t count, M, n_pad, stages;
+    uint32_t count, M, n_pad, stages;   // stages: weight-tile stages (x tiles have kXStages)
     uint32_t chunk_words, seg_words, stage_bytes, lut_entries;
-    uint32_t tmem_cols, idesc, dec_warps, pad0;
+    uint32_t tmem_cols, idesc, dec_warps, acc_cols;   // tensor memory: two accumulators of acc_cols columns
     uint32_t *status;
     uint16_t cta_begin[kMaxCtas + 1];   // CTA c takes sched[cta_begin[c] .. cta_begin[c + 1])
-    uint16_t sched[kMaxUnits];          // matrix << 13 | 128-row unit index
+    uint16_t sched[kMaxUnits];          // matrix << 13 | part << 12 | 128-row unit index
 };
 
 __host__ __device__ constexpr uint32_t unit_mat(uint32_t u) { return u >> 13; }
-__host__ __device__ constexpr uint32_t unit_idx(uint32_t u) { return u & 0x1FFFu; }
+__host__ __device__ constexpr uint32_t unit_part(uint32_t u) { return (u >> 12) & 1u; }
+__host__ __device__ constexpr uint32_t unit_idx(uint32_t u) { return u & 0xFFFu; }
+
+// The k-tiles a unit covers: all of them, or (split matrices) the first
+// kt_split or the rest. In tile order a unit is one contiguous weight range.
+struct UnitSpan {
+    uint32_t mat, ru, part, kt0, kts;
+    uint64_t lo;   // first weight of the unit (tile order)
+};
+__device__ __forceinline__ UnitSpan unit_span(const GemmBatch &B, uint32_t u) {
+    UnitSpan r;
+    r.mat = unit_mat(u);
+    r.ru = unit_idx(u);
+    r.part = unit_part(u);
+    const GemmMat &g = B.m[r.mat];
+    r.kt0 = r.part ? g.kt_split : 0u;
+    r.kts = g.kt_split ? (r.part ? g.k_tiles - g.kt_split : g.kt_split) : g.k_tiles;
+    r.lo = ((uint64_t)r.ru * g.k_tiles + r.kt0) * kTileElems;
+    return r;
+}
 
 // Shared memory of one CTA (offsets from a 1024-byte aligned base).
 struct GemmLayout {
-    uint32_t stage_stride, dec, ctl, total;
+    uint32_t stage_stride, x_off, x_stride, dec, ctl, total;
     // control block (bytes from ctl)
     static constexpr uint32_t kFullX = 0;            // u64[kMaxStages]: x tile landed
     static constexpr uint32_t kFullW = 64;           // u64[kMaxStages]: weight tile complete
     static constexpr uint32_t kEmpty = 128;          // u64[kMaxStages]: the MMAs that read the stage completed
-    static constexpr uint32_t kAccFull = 192;        // u64: a unit's accumulator is final
-    static constexpr uint32_t kAccEmpty = 200;       // u64: the epilogue has read it
-    static constexpr uint32_t kWritten = 208;        // u32[kMaxStages]: weights stored in the stage's tile
-    static constexpr uint32_t kReleased = 240;       // u32[kMaxStages]: fills of the stage consumed
-    static constexpr uint32_t kTmem = 272;           // u32: tensor-memory address
-    static constexpr uint32_t kAbort = 276;          // u32
-    static constexpr uint32_t kUnitFirst = 288;      // u32[kMaxCtaUnits]: a unit's first block
+    static constexpr uint32_t kAccFull = 192;        // u64[2]: a unit's accumulator (buffer ui % 2) is final
+    static constexpr uint32_t kAccEmpty = 208;       // u64[2]: the epilogue has read it
+    static constexpr uint32_t kWritten = 224;        // u32[kMaxStages]: weights stored in the stage's tile
+    static constexpr uint32_t kReleased = 256;       // u32[kMaxStages]: fills of the stage consumed
+    static constexpr uint32_t kTmem = 288;           // u32: tensor-memory address
+    static constexpr uint32_t kAbort = 292;          // u32
+    static constexpr uint32_t kUnitFirst = 304;      // u32[kMaxCtaUnits]: a unit's first block
     static constexpr uint32_t kUnitItem = kUnitFirst + 4 * kMaxCtaUnits;   // u32[kMaxCtaUnits + 1]: first item
     static constexpr uint32_t kUnitTile = kUnitItem + 4 * (kMaxCtaUnits + 1) + 12;   // u32[kMaxCtaUnits + 1]
     static constexpr uint32_t kCtlBytes = kUnitTile + 4 * (kMaxCtaUnits + 1) + 12;
     __host__ __device__ GemmLayout(uint32_t n_pad, uint32_t stages, uint32_t seg_words, uint32_t lut_entries,
                                    uint32_t stage_bytes, uint32_t dec_warps) {
-        stage_stride = kTileBytes + n_pad * 128u;   // weight tile, then x tile; multiple of 1024
-        dec = stages * stage_stride;
+        stage_stride = kTileBytes;            // weight tiles, then x tiles; all multiples of 1024
+        x_off = stages * stage_stride;
+        x_stride = n_pad * 128u;
+        dec = x_off + kXStages * x_stride;
         ctl = dec + CountedLayout(seg_words, lut_entries, stage_bytes, dec_warps).total;
         ctl = (ctl + 15u) & ~15u;
         total = ctl + kCtlBytes;
@@ -188,15 +214,17 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
 
     // ---- prologue: barriers, counters, tensor memory, this CTA's unit table
     if (tid == 0) {
+        for (uint32_t s = 0; s < kXStages; s++) dev::mbar_init(&full_x[s], 1);
         for (uint32_t s = 0; s < NS; s++) {
-            dev::mbar_init(&full_x[s], 1);
             dev::mbar_init(&full_w[s], 1);
             dev::mbar_init(&empty[s], 1);
             written[s] = 0;
             released[s] = 0;
         }
-        dev::mbar_init(acc_full, 1);
-        dev::mbar_init(acc_empty, 4);
+        for (uint32_t k = 0; k < 2; k++) {
+            dev::mbar_init(&acc_full[k], 1);
+            dev::mbar_init(&acc_empty[k], 4);
+        }
         *abort_flag = 0;
         dev::fence_mbar_init();
     }
@@ -205,10 +233,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
         umma::tmem_relinquish();
     }
     for (uint32_t i = tid; i < nunits; i += blockDim.x) {
-        const uint32_t u = B.sched[c0 + i];
-        const GemmMat &gm = B.m[unit_mat(u)];
-        const uint64_t lo = (uint64_t)unit_idx(u) * kTileRows * gm.cols;
-        const uint64_t hi = lo + (uint64_t)kTileRows * gm.cols;
+        const UnitSpan sp = unit_span(B, B.sched[c0 + i]);
+        const GemmMat &gm = B.m[sp.mat];
+        const uint64_t lo = sp.lo, hi = lo + (uint64_t)sp.kts * kTileElems;
         // the last block whose first weight is <= v (block 0 starts at weight 0)
         auto last_le = [&](uint64_t v) {
             uint32_t a = 0, b = gm.t.n_blocks;
@@ -221,7 +248,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
         const uint32_t first = last_le(lo), last = last_le(hi - 1);
         u_first[i] = first;
         u_item[i + 1] = last - first + 1;
-        u_tile[i + 1] = gm.k_tiles;
+        u_tile[i + 1] = sp.kts;
     }
     __syncthreads();
     if (tid == 0) {
@@ -236,7 +263,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tiles_a = dev::smem_u32(smem);   // stage s: weight tile at tiles_a + s * stride, x tile after it
+    const uint32_t tiles_a = dev::smem_u32(smem);   // weight tile of stage s at tiles_a + s * stride
+    const uint32_t tiles_x = tiles_a + G.x_off;      // x tile of x stage k at tiles_x + k * x_stride
 
     if (warp == kMmaWarp) {
         // ---- one thread: x tiles by tensor copy, MMAs, stage release
@@ -245,25 +273,25 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             const uint32_t xbytes = B.n_pad * 128u;
             uint32_t lq = 0, lu = 0, lk = 0;   // next tile whose x tile is loaded: its unit and k-tile
             auto load_x = [&]() {
-                const uint32_t s = lq % NS;
-                const uint32_t mat = unit_mat(B.sched[c0 + lu]);
+                const uint32_t s = lq % kXStages;
+                const UnitSpan sp = unit_span(B, B.sched[c0 + lu]);
                 dev::mbar_arrive_expect_tx(&full_x[s], xbytes);
-                umma::tma_load_2d(smem + s * G.stage_stride + kTileBytes, &B.xmap[mat], (int32_t)(lk * kTileCols), 0,
-                                  &full_x[s]);
+                umma::tma_load_2d(smem + G.x_off + s * G.x_stride, &B.xmap[sp.mat],
+                                  (int32_t)((sp.kt0 + lk) * kTileCols), 0, &full_x[s]);
                 lq++;
-                if (++lk == B.m[mat].k_tiles) {
+                if (++lk == sp.kts) {
                     lk = 0;
                     lu++;
                 }
             };
-            for (uint32_t j = 0; j < NS && lq < T; j++) load_x();
+            for (uint32_t j = 0; j < kXStages && lq < T; j++) load_x();
             // Event loop: retire the oldest issued tile as soon as its MMAs complete
-            // (its stage goes back to the decoders, its x buffer takes the tile NS
-            // ahead), and issue the next tile as soon as its weights and x are in.
+            // (its weight stage goes back to the decoders, its x stage takes the tile
+            // kXStages ahead), and issue the next tile as soon as its weights and x are in.
             // Phase parities are unambiguous: a stage's barriers never run more than
             // one fill ahead of this thread.
             uint32_t issued = 0, retired = 0, ui = 0, kt = 0, idle = 0;
-            uint32_t KT = nunits ? B.m[unit_mat(B.sched[c0])].k_tiles : 0u;
+            uint32_t KT = nunits ? unit_span(B, B.sched[c0]).kts : 0u;
             bool ok = true;
             while (retired < T) {
                 bool progress = false;
@@ -275,22 +303,24 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
                     progress = true;
                 }
                 if (issued < T && issued - retired < NS) {
-                    const uint32_t s = issued % NS, f = issued / NS;
-                    if (dev::mbar_test(&full_x[s], f & 1u) && dev::mbar_test(&full_w[s], f & 1u) &&
-                        (kt != 0 || ui == 0 || dev::mbar_test(acc_empty, (ui - 1) & 1u))) {
+                    const uint32_t s = issued % NS, f = issued / NS, sx = issued % kXStages;
+                    // unit ui accumulates in buffer ui % 2, free once the epilogue has read unit ui - 2
+                    if (dev::mbar_test(&full_x[sx], (issued / kXStages) & 1u) && dev::mbar_test(&full_w[s], f & 1u) &&
+                        (kt != 0 || ui < 2 || dev::mbar_test(&acc_empty[ui & 1u], ((ui >> 1) - 1) & 1u))) {
                         umma::fence_after_sync();
-                        const uint32_t a = tiles_a + s * G.stage_stride, b = a + kTileBytes;
+                        const uint32_t a = tiles_a + s * G.stage_stride, b = tiles_x + sx * G.x_stride;
+                        const uint32_t d = tmem + (ui & 1u) * B.acc_cols;
 #pragma unroll
                         for (uint32_t k = 0; k < kTileCols / 16; k++)
-                            umma::mma_bf16(tmem, umma::smem_desc_sw128(a + 32u * k), umma::smem_desc_sw128(b + 32u * k),
+                            umma::mma_bf16(d, umma::smem_desc_sw128(a + 32u * k), umma::smem_desc_sw128(b + 32u * k),
                                            B.idesc, (kt | k) != 0);
                         umma::mma_commit(&empty[s]);
-                        if (kt + 1 == KT) umma::mma_commit(acc_full);   // the unit's accumulator, once complete
+                        if (kt + 1 == KT) umma::mma_commit(&acc_full[ui & 1u]);   // the unit's accumulator, once complete
                         issued++;
                         if (++kt == KT) {
                             kt = 0;
                             ui++;
-                            KT = ui < nunits ? B.m[unit_mat(B.sched[c0 + ui])].k_tiles : 0u;
+                            KT = ui < nunits ? unit_span(B, B.sched[c0 + ui]).kts : 0u;
                         }
                         progress = true;
                     }
@@ -311,13 +341,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             }
             // before the CTA ends: every issued MMA completes, every x tile in flight lands
             while (retired < issued && dev::mbar_wait_bounded(&empty[retired % NS], (retired / NS) & 1u)) retired++;
-            for (uint32_t r = issued; r < lq; r++) dev::mbar_wait_bounded(&full_x[r % NS], (r / NS) & 1u);
+            for (uint32_t r = issued; r < lq; r++) dev::mbar_wait_bounded(&full_x[r % kXStages], (r / kXStages) & 1u);
         }
         __syncwarp();
     } else if (warp < kMmaWarp) {
         // ---- epilogue: warp w reads accumulator lanes 32 w .. 32 w + 31 (weight rows)
         for (uint32_t ui = 0; ui < nunits; ui++) {
-            if (!wait_phase(acc_full, ui & 1u, abort_flag)) {
+            if (!wait_phase(&acc_full[ui & 1u], (ui >> 1) & 1u, abort_flag)) {
                 if (!*abort_flag) bad |= LWC_DEVICE_TIMEOUT;
                 *abort_flag = 1;
                 break;
@@ -326,17 +356,29 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             const uint32_t u = B.sched[c0 + ui];
             const GemmMat &gm = B.m[unit_mat(u)];
             float *y = gm.y + (unit_idx(u) * kTileRows + warp * 32u + lane);
-            const uint32_t taddr = tmem + ((warp * 32u) << 16);
+            const uint32_t taddr = tmem + ((warp * 32u) << 16) + (ui & 1u) * B.acc_cols;
+            const bool split = gm.kt_split != 0;
             for (uint32_t c = 0; c < B.n_pad; c += 16) {
                 uint32_t v[16];
                 umma::tmem_ld16(taddr + c, v);
 #pragma unroll
-                for (uint32_t j = 0; j < 16; j++)
-                    if (c + j < B.M) y[(size_t)(c + j) * gm.rows] = __uint_as_float(v[j]);
+                for (uint32_t j = 0; j < 16; j++) {
+                    if (c + j >= B.M) continue;
+                    float *py = y + (size_t)(c + j) * gm.rows;
+                    if (!split) {
+                        *py = __uint_as_float(v[j]);
+                    } else {
+                        // the K range is split in two parts: y starts as kSplitEmpty; the part
+                        // that finds the other's product there stores the sum (IEEE addition
+                        // commutes, so the result does not depend on which part came second)
+                        const uint32_t other = atomicExch(reinterpret_cast<unsigned int *>(py), v[j]);
+                        if (other != kSplitEmpty) *py = __uint_as_float(v[j]) + __uint_as_float(other);
+                    }
+                }
             }
             umma::fence_before_sync();
             __syncwarp();
-            if (lane == 0) dev::mbar_arrive(acc_empty);
+            if (lane == 0) dev::mbar_arrive(&acc_empty[ui & 1u]);
         }
     } else {
         // ---- decoder warps: blocks of this CTA's units, in order, into the stages
@@ -415,9 +457,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
                     o0n = tn.blkoff[bn];
                     o1n = tn.blkoff[bn + 1];
                 }
-                const uint32_t uu = B.sched[c0 + cu];
-                const uint64_t ulo = (uint64_t)unit_idx(uu) * kTileRows * gm.cols;
-                const uint64_t uhi = ulo + (uint64_t)kTileRows * gm.cols;
+                const UnitSpan usp = unit_span(B, B.sched[c0 + cu]);
+                const uint64_t ulo = usp.lo, uhi = ulo + (uint64_t)usp.kts * kTileElems;
                 const bool ok = o0 <= o1 && o1 <= tn.n && o1 - o0 + 16 <= B.stage_bytes && o0 < uhi && o1 > ulo;
                 const uint64_t p_lo = ok ? max(o0, ulo) : 0, p_hi = ok ? min(o1, uhi) : 0;
                 // this unit's part of the block: 8-weight pieces [g_lo, g_hi), single weights at either end
@@ -741,8 +782,8 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
         if (cols[i] == 0 || cols[i] % kTileCols || cols[i] > (1u << 24) || d.n % cols[i])
             return fail(LWC_ERR_INVALID_ARG, "matrix %d: cols must divide n and be a multiple of 64 up to 2^24", i);
         const uint64_t rows = d.n / cols[i];
-        if (rows % kTileRows || rows / kTileRows > 8192)
-            return fail(LWC_ERR_INVALID_ARG, "matrix %d: rows must be a multiple of 128 (at most 2^20)", i);
+        if (rows % kTileRows || rows / kTileRows > 4096)
+            return fail(LWC_ERR_INVALID_ARG, "matrix %d: rows must be a multiple of 128 (at most 2^19)", i);
         if (chunk_bytes && d.chunk_bytes != chunk_bytes)
             return fail(LWC_ERR_UNSUPPORTED, "matrices of one call must share chunk_bytes");
         chunk_bytes = d.chunk_bytes;
@@ -766,10 +807,7 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
         g.rows = (uint32_t)rows;
         g.cols = (uint32_t)cols[i];
         g.k_tiles = g.cols / kTileCols;
-        for (uint32_t r = 0; r < rows / kTileRows; r++) {
-            units.push_back(n << 13 | r);
-            cost.push_back(g.k_tiles + 2);
-        }
+        g.kt_split = 0;
         max_count = std::max<uint64_t>(max_count, d.max_block_count);
         max_tables = std::max<uint64_t>(max_tables, d.n_tables);
         mats.push_back(i);
@@ -779,11 +817,37 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
         clear_error();
         return LWC_OK;
     }
-    if (units.size() > kMaxUnits) return fail(LWC_ERR_UNSUPPORTED, "more than %u 128-row units in one call", kMaxUnits);
     GemmDevice dev;
     EncodeTiledFn encode = nullptr;
     lwc_status st = gemm_device(dev, encode);
     if (st) return st;
+    // Work units: 128 rows of a matrix, all k-tiles; a matrix whose unit would
+    // take much longer than a CTA's average share has its K range split in
+    // two parts (the CTA that finishes a part second adds the two).
+    {
+        uint64_t total_cost = 0, n_units = 0;
+        for (uint32_t j = 0; j < n; j++) {
+            total_cost += (uint64_t)(B.m[j].rows / kTileRows) * (B.m[j].k_tiles + 2);
+            n_units += B.m[j].rows / kTileRows;
+        }
+        const uint64_t ctas0 = std::min<uint64_t>(n_units, (uint64_t)std::min(dev.sms, (int)kMaxCtas));
+        for (uint32_t j = 0; j < n; j++) {
+            GemmMat &g = B.m[j];
+            if (g.k_tiles >= 2 && 4 * (uint64_t)(g.k_tiles + 2) * ctas0 > 3 * total_cost) g.kt_split = g.k_tiles / 2;
+            for (uint32_t r = 0; r < g.rows / kTileRows; r++) {
+                if (!g.kt_split) {
+                    units.push_back(j << 13 | r);
+                    cost.push_back(g.k_tiles + 2);
+                } else {
+                    units.push_back(j << 13 | r);
+                    cost.push_back(g.kt_split + 2);
+                    units.push_back(j << 13 | 1u << 12 | r);
+                    cost.push_back(g.k_tiles - g.kt_split + 2);
+                }
+            }
+        }
+    }
+    if (units.size() > kMaxUnits) return fail(LWC_ERR_UNSUPPORTED, "more than %u 128-row units in one call", kMaxUnits);
     B.count = n;
     B.M = (uint32_t)M;
     B.n_pad = (uint32_t)round_up((uint64_t)M, 16);
@@ -791,7 +855,8 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     B.seg_words = (uint32_t)round_up(32ull * B.chunk_words + 2, 4);
     B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
-    B.tmem_cols = B.n_pad <= 32 ? 32 : B.n_pad <= 64 ? 64 : B.n_pad <= 128 ? 128 : 256;
+    B.acc_cols = B.n_pad <= 32 ? 32 : B.n_pad <= 64 ? 64 : B.n_pad <= 128 ? 128 : 256;
+    B.tmem_cols = 2 * B.acc_cols;   // two accumulators: a unit's epilogue overlaps the next unit's MMAs
     B.idesc = umma::instr_desc_bf16_f32(kTileRows, B.n_pad);
     B.status = d_status;
     // shared memory: the most decoder warps with at least three stages (then as many
@@ -828,6 +893,12 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     const uint32_t ctas = (uint32_t)std::min<uint64_t>(units.size(), (uint64_t)std::min(dev.sms, (int)kMaxCtas));
     if (!schedule_units(units, cost, ctas, B))
         return fail(LWC_ERR_UNSUPPORTED, "too many units per CTA (%zu units on %u CTAs)", units.size(), ctas);
+    for (uint32_t j = 0; j < n; j++)
+        if (B.m[j].kt_split) {
+            const cudaError_t e = cudaMemsetAsync(B.m[j].y, 0xFF, (size_t)M * B.m[j].rows * sizeof(float),
+                                                  reinterpret_cast<cudaStream_t>(stream));
+            if (e != cudaSuccess) return fail(LWC_ERR_CUDA, "output fill: %s", cudaGetErrorString(e));
+        }
     df11_gemm_kernel<<<ctas, (kDec0 + B.dec_warps) * 32u, (size_t)smem, reinterpret_cast<cudaStream_t>(stream)>>>(B);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "tensor-core product launch: %s", cudaGetErrorString(err));

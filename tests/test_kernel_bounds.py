@@ -384,12 +384,15 @@ def _last_le(blkoff, n_blocks, v):
 
 
 def _gemm_placement(blkoff, n_blocks, tiled, rows, cols, cta_units):
+    """cta_units: (128-row unit, first k-tile, k-tiles) in the CTA's order; a
+    unit whose K range is split in two parts appears once per part."""
     kt = cols // 64
     slots = {}      # tile sequence number -> {byte offset: weight}
     counts = {}
     t0 = 0
-    for u in cta_units:
-        lo, hi = u * 128 * cols, (u + 1) * 128 * cols
+    for u, kt0, kts in cta_units:
+        lo = (u * kt + kt0) * 8192
+        hi = lo + kts * 8192
         first, last = _last_le(blkoff, n_blocks, lo), _last_le(blkoff, n_blocks, hi - 1)
         for b in range(first, last + 1):
             o0, o1 = int(blkoff[b]), int(blkoff[b + 1])
@@ -421,12 +424,13 @@ def _gemm_placement(blkoff, n_blocks, tiled, rows, cols, cta_units):
             for q in range(qa, qz + 1):
                 tlo = lo + (q - t0) * 8192
                 counts[q] = counts.get(q, 0) + min(p_hi, tlo + 8192) - max(p_lo, tlo)
-        t0 += kt
+        t0 += kts
     return slots, counts
 
 
 @pytest.mark.parametrize("rows,cols,chunk,order", [(384, 320, 36, "plain"), (256, 64, 8, "plain"),
-                                                   (512, 192, 36, "shuffled"), (128, 1024, 12, "plain")])
+                                                   (512, 192, 36, "shuffled"), (128, 1024, 12, "plain"),
+                                                   (384, 320, 20, "split"), (256, 1024, 36, "split")])
 def test_gemm_tile_placement_model(rows, cols, chunk, order):
     import synth
     from decode_dfloat11_b200 import lwc
@@ -439,17 +443,22 @@ def test_gemm_tile_placement_model(rows, cols, chunk, order):
     assert d.flags & 2
     h = B.unpack_header(b)
     blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
-    units = list(range(rows // 128))
+    kt = cols // 64
+    units = [(u, 0, kt) for u in range(rows // 128)]
     if order == "shuffled":
         units = units[::-1]
+    if order == "split":   # each unit's K range in two parts (k-tiles kt // 2 and the rest), second parts first
+        half = kt // 2
+        units = [(u, half, kt - half) for u in range(rows // 128)] + [(u, 0, half) for u in range(rows // 128)]
     slots, counts = _gemm_placement(blkoff, h["n_blocks"], tiled, rows, cols, units)
-    kt = cols // 64
-    assert sorted(counts) == list(range(len(units) * kt))
+    n_tiles = sum(kts for _, _, kts in units)
+    assert sorted(counts) == list(range(n_tiles))
     assert all(c == 8192 for c in counts.values())
-    for k, u in enumerate(units):
-        for j in range(kt):
-            q = k * kt + j
+    q = 0
+    for u, kt0, kts in units:
+        for j in range(kt0, kt0 + kts):
             assert len(slots[q]) == 8192
             for r in (0, 1, 7, 8, 63, 127):
                 for c in (0, 5, 8, 31, 63):
                     assert slots[q][_sw128(r, c)] == w[u * 128 + r, j * 64 + c]
+            q += 1
