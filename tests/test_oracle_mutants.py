@@ -240,3 +240,25 @@ def test_chunk_offsets_off_by_one_is_caught(monkeypatch):
     monkeypatch.setattr(df11, "chunk_output_offsets", bad)
     fails(pins.test_chunk_output_offsets_match_independent_chunk_decodes, 8, 32)
     fails(pins.test_chunk_output_offsets_single_code_length)
+
+
+def _tile_order_by(order):
+    """A tile order with the tiles or their contents walked the wrong way."""
+    def f(w_bits, tile_rows=128, tile_cols=64):
+        w = np.asarray(w_bits)
+        rows, cols = w.shape
+        pieces = []
+        grid = [(i, j) for i in range(rows // tile_rows) for j in range(cols // tile_cols)]
+        if order == "tiles_by_column":
+            grid = [(i, j) for j in range(cols // tile_cols) for i in range(rows // tile_rows)]
+        for i, j in grid:
+            tile = w[i * tile_rows:(i + 1) * tile_rows, j * tile_cols:(j + 1) * tile_cols]
+            pieces.append(tile.T.reshape(-1) if order == "tile_column_major" else tile.reshape(-1))
+        return np.concatenate(pieces)
+    return f
+
+
+@pytest.mark.parametrize("order", ["tiles_by_column", "tile_column_major"])
+def test_tile_order_walked_the_wrong_way_is_caught(monkeypatch, order):
+    monkeypatch.setattr(OL, "tile_order", _tile_order_by(order))
+    fails(lpins.test_golden_tile_order)
