@@ -246,8 +246,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             return a;
         };
         const uint32_t first = last_le(lo), last = last_le(hi - 1);
-        u_first[i] = first;
-        u_item[i + 1] = last - first + 1;
+        // block offsets that are not ascending (a damaged blob) can give last < first:
+        // the unit gets no items and is reported below
+        u_first[i] = last >= first ? first : 0xFFFFFFFFu;
+        u_item[i + 1] = last >= first ? last - first + 1 : 0u;
         u_tile[i + 1] = sp.kts;
     }
     __syncthreads();
@@ -255,6 +257,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
         u_item[0] = 0;
         u_tile[0] = 0;
         for (uint32_t i = 0; i < nunits; i++) {
+            if (u_first[i] == 0xFFFFFFFFu) {
+                bad |= LWC_DEVICE_BAD_OFFSET;
+                *abort_flag = 1;
+                u_first[i] = 0;
+            }
             u_item[i + 1] += u_item[i];
             u_tile[i + 1] += u_tile[i];
         }
@@ -590,10 +597,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
                                     const uint64_t tlo = ulo + (uint64_t)(q - t0) * kTileElems;
                                     const uint32_t n_in = (uint32_t)(min(p_hi, tlo + kTileElems) - max(p_lo, tlo));
                                     const uint32_t s = q % NS;
-                                    if (atomicAdd(&written[s], n_in) + n_in == kTileElems) {   // the tile is complete
+                                    const uint32_t now = atomicAdd(&written[s], n_in) + n_in;
+                                    if (now == kTileElems) {   // the tile is complete
                                         written[s] = 0;
                                         __threadfence_block();
                                         dev::mbar_arrive(&full_w[s]);
+                                    } else if (now > kTileElems) {   // blocks overlap: a damaged blob
+                                        bad |= LWC_DEVICE_BAD_OFFSET;
+                                        *abort_flag = 1;
                                     }
                                 }
                             }

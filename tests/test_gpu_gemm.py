@@ -203,3 +203,55 @@ def test_tile_order_argument_errors():
     with pytest.raises(lwc.LwcError) as e:
         lwc.lwc_tile_order(src, 256, 128, src)
     assert e.value.status == lwc.LWC_ERR_INVALID_ARG
+
+
+def test_damaged_blobs_are_reported_and_contained():
+    """Damaged tile-order blobs (count bytes, block offsets out of range or
+    out of order, every lookup entry invalid, stream bit flips) end the
+    product with a device status, within the bounded waits, with nothing
+    written outside y; the next call on a sound blob is exact."""
+    import time
+    rows, cols, M = 384, 1024, 16
+    w = weights(rows, cols, seed=21)
+    d, b = lwc.lwc_encode_dfloat11(OL.tile_order(w), chunk_bytes=GEMM_CHUNK_BYTES)
+    assert d.n_blocks > 8
+    rng = np.random.default_rng(3)
+    cases = {}
+    x = b.copy()
+    x[d.off_counts + 32 * 5 + 7] += np.uint8(1)                 # one chunk's code count
+    cases["count"] = (x, lwc.LWC_DEVICE_BAD_COUNT)
+    x = b.copy()
+    x[d.off_blkoff + 8 * 4: d.off_blkoff + 8 * 5] = np.array([2 ** 40], np.uint64).view(np.uint8)
+    cases["offset_out_of_range"] = (x, lwc.LWC_DEVICE_BAD_OFFSET | lwc.LWC_DEVICE_BAD_COUNT)
+    x = b.copy()
+    off = np.frombuffer(x[d.off_blkoff: d.off_blkoff + 8 * (d.n_blocks + 1)].tobytes(), np.uint64).copy()
+    off[[2, 6]] = off[[6, 2]]                                   # offsets out of order
+    x[d.off_blkoff: d.off_blkoff + 8 * (d.n_blocks + 1)] = off.view(np.uint8)
+    cases["offsets_out_of_order"] = (x, lwc.LWC_DEVICE_BAD_OFFSET | lwc.LWC_DEVICE_BAD_COUNT)
+    x = b.copy()
+    x[d.off_lut: d.off_lut + 512 * d.n_tables] = 0xFF             # every lookup entry invalid
+    cases["lut"] = (x, lwc.LWC_DEVICE_BAD_CODE | lwc.LWC_DEVICE_BAD_COUNT)
+    x = b.copy()
+    x[d.off_stream + rng.integers(0, (d.total_bits + 7) // 8, 50)] ^= np.uint8(0x10)
+    cases["bit_flips"] = (x, None)
+    guard = 4096
+    xa = synth.activations_bf16(M, cols, seed=22, device="cuda")
+    for name, (blob, expect) in cases.items():
+        ybuf = torch.zeros(M * rows + 2 * guard, dtype=torch.float32, device="cuda")
+        y = ybuf[guard:guard + M * rows].view(M, rows)
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        t0 = time.perf_counter()
+        lwc.lwc_gemm_dfloat11(d, torch.from_numpy(blob).to("cuda"), cols, xa, M, y, status)
+        torch.cuda.synchronize()
+        assert time.perf_counter() - t0 < 30, name
+        got = ybuf.cpu().numpy()
+        assert np.all(got[:guard] == 0) and np.all(got[guard + M * rows:] == 0), name
+        st = int(status.item())
+        if expect is not None:
+            assert st & expect, (name, st)
+    # the context still computes exactly
+    x1 = torch.zeros((64, cols), dtype=torch.bfloat16, device="cuda")
+    x1[torch.arange(64), torch.arange(64)] = 1.0
+    d0, b0 = tiled_blob(w)
+    y = run_gemm(d0, b0, cols, x1, 64)
+    assert np.array_equal(y, OL.bf16_values(w)[:, :64].T)
