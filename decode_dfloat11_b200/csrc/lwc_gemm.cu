@@ -16,8 +16,8 @@
 // one work unit (128 rows of W, all columns) is a contiguous range of the
 // decoded stream, whose k-tiles arrive in order.
 //
-// Roles (one CTA per SM, persistent; 5 + 4..24 warps, the host's choice by
-// shared memory):
+// Roles (one CTA per SM, persistent; 5 + 4..20 warps, the host's choice by
+// block size and shared memory):
 //  * warps 5.. decode: they claim the unit's 32-chunk blocks in order (the
 //    counted decoder: stored chunk counts, multi-code symbol tables), merge
 //    each weight with its sign|mantissa byte and store it into the stage of
@@ -66,7 +66,8 @@ constexpr uint32_t kMaxCtaUnits = 64;      // units one CTA takes
 constexpr uint32_t kMaxStages = 8;         // weight-tile stages
 constexpr uint32_t kXStages = 2;           // x-tile stages (refilled from L2 by the tensor copy)
 constexpr int kPreloadUnits = 8;           // 8-weight pieces per lane whose sign|mantissa loads are issued early
-constexpr uint32_t kMaxDecWarps = 16;     // decoder warps: up to 16 (more only slowed the issue-bound decode)
+constexpr uint32_t kMaxDecWarps = 20;     // decoder warps (24 spill registers and were slower)
+constexpr uint32_t kInFlightWeights = 48 * 1024;   // blocks in flight: about six 8192-weight tiles
 constexpr uint32_t kMinDecWarps = 4;
 constexpr uint32_t kMmaWarp = 4;
 constexpr uint32_t kDec0 = 5;              // first decoder warp
@@ -870,8 +871,12 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     B.tmem_cols = 2 * B.acc_cols;   // two accumulators: a unit's epilogue overlaps the next unit's MMAs
     B.idesc = umma::instr_desc_bf16_f32(kTileRows, B.n_pad);
     B.status = d_status;
-    // shared memory: the most decoder warps with at least three stages (then as many
-    // stages as fit, up to kMaxStages); failing that, the most warps with two
+    // decoder warps: at most as many as keep about kInFlightWeights weights in flight
+    // (blocks of 36-byte chunks, ~3,600 weights: 12 warps; of 20-byte chunks: 20);
+    // then, by shared memory, the most of them with at least three weight stages
+    // (and as many stages as fit, up to kMaxStages); failing that, with two
+    uint32_t warp_cap = (uint32_t)std::min<uint64_t>(kMaxDecWarps, kInFlightWeights / std::max<uint64_t>(max_count, 1));
+    warp_cap = std::max(kMinDecWarps, warp_cap & ~1u);
     uint64_t smem = 0;
     auto fits = [&](uint32_t warps, uint32_t stages) {
         smem = GemmLayout(B.n_pad, stages, B.seg_words, B.lut_entries, B.stage_bytes, warps).total + 1024;
@@ -879,7 +884,7 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     };
     B.stages = 0;
     for (uint32_t min_stages : {3u, 2u}) {
-        for (uint32_t w = kMaxDecWarps; w >= kMinDecWarps && !B.stages; w -= 4)
+        for (uint32_t w = warp_cap; w >= kMinDecWarps && !B.stages; w -= 2)
             if (fits(w, min_stages)) {
                 B.dec_warps = w;
                 B.stages = min_stages;

@@ -122,11 +122,11 @@ def fused_linear(desc, blob, shape, x, codec: str, out=None, stream=None, status
 
 
 # Chunk size of the blobs TiledWeights makes. A 32-chunk block of 20-byte
-# chunks holds about 2,000 exponent codes, so the product's 16 decoder warps
-# keep about four 8192-weight tiles in flight (36-byte chunks: about seven,
-# more than the shared-memory stages hold at M > 16); the price is 0.13 bits
-# per weight of chunk gaps and counts. Measured on a Llama-3-8B layer (B200):
-# 20 bytes was the fastest of 16, 20, 24 and 36 for M = 16..256.
+# chunks holds about 2,000 exponent codes, so the product can run 20 decoder
+# warps with about five 8192-weight tiles in flight (36-byte chunks: 12 warps);
+# the price is 0.13 bits per weight of chunk gaps and counts. Measured on a
+# Llama-3-8B layer (B200), M = 16 / 128 / 256: 20-byte chunks 0.31 / 0.34 /
+# 0.42 ms; 24: 0.31 / 0.34 / 0.50; 28: 0.29 / 0.38 / 0.59; 36: 0.32 / 0.41 / 0.67.
 GEMM_CHUNK_BYTES = 20
 
 
