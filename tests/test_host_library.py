@@ -402,3 +402,35 @@ def test_resident_model_needs_two_buffers():
     with pytest.raises(ValueError):
         ResidentModel("dfloat11", "cpu", slots=0)
     assert ResidentModel("codebook", "cpu", slots=2).slots == 2
+
+
+def test_tensor_core_product_rejects_bad_arguments_before_any_device_work():
+    """lwc_gemm_dfloat11 checks its arguments on the host before it touches
+    the device: these calls fail the same way with or without a GPU (the
+    device pointers are never dereferenced)."""
+    from oracle import linear as OL
+    w = synth.as_u16(synth.normal_bf16((256, 128), seed=1, sigma=0.02)).reshape(256, 128)
+    d, _ = lwc.lwc_encode_dfloat11(OL.tile_order(w), chunk_bytes=20)
+    fake = ctypes.c_void_p(1 << 40)          # 16-byte aligned, never read
+    def call(desc, cols, M, blob=fake, x=fake, y=fake):
+        L = lwc.load()
+        return L.lwc_gemm_dfloat11(ctypes.byref(desc), blob, cols, x, M, y, None, None)
+    assert call(d, 128, 0) == lwc.LWC_ERR_INVALID_ARG
+    assert call(d, 128, 257) == lwc.LWC_ERR_INVALID_ARG
+    assert call(d, 96, 4) == lwc.LWC_ERR_INVALID_ARG           # cols not a multiple of 64
+    assert call(d, 256 * 128, 4) == lwc.LWC_ERR_INVALID_ARG    # rows = 1, not a multiple of 128
+    assert call(d, 128, 4, blob=None) == lwc.LWC_ERR_INVALID_ARG
+    assert call(d, 128, 4, x=ctypes.c_void_p((1 << 40) + 2)) == lwc.LWC_ERR_MISALIGNED
+    for kw in ({"chunk_counts": False}, {"threads_per_block": 64}):
+        d2, _ = lwc.lwc_encode_dfloat11(OL.tile_order(w), **kw)
+        assert call(d2, 128, 4) == lwc.LWC_ERR_UNSUPPORTED
+    d3, _ = lwc.lwc_encode_dfloat11(np.full(256 * 128, 0x3F80, np.uint16))   # one exponent value
+    assert call(d3, 128, 4) == lwc.LWC_ERR_UNSUPPORTED
+    dc, _ = lwc.lwc_encode_codebook(OL.tile_order(w))
+    assert call(dc, 128, 4) != lwc.LWC_OK                      # not a DFloat11 blob
+    # the tile order itself
+    L = lwc.load()
+    assert L.lwc_tile_order(fake, 100, 128, ctypes.c_void_p((1 << 40) + 4096), None) == lwc.LWC_ERR_INVALID_ARG
+    assert L.lwc_tile_order(fake, 256, 96, ctypes.c_void_p((1 << 40) + 4096), None) == lwc.LWC_ERR_INVALID_ARG
+    assert L.lwc_tile_order(fake, 256, 128, fake, None) == lwc.LWC_ERR_INVALID_ARG
+    assert L.lwc_tile_order(fake, 0, 128, ctypes.c_void_p((1 << 40) + 4096), None) == lwc.LWC_OK
