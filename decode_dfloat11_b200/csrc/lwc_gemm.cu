@@ -66,7 +66,7 @@ constexpr uint32_t kMaxCtaUnits = 64;      // units one CTA takes
 constexpr uint32_t kMaxStages = 8;         // weight-tile stages
 constexpr uint32_t kXStages = 2;           // x-tile stages (refilled from L2 by the tensor copy)
 constexpr int kPreloadUnits = 8;           // 8-weight pieces per lane whose sign|mantissa loads are issued early
-constexpr uint32_t kMaxDecWarps = 20;     // decoder warps (24 spill registers and were slower)
+constexpr uint32_t kMaxDecWarps = 20;     // decoder warps: 25 warps leave 80 registers a thread (24 + 5 leave 64: spills)
 constexpr uint32_t kInFlightWeights = 48 * 1024;   // blocks in flight: about six 8192-weight tiles
 constexpr uint32_t kMinDecWarps = 4;
 constexpr uint32_t kMmaWarp = 4;
@@ -120,7 +120,7 @@ __device__ __forceinline__ UnitSpan unit_span(const GemmBatch &B, uint32_t u) {
 struct GemmLayout {
     uint32_t stage_stride, x_off, x_stride, dec, ctl, total;
     // control block (bytes from ctl)
-    static constexpr uint32_t kFullX = 0;            // u64[kMaxStages]: x tile landed
+    static constexpr uint32_t kFullX = 0;            // u64[kXStages]: x tile landed
     static constexpr uint32_t kFullW = 64;           // u64[kMaxStages]: weight tile complete
     static constexpr uint32_t kEmpty = 128;          // u64[kMaxStages]: the MMAs that read the stage completed
     static constexpr uint32_t kAccFull = 192;        // u64[2]: a unit's accumulator (buffer ui % 2) is final
