@@ -619,6 +619,51 @@ def run_lwc(args, rank, world, local_rank, dist):
                 "roofline": mixed_roofline(tbytes + io, 2.0 * M * n_total, gms, peak, tc_peak)}
             del xs, ys, tb
         del tw, enc_d, dbatch
+
+        # the same for the codebook codec (the layer's matrices grouped by index width)
+        twc = TiledWeights(device, codec="codebook")
+        cidx = [twc.add(t) for t in src]
+        cbytes = twc.compressed_bytes
+        enc_c = [encode_on_device(t, "codebook") for t in src]
+        cbatch = lwc.Batch([d for d, _ in enc_c], [b for _, b in enc_c], views)
+        groups = {}
+        for i in cidx:
+            groups.setdefault(twc.descs[i].k, []).append(i)
+        lin["kernels"]["codebook_tensor_core"] = "cb_gemm_kernel<k> (tcgen05.mma, TMEM accumulator, x by TMA)"
+        for M in (16, 64, 128, 256):
+            xs = [synth.activations_bf16(M, t.shape[1], seed=900 + j, device=device) for j, t in enumerate(src)]
+            ys = [torch.empty((M, t.shape[0]), dtype=torch.float32, device=device) for t in src]
+            cbs = [lwc.LinearBatch([twc.descs[i] for i in g], [twc.blobs[i] for i in g],
+                                   [src[i].shape[1] for i in g], [xs[i] for i in g], [ys[i] for i in g], M)
+                   for g in groups.values()]
+
+            def cgemm():
+                for b in cbs:
+                    lwc.lwc_gemm_codebook_batched(b, stream=stream)
+            cgemm()
+            torch.cuda.synchronize(device)
+            for t, x, y in zip(src, xs, ys):
+                ref = x.float() @ t.float().T
+                if not torch.allclose(y, ref, rtol=1e-3, atol=1e-3 * float(ref.abs().max())):
+                    raise SystemExit("codebook tensor-core product disagrees with torch")
+            for _ in range(args.warmup):
+                cgemm()
+            gms = time_steps(cgemm, args.steps, stream) / args.steps
+
+            def unfused_cb():
+                lwc.lwc_decode_codebook_batched(cbatch, stream=stream)
+                for x, v, t in zip(xs, views, src):
+                    torch.mm(x, v.view(t.shape).T, out_dtype=torch.float32)
+            for _ in range(args.warmup):
+                unfused_cb()
+            ums = time_steps(unfused_cb, args.steps, stream) / args.steps
+            io = sum(2 * x.numel() + 4 * y.numel() for x, y in zip(xs, ys))
+            lin[f"codebook_tc_M{M}"] = {
+                "tc_ms": round(gms, 5), "decode_then_matmul_ms": round(ums, 5),
+                "speedup_vs_decode_then_matmul": round(ums / gms, 3), "launches": len(cbs),
+                "roofline": mixed_roofline(cbytes + io, 2.0 * M * n_total, gms, peak, tc_peak)}
+            del xs, ys, cbs
+        del twc, enc_c, cbatch
         result["linear"] = lin
         del src
 

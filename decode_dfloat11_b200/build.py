@@ -20,7 +20,7 @@ LIB = os.path.join(PKG, "liblwc.so")
 
 CUDA_SOURCES = ["lwc_df11.cu", "lwc_codebook.cu", "lwc_encode.cu", "lwc_gemm.cu"]
 CXX_SOURCES = ["lwc_host.cpp"]
-HEADERS = ["lwc_internal.h", "lwc_device.cuh", "lwc_df11_dev.cuh", "lwc_umma.cuh"]
+HEADERS = ["lwc_internal.h", "lwc_device.cuh", "lwc_df11_dev.cuh", "lwc_umma.cuh", "lwc_cb_dev.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

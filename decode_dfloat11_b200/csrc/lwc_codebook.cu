@@ -27,11 +27,14 @@
 #include <mutex>
 #include <vector>
 
+#include "lwc_cb_dev.cuh"
 #include "lwc_device.cuh"
 #include "lwc_internal.h"
 
 namespace lwc {
 namespace {
+
+using namespace cbdev;
 
 // Warps per CTA by index width: the 32 and 64 KB tables of k = 14 and 15
 // leave room for only two CTAs per SM, so those CTAs carry more warps sharing
@@ -67,57 +70,6 @@ struct CbBatch {
     uint32_t pad;
     uint64_t total_tiles;
     uint32_t *status;
-};
-
-// Load a lane's K words from shared memory, as wide as their alignment allows.
-template <int K>
-__device__ __forceinline__ void load_words(const uint32_t *src, uint32_t (&w)[K + 1]) {
-    if constexpr (K % 4 == 0) {
-#pragma unroll
-        for (int i = 0; i < K / 4; i++) {
-            const uint4 v = reinterpret_cast<const uint4 *>(src)[i];
-            w[4 * i] = v.x;
-            w[4 * i + 1] = v.y;
-            w[4 * i + 2] = v.z;
-            w[4 * i + 3] = v.w;
-        }
-    } else if constexpr (K % 2 == 0) {
-#pragma unroll
-        for (int i = 0; i < K / 2; i++) {
-            const uint2 v = reinterpret_cast<const uint2 *>(src)[i];
-            w[2 * i] = v.x;
-            w[2 * i + 1] = v.y;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < K; i++) w[i] = src[i];
-    }
-    w[K] = 0;
-}
-
-// Field j of width K starting at bit j*K of the word array (compile-time offsets).
-template <int K, int J>
-__device__ __forceinline__ uint32_t field(const uint32_t (&w)[K + 1]) {
-    constexpr int bit = J * K, word = bit >> 5, sh = bit & 31;
-    constexpr uint32_t mask = (1u << K) - 1u;
-    if constexpr (sh + K <= 32)
-        return (w[word] >> sh) & mask;
-    else
-        return __funnelshift_r(w[word], w[word + 1], sh) & mask;
-}
-
-template <int K, int J>
-struct Gather {
-    __device__ __forceinline__ static void run(const uint32_t (&w)[K + 1], const uint16_t *tab, uint32_t (&o)[16]) {
-        const uint32_t a = tab[field<K, J>(w)];
-        const uint32_t b = tab[field<K, J + 1>(w)];
-        o[J / 2] = a | (b << 16);
-        Gather<K, J + 2>::run(w, tab, o);
-    }
-};
-template <int K>
-struct Gather<K, 32> {
-    __device__ __forceinline__ static void run(const uint32_t (&)[K + 1], const uint16_t *, uint32_t (&)[16]) {}
 };
 
 template <int K>

@@ -44,6 +44,7 @@
 #include <numeric>
 #include <vector>
 
+#include "lwc_cb_dev.cuh"
 #include "lwc_device.cuh"
 #include "lwc_df11_dev.cuh"
 #include "lwc_internal.h"
@@ -53,6 +54,7 @@ namespace lwc {
 namespace {
 
 using namespace df11dev;
+using namespace cbdev;
 
 constexpr uint32_t kTileRows = 128;
 constexpr uint32_t kTileCols = 64;
@@ -69,6 +71,7 @@ constexpr int kPreloadUnits = 8;           // 8-weight pieces per lane whose sig
 constexpr uint32_t kMaxDecWarps = 20;     // decoder warps: 25 warps leave 80 registers a thread (24 + 5 leave 64: spills)
 constexpr uint32_t kInFlightWeights = 48 * 1024;   // blocks in flight: about six 8192-weight tiles
 constexpr uint32_t kMinDecWarps = 4;
+constexpr uint32_t kMaxCbK = 16;           // codebook index widths the product takes (1..16)
 constexpr uint32_t kMmaWarp = 4;
 constexpr uint32_t kDec0 = 5;              // first decoder warp
 constexpr uint32_t kMaxThreads = (kDec0 + kMaxDecWarps) * 32;
@@ -78,7 +81,11 @@ constexpr uint32_t kDecBarrier = 1;        // named barrier of the decoder warps
 constexpr uint32_t kSplitEmpty = 0xFFFFFFFFu;
 
 struct GemmMat {
-    Df11Tensor t;          // the blob's sections (tile order); t.out unused
+    Df11Tensor t;          // DFloat11: the blob's sections (tile order); t.out unused
+    const uint8_t *packed; // codebook: the k-bit indices (tile order)
+    const uint16_t *table; // codebook: the table (U entries)
+    uint32_t table_words;  // codebook: 32-bit words to copy from the table (2U bytes, rounded up)
+    uint32_t pad;
     float *y;              // M x rows, row-major
     uint32_t rows, cols, k_tiles, kt_split;   // kt_split: k-tiles of part 0 when the K range is split, else 0
 };
@@ -116,6 +123,22 @@ __device__ __forceinline__ UnitSpan unit_span(const GemmBatch &B, uint32_t u) {
     return r;
 }
 
+// Codebook decoder warps' shared memory: the table (2^k entries, so that
+// every k-bit index stays inside it), two mbarriers and two task buffers per
+// warp (a task = 1024 indices = 16 rows of a tile = 128 k bytes), a claim
+// counter.
+struct CbGemmLayout {
+    uint32_t tab, bars, claim, bufs, total;
+    __host__ __device__ CbGemmLayout(uint32_t k, uint32_t warps) {
+        tab = 0;
+        bars = (2u << k) < 16u ? 16u : (2u << k);
+        claim = bars + ((16u * warps + 15u) & ~15u);
+        bufs = claim + 16u;
+        total = bufs + warps * 2u * 128u * k;
+    }
+};
+__host__ __device__ inline uint32_t cb_dec_bytes(uint32_t k, uint32_t warps) { return CbGemmLayout(k, warps).total; }
+
 // Shared memory of one CTA (offsets from a 1024-byte aligned base).
 struct GemmLayout {
     uint32_t stage_stride, x_off, x_stride, dec, ctl, total;
@@ -133,13 +156,16 @@ struct GemmLayout {
     static constexpr uint32_t kUnitItem = kUnitFirst + 4 * kMaxCtaUnits;   // u32[kMaxCtaUnits + 1]: first item
     static constexpr uint32_t kUnitTile = kUnitItem + 4 * (kMaxCtaUnits + 1) + 12;   // u32[kMaxCtaUnits + 1]
     static constexpr uint32_t kCtlBytes = kUnitTile + 4 * (kMaxCtaUnits + 1) + 12;
+    // cb_k = 0: DFloat11 decoder warps (the counted decoder's layout); cb_k = k:
+    // codebook decoder warps (CbGemmLayout)
     __host__ __device__ GemmLayout(uint32_t n_pad, uint32_t stages, uint32_t seg_words, uint32_t lut_entries,
-                                   uint32_t stage_bytes, uint32_t dec_warps) {
+                                   uint32_t stage_bytes, uint32_t dec_warps, uint32_t cb_k = 0) {
         stage_stride = kTileBytes;            // weight tiles, then x tiles; all multiples of 1024
         x_off = stages * stage_stride;
         x_stride = n_pad * 128u;
         dec = x_off + kXStages * x_stride;
-        ctl = dec + CountedLayout(seg_words, lut_entries, stage_bytes, dec_warps).total;
+        ctl = dec + (cb_k ? cb_dec_bytes(cb_k, dec_warps)
+                          : CountedLayout(seg_words, lut_entries, stage_bytes, dec_warps).total);
         ctl = (ctl + 15u) & ~15u;
         total = ctl + kCtlBytes;
     }
@@ -188,13 +214,16 @@ __device__ __forceinline__ uint32_t merge1r(uint32_t s, uint32_t r) {
     return ((s & 0x7Fu) | (r & 0x80u)) | (((r & 0x7Fu) | (s & 0x80u)) << 8);
 }
 
-__global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_constant__ GemmBatch B) {
+// The kernel body; CBK = 0: DFloat11 weights, CBK = k: codebook weights with
+// k-bit indices (only the decoder warps differ).
+template <int CBK>
+__device__ __forceinline__ void gemm_body(const GemmBatch &B) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
     const uint32_t raw_a = dev::smem_u32(smem_raw);
     uint8_t *smem = smem_raw + (((raw_a + 1023u) & ~1023u) - raw_a);   // tiles need 1024-byte alignment
     const uint32_t NS = B.stages;
-    const GemmLayout G(B.n_pad, NS, B.seg_words, B.lut_entries, B.stage_bytes, B.dec_warps);
+    const GemmLayout G(B.n_pad, NS, B.seg_words, B.lut_entries, B.stage_bytes, B.dec_warps, CBK);
     uint8_t *ctl = smem + G.ctl;
     uint64_t *full_x = reinterpret_cast<uint64_t *>(ctl + GemmLayout::kFullX);
     uint64_t *full_w = reinterpret_cast<uint64_t *>(ctl + GemmLayout::kFullW);
@@ -235,6 +264,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
     }
     for (uint32_t i = tid; i < nunits; i += blockDim.x) {
         const UnitSpan sp = unit_span(B, B.sched[c0 + i]);
+        u_tile[i + 1] = sp.kts;
+        if constexpr (CBK != 0) {   // codebook decoders take whole tiles: no blocks to find
+            u_first[i] = 0;
+            u_item[i + 1] = 0;
+            continue;
+        }
         const GemmMat &gm = B.m[sp.mat];
         const uint64_t lo = sp.lo, hi = lo + (uint64_t)sp.kts * kTileElems;
         // the last block whose first weight is <= v (block 0 starts at weight 0)
@@ -251,7 +286,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
         // the unit gets no items and is reported below
         u_first[i] = last >= first ? first : 0xFFFFFFFFu;
         u_item[i + 1] = last >= first ? last - first + 1 : 0u;
-        u_tile[i + 1] = sp.kts;
     }
     __syncthreads();
     if (tid == 0) {
@@ -388,7 +422,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             __syncwarp();
             if (lane == 0) dev::mbar_arrive(&acc_empty[ui & 1u]);
         }
-    } else {
+    } else if constexpr (CBK == 0) {
         // ---- decoder warps: blocks of this CTA's units, in order, into the stages
         const uint32_t dw = warp - kDec0, dt = tid - kDec0 * 32u;
         const uint32_t DW = B.dec_warps, DT = DW * 32u;
@@ -628,6 +662,117 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
             }
             i0 = i1;
         }
+    } else {
+        // ---- codebook decoder warps: tasks of 1024 indices (16 rows of a tile), in
+        // tile order, each bulk-copied into one of the warp's two buffers, unpacked
+        // (32 fields of k bits per lane), gathered from the table and stored as four
+        // 16-byte chunks at their swizzled places in the tile's stage
+        constexpr uint32_t K = CBK, kTaskBytes = 128u * K, kTaskWords = 32u * K;
+        const uint32_t DW = B.dec_warps, DT = DW * 32u, dw = warp - kDec0, dt = tid - kDec0 * 32u;
+        const CbGemmLayout C(K, DW);
+        uint8_t *dsm = smem + G.dec;
+        uint16_t *tab = reinterpret_cast<uint16_t *>(dsm + C.tab);
+        uint64_t *cbar = reinterpret_cast<uint64_t *>(dsm + C.bars) + 2 * dw;
+        uint32_t *claim = reinterpret_cast<uint32_t *>(dsm + C.claim);
+        uint32_t *bufs = reinterpret_cast<uint32_t *>(dsm + C.bufs) + dw * 2u * kTaskWords;
+        if (lane == 0) {
+            dev::mbar_init(&cbar[0], 1);
+            dev::mbar_init(&cbar[1], 1);
+            dev::fence_mbar_init();
+        }
+        __syncwarp();
+        uint32_t copies = 0;   // copies issued; copy c uses buffer and barrier c % 2, phase (c / 2) & 1
+        // lane 0: the bulk copy of task t's packed indices into buffer `copies % 2`
+        auto issue = [&](uint32_t t, uint32_t ui) {
+            if (lane == 0) {
+                const UnitSpan sp = unit_span(B, B.sched[c0 + ui]);
+                const GemmMat &g = B.m[sp.mat];
+                const uint64_t tile = (uint64_t)sp.ru * g.k_tiles + sp.kt0 + (t / 8u - u_tile[ui]);
+                const uint32_t b = copies & 1u;
+                dev::fence_proxy_async_smem();   // this warp's reads of the buffer come before the copy's writes
+                dev::mbar_arrive_expect_tx(&cbar[b], kTaskBytes);
+                dev::bulk_g2s(bufs + b * kTaskWords, g.packed + tile * (8u * kTaskBytes) + (t % 8u) * kTaskBytes,
+                              kTaskBytes, &cbar[b]);
+            }
+            copies++;
+        };
+        for (uint32_t i0 = 0; i0 < nunits;) {
+            const uint32_t mat = unit_mat(B.sched[c0 + i0]);
+            uint32_t i1 = i0 + 1;
+            while (i1 < nunits && unit_mat(B.sched[c0 + i1]) == mat) i1++;
+            const GemmMat &gm = B.m[mat];
+            const uint32_t tb = 8u * u_tile[i0], te = 8u * u_tile[i1];   // this run's tasks
+            auto unit_of = [&](uint32_t t, uint32_t from) {
+                while (from + 1 < i1 && 8u * u_tile[from + 1] <= t) from++;
+                return from;
+            };
+            dec_sync(DT);   // every decoder warp is done with the previous table
+            for (uint32_t i = dt; i < gm.table_words; i += DT)
+                reinterpret_cast<uint32_t *>(tab)[i] = reinterpret_cast<const uint32_t *>(gm.table)[i];
+            if (dt == 0) *claim = tb + DW;
+            dec_sync(DT);
+            uint32_t t = tb + dw, ui = i0;
+            if (t < te && !warp_aborted(abort_flag)) {
+                ui = unit_of(t, ui);
+                issue(t, ui);
+            } else {
+                t = te;
+            }
+            // invariant at the loop top: the copy of task t (t < te) is copy `copies - 1`
+            while (t < te && !warp_aborted(abort_flag)) {
+                const uint32_t cur = copies - 1u;
+                uint32_t tn = 0;
+                if (lane == 0) tn = atomicAdd(claim, 1u);
+                tn = __shfl_sync(0xFFFFFFFFu, tn, 0);
+                if (tn < te) {   // the next task's copy, into the other buffer
+                    ui = unit_of(tn, ui);
+                    issue(tn, ui);
+                }
+                const uint32_t q = t / 8u, s = q % NS;
+                uint32_t free_ = 0;
+                if (lane == 0) free_ = wait_count(&released[s], q / NS, abort_flag);
+                free_ = __shfl_sync(0xFFFFFFFFu, free_, 0);
+                const bool landed = dev::mbar_wait_bounded(&cbar[cur & 1u], (cur >> 1) & 1u);
+                if (__any_sync(0xFFFFFFFFu, !landed)) {
+                    bad |= LWC_DEVICE_TIMEOUT;
+                    if (lane == 0) dev::mbar_wait_bounded(&cbar[cur & 1u], (cur >> 1) & 1u);
+                }
+                if (!free_ || __any_sync(0xFFFFFFFFu, !landed)) {
+                    *abort_flag = 1;
+                    t = tn < te ? tn : te;   // a copy still in flight is waited for below
+                    break;
+                }
+                uint32_t wv[K + 1];
+                load_words<K>(bufs + (cur & 1u) * kTaskWords + lane * K, wv);
+                uint32_t o[16];
+                Gather<K, 0>::run(wv, tab, o);
+                __syncwarp();   // the buffer is free for the copy after next
+                // 32 weights: row 16 (t % 8) + lane / 2 of the tile, columns 32 (lane % 2) .. + 31
+                const uint32_t r = 16u * (t % 8u) + (lane >> 1), c8 = (lane & 1u) * 4u;
+                const uint32_t row = tiles_a + s * G.stage_stride + r * 128u;
+#pragma unroll
+                for (uint32_t k = 0; k < 4; k++)
+                    st_shared_v4(row + ((((c8 + k) ^ r) & 7u) << 4), o[4 * k], o[4 * k + 1], o[4 * k + 2],
+                                 o[4 * k + 3]);
+                dev::fence_proxy_async_smem();   // these stores before the MMA's (async-proxy) reads
+                __syncwarp();
+                if (lane == 0) {
+                    __threadfence_block();
+                    const uint32_t now = atomicAdd(&written[s], 1024u) + 1024u;
+                    if (now == kTileElems) {   // the tile is complete
+                        written[s] = 0;
+                        __threadfence_block();
+                        dev::mbar_arrive(&full_w[s]);
+                    }
+                }
+                t = tn < te ? tn : te;
+            }
+            if (t < te) {   // the copy of task t was issued: let it land (bounded)
+                if (lane == 0) dev::mbar_wait_bounded(&cbar[(copies - 1u) & 1u], ((copies - 1u) >> 1) & 1u);
+                __syncwarp();
+            }
+            i0 = i1;
+        }
     }
     umma::fence_before_sync();
     __syncthreads();
@@ -637,6 +782,33 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
     }
     if (bad && B.status) atomicOr(B.status, bad);
 }
+
+__global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_constant__ GemmBatch B) {
+    gemm_body<0>(B);
+}
+
+template <int K>
+__global__ void __launch_bounds__(kMaxThreads, 1) cb_gemm_kernel(const __grid_constant__ GemmBatch B) {
+    gemm_body<K>(B);
+}
+
+template <int K>
+void launch_cb_gemm(const GemmBatch &B, dim3 grid, dim3 block, size_t smem, cudaStream_t s) {
+    cb_gemm_kernel<K><<<grid, block, smem, s>>>(B);
+}
+using CbGemmLaunch = void (*)(const GemmBatch &, dim3, dim3, size_t, cudaStream_t);
+const CbGemmLaunch kCbGemmKernels[kMaxCbK + 1] = {
+    nullptr, launch_cb_gemm<1>, launch_cb_gemm<2>, launch_cb_gemm<3>, launch_cb_gemm<4>, launch_cb_gemm<5>,
+    launch_cb_gemm<6>, launch_cb_gemm<7>, launch_cb_gemm<8>, launch_cb_gemm<9>, launch_cb_gemm<10>,
+    launch_cb_gemm<11>, launch_cb_gemm<12>, launch_cb_gemm<13>, launch_cb_gemm<14>, launch_cb_gemm<15>,
+    launch_cb_gemm<16>};
+const void *const kCbGemmFuncs[kMaxCbK + 1] = {
+    nullptr, (const void *)cb_gemm_kernel<1>, (const void *)cb_gemm_kernel<2>, (const void *)cb_gemm_kernel<3>,
+    (const void *)cb_gemm_kernel<4>, (const void *)cb_gemm_kernel<5>, (const void *)cb_gemm_kernel<6>,
+    (const void *)cb_gemm_kernel<7>, (const void *)cb_gemm_kernel<8>, (const void *)cb_gemm_kernel<9>,
+    (const void *)cb_gemm_kernel<10>, (const void *)cb_gemm_kernel<11>, (const void *)cb_gemm_kernel<12>,
+    (const void *)cb_gemm_kernel<13>, (const void *)cb_gemm_kernel<14>, (const void *)cb_gemm_kernel<15>,
+    (const void *)cb_gemm_kernel<16>};
 
 // Source order -> tile order (the weight order lwc_gemm_dfloat11 reads):
 // each thread moves 16-byte pieces (8 weights of one row), read in source order.
@@ -695,6 +867,8 @@ lwc_status gemm_device(GemmDevice &out, EncodeTiledFn &encode) {
         if (err == cudaSuccess)
             err = cudaFuncSetAttribute((const void *)df11_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        c.max_smem);
+        for (uint32_t k = 1; k <= kMaxCbK && err == cudaSuccess; k++)
+            err = cudaFuncSetAttribute(kCbGemmFuncs[k], cudaFuncAttributeMaxDynamicSharedMemorySize, c.max_smem);
         if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device setup: %s", cudaGetErrorString(err));
         c.ready = true;
     }
@@ -732,42 +906,9 @@ bool schedule_units(const std::vector<uint32_t> &units, const std::vector<uint32
     return true;
 }
 
-}  // namespace
-}  // namespace lwc
-
-using namespace lwc;
-
-extern "C" {
-
-lwc_status lwc_tile_order(const uint16_t *d_src, uint64_t rows, uint64_t cols, uint16_t *d_dst, lwc_stream_t stream) {
-    if (rows % kTileRows || cols % kTileCols)
-        return fail(LWC_ERR_INVALID_ARG, "rows must be a multiple of 128 and cols of 64 (got %llu x %llu)",
-                    (unsigned long long)rows, (unsigned long long)cols);
-    if (rows == 0 || cols == 0) {
-        clear_error();
-        return LWC_OK;
-    }
-    if (!d_src || !d_dst) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer");
-    if (d_src == d_dst) return fail(LWC_ERR_INVALID_ARG, "the tile order is not computed in place");
-    if (!aligned16(d_src) || !aligned16(d_dst)) return fail(LWC_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
-    if (rows > (1ull << 40) / cols) return fail(LWC_ERR_INVALID_ARG, "matrix too large");
-    int dev = 0, sms = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device query: %s", cudaGetErrorString(err));
-    const uint64_t pieces = rows * cols / 8;
-    const uint64_t grid = std::min<uint64_t>((pieces + 255) / 256, (uint64_t)sms * 8);
-    tile_order_kernel<<<(unsigned)grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        reinterpret_cast<const uint4 *>(d_src), reinterpret_cast<uint4 *>(d_dst), rows, cols);
-    err = cudaGetLastError();
-    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "tile-order launch: %s", cudaGetErrorString(err));
-    clear_error();
-    return LWC_OK;
-}
-
-lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
-                                     const uint16_t *const *d_xs, int M, float *const *d_ys, int count,
-                                     uint32_t *d_status, lwc_stream_t stream) {
+lwc_status gemm_batched(uint32_t codec, const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
+                        const uint16_t *const *d_xs, int M, float *const *d_ys, int count, uint32_t *d_status,
+                        lwc_stream_t stream) {
     if (count < 0 || (count > 0 && (!descs || !d_blobs || !cols || !d_xs || !d_ys)))
         return fail(LWC_ERR_INVALID_ARG, "bad batch arguments");
     if (count > (int)kMaxMats) return fail(LWC_ERR_UNSUPPORTED, "at most %u matrices per call", kMaxMats);
@@ -780,30 +921,44 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     std::memset(&B, 0, sizeof B);
     std::vector<uint32_t> units, cost;
     uint64_t max_count = 0, max_tables = 0;
-    uint32_t chunk_bytes = 0, n = 0;
+    uint32_t chunk_bytes = 0, n = 0, cb_k = 0;
+    const bool cb = codec == LWC_CODEC_CODEBOOK;
     std::vector<int> mats;
     for (int i = 0; i < count; i++) {
         const lwc_desc &d = descs[i];
-        lwc_status st = check_df11_desc(&d);
+        lwc_status st = cb ? check_codebook_desc(&d) : check_df11_desc(&d);
         if (st) return st;
         if (d.n == 0) continue;
-        if (d.elem != LWC_ELEM_BF16) return fail(LWC_ERR_UNSUPPORTED, "matrix %d: BF16 weights only", i);
-        if (d.threads_per_block != 32 || !(d.flags & kFlagChunkCounts) || (d.flags & kFlagSingleExponent))
-            return fail(LWC_ERR_UNSUPPORTED,
-                        "matrix %d: needs blocks of 32 chunks with stored chunk counts and more than one exponent", i);
+        if (cb) {
+            if (d.k < 1 || d.k > kMaxCbK)
+                return fail(LWC_ERR_UNSUPPORTED, "matrix %d: codebook index width %u (1..%u taken)", i, d.k, kMaxCbK);
+            if (cb_k && d.k != cb_k) return fail(LWC_ERR_UNSUPPORTED, "matrices of one call must share the index width");
+            cb_k = d.k;
+        } else {
+            if (d.elem != LWC_ELEM_BF16) return fail(LWC_ERR_UNSUPPORTED, "matrix %d: BF16 weights only", i);
+            if (d.threads_per_block != 32 || !(d.flags & kFlagChunkCounts) || (d.flags & kFlagSingleExponent))
+                return fail(LWC_ERR_UNSUPPORTED,
+                            "matrix %d: needs blocks of 32 chunks with stored chunk counts and more than one exponent", i);
+        }
         if (cols[i] == 0 || cols[i] % kTileCols || cols[i] > (1u << 24) || d.n % cols[i])
             return fail(LWC_ERR_INVALID_ARG, "matrix %d: cols must divide n and be a multiple of 64 up to 2^24", i);
         const uint64_t rows = d.n / cols[i];
         if (rows % kTileRows || rows / kTileRows > 4096)
             return fail(LWC_ERR_INVALID_ARG, "matrix %d: rows must be a multiple of 128 (at most 2^19)", i);
-        if (chunk_bytes && d.chunk_bytes != chunk_bytes)
+        if (!cb && chunk_bytes && d.chunk_bytes != chunk_bytes)
             return fail(LWC_ERR_UNSUPPORTED, "matrices of one call must share chunk_bytes");
-        chunk_bytes = d.chunk_bytes;
+        if (!cb) chunk_bytes = d.chunk_bytes;
         if (!d_blobs[i] || !d_xs[i] || !d_ys[i]) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer (matrix %d)", i);
         if (!aligned16(d_blobs[i]) || !aligned16(d_xs[i]) || (reinterpret_cast<uintptr_t>(d_ys[i]) & 3u))
             return fail(LWC_ERR_MISALIGNED, "blob and x must be 16-byte aligned, y 4-byte aligned (matrix %d)", i);
         const uint8_t *base = static_cast<const uint8_t *>(d_blobs[i]);
         GemmMat &g = B.m[n];
+        if (cb) {
+            g.packed = base + d.off_packed;
+            g.table = reinterpret_cast<const uint16_t *>(base + d.off_table);
+            g.table_words = (d.U + 1) / 2;
+        }
+        if (!cb) {
         g.t.stream = reinterpret_cast<const uint32_t *>(base + d.off_stream);
         g.t.gaps = base + d.off_gaps;
         g.t.counts = base + d.off_counts;
@@ -815,13 +970,14 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
         g.t.stream_bytes = d.stream_bytes;
         g.t.n_blocks = (uint32_t)d.n_blocks;
         g.t.n_tables = d.n_tables;
+        max_count = std::max<uint64_t>(max_count, d.max_block_count);
+        max_tables = std::max<uint64_t>(max_tables, d.n_tables);
+        }
         g.y = d_ys[i];
         g.rows = (uint32_t)rows;
         g.cols = (uint32_t)cols[i];
         g.k_tiles = g.cols / kTileCols;
         g.kt_split = 0;
-        max_count = std::max<uint64_t>(max_count, d.max_block_count);
-        max_tables = std::max<uint64_t>(max_tables, d.n_tables);
         mats.push_back(i);
         n++;
     }
@@ -876,10 +1032,10 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
     // then, by shared memory, the most of them with at least three weight stages
     // (and as many stages as fit, up to kMaxStages); failing that, with two
     uint32_t warp_cap = (uint32_t)std::min<uint64_t>(kMaxDecWarps, kInFlightWeights / std::max<uint64_t>(max_count, 1));
-    warp_cap = std::max(kMinDecWarps, warp_cap & ~1u);
+    warp_cap = cb ? kMaxDecWarps : std::max(kMinDecWarps, warp_cap & ~1u);   // codebook tasks hold 1024 weights
     uint64_t smem = 0;
     auto fits = [&](uint32_t warps, uint32_t stages) {
-        smem = GemmLayout(B.n_pad, stages, B.seg_words, B.lut_entries, B.stage_bytes, warps).total + 1024;
+        smem = GemmLayout(B.n_pad, stages, B.seg_words, B.lut_entries, B.stage_bytes, warps, cb_k).total + 1024;
         return smem <= (uint64_t)dev.max_smem;
     };
     B.stages = 0;
@@ -915,11 +1071,67 @@ lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d
                                                   reinterpret_cast<cudaStream_t>(stream));
             if (e != cudaSuccess) return fail(LWC_ERR_CUDA, "output fill: %s", cudaGetErrorString(e));
         }
-    df11_gemm_kernel<<<ctas, (kDec0 + B.dec_warps) * 32u, (size_t)smem, reinterpret_cast<cudaStream_t>(stream)>>>(B);
+    const dim3 grid(ctas), block((kDec0 + B.dec_warps) * 32u);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cb)
+        kCbGemmKernels[cb_k](B, grid, block, (size_t)smem, s);
+    else
+        df11_gemm_kernel<<<grid, block, (size_t)smem, s>>>(B);
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "tensor-core product launch: %s", cudaGetErrorString(err));
     clear_error();
     return LWC_OK;
+}
+
+}  // namespace
+}  // namespace lwc
+
+using namespace lwc;
+
+extern "C" {
+
+lwc_status lwc_tile_order(const uint16_t *d_src, uint64_t rows, uint64_t cols, uint16_t *d_dst, lwc_stream_t stream) {
+    if (rows % kTileRows || cols % kTileCols)
+        return fail(LWC_ERR_INVALID_ARG, "rows must be a multiple of 128 and cols of 64 (got %llu x %llu)",
+                    (unsigned long long)rows, (unsigned long long)cols);
+    if (rows == 0 || cols == 0) {
+        clear_error();
+        return LWC_OK;
+    }
+    if (!d_src || !d_dst) return fail(LWC_ERR_INVALID_ARG, "NULL device pointer");
+    if (d_src == d_dst) return fail(LWC_ERR_INVALID_ARG, "the tile order is not computed in place");
+    if (!aligned16(d_src) || !aligned16(d_dst)) return fail(LWC_ERR_MISALIGNED, "device pointers must be 16-byte aligned");
+    if (rows > (1ull << 40) / cols) return fail(LWC_ERR_INVALID_ARG, "matrix too large");
+    int dev = 0, sms = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "device query: %s", cudaGetErrorString(err));
+    const uint64_t pieces = rows * cols / 8;
+    const uint64_t grid = std::min<uint64_t>((pieces + 255) / 256, (uint64_t)sms * 8);
+    tile_order_kernel<<<(unsigned)grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4 *>(d_src), reinterpret_cast<uint4 *>(d_dst), rows, cols);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return fail(LWC_ERR_CUDA, "tile-order launch: %s", cudaGetErrorString(err));
+    clear_error();
+    return LWC_OK;
+}
+
+lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
+                                     const uint16_t *const *d_xs, int M, float *const *d_ys, int count,
+                                     uint32_t *d_status, lwc_stream_t stream) {
+    return gemm_batched(LWC_CODEC_DFLOAT11, descs, d_blobs, cols, d_xs, M, d_ys, count, d_status, stream);
+}
+
+lwc_status lwc_gemm_codebook_batched(const lwc_desc *descs, const void *const *d_blobs, const uint64_t *cols,
+                                     const uint16_t *const *d_xs, int M, float *const *d_ys, int count,
+                                     uint32_t *d_status, lwc_stream_t stream) {
+    return gemm_batched(LWC_CODEC_CODEBOOK, descs, d_blobs, cols, d_xs, M, d_ys, count, d_status, stream);
+}
+
+lwc_status lwc_gemm_codebook(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x, int M,
+                             float *d_y, uint32_t *d_status, lwc_stream_t stream) {
+    if (!desc) return fail(LWC_ERR_INVALID_ARG, "NULL descriptor");
+    return lwc_gemm_codebook_batched(desc, &d_blob, &cols, &d_x, M, &d_y, 1, d_status, stream);
 }
 
 lwc_status lwc_gemm_dfloat11(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x, int M,

@@ -131,15 +131,20 @@ GEMM_CHUNK_BYTES = 20
 
 
 class TiledWeights:
-    """Weight matrices held for the tensor-core product (lwc_gemm_dfloat11):
-    each rows x cols BF16 matrix (rows % 128 == 0, cols % 64 == 0) is put in
-    tile order on the GPU (lwc_tile_order) and compressed there by the
-    DFloat11 device encoder. ``gemm`` then computes y = x W^T for 1 to 256
-    activation rows with W decoded straight into the MMA's shared-memory
-    operands (the BF16 matrix is never written to device memory)."""
+    """Weight matrices held for the tensor-core product (lwc_gemm_dfloat11 /
+    lwc_gemm_codebook): each rows x cols BF16 matrix (rows % 128 == 0, cols %
+    64 == 0) is put in tile order on the GPU (lwc_tile_order) and compressed
+    there by the device encoder of ``codec``. ``gemm`` then computes y = x W^T
+    for 1 to 256 activation rows with W decoded straight into the MMA's
+    shared-memory operands (the BF16 matrix is never written to device
+    memory). A batched call takes matrices of one codec (codebook: one index
+    width)."""
 
-    def __init__(self, device):
+    def __init__(self, device, codec: str = "dfloat11"):
+        if codec not in CODECS:
+            raise ValueError(f"unknown codec {codec!r}")
         self.device = device
+        self.codec = codec
         self.descs, self.blobs, self.shapes = [], [], []
 
     def add(self, w, workspace=None, stream=None, chunk_bytes: int = GEMM_CHUNK_BYTES) -> int:
@@ -154,7 +159,8 @@ class TiledWeights:
         tiled = torch.empty_like(src)
         lwc.lwc_tile_order(src, rows, cols, tiled, stream)
         with torch.cuda.stream(stream):
-            d, b = encode_on_device(tiled, "dfloat11", workspace=workspace, stream=stream, chunk_bytes=chunk_bytes)
+            params = {"chunk_bytes": chunk_bytes} if self.codec == "dfloat11" else {}
+            d, b = encode_on_device(tiled, self.codec, workspace=workspace, stream=stream, **params)
         del tiled
         self.descs.append(d)
         self.blobs.append(b)
@@ -180,7 +186,8 @@ class TiledWeights:
         M = int(x.shape[0])
         if out is None:
             out = torch.empty((M, rows), dtype=torch.float32, device=x.device)
-        lwc.lwc_gemm_dfloat11(self.descs[index], self.blobs[index], cols, x, M, out, d_status=status, stream=stream)
+        fn = lwc.lwc_gemm_dfloat11 if self.codec == "dfloat11" else lwc.lwc_gemm_codebook
+        fn(self.descs[index], self.blobs[index], cols, x, M, out, d_status=status, stream=stream)
         return out
 
     def gemm_batched(self, indices, xs, outs=None, stream=None, status=None):
@@ -194,7 +201,8 @@ class TiledWeights:
             outs = [torch.empty((M, self.shapes[i][0]), dtype=torch.float32, device=xs[0].device) for i in indices]
         batch = lwc.LinearBatch([self.descs[i] for i in indices], [self.blobs[i] for i in indices],
                                 [self.shapes[i][1] for i in indices], xs, outs, M)
-        lwc.lwc_gemm_dfloat11_batched(batch, d_status=status, stream=stream)
+        fn = lwc.lwc_gemm_dfloat11_batched if self.codec == "dfloat11" else lwc.lwc_gemm_codebook_batched
+        fn(batch, d_status=status, stream=stream)
         return outs
 
 

@@ -45,7 +45,8 @@ EXPORTED = (
     "lwc_encode_dfloat11_elements_device_plan", "lwc_encode_codebook_device_plan",
     "lwc_encode_device_write", "lwc_encode_dfloat11_device_noalloc", "lwc_linear_codebook",
     "lwc_linear_codebook_batched", "lwc_linear_dfloat11", "lwc_linear_dfloat11_batched",
-    "lwc_tile_order", "lwc_gemm_dfloat11", "lwc_gemm_dfloat11_batched",
+    "lwc_tile_order", "lwc_gemm_dfloat11", "lwc_gemm_dfloat11_batched", "lwc_gemm_codebook",
+    "lwc_gemm_codebook_batched",
     "lwc_selftest_bounded_wait", "lwc_status_string",
     "lwc_last_error", "lwc_version",
 )
@@ -126,11 +127,13 @@ def load():
     for name in ("lwc_linear_codebook", "lwc_linear_dfloat11"):
         getattr(L, name).argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
         getattr(L, name).restype = ctypes.c_int
-    L.lwc_gemm_dfloat11.argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
-    L.lwc_gemm_dfloat11.restype = ctypes.c_int
+    for name in ("lwc_gemm_dfloat11", "lwc_gemm_codebook"):
+        getattr(L, name).argtypes = [D, _P, _u64, _P, ctypes.c_int, _P, _P, _P]
+        getattr(L, name).restype = ctypes.c_int
     L.lwc_tile_order.argtypes = [_P, _u64, _u64, _P, _P]
     L.lwc_tile_order.restype = ctypes.c_int
-    for name in ("lwc_linear_codebook_batched", "lwc_linear_dfloat11_batched", "lwc_gemm_dfloat11_batched"):
+    for name in ("lwc_linear_codebook_batched", "lwc_linear_dfloat11_batched", "lwc_gemm_dfloat11_batched",
+                 "lwc_gemm_codebook_batched"):
         getattr(L, name).argtypes = [D, ctypes.POINTER(_P), ctypes.POINTER(_u64), ctypes.POINTER(_P), ctypes.c_int,
                                      ctypes.POINTER(_P), ctypes.c_int, _P, _P]
         getattr(L, name).restype = ctypes.c_int
@@ -339,6 +342,19 @@ def lwc_gemm_dfloat11_batched(batch: LinearBatch, d_status=None, stream=None) ->
     """Several tile-order DFloat11 matrices (at most 8) in one launch."""
     b = batch
     _check(load().lwc_gemm_dfloat11_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
+                                            _stream(stream)))
+
+
+def lwc_gemm_codebook(desc: lwc_desc, d_blob, cols: int, d_x, M: int, d_y, d_status=None, stream=None) -> None:
+    """As lwc_gemm_dfloat11, for a tile-order codebook blob."""
+    _check(load().lwc_gemm_codebook(ctypes.byref(desc), _addr(d_blob), cols, _addr(d_x), M, _addr(d_y),
+                                    _addr(d_status), _stream(stream)))
+
+
+def lwc_gemm_codebook_batched(batch: LinearBatch, d_status=None, stream=None) -> None:
+    """Several tile-order codebook matrices (at most 8, one index width) in one launch."""
+    b = batch
+    _check(load().lwc_gemm_codebook_batched(b.descs, b.blobs, b.cols, b.xs, b.M, b.ys, b.count, _addr(d_status),
                                             _stream(stream)))
 
 

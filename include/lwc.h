@@ -338,6 +338,23 @@ LWC_API lwc_status lwc_gemm_dfloat11_batched(const lwc_desc *descs, const void *
                                              float *const *d_ys, int count, uint32_t *d_status,
                                              lwc_stream_t stream);
 
+/* As lwc_gemm_dfloat11, for a codebook blob of tile-ordered weights (codebook
+ * page: "Codebook Lossless Compression: когда 25% памяти значат больше, чем
+ * кажется", section "Как работает эта магия?": out[i] = table[index i]):
+ * each 1024-index run of a tile's packed indices is copied, unpacked and
+ * looked up into the shared-memory operand. Index widths k = 1..16 (a
+ * one-entry table, k = 0, gives LWC_ERR_UNSUPPORTED); at k = 16 the 128 KB
+ * table may leave no room for larger M (LWC_ERR_UNSUPPORTED). Same bound and
+ * repeatability as lwc_gemm_dfloat11. */
+LWC_API lwc_status lwc_gemm_codebook(const lwc_desc *desc, const void *d_blob, uint64_t cols, const uint16_t *d_x,
+                                     int M, float *d_y, uint32_t *d_status, lwc_stream_t stream);
+
+/* `count` (at most 8) codebook matrices with one index width in one launch. */
+LWC_API lwc_status lwc_gemm_codebook_batched(const lwc_desc *descs, const void *const *d_blobs,
+                                             const uint64_t *cols, const uint16_t *const *d_xs, int M,
+                                             float *const *d_ys, int count, uint32_t *d_status,
+                                             lwc_stream_t stream);
+
 /* ---- device encoders ------------------------------------------------------ */
 
 /* Compression of a tensor that is already in GPU memory, into a blob in GPU

@@ -255,3 +255,110 @@ def test_damaged_blobs_are_reported_and_contained():
     d0, b0 = tiled_blob(w)
     y = run_gemm(d0, b0, cols, x1, 64)
     assert np.array_equal(y, OL.bf16_values(w)[:, :64].T)
+
+
+# ---- the codebook codec -----------------------------------------------------------
+
+def cb_tiled_blob(w_u16):
+    d, b = lwc.lwc_encode_codebook(OL.tile_order(w_u16))
+    return d, torch.from_numpy(b).to("cuda")
+
+
+def run_cb_gemm(d, blob, cols, x, M):
+    rows = d.n // cols
+    y = torch.full((M, rows), float("nan"), dtype=torch.float32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_gemm_codebook(d, blob, cols, x, M, y, status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return y.cpu().numpy().astype(np.float64)
+
+
+def few_values(rows, cols, U, seed):
+    """A matrix drawing from U distinct BF16 values (index width ceil(log2 U))."""
+    vals = synth.as_u16(synth.normal_bf16((U * 4,), seed=seed, sigma=0.02))
+    vals = np.unique(vals)[:U]
+    rng = np.random.default_rng(seed)
+    return vals[rng.integers(0, len(vals), rows * cols)].reshape(rows, cols)
+
+
+@pytest.mark.parametrize("rows,cols", [(128, 64), (256, 320), (384, 1024)])
+@pytest.mark.parametrize("M", [1, 16, 33, 128, 256])
+def test_codebook_gemm_matches_oracle(rows, cols, M):
+    w = weights(rows, cols, seed=rows * 3 + cols)
+    d, blob = cb_tiled_blob(w)
+    assert d.k >= 1
+    x = synth.activations_bf16(M, cols, seed=M + 7, device="cuda")
+    check(run_cb_gemm(d, blob, cols, x, M), w, x)
+
+
+@pytest.mark.parametrize("U,M", [(2, 16), (3, 64), (17, 16), (255, 128), (1000, 40), (40000, 16), (65536, 16)])
+def test_codebook_gemm_index_widths(U, M):
+    rows, cols = 256, 192
+    w = few_values(rows, cols, U, seed=U) if U < 65536 else \
+        synth.as_u16(synth.uniform_patterns(rows * cols, seed=5)).reshape(rows, cols)
+    w = np.where(np.isfinite(OL.bf16_values(w)) & (np.abs(OL.bf16_values(w)) < 1e30), w, np.uint16(0x3F80))
+    d, blob = cb_tiled_blob(w)
+    x = synth.activations_bf16(M, cols, seed=U, device="cuda")
+    check(run_cb_gemm(d, blob, cols, x, M), w, x)
+
+
+def test_codebook_one_hot_sweep_checks_every_weight_exactly():
+    rows, cols, M = 256, 320, 64
+    w = weights(rows, cols, seed=15)
+    d, blob = cb_tiled_blob(w)
+    wv = OL.bf16_values(w)
+    for c0 in range(0, cols, M):
+        x = torch.zeros((M, cols), dtype=torch.bfloat16, device="cuda")
+        x[torch.arange(M), c0 + torch.arange(M)] = 1.0
+        assert np.array_equal(run_cb_gemm(d, blob, cols, x, M), wv[:, c0:c0 + M].T)
+
+
+@pytest.mark.parametrize("M", [16, 128])
+def test_codebook_llama3_8b_layer_sampled_rows(M):
+    tensors = list(synth.llama_layer_tensors(1, device="cuda"))
+    tw = TiledWeights(torch.device("cuda"), codec="codebook")
+    idx = [tw.add(t) for _, t in tensors]
+    ks = {tw.descs[i].k for i in idx}
+    xs = [synth.activations_bf16(M, tw.shapes[i][1], seed=400 + i, device="cuda") for i in idx]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    if len(ks) > 1:   # one launch takes one index width: group by k
+        ys = [None] * len(idx)
+        for k in ks:
+            sel = [i for i in idx if tw.descs[i].k == k]
+            for i, y in zip(sel, tw.gemm_batched(sel, [xs[i] for i in sel], status=status)):
+                ys[i] = y
+    else:
+        ys = tw.gemm_batched(idx, xs, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rng = np.random.default_rng(2)
+    for i, (_, t) in zip(idx, tensors):
+        rows, cols = tw.shapes[i]
+        pick = np.sort(rng.choice(rows, 48, replace=False))
+        w_rows = synth.as_u16(t[torch.from_numpy(pick).to("cuda")]).reshape(len(pick), cols)
+        want, mag = OL.linear(w_rows, synth.as_u16(xs[i]).reshape(M, cols))
+        got = ys[i].cpu().numpy().astype(np.float64)[:, pick]
+        assert np.all(np.abs(got - want) <= OL.float32_tree_bound(mag, cols, unit_roundoff=U_TC))
+
+
+def test_codebook_gemm_argument_errors():
+    w = weights(256, 128, seed=31)
+    d, blob = cb_tiled_blob(w)
+    x = synth.activations_bf16(4, 128, seed=32, device="cuda")
+    y = torch.empty((4, 256), dtype=torch.float32, device="cuda")
+    d1, b1 = lwc.lwc_encode_codebook(np.full(256 * 128, 0x3F80, np.uint16))   # one value: k = 0
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_gemm_codebook(d1, torch.from_numpy(b1).to("cuda"), 128, x, 4, y)
+    assert e.value.status == lwc.LWC_ERR_UNSUPPORTED
+    w2 = few_values(256, 128, 5, seed=33)
+    d2, b2 = cb_tiled_blob(w2)
+    assert d2.k != d.k
+    yb = [torch.empty((4, 256), dtype=torch.float32, device="cuda") for _ in range(2)]
+    batch = lwc.LinearBatch([d, d2], [blob, b2], [128, 128], [x, x], yb, 4)
+    with pytest.raises(lwc.LwcError) as e:
+        lwc.lwc_gemm_codebook_batched(batch)
+    assert e.value.status == lwc.LWC_ERR_UNSUPPORTED
+    dd, bd = tiled_blob(w)   # a DFloat11 blob is not a codebook blob
+    with pytest.raises(lwc.LwcError):
+        lwc.lwc_gemm_codebook(dd, bd, 128, x, 4, y)
