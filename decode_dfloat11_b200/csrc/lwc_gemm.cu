@@ -74,7 +74,9 @@ constexpr uint32_t kMinDecWarps = 4;
 constexpr uint32_t kMaxCbK = 16;           // codebook index widths the product takes (1..16)
 constexpr uint32_t kMmaWarp = 4;
 constexpr uint32_t kDec0 = 5;              // first decoder warp
+constexpr uint32_t kMaxCbDecWarps = 20;   // codebook decoder warps
 constexpr uint32_t kMaxThreads = (kDec0 + kMaxDecWarps) * 32;
+constexpr uint32_t kMaxCbThreads = (kDec0 + kMaxCbDecWarps) * 32;
 constexpr uint32_t kDecBarrier = 1;        // named barrier of the decoder warps
 // y of a matrix whose K range is split starts as this pattern (a NaN that no
 // sum of finite or infinite products yields: those NaNs are canonical)
@@ -788,7 +790,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1) df11_gemm_kernel(const __grid_
 }
 
 template <int K>
-__global__ void __launch_bounds__(kMaxThreads, 1) cb_gemm_kernel(const __grid_constant__ GemmBatch B) {
+__global__ void __launch_bounds__(kMaxCbThreads, 1) cb_gemm_kernel(const __grid_constant__ GemmBatch B) {
     gemm_body<K>(B);
 }
 
@@ -1032,7 +1034,7 @@ lwc_status gemm_batched(uint32_t codec, const lwc_desc *descs, const void *const
     // then, by shared memory, the most of them with at least three weight stages
     // (and as many stages as fit, up to kMaxStages); failing that, with two
     uint32_t warp_cap = (uint32_t)std::min<uint64_t>(kMaxDecWarps, kInFlightWeights / std::max<uint64_t>(max_count, 1));
-    warp_cap = cb ? kMaxDecWarps : std::max(kMinDecWarps, warp_cap & ~1u);   // codebook tasks hold 1024 weights
+    warp_cap = cb ? kMaxCbDecWarps : std::max(kMinDecWarps, warp_cap & ~1u);   // codebook tasks hold 1024 weights
     uint64_t smem = 0;
     auto fits = [&](uint32_t warps, uint32_t stages) {
         smem = GemmLayout(B.n_pad, stages, B.seg_words, B.lut_entries, B.stage_bytes, warps, cb_k).total + 1024;
