@@ -888,14 +888,20 @@ bool schedule_units(const std::vector<uint32_t> &units, const std::vector<uint32
     std::vector<uint32_t> order(units.size());
     std::iota(order.begin(), order.end(), 0u);
     std::stable_sort(order.begin(), order.end(), [&](uint32_t a, uint32_t b) { return cost[a] > cost[b]; });
-    std::vector<uint64_t> load(ctas, 0);
+    // min-heap of (load, CTA): the least loaded CTA, the lower index on ties
+    std::vector<std::pair<uint64_t, uint32_t>> heap;
+    heap.reserve(ctas);
+    for (uint32_t c = 0; c < ctas; c++) heap.push_back({0, c});
+    const auto later = [](const std::pair<uint64_t, uint32_t> &a, const std::pair<uint64_t, uint32_t> &b) {
+        return a > b;
+    };
     std::vector<std::vector<uint16_t>> per(ctas);
     for (uint32_t j : order) {
-        uint32_t best = 0;
-        for (uint32_t c = 1; c < ctas; c++)
-            if (load[c] < load[best]) best = c;
-        load[best] += cost[j];
-        per[best].push_back((uint16_t)units[j]);
+        std::pop_heap(heap.begin(), heap.end(), later);
+        auto &top = heap.back();
+        per[top.second].push_back((uint16_t)units[j]);
+        top.first += cost[j];
+        std::push_heap(heap.begin(), heap.end(), later);
     }
     uint32_t pos = 0;
     for (uint32_t c = 0; c < ctas; c++) {
