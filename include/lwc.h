@@ -427,7 +427,7 @@ LWC_API lwc_status lwc_encode_device_write(const void *d_src, uint64_t n, void *
  *     total_bytes is the size needed.
  *   - The first call on a device (per process) looks up the scratch array's
  *     device address for that device (cudaGetSymbolAddress, with that device
- *     current); make that first call before any stream capture.
+ *     current).
  *   - Every call on a device shares the one scratch array, which keeps the
  *     last call's contents (each call clears what must start at zero). Calls
  *     whose GPU work overlaps — from several host threads, or on several
