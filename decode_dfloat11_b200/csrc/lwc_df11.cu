@@ -1067,7 +1067,11 @@ __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_warp_k
 // The counted decoder's body. LIN = 0: merge and store the weights (decoder).
 // LIN > 0: dot them with up to LIN activation rows instead (fused linear
 // layer, BF16 elements only), as in df11_warp_body.
-template <int E, int LIN>
+// FX: the launch's codes have no word longer than 8 bits, and tensors whose
+// words all have one length take the fixed-length path (a kernel of its own:
+// with FX = 0 the path is compiled out and the variable-length path keeps its
+// registers).
+template <int E, int LIN, bool FX = false>
 __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11Lin *X) {
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
@@ -1125,6 +1129,12 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
         build_counted_tables(lut, ntab, sym, sub, first_long, tid, blockDim.x, [] { __syncthreads(); });
         __syncthreads();
         const uint32_t v0 = *first_long;
+        // A code whose words all have one length L <= 8 (then every 11-bit window
+        // decodes the same number of codes in the same number of bits, and only
+        // then): its codes are fixed-width fields, decoded by direct indexing of a
+        // 2^L-entry table (in place of the second-level tables, which such a code
+        // does not use)
+        const uint32_t fixed_len = FX ? fixed_code_length(sym, sub, tid, blockDim.x) : 0u;
 
         while (w < s_end && !dead) {
             const uint32_t b = w - tn.first_work;
@@ -1189,21 +1199,31 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
                     const bool has_next = lane + 1 < 32u || b + 1 < tn.n_blocks;
                     const uint64_t next = has_next ? (uint64_t)(lane + 1) * cbits + gapb[lane + 1] : rem_block;
                     const uint32_t end = (uint32_t)min(next, rem_block);
-                    if (cnt) {
-                        const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
-                                                            stage_a, slot_a, bad);
-                        // the last step may decode past the lane's codes (by at most 40 bits);
-                        // falling short of the next chunk's first code, or far past it, means a bad count
-                        if (got - end > 40u) bad |= LWC_DEVICE_BAD_COUNT;
-                    }
-                    __syncwarp();
-                    // the bytes of this lane's first, shared word
-                    if ((qb & 3u) && cnt) {
-                        const uint32_t hw = *slot, j0 = qb & 3u;
-                        uint8_t *hb = stage + (qb & ~3u);
-                        hb[j0] = (uint8_t)(hw >> (8 * j0));
-                        if (j0 < 3 && cnt > 1) hb[j0 + 1] = (uint8_t)(hw >> (8 * j0 + 8));
-                        if (j0 == 1 && cnt > 2) hb[3] = (uint8_t)(hw >> 24);
+                    if (FX && fixed_len) {
+                        // the block's codes lie back to back from its first chunk's first code
+                        const uint32_t start0 = gapb[0];
+                        stage_fixed(seg, last, sub, fixed_len, start0, total, (uint32_t)(o0 & 15u),
+                                    reinterpret_cast<uint32_t *>(stage), lane);
+                        // they must end where the next block's first code starts (or the stream ends)
+                        const uint64_t block_end = b + 1 < tn.n_blocks ? 32ull * cbits + gapb[32] : rem_block;
+                        if ((uint64_t)start0 + (uint64_t)total * fixed_len != block_end) bad |= LWC_DEVICE_BAD_COUNT;
+                    } else {
+                        if (cnt) {
+                            const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
+                                                                stage_a, slot_a, bad);
+                            // the last step may decode past the lane's codes (by at most 40 bits);
+                            // falling short of the next chunk's first code, or far past it, means a bad count
+                            if (got - end > 40u) bad |= LWC_DEVICE_BAD_COUNT;
+                        }
+                        __syncwarp();
+                        // the bytes of this lane's first, shared word
+                        if ((qb & 3u) && cnt) {
+                            const uint32_t hw = *slot, j0 = qb & 3u;
+                            uint8_t *hb = stage + (qb & ~3u);
+                            hb[j0] = (uint8_t)(hw >> (8 * j0));
+                            if (j0 < 3 && cnt > 1) hb[j0 + 1] = (uint8_t)(hw >> (8 * j0 + 8));
+                            if (j0 == 1 && cnt > 2) hb[3] = (uint8_t)(hw >> 24);
+                        }
                     }
                     __syncwarp();
                     // the segment is free: fetch this warp's next block while merging this one
@@ -1280,9 +1300,9 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
     if (bad && B.status) atomicOr(B.status, bad);
 }
 
-template <int E>
+template <int E, bool FX = false>
 __global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counted_kernel(const __grid_constant__ Df11Batch B) {
-    df11_counted_body<E, 0>(B, nullptr);
+    df11_counted_body<E, 0, FX>(B, nullptr);
 }
 
 // Fused decode + linear layer on blobs with stored chunk counts (BF16, blocks
@@ -1354,6 +1374,8 @@ lwc_status device_config(DeviceConfig &out) {
             (const void *)df11_decode_kernel<256, LWC_ELEM_FP16>, (const void *)df11_decode_kernel<1024, LWC_ELEM_FP16>,
             (const void *)df11_warp_kernel<LWC_ELEM_FP16>, (const void *)df11_counted_kernel<LWC_ELEM_BF16>,
             (const void *)df11_counted_kernel<LWC_ELEM_FP32>, (const void *)df11_counted_kernel<LWC_ELEM_FP16>,
+            (const void *)df11_counted_kernel<LWC_ELEM_BF16, true>, (const void *)df11_counted_kernel<LWC_ELEM_FP32, true>,
+            (const void *)df11_counted_kernel<LWC_ELEM_FP16, true>,
             (const void *)kLinKernels[0], (const void *)kLinKernels[1],
             (const void *)kLinKernels[2], (const void *)kLinKernels[3], (const void *)kCtdLinKernels[0],
             (const void *)kCtdLinKernels[1], (const void *)kCtdLinKernels[2], (const void *)kCtdLinKernels[3]};
@@ -1371,13 +1393,15 @@ lwc_status device_config(DeviceConfig &out) {
 
 
 // Decode kernels: one CTA per block (blocks of 64+ chunks), one warp per
-// block (blocks of 32 chunks), or one warp per block with stored chunk counts.
-enum KernelMode { kModeBlock, kModeWarp, kModeCounted };
+// block (blocks of 32 chunks), or one warp per block with stored chunk counts
+// (kModeCountedShort: codes of at most 8 bits, with the fixed-length path).
+enum KernelMode { kModeBlock, kModeWarp, kModeCounted, kModeCountedShort };
 
 template <int E>
 const void *df11_kernel(KernelMode mode, uint32_t T) {
-    return mode == kModeCounted ? (const void *)df11_counted_kernel<E>
-           : mode == kModeWarp  ? (const void *)df11_warp_kernel<E>
+    return mode == kModeCounted        ? (const void *)df11_counted_kernel<E>
+           : mode == kModeCountedShort ? (const void *)df11_counted_kernel<E, true>
+           : mode == kModeWarp         ? (const void *)df11_warp_kernel<E>
            : T <= 256           ? (const void *)df11_decode_kernel<256, E>
                                 : (const void *)df11_decode_kernel<1024, E>;
 }
@@ -1393,6 +1417,8 @@ void launch_df11(KernelMode mode, uint32_t T, unsigned grid, uint32_t threads, s
                  const Df11Batch &B) {
     if (mode == kModeCounted)
         df11_counted_kernel<E><<<grid, threads, smem, stream>>>(B);
+    else if (mode == kModeCountedShort)
+        df11_counted_kernel<E, true><<<grid, threads, smem, stream>>>(B);
     else if (mode == kModeWarp)
         df11_warp_kernel<E><<<grid, threads, smem, stream>>>(B);
     else if (T <= 256)
@@ -1403,7 +1429,8 @@ void launch_df11(KernelMode mode, uint32_t T, unsigned grid, uint32_t threads, s
 
 // Shared memory of a per-warp launch with w warps per CTA.
 uint64_t warp_smem(const Df11Batch &B, KernelMode mode, uint32_t w) {
-    return mode == kModeCounted ? CountedLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total
+    return mode == kModeCounted || mode == kModeCountedShort
+               ? CountedLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total
                                 : WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total;
 }
 
@@ -1455,7 +1482,10 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
-    const KernelMode mode = T != 32 ? kModeBlock : (d0.flags & kFlagChunkCounts) ? kModeCounted : kModeWarp;
+    const KernelMode mode = T != 32                           ? kModeBlock
+                            : !(d0.flags & kFlagChunkCounts) ? kModeWarp
+                            : d0.max_len <= 8                ? kModeCountedShort
+                                                             : kModeCounted;
     const bool per_warp = mode != kModeBlock;
     B.warps = per_warp ? warps_that_fit(B, cfg.max_smem, mode) : 0;
     const uint32_t threads = per_warp ? B.warps * 32u : T;
@@ -1618,7 +1648,8 @@ lwc_status lwc_decode_dfloat11_batched(const lwc_desc *descs, const void *const 
             continue;
         }
         const uint64_t counted = (d.flags & kFlagChunkCounts) ? 1 : 0;
-        keyed.push_back({(counted << 50) | ((uint64_t)d.elem << 40) | ((uint64_t)d.chunk_bytes << 20) |
+        const uint64_t short_codes = counted && d.max_len <= 8 ? 1 : 0;   // the kernel with the fixed-length path
+        keyed.push_back({(short_codes << 51) | (counted << 50) | ((uint64_t)d.elem << 40) | ((uint64_t)d.chunk_bytes << 20) |
                              d.threads_per_block,
                          i});
     }

@@ -272,5 +272,47 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
     return pos;
 }
 
+// Whole CTA (threads t = 0 .. nt - 1 are all of it), after the symbol table
+// is built: L when every symbol-table entry holds the same number c of codes
+// in the same c L bits with L <= 8, else 0. That holds exactly when every code
+// word has length L: a window that starts with copies of a code word of
+// length l decodes min(4, 11 / l) of them in l times as many bits, so equal
+// entries give every word the same length, and a word longer than 11 bits
+// leaves its windows' entries empty. For such a code, tab[v] (v < 2^L, in the
+// second-level tables' place) becomes the rotated exponent of code word v.
+__device__ __forceinline__ uint32_t fixed_code_length(const uint2 *sym, uint32_t *tab, uint32_t t, uint32_t nt) {
+    const uint32_t y0 = sym[0].y;
+    int same = y0 != 0u;
+    for (uint32_t v = t; v < (uint32_t)kFastSize; v += nt) same &= sym[v].y == y0;
+    const uint32_t c = y0 >> 11, used = y0 & 31u;
+    if (!__syncthreads_and(same) || c == 0 || used % c != 0 || used / c > 8) return 0;
+    const uint32_t L = used / c;
+    for (uint32_t v = t; v < (1u << L); v += nt) tab[v] = sym[v << (kFastBits - L)].x & 0xFFu;
+    __syncthreads();
+    return L;
+}
+
+// One warp: the staging words of n codes of fixed length L (<= 8) that lie
+// back to back from segment bit `start`; exponent i goes to staging byte
+// qb + i. Lane l writes words qb / 4 + l, + 32, ... as aligned 32-bit stores,
+// each from one 32-bit window (four fields) and four lookups in tab (2^L
+// entries); the bytes of a word outside qb .. qb + n - 1 hold what the
+// neighbouring fields decode to and are never read. Segment reads stay inside
+// the segment whatever the arguments say.
+__device__ __forceinline__ void stage_fixed(const uint32_t *seg, uint32_t last, const uint32_t *tab, uint32_t L,
+                                            uint32_t start, uint32_t n, uint32_t qb, uint32_t *stage, uint32_t lane) {
+    const uint32_t words = (qb + n + 3) >> 2, sh = 32u - L;
+    for (uint32_t k = (qb >> 2) + lane; k < words; k += 32) {
+        const int32_t i0 = (int32_t)(4 * k) - (int32_t)qb;   // the exponent of the word's byte 0 (>= -3)
+        const uint32_t p = start + (i0 > 0 ? (uint32_t)i0 : 0u) * L;
+        const uint32_t wi = p >> 5;
+        const uint32_t win = __funnelshift_l(seg[min(wi + 1, last)], seg[min(wi, last)], p);   // bits p .. p + 31
+        uint32_t x = tab[win >> sh] | (tab[(win << L) >> sh] << 8) | (tab[(win << (2 * L)) >> sh] << 16) |
+                     (tab[(win << (3 * L)) >> sh] << 24);
+        if (i0 < 0) x <<= 8u * (uint32_t)(-i0);
+        stage[k] = x;
+    }
+}
+
 }  // namespace df11dev
 }  // namespace lwc

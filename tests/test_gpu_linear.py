@@ -132,6 +132,25 @@ def test_single_value_and_single_exponent_tensors(codec):
         check(y, w.reshape(rows, cols), x, cols, codec, d)
 
 
+@pytest.mark.parametrize("L", [1, 4, 7])
+def test_fixed_length_codes(L):
+    """Flat exponent histograms over 2^L values: every code word has length L,
+    which the counted kernel reads as back-to-back L-bit fields; one-hot rows
+    check every weight of a few columns exactly."""
+    rows, cols = 37, 1040
+    w = synth.as_u16(synth.equal_exponents(rows * cols, L, seed=70 + L))
+    d, blob = encode(w, "dfloat11", chunk_bytes=20)
+    assert d.flags & 2
+    x = synth.activations_bf16(5, cols, seed=L, device="cuda")
+    check(run_linear("dfloat11", d, blob, cols, x, 5), w.reshape(rows, cols), x, cols, "dfloat11", d)
+    W = OL.bf16_values(w.reshape(rows, cols))
+    cs = [0, 1, 511, 1032, 1039]
+    x = torch.zeros((len(cs), cols), dtype=torch.bfloat16, device="cuda")
+    for m, c in enumerate(cs):
+        x[m, c] = 1.0
+    assert np.array_equal(run_linear("dfloat11", d, blob, cols, x, len(cs)), W[:, cs].T)
+
+
 def moderate(w: np.ndarray) -> np.ndarray:
     """Map exponent fields into [49, 205] (values 2^-78 .. 2^79): products with
     activations and their sums stay inside FP32's normal range, where the

@@ -229,6 +229,77 @@ def test_df11_corruption_is_contained(tpb):
             assert int(status.item()) != 0, i
 
 
+# ------------------------------------------------------------ fixed-length codes
+#
+# Flat exponent histograms over 2^L values give every code word length L; the
+# counted decoder then reads a block's codes as back-to-back L-bit fields
+# (the uniform-exponent stress tensor is L = 8). Chunk sizes whose bit count
+# is not a multiple of L make codes straddle chunks (non-zero gaps).
+
+@pytest.mark.parametrize("L", range(1, 9))
+@pytest.mark.parametrize("chunk_bytes", [8, 20, 36])
+def test_df11_fixed_length_codes(L, chunk_bytes):
+    w = synth.as_u16(synth.equal_exponents(333_333 + 17 * L, L, seed=100 + L))
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes)
+    lengths = b[d.off_lengths:d.off_lengths + 256]
+    assert set(lengths[lengths > 0].tolist()) == {L}
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = host_u16(gpu_decode(d, dev(b), status=status))
+    assert int(status.item()) == 0
+    assert np.array_equal(got, odf.decode(b))
+    assert np.array_equal(got, w)
+
+
+def test_df11_fixed_length_batched_and_device_encoded():
+    """Fixed- and variable-length tensors alternating in one launch (the CTA
+    switches paths at each tensor boundary), encoded on the device."""
+    from decode_dfloat11_b200.layers import encode_on_device
+    ws = [synth.equal_exponents(200_003, 8, seed=61, device="cuda"),
+          synth.normal_bf16((300_007,), seed=62, sigma=0.02, device="cuda"),
+          synth.equal_exponents(150_001, 3, seed=63, device="cuda"),
+          synth.equal_exponents(77_777, 6, seed=64, device="cuda"),
+          synth.normal_bf16((1_001,), seed=65, sigma=0.02, device="cuda")]
+    enc = [encode_on_device(w, "dfloat11") for w in ws]
+    outs = [torch.empty(w.numel(), dtype=torch.int16, device="cuda") for w in ws]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_batched([d for d, _ in enc], [b for _, b in enc], outs, status,
+                                    torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    for w, (d, b), o in zip(ws, enc, outs):
+        assert torch.equal(o, w.view(torch.int16).reshape(-1))
+        assert np.array_equal(host_u16(o), odf.decode(b.cpu().numpy()))
+
+
+def test_df11_fixed_length_corruption_is_contained():
+    w = synth.as_u16(synth.equal_exponents(500_000, 8, seed=9))
+    d, b = lwc.lwc_encode_dfloat11(w)
+    assert d.flags & 2
+    guard = 4096
+    cases = []
+    x = b.copy()                                   # block 1 starts one bit late
+    x[d.off_gaps + 32] ^= np.uint8(1)
+    cases.append(("gap", x))
+    x = b.copy()                                   # a chunk count one too high
+    x[d.off_counts + 2 * 32 + 5] += np.uint8(1)
+    cases.append(("count", x))
+    x = b.copy()                                   # payload bit flips: still valid codes
+    pos = d.off_stream + np.random.default_rng(1).integers(0, (d.total_bits + 7) // 8, 50)
+    x[pos] ^= np.uint8(0x10)
+    cases.append(("payload", x))
+    for name, x in cases:
+        out = torch.zeros(w.size + 2 * guard, dtype=torch.int16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        lwc.lwc_decode_dfloat11_checked(d, dev(x), out[guard:guard + w.size], status, torch.cuda.current_stream())
+        torch.cuda.synchronize()
+        got = host_u16(out)
+        assert np.all(got[:guard] == 0) and np.all(got[guard + w.size:] == 0), name   # nothing outside
+        if name == "payload":
+            assert np.array_equal(got[guard:guard + w.size], odf.decode(x)), name
+        else:
+            assert int(status.item()) & lwc.LWC_DEVICE_BAD_COUNT, name
+
+
 # ------------------------------------------------------------ full-size configs
 
 def test_llama3_8b_layer_full_size():

@@ -462,3 +462,133 @@ def test_gemm_tile_placement_model(rows, cols, chunk, order):
                 for c in (0, 5, 8, 31, 63):
                     assert slots[q][_sw128(r, c)] == w[u * 128 + r, j * 64 + c]
             q += 1
+
+
+# ---- fixed-length codes (fixed_code_length / stage_fixed, csrc/lwc_df11_dev.cuh) ----
+#
+# When every code word has one length L <= 8 (flat exponent histograms: the
+# uniform-exponent stress tensor is L = 8), the counted decoder reads the
+# block's codes as back-to-back L-bit fields: each staging word from one
+# 32-bit window and four lookups in a 2^L-entry table. Restated here: the
+# test that picks this path (all symbol-table entries equal), and the word
+# stores, checked for single writers, in-range words and segment reads, and
+# the staged bytes.
+
+def _fixed_code_length(sym):
+    y0 = sym[0][1]
+    if y0 == 0 or any(e[1] != y0 for e in sym):
+        return 0
+    c, used = y0 >> 11, y0 & 31
+    if c == 0 or used % c or used // c > 8:
+        return 0
+    return used // c
+
+
+def _stage_fixed(seg, last, tab, L, start, n, qb):
+    """stage_fixed for the whole warp: [(word, value)] in store order."""
+    stores = []
+    sh = 32 - L
+    for k in range(qb >> 2, (qb + n + 3) >> 2):
+        i0 = 4 * k - qb
+        assert i0 >= -3
+        p = start + max(i0, 0) * L
+        wi = p >> 5
+        lo_i, hi_i = min(wi + 1, last), min(wi, last)
+        assert 0 <= hi_i <= lo_i <= last
+        win = _fsl(seg[lo_i], seg[hi_i], p & 31)
+        x = 0
+        for j in range(4):
+            f = ((win << (j * L)) & 0xFFFFFFFF) >> sh
+            assert f < len(tab)
+            x |= tab[f] << (8 * j)
+        if i0 < 0:
+            x = (x << (8 * -i0)) & 0xFFFFFFFF
+        stores.append((k, x))
+    return stores
+
+
+def _blob_tables(b):
+    from oracle import blob as B
+    h = B.unpack_header(b)
+    lut = B.section(b, h["off_lut"], 512 * h["n_tables"], np.uint16).tolist()
+    return h, _counted_tables(lut)
+
+
+@pytest.mark.parametrize("L", range(1, 9))
+@pytest.mark.parametrize("chunk", [8, 12, 36])
+def test_fixed_length_staging_model(L, chunk):
+    import synth
+    from decode_dfloat11_b200 import lwc
+    from oracle import blob as B
+    from oracle import df11 as odf
+
+    w = synth.as_u16(synth.equal_exponents(60_001, L, seed=L))
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk)
+    h, (sym, sub, first_long) = _blob_tables(b)
+    lengths = B.section(b, h["off_lengths"], 256)
+    assert set(lengths[lengths > 0].tolist()) == {L}
+    assert first_long == 1 << FAST_BITS          # no code longer than the fast table's 11 bits
+    assert _fixed_code_length(sym) == L
+    if not d.flags & 2:                          # > 255 codes per chunk: no stored counts, two-pass kernel
+        assert 8 * chunk // L > 255
+        return
+    tab = [sym[v << (FAST_BITS - L)][0] & 0xFF for v in range(1 << L)]
+    exps, _ = odf.split(w)
+    words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
+    gaps = B.section(b, h["off_gaps"], h["n_blocks"] * 32)
+    counts = B.section(b, h["off_counts"], h["n_blocks"] * 32)
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
+    cw = chunk // 4
+    cbits = 32 * cw
+    seg_words = (32 * cw + 2 + 3) // 4 * 4
+    stage_bytes = (int(np.diff(blkoff).max()) + 16 + 15) // 16 * 16
+    nb = h["n_blocks"]
+    for blk in sorted({0, 1, nb // 2, nb - 2, nb - 1} & set(range(nb))):
+        o0, o1 = int(blkoff[blk]), int(blkoff[blk + 1])
+        n = o1 - o0
+        assert int(counts[blk * 32:(blk + 1) * 32].sum()) == n
+        seg = [int(x) for x in words[blk * 32 * cw:blk * 32 * cw + seg_words]]
+        seg += [0xDEADBEEF] * (seg_words - len(seg))
+        start0 = int(gaps[blk * 32])
+        rem_block = h["total_bits"] - blk * 32 * cbits
+        block_end = 32 * cbits + int(gaps[(blk + 1) * 32]) if blk + 1 < nb else rem_block
+        assert start0 + n * L == block_end, blk           # the kernel's consistency check holds
+        stores = _stage_fixed(seg, seg_words - 1, tab, L, start0, n, o0 & 15)
+        ks = [k for k, _ in stores]
+        assert len(ks) == len(set(ks)) and all(4 * k + 4 <= stage_bytes for k in ks), blk
+        stage = bytearray(b"\xAA" * stage_bytes)
+        for k, x in stores:
+            stage[4 * k:4 * k + 4] = x.to_bytes(4, "little")
+        got = np.frombuffer(bytes(stage[(o0 & 15):(o0 & 15) + n]), np.uint8)
+        assert np.array_equal(got, np.array([_rot(int(x)) for x in exps[o0:o1]], np.uint8)), blk
+
+
+@pytest.mark.parametrize("case", ["normal", "three_values", "nine_values", "two_lengths", "long_codes"])
+def test_fixed_length_test_rejects_variable_codes(case):
+    """Codes with more than one word length never take the fixed-length path,
+    however flat their histogram."""
+    import synth
+    from decode_dfloat11_b200 import lwc
+
+    rng = np.random.default_rng(5)
+    if case == "normal":
+        w = synth.as_u16(synth.normal_bf16((100_000,), seed=5, sigma=0.02))
+    elif case == "long_codes":
+        fib = [1, 1]
+        while len(fib) < 24:
+            fib.append(fib[-1] + fib[-2])
+        w = np.repeat((np.arange(24, dtype=np.uint16) << 7) | 0x8011, np.array(fib))
+    else:
+        m = {"three_values": 3, "nine_values": 9, "two_lengths": 16}[case]
+        reps = np.full(m, 1000)
+        if case == "two_lengths":
+            reps[:4] = 3000            # four exponents three times as frequent: lengths 3 and 5
+        w = np.repeat((np.arange(120, 120 + m, dtype=np.uint16) << 7), reps)
+        w |= rng.integers(0, 128, w.size).astype(np.uint16)
+    w = rng.permutation(w).astype(np.uint16)
+    d, b = lwc.lwc_encode_dfloat11(w)
+    h, (sym, _, _) = _blob_tables(b)
+    from oracle import blob as B
+    lengths = B.section(b, h["off_lengths"], 256)
+    assert len(set(lengths[lengths > 0].tolist())) > 1
+    assert _fixed_code_length(sym) == 0
