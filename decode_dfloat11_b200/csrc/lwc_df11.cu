@@ -243,6 +243,118 @@ __device__ __forceinline__ void merge_one(uint32_t s, uint32_t e, void *out, con
     }
 }
 
+// ---- fixed-length codes ------------------------------------------------------------
+//
+// When every code word has one length L, code i is stream bits [i L, i L + L)
+// (the stream is the codes back to back from bit 0), so weights are decoded
+// straight from their index: no block offsets, gaps or counts are needed
+// beyond the range a CTA owns.
+
+// Code word c (0 <= c < 32) of a 32-weight piece whose stream bits start at a
+// multiple of 32 in the words w[0..L] (MSB first).
+template <int L>
+__device__ __forceinline__ uint32_t fixed_field(const uint32_t (&w)[L + 1], int c) {
+    const int p = c * L, k = p >> 5, o = p & 31;
+    if (o + L <= 32) return (w[k] << o) >> (32 - L);
+    return __funnelshift_l(w[k + 1], w[k], (uint32_t)o) >> (32 - L);
+}
+
+// The CTA's threads t = 0 .. nt - 1: weights [ob, oe) of tensor tn, whose
+// code words all have length L (1..8); tab[v] = rotated exponent of code
+// word v. AFF: code word v stands for exponent base + v (a flat histogram over
+// consecutive exponents gives this canonical code), so a piece's exponents
+// are its fields plus base, with no lookups. Threads take 32-weight pieces in
+// turn (32 L stream bits = L words, 32 sign|mantissa bytes, two 16-weight
+// merges), lane 0 of each warp bringing the warp's pieces of the next turn
+// into L2; then the up to 31 weights at either end one by one. Stream reads
+// stay inside the stream section whatever the offsets say; the caller
+// checks ob <= oe <= n.
+template <int E, int L, bool AFF>
+__device__ __noinline__ void decode_fixed_range(const Df11Tensor &tn, const uint32_t *tab, uint32_t base,
+                                                uint64_t ob, uint64_t oe, uint32_t t, uint32_t nt) {
+    const uint64_t nwords = tn.stream_bytes >> 2;
+    const uint64_t p_lo = (ob + 31) & ~31ull, p_hi = oe & ~31ull;
+    const uint32_t base4 = base * 0x01010101u;
+    for (uint64_t g = p_lo + 32ull * t; g < p_hi; g += 32ull * nt) {
+        if ((t & 31u) == 0) {   // the warp's 1,024 weights of the next turn into L2
+            const uint64_t ga = g + 32ull * nt;
+            if (ga + 1024 <= p_hi) {
+                dev::prefetch_l2(tn.sm + ga, 1024u);
+                const uint64_t s0 = (ga / 32 * L * 4) & ~15ull, s1 = ((ga + 1024) / 32 * L * 4 + 15) & ~15ull;
+                if (s1 <= (tn.stream_bytes & ~15ull))
+                    dev::prefetch_l2(reinterpret_cast<const uint8_t *>(tn.stream) + s0, (uint32_t)(s1 - s0));
+            }
+        }
+        const uint64_t w0 = g / 32 * L;   // the piece's first stream word
+        uint32_t w[L + 1];
+        if (L % 4 == 0 && w0 + L <= nwords) {   // 16-byte aligned: w0 is a multiple of L
+#pragma unroll
+            for (int j = 0; j < L; j += 4) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(tn.stream + w0 + j));
+                w[j] = v.x;
+                w[j + 1] = v.y;
+                w[j + 2] = v.z;
+                w[j + 3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < L; j++) w[j] = w0 + j < nwords ? __ldg(tn.stream + w0 + j) : 0u;
+        }
+        w[L] = 0;
+        const uint4 s0 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g));
+        const uint4 s1 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g + 16));
+        uint32_t e[8];
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            if constexpr (AFF && L == 8) {   // four whole bytes, first code in the top one
+                e[q] = __byte_perm(w[q], 0u, 0x0123u) + base4;
+            } else if constexpr (AFF) {   // each byte stays <= 255: base + 2^L - 1 <= 255
+                e[q] = (fixed_field<L>(w, 4 * q) | (fixed_field<L>(w, 4 * q + 1) << 8) |
+                        (fixed_field<L>(w, 4 * q + 2) << 16) | (fixed_field<L>(w, 4 * q + 3) << 24)) + base4;
+            } else {
+                e[q] = tab[fixed_field<L>(w, 4 * q)] | (tab[fixed_field<L>(w, 4 * q + 1)] << 8) |
+                       (tab[fixed_field<L>(w, 4 * q + 2)] << 16) | (tab[fixed_field<L>(w, 4 * q + 3)] << 24);
+            }
+        }
+        merge_group<E, !AFF>(s0, make_uint4(e[0], e[1], e[2], e[3]), tn.out, tn.lo, g);
+        merge_group<E, !AFF>(s1, make_uint4(e[4], e[5], e[6], e[7]), tn.out, tn.lo, g + 16);
+    }
+    // the weights before the first piece (u = 0..30) and after the last (u = 31..61)
+    for (uint32_t u = t; u < 62; u += nt) {
+        const uint64_t i = u < 31 ? ob + u : (p_hi > p_lo ? p_hi : p_lo) + (u - 31);
+        const bool one = u < 31 ? i < (p_lo < oe ? p_lo : oe) : i < oe;
+        if (one) {
+            const uint64_t p = i * L, k = p >> 5;
+            const uint32_t w_a = k < nwords ? __ldg(tn.stream + k) : 0u;
+            const uint32_t w_b = k + 1 < nwords ? __ldg(tn.stream + k + 1) : 0u;
+            const uint32_t f = __funnelshift_l(w_b, w_a, (uint32_t)p & 31u) >> (32 - L);
+            merge_one<E, true>(tn.sm[i], tab[f], tn.out, tn.lo, i);
+        }
+    }
+}
+
+// mode = L | kFixedAffine (or not), from fixed_code_length.
+template <int E>
+__device__ __forceinline__ void decode_fixed(uint32_t mode, const Df11Tensor &tn, const uint32_t *tab, uint64_t ob,
+                                             uint64_t oe, uint32_t t, uint32_t nt) {
+    const uint32_t base = ((tab[0] << 1) | (tab[0] >> 7)) & 0xFFu;   // exponent of code word 0
+    switch (mode) {
+#define LWC_FIXED_CASE(L_)                                                       \
+    case L_: decode_fixed_range<E, L_, false>(tn, tab, base, ob, oe, t, nt); break; \
+    case L_ | kFixedAffine: decode_fixed_range<E, L_, true>(tn, tab, base, ob, oe, t, nt); break;
+        LWC_FIXED_CASE(1)
+        LWC_FIXED_CASE(2)
+        LWC_FIXED_CASE(3)
+        LWC_FIXED_CASE(4)
+        LWC_FIXED_CASE(5)
+        LWC_FIXED_CASE(6)
+        LWC_FIXED_CASE(7)
+        LWC_FIXED_CASE(8)
+#undef LWC_FIXED_CASE
+    default: break;
+    }
+}
+
 // ---- block scan ------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *warp_sums, uint32_t &total) {
@@ -1134,7 +1246,33 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
         // then): its codes are fixed-width fields, decoded by direct indexing of a
         // 2^L-entry table (in place of the second-level tables, which such a code
         // does not use)
-        const uint32_t fixed_len = FX ? fixed_code_length(sym, sub, tid, blockDim.x) : 0u;
+        if constexpr (FX && !LIN) {
+            if (const uint32_t fixed_mode = fixed_code_length(sym, sub, tid, blockDim.x)) {
+                const uint32_t fixed_len = fixed_mode & 15u;
+                // the copy of this warp's first block, issued before the tables: let it land
+                if (w < s_end && !dead) {
+                    const bool arrived = dev::mbar_wait_bounded(bar, items & 1u);
+                    items++;
+                    if (__any_sync(0xFFFFFFFFu, !arrived)) {
+                        bad |= LWC_DEVICE_TIMEOUT;
+                        if (lane == 0) dev::mbar_wait_bounded(bar, (items - 1) & 1u);
+                        dead = true;
+                    }
+                }
+                // this CTA's blocks of the tensor hold weights [ob, oe); adjacent CTAs share
+                // their boundary offset, so the ranges tile [0, n) when the tensor's first
+                // offset is 0, its last is n and every range is ordered
+                const uint32_t b0 = w0 - tn.first_work, b1 = s_end - tn.first_work;
+                const uint64_t ob = tn.blkoff[b0], oe = tn.blkoff[b1];
+                if (!(ob <= oe && oe <= tn.n && (b0 != 0 || ob == 0) && (b1 != tn.n_blocks || oe == tn.n)))
+                    bad |= LWC_DEVICE_BAD_OFFSET;
+                else if (tn.total_bits != tn.n * fixed_len)   // L bits per weight, nothing else
+                    bad |= LWC_DEVICE_BAD_COUNT;
+                else
+                    decode_fixed<E>(fixed_mode, tn, sub, ob, oe, tid, blockDim.x);
+                w = s_end;   // no block loop
+            }
+        }
 
         while (w < s_end && !dead) {
             const uint32_t b = w - tn.first_work;
@@ -1199,31 +1337,21 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
                     const bool has_next = lane + 1 < 32u || b + 1 < tn.n_blocks;
                     const uint64_t next = has_next ? (uint64_t)(lane + 1) * cbits + gapb[lane + 1] : rem_block;
                     const uint32_t end = (uint32_t)min(next, rem_block);
-                    if (FX && fixed_len) {
-                        // the block's codes lie back to back from its first chunk's first code
-                        const uint32_t start0 = gapb[0];
-                        stage_fixed(seg, last, sub, fixed_len, start0, total, (uint32_t)(o0 & 15u),
-                                    reinterpret_cast<uint32_t *>(stage), lane);
-                        // they must end where the next block's first code starts (or the stream ends)
-                        const uint64_t block_end = b + 1 < tn.n_blocks ? 32ull * cbits + gapb[32] : rem_block;
-                        if ((uint64_t)start0 + (uint64_t)total * fixed_len != block_end) bad |= LWC_DEVICE_BAD_COUNT;
-                    } else {
-                        if (cnt) {
-                            const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
-                                                                stage_a, slot_a, bad);
-                            // the last step may decode past the lane's codes (by at most 40 bits);
-                            // falling short of the next chunk's first code, or far past it, means a bad count
-                            if (got - end > 40u) bad |= LWC_DEVICE_BAD_COUNT;
-                        }
-                        __syncwarp();
-                        // the bytes of this lane's first, shared word
-                        if ((qb & 3u) && cnt) {
-                            const uint32_t hw = *slot, j0 = qb & 3u;
-                            uint8_t *hb = stage + (qb & ~3u);
-                            hb[j0] = (uint8_t)(hw >> (8 * j0));
-                            if (j0 < 3 && cnt > 1) hb[j0 + 1] = (uint8_t)(hw >> (8 * j0 + 8));
-                            if (j0 == 1 && cnt > 2) hb[3] = (uint8_t)(hw >> 24);
-                        }
+                    if (cnt) {
+                        const uint32_t got = decode_counted(seg, last, sym, sub, v0, lut, ntab, start, cnt, qb,
+                                                            stage_a, slot_a, bad);
+                        // the last step may decode past the lane's codes (by at most 40 bits);
+                        // falling short of the next chunk's first code, or far past it, means a bad count
+                        if (got - end > 40u) bad |= LWC_DEVICE_BAD_COUNT;
+                    }
+                    __syncwarp();
+                    // the bytes of this lane's first, shared word
+                    if ((qb & 3u) && cnt) {
+                        const uint32_t hw = *slot, j0 = qb & 3u;
+                        uint8_t *hb = stage + (qb & ~3u);
+                        hb[j0] = (uint8_t)(hw >> (8 * j0));
+                        if (j0 < 3 && cnt > 1) hb[j0 + 1] = (uint8_t)(hw >> (8 * j0 + 8));
+                        if (j0 == 1 && cnt > 2) hb[3] = (uint8_t)(hw >> 24);
                     }
                     __syncwarp();
                     // the segment is free: fetch this warp's next block while merging this one

@@ -273,45 +273,30 @@ __device__ __forceinline__ uint32_t decode_counted(const uint32_t *seg, uint32_t
 }
 
 // Whole CTA (threads t = 0 .. nt - 1 are all of it), after the symbol table
-// is built: L when every symbol-table entry holds the same number c of codes
-// in the same c L bits with L <= 8, else 0. That holds exactly when every code
-// word has length L: a window that starts with copies of a code word of
-// length l decodes min(4, 11 / l) of them in l times as many bits, so equal
-// entries give every word the same length, and a word longer than 11 bits
-// leaves its windows' entries empty. For such a code, tab[v] (v < 2^L, in the
-// second-level tables' place) becomes the rotated exponent of code word v.
+// is built: L (1..8) when every symbol-table entry holds the same number c of
+// codes in the same c L bits with L <= 8, plus kFixedAffine when code word v
+// stands for exponent e0 + v for every v; else 0. Equal entries hold exactly
+// when every code word has length L: a window that starts with copies of a
+// code word of length l decodes min(4, 11 / l) of them in l times as many
+// bits, so equal entries give every word the same length, and a word longer
+// than 11 bits leaves its windows' entries empty. For such a code, tab[v]
+// (v < 2^L, in the second-level tables' place) becomes the rotated exponent
+// of code word v.
+constexpr uint32_t kFixedAffine = 16;
+
 __device__ __forceinline__ uint32_t fixed_code_length(const uint2 *sym, uint32_t *tab, uint32_t t, uint32_t nt) {
-    const uint32_t y0 = sym[0].y;
+    const uint32_t y0 = sym[0].y, c = y0 >> 11, used = y0 & 31u;
     int same = y0 != 0u;
     for (uint32_t v = t; v < (uint32_t)kFastSize; v += nt) same &= sym[v].y == y0;
-    const uint32_t c = y0 >> 11, used = y0 & 31u;
-    if (!__syncthreads_and(same) || c == 0 || used % c != 0 || used / c > 8) return 0;
-    const uint32_t L = used / c;
+    const uint32_t L = c != 0 && used % c == 0 && used / c <= 8 ? used / c : 0u;
+    if (!__syncthreads_and(same) || L == 0) return 0;
     for (uint32_t v = t; v < (1u << L); v += nt) tab[v] = sym[v << (kFastBits - L)].x & 0xFFu;
     __syncthreads();
-    return L;
-}
-
-// One warp: the staging words of n codes of fixed length L (<= 8) that lie
-// back to back from segment bit `start`; exponent i goes to staging byte
-// qb + i. Lane l writes words qb / 4 + l, + 32, ... as aligned 32-bit stores,
-// each from one 32-bit window (four fields) and four lookups in tab (2^L
-// entries); the bytes of a word outside qb .. qb + n - 1 hold what the
-// neighbouring fields decode to and are never read. Segment reads stay inside
-// the segment whatever the arguments say.
-__device__ __forceinline__ void stage_fixed(const uint32_t *seg, uint32_t last, const uint32_t *tab, uint32_t L,
-                                            uint32_t start, uint32_t n, uint32_t qb, uint32_t *stage, uint32_t lane) {
-    const uint32_t words = (qb + n + 3) >> 2, sh = 32u - L;
-    for (uint32_t k = (qb >> 2) + lane; k < words; k += 32) {
-        const int32_t i0 = (int32_t)(4 * k) - (int32_t)qb;   // the exponent of the word's byte 0 (>= -3)
-        const uint32_t p = start + (i0 > 0 ? (uint32_t)i0 : 0u) * L;
-        const uint32_t wi = p >> 5;
-        const uint32_t win = __funnelshift_l(seg[min(wi + 1, last)], seg[min(wi, last)], p);   // bits p .. p + 31
-        uint32_t x = tab[win >> sh] | (tab[(win << L) >> sh] << 8) | (tab[(win << (2 * L)) >> sh] << 16) |
-                     (tab[(win << (3 * L)) >> sh] << 24);
-        if (i0 < 0) x <<= 8u * (uint32_t)(-i0);
-        stage[k] = x;
-    }
+    // the exponent of word v, un-rotated, against that of word 0 plus v
+    const uint32_t e0 = ((tab[0] << 1) | (tab[0] >> 7)) & 0xFFu;
+    int affine = e0 + (1u << L) - 1u <= 255u;
+    for (uint32_t v = t; v < (1u << L); v += nt) affine &= (((tab[v] << 1) | (tab[v] >> 7)) & 0xFFu) == e0 + v;
+    return __syncthreads_and(affine) ? L | kFixedAffine : L;
 }
 
 }  // namespace df11dev

@@ -202,16 +202,18 @@ def uniform_patterns(n: int, seed: int, device="cpu") -> torch.Tensor:
                          dtype=torch.int16).view(torch.bfloat16)
 
 
-def equal_exponents(n: int, bits: int, seed: int, first: int | None = None, device="cpu") -> torch.Tensor:
-    """n patterns whose exponents take 2^bits consecutive values (from `first`,
-    by default centred on 127) in equal numbers (n // 2^bits of each, the
-    remainder from the first values), in random order, with uniform sign and
-    mantissa bits: exponent frequencies as flat as they can be."""
+def equal_exponents(n: int, bits: int, seed: int, first: int | None = None, step: int = 1,
+                    device="cpu") -> torch.Tensor:
+    """n patterns whose exponents take 2^bits values first, first + step, ...
+    (by default consecutive and centred on 127) in equal numbers (n // 2^bits
+    of each, the remainder from the first values), in random order, with
+    uniform sign and mantissa bits: exponent frequencies as flat as they can
+    be."""
     m = 1 << bits
-    first = (128 - m // 2) if first is None else first
-    assert 0 <= first and first + m <= 256
+    first = (128 - step * m // 2) if first is None else first
+    assert 0 <= first and first + step * (m - 1) <= 255
     g = _gen(seed, device)
-    e = (torch.arange(n, device=device, dtype=torch.int32) % m) + first
+    e = (torch.arange(n, device=device, dtype=torch.int32) % m) * step + first
     e = e[torch.randperm(n, generator=g, device=device)]
     sm = torch.randint(0, 256, (n,), generator=g, device=device, dtype=torch.int32)
     u = ((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)

@@ -236,10 +236,13 @@ def test_df11_corruption_is_contained(tpb):
 # (the uniform-exponent stress tensor is L = 8). Chunk sizes whose bit count
 # is not a multiple of L make codes straddle chunks (non-zero gaps).
 
+@pytest.mark.parametrize("step", [1, 2])   # consecutive exponents (decoded without lookups) or not
 @pytest.mark.parametrize("L", range(1, 9))
 @pytest.mark.parametrize("chunk_bytes", [8, 20, 36])
-def test_df11_fixed_length_codes(L, chunk_bytes):
-    w = synth.as_u16(synth.equal_exponents(333_333 + 17 * L, L, seed=100 + L))
+def test_df11_fixed_length_codes(L, chunk_bytes, step):
+    if step * ((1 << L) - 1) > 255:
+        pytest.skip("2^L exponents with gaps do not fit in 8 bits")
+    w = synth.as_u16(synth.equal_exponents(333_333 + 17 * L, L, seed=100 + L, step=step))
     d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes)
     lengths = b[d.off_lengths:d.off_lengths + 256]
     assert set(lengths[lengths > 0].tolist()) == {L}
@@ -256,7 +259,7 @@ def test_df11_fixed_length_batched_and_device_encoded():
     from decode_dfloat11_b200.layers import encode_on_device
     ws = [synth.equal_exponents(200_003, 8, seed=61, device="cuda"),
           synth.normal_bf16((300_007,), seed=62, sigma=0.02, device="cuda"),
-          synth.equal_exponents(150_001, 3, seed=63, device="cuda"),
+          synth.equal_exponents(150_001, 3, seed=63, step=3, device="cuda"),
           synth.equal_exponents(77_777, 6, seed=64, device="cuda"),
           synth.normal_bf16((1_001,), seed=65, sigma=0.02, device="cuda")]
     enc = [encode_on_device(w, "dfloat11") for w in ws]
@@ -272,21 +275,30 @@ def test_df11_fixed_length_batched_and_device_encoded():
 
 
 def test_df11_fixed_length_corruption_is_contained():
+    """A fixed-length tensor is decoded from the block offsets at the ends of
+    each CTA's range and its stream: a first offset other than 0 or a last
+    other than n is reported, an interior offset out of order either is
+    reported (at a CTA boundary) or is not read, and nothing is written
+    outside the output; damaged code words decode as the oracle decodes them;
+    the gaps and counts are not read on this path."""
     w = synth.as_u16(synth.equal_exponents(500_000, 8, seed=9))
     d, b = lwc.lwc_encode_dfloat11(w)
     assert d.flags & 2
     guard = 4096
     cases = []
-    x = b.copy()                                   # block 1 starts one bit late
-    x[d.off_gaps + 32] ^= np.uint8(1)
-    cases.append(("gap", x))
-    x = b.copy()                                   # a chunk count one too high
-    x[d.off_counts + 2 * 32 + 5] += np.uint8(1)
-    cases.append(("count", x))
-    x = b.copy()                                   # payload bit flips: still valid codes
+    for name, blk, v in (("first", 0, 64), ("last", d.n_blocks, 2 ** 40), ("interior", 3, 2 ** 40)):
+        x = b.copy()
+        x[d.off_blkoff + 8 * blk: d.off_blkoff + 8 * blk + 8] = np.array([v], np.uint64).view(np.uint8)
+        cases.append((name, x))
+    x = b.copy()                                   # payload bit flips: still valid code words
     pos = d.off_stream + np.random.default_rng(1).integers(0, (d.total_bits + 7) // 8, 50)
     x[pos] ^= np.uint8(0x10)
     cases.append(("payload", x))
+    x = b.copy()                                   # gaps and counts garbage
+    rng = np.random.default_rng(2)
+    x[d.off_gaps: d.off_gaps + d.n_blocks * 32] = rng.integers(0, 256, d.n_blocks * 32)
+    x[d.off_counts: d.off_counts + d.n_blocks * 32] = rng.integers(0, 256, d.n_blocks * 32)
+    cases.append(("index", x))
     for name, x in cases:
         out = torch.zeros(w.size + 2 * guard, dtype=torch.int16, device="cuda")
         status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -294,10 +306,15 @@ def test_df11_fixed_length_corruption_is_contained():
         torch.cuda.synchronize()
         got = host_u16(out)
         assert np.all(got[:guard] == 0) and np.all(got[guard + w.size:] == 0), name   # nothing outside
-        if name == "payload":
-            assert np.array_equal(got[guard:guard + w.size], odf.decode(x)), name
+        if name in ("first", "last"):
+            assert int(status.item()) & lwc.LWC_DEVICE_BAD_OFFSET, name
+        elif name == "interior":
+            assert int(status.item()) & lwc.LWC_DEVICE_BAD_OFFSET or \
+                (int(status.item()) == 0 and np.array_equal(got[guard:guard + w.size], w)), name
+        elif name == "payload":
+            assert int(status.item()) == 0 and np.array_equal(got[guard:guard + w.size], odf.decode(x)), name
         else:
-            assert int(status.item()) & lwc.LWC_DEVICE_BAD_COUNT, name
+            assert int(status.item()) == 0 and np.array_equal(got[guard:guard + w.size], w), name
 
 
 # ------------------------------------------------------------ full-size configs

@@ -464,47 +464,78 @@ def test_gemm_tile_placement_model(rows, cols, chunk, order):
             q += 1
 
 
-# ---- fixed-length codes (fixed_code_length / stage_fixed, csrc/lwc_df11_dev.cuh) ----
+# ---- fixed-length codes (fixed_code_length, csrc/lwc_df11_dev.cuh; decode_fixed_range, csrc/lwc_df11.cu) ----
 #
 # When every code word has one length L <= 8 (flat exponent histograms: the
-# uniform-exponent stress tensor is L = 8), the counted decoder reads the
-# block's codes as back-to-back L-bit fields: each staging word from one
-# 32-bit window and four lookups in a 2^L-entry table. Restated here: the
-# test that picks this path (all symbol-table entries equal), and the word
-# stores, checked for single writers, in-range words and segment reads, and
-# the staged bytes.
+# uniform-exponent stress tensor is L = 8), code i is stream bits [iL, iL + L),
+# and a CTA decodes the weights of its blocks straight from their indices:
+# 32-weight pieces from L stream words each, the ends one by one. Restated
+# here: the test that picks this path (all symbol-table entries equal), and
+# the range decode, checked for in-range reads, every weight written once,
+# and the exponents it produces.
+
+def _unrot(e):
+    return ((e << 1) | (e >> 7)) & 0xFF
+
 
 def _fixed_code_length(sym):
+    """(L, affine) as fixed_code_length decides; (0, False) for other codes."""
     y0 = sym[0][1]
     if y0 == 0 or any(e[1] != y0 for e in sym):
-        return 0
+        return 0, False
     c, used = y0 >> 11, y0 & 31
     if c == 0 or used % c or used // c > 8:
-        return 0
-    return used // c
+        return 0, False
+    L = used // c
+    tab = [sym[v << (FAST_BITS - L)][0] & 0xFF for v in range(1 << L)]
+    e0 = _unrot(tab[0])
+    return L, e0 + (1 << L) - 1 <= 255 and all(_unrot(tab[v]) == e0 + v for v in range(1 << L))
 
 
-def _stage_fixed(seg, last, tab, L, start, n, qb):
-    """stage_fixed for the whole warp: [(word, value)] in store order."""
-    stores = []
-    sh = 32 - L
-    for k in range(qb >> 2, (qb + n + 3) >> 2):
-        i0 = 4 * k - qb
-        assert i0 >= -3
-        p = start + max(i0, 0) * L
-        wi = p >> 5
-        lo_i, hi_i = min(wi + 1, last), min(wi, last)
-        assert 0 <= hi_i <= lo_i <= last
-        win = _fsl(seg[lo_i], seg[hi_i], p & 31)
-        x = 0
-        for j in range(4):
-            f = ((win << (j * L)) & 0xFFFFFFFF) >> sh
-            assert f < len(tab)
-            x |= tab[f] << (8 * j)
-        if i0 < 0:
-            x = (x << (8 * -i0)) & 0xFFFFFFFF
-        stores.append((k, x))
-    return stores
+def _fixed_range(words, n, L, tab, ob, oe, nt, affine=False):
+    """decode_fixed_range for one CTA of nt threads: {weight: rotated exponent}
+    (the affine form computes base + field and merges unrotated; returned
+    rotated here, to compare alike)."""
+    base = _unrot(tab[0])
+    nwords = len(words)
+    out = {}
+
+    def put(i, e):
+        assert ob <= i < oe and 0 <= i < n and i not in out, i
+        out[i] = e
+
+    p_lo, p_hi = (ob + 31) & ~31, oe & ~31
+    for t in range(nt):
+        for g in range(p_lo + 32 * t, p_hi, 32 * nt):
+            w0 = g // 32 * L
+            assert w0 + L <= nwords               # the piece's words exist: no read is clamped
+            w = [int(words[w0 + j]) for j in range(L)] + [0]
+            if affine and L == 8:   # whole bytes, byte-swapped, plus base in every byte
+                for q in range(8):
+                    x = int.from_bytes(w[q].to_bytes(4, "big"), "little") + base * 0x01010101
+                    assert x < 1 << 32
+                    for j in range(4):
+                        put(g + 4 * q + j, _rot((x >> (8 * j)) & 0xFF))
+                continue
+            for c in range(32):
+                p = c * L
+                k, o = p >> 5, p & 31
+                f = (((w[k] << 32 | w[k + 1]) << o) >> (64 - L)) & ((1 << L) - 1)
+                assert f < len(tab)
+                if affine:
+                    assert base + f <= 255
+                    put(g + c, _rot(base + f))
+                else:
+                    put(g + c, tab[f])
+        for u in range(t, 62, nt):
+            i = ob + u if u < 31 else max(p_hi, p_lo) + (u - 31)
+            if i < min(p_lo, oe) if u < 31 else i < oe:
+                p = i * L
+                k = p >> 5
+                wa = int(words[k]) if k < nwords else 0
+                wb = int(words[k + 1]) if k + 1 < nwords else 0
+                put(i, tab[_fsl(wb, wa, p & 31) >> (32 - L)])
+    return out
 
 
 def _blob_tables(b):
@@ -514,53 +545,43 @@ def _blob_tables(b):
     return h, _counted_tables(lut)
 
 
+@pytest.mark.parametrize("step", [1, 2])   # consecutive exponents (an affine code) or every other one
 @pytest.mark.parametrize("L", range(1, 9))
 @pytest.mark.parametrize("chunk", [8, 12, 36])
-def test_fixed_length_staging_model(L, chunk):
+def test_fixed_length_range_model(L, chunk, step):
     import synth
     from decode_dfloat11_b200 import lwc
     from oracle import blob as B
     from oracle import df11 as odf
 
-    w = synth.as_u16(synth.equal_exponents(60_001, L, seed=L))
+    if step * ((1 << L) - 1) > 255:
+        pytest.skip("2^L exponents with gaps do not fit in 8 bits")
+    w = synth.as_u16(synth.equal_exponents(20_001 + 37 * L, L, seed=L, step=step))
     d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk)
     h, (sym, sub, first_long) = _blob_tables(b)
     lengths = B.section(b, h["off_lengths"], 256)
     assert set(lengths[lengths > 0].tolist()) == {L}
     assert first_long == 1 << FAST_BITS          # no code longer than the fast table's 11 bits
-    assert _fixed_code_length(sym) == L
-    if not d.flags & 2:                          # > 255 codes per chunk: no stored counts, two-pass kernel
-        assert 8 * chunk // L > 255
-        return
+    assert _fixed_code_length(sym) == (L, step == 1)   # canonical codes of consecutive exponents
+    assert h["total_bits"] == L * w.size          # the kernel's precondition holds for a valid blob
     tab = [sym[v << (FAST_BITS - L)][0] & 0xFF for v in range(1 << L)]
     exps, _ = odf.split(w)
     words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
-    gaps = B.section(b, h["off_gaps"], h["n_blocks"] * 32)
-    counts = B.section(b, h["off_counts"], h["n_blocks"] * 32)
-    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64)
-    cw = chunk // 4
-    cbits = 32 * cw
-    seg_words = (32 * cw + 2 + 3) // 4 * 4
-    stage_bytes = (int(np.diff(blkoff).max()) + 16 + 15) // 16 * 16
+    blkoff = B.section(b, h["off_blkoff"], 8 * (h["n_blocks"] + 1), np.uint64).astype(int)
     nb = h["n_blocks"]
-    for blk in sorted({0, 1, nb // 2, nb - 2, nb - 1} & set(range(nb))):
-        o0, o1 = int(blkoff[blk]), int(blkoff[blk + 1])
-        n = o1 - o0
-        assert int(counts[blk * 32:(blk + 1) * 32].sum()) == n
-        seg = [int(x) for x in words[blk * 32 * cw:blk * 32 * cw + seg_words]]
-        seg += [0xDEADBEEF] * (seg_words - len(seg))
-        start0 = int(gaps[blk * 32])
-        rem_block = h["total_bits"] - blk * 32 * cbits
-        block_end = 32 * cbits + int(gaps[(blk + 1) * 32]) if blk + 1 < nb else rem_block
-        assert start0 + n * L == block_end, blk           # the kernel's consistency check holds
-        stores = _stage_fixed(seg, seg_words - 1, tab, L, start0, n, o0 & 15)
-        ks = [k for k, _ in stores]
-        assert len(ks) == len(set(ks)) and all(4 * k + 4 <= stage_bytes for k in ks), blk
-        stage = bytearray(b"\xAA" * stage_bytes)
-        for k, x in stores:
-            stage[4 * k:4 * k + 4] = x.to_bytes(4, "little")
-        got = np.frombuffer(bytes(stage[(o0 & 15):(o0 & 15) + n]), np.uint8)
-        assert np.array_equal(got, np.array([_rot(int(x)) for x in exps[o0:o1]], np.uint8)), blk
+    # CTA ranges as the launch splits the work list: G CTAs over nb blocks
+    for G in (1, 3, 296):
+        done = {}
+        for cta in range(G):
+            b0, b1 = nb * cta // G, nb * (cta + 1) // G
+            if b0 >= b1:
+                continue
+            got = _fixed_range(words, w.size, L, tab, int(blkoff[b0]), int(blkoff[b1]), 32 if G == 3 else 576,
+                               affine=_fixed_code_length(sym)[1])
+            assert not (set(got) & set(done))
+            done.update(got)
+        assert sorted(done) == list(range(w.size))
+        assert [done[i] for i in range(w.size)] == [_rot(int(x)) for x in exps]
 
 
 @pytest.mark.parametrize("case", ["normal", "three_values", "nine_values", "two_lengths", "long_codes"])
@@ -591,4 +612,4 @@ def test_fixed_length_test_rejects_variable_codes(case):
     from oracle import blob as B
     lengths = B.section(b, h["off_lengths"], 256)
     assert len(set(lengths[lengths > 0].tolist())) > 1
-    assert _fixed_code_length(sym) == 0
+    assert _fixed_code_length(sym) == (0, False)
