@@ -28,7 +28,10 @@
 // one warp decodes one block with a warp scan and its own segment buffer,
 // staging area and mbarrier, so no CTA-wide barrier sits on the per-block
 // path; 18 warps per CTA share the tables. df11_decode_kernel (blocks of 64+
-// chunks): one block per CTA and a block scan.
+// chunks): one block per CTA and a block scan. Blobs that store each chunk's
+// code count take df11_counted_kernel (the first phase read, not recomputed);
+// its instance for codes of at most 8 bits also decodes codes whose words all
+// have one length straight from the weight index (decode_fixed_range).
 //
 // Memory pipeline: as soon as pass 2 of an item no longer needs the shared
 // stream segment, the bulk-copy (TMA) engine starts bringing in the segment
@@ -259,6 +262,51 @@ __device__ __forceinline__ uint32_t fixed_field(const uint32_t (&w)[L + 1], int 
     return __funnelshift_l(w[k + 1], w[k], (uint32_t)o) >> (32 - L);
 }
 
+// The stream words (w[0..L-1], w[L] = 0) and sign|mantissa bytes of the
+// 32-weight piece at weight g (a multiple of 32).
+template <int L>
+__device__ __forceinline__ void fixed_load(const Df11Tensor &tn, uint64_t nwords, uint64_t g, uint32_t (&w)[L + 1],
+                                           uint4 &s0, uint4 &s1) {
+    const uint64_t w0 = g / 32 * L;   // the piece's first stream word
+    if (L % 4 == 0 && w0 + L <= nwords) {   // 16-byte aligned: w0 is a multiple of L
+#pragma unroll
+        for (int j = 0; j < L; j += 4) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(tn.stream + w0 + j));
+            w[j] = v.x;
+            w[j + 1] = v.y;
+            w[j + 2] = v.z;
+            w[j + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < L; j++) w[j] = w0 + j < nwords ? __ldg(tn.stream + w0 + j) : 0u;
+    }
+    w[L] = 0;
+    s0 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g));
+    s1 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g + 16));
+}
+
+// Decodes and merges the piece at weight g (see decode_fixed_range).
+template <int E, int L, bool AFF>
+__device__ __forceinline__ void fixed_emit(const Df11Tensor &tn, const uint32_t *tab, uint32_t base4, uint64_t g,
+                                           const uint32_t (&w)[L + 1], const uint4 &s0, const uint4 &s1) {
+    uint32_t e[8];
+#pragma unroll
+    for (int q = 0; q < 8; q++) {
+        if constexpr (AFF && L == 8) {   // four whole bytes, first code in the top one
+            e[q] = __byte_perm(w[q], 0u, 0x0123u) + base4;
+        } else if constexpr (AFF) {   // each byte stays <= 255: base + 2^L - 1 <= 255
+            e[q] = (fixed_field<L>(w, 4 * q) | (fixed_field<L>(w, 4 * q + 1) << 8) |
+                    (fixed_field<L>(w, 4 * q + 2) << 16) | (fixed_field<L>(w, 4 * q + 3) << 24)) + base4;
+        } else {
+            e[q] = tab[fixed_field<L>(w, 4 * q)] | (tab[fixed_field<L>(w, 4 * q + 1)] << 8) |
+                   (tab[fixed_field<L>(w, 4 * q + 2)] << 16) | (tab[fixed_field<L>(w, 4 * q + 3)] << 24);
+        }
+    }
+    merge_group<E, !AFF>(s0, make_uint4(e[0], e[1], e[2], e[3]), tn.out, tn.lo, g);
+    merge_group<E, !AFF>(s1, make_uint4(e[4], e[5], e[6], e[7]), tn.out, tn.lo, g + 16);
+}
+
 // The CTA's threads t = 0 .. nt - 1: weights [ob, oe) of tensor tn, whose
 // code words all have length L (1..8); tab[v] = rotated exponent of code
 // word v. AFF: code word v stands for exponent base + v (a flat histogram over
@@ -285,39 +333,10 @@ __device__ __noinline__ void decode_fixed_range(const Df11Tensor &tn, const uint
                     dev::prefetch_l2(reinterpret_cast<const uint8_t *>(tn.stream) + s0, (uint32_t)(s1 - s0));
             }
         }
-        const uint64_t w0 = g / 32 * L;   // the piece's first stream word
         uint32_t w[L + 1];
-        if (L % 4 == 0 && w0 + L <= nwords) {   // 16-byte aligned: w0 is a multiple of L
-#pragma unroll
-            for (int j = 0; j < L; j += 4) {
-                const uint4 v = __ldg(reinterpret_cast<const uint4 *>(tn.stream + w0 + j));
-                w[j] = v.x;
-                w[j + 1] = v.y;
-                w[j + 2] = v.z;
-                w[j + 3] = v.w;
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < L; j++) w[j] = w0 + j < nwords ? __ldg(tn.stream + w0 + j) : 0u;
-        }
-        w[L] = 0;
-        const uint4 s0 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g));
-        const uint4 s1 = __ldg(reinterpret_cast<const uint4 *>(tn.sm + g + 16));
-        uint32_t e[8];
-#pragma unroll
-        for (int q = 0; q < 8; q++) {
-            if constexpr (AFF && L == 8) {   // four whole bytes, first code in the top one
-                e[q] = __byte_perm(w[q], 0u, 0x0123u) + base4;
-            } else if constexpr (AFF) {   // each byte stays <= 255: base + 2^L - 1 <= 255
-                e[q] = (fixed_field<L>(w, 4 * q) | (fixed_field<L>(w, 4 * q + 1) << 8) |
-                        (fixed_field<L>(w, 4 * q + 2) << 16) | (fixed_field<L>(w, 4 * q + 3) << 24)) + base4;
-            } else {
-                e[q] = tab[fixed_field<L>(w, 4 * q)] | (tab[fixed_field<L>(w, 4 * q + 1)] << 8) |
-                       (tab[fixed_field<L>(w, 4 * q + 2)] << 16) | (tab[fixed_field<L>(w, 4 * q + 3)] << 24);
-            }
-        }
-        merge_group<E, !AFF>(s0, make_uint4(e[0], e[1], e[2], e[3]), tn.out, tn.lo, g);
-        merge_group<E, !AFF>(s1, make_uint4(e[4], e[5], e[6], e[7]), tn.out, tn.lo, g + 16);
+        uint4 s0, s1;
+        fixed_load<L>(tn, nwords, g, w, s0, s1);
+        fixed_emit<E, L, AFF>(tn, tab, base4, g, w, s0, s1);
     }
     // the weights before the first piece (u = 0..30) and after the last (u = 31..61)
     for (uint32_t u = t; u < 62; u += nt) {
