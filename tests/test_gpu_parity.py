@@ -253,6 +253,27 @@ def test_df11_fixed_length_codes(L, chunk_bytes, step):
     assert np.array_equal(got, w)
 
 
+@pytest.mark.parametrize("chunk_bytes", [8, 20, 36])
+def test_df11_short_variable_length_codes(chunk_bytes):
+    """Codes of at most 8 bits with more than one length (geometric exponent
+    frequencies 2^7 : 2^6 : ... : 1 over 8 exponents, lengths 1..7): the kernel
+    instance launched for short codes, on its block path."""
+    rng = np.random.default_rng(chunk_bytes)
+    counts = 1 << np.arange(7, -1, -1)
+    e = np.repeat(np.arange(120, 128), counts * 2_000)
+    w = ((e.astype(np.uint16) << 7) | rng.integers(0, 128, e.size).astype(np.uint16)
+         | (rng.integers(0, 2, e.size).astype(np.uint16) << 15))
+    w = rng.permutation(w).astype(np.uint16)
+    d, b = lwc.lwc_encode_dfloat11(w, chunk_bytes=chunk_bytes)
+    lengths = b[d.off_lengths:d.off_lengths + 256]
+    assert d.max_len <= 8 and len(set(lengths[lengths > 0].tolist())) > 1
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    got = host_u16(gpu_decode(d, dev(b), status=status))
+    assert int(status.item()) == 0
+    assert np.array_equal(got, odf.decode(b))
+    assert np.array_equal(got, w)
+
+
 def test_df11_fixed_length_batched_and_device_encoded():
     """Fixed- and variable-length tensors alternating in one launch (the CTA
     switches paths at each tensor boundary), encoded on the device."""
