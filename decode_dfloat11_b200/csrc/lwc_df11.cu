@@ -673,6 +673,14 @@ __global__ void __launch_bounds__(kMaxThreads, kCtasPerSm * 256 / kMaxThreads > 
 // 18 of them).
 constexpr uint32_t kWarpsPerCta = 18;   // 2 CTAs (36 warps) per SM fit registers and shared memory
 constexpr int kWarpCtasPerSm = 2;
+// The counted decoder's wide form: one CTA of 32 warps per SM. The SM's
+// schedulers do not serve two CTAs evenly, so of two CTAs with equal shares one
+// finishes early and its sibling runs the rest with half the warps; with one
+// CTA every warp claims from the same counter. That outweighs the four fewer
+// warps on long launches (a Llama-3-70B layer: 0.580 -> 0.572 ms; the model
+// pass 2.4 % faster) but not on short ones (a Llama-3-8B layer: 0.164 -> 0.170).
+constexpr uint32_t kWideWarpsPerCta = 32;
+constexpr uint64_t kWideMinWeights = 512ull << 20;   // launches of at least this many weights
 constexpr int kWarpMergeRegs = 3;       // 16-weight merge groups per lane whose loads are issued early
 
 struct WarpLayout {
@@ -1447,8 +1455,9 @@ __device__ __forceinline__ void df11_counted_body(const Df11Batch &B, const Df11
     if (bad && B.status) atomicOr(B.status, bad);
 }
 
-template <int E, bool FX = false>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, kWarpCtasPerSm) df11_counted_kernel(const __grid_constant__ Df11Batch B) {
+template <int E, bool FX = false, bool WIDE = false>
+__global__ void __launch_bounds__(WIDE ? kWideWarpsPerCta * 32 : kWarpsPerCta * 32, WIDE ? 1 : kWarpCtasPerSm)
+    df11_counted_kernel(const __grid_constant__ Df11Batch B) {
     df11_counted_body<E, 0, FX>(B, nullptr);
 }
 
@@ -1523,6 +1532,9 @@ lwc_status device_config(DeviceConfig &out) {
             (const void *)df11_counted_kernel<LWC_ELEM_FP32>, (const void *)df11_counted_kernel<LWC_ELEM_FP16>,
             (const void *)df11_counted_kernel<LWC_ELEM_BF16, true>, (const void *)df11_counted_kernel<LWC_ELEM_FP32, true>,
             (const void *)df11_counted_kernel<LWC_ELEM_FP16, true>,
+            (const void *)df11_counted_kernel<LWC_ELEM_BF16, false, true>,
+            (const void *)df11_counted_kernel<LWC_ELEM_FP32, false, true>,
+            (const void *)df11_counted_kernel<LWC_ELEM_FP16, false, true>,
             (const void *)kLinKernels[0], (const void *)kLinKernels[1],
             (const void *)kLinKernels[2], (const void *)kLinKernels[3], (const void *)kCtdLinKernels[0],
             (const void *)kCtdLinKernels[1], (const void *)kCtdLinKernels[2], (const void *)kCtdLinKernels[3]};
@@ -1541,13 +1553,15 @@ lwc_status device_config(DeviceConfig &out) {
 
 // Decode kernels: one CTA per block (blocks of 64+ chunks), one warp per
 // block (blocks of 32 chunks), or one warp per block with stored chunk counts
-// (kModeCountedShort: codes of at most 8 bits, with the fixed-length path).
-enum KernelMode { kModeBlock, kModeWarp, kModeCounted, kModeCountedShort };
+// (kModeCountedShort: codes of at most 8 bits, with the fixed-length path;
+// kModeCountedWide: one CTA of 32 warps per SM, for long launches).
+enum KernelMode { kModeBlock, kModeWarp, kModeCounted, kModeCountedShort, kModeCountedWide };
 
 template <int E>
 const void *df11_kernel(KernelMode mode, uint32_t T) {
     return mode == kModeCounted        ? (const void *)df11_counted_kernel<E>
            : mode == kModeCountedShort ? (const void *)df11_counted_kernel<E, true>
+           : mode == kModeCountedWide  ? (const void *)df11_counted_kernel<E, false, true>
            : mode == kModeWarp         ? (const void *)df11_warp_kernel<E>
            : T <= 256           ? (const void *)df11_decode_kernel<256, E>
                                 : (const void *)df11_decode_kernel<1024, E>;
@@ -1564,6 +1578,8 @@ void launch_df11(KernelMode mode, uint32_t T, unsigned grid, uint32_t threads, s
                  const Df11Batch &B) {
     if (mode == kModeCounted)
         df11_counted_kernel<E><<<grid, threads, smem, stream>>>(B);
+    else if (mode == kModeCountedWide)
+        df11_counted_kernel<E, false, true><<<grid, threads, smem, stream>>>(B);
     else if (mode == kModeCountedShort)
         df11_counted_kernel<E, true><<<grid, threads, smem, stream>>>(B);
     else if (mode == kModeWarp)
@@ -1576,7 +1592,7 @@ void launch_df11(KernelMode mode, uint32_t T, unsigned grid, uint32_t threads, s
 
 // Shared memory of a per-warp launch with w warps per CTA.
 uint64_t warp_smem(const Df11Batch &B, KernelMode mode, uint32_t w) {
-    return mode == kModeCounted || mode == kModeCountedShort
+    return mode == kModeCounted || mode == kModeCountedShort || mode == kModeCountedWide
                ? CountedLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total
                                 : WarpLayout(B.seg_words, B.lut_entries, B.stage_bytes, w).total;
 }
@@ -1584,7 +1600,7 @@ uint64_t warp_smem(const Df11Batch &B, KernelMode mode, uint32_t w) {
 // Warps per CTA of the per-warp kernels: kWarpsPerCta, or fewer when one
 // warp's segment buffer and staging area are large (long chunks).
 uint32_t warps_that_fit(const Df11Batch &B, int max_smem, KernelMode mode = kModeWarp) {
-    uint32_t w = kWarpsPerCta;
+    uint32_t w = mode == kModeCountedWide ? kWideWarpsPerCta : kWarpsPerCta;
     while (w > 1 && warp_smem(B, mode, w) > (uint64_t)max_smem) w--;
     return w;
 }
@@ -1629,9 +1645,12 @@ lwc_status launch_group(const std::vector<int> &idx, const lwc_desc *descs, cons
     B.stage_bytes = (uint32_t)round_up(max_count + 16, 16);
     B.lut_entries = (uint32_t)(max_tables * 256);
     B.status = d_status;
+    uint64_t weights = 0;
+    for (const int i : idx) weights += descs[i].n;
     const KernelMode mode = T != 32                           ? kModeBlock
                             : !(d0.flags & kFlagChunkCounts) ? kModeWarp
                             : d0.max_len <= 8                ? kModeCountedShort
+                            : weights >= kWideMinWeights     ? kModeCountedWide
                                                              : kModeCounted;
     const bool per_warp = mode != kModeBlock;
     B.warps = per_warp ? warps_that_fit(B, cfg.max_smem, mode) : 0;
