@@ -477,3 +477,32 @@ def test_df11_fp32_full_size():
     got = gpu_decode_elements(d, dev(b), B.ELEM_FP32, xh.size)
     assert np.array_equal(got, xh)
     assert 8.0 * d.total_bytes / d.n < 28.0
+
+
+@pytest.mark.parametrize("elem", [B.ELEM_FP32, B.ELEM_FP16])
+def test_df11_wide_form_elements(elem):
+    """A launch of at least 512 M weights takes the counted decoder's wide form
+    (one 32-warp CTA per SM): 2^29 + 12,345 FP32 / FP16 elements encoded on the
+    device, decoded, compared with the input, and sampled block ranges of the
+    coded 16-bit patterns compared with the oracle's block-range decode."""
+    from decode_dfloat11_b200.layers import encode_on_device
+    n = (1 << 29) + 12_345
+    g = torch.Generator(device="cuda").manual_seed(90 + elem)
+    x = torch.randn(n, generator=g, device="cuda") * 0.02
+    x = x if elem == B.ELEM_FP32 else x.to(torch.float16)
+    d, blob = encode_on_device(x, "dfloat11")
+    assert d.elem == elem and d.flags & 2 and d.max_len > 8
+    out = torch.empty(n, dtype=torch.int32 if elem == B.ELEM_FP32 else torch.int16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lwc.lwc_decode_dfloat11_checked(d, blob, out, status, torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(out, x.view(torch.int32 if elem == B.ELEM_FP32 else torch.int16))
+    hb = blob.cpu().numpy()
+    xs = x.view(torch.int32 if elem == B.ELEM_FP32 else torch.int16).cpu().numpy()
+    xs = xs.view(np.uint32) if elem == B.ELEM_FP32 else xs.view(np.uint16)
+    blkoff = B.section(hb, d.off_blkoff, 8 * (d.n_blocks + 1), np.uint64)
+    for b0 in (0, d.n_blocks // 3, d.n_blocks - 3):
+        v = odf.decode_blocks(hb, b0, b0 + 3)
+        i0, i1 = int(blkoff[b0]), int(blkoff[b0 + 3])
+        assert np.array_equal(v, odf.split_elements(xs[i0:i1], elem)[0]), b0
