@@ -90,6 +90,40 @@ def test_uniform_exponents_maximal_spread():
     assert 15.9 < df11.bits_per_weight(b) < 16.6
 
 
+@pytest.mark.parametrize("L", range(1, 9))
+def test_flat_histograms_give_fixed_length_affine_codes(L):
+    """2^L consecutive exponents in equal numbers: Huffman merges them in
+    pairs level by level, so every code word has length L, and canonical codes
+    of one length follow symbol order, so exponent e0 + v gets word v; the
+    stream is then L-bit fields, weight i's at bits [iL, iL + L). This is what
+    the decoder's fixed-length path relies on."""
+    w = synth.as_u16(synth.equal_exponents(2048 * (1 << L) + 5, L, seed=L))
+    counts, lengths, _ = df11.code_for(w)
+    present = [e for e in range(256) if lengths[e]]
+    e0 = present[0]
+    assert present == list(range(e0, e0 + (1 << L)))
+    assert {lengths[e] for e in present} == {L}
+    codes = H.canonical_codes(lengths)
+    assert [codes[e] for e in present] == list(range(1 << L))
+    b = df11.encode(w)
+    h = B.unpack_header(b)
+    assert h["total_bits"] == L * w.size
+    words = B.section(b, h["off_stream"], h["stream_bytes"], np.uint32)
+    bits = "".join(format(int(x), "032b") for x in words[: (L * w.size + 31) // 32])
+    e = (w >> 7) & 0xFF
+    for i in list(range(0, w.size, 97)) + [w.size - 1]:
+        assert int(bits[i * L:(i + 1) * L], 2) == int(e[i]) - e0, i
+
+
+def test_unequal_histogram_is_not_fixed_length():
+    # counts 4000 : 1000 : 1000 : 1000 over four exponents: lengths (1, 2, 3, 3)
+    # cost 12,000 bits against 14,000 for four 2-bit codes, so the code has
+    # several lengths and the fixed-length path must not apply
+    w = np.repeat(np.array([120, 121, 122, 123], np.uint16) << 7, [4000, 1000, 1000, 1000])
+    counts, lengths, _ = df11.code_for(w)
+    assert sorted(l for l in lengths if l) == [1, 2, 3, 3]
+
+
 # ------------------------------------------------------- code properties
 
 def code_strings(lengths, codes):
